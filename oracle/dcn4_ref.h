@@ -1,0 +1,105 @@
+/*
+ * dcn4_ref.h — plain, slow CPU oracle for the DCNv4 core spatial aggregation.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the test suite, the smoke check and the
+ * benchmark's CPU-baseline / reference arm may load this library.  The product
+ * path (libdcn4) never links, loads or calls it, and it shares no code, header,
+ * table or helper with the GPU path.
+ *
+ * What it computes (CVPR'24 "Efficient Deformable ConvNets: Rethinking Dynamic
+ * and Sparse Operator for Vision Applications", summarised on the CSDN page
+ * "DCNv4论文解析", section 1.2 "回顾DCNv3" equation, with the softmax removed as in
+ * section 2.1 "增强动态特性"):
+ *
+ *     y_g(p0) = sum_k  m_gk * x_g(p0 + p_k + offset_scale * dp_gk)
+ *     y       = concat_g y_g                      (channels-last)
+ *
+ * x_g(.) is bilinear interpolation of group g's C' channels of the zero-extended
+ * image (section 2.2, "GPU效率的理论分析": four coefficients per sampling point).
+ * p_k enumerates a kh x kw convolution grid with stride / pad / dilation; with
+ * remove_center the centre cell is skipped (DCNv4 module signature on the
+ * mhpn.cn architecture page, "参数remove_center").
+ *
+ * Layouts (all dense, row-major, channels last):
+ *   value        [N, H, W, G*Cg]
+ *   offset_mask  [N, Ho, Wo, P]; group g owns entries [g*3K, (g+1)*3K):
+ *                K pairs (dx_k, dy_k) followed by K masks m_k; [G*3K, P) is
+ *                padding and is never read.
+ *   out          [N, Ho, Wo, G*Cg]
+ *   grad_*       same shape as the tensor they are the gradient of.
+ *
+ * Grid order: k runs over the kernel columns (x) in the outer loop and the
+ * kernel rows (y) in the inner loop, i.e. k = iw*kh + ih before the centre is
+ * removed; the centre cell (kw/2, kh/2) is skipped when remove_center != 0 and
+ * later cells keep their relative order.  dx moves the sample along W, dy
+ * along H.
+ *
+ * Sampling location for output (ho, wo), grid cell (ih, iw):
+ *     h = ho*sh - ph + ih*dh + offset_scale*dy,   w = wo*sw - pw + iw*dw + offset_scale*dx
+ * In location_fp32 mode the location is formed as one fp32 fused multiply-add
+ * fmaf(offset_scale, d, base) — the precision in which the GPU kernels decide
+ * which bilinear cell a sample falls in — and all later arithmetic stays in
+ * double.  Otherwise the location is formed in double.
+ *
+ * Element storage: REF_F32, REF_F16 (IEEE binary16), REF_BF16 (upper half of an
+ * IEEE binary32) and REF_F64 (for finite-difference tests).  Every element is
+ * decoded exactly into a double by this file's own bit-level decoders.
+ * Outputs and gradients are written as double.
+ */
+#ifndef DCN4_REF_H
+#define DCN4_REF_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum { REF_F32 = 0, REF_F16 = 1, REF_BF16 = 2, REF_F64 = 3 };
+
+typedef struct {
+    int N, H, W;          /* input batch and spatial size                      */
+    int G, Cg;            /* groups and channels per group (C = G*Cg)          */
+    int kh, kw;           /* kernel grid                                       */
+    int sh, sw;           /* stride                                            */
+    int ph, pw;           /* padding                                           */
+    int dh, dw;           /* dilation                                          */
+    double offset_scale;  /* multiplies the learned offsets only               */
+    int remove_center;    /* 1: skip the centre grid cell (odd kh, kw only)    */
+    int P;                /* row length of offset_mask, >= G*3K                */
+    int dtype;            /* REF_* storage type of value/offset_mask/grad_out  */
+    int location_fp32;    /* 1: form the sampling location with an fp32 fma    */
+} ref_problem;
+
+/* Output size of the grid: Ho = (H + 2ph - (dh*(kh-1)+1)) / sh + 1 (floor).
+ * Returns 0, or -1 when the problem is malformed. */
+int ref_output_dims(const ref_problem* p, int* Ho, int* Wo);
+
+/* Number of sampling points K = kh*kw - (remove_center ? 1 : 0). */
+int ref_num_points(const ref_problem* p);
+
+/* Forward: out[N,Ho,Wo,G*Cg] (double).  nthreads > 1 splits output rows
+ * across std::thread workers; each output element is computed by one thread in the
+ * same order.  Returns 0 or -1. */
+int ref_forward(const ref_problem* p, const void* value, const void* offset_mask,
+                double* out, int nthreads);
+
+/* Backward for grad_out (stored in p->dtype):
+ *   grad_value       [N,H,W,G*Cg]  = adjoint of the forward in value
+ *   grad_offset_mask [N,Ho,Wo,P]   = d<grad_out, y>/d offset_mask; the padding
+ *                                    tail [G*3K, P) is written as 0.
+ * The bilinear derivative at an integer coordinate is the one-sided one of
+ * the cell that floor() selects.  nthreads > 1 splits the batch across
+ * std::thread workers (images are independent).  Returns 0 or -1. */
+int ref_backward(const ref_problem* p, const void* value, const void* offset_mask,
+                 const void* grad_out, double* grad_value, double* grad_offset_mask,
+                 int nthreads);
+
+/* Exact decode of n stored elements into doubles. */
+void ref_decode(int dtype, const void* src, double* dst, int64_t n);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DCN4_REF_H */

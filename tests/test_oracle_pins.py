@@ -1,0 +1,493 @@
+"""Pins of the CPU oracle against things other than itself (CPU only).
+
+The pages print no worked numeric example, so the oracle is pinned by:
+  * library routines that compute special cases of the operator on the host
+    (grouped conv2d, grid_sample, torchvision's deform_conv2d);
+  * exact special cases (integer offsets are plain gathers, far-off-image
+    samples are zero, remove_center is a zero centre mask, offset_scale only
+    scales the offsets);
+  * identities the mathematics fixes (linearity in value and mask, the
+    adjoint identity for grad_value, <grad_mask, m> = <grad_out, y>);
+  * central finite differences for grad_offset / grad_mask.
+
+The operator is the DCNv3 aggregation of the CSDN summary of "Efficient
+Deformable ConvNets" (section 1.2 equation) without the softmax (section 2.1),
+sampled bilinearly (section 2.2), with offset_scale / remove_center from the
+DCNv4 module signature on the mhpn.cn architecture page.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+import dcn4_inputs as gen
+import oracle
+
+torch.set_default_dtype(torch.float64)
+
+
+def rand_problem_inputs(prob: oracle.Problem, seed: int, offset=("uniform", -2.0, 2.0),
+                        mask=("normal", 0.0, 1.0)):
+    Ho, Wo = oracle.output_dims(prob)
+    w = gen.custom(N=prob.N, H=prob.H, W=prob.W, G=prob.G, Cg=prob.Cg, Ho=Ho, Wo=Wo, K=prob.K,
+                   P=prob.row, dtype=prob.dtype, offset=offset, mask=mask)
+    return gen.make_inputs(w, seed=seed), Ho, Wo
+
+
+def split_om(om: np.ndarray, G: int, K: int):
+    """offset_mask rows -> (dx [..,G,K], dy [..,G,K], m [..,G,K]) as float64 views of storage."""
+    body = om[..., : G * 3 * K].reshape(om.shape[:-1] + (G, 3 * K))
+    pairs = body[..., : 2 * K].reshape(om.shape[:-1] + (G, K, 2))
+    return pairs[..., 0], pairs[..., 1], body[..., 2 * K:]
+
+
+def cells(kh, kw, remove_center):
+    """Grid cells (ih, iw) in k order: columns outer, rows inner, centre optionally dropped."""
+    out = []
+    for iw in range(kw):
+        for ih in range(kh):
+            if remove_center and ih == kh // 2 and iw == kw // 2:
+                continue
+            out.append((ih, iw))
+    return out
+
+
+def rel_err(a, b):
+    scale = max(np.max(np.abs(b)), 1e-300)
+    return np.max(np.abs(a - b)) / scale
+
+
+GEOMS = [
+    dict(kh=3, kw=3, sh=1, sw=1, ph=1, pw=1, dh=1, dw=1),
+    dict(kh=3, kw=3, sh=2, sw=1, ph=0, pw=2, dh=1, dw=2),
+    dict(kh=3, kw=5, sh=1, sw=2, ph=2, pw=1, dh=2, dw=1),
+    dict(kh=1, kw=3, sh=1, sw=1, ph=0, pw=1, dh=1, dw=1),
+]
+
+
+# ---------------------------------------------------------------------------
+# Decoders
+# ---------------------------------------------------------------------------
+
+def test_decode_f16_all_patterns():
+    bits = np.arange(1 << 16, dtype=np.uint16)
+    got = oracle.decode("f16", bits.view(np.float16))
+    want = bits.view(np.float16).astype(np.float64)
+    np.testing.assert_array_equal(np.isnan(got), np.isnan(want))
+    ok = ~np.isnan(want)
+    np.testing.assert_array_equal(got[ok], want[ok])
+
+
+def test_decode_bf16_all_patterns():
+    bits = np.arange(1 << 16, dtype=np.uint16)
+    got = oracle.decode("bf16", bits)
+    want = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(torch.float64).numpy()
+    np.testing.assert_array_equal(np.isnan(got), np.isnan(want))
+    ok = ~np.isnan(want)
+    np.testing.assert_array_equal(got[ok], want[ok])
+
+
+# ---------------------------------------------------------------------------
+# Geometry: zero offsets + per-(g,k) constant mask == grouped convolution
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("geom", GEOMS)
+@pytest.mark.parametrize("remove_center", [0, 1])
+def test_zero_offsets_equal_grouped_conv(geom, remove_center):
+    if remove_center and (geom["kh"] % 2 == 0 or geom["kw"] % 2 == 0):
+        pytest.skip("remove_center needs odd kernels")
+    prob = oracle.Problem(N=2, H=7, W=9, G=3, Cg=2, remove_center=remove_center, dtype="f64", **geom)
+    inp, Ho, Wo = rand_problem_inputs(prob, seed=11)
+    K = prob.K
+    rng = np.random.default_rng(3)
+    wk = rng.normal(size=(prob.G, K))                 # one weight per (group, grid point)
+    om = inp["offset_mask"]
+    dx, dy, m = split_om(om, prob.G, K)
+    dx[...] = 0.0
+    dy[...] = 0.0
+    m[...] = wk                                        # broadcast over pixels
+    y = oracle.forward(prob, inp["value"], om)
+
+    # depthwise conv2d weight [C, 1, kh, kw]: channel c of group g gets wk[g, k(ih, iw)]
+    weight = np.zeros((prob.C, 1, prob.kh, prob.kw))
+    for k, (ih, iw) in enumerate(cells(prob.kh, prob.kw, remove_center)):
+        for g in range(prob.G):
+            weight[g * prob.Cg:(g + 1) * prob.Cg, 0, ih, iw] = wk[g, k]
+    x = torch.from_numpy(inp["value"]).permute(0, 3, 1, 2)
+    ref = F.conv2d(x, torch.from_numpy(weight), stride=(prob.sh, prob.sw), padding=(prob.ph, prob.pw),
+                   dilation=(prob.dh, prob.dw), groups=prob.C).permute(0, 2, 3, 1).numpy()
+    assert ref.shape == y.shape
+    assert rel_err(y, ref) < 1e-13
+
+
+def test_output_dims_match_conv2d():
+    for geom in GEOMS:
+        for H, W in [(5, 6), (8, 8), (13, 4)]:
+            prob = oracle.Problem(N=1, H=H, W=W, G=1, Cg=1, dtype="f64", **geom)
+            x = torch.zeros(1, 1, H, W)
+            try:
+                ref = F.conv2d(x, torch.zeros(1, 1, prob.kh, prob.kw), stride=(prob.sh, prob.sw),
+                               padding=(prob.ph, prob.pw), dilation=(prob.dh, prob.dw)).shape[2:]
+            except RuntimeError:
+                continue
+            assert oracle.output_dims(prob) == tuple(ref)
+
+
+# ---------------------------------------------------------------------------
+# Integer offsets: exact shifted gathers
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("geom", GEOMS[:3])
+def test_integer_offsets_exact_gather(geom):
+    prob = oracle.Problem(N=2, H=6, W=7, G=2, Cg=3, dtype="f32", **geom)
+    inp, Ho, Wo = rand_problem_inputs(prob, seed=5)
+    K = prob.K
+    om = inp["offset_mask"]
+    dx, dy, m = split_om(om, prob.G, K)
+    rng = np.random.default_rng(9)
+    dx[...] = rng.integers(-3, 4, size=dx.shape).astype(np.float32)
+    dy[...] = rng.integers(-3, 4, size=dy.shape).astype(np.float32)
+    y = oracle.forward(prob, inp["value"], om)
+
+    x = inp["value"].astype(np.float64)
+    want = np.zeros_like(y)
+    for n in range(prob.N):
+        for ho in range(Ho):
+            for wo in range(Wo):
+                for g in range(prob.G):
+                    for k, (ih, iw) in enumerate(cells(prob.kh, prob.kw, 0)):
+                        yy = ho * prob.sh - prob.ph + ih * prob.dh + int(dy[n, ho, wo, g, k])
+                        xx = wo * prob.sw - prob.pw + iw * prob.dw + int(dx[n, ho, wo, g, k])
+                        if 0 <= yy < prob.H and 0 <= xx < prob.W:
+                            sl = slice(g * prob.Cg, (g + 1) * prob.Cg)
+                            want[n, ho, wo, sl] += float(m[n, ho, wo, g, k]) * x[n, yy, xx, sl]
+    np.testing.assert_array_equal(y, want)
+
+
+# ---------------------------------------------------------------------------
+# Bilinear sampling + zero padding == grid_sample(align_corners=True, zeros)
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("offset", [("uniform", -2.0, 2.0), ("uniform", -6.0, 6.0)])
+def test_single_point_matches_grid_sample(offset):
+    prob = oracle.Problem(N=2, H=6, W=8, G=2, Cg=3, dtype="f64", offset_scale=0.75)
+    inp, Ho, Wo = rand_problem_inputs(prob, seed=21, offset=offset)
+    K = prob.K
+    om0 = inp["offset_mask"]
+    for k, (ih, iw) in enumerate(cells(3, 3, 0)):
+        om = om0.copy()
+        dx, dy, m = split_om(om, prob.G, K)
+        m[...] = 0.0
+        m[..., k] = 1.0
+        y = oracle.forward(prob, inp["value"], om)
+        ho = np.arange(Ho)[:, None]
+        wo = np.arange(Wo)[None, :]
+        for g in range(prob.G):
+            h = (ho * prob.sh - prob.ph + ih * prob.dh) + prob.offset_scale * dy[..., g, k]
+            w = (wo * prob.sw - prob.pw + iw * prob.dw) + prob.offset_scale * dx[..., g, k]
+            grid = np.stack([2.0 * w / (prob.W - 1) - 1.0, 2.0 * h / (prob.H - 1) - 1.0], axis=-1)
+            x = torch.from_numpy(inp["value"][..., g * prob.Cg:(g + 1) * prob.Cg]).permute(0, 3, 1, 2)
+            ref = F.grid_sample(x, torch.from_numpy(grid), mode="bilinear", padding_mode="zeros",
+                                align_corners=True).permute(0, 2, 3, 1).numpy()
+            got = y[..., g * prob.Cg:(g + 1) * prob.Cg]
+            assert rel_err(got, ref) < 1e-12
+
+
+# ---------------------------------------------------------------------------
+# Whole operator == torchvision.ops.deform_conv2d with a depthwise all-ones weight
+# ---------------------------------------------------------------------------
+
+def _torchvision():
+    tv = pytest.importorskip("torchvision")
+    return tv.ops.deform_conv2d
+
+
+def test_torchvision_offset_layout_probe():
+    """torchvision's offset channels per kernel position are (row shift, column shift), row-major."""
+    deform_conv2d = _torchvision()
+    H = W = 5
+    ramp_h = torch.arange(H, dtype=torch.float64)[:, None].expand(H, W).reshape(1, 1, H, W)
+    ramp_w = torch.arange(W, dtype=torch.float64)[None, :].expand(H, W).reshape(1, 1, H, W)
+    weight = torch.zeros(1, 1, 3, 3)
+    weight[0, 0, 0, 1] = 1.0                         # kernel position (i=0, j=1) -> index 1
+    off = torch.zeros(1, 18, H, W)
+    off[0, 2 * 1] = 0.5                              # first channel of position 1
+    a = deform_conv2d(ramp_h, off, weight, padding=1)
+    b = deform_conv2d(ramp_h, torch.zeros_like(off), weight, padding=1)
+    assert torch.allclose((a - b)[0, 0, 2, 2], torch.tensor(0.5))   # moved along rows
+    c = deform_conv2d(ramp_w, off, weight, padding=1)
+    d = deform_conv2d(ramp_w, torch.zeros_like(off), weight, padding=1)
+    assert torch.allclose((c - d)[0, 0, 2, 2], torch.tensor(0.0))
+
+
+@pytest.mark.parametrize("geom", GEOMS)
+@pytest.mark.parametrize("remove_center,scale", [(0, 1.0), (1, 0.5), (0, 1.7)])
+def test_matches_torchvision_deform_conv2d(geom, remove_center, scale):
+    deform_conv2d = _torchvision()
+    if remove_center and (geom["kh"] % 2 == 0 or geom["kw"] % 2 == 0):
+        pytest.skip("remove_center needs odd kernels")
+    prob = oracle.Problem(N=2, H=9, W=7, G=3, Cg=2, dtype="f64", offset_scale=scale,
+                          remove_center=remove_center, **geom)
+    inp, Ho, Wo = rand_problem_inputs(prob, seed=31, offset=("normal", 0.0, 2.0))
+    y = oracle.forward(prob, inp["value"], inp["offset_mask"])
+    dx, dy, m = split_om(inp["offset_mask"], prob.G, prob.K)
+    kh, kw = prob.kh, prob.kw
+    off_tv = np.zeros((prob.N, prob.G, kh * kw, 2, Ho, Wo))
+    mask_tv = np.zeros((prob.N, prob.G, kh * kw, Ho, Wo))
+    for k, (ih, iw) in enumerate(cells(kh, kw, remove_center)):
+        j = ih * kw + iw
+        off_tv[:, :, j, 0] = np.moveaxis(scale * dy[..., k], 3, 1)
+        off_tv[:, :, j, 1] = np.moveaxis(scale * dx[..., k], 3, 1)
+        mask_tv[:, :, j] = np.moveaxis(m[..., k], 3, 1)
+    x = torch.from_numpy(inp["value"]).permute(0, 3, 1, 2).contiguous()
+    ref = deform_conv2d(x, torch.from_numpy(off_tv.reshape(prob.N, -1, Ho, Wo)),
+                        torch.ones(prob.C, 1, kh, kw), stride=(prob.sh, prob.sw),
+                        padding=(prob.ph, prob.pw), dilation=(prob.dh, prob.dw),
+                        mask=torch.from_numpy(mask_tv.reshape(prob.N, -1, Ho, Wo)))
+    ref = ref.permute(0, 2, 3, 1).numpy()
+    assert rel_err(y, ref) < 1e-12
+
+
+# ---------------------------------------------------------------------------
+# Structural identities and special cases
+# ---------------------------------------------------------------------------
+
+def _tiny(dtype="f64", **kw):
+    base = dict(N=2, H=6, W=5, G=2, Cg=3, dtype=dtype)
+    base.update(kw)
+    return oracle.Problem(**base)
+
+
+def test_linear_in_value_and_mask():
+    prob = _tiny()
+    a, Ho, Wo = rand_problem_inputs(prob, seed=1)
+    b, _, _ = rand_problem_inputs(prob, seed=2)
+    y1 = oracle.forward(prob, a["value"], a["offset_mask"])
+    y2 = oracle.forward(prob, b["value"], a["offset_mask"])
+    y12 = oracle.forward(prob, 2.5 * a["value"] - 0.75 * b["value"], a["offset_mask"])
+    assert rel_err(y12, 2.5 * y1 - 0.75 * y2) < 1e-13
+    om2 = a["offset_mask"].copy()
+    _, _, m2 = split_om(om2, prob.G, prob.K)
+    _, _, m1 = split_om(b["offset_mask"], prob.G, prob.K)
+    om_sum = a["offset_mask"].copy()
+    _, _, ms = split_om(om_sum, prob.G, prob.K)
+    ms[...] = 3.0 * m2 + m1
+    om_b = a["offset_mask"].copy()
+    _, _, mb = split_om(om_b, prob.G, prob.K)
+    mb[...] = m1
+    ya = oracle.forward(prob, a["value"], a["offset_mask"])
+    yb = oracle.forward(prob, a["value"], om_b)
+    ys = oracle.forward(prob, a["value"], om_sum)
+    assert rel_err(ys, 3.0 * ya + yb) < 1e-13
+
+
+def test_remove_center_is_zero_centre_mask():
+    p8 = _tiny(remove_center=1)
+    p9 = _tiny(remove_center=0)
+    inp, Ho, Wo = rand_problem_inputs(p8, seed=4)
+    dx8, dy8, m8 = split_om(inp["offset_mask"], p8.G, 8)
+    om9 = np.full(inp["offset_mask"].shape[:-1] + (p9.row,), np.nan)
+    dx9, dy9, m9 = split_om(om9, p9.G, 9)
+    order9 = cells(3, 3, 0)
+    order8 = cells(3, 3, 1)
+    for k8, c in enumerate(order8):
+        k9 = order9.index(c)
+        dx9[..., k9], dy9[..., k9], m9[..., k9] = dx8[..., k8], dy8[..., k8], m8[..., k8]
+    kc = order9.index((1, 1))
+    dx9[..., kc], dy9[..., kc], m9[..., kc] = 0.3, -0.2, 0.0
+    y8 = oracle.forward(p8, inp["value"], inp["offset_mask"])
+    y9 = oracle.forward(p9, inp["value"], om9)
+    np.testing.assert_array_equal(y8, y9)
+
+
+def test_offset_scale_scales_offsets_only():
+    p_half = _tiny(offset_scale=0.5)
+    p_one = _tiny(offset_scale=1.0)
+    inp, Ho, Wo = rand_problem_inputs(p_half, seed=6, offset=("normal", 0.0, 2.0))
+    om_scaled = inp["offset_mask"].copy()
+    dx, dy, _ = split_om(om_scaled, p_half.G, p_half.K)
+    dx *= 0.5
+    dy *= 0.5
+    np.testing.assert_array_equal(oracle.forward(p_half, inp["value"], inp["offset_mask"]),
+                                  oracle.forward(p_one, inp["value"], om_scaled))
+    p_odd = _tiny(offset_scale=0.3)
+    om_odd = inp["offset_mask"].copy()
+    dx, dy, _ = split_om(om_odd, p_odd.G, p_odd.K)
+    dx *= 0.3
+    dy *= 0.3
+    assert rel_err(oracle.forward(p_odd, inp["value"], inp["offset_mask"]),
+                   oracle.forward(p_one, inp["value"], om_odd)) < 1e-13
+
+
+def test_far_off_image_is_zero():
+    prob = _tiny()
+    inp, Ho, Wo = rand_problem_inputs(prob, seed=8)
+    gy = inp["grad_out"]
+    for far in (1e3, -1e3, 7.0, -2.0 - 1e-9 - 8.0):
+        om = inp["offset_mask"].copy()
+        dx, dy, _ = split_om(om, prob.G, prob.K)
+        dy[...] = far
+        y = oracle.forward(prob, inp["value"], om)
+        assert np.all(y == 0.0)
+        gv, gom = oracle.backward(prob, inp["value"], om, gy)
+        assert np.all(gv == 0.0) and np.all(gom == 0.0)
+
+
+def test_padding_tail_ignored_and_zeroed():
+    prob = _tiny(P=48)                                 # G*3K = 54 -> force a bigger row
+    prob = _tiny(P=64)
+    inp, Ho, Wo = rand_problem_inputs(prob, seed=12)
+    om_nan = inp["offset_mask"]
+    assert np.all(np.isnan(om_nan[..., prob.G * 3 * prob.K:]))
+    om_zero = om_nan.copy()
+    om_zero[..., prob.G * 3 * prob.K:] = 0.0
+    y_nan = oracle.forward(prob, inp["value"], om_nan)
+    assert np.all(np.isfinite(y_nan))
+    np.testing.assert_array_equal(y_nan, oracle.forward(prob, inp["value"], om_zero))
+    gv, gom = oracle.backward(prob, inp["value"], om_nan, inp["grad_out"])
+    assert np.all(gom[..., prob.G * 3 * prob.K:] == 0.0)
+    assert np.all(np.isfinite(gv)) and np.all(np.isfinite(gom))
+
+
+def test_storage_types_agree_on_representable_inputs():
+    """The same numbers stored as f16 / bf16 / f32 / f64 give the same result."""
+    p64 = _tiny()
+    inp, Ho, Wo = rand_problem_inputs(p64, seed=13)
+    v = gen.bf16_bits_to_f64(gen.f64_to_bf16_bits(inp["value"]))          # bf16-representable
+    om = inp["offset_mask"].copy()
+    om = np.where(np.isnan(om), 0.0, om)
+    om = np.round(om * 64.0) / 64.0                                           # exact in all 4 types
+    y64 = oracle.forward(p64, v, om)
+    for dt in ("f32", "f16", "bf16"):
+        p = _tiny(dtype=dt)
+        y = oracle.forward(p, gen.to_storage(v, dt), gen.to_storage(om, dt))
+        np.testing.assert_array_equal(y, y64)
+
+
+def test_location_fp32_mode():
+    prob = _tiny(dtype="f32", offset_scale=0.7)
+    inp, Ho, Wo = rand_problem_inputs(prob, seed=14)
+    y64 = oracle.forward(prob, inp["value"], inp["offset_mask"])
+    prob32 = _tiny(dtype="f32", offset_scale=0.7, location_fp32=True)
+    y32 = oracle.forward(prob32, inp["value"], inp["offset_mask"])
+    assert 0.0 < rel_err(y32, y64) < 1e-6
+    # integer offsets with a power-of-two scale: locations exact in both modes
+    om = inp["offset_mask"].copy()
+    dx, dy, _ = split_om(om, prob.G, prob.K)
+    dx[...] = np.round(dx)
+    dy[...] = np.round(dy)
+    pa = _tiny(dtype="f32", offset_scale=0.5)
+    pb = _tiny(dtype="f32", offset_scale=0.5, location_fp32=True)
+    np.testing.assert_array_equal(oracle.forward(pa, inp["value"], om), oracle.forward(pb, inp["value"], om))
+
+
+def test_threads_do_not_change_results():
+    prob = _tiny(N=3)
+    inp, Ho, Wo = rand_problem_inputs(prob, seed=15)
+    y1 = oracle.forward(prob, inp["value"], inp["offset_mask"], nthreads=1)
+    y4 = oracle.forward(prob, inp["value"], inp["offset_mask"], nthreads=4)
+    np.testing.assert_array_equal(y1, y4)
+    g1 = oracle.backward(prob, inp["value"], inp["offset_mask"], inp["grad_out"], nthreads=1)
+    g3 = oracle.backward(prob, inp["value"], inp["offset_mask"], inp["grad_out"], nthreads=3)
+    for a, b in zip(g1, g3):
+        np.testing.assert_array_equal(a, b)
+
+
+# ---------------------------------------------------------------------------
+# Backward
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("geom", GEOMS[:3])
+def test_grad_value_is_adjoint(geom):
+    prob = oracle.Problem(N=2, H=7, W=6, G=2, Cg=3, dtype="f64", offset_scale=0.8, **geom)
+    inp, Ho, Wo = rand_problem_inputs(prob, seed=17, offset=("normal", 0.0, 2.0))
+    rng = np.random.default_rng(0)
+    v2 = rng.normal(size=inp["value"].shape)
+    gy = inp["grad_out"]
+    gv, _ = oracle.backward(prob, inp["value"], inp["offset_mask"], gy)
+    lhs = np.sum(gy * oracle.forward(prob, v2, inp["offset_mask"]))
+    rhs = np.sum(gv * v2)
+    assert abs(lhs - rhs) <= 1e-12 * (np.sum(np.abs(gy)) * np.max(np.abs(v2)))
+    # grad_value does not depend on value (the operator is linear in value)
+    gv2, _ = oracle.backward(prob, v2, inp["offset_mask"], gy)
+    np.testing.assert_array_equal(gv, gv2)
+
+
+def test_grad_mask_identities():
+    prob = _tiny(remove_center=1, offset_scale=0.5)
+    inp, Ho, Wo = rand_problem_inputs(prob, seed=19)
+    gy = inp["grad_out"]
+    om = inp["offset_mask"]
+    y = oracle.forward(prob, inp["value"], om)
+    _, gom = oracle.backward(prob, inp["value"], om, gy)
+    _, _, m = split_om(om, prob.G, prob.K)
+    _, _, gm = split_om(gom, prob.G, prob.K)
+    assert abs(np.sum(gm * m) - np.sum(gy * y)) < 1e-12 * np.sum(np.abs(gy * y))
+    # elementwise: gm[k] = sum_c gy * S_k with S_k from a one-hot mask
+    C = prob.C
+    for k in range(prob.K):
+        om_k = om.copy()
+        _, _, mk = split_om(om_k, prob.G, prob.K)
+        mk[...] = 0.0
+        mk[..., k] = 1.0
+        S = oracle.forward(prob, inp["value"], om_k).reshape(prob.N, Ho, Wo, prob.G, prob.Cg)
+        want = np.sum(gy.reshape(prob.N, Ho, Wo, prob.G, prob.Cg) * S, axis=-1)
+        assert rel_err(gm[..., k], want) < 1e-13
+    assert C == prob.G * prob.Cg
+
+
+@pytest.mark.parametrize("scale,remove_center", [(1.0, 0), (0.5, 1), (1.3, 0)])
+def test_grad_offset_mask_finite_differences(scale, remove_center):
+    prob = oracle.Problem(N=1, H=8, W=8, G=2, Cg=4, dtype="f64", offset_scale=scale,
+                          remove_center=remove_center)
+    inp, Ho, Wo = rand_problem_inputs(prob, seed=23)
+    om = inp["offset_mask"].copy()
+    om[..., prob.G * 3 * prob.K:] = 0.0
+    dx, dy, _ = split_om(om, prob.G, prob.K)
+    # keep every location >= 1e-3 away from an integer (a cell boundary)
+    for d in (dx, dy):
+        frac = np.mod(scale * d, 1.0)
+        bad = (frac < 1e-3) | (frac > 1 - 1e-3)
+        d[bad] += 0.01
+    gy = inp["grad_out"]
+    _, gom = oracle.backward(prob, inp["value"], om, gy)
+    eps = 1e-6
+    G, K, Cg = prob.G, prob.K, prob.Cg
+    body = G * 3 * K
+    for e in range(3 * K):
+        plus, minus = om.copy(), om.copy()
+        idx = np.arange(G) * 3 * K + e
+        plus[..., idx] += eps
+        minus[..., idx] -= eps
+        yp = oracle.forward(prob, inp["value"], plus).reshape(1, Ho, Wo, G, Cg)
+        ym = oracle.forward(prob, inp["value"], minus).reshape(1, Ho, Wo, G, Cg)
+        fd = np.sum(gy.reshape(1, Ho, Wo, G, Cg) * (yp - ym), axis=-1) / (2 * eps)
+        got = gom[..., idx]
+        scale_ref = max(np.max(np.abs(gom[..., :body])), 1e-12)
+        assert np.max(np.abs(got - fd)) / scale_ref < 1e-6, f"entry {e}"
+
+
+def test_grad_offset_zero_offsets_at_border_uses_floor_cell():
+    """At an integer location the derivative is the one of the cell floor() picks."""
+    prob = oracle.Problem(N=1, H=4, W=4, G=1, Cg=1, dtype="f64")
+    value = np.arange(16, dtype=np.float64).reshape(1, 4, 4, 1) + 1.0
+    Ho, Wo = oracle.output_dims(prob)
+    om = np.zeros((1, Ho, Wo, prob.row))
+    _, _, m = split_om(om, 1, 9)
+    m[...] = 1.0
+    gy = np.zeros((1, Ho, Wo, 1))
+    gy[0, 0, 0, 0] = 1.0
+    _, gom = oracle.backward(prob, value, om, gy)
+    dxg, dyg, _ = split_om(gom, 1, 9)
+    # k = 0 is cell (ih=0, iw=0): location (-1, -1); floor cell rows {-1, 0}, cols {-1, 0}
+    # dS/dh = (1-lw)(v10 - v00) + lw(v11 - v01) with lw = 0 -> v[0,-1] - v[-1,-1] = 0 (col -1 is outside)
+    assert dyg[0, 0, 0, 0, 0] == 0.0 and dxg[0, 0, 0, 0, 0] == 0.0
+    # k = 1 is cell (ih=1, iw=0): location (0, -1): dS/dw = (1-lh)(v01 - v00) = v[0,0] - 0 = 1
+    assert dxg[0, 0, 0, 0, 1] == 1.0
+    # dS/dh = (1-lw)(v10 - v00) = v[1,-1] - v[0,-1] = 0 (column -1 is outside)
+    assert dyg[0, 0, 0, 0, 1] == 0.0
+    # k = 4 is the centre (1, 1): location (0, 0): dS/dh = v[1,0]-v[0,0] = 4, dS/dw = v[0,1]-v[0,0] = 1
+    assert dyg[0, 0, 0, 0, 4] == 4.0 and dxg[0, 0, 0, 0, 4] == 1.0
+    assert math.isfinite(float(np.sum(gom)))
