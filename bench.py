@@ -1,0 +1,423 @@
+#!/usr/bin/env python
+"""Benchmark of the DCNv4 core operator on B200: one forward + backward step.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
+                    [--workload NAME] [--no-cpu-baseline] [--no-e2e]
+
+A step is one pass of the whole path over one batch: dcn4_forward followed by
+dcn4_backward on the first-stage backbone workload (N64 H56 W56 C64 G4, C'=16,
+3x3, fp16; inputs seeded, see dcn4_inputs).  Inputs are resident in HBM; the
+L2 cache is flushed (a 256 MiB write) between timed steps, outside the timed
+events.  Each step is timed with CUDA events on the launching stream, with a
+barrier + synchronize around the K timed steps; multi-GPU runs (torchrun, one
+rank per GPU, NCCL) report the max over ranks.  Every rank runs the full
+batch: the operator is independent per image, so there is no collective on the
+data path (weak scaling, replicas).
+
+Rank 0 prints one JSON line.  value = microseconds per forward+backward step
+(lower is better); the line also carries per-kernel times, achieved HBM GB/s
+against the algorithmic byte model, the roofline of the dominant launch, an
+end-to-end figure through host buffers, clocks sampled during the timed loop,
+and a CPU-oracle baseline.
+
+--impl reference times the CPU oracle (the only other implementation of the
+operator) on the host cores, on a bounded sample of the same workload per
+step, scaled to the full batch.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import dcn4_inputs as gen  # noqa: E402
+
+METRIC = "DCNv4 core fwd/bwd µs per call and achieved HBM GB/s (% of B200 peak)"
+L2_FLUSH_BYTES = 256 << 20
+FALLBACK_HBM_GBS = 6650.0
+ELEM_BYTES = {"f32": 4, "f16": 2, "bf16": 2}
+
+
+# ---------------------------------------------------------------------------
+# Byte model (compulsory HBM traffic per call)
+# ---------------------------------------------------------------------------
+
+def byte_model(w: gen.Workload) -> dict:
+    """value + offset_mask + out (forward); + grad_out read, grad_value and
+    grad_offset_mask written (backward)."""
+    b = ELEM_BYTES[w.dtype]
+    value = w.N * w.H * w.W * w.C * b
+    om = w.N * w.Ho * w.Wo * w.P * b
+    out = w.N * w.Ho * w.Wo * w.C * b
+    return {"fwd": value + om + out, "bwd": value + om + out + value + om}
+
+
+def measured_peaks() -> dict:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return {"hbm_gbs": FALLBACK_HBM_GBS, "source": "fallback"}
+
+
+# ---------------------------------------------------------------------------
+# Clock sampling (nvidia-smi in the background during the timed loop)
+# ---------------------------------------------------------------------------
+
+CLOCK_QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+
+class ClockSampler:
+    def __init__(self, gpu_index: int, period_ms: int = 100):
+        self.samples: list[tuple[float, list[str]]] = []
+        self.proc = None
+        self.gpu_index = gpu_index
+        self.period_ms = period_ms
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={CLOCK_QUERY}", "--format=csv,noheader,nounits",
+                 f"-lms", str(self.period_ms), "-i", str(self.gpu_index)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.samples.append((time.time(), [x.strip() for x in line.split(",")]))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+
+def summarize_clocks(samples, t0: float, t1: float) -> dict:
+    """Median SM clock and the throttle reasons seen in [t0, t1] (all samples if none fall inside)."""
+    inside = [s for t, s in samples if t0 <= t <= t1]
+    window = "timed loop"
+    if not inside:
+        inside = [s for _, s in samples]
+        window = "whole run (timed loop shorter than the sampling period)"
+    if not inside:
+        return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "window": "unavailable"}
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    sm, smax, reasons = [], [], set()
+    for s in inside:
+        try:
+            sm.append(float(s[1]))
+            smax.append(float(s[2]))
+        except (ValueError, IndexError):
+            continue
+        for i, n in enumerate(names):
+            if len(s) > 5 + i and s[5 + i].lower().startswith("active"):
+                reasons.add(n)
+    return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+            "reasons": sorted(reasons), "samples": len(inside), "window": window}
+
+
+# ---------------------------------------------------------------------------
+# Distributed plumbing
+# ---------------------------------------------------------------------------
+
+def dist_env() -> tuple[int, int, int]:
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def max_over_ranks(x: float, device=None) -> float:
+    """Max of a per-rank scalar (identity when not distributed)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(device=None):
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        if device is not None and device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (baseline / reference arm)
+# ---------------------------------------------------------------------------
+
+def time_oracle(w: gen.Workload, images: int, inp=None) -> dict:
+    """Forward + backward of the oracle on `images` images of the workload,
+    scaled to µs per full-batch call."""
+    import oracle
+    threads = oracle.host_threads()
+    sub = gen.custom(**{**w.__dict__, "N": images, "name": w.name + "_sample"})
+    if inp is None:
+        inp = gen.make_inputs(sub, tail_fill=0.0)
+    prob = oracle.Problem(dtype=w.dtype, location_fp32=True, **sub.geometry())
+    t0 = time.perf_counter()
+    oracle.forward(prob, inp["value"], inp["offset_mask"], nthreads=threads)
+    oracle.backward(prob, inp["value"], inp["offset_mask"], inp["grad_out"], nthreads=threads)
+    dt = time.perf_counter() - t0
+    us_full = dt * 1e6 * w.N / images
+    return {"value": round(us_full, 1), "unit": "us/call", "cores": threads, "kind": "oracle",
+            "sample": f"forward+backward of {images} of {w.N} images, {threads} threads, "
+                      f"{dt:.2f} s, scaled x{w.N / images:g} to the full batch",
+            "seconds": dt}
+
+
+def oracle_sample_images(w: gen.Workload, target_s: float = 15.0) -> int:
+    """Images of the workload the oracle handles in about target_s seconds."""
+    probe = time_oracle(w, 1)
+    per = max(probe["seconds"], 1e-3)
+    return int(max(1, min(w.N, target_s // per)))
+
+
+def run_reference(args, w: gen.Workload) -> dict:
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return {}
+    imgs = max(1, min(w.N, args.reference_images))
+    sub = gen.custom(**{**w.__dict__, "N": imgs, "name": w.name + "_sample"})
+    inp = gen.make_inputs(sub, tail_fill=0.0)
+    for _ in range(args.warmup):
+        time_oracle(w, imgs, inp)
+    times = [time_oracle(w, imgs, inp) for _ in range(args.steps)]
+    us = statistics.mean(t["value"] for t in times)
+    cb = dict(times[0])
+    cb["value"] = round(us, 1)
+    cb.pop("seconds", None)
+    cb["sample"] = f"each step: forward+backward of {imgs} of {w.N} images, scaled to the full batch"
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(us, 1), "unit": "us/call",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(us / 1e3, 4),
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": f"{w.name}: {w.describe()}, forward+backward",
+                                        "parallelism": "oracle on host cores"},
+        "cpu_baseline": cb,
+        "e2e": {"value": round(us, 1), "unit": "us/call", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+# ---------------------------------------------------------------------------
+# Native arm
+# ---------------------------------------------------------------------------
+
+def run_native(args, w: gen.Workload) -> dict:
+    import torch
+    import torch.distributed as dist
+
+    rank, world, local = dist_env()
+    if world > 1:
+        torch.cuda.set_device(local)
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+
+    import deformable_convolution_sampling_b200 as dcn
+
+    tdt = {"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16}[w.dtype]
+    inp = gen.make_inputs(w, tail_fill=0.0)
+
+    def host_tensor(a):
+        import numpy as np
+        a = np.ascontiguousarray(a)
+        t = torch.from_numpy(a.view(np.int16)).view(tdt) if w.dtype == "bf16" else torch.from_numpy(a)
+        return t.pin_memory()
+
+    h_v, h_om, h_gy = host_tensor(inp["value"]), host_tensor(inp["offset_mask"]), host_tensor(inp["grad_out"])
+    v, om, gy = h_v.to(dev), h_om.to(dev), h_gy.to(dev)
+    p = dcn.make_params(dtype=w.dtype, **w.geometry())
+    st, Ho, Wo = dcn.dcn4_output_dims(p)
+    dcn.check(st)
+    out = torch.empty((w.N, Ho, Wo, w.C), dtype=tdt, device=dev)
+    gv = torch.empty_like(v)
+    gom = torch.empty((w.N, Ho, Wo, w.P), dtype=tdt, device=dev)
+    ws_bytes = dcn.dcn4_backward_workspace_size(p)
+    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    sh = stream.cuda_stream
+    ptr = dict(v=v.data_ptr(), om=om.data_ptr(), gy=gy.data_ptr(), out=out.data_ptr(), gv=gv.data_ptr(),
+               gom=gom.data_ptr(), ws=ws.data_ptr())
+
+    def fwd():
+        dcn.check(dcn.dcn4_forward(p, ptr["v"], ptr["om"], ptr["out"], sh))
+
+    def bwd():
+        dcn.check(dcn.dcn4_backward(p, ptr["v"], ptr["om"], ptr["gy"], ptr["gv"], ptr["gom"], ptr["ws"],
+                                    ws_bytes, sh))
+
+    launches_per_step = 1 + (2 if w.dtype != "f32" else 1)  # forward; backward kernel (+ finalize)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        fwd()
+        bwd()
+    torch.cuda.synchronize(dev)
+
+    sampler = ClockSampler(local if world > 1 else torch.cuda.current_device())
+    sampler.start()
+    time.sleep(0.3)
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    barrier(dev)
+    torch.cuda.synchronize(dev)
+    t0 = time.time()
+    for i in range(K):
+        flush.zero_()
+        ev[i][0].record(stream)
+        fwd()
+        ev[i][1].record(stream)
+        bwd()
+        ev[i][2].record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(dev)
+    t1 = time.time()
+    time.sleep(0.25)
+    sampler.stop()
+
+    fwd_ms = [e[0].elapsed_time(e[1]) for e in ev]
+    bwd_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    step_ms = statistics.mean(f + b for f, b in zip(fwd_ms, bwd_ms))
+    step_ms_max = max_over_ranks(step_ms, dev)
+    fwd_us = max_over_ranks(statistics.mean(fwd_ms) * 1e3, dev)
+    bwd_us = max_over_ranks(statistics.mean(bwd_ms) * 1e3, dev)
+
+    # End to end through host buffers: pinned host -> device copies of the
+    # inputs, forward + backward, device -> pinned host copies of the results.
+    e2e = None
+    if not args.no_e2e:
+        h_out = torch.empty(out.shape, dtype=tdt).pin_memory()
+        h_gv = torch.empty(gv.shape, dtype=tdt).pin_memory()
+        h_gom = torch.empty(gom.shape, dtype=tdt).pin_memory()
+
+        def e2e_step():
+            v.copy_(h_v, non_blocking=True)
+            om.copy_(h_om, non_blocking=True)
+            gy.copy_(h_gy, non_blocking=True)
+            fwd()
+            bwd()
+            h_out.copy_(out, non_blocking=True)
+            h_gv.copy_(gv, non_blocking=True)
+            h_gom.copy_(gom, non_blocking=True)
+
+        for _ in range(max(3, args.warmup // 10)):
+            e2e_step()
+        ke = max(3, min(K, 50))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(dev)
+        torch.cuda.synchronize(dev)
+        e0.record(stream)
+        for _ in range(ke):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_us = max_over_ranks(e0.elapsed_time(e1) * 1e3 / ke, dev)
+        bi = sum(t.numel() * t.element_size() for t in (h_v, h_om, h_gy))
+        bo = sum(t.numel() * t.element_size() for t in (h_out, h_gv, h_gom))
+        e2e = {"value": round(e2e_us, 2), "unit": "us/call", "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo,
+               "steps": ke}
+
+    bm = byte_model(w)
+    peaks = measured_peaks()
+    fwd_gbs = bm["fwd"] / (fwd_us * 1e-6) / 1e9
+    bwd_gbs = bm["bwd"] / (bwd_us * 1e-6) / 1e9
+    step_gbs = (bm["fwd"] + bm["bwd"]) / (step_ms_max * 1e-3) / 1e9
+    dominant = "bwd" if bwd_us >= fwd_us else "fwd"
+    dom_gbs = bwd_gbs if dominant == "bwd" else fwd_gbs
+    roofline = {
+        "bound": "hbm", "kernel": "dcn4_backward (accumulator memset + gradient kernel + fp32->dtype finalize)"
+        if dominant == "bwd" else "dcn4_forward kernel",
+        "achieved": round(dom_gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+        "frac": round(dom_gbs / peaks["hbm_gbs"], 4), "peak_source": peaks["source"],
+        "traffic": args.traffic_bytes,
+        "algorithmic_bytes": bm[dominant],
+    }
+
+    clocks = summarize_clocks(sampler.samples, t0, t1)
+    result = {
+        "metric": METRIC, "value": round(step_ms_max * 1e3, 2), "unit": "us/call",
+        "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": round(step_ms_max, 5),
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
+        "data": "synthetic",
+        "config": {"workload": f"{w.name}: {w.describe()}, forward+backward",
+                   "global_batch": w.N * world, "parallelism": f"replicas x{world} (batch per GPU {w.N})",
+                   "l2": "flushed between timed steps (256 MiB write outside the events)"},
+        "fwd_us": round(fwd_us, 2), "bwd_us": round(bwd_us, 2),
+        "fwd_gbs": round(fwd_gbs, 1), "bwd_gbs": round(bwd_gbs, 1), "step_gbs": round(step_gbs, 1),
+        "fwd_frac_hbm": round(fwd_gbs / peaks["hbm_gbs"], 4), "bwd_frac_hbm": round(bwd_gbs / peaks["hbm_gbs"], 4),
+        "fwd_frac_8tbs": round(fwd_gbs / 8000.0, 4), "bwd_frac_8tbs": round(bwd_gbs / 8000.0, 4),
+        "bytes_per_call": bm,
+        "roofline": roofline,
+        "gpu_launches": launches_per_step * K,
+        "clocks": clocks,
+    }
+    if e2e is not None:
+        result["e2e"] = e2e
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        n_img = oracle_sample_images(w, args.cpu_seconds)
+        cb = time_oracle(w, n_img)
+        cb.pop("seconds", None)
+        result["cpu_baseline"] = cb
+    if world > 1:
+        dist.destroy_process_group()
+    return result
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--workload", default="stage1_f16", choices=sorted(gen.WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0,
+                    help="target seconds of oracle work for the cpu_baseline sample")
+    ap.add_argument("--reference-images", type=int, default=1,
+                    help="images of the batch the reference arm runs per step")
+    ap.add_argument("--traffic-bytes", type=float, default=None,
+                    help="DRAM bytes per launch of the dominant kernel from an ncu capture (null if unknown)")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    w = gen.WORKLOADS[args.workload]
+    rank, world, _ = dist_env()
+    if args.impl == "reference":
+        res = run_reference(args, w)
+    else:
+        res = run_native(args, w)
+    if rank == 0 and res:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

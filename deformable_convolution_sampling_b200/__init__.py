@@ -1,0 +1,193 @@
+"""Python binding of libdcn4, the sm_100a DCNv4 core spatial aggregation.
+
+The C ABI (include/dcn4.h) is exposed under the same names -- ``dcn4_forward``,
+``dcn4_backward``, ``dcn4_output_dims`` ... -- taking a :class:`dcn4_params`
+and raw device pointers.  They only marshal arguments: every step of the
+operator runs in the library's CUDA kernels.  There is no CPU fallback; if the
+library is not built, importing this package fails.
+
+``forward`` / ``backward`` are conveniences over the same calls for torch
+tensors (torch provides device memory and streams only).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libdcn4.so")
+
+DCN4_F32, DCN4_F16, DCN4_BF16 = 0, 1, 2
+STATUS = {
+    0: "DCN4_OK", -1: "DCN4_ERR_NULL", -2: "DCN4_ERR_BAD_SHAPE", -3: "DCN4_ERR_BAD_P",
+    -4: "DCN4_ERR_MISALIGNED", -5: "DCN4_ERR_UNSUPPORTED", -6: "DCN4_ERR_WORKSPACE",
+    -7: "DCN4_ERR_LAUNCH", -8: "DCN4_ERR_DTYPE",
+}
+DTYPE_NAMES = {"f32": DCN4_F32, "f16": DCN4_F16, "bf16": DCN4_BF16}
+
+
+class Dcn4Error(RuntimeError):
+    def __init__(self, status: int, detail: str):
+        super().__init__(f"{STATUS.get(status, status)}: {detail}")
+        self.status = status
+
+
+class dcn4_params(ctypes.Structure):
+    """Mirror of the C struct dcn4_params."""
+
+    _fields_ = [
+        ("N", ctypes.c_int), ("H", ctypes.c_int), ("W", ctypes.c_int),
+        ("G", ctypes.c_int), ("Cg", ctypes.c_int),
+        ("kh", ctypes.c_int), ("kw", ctypes.c_int),
+        ("sh", ctypes.c_int), ("sw", ctypes.c_int),
+        ("ph", ctypes.c_int), ("pw", ctypes.c_int),
+        ("dh", ctypes.c_int), ("dw", ctypes.c_int),
+        ("offset_scale", ctypes.c_float),
+        ("remove_center", ctypes.c_int),
+        ("P", ctypes.c_int),
+        ("dtype", ctypes.c_int),
+    ]
+
+
+def make_params(*, N, H, W, G, Cg, kh=3, kw=3, sh=1, sw=1, ph=1, pw=1, dh=1, dw=1,
+                offset_scale=1.0, remove_center=0, P=None, dtype="f32") -> dcn4_params:
+    """Build a dcn4_params; P defaults to the smallest valid padded row."""
+    if isinstance(dtype, str):
+        dtype = DTYPE_NAMES[dtype]
+    if P is None:
+        P = dcn4_padded_offset_dim(G, kh * kw - (1 if remove_center else 0))
+    return dcn4_params(N, H, W, G, Cg, kh, kw, sh, sw, ph, pw, dh, dw, float(offset_scale),
+                       1 if remove_center else 0, P, dtype)
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is not built; run `python deformable_convolution_sampling_b200/build.py` "
+            "(there is no CPU fallback)")
+    L = ctypes.CDLL(LIB_PATH)
+    P = ctypes.POINTER(dcn4_params)
+    vp, ip = ctypes.c_void_p, ctypes.POINTER(ctypes.c_int)
+    sig = {
+        "dcn4_version": ([], ctypes.c_int),
+        "dcn4_num_points": ([P], ctypes.c_int),
+        "dcn4_padded_offset_dim": ([ctypes.c_int, ctypes.c_int], ctypes.c_int),
+        "dcn4_output_dims": ([P, ip, ip], ctypes.c_int),
+        "dcn4_check_params": ([P], ctypes.c_int),
+        "dcn4_forward": ([P, vp, vp, vp, vp], ctypes.c_int),
+        "dcn4_backward_workspace_size": ([P], ctypes.c_size_t),
+        "dcn4_backward": ([P, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp], ctypes.c_int),
+        "dcn4_status_string": ([ctypes.c_int], ctypes.c_char_p),
+        "dcn4_last_error": ([], ctypes.c_char_p),
+    }
+    for name, (args, res) in sig.items():
+        fn = getattr(L, name)
+        fn.argtypes = args
+        fn.restype = res
+    return L
+
+
+lib = _load()
+
+
+# ---------------------------------------------------------------------------
+# Same-name wrappers of the C ABI (pointers are ints or None; stream is a
+# cudaStream_t handle as an int, 0 / None for the legacy default stream).
+# ---------------------------------------------------------------------------
+
+def dcn4_version() -> int:
+    return lib.dcn4_version()
+
+
+def dcn4_num_points(p: dcn4_params) -> int:
+    return lib.dcn4_num_points(ctypes.byref(p))
+
+
+def dcn4_padded_offset_dim(G: int, K: int) -> int:
+    return lib.dcn4_padded_offset_dim(G, K)
+
+
+def dcn4_output_dims(p: dcn4_params) -> tuple[int, int, int]:
+    ho, wo = ctypes.c_int(), ctypes.c_int()
+    st = lib.dcn4_output_dims(ctypes.byref(p), ctypes.byref(ho), ctypes.byref(wo))
+    return st, ho.value, wo.value
+
+
+def dcn4_check_params(p: dcn4_params) -> int:
+    return lib.dcn4_check_params(ctypes.byref(p))
+
+
+def dcn4_forward(p: dcn4_params, value, offset_mask, out, stream=None) -> int:
+    return lib.dcn4_forward(ctypes.byref(p), value, offset_mask, out, stream)
+
+
+def dcn4_backward_workspace_size(p: dcn4_params) -> int:
+    return lib.dcn4_backward_workspace_size(ctypes.byref(p))
+
+
+def dcn4_backward(p: dcn4_params, value, offset_mask, grad_out, grad_value, grad_offset_mask,
+                  workspace, workspace_bytes: int, stream=None) -> int:
+    return lib.dcn4_backward(ctypes.byref(p), value, offset_mask, grad_out, grad_value,
+                             grad_offset_mask, workspace, workspace_bytes, stream)
+
+
+def dcn4_status_string(status: int) -> str:
+    return lib.dcn4_status_string(status).decode()
+
+
+def dcn4_last_error() -> str:
+    return lib.dcn4_last_error().decode()
+
+
+def check(status: int) -> None:
+    """Raise Dcn4Error for a negative status."""
+    if status != 0:
+        raise Dcn4Error(status, dcn4_last_error())
+
+
+# ---------------------------------------------------------------------------
+# torch conveniences (device memory and the current stream come from torch)
+# ---------------------------------------------------------------------------
+
+def _torch_dtype(code: int):
+    import torch
+    return {DCN4_F32: torch.float32, DCN4_F16: torch.float16, DCN4_BF16: torch.bfloat16}[code]
+
+
+def _stream_handle(device):
+    import torch
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def forward(p: dcn4_params, value, offset_mask, out=None):
+    """y[N,Ho,Wo,C] for CUDA tensors value[N,H,W,C] and offset_mask[N,Ho,Wo,P]."""
+    import torch
+    st, Ho, Wo = dcn4_output_dims(p)
+    check(st)
+    if out is None:
+        out = torch.empty((p.N, Ho, Wo, p.G * p.Cg), dtype=_torch_dtype(p.dtype), device=value.device)
+    check(dcn4_forward(p, value.data_ptr(), offset_mask.data_ptr(), out.data_ptr(),
+                       _stream_handle(value.device)))
+    return out
+
+
+def backward(p: dcn4_params, value, offset_mask, grad_out, grad_value=None, grad_offset_mask=None,
+             workspace=None):
+    """(grad_value[N,H,W,C], grad_offset_mask[N,Ho,Wo,P]) for CUDA tensors."""
+    import torch
+    st, Ho, Wo = dcn4_output_dims(p)
+    check(st)
+    dt = _torch_dtype(p.dtype)
+    if grad_value is None:
+        grad_value = torch.empty_like(value, dtype=dt)
+    if grad_offset_mask is None:
+        grad_offset_mask = torch.empty((p.N, Ho, Wo, p.P), dtype=dt, device=value.device)
+    need = dcn4_backward_workspace_size(p)
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=value.device)
+    ws_ptr = workspace.data_ptr() if workspace is not None else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    check(dcn4_backward(p, value.data_ptr(), offset_mask.data_ptr(), grad_out.data_ptr(),
+                        grad_value.data_ptr(), grad_offset_mask.data_ptr(), ws_ptr, ws_bytes,
+                        _stream_handle(value.device)))
+    return grad_value, grad_offset_mask

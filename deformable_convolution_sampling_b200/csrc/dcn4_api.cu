@@ -1,0 +1,263 @@
+// dcn4_api.cu — the C ABI of libdcn4 (declared in include/dcn4.h).
+//
+// Host side only: validates a call completely before anything reaches the GPU,
+// derives the launch geometry from the shape (no tuning tables), and launches
+// the kernels of dcn4_forward.cu / dcn4_backward.cu on the caller's stream.
+#include <cmath>
+#include <cstdarg>
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+
+#include <algorithm>
+
+#include "dcn4.h"
+#include "dcn4_common.cuh"
+
+namespace {
+
+thread_local char g_last_error[512] = "";
+
+int fail(int status, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+int fail(int status, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_last_error, sizeof g_last_error, fmt, ap);
+    va_end(ap);
+    return status;
+}
+
+int elem_bytes(int dtype) { return dtype == DCN4_F32 ? 4 : 2; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned32(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
+
+// Threads of one CTA aim at 256: enough warps per SM to hide gather latency
+// while keeping each CTA's offset_mask rows small in shared memory.
+constexpr int kTargetThreads = 256;
+constexpr size_t kSmemDefault = 48 * 1024;
+constexpr size_t kSmemMax = 227 * 1024;
+// grad_value pass: up to 1024 threads and 256 input pixels per CTA; sample
+// records get what is left of this shared-memory budget after the bins.
+constexpr int kValueThreads = 1024;
+constexpr int kValuePixels = 256;
+constexpr size_t kValueSmem = 200 * 1024;
+
+// Validates p and fills the kernel geometry.  Touches no GPU state.
+// wide: the gathered and stored tensors are 32-byte aligned, so a thread may
+// move a 32-byte channel slice with one 256-bit access.
+int make_geometry(const dcn4_params* p, bool backward, bool wide, dcn4::Geometry* g) {
+    if (!p) return fail(DCN4_ERR_NULL, "params is NULL");
+    if (p->dtype != DCN4_F32 && p->dtype != DCN4_F16 && p->dtype != DCN4_BF16)
+        return fail(DCN4_ERR_DTYPE, "dtype %d is not a dcn4_dtype", p->dtype);
+    if (p->N < 0 || p->H < 1 || p->W < 1 || p->G < 1 || p->Cg < 1)
+        return fail(DCN4_ERR_BAD_SHAPE, "need N >= 0 and H, W, G, Cg >= 1 (got N=%d H=%d W=%d G=%d Cg=%d)", p->N, p->H,
+                    p->W, p->G, p->Cg);
+    if (p->kh < 1 || p->kw < 1 || p->sh < 1 || p->sw < 1 || p->dh < 1 || p->dw < 1 || p->ph < 0 || p->pw < 0)
+        return fail(DCN4_ERR_BAD_SHAPE, "need kernel, stride, dilation >= 1 and padding >= 0");
+    if (p->remove_center != 0 && p->remove_center != 1)
+        return fail(DCN4_ERR_BAD_SHAPE, "remove_center must be 0 or 1");
+    if (p->remove_center && (p->kh % 2 == 0 || p->kw % 2 == 0))
+        return fail(DCN4_ERR_BAD_SHAPE, "remove_center needs odd kh and kw");
+    if (!std::isfinite(p->offset_scale)) return fail(DCN4_ERR_BAD_SHAPE, "offset_scale is not finite");
+    if (static_cast<long long>(p->kh) * p->kw > 1024) return fail(DCN4_ERR_UNSUPPORTED, "kh*kw > 1024");
+    const int K = p->kh * p->kw - p->remove_center;
+    if (K < 1) return fail(DCN4_ERR_BAD_SHAPE, "no sampling point left");
+    const long long body = 3LL * p->G * K;
+    if (body > (1LL << 30) || p->P < body || p->P % 8 != 0)
+        return fail(DCN4_ERR_BAD_P, "P=%d must be a multiple of 8 and >= G*3K=%lld", p->P, body);
+    const long long eff_h = static_cast<long long>(p->dh) * (p->kh - 1) + 1;
+    const long long eff_w = static_cast<long long>(p->dw) * (p->kw - 1) + 1;
+    const long long num_h = p->H + 2LL * p->ph - eff_h, num_w = p->W + 2LL * p->pw - eff_w;
+    if (num_h < 0 || num_w < 0) return fail(DCN4_ERR_BAD_SHAPE, "the kernel grid does not fit the padded input");
+    const long long Ho = num_h / p->sh + 1, Wo = num_w / p->sw + 1;
+    if (p->H >= (1 << 24) || p->W >= (1 << 24) || Ho >= (1 << 24) || Wo >= (1 << 24))
+        return fail(DCN4_ERR_UNSUPPORTED, "H, W, Ho, Wo must be < 2^24");
+    if (p->ph >= (1 << 24) || p->pw >= (1 << 24) || eff_h >= (1 << 24) || eff_w >= (1 << 24) ||
+        static_cast<long long>(p->sh) * Ho >= (1 << 24) || static_cast<long long>(p->sw) * Wo >= (1 << 24))
+        return fail(DCN4_ERR_UNSUPPORTED, "grid coordinates must stay below 2^24");
+    const long long C = static_cast<long long>(p->G) * p->Cg;
+    if (static_cast<long long>(p->H) * p->W * C >= (1LL << 31))
+        return fail(DCN4_ERR_UNSUPPORTED, "H*W*C must be < 2^31 per image");
+    const int eb = elem_bytes(p->dtype);
+    const long long slice_bytes = static_cast<long long>(p->Cg) * eb;
+    if (slice_bytes % 16 != 0)
+        return fail(DCN4_ERR_UNSUPPORTED, "Cg*sizeof(dtype)=%lld must be a multiple of 16 bytes", slice_bytes);
+    const long long vec = (wide && slice_bytes % 32 == 0) ? 2 : 1;
+    const long long nslice = slice_bytes / (16 * vec);
+    if (nslice > 32 || (nslice & (nslice - 1)) != 0)
+        return fail(DCN4_ERR_UNSUPPORTED, "Cg*sizeof(dtype)/32 must be a power of two <= 32 (Cg=%d)", p->Cg);
+    const long long lanes_pp = p->G * nslice;
+    if (lanes_pp > kTargetThreads)
+        return fail(DCN4_ERR_UNSUPPORTED, "G * slices per group = %lld exceeds %d threads", lanes_pp, kTargetThreads);
+    const long long total_pix = static_cast<long long>(p->N) * Ho * Wo;
+    if (Ho * Wo >= (1LL << 31)) return fail(DCN4_ERR_UNSUPPORTED, "Ho*Wo must be < 2^31");
+    if (total_pix > (1LL << 40)) return fail(DCN4_ERR_UNSUPPORTED, "N*Ho*Wo too large");
+
+    // Output pixels per CTA: fill kTargetThreads, then shrink until the
+    // shared-memory rows fit the default 48 KB (or, for very long rows, the
+    // per-CTA maximum).
+    const size_t row_bytes = static_cast<size_t>(p->P) * (eb + (backward ? 4 : 0));
+    long long ppc = kTargetThreads / lanes_pp;
+    while (ppc > 1 && ppc * row_bytes > kSmemDefault) --ppc;
+    if (ppc * row_bytes > kSmemMax) return fail(DCN4_ERR_UNSUPPORTED, "P=%d rows do not fit shared memory", p->P);
+    // A CTA covers a TH x TW tile of output pixels of one image: as square as
+    // the pixel budget allows (TW a power of two), clipped to the image.
+    long long TW = 1;
+    while (TW * TW < ppc && TW * 2 <= ppc) TW *= 2;
+    while (TW > 1 && TW / 2 >= Wo) TW /= 2;
+    long long TH = ppc / TW;
+    if (TH > Ho) TH = Ho;
+    const long long tiles_h = (Ho + TH - 1) / TH, tiles_w = (Wo + TW - 1) / TW;
+    if (static_cast<long long>(p->N) * tiles_h * tiles_w > 0x7fffffffLL)
+        return fail(DCN4_ERR_UNSUPPORTED, "grid too large");
+
+    g->N = p->N; g->H = p->H; g->W = p->W; g->G = p->G; g->Cg = p->Cg; g->C = static_cast<int>(C);
+    g->Ho = static_cast<int>(Ho); g->Wo = static_cast<int>(Wo); g->P = p->P; g->K = K;
+    g->kh = p->kh; g->kw = p->kw; g->sh = p->sh; g->sw = p->sw; g->ph = p->ph; g->pw = p->pw;
+    g->dh = p->dh; g->dw = p->dw; g->s = p->offset_scale; g->remove_center = p->remove_center;
+    g->vec = static_cast<int>(vec);
+    g->nslice = static_cast<int>(nslice);
+    g->pix_per_cta = static_cast<int>(TH * TW);
+    g->total_pix = total_pix;
+    g->TH = static_cast<int>(TH);
+    g->TW = static_cast<int>(TW);
+    g->tiles_h = static_cast<int>(tiles_h);
+    g->tiles_w = static_cast<int>(tiles_w);
+
+    // grad_value pass: BH x BW input pixels per CTA (all groups).
+    long long bpix = std::min<long long>(kValuePixels, kValueThreads / lanes_pp);
+    long long BW = 1;
+    while (BW * BW < bpix && BW * 2 <= bpix) BW *= 2;
+    while (BW > 1 && BW / 2 >= p->W) BW /= 2;
+    long long BH = std::max<long long>(1, bpix / BW);
+    if (BH > p->H) BH = p->H;
+    long long bthreads = (BH * BW * lanes_pp + 31) / 32 * 32;
+    const long long GK = static_cast<long long>(p->G) * K;
+    if (GK > kValueThreads) return fail(DCN4_ERR_UNSUPPORTED, "G*K = %lld exceeds %d", GK, kValueThreads);
+    if (bthreads < GK) bthreads = (GK + 31) / 32 * 32;
+    const long long nbins = static_cast<long long>(p->G) * (BH + 1) * (BW + 1);
+    const long long bin_bytes = (2 * nbins * 4 + 15) / 16 * 16;
+    if (bin_bytes + 1024 * 16 > static_cast<long long>(kValueSmem))
+        return fail(DCN4_ERR_UNSUPPORTED, "too many groups for the grad_value tile");
+    // Records: room for about twice the expected number of samples per tile
+    // (K per cell for every output pixel per input pixel), within the budget.
+    const long long expect = nbins * K * std::max<long long>(1, (Ho * Wo + p->H * p->W - 1) / (p->H * p->W));
+    long long bcap = (static_cast<long long>(kValueSmem) - bin_bytes) / 16;
+    bcap = std::max<long long>(1024, std::min(bcap, 2 * expect));
+    const long long btiles_h = (p->H + BH - 1) / BH, btiles_w = (p->W + BW - 1) / BW;
+    if (static_cast<long long>(p->N) * btiles_h * btiles_w > 0x7fffffffLL)
+        return fail(DCN4_ERR_UNSUPPORTED, "grid too large");
+    g->BH = static_cast<int>(BH);
+    g->BW = static_cast<int>(BW);
+    g->btiles_h = static_cast<int>(btiles_h);
+    g->btiles_w = static_cast<int>(btiles_w);
+    g->bthreads = static_cast<int>(bthreads);
+    g->bcap = static_cast<int>(bcap);
+    return DCN4_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int dcn4_version(void) { return DCN4_VERSION; }
+
+int dcn4_num_points(const dcn4_params* p) {
+    if (!p) return fail(DCN4_ERR_NULL, "params is NULL");
+    if (p->kh < 1 || p->kw < 1 || (p->remove_center != 0 && p->remove_center != 1))
+        return fail(DCN4_ERR_BAD_SHAPE, "bad kernel size or remove_center");
+    const int K = p->kh * p->kw - p->remove_center;
+    return K >= 1 ? K : fail(DCN4_ERR_BAD_SHAPE, "no sampling point left");
+}
+
+int dcn4_padded_offset_dim(int G, int K) {
+    if (G < 1 || K < 1 || static_cast<long long>(G) * K > (1LL << 28))
+        return fail(DCN4_ERR_BAD_SHAPE, "need G >= 1 and K >= 1");
+    return (G * 3 * K + 7) / 8 * 8;
+}
+
+int dcn4_output_dims(const dcn4_params* p, int* Ho, int* Wo) {
+    if (!Ho || !Wo) return fail(DCN4_ERR_NULL, "Ho/Wo is NULL");
+    dcn4::Geometry g;
+    const int st = make_geometry(p, false, true, &g);
+    if (st != DCN4_OK) return st;
+    *Ho = g.Ho;
+    *Wo = g.Wo;
+    return DCN4_OK;
+}
+
+int dcn4_check_params(const dcn4_params* p) {
+    dcn4::Geometry g;
+    for (int backward = 0; backward < 2; ++backward)
+        for (int wide = 0; wide < 2; ++wide) {
+            const int st = make_geometry(p, backward, wide, &g);
+            if (st != DCN4_OK) return st;
+        }
+    return DCN4_OK;
+}
+
+int dcn4_forward(const dcn4_params* p, const void* value, const void* offset_mask, void* out, void* stream) {
+    dcn4::Geometry g;
+    const int st = make_geometry(p, false, aligned32(value) && aligned32(out), &g);
+    if (st != DCN4_OK) return st;
+    if (g.total_pix == 0) return DCN4_OK;
+    if (!value || !offset_mask || !out) return fail(DCN4_ERR_NULL, "value, offset_mask and out must be non-NULL");
+    if (!aligned16(value) || !aligned16(offset_mask) || !aligned16(out))
+        return fail(DCN4_ERR_MISALIGNED, "value, offset_mask and out must be 16-byte aligned");
+    const cudaError_t e =
+        dcn4::launch_forward(g, p->dtype, value, offset_mask, out, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return fail(DCN4_ERR_LAUNCH, "forward launch: %s", cudaGetErrorString(e));
+    return DCN4_OK;
+}
+
+size_t dcn4_backward_workspace_size(const dcn4_params* p) {
+    dcn4::Geometry g;
+    if (make_geometry(p, true, true, &g) != DCN4_OK) return 0;
+    return (static_cast<size_t>(g.N) * sizeof(int) + 255) / 256 * 256;  // one reach word per image
+}
+
+int dcn4_backward(const dcn4_params* p, const void* value, const void* offset_mask, const void* grad_out,
+                  void* grad_value, void* grad_offset_mask, void* workspace, size_t workspace_bytes, void* stream) {
+    dcn4::Geometry g;
+    const int st = make_geometry(p, true, aligned32(value) && aligned32(grad_out) && aligned32(grad_value), &g);
+    if (st != DCN4_OK) return st;
+    if (g.total_pix == 0) return DCN4_OK;
+    if (!value || !offset_mask || !grad_out || !grad_value || !grad_offset_mask)
+        return fail(DCN4_ERR_NULL, "value, offset_mask, grad_out, grad_value and grad_offset_mask must be non-NULL");
+    if (!aligned16(value) || !aligned16(offset_mask) || !aligned16(grad_out) || !aligned16(grad_value) ||
+        !aligned16(grad_offset_mask))
+        return fail(DCN4_ERR_MISALIGNED, "tensor pointers must be 16-byte aligned");
+    const size_t need = dcn4_backward_workspace_size(p);
+    if (!workspace || workspace_bytes < need)
+        return fail(DCN4_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, workspace_bytes);
+    if (!aligned16(workspace)) return fail(DCN4_ERR_MISALIGNED, "workspace must be 16-byte aligned");
+    int* reach = static_cast<int*>(workspace);
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemsetAsync(reach, 0xff, static_cast<size_t>(g.N) * sizeof(int), s);  // reach = -1
+    if (e != cudaSuccess) return fail(DCN4_ERR_LAUNCH, "reach reset: %s", cudaGetErrorString(e));
+    e = dcn4::launch_backward_samples(g, p->dtype, value, offset_mask, grad_out, grad_offset_mask, reach, s);
+    if (e != cudaSuccess) return fail(DCN4_ERR_LAUNCH, "grad_offset_mask launch: %s", cudaGetErrorString(e));
+    e = dcn4::launch_backward_value(g, p->dtype, offset_mask, grad_out, grad_value, reach, s);
+    if (e != cudaSuccess) return fail(DCN4_ERR_LAUNCH, "grad_value launch: %s", cudaGetErrorString(e));
+    return DCN4_OK;
+}
+
+const char* dcn4_status_string(int status) {
+    switch (status) {
+        case DCN4_OK: return "DCN4_OK";
+        case DCN4_ERR_NULL: return "DCN4_ERR_NULL";
+        case DCN4_ERR_BAD_SHAPE: return "DCN4_ERR_BAD_SHAPE";
+        case DCN4_ERR_BAD_P: return "DCN4_ERR_BAD_P";
+        case DCN4_ERR_MISALIGNED: return "DCN4_ERR_MISALIGNED";
+        case DCN4_ERR_UNSUPPORTED: return "DCN4_ERR_UNSUPPORTED";
+        case DCN4_ERR_WORKSPACE: return "DCN4_ERR_WORKSPACE";
+        case DCN4_ERR_LAUNCH: return "DCN4_ERR_LAUNCH";
+        case DCN4_ERR_DTYPE: return "DCN4_ERR_DTYPE";
+        default: return "DCN4_UNKNOWN_STATUS";
+    }
+}
+
+const char* dcn4_last_error(void) { return g_last_error; }
+
+}  // extern "C"

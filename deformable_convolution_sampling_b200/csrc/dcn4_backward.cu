@@ -1,0 +1,513 @@
+// dcn4_backward.cu — gradients of the DCNv4 core spatial aggregation.
+//
+// For every sample (output pixel p, group g, point k) with location
+// (h, w) = anchor + s*(dy, dx), bilinear cell corners v_ab and weights
+// w_ab = (a ? lh : 1-lh)(b ? lw : 1-lw), and gy = grad_out of (p, g):
+//   d/d m_k   = <gy, S>,                        S = sum_ab w_ab v_ab
+//   d/d dx_k  = s * m_k * <gy, dS/dw>,          dS/dw = (1-lh)(v01 - v00) + lh(v11 - v10)
+//   d/d dy_k  = s * m_k * <gy, dS/dh>,          dS/dh = (1-lw)(v10 - v00) + lw(v11 - v01)
+//   grad_value[corner ab] += m_k * w_ab * gy     (every in-image corner)
+// where <.,.> sums over the group's C' channels.
+//
+// Two kernels, no atomics on gradient data:
+//
+// samples_kernel (output tiles, the forward's mapping).  The three per-sample
+//   gradients follow from the four per-corner dot products d_ab = <gy, v_ab>:
+//   each corner slice is gathered once (256-bit load), dotted with gy in fp32,
+//   reduced over the threads sharing the group, and the grad_offset_mask rows
+//   (padding tail = 0) are assembled in shared memory and stored once.  It
+//   also records, per image, the reach R: the largest distance (per
+//   coordinate, in pixels) between a grid anchor and a corner of a cell that
+//   touches the image.
+//
+// value_kernel (input tiles).  grad_value is pulled, not scattered: a CTA owns
+//   a BH x BW tile of input pixels (all groups) and writes each of their
+//   grad_value elements exactly once.  The samples that can touch the tile come
+//   from output pixels whose anchors lie within R of it; the CTA re-forms those
+//   samples' locations (the same fp32 fma as the forward, so the same cells),
+//   counting-sorts the ones whose cell touches the tile by (group, cell) in
+//   shared memory, then each thread sums m * w_ab * gy over the samples of the
+//   four cells its pixel is a corner of.  Should the sorted samples not fit in
+//   shared memory (a pathological concentration of samples), the CTA falls
+//   back to having each thread scan the candidate samples directly: slower,
+//   same result.
+#include "dcn4_common.cuh"
+
+namespace dcn4 {
+namespace {
+
+__device__ __forceinline__ int floor_div(int a, int b) { return a >= 0 ? a / b : -((-a + b - 1) / b); }
+__device__ __forceinline__ int ceil_div(int a, int b) { return -floor_div(-a, b); }
+
+// <gy, the VEC x 16 bytes of channels at src>, in fp32.
+template <typename T, int VEC>
+__device__ __forceinline__ float corner_dot(const float2* gy, const T* src) {
+    constexpr int PAIRS = Elem<T>::per16 / 2;
+    uint4 raw[VEC];
+    if constexpr (VEC == 2) {
+        ld_gather32(src, raw[0], raw[1]);
+    } else {
+        raw[0] = ld_gather(src);
+    }
+    float2 d = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int v = 0; v < VEC; ++v) {
+        float2 f[PAIRS];
+        unpack(raw[v], f, T());
+#pragma unroll
+        for (int i = 0; i < PAIRS; ++i) d = __ffma2_rn(gy[v * PAIRS + i], f[i], d);
+    }
+    return d.x + d.y;
+}
+
+// gy (this thread's VEC x 16 bytes of grad_out channels) as fp32 pairs.
+template <typename T, int VEC>
+__device__ __forceinline__ void load_gy(float2* gy, const T* src) {
+    constexpr int HALF = Elem<T>::per16 / 2;
+    uint4 raw[VEC];
+    if constexpr (VEC == 2) {
+        ld_gather32(src, raw[0], raw[1]);
+    } else {
+        raw[0] = ld_gather(src);
+    }
+#pragma unroll
+    for (int v = 0; v < VEC; ++v) unpack(raw[v], gy + v * HALF, T());
+}
+
+// Grid cell (ih, iw) of sampling point k (columns outer, rows inner, centre
+// skipped when remove_center is set).
+__device__ __forceinline__ void grid_cell_of(const Geometry& g, int k, int& ih, int& iw) {
+    int idx = k;
+    if (g.remove_center) {
+        const int centre = (g.kw / 2) * g.kh + g.kh / 2;
+        if (idx >= centre) ++idx;
+    }
+    iw = idx / g.kh;
+    ih = idx - iw * g.kh;
+}
+
+// ---------------------------------------------------------------------------
+// grad_offset_mask + reach
+// ---------------------------------------------------------------------------
+template <typename T, int VEC, int KH, int KW, bool RC>
+__global__ void __launch_bounds__(256) samples_kernel(const Geometry g, const T* __restrict__ value,
+                                                      const T* __restrict__ om, const T* __restrict__ gout,
+                                                      T* __restrict__ gom, int* __restrict__ reach) {
+    extern __shared__ __align__(16) unsigned char smem[];
+    __shared__ int s_reach;
+    constexpr int EPV = Elem<T>::per16;
+    constexpr int PAIRS = VEC * EPV / 2;
+    const int tile_elems = g.TH * g.TW * g.P;
+    T* om_s = reinterpret_cast<T*>(smem);
+    float* gom_s = reinterpret_cast<float*>(smem + tile_elems * sizeof(T));  // P % 8 == 0 keeps this 16-byte aligned
+
+    const Tile t = tile_of_block(g);
+    stage_tile_rows(om_s, om, g, t);
+    for (int i = threadIdx.x; i < tile_elems; i += blockDim.x) gom_s[i] = 0.f;
+    if (threadIdx.x == 0) s_reach = -1;
+    __syncthreads();
+
+    const int lanes_pp = g.G * g.nslice;
+    const int lp = threadIdx.x / lanes_pp;
+    const int py = lp / g.TW;
+    const int px = lp - py * g.TW;
+    // Threads past the tile edge stay in the loop (their samples touch
+    // nothing) so that every lane of a warp reaches the shuffles.
+    const bool active = py < t.th && px < t.tw;
+    const int r = threadIdx.x - lp * lanes_pp;
+    const int grp = r / g.nslice;
+    const int sl = r - grp * g.nslice;
+    const int ho = t.ho0 + (active ? py : 0), wo = t.wo0 + (active ? px : 0);
+    const int lrow = (active ? lp : 0) * g.P + grp * 3 * (KH > 0 ? KH * KW - (RC ? 1 : 0) : g.K);
+
+    const int K = KH > 0 ? KH * KW - (RC ? 1 : 0) : g.K;
+    const int kh = KH > 0 ? KH : g.kh;
+    const int kw = KW > 0 ? KW : g.kw;
+    const bool rc = KH > 0 ? RC : g.remove_center != 0;
+    const T* row = om_s + lrow;
+    const int ch_off = grp * g.Cg + sl * (VEC * EPV);
+    const T* img = value + static_cast<long long>(t.n) * g.H * g.W * g.C + ch_off;
+    const int hb = ho * g.sh - g.ph, wb = wo * g.sw - g.pw;
+
+    float2 gy[PAIRS];
+    load_gy<T, VEC>(gy, gout + ((static_cast<long long>(t.n) * g.Ho + ho) * g.Wo + wo) * g.C + ch_off);
+    int my_reach = -1;
+
+    int k = 0;
+#pragma unroll
+    for (int iw = 0; iw < kw; ++iw) {
+        const int aw = wb + iw * g.dw;  // anchor column
+#pragma unroll
+        for (int ih = 0; ih < kh; ++ih) {
+            if (rc && iw == kw / 2 && ih == kh / 2) continue;
+            const int kk = k++;
+            const int ah = hb + ih * g.dh;  // anchor row
+            const float dx = to_f32(row[2 * kk]);
+            const float dy = to_f32(row[2 * kk + 1]);
+            const float m = to_f32(row[2 * K + kk]);
+            const float h = active ? __fmaf_rn(g.s, dy, static_cast<float>(ah)) : -2.f;
+            const float w = __fmaf_rn(g.s, dx, static_cast<float>(aw));
+            const Cell<T> cell = bilinear_cell(g, img, h, w);
+            float d00 = corner_dot<T, VEC>(gy, cell.c[0]);
+            float d01 = corner_dot<T, VEC>(gy, cell.c[1]);
+            float d10 = corner_dot<T, VEC>(gy, cell.c[2]);
+            float d11 = corner_dot<T, VEC>(gy, cell.c[3]);
+            for (int off = g.nslice >> 1; off > 0; off >>= 1) {
+                d00 += __shfl_xor_sync(0xffffffffu, d00, off);
+                d01 += __shfl_xor_sync(0xffffffffu, d01, off);
+                d10 += __shfl_xor_sync(0xffffffffu, d10, off);
+                d11 += __shfl_xor_sync(0xffffffffu, d11, off);
+            }
+            if (cell.any) {
+                if (sl == 0) {
+                    const float hl = 1.f - cell.lh, wl = 1.f - cell.lw;
+                    const float sm = g.s * m;
+                    float* gr = gom_s + lrow;
+                    gr[2 * kk] = sm * (hl * (d01 - d00) + cell.lh * (d11 - d10));
+                    gr[2 * kk + 1] = sm * (wl * (d10 - d00) + cell.lw * (d11 - d01));
+                    gr[2 * K + kk] = hl * (wl * d00 + cell.lw * d01) + cell.lh * (wl * d10 + cell.lw * d11);
+                }
+                const int dh = max(abs(cell.h0 - ah), abs(cell.h0 + 1 - ah));
+                const int dw = max(abs(cell.w0 - aw), abs(cell.w0 + 1 - aw));
+                my_reach = max(my_reach, max(dh, dw));
+            }
+        }
+    }
+
+    for (int off = 16; off > 0; off >>= 1) my_reach = max(my_reach, __shfl_xor_sync(0xffffffffu, my_reach, off));
+    if ((threadIdx.x & 31) == 0 && my_reach >= 0) atomicMax(&s_reach, my_reach);
+    __syncthreads();
+    if (threadIdx.x == 0 && s_reach >= 0) atomicMax(reach + t.n, s_reach);
+
+    // grad_offset_mask rows of the tile, 16-byte stores.
+    const int row_vecs = t.tw * g.P / EPV;
+    for (int i = threadIdx.x; i < t.th * row_vecs; i += blockDim.x) {
+        const int rr = i / row_vecs;
+        const int c = i - rr * row_vecs;
+        const float2* src = reinterpret_cast<const float2*>(gom_s + rr * g.TW * g.P + c * EPV);
+        float2 f[EPV / 2];
+#pragma unroll
+        for (int j = 0; j < EPV / 2; ++j) f[j] = src[j];
+        const long long grow = (static_cast<long long>(t.n) * g.Ho + t.ho0 + rr) * g.Wo + t.wo0;
+        st_global(gom + grow * g.P + c * EPV, pack(f, T()));
+    }
+}
+
+// ---------------------------------------------------------------------------
+// grad_value (pull over a counting sort of the samples touching the tile)
+// ---------------------------------------------------------------------------
+
+// acc += wt * gy slice at src.
+template <typename T, int VEC>
+__device__ __forceinline__ void accumulate(float2* acc, const T* src, float wt) {
+    constexpr int PAIRS = Elem<T>::per16 / 2;
+    const float2 w2 = make_float2(wt, wt);
+    uint4 raw[VEC];
+    if constexpr (VEC == 2) {
+        ld_gather32(src, raw[0], raw[1]);
+    } else {
+        raw[0] = ld_gather(src);
+    }
+#pragma unroll
+    for (int v = 0; v < VEC; ++v) {
+        float2 f[PAIRS];
+        unpack(raw[v], f, T());
+#pragma unroll
+        for (int i = 0; i < PAIRS; ++i) acc[v * PAIRS + i] = __ffma2_rn(w2, f[i], acc[v * PAIRS + i]);
+    }
+}
+
+// One candidate sample of the tile scan: the cell it falls in.
+struct Candidate {
+    int h0, w0;
+    float lh, lw;
+    bool any;
+};
+
+template <typename T>
+__device__ __forceinline__ Candidate candidate(const Geometry& g, const T* om_row, int k, int ho, int wo, int ih,
+                                               int iw) {
+    const float dx = to_f32(om_row[2 * k]);
+    const float dy = to_f32(om_row[2 * k + 1]);
+    const float h = __fmaf_rn(g.s, dy, static_cast<float>(ho * g.sh - g.ph + ih * g.dh));
+    const float w = __fmaf_rn(g.s, dx, static_cast<float>(wo * g.sw - g.pw + iw * g.dw));
+    Candidate c;
+    c.any = h >= -1.f && h < static_cast<float>(g.H) && w >= -1.f && w < static_cast<float>(g.W);
+    const float hc = c.any ? h : 0.f, wc = c.any ? w : 0.f;
+    const float h0f = floorf(hc), w0f = floorf(wc);
+    c.lh = hc - h0f;
+    c.lw = wc - w0f;
+    c.h0 = static_cast<int>(h0f);
+    c.w0 = static_cast<int>(w0f);
+    return c;
+}
+
+template <typename T, int VEC>
+__global__ void __launch_bounds__(1024) value_kernel(const Geometry g, const T* __restrict__ om,
+                                                     const T* __restrict__ gout, T* __restrict__ gvalue,
+                                                     const int* __restrict__ reach) {
+    extern __shared__ __align__(16) unsigned char smem[];
+    __shared__ int s_warp[32];
+    __shared__ int s_total;
+    constexpr int EPV = Elem<T>::per16;
+    constexpr int PAIRS = VEC * EPV / 2;
+
+    // Input tile of this CTA.
+    const int per_img = g.btiles_h * g.btiles_w;
+    const int n = blockIdx.x / per_img;
+    const int tr = blockIdx.x - n * per_img;
+    const int by = tr / g.btiles_w;
+    const int y0 = by * g.BH, x0 = (tr - by * g.btiles_w) * g.BW;
+    const int bh = min(g.BH, g.H - y0), bw = min(g.BW, g.W - x0);
+    const int cells_w = g.BW + 1;
+    const int cells = (g.BH + 1) * cells_w;
+    const int nbins = g.G * cells;
+    int* cnt = reinterpret_cast<int*>(smem);
+    int* cur = cnt + nbins;
+    float4* rec = reinterpret_cast<float4*>(smem + ((2 * nbins * sizeof(int) + 15) / 16) * 16);
+
+    // Output pixels whose samples can touch the tile: anchors within R of it.
+    const int R = reach[n];
+    int ho_lo = 0, ho_hi = -1, wo_lo = 0, wo_hi = -1;
+    if (R >= 0) {
+        ho_lo = max(0, ceil_div(y0 - R + g.ph - (g.kh - 1) * g.dh, g.sh));
+        ho_hi = min(g.Ho - 1, floor_div(y0 + bh - 1 + R + g.ph, g.sh));
+        wo_lo = max(0, ceil_div(x0 - R + g.pw - (g.kw - 1) * g.dw, g.sw));
+        wo_hi = min(g.Wo - 1, floor_div(x0 + bw - 1 + R + g.pw, g.sw));
+    }
+    const int e_w = max(0, wo_hi - wo_lo + 1);
+    const int e_cnt = e_w * max(0, ho_hi - ho_lo + 1);
+
+    // Scan mapping: thread -> fixed (group, point), a slot of pixels per step.
+    const int GK = g.G * g.K;
+    const int spt = blockDim.x / GK;
+    const int tslot = threadIdx.x / GK;
+    const int gk = threadIdx.x - tslot * GK;
+    const bool scanner = tslot < spt;
+    const int sg = gk / g.K;
+    const int sk = gk - sg * g.K;
+    int s_ih, s_iw;
+    grid_cell_of(g, sk, s_ih, s_iw);
+    const T* om_img = om + static_cast<long long>(n) * g.Ho * g.Wo * g.P + sg * 3 * g.K;
+
+    for (int i = threadIdx.x; i < nbins; i += blockDim.x) cnt[i] = 0;
+    __syncthreads();
+
+    // Pass 1: count the samples of each (group, cell).
+    if (scanner) {
+        for (int e = tslot; e < e_cnt; e += spt) {
+            const int eh = e / e_w;
+            const int ho = ho_lo + eh, wo = wo_lo + (e - eh * e_w);
+            const Candidate c = candidate(g, om_img + static_cast<long long>(ho * g.Wo + wo) * g.P, sk, ho, wo, s_ih, s_iw);
+            const int ch = c.h0 - (y0 - 1), cw = c.w0 - (x0 - 1);
+            if (c.any && ch >= 0 && ch <= bh && cw >= 0 && cw <= bw) atomicAdd(&cnt[sg * cells + ch * cells_w + cw], 1);
+        }
+    }
+    __syncthreads();
+
+    // Exclusive scan of the counts -> cursors (block-wide, thread-contiguous chunks).
+    {
+        const int per = (nbins + blockDim.x - 1) / blockDim.x;
+        const int b0 = threadIdx.x * per;
+        int local = 0;
+        for (int b = b0; b < min(nbins, b0 + per); ++b) local += cnt[b];
+        const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+        int incl = local;
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        if (lane == 31) s_warp[wid] = incl;
+        __syncthreads();
+        if (wid == 0) {
+            const int nw = (blockDim.x + 31) >> 5;
+            int v = lane < nw ? s_warp[lane] : 0;
+            for (int o = 1; o < 32; o <<= 1) {
+                const int u = __shfl_up_sync(0xffffffffu, v, o);
+                if (lane >= o) v += u;
+            }
+            if (lane < nw) s_warp[lane] = v;  // inclusive warp totals
+            if (lane == nw - 1) s_total = v;
+        }
+        __syncthreads();
+        int run = incl - local + (wid > 0 ? s_warp[wid - 1] : 0);
+        for (int b = b0; b < min(nbins, b0 + per); ++b) {
+            cur[b] = run;
+            run += cnt[b];
+        }
+    }
+    __syncthreads();
+    const bool sorted = s_total <= g.bcap;
+
+    // Pass 2: place each sample's record (image pixel of p, m(1-lh), m lh, lw) in its bin.
+    if (sorted && scanner) {
+        for (int e = tslot; e < e_cnt; e += spt) {
+            const int eh = e / e_w;
+            const int ho = ho_lo + eh, wo = wo_lo + (e - eh * e_w);
+            const T* orow = om_img + static_cast<long long>(ho * g.Wo + wo) * g.P;
+            const Candidate c = candidate(g, orow, sk, ho, wo, s_ih, s_iw);
+            const int ch = c.h0 - (y0 - 1), cw = c.w0 - (x0 - 1);
+            if (c.any && ch >= 0 && ch <= bh && cw >= 0 && cw <= bw) {
+                const int slot = atomicAdd(&cur[sg * cells + ch * cells_w + cw], 1);
+                const float m = to_f32(orow[2 * g.K + sk]);
+                const float b = m * c.lh;
+                rec[slot] = make_float4(__int_as_float(ho * g.Wo + wo), m - b, b, c.lw);
+            }
+        }
+    }
+    __syncthreads();
+
+    // Pull: thread -> (input pixel q of the tile, group, slice).
+    const int lanes_pp = g.G * g.nslice;
+    const int q = threadIdx.x / lanes_pp;
+    const int qy = q / g.BW, qx = q - (q / g.BW) * g.BW;
+    if (q >= g.BH * g.BW || qy >= bh || qx >= bw) return;
+    const int rr = threadIdx.x - q * lanes_pp;
+    const int grp = rr / g.nslice;
+    const int sl = rr - grp * g.nslice;
+    const int ch_off = grp * g.Cg + sl * (VEC * EPV);
+    const T* gy_img = gout + static_cast<long long>(n) * g.Ho * g.Wo * g.C + ch_off;
+
+    float2 acc[PAIRS];
+#pragma unroll
+    for (int i = 0; i < PAIRS; ++i) acc[i] = make_float2(0.f, 0.f);
+
+    if (sorted) {
+        // q is corner (a, b) of the cell with top-left (qy - a, qx - b).
+#pragma unroll
+        for (int a = 0; a < 2; ++a) {
+#pragma unroll
+            for (int b = 0; b < 2; ++b) {
+                const int bin = grp * cells + (qy - a + 1) * cells_w + (qx - b + 1);
+                const int end = cur[bin];
+                for (int j = end - cnt[bin]; j < end; ++j) {
+                    const float4 rcd = rec[j];
+                    const float wt = (a ? rcd.z : rcd.y) * (b ? rcd.w : 1.f - rcd.w);
+                    accumulate<T, VEC>(acc, gy_img + static_cast<long long>(__float_as_int(rcd.x)) * g.C, wt);
+                }
+            }
+        }
+    } else {
+        // Overflow path: scan every candidate sample of this group directly.
+        const int gy_abs = y0 + qy, gx_abs = x0 + qx;
+        const T* om_g = om + static_cast<long long>(n) * g.Ho * g.Wo * g.P + grp * 3 * g.K;
+        for (int e = 0; e < e_cnt; ++e) {
+            const int eh = e / e_w;
+            const int ho = ho_lo + eh, wo = wo_lo + (e - eh * e_w);
+            const T* orow = om_g + static_cast<long long>(ho * g.Wo + wo) * g.P;
+            for (int k = 0; k < g.K; ++k) {
+                int ih, iw;
+                grid_cell_of(g, k, ih, iw);
+                const Candidate c = candidate(g, orow, k, ho, wo, ih, iw);
+                const int a = gy_abs - c.h0, b = gx_abs - c.w0;
+                if (c.any && a >= 0 && a <= 1 && b >= 0 && b <= 1) {
+                    const float m = to_f32(orow[2 * g.K + k]);
+                    const float wt = m * (a ? c.lh : 1.f - c.lh) * (b ? c.lw : 1.f - c.lw);
+                    accumulate<T, VEC>(acc, gy_img + static_cast<long long>(ho * g.Wo + wo) * g.C, wt);
+                }
+            }
+        }
+    }
+
+    T* dst = gvalue + ((static_cast<long long>(n) * g.H + y0 + qy) * g.W + x0 + qx) * g.C + ch_off;
+    if constexpr (VEC == 2) {
+        st_global32(dst, pack(acc, T()), pack(acc + EPV / 2, T()));
+    } else {
+        st_global(dst, pack(acc, T()));
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Launchers
+// ---------------------------------------------------------------------------
+
+template <typename Kern>
+cudaError_t allow_smem(Kern kern, size_t smem) {
+    if (smem <= 48 * 1024) return cudaSuccess;
+    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+}
+
+template <typename T, int VEC, int KH, int KW, bool RC>
+cudaError_t launch_samples_typed(const Geometry& g, const void* value, const void* om, const void* gout, void* gom,
+                                 int* reach, cudaStream_t stream) {
+    const size_t smem = backward_smem_bytes(g, sizeof(T));
+    auto kern = samples_kernel<T, VEC, KH, KW, RC>;
+    cudaError_t e = allow_smem(kern, smem);
+    if (e != cudaSuccess) return e;
+    const long long blocks = static_cast<long long>(g.N) * g.tiles_h * g.tiles_w;
+    const int threads = (g.pix_per_cta * g.G * g.nslice + 31) / 32 * 32;  // whole warps (shuffles)
+    kern<<<static_cast<unsigned>(blocks), threads, smem, stream>>>(g, static_cast<const T*>(value),
+                                                                   static_cast<const T*>(om), static_cast<const T*>(gout),
+                                                                   static_cast<T*>(gom), reach);
+    return cudaGetLastError();
+}
+
+template <typename T, int VEC>
+cudaError_t launch_samples_grid(const Geometry& g, const void* value, const void* om, const void* gout, void* gom,
+                                int* reach, cudaStream_t stream) {
+    if (g.kh == 3 && g.kw == 3) {
+        return g.remove_center ? launch_samples_typed<T, VEC, 3, 3, true>(g, value, om, gout, gom, reach, stream)
+                               : launch_samples_typed<T, VEC, 3, 3, false>(g, value, om, gout, gom, reach, stream);
+    }
+    return launch_samples_typed<T, VEC, 0, 0, false>(g, value, om, gout, gom, reach, stream);
+}
+
+template <typename T>
+cudaError_t launch_samples_vec(const Geometry& g, const void* value, const void* om, const void* gout, void* gom,
+                               int* reach, cudaStream_t stream) {
+    return g.vec == 2 ? launch_samples_grid<T, 2>(g, value, om, gout, gom, reach, stream)
+                      : launch_samples_grid<T, 1>(g, value, om, gout, gom, reach, stream);
+}
+
+template <typename T, int VEC>
+cudaError_t launch_value_typed(const Geometry& g, const void* om, const void* gout, void* gvalue, const int* reach,
+                               cudaStream_t stream) {
+    const size_t smem = backward_value_smem_bytes(g);
+    auto kern = value_kernel<T, VEC>;
+    cudaError_t e = allow_smem(kern, smem);
+    if (e != cudaSuccess) return e;
+    const long long blocks = static_cast<long long>(g.N) * g.btiles_h * g.btiles_w;
+    kern<<<static_cast<unsigned>(blocks), g.bthreads, smem, stream>>>(
+        g, static_cast<const T*>(om), static_cast<const T*>(gout), static_cast<T*>(gvalue), reach);
+    return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t launch_value_vec(const Geometry& g, const void* om, const void* gout, void* gvalue, const int* reach,
+                             cudaStream_t stream) {
+    return g.vec == 2 ? launch_value_typed<T, 2>(g, om, gout, gvalue, reach, stream)
+                      : launch_value_typed<T, 1>(g, om, gout, gvalue, reach, stream);
+}
+
+}  // namespace
+
+size_t backward_smem_bytes(const Geometry& g, int elem_bytes) {
+    return static_cast<size_t>(g.TH) * g.TW * g.P * (elem_bytes + 4);
+}
+
+size_t backward_value_smem_bytes(const Geometry& g) {
+    const size_t nbins = static_cast<size_t>(g.G) * (g.BH + 1) * (g.BW + 1);
+    return (2 * nbins * sizeof(int) + 15) / 16 * 16 + static_cast<size_t>(g.bcap) * 16;
+}
+
+cudaError_t launch_backward_samples(const Geometry& g, int dtype, const void* value, const void* om, const void* gout,
+                                    void* gom, int* reach, cudaStream_t stream) {
+    switch (dtype) {
+        case 0: return launch_samples_vec<float>(g, value, om, gout, gom, reach, stream);
+        case 1: return launch_samples_vec<__half>(g, value, om, gout, gom, reach, stream);
+        case 2: return launch_samples_vec<__nv_bfloat16>(g, value, om, gout, gom, reach, stream);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t launch_backward_value(const Geometry& g, int dtype, const void* om, const void* gout, void* gvalue,
+                                  const int* reach, cudaStream_t stream) {
+    switch (dtype) {
+        case 0: return launch_value_vec<float>(g, om, gout, gvalue, reach, stream);
+        case 1: return launch_value_vec<__half>(g, om, gout, gvalue, reach, stream);
+        case 2: return launch_value_vec<__nv_bfloat16>(g, om, gout, gvalue, reach, stream);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace dcn4

@@ -1,0 +1,248 @@
+// dcn4_common.cuh — device-side helpers shared by the libdcn4 kernels.
+//
+// Element access is in 16-byte vectors (8 x fp16/bf16 or 4 x fp32): the C'
+// channels of a group are contiguous in the channels-last layout, so one
+// 128-bit instruction moves a whole run of them (CSDN summary of "Efficient
+// Deformable ConvNets", section 2.2, "消除冗余内存指令").
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+namespace dcn4 {
+
+// Problem geometry with the derived sizes the kernels need (filled on the host).
+struct Geometry {
+    int N, H, W, G, Cg, C, Ho, Wo, P, K;
+    int kh, kw, sh, sw, ph, pw, dh, dw;
+    float s;              // offset_scale
+    int remove_center;
+    int vec;              // 16-byte vectors per thread slice: 2 (one 32-byte access) or 1
+    int nslice;           // threads cooperating on one (pixel, group): power of two <= 32
+    int pix_per_cta;      // output pixels handled by one CTA (= TH * TW)
+    long long total_pix;  // N * Ho * Wo
+    int TH, TW;           // output tile of one CTA (rows x columns of one image)
+    int tiles_h, tiles_w; // tiles per image
+    // grad_value pass: input tiles of BH x BW pixels, bthreads threads per CTA,
+    // room for bcap sample records in shared memory.
+    int BH, BW, btiles_h, btiles_w, bthreads, bcap;
+};
+
+template <typename T>
+struct Elem;
+template <>
+struct Elem<float> {
+    static constexpr int per16 = 4;
+};
+template <>
+struct Elem<__half> {
+    static constexpr int per16 = 8;
+};
+template <>
+struct Elem<__nv_bfloat16> {
+    static constexpr int per16 = 8;
+};
+
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__half x) { return __half2float(x); }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+// ---------------------------------------------------------------------------
+// 16-byte vector <-> float pairs
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void unpack(const uint4& r, float2* f, float) {
+    f[0] = make_float2(__uint_as_float(r.x), __uint_as_float(r.y));
+    f[1] = make_float2(__uint_as_float(r.z), __uint_as_float(r.w));
+}
+__device__ __forceinline__ void unpack(const uint4& r, float2* f, __half) {
+    const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        __half2 h;
+        memcpy(&h, &w[i], 4);
+        f[i] = __half22float2(h);
+    }
+}
+__device__ __forceinline__ void unpack(const uint4& r, float2* f, __nv_bfloat16) {
+    // bfloat16 is the upper half of a binary32: widen by placing the bits there.
+    const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) f[i] = make_float2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xffff0000u));
+}
+
+__device__ __forceinline__ uint4 pack(const float2* f, float) {
+    return make_uint4(__float_as_uint(f[0].x), __float_as_uint(f[0].y), __float_as_uint(f[1].x),
+                      __float_as_uint(f[1].y));
+}
+__device__ __forceinline__ uint4 pack(const float2* f, __half) {
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const __half2 h = __float22half2_rn(f[i]);
+        memcpy(&w[i], &h, 4);
+    }
+    return make_uint4(w[0], w[1], w[2], w[3]);
+}
+__device__ __forceinline__ uint4 pack(const float2* f, __nv_bfloat16) {
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const __nv_bfloat162 h = __float22bfloat162_rn(f[i]);
+        memcpy(&w[i], &h, 4);
+    }
+    return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// ---------------------------------------------------------------------------
+// Global memory access
+// ---------------------------------------------------------------------------
+
+// Read-only gather through L1 (value rows are re-read by neighbouring samples).
+__device__ __forceinline__ uint4 ld_gather(const void* p) {
+    return __ldg(reinterpret_cast<const uint4*>(p));
+}
+
+// 32-byte read-only gather (one full sector per thread, sm_100 256-bit load).
+__device__ __forceinline__ void ld_gather32(const void* p, uint4& lo, uint4& hi) {
+    asm volatile("ld.global.nc.v8.u32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                 : "=r"(lo.x), "=r"(lo.y), "=r"(lo.z), "=r"(lo.w), "=r"(hi.x), "=r"(hi.y), "=r"(hi.z), "=r"(hi.w)
+                 : "l"(p));
+}
+
+// 32-byte store (sm_100 256-bit store).
+__device__ __forceinline__ void st_global32(void* p, const uint4& lo, const uint4& hi) {
+    asm volatile("st.global.v8.u32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(lo.x), "r"(lo.y),
+                 "r"(lo.z), "r"(lo.w), "r"(hi.x), "r"(hi.y), "r"(hi.z), "r"(hi.w)
+                 : "memory");
+}
+
+// Streaming read that is used once (offset_mask rows, grad_out): do not keep in L1.
+__device__ __forceinline__ uint4 ld_stream(const void* p) {
+    uint4 r;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "l"(p));
+    return r;
+}
+
+__device__ __forceinline__ void st_global(void* p, const uint4& v) {
+    *reinterpret_cast<uint4*>(p) = v;
+}
+
+// Output pixel index -> (n, ho, wo).
+__device__ __forceinline__ void pixel_coords(const Geometry& g, long long pix, int& n, int& ho, int& wo) {
+    const long long hw = static_cast<long long>(g.Ho) * g.Wo;
+    n = static_cast<int>(pix / hw);
+    const int rem = static_cast<int>(pix - static_cast<long long>(n) * hw);
+    ho = rem / g.Wo;
+    wo = rem - ho * g.Wo;
+}
+
+// Copies `bytes` (a multiple of 16) of contiguous global memory into shared
+// memory with the whole CTA, 16 bytes per thread per step.
+__device__ __forceinline__ void stage_rows(void* dst_smem, const void* src, int bytes) {
+    uint4* d = reinterpret_cast<uint4*>(dst_smem);
+    const char* s = reinterpret_cast<const char*>(src);
+    for (int i = threadIdx.x; i < bytes / 16; i += blockDim.x) d[i] = ld_stream(s + 16ll * i);
+}
+
+// One CTA's output tile: image n, rows [ho0, ho0 + th), columns [wo0, wo0 + tw).
+struct Tile {
+    int n, ho0, wo0, th, tw;
+};
+
+__device__ __forceinline__ Tile tile_of_block(const Geometry& g) {
+    const int per_img = g.tiles_h * g.tiles_w;
+    Tile t;
+    t.n = blockIdx.x / per_img;
+    const int r = blockIdx.x - t.n * per_img;
+    const int ty = r / g.tiles_w;
+    const int tx = r - ty * g.tiles_w;
+    t.ho0 = ty * g.TH;
+    t.wo0 = tx * g.TW;
+    t.th = min(g.TH, g.Ho - t.ho0);
+    t.tw = min(g.TW, g.Wo - t.wo0);
+    return t;
+}
+
+// Copies the P-wide rows of a tile of pixels (row-major [th][tw] in a [*, Ho, Wo, P]
+// tensor) into shared memory laid out [TH][TW][P]; 16 bytes per thread per step.
+template <typename T>
+__device__ __forceinline__ void stage_tile_rows(T* dst_smem, const T* src, const Geometry& g, const Tile& t) {
+    const int row_chunks = t.tw * g.P * static_cast<int>(sizeof(T)) / 16;  // 16-byte chunks per tile row
+    const int total = t.th * row_chunks;
+    for (int i = threadIdx.x; i < total; i += blockDim.x) {
+        const int r = i / row_chunks;
+        const int c = i - r * row_chunks;
+        const long long grow = (static_cast<long long>(t.n) * g.Ho + t.ho0 + r) * g.Wo + t.wo0;
+        const char* s = reinterpret_cast<const char*>(src + grow * g.P) + 16ll * c;
+        char* d = reinterpret_cast<char*>(dst_smem + r * g.TW * g.P) + 16 * c;
+        *reinterpret_cast<uint4*>(d) = ld_stream(s);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Bilinear cell of one sample, branch-free
+// ---------------------------------------------------------------------------
+
+// 32 zero bytes: the gather address of a corner outside the image, so every
+// corner can be loaded unconditionally (its value then contributes 0).  One
+// copy per translation unit (device code is not relocatable).
+static __device__ __align__(32) const uint4 g_zero_slice[2] = {};
+
+// The four corners of the cell that floor() selects for location (h, w):
+// c[0] = (h0, w0), c[1] = (h0, w0+1), c[2] = (h0+1, w0), c[3] = (h0+1, w0+1),
+// with bilinear weights wt[] = (1-lh)(1-lw), (1-lh)lw, lh(1-lw), lh lw.  A
+// corner outside [0,H) x [0,W) gets the zero slice as its address; a location
+// that touches no pixel (h < -1, h >= H, w < -1, w >= W, or NaN) gets it for
+// all four.  `img` points at this thread's channels of pixel (0, 0) of the image.
+template <typename T>
+struct Cell {
+    const T* c[4];
+    float lh, lw;
+    int h0, w0;  // top-left corner of the cell (meaningful when any)
+    bool any;    // some corner is inside the image
+};
+
+template <typename T>
+__device__ __forceinline__ Cell<T> bilinear_cell(const Geometry& g, const T* img, float h, float w) {
+    Cell<T> cell;
+    cell.any = h >= -1.f && h < static_cast<float>(g.H) && w >= -1.f && w < static_cast<float>(g.W);
+    const float hc = cell.any ? h : 0.f, wc = cell.any ? w : 0.f;
+    const float h0f = floorf(hc), w0f = floorf(wc);
+    cell.lh = hc - h0f;
+    cell.lw = wc - w0f;
+    const int h0 = static_cast<int>(h0f), w0 = static_cast<int>(w0f);
+    cell.h0 = h0;
+    cell.w0 = w0;
+    const bool y0 = cell.any && h0 >= 0, y1 = cell.any && h0 + 1 < g.H;
+    const bool x0 = w0 >= 0, x1 = w0 + 1 < g.W;
+    const T* zero = reinterpret_cast<const T*>(g_zero_slice);
+    const T* p00 = img + (h0 * g.W + w0) * g.C;
+    cell.c[0] = (y0 && x0) ? p00 : zero;
+    cell.c[1] = (y0 && x1) ? p00 + g.C : zero;
+    cell.c[2] = (y1 && x0) ? p00 + g.W * g.C : zero;
+    cell.c[3] = (y1 && x1) ? p00 + g.W * g.C + g.C : zero;
+    return cell;
+}
+
+}  // namespace dcn4
+
+// Host-side launchers (defined in dcn4_forward.cu / dcn4_backward.cu).
+namespace dcn4 {
+cudaError_t launch_forward(const Geometry& g, int dtype, const void* value, const void* om, void* out,
+                           cudaStream_t stream);
+// grad_offset_mask and the per-image reach (int[N], pre-filled with -1).
+cudaError_t launch_backward_samples(const Geometry& g, int dtype, const void* value, const void* om,
+                                    const void* gout, void* gom, int* reach, cudaStream_t stream);
+// grad_value from the reach written by launch_backward_samples.
+cudaError_t launch_backward_value(const Geometry& g, int dtype, const void* om, const void* gout, void* gvalue,
+                                  const int* reach, cudaStream_t stream);
+// Dynamic shared memory bytes of one CTA.
+size_t forward_smem_bytes(const Geometry& g, int elem_bytes);
+size_t backward_smem_bytes(const Geometry& g, int elem_bytes);
+size_t backward_value_smem_bytes(const Geometry& g);
+}  // namespace dcn4

@@ -1,0 +1,153 @@
+/*
+ * dcn4.h — C ABI of libdcn4, the sm_100a (B200) DCNv4 core spatial aggregation.
+ *
+ * The operation (CSDN summary of "Efficient Deformable ConvNets: Rethinking
+ * Dynamic and Sparse Operator for Vision Applications", section 1.2 equation,
+ * with the softmax over K removed as section 2.1 "增强动态特性" describes):
+ *
+ *     y_g(p0) = sum_{k<K} m_gk * x_g(p0 + p_k + offset_scale * dp_gk),   y = concat_g y_g
+ *
+ * for every output pixel p0 and group g.  x_g(.) is bilinear interpolation of
+ * the C' = Cg channels of group g (section 2.2: four coefficients per sample);
+ * a bilinear corner outside the image contributes zero.  p_k runs over a
+ * kh x kw convolution grid with stride, padding and dilation; remove_center
+ * drops the centre cell so K = kh*kw - 1 (DCNv4 module / dcnv4_cuda_forward
+ * signatures on the mhpn.cn architecture page).  The modulation scalars m_gk
+ * are unbounded (no softmax).
+ *
+ * Sampling location of grid cell (ih, iw) for output pixel (ho, wo):
+ *     h = ho*sh - ph + ih*dh + offset_scale*dy,   w = wo*sw - pw + iw*dw + offset_scale*dx
+ * formed in fp32 as fmaf(offset_scale, d, base) (one rounding).  The grid is
+ * enumerated with the kernel column outer and the kernel row inner,
+ * k = iw*kh + ih, skipping the centre (iw, ih) = (kw/2, kh/2) when
+ * remove_center is set; dx moves along W and dy along H.
+ *
+ * Layouts (dense, contiguous, channels last; C = G*Cg):
+ *   value            [N, H,  W,  C]   dtype
+ *   offset_mask      [N, Ho, Wo, P]   dtype.  Group g owns entries [g*3K, (g+1)*3K):
+ *                                     K pairs (dx_k, dy_k), then K masks m_k.
+ *                                     Entries [G*3K, P) are padding: never read.
+ *   out / grad_out   [N, Ho, Wo, C]   dtype
+ *   grad_value       [N, H,  W,  C]   dtype
+ *   grad_offset_mask [N, Ho, Wo, P]   dtype; the padding tail is written as 0.
+ * P is a multiple of 8 and >= G*3K ("padded_offset_dim divisible by 8" on the
+ * mhpn.cn page); dcn4_padded_offset_dim() gives the smallest such P.
+ *
+ * Precision: inputs are converted to fp32, every sum is accumulated in fp32,
+ * and results are rounded once to dtype (round to nearest even).
+ *
+ * Ownership and execution: the caller owns every buffer (device memory) and
+ * the stream.  The library allocates nothing and keeps no state between
+ * calls; every call is asynchronous and ordered on `stream` (a cudaStream_t;
+ * NULL is the legacy default stream).  Inputs must not alias outputs.
+ *
+ * Preconditions checked on the host before anything is launched (a failed
+ * check launches nothing and returns a negative status):
+ *   - non-NULL pointers (except when N == 0, which is a successful no-op);
+ *   - every pointer 16-byte aligned;
+ *   - Cg * sizeof(dtype) a multiple of 16 bytes (fp32: Cg % 4 == 0, fp16/bf16:
+ *     Cg % 8 == 0) and Cg * sizeof(dtype) / 32 (rounded up) a power of two <= 32;
+ *   - H, W < 2^24 and H*W*C < 2^31 (per image), Ho >= 1, Wo >= 1;
+ *   - remove_center only with odd kh and kw.
+ * Errors are returned, never raised: no abort, no exception, no device trap.
+ */
+#ifndef DCN4_H
+#define DCN4_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define DCN4_VERSION 100  /* 1.0.0 */
+
+typedef enum {
+    DCN4_F32 = 0,   /* IEEE binary32            */
+    DCN4_F16 = 1,   /* IEEE binary16            */
+    DCN4_BF16 = 2   /* bfloat16 (upper half of binary32) */
+} dcn4_dtype;
+
+typedef enum {
+    DCN4_OK = 0,
+    DCN4_ERR_NULL = -1,         /* a required pointer is NULL                         */
+    DCN4_ERR_BAD_SHAPE = -2,    /* non-positive size, empty output grid, bad geometry */
+    DCN4_ERR_BAD_P = -3,        /* P < G*3K or P not a multiple of 8                  */
+    DCN4_ERR_MISALIGNED = -4,   /* a pointer is not 16-byte aligned                   */
+    DCN4_ERR_UNSUPPORTED = -5,  /* valid operator, but outside this build's kernels   */
+    DCN4_ERR_WORKSPACE = -6,    /* workspace missing or smaller than required         */
+    DCN4_ERR_LAUNCH = -7,       /* the CUDA launch failed; see dcn4_last_error()      */
+    DCN4_ERR_DTYPE = -8         /* dtype is not a dcn4_dtype                          */
+} dcn4_status;
+
+/* Geometry of one call.  All fields are read, none is written. */
+typedef struct {
+    int N, H, W;          /* value is [N, H, W, G*Cg]                           */
+    int G, Cg;            /* groups, channels per group                         */
+    int kh, kw;           /* sampling grid (kernel) size                        */
+    int sh, sw;           /* stride  (>= 1)                                     */
+    int ph, pw;           /* padding (>= 0)                                     */
+    int dh, dw;           /* dilation (>= 1)                                    */
+    float offset_scale;   /* multiplies the learned offsets, not the grid      */
+    int remove_center;    /* 0 or 1                                             */
+    int P;                /* row length of offset_mask / grad_offset_mask       */
+    int dtype;            /* dcn4_dtype of every tensor argument                */
+} dcn4_params;
+
+/* Library version (DCN4_VERSION of the build). */
+int dcn4_version(void);
+
+/* Number of sampling points K = kh*kw - remove_center, or a negative status. */
+int dcn4_num_points(const dcn4_params* p);
+
+/* Smallest valid P for G groups of K points: G*3K rounded up to a multiple of 8.
+ * Returns a negative status for G < 1 or K < 1. */
+int dcn4_padded_offset_dim(int G, int K);
+
+/* Output grid: Ho = (H + 2*ph - (dh*(kh-1) + 1)) / sh + 1 (floor), likewise Wo.
+ * Writes *Ho, *Wo and returns DCN4_OK, or a negative status. */
+int dcn4_output_dims(const dcn4_params* p, int* Ho, int* Wo);
+
+/* Host-only validation of p (shape, P, dtype, supported sizes); touches no
+ * GPU.  Returns DCN4_OK or the status dcn4_forward would return. */
+int dcn4_check_params(const dcn4_params* p);
+
+/* Forward: out = y.  Reads value and offset_mask, writes every element of out.
+ * One kernel launch on `stream`. */
+int dcn4_forward(const dcn4_params* p, const void* value, const void* offset_mask, void* out,
+                 void* stream);
+
+/* Bytes of device workspace dcn4_backward needs: one 32-bit word per image
+ * (N*4 rounded up to 256), whatever the dtype; 0 if p is invalid. */
+size_t dcn4_backward_workspace_size(const dcn4_params* p);
+
+/* Backward of the forward for upstream gradient grad_out:
+ *   grad_value       = sum over samples of m_gk * bilinear_weight * grad_out (scatter-add)
+ *   grad_offset_mask = (d/d dx, d/d dy) = offset_scale * m_gk * <grad_out, dS/dw, dS/dh>
+ *                      and d/d m_gk = <grad_out, S> per (pixel, group, k);
+ * S is the bilinear sample, and its derivative at an integer coordinate is the
+ * one of the cell floor() selects.  Both gradients are overwritten (not
+ * accumulated into); the offset_mask padding tail is written as 0.
+ * `workspace` (device, 16-byte aligned, >= dcn4_backward_workspace_size bytes)
+ * is scratch, clobbered by the call: it receives, per image, how far any
+ * sample reaches from its grid position.
+ * Launches, on `stream`: a memset of that word per image, one kernel for
+ * grad_offset_mask (and the reach), and one for grad_value.  grad_value is
+ * not scattered with atomics: each element is summed by one thread in fp32
+ * (over the samples sorted by cell) and written once, so results are
+ * deterministic up to the order in which samples of one cell are added. */
+int dcn4_backward(const dcn4_params* p, const void* value, const void* offset_mask,
+                  const void* grad_out, void* grad_value, void* grad_offset_mask,
+                  void* workspace, size_t workspace_bytes, void* stream);
+
+/* Name of a dcn4_status. */
+const char* dcn4_status_string(int status);
+
+/* Detail of the last failing call on this host thread ("" if none). */
+const char* dcn4_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DCN4_H */

@@ -1,0 +1,136 @@
+"""The C-ABI library loads, exports every declared symbol, and validates
+calls on the host before touching a GPU (CPU only: no kernel is launched)."""
+import ctypes
+import os
+import re
+import shutil
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "dcn4.h")
+
+
+@pytest.fixture(scope="module")
+def dcn():
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "dcn4_build", os.path.join(ROOT, "deformable_convolution_sampling_b200", "build.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    mod.build()
+    import deformable_convolution_sampling_b200 as d
+    return d
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(dcn4_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("dcn4_forward", "dcn4_backward", "dcn4_backward_workspace_size", "dcn4_output_dims",
+                     "dcn4_padded_offset_dim", "dcn4_status_string", "dcn4_last_error", "dcn4_check_params"):
+        assert required in names
+
+
+def test_every_declared_symbol_is_exported(dcn):
+    raw = ctypes.CDLL(dcn.LIB_PATH)
+    for name in declared_functions():
+        assert hasattr(raw, name), f"{name} declared in dcn4.h but not exported"
+    out = subprocess.run(["nm", "-D", "--defined-only", dcn.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT (dcn4_\w+)", out))
+    assert exported == set(declared_functions()), exported ^ set(declared_functions())
+
+
+def test_library_does_not_link_the_oracle(dcn):
+    out = subprocess.run(["ldd", dcn.LIB_PATH], capture_output=True, text=True).stdout
+    assert "oracle" not in out
+    syms = subprocess.run(["nm", "-D", dcn.LIB_PATH], capture_output=True, text=True).stdout
+    assert "ref_forward" not in syms and "ref_backward" not in syms
+
+
+def test_padded_offset_dim_and_points(dcn):
+    assert dcn.dcn4_padded_offset_dim(2, 9) == 56
+    assert dcn.dcn4_padded_offset_dim(4, 9) == 112
+    assert dcn.dcn4_padded_offset_dim(16, 9) == 432
+    assert dcn.dcn4_padded_offset_dim(4, 8) == 96
+    assert dcn.dcn4_padded_offset_dim(0, 9) < 0
+    p = dcn.make_params(N=1, H=8, W=8, G=2, Cg=8, remove_center=1, dtype="f32")
+    assert dcn.dcn4_num_points(p) == 8
+
+
+def test_output_dims_agree_with_the_oracle(dcn):
+    import oracle
+    for (kh, kw, sh, sw, ph, pw, dh, dw) in [(3, 3, 1, 1, 1, 1, 1, 1), (3, 5, 2, 1, 0, 2, 2, 1),
+                                             (1, 3, 3, 2, 0, 0, 1, 3), (5, 5, 2, 2, 2, 2, 1, 1)]:
+        for H, W in [(7, 9), (16, 5), (33, 33)]:
+            geo = dict(N=1, H=H, W=W, G=2, Cg=8, kh=kh, kw=kw, sh=sh, sw=sw, ph=ph, pw=pw, dh=dh, dw=dw)
+            try:
+                want = oracle.output_dims(oracle.Problem(dtype="f32", **geo))
+            except ValueError:
+                want = None
+            st, ho, wo = dcn.dcn4_output_dims(dcn.make_params(dtype="f16", **geo))
+            if want is None:
+                assert st == -2
+            else:
+                assert st == 0 and (ho, wo) == want
+
+
+def test_workspace_size(dcn):
+    """One reach word per image, rounded up to 256 bytes, for every dtype."""
+    p = dcn.make_params(N=64, H=56, W=56, G=4, Cg=16, dtype="f16")
+    assert dcn.dcn4_backward_workspace_size(p) == 256
+    p = dcn.make_params(N=100, H=8, W=8, G=2, Cg=8, dtype="f32")
+    assert dcn.dcn4_backward_workspace_size(p) == 512
+    p.Cg = 6
+    assert dcn.dcn4_backward_workspace_size(p) == 0
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("dtype", 7, -8), ("N", -1, -2), ("H", 0, -2), ("G", 0, -2), ("Cg", 0, -2), ("kh", 0, -2),
+    ("sh", 0, -2), ("ph", -1, -2), ("dh", 0, -2), ("remove_center", 2, -2), ("P", 50, -3),
+    ("P", 60, -3), ("Cg", 4, -5), ("Cg", 24, -5), ("Cg", 48, -5), ("H", 1 << 24, -5),
+])
+def test_invalid_params_are_rejected_before_launch(dcn, field, value, status):
+    p = dcn.make_params(N=2, H=8, W=8, G=2, Cg=8, dtype="f16")
+    setattr(p, field, value)
+    assert dcn.dcn4_check_params(p) == status
+    # pointers that would fault if used: the call must fail before any launch
+    assert dcn.dcn4_forward(p, 16, 32, 48, None) == status
+    assert dcn.dcn4_last_error() != ""
+
+
+def test_remove_center_needs_odd_kernel(dcn):
+    p = dcn.make_params(N=1, H=8, W=8, G=2, Cg=8, kh=2, kw=3, ph=0, dtype="f16", P=48)
+    p.remove_center = 1
+    assert dcn.dcn4_check_params(p) == -2
+
+
+def test_null_and_misaligned_pointers(dcn):
+    p = dcn.make_params(N=1, H=8, W=8, G=2, Cg=8, dtype="f16")
+    assert dcn.dcn4_forward(p, None, 16, 32, None) == -1
+    assert dcn.dcn4_forward(p, 16, 18, 32, None) == -4
+    assert dcn.dcn4_backward(p, 16, 32, 48, 64, None, 96, 1 << 20, None) == -1
+    assert dcn.dcn4_backward(p, 16, 32, 48, 64, 80, 97, 1 << 20, None) == -4
+    assert dcn.dcn4_backward(p, 16, 32, 48, 64, 80, None, 0, None) == -6
+    assert dcn.dcn4_backward(p, 16, 32, 48, 64, 80, 96, 100, None) == -6
+    assert dcn.lib.dcn4_forward(None, None, None, None, None) == -1
+
+
+def test_status_strings(dcn):
+    for code, name in dcn.STATUS.items():
+        assert dcn.dcn4_status_string(code) == name
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    pkg = tmp_path / "deformable_convolution_sampling_b200"
+    pkg.mkdir()
+    shutil.copy(os.path.join(ROOT, "deformable_convolution_sampling_b200", "__init__.py"), pkg)
+    r = subprocess.run([sys.executable, "-c", "import deformable_convolution_sampling_b200"], cwd=tmp_path,
+                       capture_output=True, text=True)
+    assert r.returncode != 0 and "ImportError" in r.stderr and "no CPU fallback" in r.stderr
