@@ -40,7 +40,10 @@ constexpr size_t kSmemMax = 227 * 1024;
 // grad_value pass: up to 1024 threads and 256 input pixels per CTA; sample
 // records get what is left of this shared-memory budget after the bins.
 constexpr int kValueThreads = 1024;
-constexpr int kValuePixels = 256;
+#ifndef DCN4_VALUE_PIXELS
+#define DCN4_VALUE_PIXELS 256
+#endif
+constexpr int kValuePixels = DCN4_VALUE_PIXELS;
 constexpr size_t kValueSmem = 200 * 1024;
 
 // Validates p and fills the kernel geometry.  Touches no GPU state.
@@ -140,11 +143,12 @@ int make_geometry(const dcn4_params* p, bool backward, bool wide, dcn4::Geometry
     const long long bin_bytes = (2 * nbins * 4 + 15) / 16 * 16;
     if (bin_bytes + 1024 * 16 > static_cast<long long>(kValueSmem))
         return fail(DCN4_ERR_UNSUPPORTED, "too many groups for the grad_value tile");
-    // Records: room for about twice the expected number of samples per tile
-    // (K per cell for every output pixel per input pixel), within the budget.
+    // Records: room for 1.25x the expected number of samples per tile (K per
+    // cell for every output pixel per input pixel), within the budget; the
+    // rest of the shared memory stays L1 for the grad_out gathers.
     const long long expect = nbins * K * std::max<long long>(1, (Ho * Wo + p->H * p->W - 1) / (p->H * p->W));
     long long bcap = (static_cast<long long>(kValueSmem) - bin_bytes) / 16;
-    bcap = std::max<long long>(1024, std::min(bcap, 2 * expect));
+    bcap = std::max<long long>(1024, std::min(bcap, expect + expect / 4 + 256));
     const long long btiles_h = (p->H + BH - 1) / BH, btiles_w = (p->W + BW - 1) / BW;
     if (static_cast<long long>(p->N) * btiles_h * btiles_w > 0x7fffffffLL)
         return fail(DCN4_ERR_UNSUPPORTED, "grid too large");
@@ -156,6 +160,12 @@ int make_geometry(const dcn4_params* p, bool backward, bool wide, dcn4::Geometry
     g->bcap = static_cast<int>(bcap);
     return DCN4_OK;
 }
+
+// Backward workspace: one reach word per image, one cell bounding box (4
+// bytes) per output pixel (each rounded up to 256 bytes), then one 2-byte cell
+// code per sample.
+size_t reach_bytes(const dcn4::Geometry& g) { return (static_cast<size_t>(g.N) * sizeof(int) + 255) / 256 * 256; }
+size_t box_bytes(const dcn4::Geometry& g) { return (static_cast<size_t>(g.total_pix) * 4 + 255) / 256 * 256; }
 
 }  // namespace
 
@@ -214,7 +224,7 @@ int dcn4_forward(const dcn4_params* p, const void* value, const void* offset_mas
 size_t dcn4_backward_workspace_size(const dcn4_params* p) {
     dcn4::Geometry g;
     if (make_geometry(p, true, true, &g) != DCN4_OK) return 0;
-    return (static_cast<size_t>(g.N) * sizeof(int) + 255) / 256 * 256;  // one reach word per image
+    return reach_bytes(g) + box_bytes(g) + static_cast<size_t>(g.total_pix) * g.G * g.K * sizeof(uint16_t);
 }
 
 int dcn4_backward(const dcn4_params* p, const void* value, const void* offset_mask, const void* grad_out,
@@ -233,12 +243,14 @@ int dcn4_backward(const dcn4_params* p, const void* value, const void* offset_ma
         return fail(DCN4_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, workspace_bytes);
     if (!aligned16(workspace)) return fail(DCN4_ERR_MISALIGNED, "workspace must be 16-byte aligned");
     int* reach = static_cast<int*>(workspace);
+    uint32_t* boxes = reinterpret_cast<uint32_t*>(static_cast<char*>(workspace) + reach_bytes(g));
+    uint16_t* codes = reinterpret_cast<uint16_t*>(static_cast<char*>(workspace) + reach_bytes(g) + box_bytes(g));
     const cudaStream_t s = static_cast<cudaStream_t>(stream);
     cudaError_t e = cudaMemsetAsync(reach, 0xff, static_cast<size_t>(g.N) * sizeof(int), s);  // reach = -1
     if (e != cudaSuccess) return fail(DCN4_ERR_LAUNCH, "reach reset: %s", cudaGetErrorString(e));
-    e = dcn4::launch_backward_samples(g, p->dtype, value, offset_mask, grad_out, grad_offset_mask, reach, s);
+    e = dcn4::launch_backward_samples(g, p->dtype, value, offset_mask, grad_out, grad_offset_mask, reach, codes, boxes, s);
     if (e != cudaSuccess) return fail(DCN4_ERR_LAUNCH, "grad_offset_mask launch: %s", cudaGetErrorString(e));
-    e = dcn4::launch_backward_value(g, p->dtype, offset_mask, grad_out, grad_value, reach, s);
+    e = dcn4::launch_backward_value(g, p->dtype, offset_mask, grad_out, grad_value, reach, codes, boxes, s);
     if (e != cudaSuccess) return fail(DCN4_ERR_LAUNCH, "grad_value launch: %s", cudaGetErrorString(e));
     return DCN4_OK;
 }

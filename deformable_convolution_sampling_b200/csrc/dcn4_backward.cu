@@ -18,14 +18,16 @@
 //   (padding tail = 0) are assembled in shared memory and stored once.  It
 //   also records, per image, the reach R: the largest distance (per
 //   coordinate, in pixels) between a grid anchor and a corner of a cell that
-//   touches the image.
+//   touches the image; and, per sample, a 2-byte code of its cell relative to
+//   its anchor.
 //
 // value_kernel (input tiles).  grad_value is pulled, not scattered: a CTA owns
 //   a BH x BW tile of input pixels (all groups) and writes each of their
 //   grad_value elements exactly once.  The samples that can touch the tile come
-//   from output pixels whose anchors lie within R of it; the CTA re-forms those
-//   samples' locations (the same fp32 fma as the forward, so the same cells),
-//   counting-sorts the ones whose cell touches the tile by (group, cell) in
+//   from output pixels whose anchors lie within R of it; the CTA reads those
+//   samples' cell codes, re-forms the locations of the ones whose cell touches
+//   the tile (the same fp32 fma as the forward, so the same cells), and
+//   counting-sorts them by (group, cell) in
 //   shared memory, then each thread sums m * w_ab * gy over the samples of the
 //   four cells its pixel is a corner of.  Should the sorted samples not fit in
 //   shared memory (a pathological concentration of samples), the CTA falls
@@ -74,6 +76,23 @@ __device__ __forceinline__ void load_gy(float2* gy, const T* src) {
     for (int v = 0; v < VEC; ++v) unpack(raw[v], gy + v * HALF, T());
 }
 
+// Cell code of a sample: the offset of its cell's top-left corner from the
+// grid anchor, (row, column) as two int8 (low byte = row).  A sample that
+// touches no pixel is kCodeNone.  Offsets beyond +-126 are clamped: the
+// grad_value pass only trusts codes for images whose reach is at most 126.
+constexpr uint16_t kCodeNone = 0x8080;
+constexpr int kCodeReach = 126;
+// Candidate output pixels a grad_value CTA lists in shared memory (beyond that
+// it walks its whole candidate window instead).
+constexpr int kListCap = 4096;
+
+__device__ __forceinline__ uint16_t cell_code(bool any, int dh, int dw) {
+    if (!any) return kCodeNone;
+    dh = min(127, max(-127, dh));
+    dw = min(127, max(-127, dw));
+    return static_cast<uint16_t>((dh & 0xff) | ((dw & 0xff) << 8));
+}
+
 // Grid cell (ih, iw) of sampling point k (columns outer, rows inner, centre
 // skipped when remove_center is set).
 __device__ __forceinline__ void grid_cell_of(const Geometry& g, int k, int& ih, int& iw) {
@@ -92,9 +111,11 @@ __device__ __forceinline__ void grid_cell_of(const Geometry& g, int k, int& ih, 
 template <typename T, int VEC, int KH, int KW, bool RC>
 __global__ void __launch_bounds__(256) samples_kernel(const Geometry g, const T* __restrict__ value,
                                                       const T* __restrict__ om, const T* __restrict__ gout,
-                                                      T* __restrict__ gom, int* __restrict__ reach) {
+                                                      T* __restrict__ gom, int* __restrict__ reach,
+                                                      uint16_t* __restrict__ codes, uint32_t* __restrict__ boxes) {
     extern __shared__ __align__(16) unsigned char smem[];
     __shared__ int s_reach;
+    __shared__ int s_box[4 * 256];  // per tile pixel: min/max cell row, min/max cell column (relative)
     constexpr int EPV = Elem<T>::per16;
     constexpr int PAIRS = VEC * EPV / 2;
     const int tile_elems = g.TH * g.TW * g.P;
@@ -104,6 +125,12 @@ __global__ void __launch_bounds__(256) samples_kernel(const Geometry g, const T*
     const Tile t = tile_of_block(g);
     stage_tile_rows(om_s, om, g, t);
     for (int i = threadIdx.x; i < tile_elems; i += blockDim.x) gom_s[i] = 0.f;
+    for (int i = threadIdx.x; i < g.TH * g.TW; i += blockDim.x) {
+        s_box[4 * i] = 127;
+        s_box[4 * i + 1] = -128;
+        s_box[4 * i + 2] = 127;
+        s_box[4 * i + 3] = -128;
+    }
     if (threadIdx.x == 0) s_reach = -1;
     __syncthreads();
 
@@ -130,8 +157,12 @@ __global__ void __launch_bounds__(256) samples_kernel(const Geometry g, const T*
     const int hb = ho * g.sh - g.ph, wb = wo * g.sw - g.pw;
 
     float2 gy[PAIRS];
-    load_gy<T, VEC>(gy, gout + ((static_cast<long long>(t.n) * g.Ho + ho) * g.Wo + wo) * g.C + ch_off);
+    const long long pix = (static_cast<long long>(t.n) * g.Ho + ho) * g.Wo + wo;
+    load_gy<T, VEC>(gy, gout + pix * g.C + ch_off);
+    uint16_t* code = codes + (pix * g.G + grp) * K;  // codes[N, Ho, Wo, G, K]
+    const bool writer = active && sl == 0;
     int my_reach = -1;
+    int bmin_h = 127, bmax_h = -128, bmin_w = 127, bmax_w = -128;  // cells relative to (hb, wb)
 
     int k = 0;
 #pragma unroll
@@ -170,14 +201,32 @@ __global__ void __launch_bounds__(256) samples_kernel(const Geometry g, const T*
                 const int dh = max(abs(cell.h0 - ah), abs(cell.h0 + 1 - ah));
                 const int dw = max(abs(cell.w0 - aw), abs(cell.w0 + 1 - aw));
                 my_reach = max(my_reach, max(dh, dw));
+                bmin_h = min(bmin_h, cell.h0 - hb);
+                bmax_h = max(bmax_h, cell.h0 - hb);
+                bmin_w = min(bmin_w, cell.w0 - wb);
+                bmax_w = max(bmax_w, cell.w0 - wb);
             }
+            if (writer) code[kk] = cell_code(cell.any, cell.h0 - ah, cell.w0 - aw);
         }
     }
 
     for (int off = 16; off > 0; off >>= 1) my_reach = max(my_reach, __shfl_xor_sync(0xffffffffu, my_reach, off));
     if ((threadIdx.x & 31) == 0 && my_reach >= 0) atomicMax(&s_reach, my_reach);
+    if (writer && bmax_h >= bmin_h) {
+        atomicMin(&s_box[4 * lp], max(-127, bmin_h));
+        atomicMax(&s_box[4 * lp + 1], min(127, bmax_h));
+        atomicMin(&s_box[4 * lp + 2], max(-127, bmin_w));
+        atomicMax(&s_box[4 * lp + 3], min(127, bmax_w));
+    }
     __syncthreads();
     if (threadIdx.x == 0 && s_reach >= 0) atomicMax(reach + t.n, s_reach);
+    for (int i = threadIdx.x; i < t.th * g.TW; i += blockDim.x) {
+        const int r2 = i / g.TW, c2 = i - r2 * g.TW;
+        if (c2 >= t.tw) continue;
+        const long long bp = (static_cast<long long>(t.n) * g.Ho + t.ho0 + r2) * g.Wo + t.wo0 + c2;
+        boxes[bp] = (s_box[4 * i] & 0xff) | ((s_box[4 * i + 1] & 0xff) << 8) | ((s_box[4 * i + 2] & 0xff) << 16) |
+                    (static_cast<uint32_t>(s_box[4 * i + 3] & 0xff) << 24);
+    }
 
     // grad_offset_mask rows of the tile, 16-byte stores.
     const int row_vecs = t.tw * g.P / EPV;
@@ -245,10 +294,14 @@ __device__ __forceinline__ Candidate candidate(const Geometry& g, const T* om_ro
 template <typename T, int VEC>
 __global__ void __launch_bounds__(1024) value_kernel(const Geometry g, const T* __restrict__ om,
                                                      const T* __restrict__ gout, T* __restrict__ gvalue,
-                                                     const int* __restrict__ reach) {
+                                                     const int* __restrict__ reach,
+                                                     const uint16_t* __restrict__ codes,
+                                                     const uint32_t* __restrict__ boxes) {
     extern __shared__ __align__(16) unsigned char smem[];
     __shared__ int s_warp[32];
     __shared__ int s_total;
+    __shared__ int s_nlist;
+    __shared__ uint32_t s_list[kListCap];  // output pixels whose cells reach the tile: (ho << 16) | wo
     constexpr int EPV = Elem<T>::per16;
     constexpr int PAIRS = VEC * EPV / 2;
 
@@ -266,8 +319,16 @@ __global__ void __launch_bounds__(1024) value_kernel(const Geometry g, const T* 
     int* cur = cnt + nbins;
     float4* rec = reinterpret_cast<float4*>(smem + ((2 * nbins * sizeof(int) + 15) / 16) * 16);
 
-    // Output pixels whose samples can touch the tile: anchors within R of it.
+    // Samples that can touch the tile come from output pixels whose anchor
+    // (for the sample's grid point) lies within R of the tile.
     const int R = reach[n];
+
+    // Candidate output pixels: anchors within R of the tile (the union over
+    // grid points).  Each is kept if the bounding box of its samples' cells
+    // (from the sample pass) meets the tile's cells.
+    const int GK = g.G * g.K;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+    const bool use_codes = R <= kCodeReach;  // else cells are re-formed from the offsets
     int ho_lo = 0, ho_hi = -1, wo_lo = 0, wo_hi = -1;
     if (R >= 0) {
         ho_lo = max(0, ceil_div(y0 - R + g.ph - (g.kh - 1) * g.dh, g.sh));
@@ -277,9 +338,44 @@ __global__ void __launch_bounds__(1024) value_kernel(const Geometry g, const T* 
     }
     const int e_w = max(0, wo_hi - wo_lo + 1);
     const int e_cnt = e_w * max(0, ho_hi - ho_lo + 1);
+    const long long pix0 = static_cast<long long>(n) * g.Ho * g.Wo;
 
-    // Scan mapping: thread -> fixed (group, point), a slot of pixels per step.
-    const int GK = g.G * g.K;
+    if (threadIdx.x == 0) s_nlist = 0;
+    for (int i = threadIdx.x; i < nbins; i += blockDim.x) cnt[i] = 0;
+    __syncthreads();
+    if (use_codes && R + max((g.kh - 1) * g.dh, (g.kw - 1) * g.dw) <= 127) {
+        for (int e0 = warp * 32; e0 < e_cnt; e0 += nwarps * 32) {
+            const int e = e0 + lane;
+            bool keep = false;
+            int ho = 0, wo = 0;
+            if (e < e_cnt) {
+                ho = ho_lo + e / e_w;
+                wo = wo_lo + (e - (e / e_w) * e_w);
+                const uint32_t box = boxes[pix0 + static_cast<long long>(ho) * g.Wo + wo];
+                const int bh0 = ho * g.sh - g.ph, bw0 = wo * g.sw - g.pw;
+                const int rmin = bh0 + static_cast<int8_t>(box & 0xff), rmax = bh0 + static_cast<int8_t>((box >> 8) & 0xff);
+                const int cmin = bw0 + static_cast<int8_t>((box >> 16) & 0xff), cmax = bw0 + static_cast<int8_t>(box >> 24);
+                keep = rmax >= y0 - 1 && rmin <= y0 + bh - 1 && cmax >= x0 - 1 && cmin <= x0 + bw - 1;
+            }
+            const unsigned ball = __ballot_sync(0xffffffffu, keep);
+            int base = 0;
+            if (lane == 0 && ball) base = atomicAdd(&s_nlist, __popc(ball));
+            base = __shfl_sync(0xffffffffu, base, 0);
+            const int pos = base + __popc(ball & ((1u << lane) - 1));
+            if (keep && pos < kListCap) s_list[pos] = (static_cast<uint32_t>(ho) << 16) | static_cast<uint32_t>(wo);
+        }
+    }
+    __syncthreads();
+    // The list is used when codes are valid, coordinates fit 16 bits and it did not overflow.
+    // (Boxes are relative to the pixel's grid origin, so they also span the
+    // grid itself: they are exact only while that stays within int8.)
+    const bool listed = use_codes && R + max((g.kh - 1) * g.dh, (g.kw - 1) * g.dw) <= 127 && s_nlist <= kListCap &&
+                        g.Ho <= 65535 && g.Wo <= 65535;
+    const int nlist = s_nlist;
+
+    // Scan mapping: each thread keeps one (group, point) and walks the listed
+    // pixels (or, without a list, every pixel whose anchor for that point is
+    // within R of the tile), a slot of pixels at a time.
     const int spt = blockDim.x / GK;
     const int tslot = threadIdx.x / GK;
     const int gk = threadIdx.x - tslot * GK;
@@ -288,74 +384,109 @@ __global__ void __launch_bounds__(1024) value_kernel(const Geometry g, const T* 
     const int sk = gk - sg * g.K;
     int s_ih, s_iw;
     grid_cell_of(g, sk, s_ih, s_iw);
-    const T* om_img = om + static_cast<long long>(n) * g.Ho * g.Wo * g.P + sg * 3 * g.K;
-
-    for (int i = threadIdx.x; i < nbins; i += blockDim.x) cnt[i] = 0;
-    __syncthreads();
-
-    // Pass 1: count the samples of each (group, cell).
-    if (scanner) {
-        for (int e = tslot; e < e_cnt; e += spt) {
-            const int eh = e / e_w;
-            const int ho = ho_lo + eh, wo = wo_lo + (e - eh * e_w);
-            const Candidate c = candidate(g, om_img + static_cast<long long>(ho * g.Wo + wo) * g.P, sk, ho, wo, s_ih, s_iw);
-            const int ch = c.h0 - (y0 - 1), cw = c.w0 - (x0 - 1);
-            if (c.any && ch >= 0 && ch <= bh && cw >= 0 && cw <= bw) atomicAdd(&cnt[sg * cells + ch * cells_w + cw], 1);
-        }
+    const int ah0 = s_ih * g.dh - g.ph, aw0 = s_iw * g.dw - g.pw;  // anchor = (ho*sh + ah0, wo*sw + aw0)
+    int kh_lo = 0, kh_hi = -1, kw_lo = 0, kw_hi = -1;
+    if (R >= 0) {
+        kh_lo = max(0, ceil_div(y0 - R - ah0, g.sh));
+        kh_hi = min(g.Ho - 1, floor_div(y0 + bh - 1 + R - ah0, g.sh));
+        kw_lo = max(0, ceil_div(x0 - R - aw0, g.sw));
+        kw_hi = min(g.Wo - 1, floor_div(x0 + bw - 1 + R - aw0, g.sw));
     }
-    __syncthreads();
+    const int k_w = max(0, kw_hi - kw_lo + 1);
+    const int k_cnt = listed ? nlist : k_w * max(0, kh_hi - kh_lo + 1);
+    const uint16_t* code_n = codes + pix0 * GK + gk;
+    const T* om_n = om + pix0 * g.P + sg * 3 * g.K;
 
-    // Exclusive scan of the counts -> cursors (block-wide, thread-contiguous chunks).
-    {
-        const int per = (nbins + blockDim.x - 1) / blockDim.x;
-        const int b0 = threadIdx.x * per;
-        int local = 0;
-        for (int b = b0; b < min(nbins, b0 + per); ++b) local += cnt[b];
-        const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-        int incl = local;
-        for (int o = 1; o < 32; o <<= 1) {
-            const int v = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += v;
-        }
-        if (lane == 31) s_warp[wid] = incl;
-        __syncthreads();
-        if (wid == 0) {
-            const int nw = (blockDim.x + 31) >> 5;
-            int v = lane < nw ? s_warp[lane] : 0;
+    // Pass 0 counts the samples of each (group, cell); pass 1 places their
+    // records (image pixel of p, m(1-lh), m lh, lw) in bin order.
+    bool sorted = true;
+    for (int pass = 0; pass < 2; ++pass) {
+        if (pass == 1) {
+            // Exclusive scan of the counts -> cursors (block-wide, thread-contiguous chunks).
+            const int per = (nbins + blockDim.x - 1) / blockDim.x;
+            const int b0 = threadIdx.x * per;
+            int local = 0;
+            for (int b = b0; b < min(nbins, b0 + per); ++b) local += cnt[b];
+            int incl = local;
             for (int o = 1; o < 32; o <<= 1) {
-                const int u = __shfl_up_sync(0xffffffffu, v, o);
-                if (lane >= o) v += u;
+                const int v = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += v;
             }
-            if (lane < nw) s_warp[lane] = v;  // inclusive warp totals
-            if (lane == nw - 1) s_total = v;
+            if (lane == 31) s_warp[warp] = incl;
+            __syncthreads();
+            if (warp == 0) {
+                int v = lane < nwarps ? s_warp[lane] : 0;
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int u = __shfl_up_sync(0xffffffffu, v, o);
+                    if (lane >= o) v += u;
+                }
+                if (lane < nwarps) s_warp[lane] = v;  // inclusive warp totals
+                if (lane == nwarps - 1) s_total = v;
+            }
+            __syncthreads();
+            int run = incl - local + (warp > 0 ? s_warp[warp - 1] : 0);
+            for (int b = b0; b < min(nbins, b0 + per); ++b) {
+                cur[b] = run;
+                run += cnt[b];
+            }
+            __syncthreads();
+            sorted = s_total <= g.bcap;
+            if (!sorted) break;
+        }
+        if (scanner && tslot < k_cnt) {
+            int ho = 0, wo = 0;
+            if (!listed) {
+                const int eh = tslot / k_w;
+                ho = kh_lo + eh;
+                wo = kw_lo + tslot - eh * k_w;
+            }
+            for (int e = tslot; e < k_cnt; e += spt) {
+                if (listed) {
+                    const uint32_t lv = s_list[e];
+                    ho = static_cast<int>(lv >> 16);
+                    wo = static_cast<int>(lv & 0xffff);
+                }
+                const long long pix = static_cast<long long>(ho) * g.Wo + wo;
+                int h0, w0;
+                bool any;
+                Candidate c;
+                if (use_codes) {
+                    const uint16_t cd = code_n[pix * GK];
+                    any = cd != kCodeNone;
+                    h0 = ho * g.sh + ah0 + static_cast<int8_t>(cd & 0xff);
+                    w0 = wo * g.sw + aw0 + static_cast<int8_t>(cd >> 8);
+                } else {
+                    c = candidate(g, om_n + pix * g.P, sk, ho, wo, s_ih, s_iw);
+                    any = c.any;
+                    h0 = c.h0;
+                    w0 = c.w0;
+                }
+                const int ch = h0 - (y0 - 1), cw = w0 - (x0 - 1);
+                if (any && static_cast<unsigned>(ch) <= static_cast<unsigned>(bh) &&
+                    static_cast<unsigned>(cw) <= static_cast<unsigned>(bw)) {
+                    const int bin = sg * cells + ch * cells_w + cw;
+                    if (pass == 0) {
+                        atomicAdd(&cnt[bin], 1);
+                    } else {
+                        const T* orow = om_n + pix * g.P;
+                        if (use_codes) c = candidate(g, orow, sk, ho, wo, s_ih, s_iw);
+                        const int slot = atomicAdd(&cur[bin], 1);
+                        const float m = to_f32(orow[2 * g.K + sk]);
+                        const float b = m * c.lh;
+                        rec[slot] = make_float4(__int_as_float(static_cast<int>(pix)), m - b, b, c.lw);
+                    }
+                }
+                if (!listed) {  // next pixel of this slot
+                    wo += spt;
+                    while (wo > kw_hi) {
+                        wo -= k_w;
+                        ++ho;
+                    }
+                }
+            }
         }
         __syncthreads();
-        int run = incl - local + (wid > 0 ? s_warp[wid - 1] : 0);
-        for (int b = b0; b < min(nbins, b0 + per); ++b) {
-            cur[b] = run;
-            run += cnt[b];
-        }
     }
-    __syncthreads();
-    const bool sorted = s_total <= g.bcap;
-
-    // Pass 2: place each sample's record (image pixel of p, m(1-lh), m lh, lw) in its bin.
-    if (sorted && scanner) {
-        for (int e = tslot; e < e_cnt; e += spt) {
-            const int eh = e / e_w;
-            const int ho = ho_lo + eh, wo = wo_lo + (e - eh * e_w);
-            const T* orow = om_img + static_cast<long long>(ho * g.Wo + wo) * g.P;
-            const Candidate c = candidate(g, orow, sk, ho, wo, s_ih, s_iw);
-            const int ch = c.h0 - (y0 - 1), cw = c.w0 - (x0 - 1);
-            if (c.any && ch >= 0 && ch <= bh && cw >= 0 && cw <= bw) {
-                const int slot = atomicAdd(&cur[sg * cells + ch * cells_w + cw], 1);
-                const float m = to_f32(orow[2 * g.K + sk]);
-                const float b = m * c.lh;
-                rec[slot] = make_float4(__int_as_float(ho * g.Wo + wo), m - b, b, c.lw);
-            }
-        }
-    }
-    __syncthreads();
 
     // Pull: thread -> (input pixel q of the tile, group, slice).
     const int lanes_pp = g.G * g.nslice;
@@ -380,6 +511,7 @@ __global__ void __launch_bounds__(1024) value_kernel(const Geometry g, const T* 
             for (int b = 0; b < 2; ++b) {
                 const int bin = grp * cells + (qy - a + 1) * cells_w + (qx - b + 1);
                 const int end = cur[bin];
+#pragma unroll 2
                 for (int j = end - cnt[bin]; j < end; ++j) {
                     const float4 rcd = rec[j];
                     const float wt = (a ? rcd.z : rcd.y) * (b ? rcd.w : 1.f - rcd.w);
@@ -389,11 +521,17 @@ __global__ void __launch_bounds__(1024) value_kernel(const Geometry g, const T* 
         }
     } else {
         // Overflow path: scan every candidate sample of this group directly.
+        const int uh_lo = max(0, ceil_div(y0 - R + g.ph - (g.kh - 1) * g.dh, g.sh));
+        const int uh_hi = min(g.Ho - 1, floor_div(y0 + bh - 1 + R + g.ph, g.sh));
+        const int uw_lo = max(0, ceil_div(x0 - R + g.pw - (g.kw - 1) * g.dw, g.sw));
+        const int uw_hi = min(g.Wo - 1, floor_div(x0 + bw - 1 + R + g.pw, g.sw));
+        const int u_w = max(0, uw_hi - uw_lo + 1);
+        const int u_cnt = u_w * max(0, uh_hi - uh_lo + 1);
         const int gy_abs = y0 + qy, gx_abs = x0 + qx;
         const T* om_g = om + static_cast<long long>(n) * g.Ho * g.Wo * g.P + grp * 3 * g.K;
-        for (int e = 0; e < e_cnt; ++e) {
-            const int eh = e / e_w;
-            const int ho = ho_lo + eh, wo = wo_lo + (e - eh * e_w);
+        for (int e = 0; e < u_cnt; ++e) {
+            const int eh = e / u_w;
+            const int ho = uh_lo + eh, wo = uw_lo + (e - eh * u_w);
             const T* orow = om_g + static_cast<long long>(ho * g.Wo + wo) * g.P;
             for (int k = 0; k < g.K; ++k) {
                 int ih, iw;
@@ -421,15 +559,16 @@ __global__ void __launch_bounds__(1024) value_kernel(const Geometry g, const T* 
 // Launchers
 // ---------------------------------------------------------------------------
 
+// Opt the kernel in to `smem` bytes of dynamic shared memory (needed whenever
+// static + dynamic exceed the 48 KB default).
 template <typename Kern>
 cudaError_t allow_smem(Kern kern, size_t smem) {
-    if (smem <= 48 * 1024) return cudaSuccess;
     return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
 }
 
 template <typename T, int VEC, int KH, int KW, bool RC>
 cudaError_t launch_samples_typed(const Geometry& g, const void* value, const void* om, const void* gout, void* gom,
-                                 int* reach, cudaStream_t stream) {
+                                 int* reach, uint16_t* codes, uint32_t* boxes, cudaStream_t stream) {
     const size_t smem = backward_smem_bytes(g, sizeof(T));
     auto kern = samples_kernel<T, VEC, KH, KW, RC>;
     cudaError_t e = allow_smem(kern, smem);
@@ -438,45 +577,46 @@ cudaError_t launch_samples_typed(const Geometry& g, const void* value, const voi
     const int threads = (g.pix_per_cta * g.G * g.nslice + 31) / 32 * 32;  // whole warps (shuffles)
     kern<<<static_cast<unsigned>(blocks), threads, smem, stream>>>(g, static_cast<const T*>(value),
                                                                    static_cast<const T*>(om), static_cast<const T*>(gout),
-                                                                   static_cast<T*>(gom), reach);
+                                                                   static_cast<T*>(gom), reach, codes, boxes);
     return cudaGetLastError();
 }
 
 template <typename T, int VEC>
 cudaError_t launch_samples_grid(const Geometry& g, const void* value, const void* om, const void* gout, void* gom,
-                                int* reach, cudaStream_t stream) {
+                                int* reach, uint16_t* codes, uint32_t* boxes, cudaStream_t stream) {
     if (g.kh == 3 && g.kw == 3) {
-        return g.remove_center ? launch_samples_typed<T, VEC, 3, 3, true>(g, value, om, gout, gom, reach, stream)
-                               : launch_samples_typed<T, VEC, 3, 3, false>(g, value, om, gout, gom, reach, stream);
+        return g.remove_center
+                   ? launch_samples_typed<T, VEC, 3, 3, true>(g, value, om, gout, gom, reach, codes, boxes, stream)
+                   : launch_samples_typed<T, VEC, 3, 3, false>(g, value, om, gout, gom, reach, codes, boxes, stream);
     }
-    return launch_samples_typed<T, VEC, 0, 0, false>(g, value, om, gout, gom, reach, stream);
+    return launch_samples_typed<T, VEC, 0, 0, false>(g, value, om, gout, gom, reach, codes, boxes, stream);
 }
 
 template <typename T>
 cudaError_t launch_samples_vec(const Geometry& g, const void* value, const void* om, const void* gout, void* gom,
-                               int* reach, cudaStream_t stream) {
-    return g.vec == 2 ? launch_samples_grid<T, 2>(g, value, om, gout, gom, reach, stream)
-                      : launch_samples_grid<T, 1>(g, value, om, gout, gom, reach, stream);
+                               int* reach, uint16_t* codes, uint32_t* boxes, cudaStream_t stream) {
+    return g.vec == 2 ? launch_samples_grid<T, 2>(g, value, om, gout, gom, reach, codes, boxes, stream)
+                      : launch_samples_grid<T, 1>(g, value, om, gout, gom, reach, codes, boxes, stream);
 }
 
 template <typename T, int VEC>
 cudaError_t launch_value_typed(const Geometry& g, const void* om, const void* gout, void* gvalue, const int* reach,
-                               cudaStream_t stream) {
+                               const uint16_t* codes, const uint32_t* boxes, cudaStream_t stream) {
     const size_t smem = backward_value_smem_bytes(g);
     auto kern = value_kernel<T, VEC>;
     cudaError_t e = allow_smem(kern, smem);
     if (e != cudaSuccess) return e;
     const long long blocks = static_cast<long long>(g.N) * g.btiles_h * g.btiles_w;
     kern<<<static_cast<unsigned>(blocks), g.bthreads, smem, stream>>>(
-        g, static_cast<const T*>(om), static_cast<const T*>(gout), static_cast<T*>(gvalue), reach);
+        g, static_cast<const T*>(om), static_cast<const T*>(gout), static_cast<T*>(gvalue), reach, codes, boxes);
     return cudaGetLastError();
 }
 
 template <typename T>
 cudaError_t launch_value_vec(const Geometry& g, const void* om, const void* gout, void* gvalue, const int* reach,
-                             cudaStream_t stream) {
-    return g.vec == 2 ? launch_value_typed<T, 2>(g, om, gout, gvalue, reach, stream)
-                      : launch_value_typed<T, 1>(g, om, gout, gvalue, reach, stream);
+                             const uint16_t* codes, const uint32_t* boxes, cudaStream_t stream) {
+    return g.vec == 2 ? launch_value_typed<T, 2>(g, om, gout, gvalue, reach, codes, boxes, stream)
+                      : launch_value_typed<T, 1>(g, om, gout, gvalue, reach, codes, boxes, stream);
 }
 
 }  // namespace
@@ -491,21 +631,22 @@ size_t backward_value_smem_bytes(const Geometry& g) {
 }
 
 cudaError_t launch_backward_samples(const Geometry& g, int dtype, const void* value, const void* om, const void* gout,
-                                    void* gom, int* reach, cudaStream_t stream) {
+                                    void* gom, int* reach, uint16_t* codes, uint32_t* boxes, cudaStream_t stream) {
     switch (dtype) {
-        case 0: return launch_samples_vec<float>(g, value, om, gout, gom, reach, stream);
-        case 1: return launch_samples_vec<__half>(g, value, om, gout, gom, reach, stream);
-        case 2: return launch_samples_vec<__nv_bfloat16>(g, value, om, gout, gom, reach, stream);
+        case 0: return launch_samples_vec<float>(g, value, om, gout, gom, reach, codes, boxes, stream);
+        case 1: return launch_samples_vec<__half>(g, value, om, gout, gom, reach, codes, boxes, stream);
+        case 2: return launch_samples_vec<__nv_bfloat16>(g, value, om, gout, gom, reach, codes, boxes, stream);
         default: return cudaErrorInvalidValue;
     }
 }
 
 cudaError_t launch_backward_value(const Geometry& g, int dtype, const void* om, const void* gout, void* gvalue,
-                                  const int* reach, cudaStream_t stream) {
+                                  const int* reach, const uint16_t* codes, const uint32_t* boxes,
+                                  cudaStream_t stream) {
     switch (dtype) {
-        case 0: return launch_value_vec<float>(g, om, gout, gvalue, reach, stream);
-        case 1: return launch_value_vec<__half>(g, om, gout, gvalue, reach, stream);
-        case 2: return launch_value_vec<__nv_bfloat16>(g, om, gout, gvalue, reach, stream);
+        case 0: return launch_value_vec<float>(g, om, gout, gvalue, reach, codes, boxes, stream);
+        case 1: return launch_value_vec<__half>(g, om, gout, gvalue, reach, codes, boxes, stream);
+        case 2: return launch_value_vec<__nv_bfloat16>(g, om, gout, gvalue, reach, codes, boxes, stream);
         default: return cudaErrorInvalidValue;
     }
 }

@@ -236,11 +236,15 @@ namespace dcn4 {
 cudaError_t launch_forward(const Geometry& g, int dtype, const void* value, const void* om, void* out,
                            cudaStream_t stream);
 // grad_offset_mask and the per-image reach (int[N], pre-filled with -1).
+// Also writes one 2-byte cell code per sample, codes[N, Ho, Wo, G, K], and the
+// bounding box of each output pixel's cells, boxes[N, Ho, Wo].
 cudaError_t launch_backward_samples(const Geometry& g, int dtype, const void* value, const void* om,
-                                    const void* gout, void* gom, int* reach, cudaStream_t stream);
-// grad_value from the reach written by launch_backward_samples.
+                                    const void* gout, void* gom, int* reach, uint16_t* codes, uint32_t* boxes,
+                                    cudaStream_t stream);
+// grad_value from the reach, cell codes and boxes written by launch_backward_samples.
 cudaError_t launch_backward_value(const Geometry& g, int dtype, const void* om, const void* gout, void* gvalue,
-                                  const int* reach, cudaStream_t stream);
+                                  const int* reach, const uint16_t* codes, const uint32_t* boxes,
+                                  cudaStream_t stream);
 // Dynamic shared memory bytes of one CTA.
 size_t forward_smem_bytes(const Geometry& g, int elem_bytes);
 size_t backward_smem_bytes(const Geometry& g, int elem_bytes);

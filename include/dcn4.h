@@ -117,8 +117,10 @@ int dcn4_check_params(const dcn4_params* p);
 int dcn4_forward(const dcn4_params* p, const void* value, const void* offset_mask, void* out,
                  void* stream);
 
-/* Bytes of device workspace dcn4_backward needs: one 32-bit word per image
- * (N*4 rounded up to 256), whatever the dtype; 0 if p is invalid. */
+/* Bytes of device workspace dcn4_backward needs, whatever the dtype:
+ * one 32-bit word per image (N*4 rounded up to 256), one 32-bit cell box per
+ * output pixel (N*Ho*Wo*4 rounded up to 256) and one 16-bit cell code per
+ * sample (N*Ho*Wo*G*K*2); 0 if p is invalid. */
 size_t dcn4_backward_workspace_size(const dcn4_params* p);
 
 /* Backward of the forward for upstream gradient grad_out:
@@ -130,7 +132,8 @@ size_t dcn4_backward_workspace_size(const dcn4_params* p);
  * accumulated into); the offset_mask padding tail is written as 0.
  * `workspace` (device, 16-byte aligned, >= dcn4_backward_workspace_size bytes)
  * is scratch, clobbered by the call: it receives, per image, how far any
- * sample reaches from its grid position.
+ * sample reaches from its grid position, and per sample the bilinear cell it
+ * falls in relative to that position.
  * Launches, on `stream`: a memset of that word per image, one kernel for
  * grad_offset_mask (and the reach), and one for grad_value.  grad_value is
  * not scattered with atomics: each element is summed by one thread in fp32
