@@ -79,6 +79,9 @@ def _load() -> ctypes.CDLL:
         "dcn4_backward": ([P, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp], ctypes.c_int),
         "dcn4_status_string": ([ctypes.c_int], ctypes.c_char_p),
         "dcn4_last_error": ([], ctypes.c_char_p),
+        "dcn4_backward_noalloc": ([P, vp, vp, vp, vp, vp, vp], ctypes.c_int),
+        "dcn4_backward_noalloc_capacity": ([], ctypes.c_size_t),
+        "dcn4_noalloc_last_error": ([], ctypes.c_char_p),
     }
     for name, (args, res) in sig.items():
         fn = getattr(L, name)
@@ -129,6 +132,22 @@ def dcn4_backward(p: dcn4_params, value, offset_mask, grad_out, grad_value, grad
                   workspace, workspace_bytes: int, stream=None) -> int:
     return lib.dcn4_backward(ctypes.byref(p), value, offset_mask, grad_out, grad_value,
                              grad_offset_mask, workspace, workspace_bytes, stream)
+
+
+def dcn4_backward_noalloc(p: dcn4_params, value, offset_mask, grad_out, grad_value, grad_offset_mask,
+                          stream=None) -> int:
+    """dcn4_backward with the library's built-in scratch area instead of a workspace
+    (for callers that cannot provide device memory when they call)."""
+    return lib.dcn4_backward_noalloc(ctypes.byref(p), value, offset_mask, grad_out, grad_value,
+                                     grad_offset_mask, stream)
+
+
+def dcn4_backward_noalloc_capacity() -> int:
+    return lib.dcn4_backward_noalloc_capacity()
+
+
+def dcn4_noalloc_last_error() -> str:
+    return lib.dcn4_noalloc_last_error().decode()
 
 
 def dcn4_status_string(status: int) -> str:

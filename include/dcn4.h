@@ -143,6 +143,41 @@ int dcn4_backward(const dcn4_params* p, const void* value, const void* offset_ma
                   const void* grad_out, void* grad_value, void* grad_offset_mask,
                   void* workspace, size_t workspace_bytes, void* stream);
 
+/* ---------------------------------------------------------------------------
+ * Backward without a caller-provided workspace.
+ *
+ * This entry point has no counterpart in the paper: it exists for callers that
+ * cannot give the library device memory when they call it, such as a plugin
+ * inside a host runtime that owns every device buffer and offers no
+ * allocator, or a service that fixes its device-memory budget at start-up.
+ * It computes exactly what dcn4_backward computes, taking its scratch from a
+ * fixed area that this library reserves on every device that loads it
+ * (DCN4_NOALLOC_SCRATCH_BYTES, 64 MiB, held until the process exits); it calls
+ * no cudaMalloc, cudaFree or allocating library routine.
+ *   - Sizes: the problem's dcn4_backward_workspace_size must not exceed
+ *     dcn4_backward_noalloc_capacity(); larger problems are rejected with
+ *     DCN4_ERR_WORKSPACE before anything is launched (detail in
+ *     dcn4_noalloc_last_error()).
+ *   - Set-up: the first call on a device (made with that device current) looks
+ *     up the area's device address; make that first call before any stream
+ *     capture begins.
+ *   - Sharing: every call on a device uses the same area, which keeps the
+ *     last call's contents (each call resets what it needs).  Calls whose
+ *     executions overlap on the GPU (different streams, no ordering between
+ *     them) race on the area and give wrong results: order them.
+ * Arguments, layouts, errors and launches are those of dcn4_backward. */
+#define DCN4_NOALLOC_SCRATCH_BYTES (64u << 20)
+
+int dcn4_backward_noalloc(const dcn4_params* p, const void* value, const void* offset_mask,
+                          const void* grad_out, void* grad_value, void* grad_offset_mask, void* stream);
+
+/* Bytes of scratch dcn4_backward_noalloc can use (DCN4_NOALLOC_SCRATCH_BYTES). */
+size_t dcn4_backward_noalloc_capacity(void);
+
+/* Detail of the last failing dcn4_backward_noalloc size or set-up check on
+ * this host thread ("" if none; launch errors are in dcn4_last_error()). */
+const char* dcn4_noalloc_last_error(void);
+
 /* Name of a dcn4_status. */
 const char* dcn4_status_string(int status);
 
