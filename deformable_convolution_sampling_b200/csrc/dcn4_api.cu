@@ -39,12 +39,10 @@ constexpr size_t kSmemDefault = 48 * 1024;
 constexpr size_t kSmemMax = 227 * 1024;
 // grad_value pass: up to 1024 threads and 256 input pixels per CTA; sample
 // records get what is left of this shared-memory budget after the bins.
-constexpr int kValueThreads = 1024;
-#ifndef DCN4_VALUE_PIXELS
-#define DCN4_VALUE_PIXELS 256
-#endif
-constexpr int kValuePixels = DCN4_VALUE_PIXELS;
+constexpr int kValueThreads = 512;
+constexpr int kValuePixels = 128;
 constexpr size_t kValueSmem = 200 * 1024;
+constexpr int kValueListCap = 2048;  // candidate-pixel list entries (4 bytes each) per CTA
 
 // Validates p and fills the kernel geometry.  Touches no GPU state.
 // wide: the gathered and stored tensors are 32-byte aligned, so a thread may
@@ -100,7 +98,7 @@ int make_geometry(const dcn4_params* p, bool backward, bool wide, dcn4::Geometry
     // Output pixels per CTA: fill kTargetThreads, then shrink until the
     // shared-memory rows fit the default 48 KB (or, for very long rows, the
     // per-CTA maximum).
-    const size_t row_bytes = static_cast<size_t>(p->P) * (eb + (backward ? 4 : 0));
+    const size_t row_bytes = static_cast<size_t>(p->P) * eb * (backward ? 2 : 1);
     long long ppc = kTargetThreads / lanes_pp;
     while (ppc > 1 && ppc * row_bytes > kSmemDefault) --ppc;
     if (ppc * row_bytes > kSmemMax) return fail(DCN4_ERR_UNSUPPORTED, "P=%d rows do not fit shared memory", p->P);
@@ -140,14 +138,15 @@ int make_geometry(const dcn4_params* p, bool backward, bool wide, dcn4::Geometry
     if (GK > kValueThreads) return fail(DCN4_ERR_UNSUPPORTED, "G*K = %lld exceeds %d", GK, kValueThreads);
     if (bthreads < GK) bthreads = (GK + 31) / 32 * 32;
     const long long nbins = static_cast<long long>(p->G) * (BH + 1) * (BW + 1);
-    const long long bin_bytes = (2 * nbins * 4 + 15) / 16 * 16;
-    if (bin_bytes + 1024 * 16 > static_cast<long long>(kValueSmem))
+    const long long bin_bytes = ((2 * nbins + kValueListCap) * 4 + 15) / 16 * 16;
+    const long long brec = eb == 2 ? 8 : 16;
+    if (bin_bytes + 1024 * brec > static_cast<long long>(kValueSmem))
         return fail(DCN4_ERR_UNSUPPORTED, "too many groups for the grad_value tile");
     // Records: room for 1.25x the expected number of samples per tile (K per
     // cell for every output pixel per input pixel), within the budget; the
     // rest of the shared memory stays L1 for the grad_out gathers.
     const long long expect = nbins * K * std::max<long long>(1, (Ho * Wo + p->H * p->W - 1) / (p->H * p->W));
-    long long bcap = (static_cast<long long>(kValueSmem) - bin_bytes) / 16;
+    long long bcap = (static_cast<long long>(kValueSmem) - bin_bytes) / brec;
     bcap = std::max<long long>(1024, std::min(bcap, expect + expect / 4 + 256));
     const long long btiles_h = (p->H + BH - 1) / BH, btiles_w = (p->W + BW - 1) / BW;
     if (static_cast<long long>(p->N) * btiles_h * btiles_w > 0x7fffffffLL)
@@ -158,6 +157,7 @@ int make_geometry(const dcn4_params* p, bool backward, bool wide, dcn4::Geometry
     g->btiles_w = static_cast<int>(btiles_w);
     g->bthreads = static_cast<int>(bthreads);
     g->bcap = static_cast<int>(bcap);
+    g->brec = static_cast<int>(brec);
     return DCN4_OK;
 }
 

@@ -84,7 +84,7 @@ constexpr uint16_t kCodeNone = 0x8080;
 constexpr int kCodeReach = 126;
 // Candidate output pixels a grad_value CTA lists in shared memory (beyond that
 // it walks its whole candidate window instead).
-constexpr int kListCap = 4096;
+constexpr int kListCap = 2048;
 
 __device__ __forceinline__ uint16_t cell_code(bool any, int dh, int dw) {
     if (!any) return kCodeNone;
@@ -120,11 +120,11 @@ __global__ void __launch_bounds__(256) samples_kernel(const Geometry g, const T*
     constexpr int PAIRS = VEC * EPV / 2;
     const int tile_elems = g.TH * g.TW * g.P;
     T* om_s = reinterpret_cast<T*>(smem);
-    float* gom_s = reinterpret_cast<float*>(smem + tile_elems * sizeof(T));  // P % 8 == 0 keeps this 16-byte aligned
+    T* gom_s = reinterpret_cast<T*>(smem + tile_elems * sizeof(T));  // P % 8 == 0 keeps this 16-byte aligned
 
     const Tile t = tile_of_block(g);
     stage_tile_rows(om_s, om, g, t);
-    for (int i = threadIdx.x; i < tile_elems; i += blockDim.x) gom_s[i] = 0.f;
+    for (int i = threadIdx.x; i < tile_elems; i += blockDim.x) gom_s[i] = static_cast<T>(0.f);
     for (int i = threadIdx.x; i < g.TH * g.TW; i += blockDim.x) {
         s_box[4 * i] = 127;
         s_box[4 * i + 1] = -128;
@@ -193,10 +193,10 @@ __global__ void __launch_bounds__(256) samples_kernel(const Geometry g, const T*
                 if (sl == 0) {
                     const float hl = 1.f - cell.lh, wl = 1.f - cell.lw;
                     const float sm = g.s * m;
-                    float* gr = gom_s + lrow;
-                    gr[2 * kk] = sm * (hl * (d01 - d00) + cell.lh * (d11 - d10));
-                    gr[2 * kk + 1] = sm * (wl * (d10 - d00) + cell.lw * (d11 - d01));
-                    gr[2 * K + kk] = hl * (wl * d00 + cell.lw * d01) + cell.lh * (wl * d10 + cell.lw * d11);
+                    T* gr = gom_s + lrow;  // rounded once, to the I/O dtype
+                    gr[2 * kk] = from_f32<T>(sm * (hl * (d01 - d00) + cell.lh * (d11 - d10)));
+                    gr[2 * kk + 1] = from_f32<T>(sm * (wl * (d10 - d00) + cell.lw * (d11 - d01)));
+                    gr[2 * K + kk] = from_f32<T>(hl * (wl * d00 + cell.lw * d01) + cell.lh * (wl * d10 + cell.lw * d11));
                 }
                 const int dh = max(abs(cell.h0 - ah), abs(cell.h0 + 1 - ah));
                 const int dw = max(abs(cell.w0 - aw), abs(cell.w0 + 1 - aw));
@@ -233,12 +233,8 @@ __global__ void __launch_bounds__(256) samples_kernel(const Geometry g, const T*
     for (int i = threadIdx.x; i < t.th * row_vecs; i += blockDim.x) {
         const int rr = i / row_vecs;
         const int c = i - rr * row_vecs;
-        const float2* src = reinterpret_cast<const float2*>(gom_s + rr * g.TW * g.P + c * EPV);
-        float2 f[EPV / 2];
-#pragma unroll
-        for (int j = 0; j < EPV / 2; ++j) f[j] = src[j];
         const long long grow = (static_cast<long long>(t.n) * g.Ho + t.ho0 + rr) * g.Wo + t.wo0;
-        st_global(gom + grow * g.P + c * EPV, pack(f, T()));
+        st_global(gom + grow * g.P + c * EPV, *reinterpret_cast<const uint4*>(gom_s + rr * g.TW * g.P + c * EPV));
     }
 }
 
@@ -274,10 +270,24 @@ struct Candidate {
 };
 
 template <typename T>
+__device__ __forceinline__ float ld_stream_elem(const T* p) {
+    if constexpr (sizeof(T) == 2) {
+        const uint16_t b = ld_stream_u16(p);
+        T x;
+        memcpy(&x, &b, 2);
+        return to_f32(x);
+    } else {
+        float x;
+        asm volatile("ld.global.nc.L1::no_allocate.f32 %0, [%1];" : "=f"(x) : "l"(p));
+        return x;
+    }
+}
+
+template <typename T>
 __device__ __forceinline__ Candidate candidate(const Geometry& g, const T* om_row, int k, int ho, int wo, int ih,
                                                int iw) {
-    const float dx = to_f32(om_row[2 * k]);
-    const float dy = to_f32(om_row[2 * k + 1]);
+    const float dx = ld_stream_elem(om_row + 2 * k);
+    const float dy = ld_stream_elem(om_row + 2 * k + 1);
     const float h = __fmaf_rn(g.s, dy, static_cast<float>(ho * g.sh - g.ph + ih * g.dh));
     const float w = __fmaf_rn(g.s, dx, static_cast<float>(wo * g.sw - g.pw + iw * g.dw));
     Candidate c;
@@ -291,17 +301,35 @@ __device__ __forceinline__ Candidate candidate(const Geometry& g, const T* om_ro
     return c;
 }
 
-template <typename T, int VEC>
-__global__ void __launch_bounds__(1024) value_kernel(const Geometry g, const T* __restrict__ om,
-                                                     const T* __restrict__ gout, T* __restrict__ gvalue,
-                                                     const int* __restrict__ reach,
-                                                     const uint16_t* __restrict__ codes,
-                                                     const uint32_t* __restrict__ boxes) {
+// Sample records of the grad_value sort.  Wide (16 bytes, fp32 I/O): image
+// pixel index of p, m(1-lh), m lh, lw.  Compact (8 bytes, 16-bit I/O): index of
+// p in the CTA's candidate list, the mask's own 16 bits, and lh, lw as 16-bit
+// fixed point (error below 2^-17, far under the I/O rounding).
+__device__ __forceinline__ uint32_t fix16(float f) { return min(65535u, static_cast<uint32_t>(f * 65536.f + 0.5f)); }
+
+template <typename T>
+__device__ __forceinline__ uint16_t raw_bits(T x) {
+    uint16_t b;
+    memcpy(&b, &x, 2);
+    return b;
+}
+__device__ __forceinline__ float from_bits(uint16_t b, __half) {
+    __half h;
+    memcpy(&h, &b, 2);
+    return __half2float(h);
+}
+__device__ __forceinline__ float from_bits(uint16_t b, __nv_bfloat16) { return __uint_as_float(static_cast<uint32_t>(b) << 16); }
+
+template <typename T, int VEC, bool COMPACT>
+__global__ void __launch_bounds__(512, 2) value_kernel(const Geometry g, const T* __restrict__ om,
+                                                       const T* __restrict__ gout, T* __restrict__ gvalue,
+                                                       const int* __restrict__ reach,
+                                                       const uint16_t* __restrict__ codes,
+                                                       const uint32_t* __restrict__ boxes) {
     extern __shared__ __align__(16) unsigned char smem[];
     __shared__ int s_warp[32];
     __shared__ int s_total;
     __shared__ int s_nlist;
-    __shared__ uint32_t s_list[kListCap];  // output pixels whose cells reach the tile: (ho << 16) | wo
     constexpr int EPV = Elem<T>::per16;
     constexpr int PAIRS = VEC * EPV / 2;
 
@@ -317,18 +345,18 @@ __global__ void __launch_bounds__(1024) value_kernel(const Geometry g, const T* 
     const int nbins = g.G * cells;
     int* cnt = reinterpret_cast<int*>(smem);
     int* cur = cnt + nbins;
-    float4* rec = reinterpret_cast<float4*>(smem + ((2 * nbins * sizeof(int) + 15) / 16) * 16);
+    uint32_t* s_list = reinterpret_cast<uint32_t*>(cur + nbins);  // candidate pixels: (ho << 16) | wo
+    unsigned char* rec_base = smem + ((2 * nbins + kListCap) * sizeof(int) + 15) / 16 * 16;
+    float4* rec_w = reinterpret_cast<float4*>(rec_base);
+    uint2* rec_c = reinterpret_cast<uint2*>(rec_base);
 
     // Samples that can touch the tile come from output pixels whose anchor
     // (for the sample's grid point) lies within R of the tile.
     const int R = reach[n];
-
-    // Candidate output pixels: anchors within R of the tile (the union over
-    // grid points).  Each is kept if the bounding box of its samples' cells
-    // (from the sample pass) meets the tile's cells.
     const int GK = g.G * g.K;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
     const bool use_codes = R <= kCodeReach;  // else cells are re-formed from the offsets
+    const bool boxes_exact = use_codes && R + max((g.kh - 1) * g.dh, (g.kw - 1) * g.dw) <= 127;
     int ho_lo = 0, ho_hi = -1, wo_lo = 0, wo_hi = -1;
     if (R >= 0) {
         ho_lo = max(0, ceil_div(y0 - R + g.ph - (g.kh - 1) * g.dh, g.sh));
@@ -343,14 +371,17 @@ __global__ void __launch_bounds__(1024) value_kernel(const Geometry g, const T* 
     if (threadIdx.x == 0) s_nlist = 0;
     for (int i = threadIdx.x; i < nbins; i += blockDim.x) cnt[i] = 0;
     __syncthreads();
-    if (use_codes && R + max((g.kh - 1) * g.dh, (g.kw - 1) * g.dw) <= 127) {
+
+    // List the candidate pixels whose cell bounding box meets the tile's cells.
+    if (boxes_exact) {
         for (int e0 = warp * 32; e0 < e_cnt; e0 += nwarps * 32) {
             const int e = e0 + lane;
             bool keep = false;
             int ho = 0, wo = 0;
             if (e < e_cnt) {
-                ho = ho_lo + e / e_w;
-                wo = wo_lo + (e - (e / e_w) * e_w);
+                const int eh = e / e_w;
+                ho = ho_lo + eh;
+                wo = wo_lo + (e - eh * e_w);
                 const uint32_t box = boxes[pix0 + static_cast<long long>(ho) * g.Wo + wo];
                 const int bh0 = ho * g.sh - g.ph, bw0 = wo * g.sw - g.pw;
                 const int rmin = bh0 + static_cast<int8_t>(box & 0xff), rmax = bh0 + static_cast<int8_t>((box >> 8) & 0xff);
@@ -366,11 +397,7 @@ __global__ void __launch_bounds__(1024) value_kernel(const Geometry g, const T* 
         }
     }
     __syncthreads();
-    // The list is used when codes are valid, coordinates fit 16 bits and it did not overflow.
-    // (Boxes are relative to the pixel's grid origin, so they also span the
-    // grid itself: they are exact only while that stays within int8.)
-    const bool listed = use_codes && R + max((g.kh - 1) * g.dh, (g.kw - 1) * g.dw) <= 127 && s_nlist <= kListCap &&
-                        g.Ho <= 65535 && g.Wo <= 65535;
+    const bool listed = boxes_exact && s_nlist <= kListCap && g.Ho <= 65535 && g.Wo <= 65535;
     const int nlist = s_nlist;
 
     // Scan mapping: each thread keeps one (group, point) and walks the listed
@@ -397,8 +424,7 @@ __global__ void __launch_bounds__(1024) value_kernel(const Geometry g, const T* 
     const uint16_t* code_n = codes + pix0 * GK + gk;
     const T* om_n = om + pix0 * g.P + sg * 3 * g.K;
 
-    // Pass 0 counts the samples of each (group, cell); pass 1 places their
-    // records (image pixel of p, m(1-lh), m lh, lw) in bin order.
+    // Pass 0 counts the samples of each (group, cell); pass 1 places their records in bin order.
     bool sorted = true;
     for (int pass = 0; pass < 2; ++pass) {
         if (pass == 1) {
@@ -433,25 +459,54 @@ __global__ void __launch_bounds__(1024) value_kernel(const Geometry g, const T* 
             sorted = s_total <= g.bcap;
             if (!sorted) break;
         }
-        if (scanner && tslot < k_cnt) {
+        if (scanner && listed) {
+            // Lean walk over the listed pixels: 32-bit math, constants hoisted.
+            const int Wo = g.Wo, sh = g.sh, sw = g.sw;
+            const int hbase = ah0 - (y0 - 1), wbase = aw0 - (x0 - 1);  // cell row/col relative to the tile's cells
+            const int binbase = sg * cells;
+            for (int e = tslot; e < nlist; e += spt) {
+                const uint32_t lv = s_list[e];
+                const int ho = static_cast<int>(lv >> 16), wo = static_cast<int>(lv & 0xffff);
+                const int pix = ho * Wo + wo;
+                const uint16_t cd = ld_stream_u16(code_n + static_cast<long long>(pix) * GK);
+                const int ch = ho * sh + hbase + static_cast<int8_t>(cd & 0xff);
+                const int cw = wo * sw + wbase + static_cast<int8_t>(cd >> 8);
+                if (cd == kCodeNone || static_cast<unsigned>(ch) > static_cast<unsigned>(bh) ||
+                    static_cast<unsigned>(cw) > static_cast<unsigned>(bw))
+                    continue;
+                const int bin = binbase + ch * cells_w + cw;
+                if (pass == 0) {
+                    atomicAdd(&cnt[bin], 1);
+                } else {
+                    const T* orow = om_n + static_cast<long long>(pix) * g.P;
+                    const Candidate c = candidate(g, orow, sk, ho, wo, s_ih, s_iw);
+                    const int slot = atomicAdd(&cur[bin], 1);
+                    const float mf = ld_stream_elem(orow + 2 * g.K + sk);
+                    if constexpr (COMPACT) {
+                        const T mt = static_cast<T>(mf);  // exact: mf came from a T
+                        rec_c[slot] = make_uint2(static_cast<uint32_t>(e) | (static_cast<uint32_t>(raw_bits(mt)) << 16),
+                                                 fix16(c.lh) | (fix16(c.lw) << 16));
+                    } else {
+                        const float b = mf * c.lh;
+                        rec_w[slot] = make_float4(__int_as_float(pix), mf - b, b, c.lw);
+                    }
+                }
+            }
+        } else if (scanner) {
+            // Without a list: every pixel whose anchor for this point lies within R.
             int ho = 0, wo = 0;
-            if (!listed) {
+            if (tslot < k_cnt) {
                 const int eh = tslot / k_w;
                 ho = kh_lo + eh;
                 wo = kw_lo + tslot - eh * k_w;
             }
             for (int e = tslot; e < k_cnt; e += spt) {
-                if (listed) {
-                    const uint32_t lv = s_list[e];
-                    ho = static_cast<int>(lv >> 16);
-                    wo = static_cast<int>(lv & 0xffff);
-                }
                 const long long pix = static_cast<long long>(ho) * g.Wo + wo;
                 int h0, w0;
                 bool any;
                 Candidate c;
                 if (use_codes) {
-                    const uint16_t cd = code_n[pix * GK];
+                    const uint16_t cd = ld_stream_u16(code_n + pix * GK);
                     any = cd != kCodeNone;
                     h0 = ho * g.sh + ah0 + static_cast<int8_t>(cd & 0xff);
                     w0 = wo * g.sw + aw0 + static_cast<int8_t>(cd >> 8);
@@ -467,26 +522,26 @@ __global__ void __launch_bounds__(1024) value_kernel(const Geometry g, const T* 
                     const int bin = sg * cells + ch * cells_w + cw;
                     if (pass == 0) {
                         atomicAdd(&cnt[bin], 1);
-                    } else {
+                    } else if constexpr (!COMPACT) {  // compact records need the list (direct path instead)
                         const T* orow = om_n + pix * g.P;
                         if (use_codes) c = candidate(g, orow, sk, ho, wo, s_ih, s_iw);
                         const int slot = atomicAdd(&cur[bin], 1);
-                        const float m = to_f32(orow[2 * g.K + sk]);
-                        const float b = m * c.lh;
-                        rec[slot] = make_float4(__int_as_float(static_cast<int>(pix)), m - b, b, c.lw);
+                        const float mf = ld_stream_elem(orow + 2 * g.K + sk);
+                        const float b = mf * c.lh;
+                        rec_w[slot] = make_float4(__int_as_float(static_cast<int>(pix)), mf - b, b, c.lw);
                     }
                 }
-                if (!listed) {  // next pixel of this slot
-                    wo += spt;
-                    while (wo > kw_hi) {
-                        wo -= k_w;
-                        ++ho;
-                    }
+                wo += spt;  // next pixel of this slot
+                while (wo > kw_hi) {
+                    wo -= k_w;
+                    ++ho;
                 }
             }
         }
         __syncthreads();
     }
+    // Compact records need the list; without it the tile takes the direct path.
+    if (COMPACT && !listed) sorted = false;
 
     // Pull: thread -> (input pixel q of the tile, group, slice).
     const int lanes_pp = g.G * g.nslice;
@@ -497,7 +552,7 @@ __global__ void __launch_bounds__(1024) value_kernel(const Geometry g, const T* 
     const int grp = rr / g.nslice;
     const int sl = rr - grp * g.nslice;
     const int ch_off = grp * g.Cg + sl * (VEC * EPV);
-    const T* gy_img = gout + static_cast<long long>(n) * g.Ho * g.Wo * g.C + ch_off;
+    const T* gy_img = gout + pix0 * g.C + ch_off;
 
     float2 acc[PAIRS];
 #pragma unroll
@@ -511,24 +566,79 @@ __global__ void __launch_bounds__(1024) value_kernel(const Geometry g, const T* 
             for (int b = 0; b < 2; ++b) {
                 const int bin = grp * cells + (qy - a + 1) * cells_w + (qx - b + 1);
                 const int end = cur[bin];
-#pragma unroll 2
-                for (int j = end - cnt[bin]; j < end; ++j) {
-                    const float4 rcd = rec[j];
-                    const float wt = (a ? rcd.z : rcd.y) * (b ? rcd.w : 1.f - rcd.w);
-                    accumulate<T, VEC>(acc, gy_img + static_cast<long long>(__float_as_int(rcd.x)) * g.C, wt);
+                int j = end - cnt[bin];
+                // Two records per step, so two grad_out gathers are in flight.
+                for (; j + 1 < end; j += 2) {
+                    const T* src[2];
+                    float wt[2];
+#pragma unroll
+                    for (int u = 0; u < 2; ++u) {
+                        if constexpr (COMPACT) {
+                            const uint2 r = rec_c[j + u];
+                            const uint32_t lv = s_list[r.x & 0xffff];
+                            const float m = from_bits(static_cast<uint16_t>(r.x >> 16), T());
+                            const float hq = static_cast<float>(a ? (r.y & 0xffff) : 65536u - (r.y & 0xffff));
+                            const float wq = static_cast<float>(b ? (r.y >> 16) : 65536u - (r.y >> 16));
+                            wt[u] = m * (hq * wq) * 0x1p-32f;
+                            src[u] = gy_img + ((lv >> 16) * static_cast<long long>(g.Wo) + (lv & 0xffff)) * g.C;
+                        } else {
+                            const float4 r = rec_w[j + u];
+                            wt[u] = (a ? r.z : r.y) * (b ? r.w : 1.f - r.w);
+                            src[u] = gy_img + static_cast<long long>(__float_as_int(r.x)) * g.C;
+                        }
+                    }
+                    uint4 raw[2][VEC];
+#pragma unroll
+                    for (int u = 0; u < 2; ++u) {
+                        if constexpr (VEC == 2) {
+                            ld_keep32(src[u], raw[u][0], raw[u][1]);
+                        } else {
+                            raw[u][0] = ld_keep16(src[u]);
+                        }
+                    }
+#pragma unroll
+                    for (int u = 0; u < 2; ++u) {
+                        const float2 w2 = make_float2(wt[u], wt[u]);
+#pragma unroll
+                        for (int v = 0; v < VEC; ++v) {
+                            float2 f[EPV / 2];
+                            unpack(raw[u][v], f, T());
+#pragma unroll
+                            for (int i = 0; i < EPV / 2; ++i)
+                                acc[v * (EPV / 2) + i] = __ffma2_rn(w2, f[i], acc[v * (EPV / 2) + i]);
+                        }
+                    }
+                }
+                if (j < end) {
+                    const T* src;
+                    float wt;
+                    if constexpr (COMPACT) {
+                        const uint2 r = rec_c[j];
+                        const uint32_t lv = s_list[r.x & 0xffff];
+                        const float m = from_bits(static_cast<uint16_t>(r.x >> 16), T());
+                        const float hq = static_cast<float>(a ? (r.y & 0xffff) : 65536u - (r.y & 0xffff));
+                        const float wq = static_cast<float>(b ? (r.y >> 16) : 65536u - (r.y >> 16));
+                        wt = m * (hq * wq) * 0x1p-32f;
+                        src = gy_img + ((lv >> 16) * static_cast<long long>(g.Wo) + (lv & 0xffff)) * g.C;
+                    } else {
+                        const float4 r = rec_w[j];
+                        wt = (a ? r.z : r.y) * (b ? r.w : 1.f - r.w);
+                        src = gy_img + static_cast<long long>(__float_as_int(r.x)) * g.C;
+                    }
+                    accumulate<T, VEC>(acc, src, wt);
                 }
             }
         }
     } else {
-        // Overflow path: scan every candidate sample of this group directly.
+        // Direct path: scan every candidate sample of this group.
         const int uh_lo = max(0, ceil_div(y0 - R + g.ph - (g.kh - 1) * g.dh, g.sh));
         const int uh_hi = min(g.Ho - 1, floor_div(y0 + bh - 1 + R + g.ph, g.sh));
         const int uw_lo = max(0, ceil_div(x0 - R + g.pw - (g.kw - 1) * g.dw, g.sw));
         const int uw_hi = min(g.Wo - 1, floor_div(x0 + bw - 1 + R + g.pw, g.sw));
         const int u_w = max(0, uw_hi - uw_lo + 1);
-        const int u_cnt = u_w * max(0, uh_hi - uh_lo + 1);
+        const int u_cnt = R >= 0 ? u_w * max(0, uh_hi - uh_lo + 1) : 0;
         const int gy_abs = y0 + qy, gx_abs = x0 + qx;
-        const T* om_g = om + static_cast<long long>(n) * g.Ho * g.Wo * g.P + grp * 3 * g.K;
+        const T* om_g = om + pix0 * g.P + grp * 3 * g.K;
         for (int e = 0; e < u_cnt; ++e) {
             const int eh = e / u_w;
             const int ho = uh_lo + eh, wo = uw_lo + (e - eh * u_w);
@@ -603,7 +713,7 @@ template <typename T, int VEC>
 cudaError_t launch_value_typed(const Geometry& g, const void* om, const void* gout, void* gvalue, const int* reach,
                                const uint16_t* codes, const uint32_t* boxes, cudaStream_t stream) {
     const size_t smem = backward_value_smem_bytes(g);
-    auto kern = value_kernel<T, VEC>;
+    auto kern = value_kernel<T, VEC, sizeof(T) == 2>;
     cudaError_t e = allow_smem(kern, smem);
     if (e != cudaSuccess) return e;
     const long long blocks = static_cast<long long>(g.N) * g.btiles_h * g.btiles_w;
@@ -622,12 +732,12 @@ cudaError_t launch_value_vec(const Geometry& g, const void* om, const void* gout
 }  // namespace
 
 size_t backward_smem_bytes(const Geometry& g, int elem_bytes) {
-    return static_cast<size_t>(g.TH) * g.TW * g.P * (elem_bytes + 4);
+    return static_cast<size_t>(g.TH) * g.TW * g.P * elem_bytes * 2;
 }
 
 size_t backward_value_smem_bytes(const Geometry& g) {
     const size_t nbins = static_cast<size_t>(g.G) * (g.BH + 1) * (g.BW + 1);
-    return (2 * nbins * sizeof(int) + 15) / 16 * 16 + static_cast<size_t>(g.bcap) * 16;
+    return ((2 * nbins + kListCap) * sizeof(int) + 15) / 16 * 16 + static_cast<size_t>(g.bcap) * g.brec;
 }
 
 cudaError_t launch_backward_samples(const Geometry& g, int dtype, const void* value, const void* om, const void* gout,

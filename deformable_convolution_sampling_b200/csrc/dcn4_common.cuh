@@ -29,6 +29,7 @@ struct Geometry {
     // grad_value pass: input tiles of BH x BW pixels, bthreads threads per CTA,
     // room for bcap sample records in shared memory.
     int BH, BW, btiles_h, btiles_w, bthreads, bcap;
+    int brec;  // bytes per sample record: 8 (16-bit dtypes) or 16 (fp32)
 };
 
 template <typename T>
@@ -45,6 +46,15 @@ template <>
 struct Elem<__nv_bfloat16> {
     static constexpr int per16 = 8;
 };
+
+template <typename T>
+__device__ __forceinline__ T from_f32(float x);
+template <>
+__device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <>
+__device__ __forceinline__ __half from_f32<__half>(float x) { return __float2half_rn(x); }
+template <>
+__device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
 
 __device__ __forceinline__ float to_f32(float x) { return x; }
 __device__ __forceinline__ float to_f32(__half x) { return __half2float(x); }
@@ -110,6 +120,27 @@ __device__ __forceinline__ void ld_gather32(const void* p, uint4& lo, uint4& hi)
     asm volatile("ld.global.nc.v8.u32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
                  : "=r"(lo.x), "=r"(lo.y), "=r"(lo.z), "=r"(lo.w), "=r"(hi.x), "=r"(hi.y), "=r"(hi.z), "=r"(hi.w)
                  : "l"(p));
+}
+
+// 32-byte read-only gather that should stay in L1 (evicted last).
+__device__ __forceinline__ void ld_keep32(const void* p, uint4& lo, uint4& hi) {
+    asm volatile("ld.global.nc.L1::evict_last.v8.u32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                 : "=r"(lo.x), "=r"(lo.y), "=r"(lo.z), "=r"(lo.w), "=r"(hi.x), "=r"(hi.y), "=r"(hi.z), "=r"(hi.w)
+                 : "l"(p));
+}
+__device__ __forceinline__ uint4 ld_keep16(const void* p) {
+    uint4 r;
+    asm volatile("ld.global.nc.L1::evict_last.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "l"(p));
+    return r;
+}
+
+// 2-byte read that bypasses L1 (used once; keeps L1 for the gathers).
+__device__ __forceinline__ uint16_t ld_stream_u16(const void* p) {
+    unsigned short r;
+    asm volatile("ld.global.nc.L1::no_allocate.u16 %0, [%1];" : "=h"(r) : "l"(p));
+    return r;
 }
 
 // 32-byte store (sm_100 256-bit store).
