@@ -52,13 +52,49 @@ ELEM_BYTES = {"f32": 4, "f16": 2, "bf16": 2}
 # ---------------------------------------------------------------------------
 
 def byte_model(w: gen.Workload) -> dict:
-    """value + offset_mask + out (forward); + grad_out read, grad_value and
-    grad_offset_mask written (backward)."""
+    """Compulsory HBM bytes per call.  forward: value + offset_mask read, out
+    written.  backward: value + offset_mask + grad_out read, grad_value +
+    grad_offset_mask written.  Per backward kernel: the offset/mask stage reads
+    value, offset_mask, grad_out and writes grad_offset_mask; the value stage
+    reads offset_mask and grad_out and writes grad_value."""
     b = ELEM_BYTES[w.dtype]
     value = w.N * w.H * w.W * w.C * b
     om = w.N * w.Ho * w.Wo * w.P * b
     out = w.N * w.Ho * w.Wo * w.C * b
-    return {"fwd": value + om + out, "bwd": value + om + out + value + om}
+    return {"fwd": value + om + out, "bwd": value + om + out + value + om,
+            "bwd_offset_mask": value + om + out + om, "bwd_value": om + out + value}
+
+
+KERNELS = {"fwd": "forward_kernel", "bwd_offset_mask": "samples_kernel", "bwd_value": "value_kernel"}
+
+
+def kernel_sources_sha() -> str:
+    """sha256 over the CUDA sources: a DRAM-traffic capture is only reported
+    while the kernels are the ones it measured."""
+    import glob
+    import hashlib
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(ROOT, "deformable_convolution_sampling_b200", "csrc", "*.cu*"))):
+        with open(f, "rb") as fh:
+            h.update(os.path.basename(f).encode())
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def recorded_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch of `kernel` on `workload` from profiles/dram_traffic.txt,
+    or None when absent or captured from other kernel sources."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    try:
+        lines = open(path).read().splitlines()
+    except OSError:
+        return None
+    sha = kernel_sources_sha()
+    for line in lines:
+        parts = line.split()
+        if len(parts) >= 4 and not line.startswith("#") and parts[0] == kernel and parts[1] == workload:
+            return int(float(parts[2])) if parts[3] == sha else None
+    return None
 
 
 def measured_peaks() -> dict:
@@ -270,45 +306,52 @@ def run_native(args, w: gen.Workload) -> dict:
     def fwd():
         dcn.check(dcn.dcn4_forward(p, ptr["v"], ptr["om"], ptr["out"], sh))
 
-    def bwd():
-        dcn.check(dcn.dcn4_backward(p, ptr["v"], ptr["om"], ptr["gy"], ptr["gv"], ptr["gom"], ptr["ws"],
-                                    ws_bytes, sh))
+    def bwd_om():
+        dcn.check(dcn.dcn4_backward_offset_mask(p, ptr["v"], ptr["om"], ptr["gy"], ptr["gom"], ptr["ws"], ws_bytes, sh))
 
-    launches_per_step = 1 + (2 if w.dtype != "f32" else 1)  # forward; backward kernel (+ finalize)
+    def bwd_val():
+        dcn.check(dcn.dcn4_backward_value(p, ptr["om"], ptr["gy"], ptr["gv"], ptr["ws"], ws_bytes, sh))
+
+    def bwd():
+        bwd_om()
+        bwd_val()
+
+    stages = [("fwd", fwd), ("bwd_offset_mask", bwd_om), ("bwd_value", bwd_val)]
+    launches_per_step = len(stages)  # forward, grad_offset_mask kernel, grad_value kernel (+ a 4N-byte memset)
 
     for _ in range(args.warmup):
         flush.zero_()
-        fwd()
-        bwd()
+        for _, fn in stages:
+            fn()
     torch.cuda.synchronize(dev)
 
     sampler = ClockSampler(local if world > 1 else torch.cuda.current_device())
     sampler.start()
     time.sleep(0.3)
     K = args.steps
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(stages) + 1)] for _ in range(K)]
     barrier(dev)
     torch.cuda.synchronize(dev)
     t0 = time.time()
     for i in range(K):
         flush.zero_()
         ev[i][0].record(stream)
-        fwd()
-        ev[i][1].record(stream)
-        bwd()
-        ev[i][2].record(stream)
+        for j, (_, fn) in enumerate(stages):
+            fn()
+            ev[i][j + 1].record(stream)
     torch.cuda.synchronize(dev)
     barrier(dev)
     t1 = time.time()
     time.sleep(0.25)
     sampler.stop()
 
-    fwd_ms = [e[0].elapsed_time(e[1]) for e in ev]
-    bwd_ms = [e[1].elapsed_time(e[2]) for e in ev]
-    step_ms = statistics.mean(f + b for f, b in zip(fwd_ms, bwd_ms))
+    stage_us = {}
+    for j, (name, _) in enumerate(stages):
+        stage_us[name] = max_over_ranks(statistics.mean(e[j].elapsed_time(e[j + 1]) for e in ev) * 1e3, dev)
+    step_ms = statistics.mean(e[0].elapsed_time(e[-1]) for e in ev)
     step_ms_max = max_over_ranks(step_ms, dev)
-    fwd_us = max_over_ranks(statistics.mean(fwd_ms) * 1e3, dev)
-    bwd_us = max_over_ranks(statistics.mean(bwd_ms) * 1e3, dev)
+    fwd_us = stage_us["fwd"]
+    bwd_us = stage_us["bwd_offset_mask"] + stage_us["bwd_value"]
 
     # End to end through host buffers: pinned host -> device copies of the
     # inputs, forward + backward, device -> pinned host copies of the results.
@@ -350,14 +393,13 @@ def run_native(args, w: gen.Workload) -> dict:
     fwd_gbs = bm["fwd"] / (fwd_us * 1e-6) / 1e9
     bwd_gbs = bm["bwd"] / (bwd_us * 1e-6) / 1e9
     step_gbs = (bm["fwd"] + bm["bwd"]) / (step_ms_max * 1e-3) / 1e9
-    dominant = "bwd" if bwd_us >= fwd_us else "fwd"
-    dom_gbs = bwd_gbs if dominant == "bwd" else fwd_gbs
+    dominant = max(stage_us, key=stage_us.get)
+    dom_gbs = bm[dominant] / (stage_us[dominant] * 1e-6) / 1e9
     roofline = {
-        "bound": "hbm", "kernel": "dcn4_backward (accumulator memset + gradient kernel + fp32->dtype finalize)"
-        if dominant == "bwd" else "dcn4_forward kernel",
+        "bound": "hbm", "kernel": KERNELS[dominant], "launch_us": round(stage_us[dominant], 2),
         "achieved": round(dom_gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
         "frac": round(dom_gbs / peaks["hbm_gbs"], 4), "peak_source": peaks["source"],
-        "traffic": args.traffic_bytes,
+        "traffic": recorded_traffic(KERNELS[dominant], w.name),
         "algorithmic_bytes": bm[dominant],
     }
 
@@ -371,6 +413,7 @@ def run_native(args, w: gen.Workload) -> dict:
                    "global_batch": w.N * world, "parallelism": f"replicas x{world} (batch per GPU {w.N})",
                    "l2": "flushed between timed steps (256 MiB write outside the events)"},
         "fwd_us": round(fwd_us, 2), "bwd_us": round(bwd_us, 2),
+        "kernel_us": {KERNELS[k]: round(v, 2) for k, v in stage_us.items()},
         "fwd_gbs": round(fwd_gbs, 1), "bwd_gbs": round(bwd_gbs, 1), "step_gbs": round(step_gbs, 1),
         "fwd_frac_hbm": round(fwd_gbs / peaks["hbm_gbs"], 4), "bwd_frac_hbm": round(bwd_gbs / peaks["hbm_gbs"], 4),
         "fwd_frac_8tbs": round(fwd_gbs / 8000.0, 4), "bwd_frac_8tbs": round(bwd_gbs / 8000.0, 4),
@@ -404,8 +447,6 @@ def main(argv=None):
                     help="target seconds of oracle work for the cpu_baseline sample")
     ap.add_argument("--reference-images", type=int, default=1,
                     help="images of the batch the reference arm runs per step")
-    ap.add_argument("--traffic-bytes", type=float, default=None,
-                    help="DRAM bytes per launch of the dominant kernel from an ncu capture (null if unknown)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

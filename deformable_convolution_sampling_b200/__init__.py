@@ -79,6 +79,8 @@ def _load() -> ctypes.CDLL:
         "dcn4_backward": ([P, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp], ctypes.c_int),
         "dcn4_status_string": ([ctypes.c_int], ctypes.c_char_p),
         "dcn4_last_error": ([], ctypes.c_char_p),
+        "dcn4_backward_offset_mask": ([P, vp, vp, vp, vp, vp, ctypes.c_size_t, vp], ctypes.c_int),
+        "dcn4_backward_value": ([P, vp, vp, vp, vp, ctypes.c_size_t, vp], ctypes.c_int),
         "dcn4_backward_noalloc": ([P, vp, vp, vp, vp, vp, vp], ctypes.c_int),
         "dcn4_backward_noalloc_capacity": ([], ctypes.c_size_t),
         "dcn4_noalloc_last_error": ([], ctypes.c_char_p),
@@ -132,6 +134,18 @@ def dcn4_backward(p: dcn4_params, value, offset_mask, grad_out, grad_value, grad
                   workspace, workspace_bytes: int, stream=None) -> int:
     return lib.dcn4_backward(ctypes.byref(p), value, offset_mask, grad_out, grad_value,
                              grad_offset_mask, workspace, workspace_bytes, stream)
+
+
+def dcn4_backward_offset_mask(p: dcn4_params, value, offset_mask, grad_out, grad_offset_mask, workspace,
+                              workspace_bytes: int, stream=None) -> int:
+    return lib.dcn4_backward_offset_mask(ctypes.byref(p), value, offset_mask, grad_out, grad_offset_mask,
+                                         workspace, workspace_bytes, stream)
+
+
+def dcn4_backward_value(p: dcn4_params, offset_mask, grad_out, grad_value, workspace, workspace_bytes: int,
+                        stream=None) -> int:
+    return lib.dcn4_backward_value(ctypes.byref(p), offset_mask, grad_out, grad_value, workspace,
+                                   workspace_bytes, stream)
 
 
 def dcn4_backward_noalloc(p: dcn4_params, value, offset_mask, grad_out, grad_value, grad_offset_mask,

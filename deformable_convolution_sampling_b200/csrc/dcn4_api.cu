@@ -227,16 +227,15 @@ size_t dcn4_backward_workspace_size(const dcn4_params* p) {
     return reach_bytes(g) + box_bytes(g) + static_cast<size_t>(g.total_pix) * g.G * g.K * sizeof(uint16_t);
 }
 
-int dcn4_backward(const dcn4_params* p, const void* value, const void* offset_mask, const void* grad_out,
-                  void* grad_value, void* grad_offset_mask, void* workspace, size_t workspace_bytes, void* stream) {
+int dcn4_backward_offset_mask(const dcn4_params* p, const void* value, const void* offset_mask, const void* grad_out,
+                              void* grad_offset_mask, void* workspace, size_t workspace_bytes, void* stream) {
     dcn4::Geometry g;
-    const int st = make_geometry(p, true, aligned32(value) && aligned32(grad_out) && aligned32(grad_value), &g);
+    const int st = make_geometry(p, true, aligned32(value) && aligned32(grad_out), &g);
     if (st != DCN4_OK) return st;
     if (g.total_pix == 0) return DCN4_OK;
-    if (!value || !offset_mask || !grad_out || !grad_value || !grad_offset_mask)
-        return fail(DCN4_ERR_NULL, "value, offset_mask, grad_out, grad_value and grad_offset_mask must be non-NULL");
-    if (!aligned16(value) || !aligned16(offset_mask) || !aligned16(grad_out) || !aligned16(grad_value) ||
-        !aligned16(grad_offset_mask))
+    if (!value || !offset_mask || !grad_out || !grad_offset_mask)
+        return fail(DCN4_ERR_NULL, "value, offset_mask, grad_out and grad_offset_mask must be non-NULL");
+    if (!aligned16(value) || !aligned16(offset_mask) || !aligned16(grad_out) || !aligned16(grad_offset_mask))
         return fail(DCN4_ERR_MISALIGNED, "tensor pointers must be 16-byte aligned");
     const size_t need = dcn4_backward_workspace_size(p);
     if (!workspace || workspace_bytes < need)
@@ -250,9 +249,46 @@ int dcn4_backward(const dcn4_params* p, const void* value, const void* offset_ma
     if (e != cudaSuccess) return fail(DCN4_ERR_LAUNCH, "reach reset: %s", cudaGetErrorString(e));
     e = dcn4::launch_backward_samples(g, p->dtype, value, offset_mask, grad_out, grad_offset_mask, reach, codes, boxes, s);
     if (e != cudaSuccess) return fail(DCN4_ERR_LAUNCH, "grad_offset_mask launch: %s", cudaGetErrorString(e));
-    e = dcn4::launch_backward_value(g, p->dtype, offset_mask, grad_out, grad_value, reach, codes, boxes, s);
+    return DCN4_OK;
+}
+
+int dcn4_backward_value(const dcn4_params* p, const void* offset_mask, const void* grad_out, void* grad_value,
+                        const void* workspace, size_t workspace_bytes, void* stream) {
+    dcn4::Geometry g;
+    const int st = make_geometry(p, true, aligned32(grad_out) && aligned32(grad_value), &g);
+    if (st != DCN4_OK) return st;
+    if (g.total_pix == 0) return DCN4_OK;
+    if (!offset_mask || !grad_out || !grad_value)
+        return fail(DCN4_ERR_NULL, "offset_mask, grad_out and grad_value must be non-NULL");
+    if (!aligned16(offset_mask) || !aligned16(grad_out) || !aligned16(grad_value))
+        return fail(DCN4_ERR_MISALIGNED, "tensor pointers must be 16-byte aligned");
+    const size_t need = dcn4_backward_workspace_size(p);
+    if (!workspace || workspace_bytes < need)
+        return fail(DCN4_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, workspace_bytes);
+    if (!aligned16(workspace)) return fail(DCN4_ERR_MISALIGNED, "workspace must be 16-byte aligned");
+    const int* reach = static_cast<const int*>(workspace);
+    const uint32_t* boxes = reinterpret_cast<const uint32_t*>(static_cast<const char*>(workspace) + reach_bytes(g));
+    const uint16_t* codes =
+        reinterpret_cast<const uint16_t*>(static_cast<const char*>(workspace) + reach_bytes(g) + box_bytes(g));
+    const cudaError_t e = dcn4::launch_backward_value(g, p->dtype, offset_mask, grad_out, grad_value, reach, codes,
+                                                      boxes, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return fail(DCN4_ERR_LAUNCH, "grad_value launch: %s", cudaGetErrorString(e));
     return DCN4_OK;
+}
+
+int dcn4_backward(const dcn4_params* p, const void* value, const void* offset_mask, const void* grad_out,
+                  void* grad_value, void* grad_offset_mask, void* workspace, size_t workspace_bytes, void* stream) {
+    // Check everything the second stage needs before launching the first.
+    dcn4::Geometry g;
+    const int st = make_geometry(p, true, false, &g);
+    if (st != DCN4_OK) return st;
+    if (g.total_pix == 0) return DCN4_OK;
+    if (!grad_value) return fail(DCN4_ERR_NULL, "grad_value must be non-NULL");
+    if (!aligned16(grad_value)) return fail(DCN4_ERR_MISALIGNED, "tensor pointers must be 16-byte aligned");
+    const int a = dcn4_backward_offset_mask(p, value, offset_mask, grad_out, grad_offset_mask, workspace,
+                                            workspace_bytes, stream);
+    if (a != DCN4_OK) return a;
+    return dcn4_backward_value(p, offset_mask, grad_out, grad_value, workspace, workspace_bytes, stream);
 }
 
 const char* dcn4_status_string(int status) {

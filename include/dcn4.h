@@ -178,6 +178,22 @@ size_t dcn4_backward_noalloc_capacity(void);
  * this host thread ("" if none; launch errors are in dcn4_last_error()). */
 const char* dcn4_noalloc_last_error(void);
 
+/* The two stages of dcn4_backward, callable on their own (same arguments,
+ * layouts and errors as dcn4_backward):
+ *   dcn4_backward_offset_mask writes grad_offset_mask and fills `workspace`
+ *     (the per-image reach, per-pixel cell boxes and per-sample cell codes);
+ *     launches a memset of one word per image and one kernel.
+ *   dcn4_backward_value writes grad_value from offset_mask, grad_out and a
+ *     workspace filled by dcn4_backward_offset_mask for the same offset_mask
+ *     (and the same params), ordered before it; one kernel.
+ * dcn4_backward(...) is dcn4_backward_offset_mask(...) then
+ * dcn4_backward_value(...) on the same stream. */
+int dcn4_backward_offset_mask(const dcn4_params* p, const void* value, const void* offset_mask,
+                              const void* grad_out, void* grad_offset_mask, void* workspace,
+                              size_t workspace_bytes, void* stream);
+int dcn4_backward_value(const dcn4_params* p, const void* offset_mask, const void* grad_out,
+                        void* grad_value, const void* workspace, size_t workspace_bytes, void* stream);
+
 /* Name of a dcn4_status. */
 const char* dcn4_status_string(int status);
 

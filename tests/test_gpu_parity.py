@@ -274,3 +274,28 @@ def test_images_with_different_reach():
     inp["offset_mask"][2, ..., : w.G * 27] = zero.reshape(w.Ho, w.Wo, w.G * 27)
     _check_forward(w, inp)
     _check_backward(w, inp)
+
+
+def test_backward_stages_equal_backward():
+    """dcn4_backward_offset_mask then dcn4_backward_value == dcn4_backward."""
+    import torch
+    import deformable_convolution_sampling_b200 as dcn
+    w = gen.WORKLOADS["train_bf16_k8"]
+    inp = gen.make_inputs(gen.custom(**{**w.__dict__, "N": 4, "name": "stages"}))
+    p = dcn.make_params(dtype=w.dtype, **{**w.geometry(), "N": 4})
+    v, om, gy = (to_device(inp[k], w.dtype) for k in ("value", "offset_mask", "grad_out"))
+    gv_ref, gom_ref = dcn.backward(p, v, om, gy)
+    nbytes = dcn.dcn4_backward_workspace_size(p)
+    ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    gv, gom = torch.empty_like(gv_ref), torch.empty_like(gom_ref)
+    s = torch.cuda.current_stream().cuda_stream
+    dcn.check(dcn.dcn4_backward_offset_mask(p, v.data_ptr(), om.data_ptr(), gy.data_ptr(), gom.data_ptr(),
+                                            ws.data_ptr(), nbytes, s))
+    dcn.check(dcn.dcn4_backward_value(p, om.data_ptr(), gy.data_ptr(), gv.data_ptr(), ws.data_ptr(), nbytes, s))
+    torch.cuda.synchronize()
+    assert torch.equal(gom.view(torch.int16), gom_ref.view(torch.int16))
+    # grad_value sums the samples of a cell in the order the shared-memory sort placed
+    # them, which may differ between calls: one bfloat16 ulp apart at most, plus fp32
+    # summation noise where the sum cancels to almost nothing.
+    a, b = to_f64(gv), to_f64(gv_ref)
+    assert np.all(np.abs(a - b) <= 2.0 ** -7 * np.maximum(np.abs(a), np.abs(b)) + 2.0 ** -20 * np.abs(b).max())
