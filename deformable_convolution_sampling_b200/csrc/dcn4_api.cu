@@ -162,8 +162,8 @@ int make_geometry(const dcn4_params* p, bool backward, bool wide, dcn4::Geometry
 }
 
 // Backward workspace: one reach word per image, one cell bounding box (4
-// bytes) per output pixel (each rounded up to 256 bytes), then one 2-byte cell
-// code per sample.
+// bytes) per output pixel (each rounded up to 256 bytes), then one entry per
+// sample (2 bytes for fp32, 8 for 16-bit dtypes).
 size_t reach_bytes(const dcn4::Geometry& g) { return (static_cast<size_t>(g.N) * sizeof(int) + 255) / 256 * 256; }
 size_t box_bytes(const dcn4::Geometry& g) { return (static_cast<size_t>(g.total_pix) * 4 + 255) / 256 * 256; }
 
@@ -224,7 +224,8 @@ int dcn4_forward(const dcn4_params* p, const void* value, const void* offset_mas
 size_t dcn4_backward_workspace_size(const dcn4_params* p) {
     dcn4::Geometry g;
     if (make_geometry(p, true, true, &g) != DCN4_OK) return 0;
-    return reach_bytes(g) + box_bytes(g) + static_cast<size_t>(g.total_pix) * g.G * g.K * sizeof(uint16_t);
+    const size_t entry = p->dtype == DCN4_F32 ? 2 : 8;  // cell code, or code + mask + fixed-point lh, lw
+    return reach_bytes(g) + box_bytes(g) + static_cast<size_t>(g.total_pix) * g.G * g.K * entry;
 }
 
 int dcn4_backward_offset_mask(const dcn4_params* p, const void* value, const void* offset_mask, const void* grad_out,
@@ -243,7 +244,7 @@ int dcn4_backward_offset_mask(const dcn4_params* p, const void* value, const voi
     if (!aligned16(workspace)) return fail(DCN4_ERR_MISALIGNED, "workspace must be 16-byte aligned");
     int* reach = static_cast<int*>(workspace);
     uint32_t* boxes = reinterpret_cast<uint32_t*>(static_cast<char*>(workspace) + reach_bytes(g));
-    uint16_t* codes = reinterpret_cast<uint16_t*>(static_cast<char*>(workspace) + reach_bytes(g) + box_bytes(g));
+    void* codes = static_cast<char*>(workspace) + reach_bytes(g) + box_bytes(g);
     const cudaStream_t s = static_cast<cudaStream_t>(stream);
     cudaError_t e = cudaMemsetAsync(reach, 0xff, static_cast<size_t>(g.N) * sizeof(int), s);  // reach = -1
     if (e != cudaSuccess) return fail(DCN4_ERR_LAUNCH, "reach reset: %s", cudaGetErrorString(e));
@@ -268,8 +269,7 @@ int dcn4_backward_value(const dcn4_params* p, const void* offset_mask, const voi
     if (!aligned16(workspace)) return fail(DCN4_ERR_MISALIGNED, "workspace must be 16-byte aligned");
     const int* reach = static_cast<const int*>(workspace);
     const uint32_t* boxes = reinterpret_cast<const uint32_t*>(static_cast<const char*>(workspace) + reach_bytes(g));
-    const uint16_t* codes =
-        reinterpret_cast<const uint16_t*>(static_cast<const char*>(workspace) + reach_bytes(g) + box_bytes(g));
+    const void* codes = static_cast<const char*>(workspace) + reach_bytes(g) + box_bytes(g);
     const cudaError_t e = dcn4::launch_backward_value(g, p->dtype, offset_mask, grad_out, grad_value, reach, codes,
                                                       boxes, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return fail(DCN4_ERR_LAUNCH, "grad_value launch: %s", cudaGetErrorString(e));

@@ -33,6 +33,8 @@
 //   shared memory (a pathological concentration of samples), the CTA falls
 //   back to having each thread scan the candidate samples directly: slower,
 //   same result.
+#include <type_traits>
+
 #include "dcn4_common.cuh"
 
 namespace dcn4 {
@@ -93,6 +95,23 @@ __device__ __forceinline__ uint16_t cell_code(bool any, int dh, int dw) {
     return static_cast<uint16_t>((dh & 0xff) | ((dw & 0xff) << 8));
 }
 
+// Per-sample entry the sample pass leaves for the grad_value pass.  fp32 I/O:
+// the 2-byte cell code (the grad_value pass re-forms the exact weights from
+// the offsets).  16-bit I/O: an 8-byte record — cell code, the mask's own 16
+// bits, lh and lw as 16-bit fixed point — so the grad_value pass never reads
+// the offsets.
+template <typename T>
+using SampleEntry = std::conditional_t<sizeof(T) == 2, uint64_t, uint16_t>;
+
+__device__ __forceinline__ uint32_t fix16(float f) { return min(65535u, static_cast<uint32_t>(f * 65536.f + 0.5f)); }
+
+template <typename T>
+__device__ __forceinline__ uint16_t raw_bits(T x) {
+    uint16_t b;
+    memcpy(&b, &x, 2);
+    return b;
+}
+
 // Grid cell (ih, iw) of sampling point k (columns outer, rows inner, centre
 // skipped when remove_center is set).
 __device__ __forceinline__ void grid_cell_of(const Geometry& g, int k, int& ih, int& iw) {
@@ -112,7 +131,7 @@ template <typename T, int VEC, int KH, int KW, bool RC>
 __global__ void __launch_bounds__(256) samples_kernel(const Geometry g, const T* __restrict__ value,
                                                       const T* __restrict__ om, const T* __restrict__ gout,
                                                       T* __restrict__ gom, int* __restrict__ reach,
-                                                      uint16_t* __restrict__ codes, uint32_t* __restrict__ boxes) {
+                                                      void* __restrict__ codes, uint32_t* __restrict__ boxes) {
     extern __shared__ __align__(16) unsigned char smem[];
     __shared__ int s_reach;
     __shared__ int s_box[4 * 256];  // per tile pixel: min/max cell row, min/max cell column (relative)
@@ -159,7 +178,7 @@ __global__ void __launch_bounds__(256) samples_kernel(const Geometry g, const T*
     float2 gy[PAIRS];
     const long long pix = (static_cast<long long>(t.n) * g.Ho + ho) * g.Wo + wo;
     load_gy<T, VEC>(gy, gout + pix * g.C + ch_off);
-    uint16_t* code = codes + (pix * g.G + grp) * K;  // codes[N, Ho, Wo, G, K]
+    SampleEntry<T>* code = static_cast<SampleEntry<T>*>(codes) + (pix * g.G + grp) * K;  // [N, Ho, Wo, G, K]
     const bool writer = active && sl == 0;
     int my_reach = -1;
     int bmin_h = 127, bmax_h = -128, bmin_w = 127, bmax_w = -128;  // cells relative to (hb, wb)
@@ -206,7 +225,15 @@ __global__ void __launch_bounds__(256) samples_kernel(const Geometry g, const T*
                 bmin_w = min(bmin_w, cell.w0 - wb);
                 bmax_w = max(bmax_w, cell.w0 - wb);
             }
-            if (writer) code[kk] = cell_code(cell.any, cell.h0 - ah, cell.w0 - aw);
+            if (writer) {
+                const uint16_t cd = cell_code(cell.any, cell.h0 - ah, cell.w0 - aw);
+                if constexpr (sizeof(T) == 2) {
+                    code[kk] = static_cast<uint64_t>(cd) | (static_cast<uint64_t>(raw_bits(row[2 * K + kk])) << 16) |
+                               (static_cast<uint64_t>(fix16(cell.lh)) << 32) | (static_cast<uint64_t>(fix16(cell.lw)) << 48);
+                } else {
+                    code[kk] = cd;
+                }
+            }
         }
     }
 
@@ -305,14 +332,6 @@ __device__ __forceinline__ Candidate candidate(const Geometry& g, const T* om_ro
 // pixel index of p, m(1-lh), m lh, lw.  Compact (8 bytes, 16-bit I/O): index of
 // p in the CTA's candidate list, the mask's own 16 bits, and lh, lw as 16-bit
 // fixed point (error below 2^-17, far under the I/O rounding).
-__device__ __forceinline__ uint32_t fix16(float f) { return min(65535u, static_cast<uint32_t>(f * 65536.f + 0.5f)); }
-
-template <typename T>
-__device__ __forceinline__ uint16_t raw_bits(T x) {
-    uint16_t b;
-    memcpy(&b, &x, 2);
-    return b;
-}
 __device__ __forceinline__ float from_bits(uint16_t b, __half) {
     __half h;
     memcpy(&h, &b, 2);
@@ -324,7 +343,7 @@ template <typename T, int VEC, bool COMPACT>
 __global__ void __launch_bounds__(512, 2) value_kernel(const Geometry g, const T* __restrict__ om,
                                                        const T* __restrict__ gout, T* __restrict__ gvalue,
                                                        const int* __restrict__ reach,
-                                                       const uint16_t* __restrict__ codes,
+                                                       const void* __restrict__ codes,
                                                        const uint32_t* __restrict__ boxes) {
     extern __shared__ __align__(16) unsigned char smem[];
     __shared__ int s_warp[32];
@@ -421,7 +440,7 @@ __global__ void __launch_bounds__(512, 2) value_kernel(const Geometry g, const T
     }
     const int k_w = max(0, kw_hi - kw_lo + 1);
     const int k_cnt = listed ? nlist : k_w * max(0, kh_hi - kh_lo + 1);
-    const uint16_t* code_n = codes + pix0 * GK + gk;
+    const SampleEntry<T>* code_n = static_cast<const SampleEntry<T>*>(codes) + pix0 * GK + gk;
     const T* om_n = om + pix0 * g.P + sg * 3 * g.K;
 
     // Pass 0 counts the samples of each (group, cell); pass 1 places their records in bin order.
@@ -468,7 +487,13 @@ __global__ void __launch_bounds__(512, 2) value_kernel(const Geometry g, const T
                 const uint32_t lv = s_list[e];
                 const int ho = static_cast<int>(lv >> 16), wo = static_cast<int>(lv & 0xffff);
                 const int pix = ho * Wo + wo;
-                const uint16_t cd = ld_stream_u16(code_n + static_cast<long long>(pix) * GK);
+                SampleEntry<T> sr;
+                if constexpr (COMPACT) {
+                    sr = ld_stream_u64(code_n + static_cast<long long>(pix) * GK);
+                } else {
+                    sr = ld_stream_u16(code_n + static_cast<long long>(pix) * GK);
+                }
+                const uint16_t cd = static_cast<uint16_t>(sr & 0xffff);
                 const int ch = ho * sh + hbase + static_cast<int8_t>(cd & 0xff);
                 const int cw = wo * sw + wbase + static_cast<int8_t>(cd >> 8);
                 if (cd == kCodeNone || static_cast<unsigned>(ch) > static_cast<unsigned>(bh) ||
@@ -478,15 +503,15 @@ __global__ void __launch_bounds__(512, 2) value_kernel(const Geometry g, const T
                 if (pass == 0) {
                     atomicAdd(&cnt[bin], 1);
                 } else {
-                    const T* orow = om_n + static_cast<long long>(pix) * g.P;
-                    const Candidate c = candidate(g, orow, sk, ho, wo, s_ih, s_iw);
                     const int slot = atomicAdd(&cur[bin], 1);
-                    const float mf = ld_stream_elem(orow + 2 * g.K + sk);
                     if constexpr (COMPACT) {
-                        const T mt = static_cast<T>(mf);  // exact: mf came from a T
-                        rec_c[slot] = make_uint2(static_cast<uint32_t>(e) | (static_cast<uint32_t>(raw_bits(mt)) << 16),
-                                                 fix16(c.lh) | (fix16(c.lw) << 16));
+                        // the sample pass already left the mask bits and fixed-point lh, lw
+                        rec_c[slot] = make_uint2(static_cast<uint32_t>(e) | (static_cast<uint32_t>(sr) & 0xffff0000u),
+                                                 static_cast<uint32_t>(sr >> 32));
                     } else {
+                        const T* orow = om_n + static_cast<long long>(pix) * g.P;
+                        const Candidate c = candidate(g, orow, sk, ho, wo, s_ih, s_iw);
+                        const float mf = ld_stream_elem(orow + 2 * g.K + sk);
                         const float b = mf * c.lh;
                         rec_w[slot] = make_float4(__int_as_float(pix), mf - b, b, c.lw);
                     }
@@ -506,7 +531,12 @@ __global__ void __launch_bounds__(512, 2) value_kernel(const Geometry g, const T
                 bool any;
                 Candidate c;
                 if (use_codes) {
-                    const uint16_t cd = ld_stream_u16(code_n + pix * GK);
+                    uint16_t cd;
+                    if constexpr (COMPACT) {
+                        cd = static_cast<uint16_t>(ld_stream_u64(code_n + pix * GK) & 0xffff);
+                    } else {
+                        cd = ld_stream_u16(code_n + pix * GK);
+                    }
                     any = cd != kCodeNone;
                     h0 = ho * g.sh + ah0 + static_cast<int8_t>(cd & 0xff);
                     w0 = wo * g.sw + aw0 + static_cast<int8_t>(cd >> 8);
@@ -678,7 +708,7 @@ cudaError_t allow_smem(Kern kern, size_t smem) {
 
 template <typename T, int VEC, int KH, int KW, bool RC>
 cudaError_t launch_samples_typed(const Geometry& g, const void* value, const void* om, const void* gout, void* gom,
-                                 int* reach, uint16_t* codes, uint32_t* boxes, cudaStream_t stream) {
+                                 int* reach, void* codes, uint32_t* boxes, cudaStream_t stream) {
     const size_t smem = backward_smem_bytes(g, sizeof(T));
     auto kern = samples_kernel<T, VEC, KH, KW, RC>;
     cudaError_t e = allow_smem(kern, smem);
@@ -693,7 +723,7 @@ cudaError_t launch_samples_typed(const Geometry& g, const void* value, const voi
 
 template <typename T, int VEC>
 cudaError_t launch_samples_grid(const Geometry& g, const void* value, const void* om, const void* gout, void* gom,
-                                int* reach, uint16_t* codes, uint32_t* boxes, cudaStream_t stream) {
+                                int* reach, void* codes, uint32_t* boxes, cudaStream_t stream) {
     if (g.kh == 3 && g.kw == 3) {
         return g.remove_center
                    ? launch_samples_typed<T, VEC, 3, 3, true>(g, value, om, gout, gom, reach, codes, boxes, stream)
@@ -704,14 +734,14 @@ cudaError_t launch_samples_grid(const Geometry& g, const void* value, const void
 
 template <typename T>
 cudaError_t launch_samples_vec(const Geometry& g, const void* value, const void* om, const void* gout, void* gom,
-                               int* reach, uint16_t* codes, uint32_t* boxes, cudaStream_t stream) {
+                               int* reach, void* codes, uint32_t* boxes, cudaStream_t stream) {
     return g.vec == 2 ? launch_samples_grid<T, 2>(g, value, om, gout, gom, reach, codes, boxes, stream)
                       : launch_samples_grid<T, 1>(g, value, om, gout, gom, reach, codes, boxes, stream);
 }
 
 template <typename T, int VEC>
 cudaError_t launch_value_typed(const Geometry& g, const void* om, const void* gout, void* gvalue, const int* reach,
-                               const uint16_t* codes, const uint32_t* boxes, cudaStream_t stream) {
+                               const void* codes, const uint32_t* boxes, cudaStream_t stream) {
     const size_t smem = backward_value_smem_bytes(g);
     auto kern = value_kernel<T, VEC, sizeof(T) == 2>;
     cudaError_t e = allow_smem(kern, smem);
@@ -724,7 +754,7 @@ cudaError_t launch_value_typed(const Geometry& g, const void* om, const void* go
 
 template <typename T>
 cudaError_t launch_value_vec(const Geometry& g, const void* om, const void* gout, void* gvalue, const int* reach,
-                             const uint16_t* codes, const uint32_t* boxes, cudaStream_t stream) {
+                             const void* codes, const uint32_t* boxes, cudaStream_t stream) {
     return g.vec == 2 ? launch_value_typed<T, 2>(g, om, gout, gvalue, reach, codes, boxes, stream)
                       : launch_value_typed<T, 1>(g, om, gout, gvalue, reach, codes, boxes, stream);
 }
@@ -741,7 +771,7 @@ size_t backward_value_smem_bytes(const Geometry& g) {
 }
 
 cudaError_t launch_backward_samples(const Geometry& g, int dtype, const void* value, const void* om, const void* gout,
-                                    void* gom, int* reach, uint16_t* codes, uint32_t* boxes, cudaStream_t stream) {
+                                    void* gom, int* reach, void* codes, uint32_t* boxes, cudaStream_t stream) {
     switch (dtype) {
         case 0: return launch_samples_vec<float>(g, value, om, gout, gom, reach, codes, boxes, stream);
         case 1: return launch_samples_vec<__half>(g, value, om, gout, gom, reach, codes, boxes, stream);
@@ -751,7 +781,7 @@ cudaError_t launch_backward_samples(const Geometry& g, int dtype, const void* va
 }
 
 cudaError_t launch_backward_value(const Geometry& g, int dtype, const void* om, const void* gout, void* gvalue,
-                                  const int* reach, const uint16_t* codes, const uint32_t* boxes,
+                                  const int* reach, const void* codes, const uint32_t* boxes,
                                   cudaStream_t stream) {
     switch (dtype) {
         case 0: return launch_value_vec<float>(g, om, gout, gvalue, reach, codes, boxes, stream);

@@ -143,6 +143,12 @@ __device__ __forceinline__ uint16_t ld_stream_u16(const void* p) {
     return r;
 }
 
+__device__ __forceinline__ uint64_t ld_stream_u64(const void* p) {
+    unsigned long long r;
+    asm volatile("ld.global.nc.L1::no_allocate.u64 %0, [%1];" : "=l"(r) : "l"(p));
+    return r;
+}
+
 // 32-byte store (sm_100 256-bit store).
 __device__ __forceinline__ void st_global32(void* p, const uint4& lo, const uint4& hi) {
     asm volatile("st.global.v8.u32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(lo.x), "r"(lo.y),
@@ -267,14 +273,15 @@ namespace dcn4 {
 cudaError_t launch_forward(const Geometry& g, int dtype, const void* value, const void* om, void* out,
                            cudaStream_t stream);
 // grad_offset_mask and the per-image reach (int[N], pre-filled with -1).
-// Also writes one 2-byte cell code per sample, codes[N, Ho, Wo, G, K], and the
+// Also writes one entry per sample, codes[N, Ho, Wo, G, K] (a 2-byte cell code for
+// fp32, an 8-byte record for 16-bit dtypes), and the
 // bounding box of each output pixel's cells, boxes[N, Ho, Wo].
 cudaError_t launch_backward_samples(const Geometry& g, int dtype, const void* value, const void* om,
-                                    const void* gout, void* gom, int* reach, uint16_t* codes, uint32_t* boxes,
+                                    const void* gout, void* gom, int* reach, void* codes, uint32_t* boxes,
                                     cudaStream_t stream);
 // grad_value from the reach, cell codes and boxes written by launch_backward_samples.
 cudaError_t launch_backward_value(const Geometry& g, int dtype, const void* om, const void* gout, void* gvalue,
-                                  const int* reach, const uint16_t* codes, const uint32_t* boxes,
+                                  const int* reach, const void* codes, const uint32_t* boxes,
                                   cudaStream_t stream);
 // Dynamic shared memory bytes of one CTA.
 size_t forward_smem_bytes(const Geometry& g, int elem_bytes);

@@ -117,10 +117,11 @@ int dcn4_check_params(const dcn4_params* p);
 int dcn4_forward(const dcn4_params* p, const void* value, const void* offset_mask, void* out,
                  void* stream);
 
-/* Bytes of device workspace dcn4_backward needs, whatever the dtype:
- * one 32-bit word per image (N*4 rounded up to 256), one 32-bit cell box per
- * output pixel (N*Ho*Wo*4 rounded up to 256) and one 16-bit cell code per
- * sample (N*Ho*Wo*G*K*2); 0 if p is invalid. */
+/* Bytes of device workspace dcn4_backward needs: one 32-bit word per image
+ * (N*4 rounded up to 256), one 32-bit cell box per output pixel (N*Ho*Wo*4
+ * rounded up to 256) and one entry per sample, N*Ho*Wo*G*K of them: a 2-byte
+ * cell code for fp32, an 8-byte record (cell code, mask bits, fixed-point
+ * bilinear fractions) for fp16/bf16; 0 if p is invalid. */
 size_t dcn4_backward_workspace_size(const dcn4_params* p);
 
 /* Backward of the forward for upstream gradient grad_out:
