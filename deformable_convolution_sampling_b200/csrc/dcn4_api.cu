@@ -37,12 +37,15 @@ bool aligned32(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31u) ==
 constexpr int kTargetThreads = 256;
 constexpr size_t kSmemDefault = 48 * 1024;
 constexpr size_t kSmemMax = 227 * 1024;
-// grad_value pass: up to 1024 threads and 256 input pixels per CTA; sample
-// records get what is left of this shared-memory budget after the bins.
-constexpr int kValueThreads = 512;
-constexpr int kValuePixels = 128;
-constexpr size_t kValueSmem = 200 * 1024;
-constexpr int kValueListCap = 2048;  // candidate-pixel list entries (4 bytes each) per CTA
+// grad_value pass: 256 threads per CTA and two CTAs per SM, so each CTA's
+// bins, candidate list and sample records share this shared-memory budget.
+constexpr int kValueThreads = 256;
+constexpr size_t kValueSmem = 112 * 1024;
+constexpr int kValueMaxBH = 16;    // input rows per tile at most
+constexpr int kValueMaxGK = 512;   // groups x points at most
+// grad_offset_mask pass: shared memory at most for its offset_mask tiles plus
+// the staging of the records it files (beyond it the grad_value pass rescans).
+constexpr size_t kFileSmem = 96 * 1024;
 
 // Validates p and fills the kernel geometry.  Touches no GPU state.
 // wide: the gathered and stored tensors are 32-byte aligned, so a thread may
@@ -126,46 +129,96 @@ int make_geometry(const dcn4_params* p, bool backward, bool wide, dcn4::Geometry
     g->tiles_h = static_cast<int>(tiles_h);
     g->tiles_w = static_cast<int>(tiles_w);
 
-    // grad_value pass: BH x BW input pixels per CTA (all groups).
-    long long bpix = std::min<long long>(kValuePixels, kValueThreads / lanes_pp);
-    long long BW = 1;
-    while (BW * BW < bpix && BW * 2 <= bpix) BW *= 2;
-    while (BW > 1 && BW / 2 >= p->W) BW /= 2;
-    long long BH = std::max<long long>(1, bpix / BW);
-    if (BH > p->H) BH = p->H;
-    long long bthreads = (BH * BW * lanes_pp + 31) / 32 * 32;
+    // grad_value pass: tiles of BH x BW input pixels.  A strip of LW lanes
+    // (one per cell column, BW + 1 of them) covers the tile's width: LW = 32
+    // for images at least 16 wide (BW = 31), narrower strips otherwise.
     const long long GK = static_cast<long long>(p->G) * K;
-    if (GK > kValueThreads) return fail(DCN4_ERR_UNSUPPORTED, "G*K = %lld exceeds %d", GK, kValueThreads);
-    if (bthreads < GK) bthreads = (GK + 31) / 32 * 32;
-    const long long nbins = static_cast<long long>(p->G) * (BH + 1) * (BW + 1);
-    const long long bin_bytes = ((2 * nbins + kValueListCap) * 4 + 15) / 16 * 16;
+    if (GK > kValueMaxGK) return fail(DCN4_ERR_UNSUPPORTED, "G*K = %lld exceeds %d", GK, kValueMaxGK);
+    const int LW = p->W >= 16 ? 32 : p->W >= 8 ? 16 : 8;
+    const long long BW = std::min<long long>(p->W, LW - 1);
     const long long brec = eb == 2 ? 8 : 16;
-    if (bin_bytes + 1024 * brec > static_cast<long long>(kValueSmem))
-        return fail(DCN4_ERR_UNSUPPORTED, "too many groups for the grad_value tile");
-    // Records: room for 1.25x the expected number of samples per tile (K per
-    // cell for every output pixel per input pixel), within the budget; the
-    // rest of the shared memory stays L1 for the grad_out gathers.
-    const long long expect = nbins * K * std::max<long long>(1, (Ho * Wo + p->H * p->W - 1) / (p->H * p->W));
-    long long bcap = (static_cast<long long>(kValueSmem) - bin_bytes) / brec;
-    bcap = std::max<long long>(1024, std::min(bcap, expect + expect / 4 + 256));
+    // Samples per cell per group: K for each output pixel per input pixel.
+    const long long dens = K * std::max<long long>(1, (Ho * Wo + static_cast<long long>(p->H) * p->W - 1) /
+                                                          (static_cast<long long>(p->H) * p->W));
+    g->G = p->G;
+    g->K = K;
+    g->BW = static_cast<int>(BW);
+    g->brec = static_cast<int>(brec);
+    // Tallest tile (<= kValueMaxBH rows) whose records fit the budget with a
+    // margin over the expected count (records beyond it send the tile to the
+    // direct path).
+    long long BH = std::min<long long>(kValueMaxBH, p->H);
+    for (;; --BH) {
+        const long long expect = static_cast<long long>(p->G) * (BH + 1) * (BW + 1) * dens;
+        g->BH = static_cast<int>(BH);
+        g->bcap = static_cast<int>(std::min<long long>(expect + expect / 16 + 512, 1LL << 24));
+        if (dcn4::backward_value_smem_bytes(*g) <= kValueSmem || BH == 1) break;
+    }
+    if (dcn4::backward_value_smem_bytes(*g) > kValueSmem) {
+        g->bcap = 0;
+        const size_t fixed = dcn4::backward_value_smem_bytes(*g);
+        if (fixed + 1024 * brec > kValueSmem) return fail(DCN4_ERR_UNSUPPORTED, "too many groups for the grad_value tile");
+        g->bcap = static_cast<int>((kValueSmem - fixed) / brec);
+    }
+    // Segments: enough (group, slice, segment) strips for every strip slot of the CTA.
+    const long long slots = (kValueThreads / 32) * (32 / LW);
+    long long nseg = std::min<long long>(BH, std::max<long long>(1, (slots + lanes_pp - 1) / lanes_pp));
+    const long long BS = (BH + nseg - 1) / nseg;
+    nseg = (BH + BS - 1) / BS;
     const long long btiles_h = (p->H + BH - 1) / BH, btiles_w = (p->W + BW - 1) / BW;
     if (static_cast<long long>(p->N) * btiles_h * btiles_w > 0x7fffffffLL)
         return fail(DCN4_ERR_UNSUPPORTED, "grid too large");
-    g->BH = static_cast<int>(BH);
-    g->BW = static_cast<int>(BW);
     g->btiles_h = static_cast<int>(btiles_h);
     g->btiles_w = static_cast<int>(btiles_w);
-    g->bthreads = static_cast<int>(bthreads);
-    g->bcap = static_cast<int>(bcap);
-    g->brec = static_cast<int>(brec);
+    g->bthreads = kValueThreads;
+    g->LW = LW;
+    g->BS = static_cast<int>(BS);
+    g->nseg = static_cast<int>(nseg);
+    // Buckets for 16-bit dtypes, when a record can name its output pixel as
+    // (ho << 16) | wo and its bin in 16 bits.
+    const long long nbins = static_cast<long long>(p->G) * (BH + 1) * (BW + 1);
+    g->buckets = eb == 2 && Ho <= 65535 && Wo <= 65535 && nbins <= 65535;
+
+    g->bh_magic = 0xffffffffu / static_cast<uint32_t>(BH) + 1u;  // BH, BW >= 2 use __umulhi; 1 is special-cased
+    g->bw_magic = 0xffffffffu / static_cast<uint32_t>(BW) + 1u;
+    // ... and when the grad_offset_mask CTA can stage its records in shared memory.
+    if (g->buckets && (dcn4::backward_smem_bytes(*g, eb) > kFileSmem ||
+                       static_cast<long long>(K) * dcn4::samples_threads(*g) > (1 << 13)))
+        g->buckets = 0;
     return DCN4_OK;
 }
 
-// Backward workspace: one reach word per image, one cell bounding box (4
-// bytes) per output pixel (each rounded up to 256 bytes), then one entry per
-// sample (2 bytes for fp32, 8 for 16-bit dtypes).
-size_t reach_bytes(const dcn4::Geometry& g) { return (static_cast<size_t>(g.N) * sizeof(int) + 255) / 256 * 256; }
-size_t box_bytes(const dcn4::Geometry& g) { return (static_cast<size_t>(g.total_pix) * 4 + 255) / 256 * 256; }
+// Backward workspace, each part starting on a 256-byte boundary: one reach
+// word per image, one cell bounding box (4 bytes) per output pixel; then for
+// fp32 a 2-byte cell code per sample, for 16-bit dtypes (with buckets) one
+// record counter per grad_value tile and each tile's bucket of bcap 12-byte
+// records (4-byte output pixel + 8-byte bin, mask bits and fractions).
+size_t round256(size_t b) { return (b + 255) / 256 * 256; }
+size_t reach_bytes(const dcn4::Geometry& g) { return round256(static_cast<size_t>(g.N) * sizeof(int)); }
+size_t box_bytes(const dcn4::Geometry& g) { return round256(static_cast<size_t>(g.total_pix) * 4); }
+size_t num_samples(const dcn4::Geometry& g) { return static_cast<size_t>(g.total_pix) * g.G * g.K; }
+size_t num_value_tiles(const dcn4::Geometry& g) { return static_cast<size_t>(g.N) * g.btiles_h * g.btiles_w; }
+size_t count_bytes(const dcn4::Geometry& g) { return round256(num_value_tiles(g) * sizeof(int)); }
+size_t workspace_bytes(const dcn4::Geometry& g, int dtype) {
+    size_t b = reach_bytes(g) + box_bytes(g);
+    if (dtype == DCN4_F32) return b + round256(num_samples(g) * 2);
+    if (!g.buckets) return b;
+    const size_t recs = num_value_tiles(g) * static_cast<size_t>(g.bcap);
+    return b + count_bytes(g) + round256(recs * 4) + recs * 8;
+}
+dcn4::SampleArrays sample_arrays(const dcn4::Geometry& g, int dtype, const void* workspace) {
+    char* base = static_cast<char*>(const_cast<void*>(workspace)) + reach_bytes(g) + box_bytes(g);
+    dcn4::SampleArrays sa = {};
+    if (dtype == DCN4_F32) {
+        sa.code = reinterpret_cast<uint16_t*>(base);
+    } else if (g.buckets) {
+        const size_t recs = num_value_tiles(g) * static_cast<size_t>(g.bcap);
+        sa.tile_count = reinterpret_cast<int*>(base);
+        sa.bucket_pix = reinterpret_cast<uint32_t*>(base + count_bytes(g));
+        sa.bucket_rec = reinterpret_cast<uint64_t*>(base + count_bytes(g) + round256(recs * 4));
+    }
+    return sa;
+}
 
 }  // namespace
 
@@ -224,8 +277,7 @@ int dcn4_forward(const dcn4_params* p, const void* value, const void* offset_mas
 size_t dcn4_backward_workspace_size(const dcn4_params* p) {
     dcn4::Geometry g;
     if (make_geometry(p, true, true, &g) != DCN4_OK) return 0;
-    const size_t entry = p->dtype == DCN4_F32 ? 2 : 8;  // cell code, or code + mask + fixed-point lh, lw
-    return reach_bytes(g) + box_bytes(g) + static_cast<size_t>(g.total_pix) * g.G * g.K * entry;
+    return workspace_bytes(g, p->dtype);
 }
 
 int dcn4_backward_offset_mask(const dcn4_params* p, const void* value, const void* offset_mask, const void* grad_out,
@@ -244,12 +296,17 @@ int dcn4_backward_offset_mask(const dcn4_params* p, const void* value, const voi
     if (!aligned16(workspace)) return fail(DCN4_ERR_MISALIGNED, "workspace must be 16-byte aligned");
     int* reach = static_cast<int*>(workspace);
     uint32_t* boxes = reinterpret_cast<uint32_t*>(static_cast<char*>(workspace) + reach_bytes(g));
-    void* codes = static_cast<char*>(workspace) + reach_bytes(g) + box_bytes(g);
+    const dcn4::SampleArrays sa = sample_arrays(g, p->dtype, workspace);
     const cudaStream_t s = static_cast<cudaStream_t>(stream);
     cudaError_t e = cudaMemsetAsync(reach, 0xff, static_cast<size_t>(g.N) * sizeof(int), s);  // reach = -1
     if (e != cudaSuccess) return fail(DCN4_ERR_LAUNCH, "reach reset: %s", cudaGetErrorString(e));
-    e = dcn4::launch_backward_samples(g, p->dtype, value, offset_mask, grad_out, grad_offset_mask, reach, codes, boxes, s);
+    if (g.buckets) {
+        e = cudaMemsetAsync(sa.tile_count, 0, num_value_tiles(g) * sizeof(int), s);
+        if (e != cudaSuccess) return fail(DCN4_ERR_LAUNCH, "bucket reset: %s", cudaGetErrorString(e));
+    }
+    e = dcn4::launch_backward_samples(g, p->dtype, value, offset_mask, grad_out, grad_offset_mask, reach, sa, boxes, s);
     if (e != cudaSuccess) return fail(DCN4_ERR_LAUNCH, "grad_offset_mask launch: %s", cudaGetErrorString(e));
+
     return DCN4_OK;
 }
 
@@ -269,8 +326,8 @@ int dcn4_backward_value(const dcn4_params* p, const void* offset_mask, const voi
     if (!aligned16(workspace)) return fail(DCN4_ERR_MISALIGNED, "workspace must be 16-byte aligned");
     const int* reach = static_cast<const int*>(workspace);
     const uint32_t* boxes = reinterpret_cast<const uint32_t*>(static_cast<const char*>(workspace) + reach_bytes(g));
-    const void* codes = static_cast<const char*>(workspace) + reach_bytes(g) + box_bytes(g);
-    const cudaError_t e = dcn4::launch_backward_value(g, p->dtype, offset_mask, grad_out, grad_value, reach, codes,
+    const dcn4::SampleArrays sa = sample_arrays(g, p->dtype, workspace);
+    const cudaError_t e = dcn4::launch_backward_value(g, p->dtype, offset_mask, grad_out, grad_value, reach, sa,
                                                       boxes, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return fail(DCN4_ERR_LAUNCH, "grad_value launch: %s", cudaGetErrorString(e));
     return DCN4_OK;

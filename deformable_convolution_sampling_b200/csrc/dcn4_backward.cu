@@ -18,18 +18,19 @@
 //   (padding tail = 0) are assembled in shared memory and stored once.  It
 //   also records, per image, the reach R: the largest distance (per
 //   coordinate, in pixels) between a grid anchor and a corner of a cell that
-//   touches the image; and, per sample, a 2-byte code of its cell relative to
-//   its anchor.
+//   touches the image; per output pixel, the bounding box of its samples'
+//   cells; and, per sample, a 2-byte code of its cell relative to its anchor
+//   (for 16-bit dtypes also the mask bits and fixed-point lh, lw).
 //
 // value_kernel (input tiles).  grad_value is pulled, not scattered: a CTA owns
 //   a BH x BW tile of input pixels (all groups) and writes each of their
 //   grad_value elements exactly once.  The samples that can touch the tile come
-//   from output pixels whose anchors lie within R of it; the CTA reads those
-//   samples' cell codes, re-forms the locations of the ones whose cell touches
-//   the tile (the same fp32 fma as the forward, so the same cells), and
-//   counting-sorts them by (group, cell) in
-//   shared memory, then each thread sums m * w_ab * gy over the samples of the
-//   four cells its pixel is a corner of.  Should the sorted samples not fit in
+//   from output pixels whose anchors lie within R of it and whose cell box
+//   meets the tile; the CTA reads those samples' cell codes and counting-sorts
+//   the ones whose cell touches the tile by (group, cell) in shared memory.
+//   Then lanes own cell columns and walk cell rows: each sample is read once
+//   and added to its cell's four corners, and a shuffle joins the corners a
+//   pixel shares with the next column.  Should the sorted samples not fit in
 //   shared memory (a pathological concentration of samples), the CTA falls
 //   back to having each thread scan the candidate samples directly: slower,
 //   same result.
@@ -95,13 +96,12 @@ __device__ __forceinline__ uint16_t cell_code(bool any, int dh, int dw) {
     return static_cast<uint16_t>((dh & 0xff) | ((dw & 0xff) << 8));
 }
 
-// Per-sample entry the sample pass leaves for the grad_value pass.  fp32 I/O:
-// the 2-byte cell code (the grad_value pass re-forms the exact weights from
-// the offsets).  16-bit I/O: an 8-byte record — cell code, the mask's own 16
-// bits, lh and lw as 16-bit fixed point — so the grad_value pass never reads
-// the offsets.
-template <typename T>
-using SampleEntry = std::conditional_t<sizeof(T) == 2, uint64_t, uint16_t>;
+// Per-sample entries the sample pass leaves for the grad_value pass.  fp32
+// I/O: the 2-byte cell code only (the grad_value pass re-forms the exact
+// weights from the offsets).  16-bit I/O: also the mask's own 16 bits and lh,
+// lw as 16-bit fixed point, so the grad_value pass never reads the offsets.
+// The three live in separate arrays: the scan that filters candidates reads
+// only the codes.
 
 __device__ __forceinline__ uint32_t fix16(float f) { return min(65535u, static_cast<uint32_t>(f * 65536.f + 0.5f)); }
 
@@ -125,16 +125,58 @@ __device__ __forceinline__ void grid_cell_of(const Geometry& g, int k, int& ih, 
 }
 
 // ---------------------------------------------------------------------------
+// Filing (16-bit dtypes, when g.buckets): the grad_offset_mask CTA files each
+// sample under every grad_value tile whose cells hold it -- the tile holding
+// the cell's top-left pixel (h0, w0) (tile row 0 for h0 = -1, likewise for
+// columns), and the next tile down / right as well when the cell straddles
+// that boundary.  Records are staged in shared memory with their rank among
+// the CTA's records for the same tile; after the samples the CTA takes one
+// range per tile from the tile's global counter and writes its records there
+// (records of one tile keep no particular order).  Tiles are named by their
+// place in a kFileWin x kFileWin window of tiles around the CTA's anchors; a
+// record for a tile outside the window, or beyond the staging room, marks the
+// tile kBucketOverflow instead, and that tile rescans the offsets.
+// ---------------------------------------------------------------------------
+constexpr int kFileWin = 8;
+
+// Staging of one (sample, thread): the record for the cell's own tile (bin
+// included) and a meta word: window slot of that tile (6 bits), the record's
+// rank there and the ranks of its copies for the tile below, right and
+// below-right (13 bits each), a flag per copy (bits 58-60), and bit 61 when
+// the own-tile record exists.  A copy's bin follows from the cell's: a cell
+// on the bottom border (cell row BH) is cell row 0 below, one on the right
+// border (cell column BW) is cell column 0 to the right.
+struct FileStage {
+    uint64_t* rec;   // [K][threads]
+    uint64_t* meta;  // [K][threads]
+    int wy0, wx0;    // window origin (tile row, tile column)
+};
+constexpr int kRankBits = 13;  // ranks < K * threads <= 2^13 (checked on the host)
+
+__device__ __forceinline__ int window_slot(const FileStage& fs, int ty, int tx) {
+    const int dy = ty - fs.wy0, dx = tx - fs.wx0;
+    return (static_cast<unsigned>(dy) < static_cast<unsigned>(kFileWin) &&
+            static_cast<unsigned>(dx) < static_cast<unsigned>(kFileWin))
+               ? dy * kFileWin + dx
+               : -1;
+}
+
+__device__ __forceinline__ int tile_index(const Geometry& g, int n, int ty, int tx) {
+    return (n * g.btiles_h + ty) * g.btiles_w + tx;
+}
+
+// ---------------------------------------------------------------------------
 // grad_offset_mask + reach
 // ---------------------------------------------------------------------------
 template <typename T, int VEC, int KH, int KW, bool RC>
-__global__ void __launch_bounds__(256) samples_kernel(const Geometry g, const T* __restrict__ value,
+__global__ void __launch_bounds__(256, 3) samples_kernel(const Geometry g, const T* __restrict__ value,
                                                       const T* __restrict__ om, const T* __restrict__ gout,
                                                       T* __restrict__ gom, int* __restrict__ reach,
-                                                      void* __restrict__ codes, uint32_t* __restrict__ boxes) {
+                                                      const SampleArrays sa, uint32_t* __restrict__ boxes) {
     extern __shared__ __align__(16) unsigned char smem[];
     __shared__ int s_reach;
     __shared__ int s_box[4 * 256];  // per tile pixel: min/max cell row, min/max cell column (relative)
+    __shared__ int s_fcnt[kFileWin * kFileWin], s_fbase[kFileWin * kFileWin];
     constexpr int EPV = Elem<T>::per16;
     constexpr int PAIRS = VEC * EPV / 2;
     const int tile_elems = g.TH * g.TW * g.P;
@@ -142,6 +184,24 @@ __global__ void __launch_bounds__(256) samples_kernel(const Geometry g, const T*
     T* gom_s = reinterpret_cast<T*>(smem + tile_elems * sizeof(T));  // P % 8 == 0 keeps this 16-byte aligned
 
     const Tile t = tile_of_block(g);
+    const int K = KH > 0 ? KH * KW - (RC ? 1 : 0) : g.K;
+    const int kh = KH > 0 ? KH : g.kh;
+    const int kw = KW > 0 ? KW : g.kw;
+    const bool rc = KH > 0 ? RC : g.remove_center != 0;
+    const bool filing = sizeof(T) == 2 && g.buckets != 0;
+    FileStage fs;
+    if (filing) {
+        // staging after the two offset_mask tiles
+        unsigned char* st = smem + 2 * static_cast<size_t>(tile_elems) * sizeof(T);
+        fs.rec = reinterpret_cast<uint64_t*>(st);
+        fs.meta = fs.rec + K * blockDim.x;
+        // window of tiles centred on the anchors of this CTA's grid
+        const int amid_h = t.ho0 * g.sh - g.ph + ((t.th - 1) * g.sh + (kh - 1) * g.dh) / 2;
+        const int amid_w = t.wo0 * g.sw - g.pw + ((t.tw - 1) * g.sw + (kw - 1) * g.dw) / 2;
+        fs.wy0 = max(0, max(0, amid_h) / g.BH - kFileWin / 2);
+        fs.wx0 = max(0, max(0, amid_w) / g.BW - kFileWin / 2);
+        for (int i = threadIdx.x; i < kFileWin * kFileWin; i += blockDim.x) s_fcnt[i] = 0;
+    }
     stage_tile_rows(om_s, om, g, t);
     for (int i = threadIdx.x; i < tile_elems; i += blockDim.x) gom_s[i] = static_cast<T>(0.f);
     for (int i = threadIdx.x; i < g.TH * g.TW; i += blockDim.x) {
@@ -164,12 +224,7 @@ __global__ void __launch_bounds__(256) samples_kernel(const Geometry g, const T*
     const int grp = r / g.nslice;
     const int sl = r - grp * g.nslice;
     const int ho = t.ho0 + (active ? py : 0), wo = t.wo0 + (active ? px : 0);
-    const int lrow = (active ? lp : 0) * g.P + grp * 3 * (KH > 0 ? KH * KW - (RC ? 1 : 0) : g.K);
-
-    const int K = KH > 0 ? KH * KW - (RC ? 1 : 0) : g.K;
-    const int kh = KH > 0 ? KH : g.kh;
-    const int kw = KW > 0 ? KW : g.kw;
-    const bool rc = KH > 0 ? RC : g.remove_center != 0;
+    const int lrow = (active ? lp : 0) * g.P + grp * 3 * K;
     const T* row = om_s + lrow;
     const int ch_off = grp * g.Cg + sl * (VEC * EPV);
     const T* img = value + static_cast<long long>(t.n) * g.H * g.W * g.C + ch_off;
@@ -178,7 +233,7 @@ __global__ void __launch_bounds__(256) samples_kernel(const Geometry g, const T*
     float2 gy[PAIRS];
     const long long pix = (static_cast<long long>(t.n) * g.Ho + ho) * g.Wo + wo;
     load_gy<T, VEC>(gy, gout + pix * g.C + ch_off);
-    SampleEntry<T>* code = static_cast<SampleEntry<T>*>(codes) + (pix * g.G + grp) * K;  // [N, Ho, Wo, G, K]
+    const long long s0 = (pix * g.G + grp) * K;  // first entry of this (pixel, group): [N, Ho, Wo, G, K]
     const bool writer = active && sl == 0;
     int my_reach = -1;
     int bmin_h = 127, bmax_h = -128, bmin_w = 127, bmax_w = -128;  // cells relative to (hb, wb)
@@ -225,14 +280,53 @@ __global__ void __launch_bounds__(256) samples_kernel(const Geometry g, const T*
                 bmin_w = min(bmin_w, cell.w0 - wb);
                 bmax_w = max(bmax_w, cell.w0 - wb);
             }
-            if (writer) {
-                const uint16_t cd = cell_code(cell.any, cell.h0 - ah, cell.w0 - aw);
-                if constexpr (sizeof(T) == 2) {
-                    code[kk] = static_cast<uint64_t>(cd) | (static_cast<uint64_t>(raw_bits(row[2 * K + kk])) << 16) |
-                               (static_cast<uint64_t>(fix16(cell.lh)) << 32) | (static_cast<uint64_t>(fix16(cell.lw)) << 48);
-                } else {
-                    code[kk] = cd;
+            if constexpr (sizeof(T) == 2) {
+                if (filing) {
+                    const bool has = writer && cell.any;
+                    const int h0 = cell.h0, w0 = cell.w0;
+                    const int ta = h0 < 0 ? 0 : g.BH == 1 ? h0 : static_cast<int>(__umulhi(static_cast<uint32_t>(h0), g.bh_magic));
+                    const int ua = w0 < 0 ? 0 : g.BW == 1 ? w0 : static_cast<int>(__umulhi(static_cast<uint32_t>(w0), g.bw_magic));
+                    const int cy = h0 + 1 - ta * g.BH, cx = w0 + 1 - ua * g.BW;
+                    const int gbase = grp * (g.BH + 1) * (g.BW + 1);
+                    const uint64_t rec = (static_cast<uint64_t>(raw_bits(row[2 * K + kk])) << 16) |
+                                         (static_cast<uint64_t>(fix16(cell.lh)) << 32) |
+                                         (static_cast<uint64_t>(fix16(cell.lw)) << 48);
+                    const int dl0 = has ? window_slot(fs, ta, ua) : -1;
+                    if (has && dl0 < 0) atomicOr(sa.tile_count + tile_index(g, t.n, ta, ua), kBucketOverflow);
+                    // rank among the CTA's records for the tile: one shared atomic per distinct tile in the warp
+                    const unsigned okm = __ballot_sync(0xffffffffu, dl0 >= 0);
+                    uint64_t meta = 0;
+                    if (dl0 >= 0) {
+                        const int lane = threadIdx.x & 31;
+                        const unsigned peers = __match_any_sync(okm, dl0);
+                        const int leader = __ffs(peers) - 1;
+                        int base = 0;
+                        if (lane == leader) base = atomicAdd(s_fcnt + dl0, __popc(peers));
+                        base = __shfl_sync(peers, base, leader);
+                        const int rank = base + __popc(peers & ((1u << lane) - 1));
+                        meta = static_cast<uint64_t>(dl0) | (static_cast<uint64_t>(rank) << 6) | (1ull << 61);
+                        // copies for the next tiles when the cell straddles a border
+                        const bool dup_r = h0 >= 0 && h0 + 1 < g.H && h0 + 1 == (ta + 1) * g.BH;
+                        const bool dup_c = w0 >= 0 && w0 + 1 < g.W && w0 + 1 == (ua + 1) * g.BW;
+#pragma unroll
+                        for (int d = 1; d < 4; ++d) {
+                            if (!((d == 1 && dup_r) || (d == 2 && dup_c) || (d == 3 && dup_r && dup_c))) continue;
+                            const int ty = ta + (d & 1), tx = ua + (d >> 1);
+                            const int dl = window_slot(fs, ty, tx);
+                            if (dl < 0) {
+                                atomicOr(sa.tile_count + tile_index(g, t.n, ty, tx), kBucketOverflow);
+                                continue;
+                            }
+                            const int r = atomicAdd(s_fcnt + dl, 1);
+                            meta |= (static_cast<uint64_t>(r) << (6 + kRankBits * d)) | (1ull << (57 + d));
+                        }
+                    }
+                    const int at = kk * blockDim.x + threadIdx.x;
+                    fs.meta[at] = meta;
+                    fs.rec[at] = rec | static_cast<uint64_t>(gbase + cy * (g.BW + 1) + cx);
                 }
+            } else {
+                if (writer) sa.code[s0 + kk] = cell_code(cell.any, cell.h0 - ah, cell.w0 - aw);
             }
         }
     }
@@ -246,6 +340,44 @@ __global__ void __launch_bounds__(256) samples_kernel(const Geometry g, const T*
         atomicMax(&s_box[4 * lp + 3], min(127, bmax_w));
     }
     __syncthreads();
+    if (filing) {
+        // One range per window tile from its global counter, then the staged records.
+        for (int i = threadIdx.x; i < kFileWin * kFileWin; i += blockDim.x) {
+            s_fbase[i] = 0;
+            if (s_fcnt[i] > 0)
+                s_fbase[i] = atomicAdd(sa.tile_count + tile_index(g, t.n, fs.wy0 + i / kFileWin, fs.wx0 + i % kFileWin),
+                                       s_fcnt[i]);
+        }
+        __syncthreads();
+        const uint32_t pixv = (static_cast<uint32_t>(ho) << 16) | static_cast<uint32_t>(wo);
+        auto put = [&](int dl, int rank, uint64_t rec) {
+            const int slot = s_fbase[dl] + rank;
+            if (static_cast<unsigned>(slot) >= static_cast<unsigned>(g.bcap)) return;  // the tile rescans
+            const long long at = static_cast<long long>(tile_index(g, t.n, fs.wy0 + dl / kFileWin, fs.wx0 + dl % kFileWin)) *
+                                     g.bcap + slot;
+            sa.bucket_pix[at] = pixv;
+            sa.bucket_rec[at] = rec;
+        };
+        const int rmask = (1 << kRankBits) - 1;
+        for (int kk = 0; kk < K; ++kk) {
+            const int at = kk * blockDim.x + threadIdx.x;
+            const uint64_t meta = fs.meta[at];
+            if (!((meta >> 61) & 1)) continue;
+            const uint64_t rec = fs.rec[at];
+            const int dl0 = static_cast<int>(meta & 63);
+            put(dl0, static_cast<int>(meta >> 6) & rmask, rec);
+            const uint64_t body = rec & ~0xffffull;
+            const int bin = static_cast<int>(rec & 0xffff);
+            if ((meta >> 58) & 1)  // below: cell row 0 there
+                put(dl0 + kFileWin, static_cast<int>(meta >> (6 + kRankBits)) & rmask,
+                    body | static_cast<uint64_t>(bin - g.BH * (g.BW + 1)));
+            if ((meta >> 59) & 1)  // right: cell column 0 there
+                put(dl0 + 1, static_cast<int>(meta >> (6 + 2 * kRankBits)) & rmask, body | static_cast<uint64_t>(bin - g.BW));
+            if ((meta >> 60) & 1)  // below-right
+                put(dl0 + kFileWin + 1, static_cast<int>(meta >> (6 + 3 * kRankBits)) & rmask,
+                    body | static_cast<uint64_t>(bin - g.BH * (g.BW + 1) - g.BW));
+        }
+    }
     if (threadIdx.x == 0 && s_reach >= 0) atomicMax(reach + t.n, s_reach);
     for (int i = threadIdx.x; i < t.th * g.TW; i += blockDim.x) {
         const int r2 = i / g.TW, c2 = i - r2 * g.TW;
@@ -328,9 +460,10 @@ __device__ __forceinline__ Candidate candidate(const Geometry& g, const T* om_ro
     return c;
 }
 
-// Sample records of the grad_value sort.  Wide (16 bytes, fp32 I/O): image
-// pixel index of p, m(1-lh), m lh, lw.  Compact (8 bytes, 16-bit I/O): index of
-// p in the CTA's candidate list, the mask's own 16 bits, and lh, lw as 16-bit
+// Sample records of the grad_value sort.  Wide (16 bytes, fp32 I/O): grad_out
+// offset of the sample's output pixel p, m(1-lh), m lh, lw.  Compact (8 bytes,
+// 16-bit I/O): p relative to the tile's reference output pixel (ho_ref - 64,
+// wo_ref - 64) as 7 + 7 bits, the mask's own 16 bits, and lh, lw as 16-bit
 // fixed point (error below 2^-17, far under the I/O rounding).
 __device__ __forceinline__ float from_bits(uint16_t b, __half) {
     __half h;
@@ -339,16 +472,170 @@ __device__ __forceinline__ float from_bits(uint16_t b, __half) {
 }
 __device__ __forceinline__ float from_bits(uint16_t b, __nv_bfloat16) { return __uint_as_float(static_cast<uint32_t>(b) << 16); }
 
+// Where a record's grad_out slice is: compact records add their 7-bit row and
+// column to `ref` (row stride `row`, column stride `col`, in elements); wide
+// records carry the offset from `ref` themselves.
+template <typename T>
+struct GySource {
+    const T* ref;
+    int row, col;
+};
+
+// Adds U consecutive sorted records (from index j) of one cell to the partial
+// sums of its four corners: t0/t1 = top-left/top-right, b0/b1 = bottom-left/
+// bottom-right.  All U grad_out gathers are issued before any is used.
+template <typename T, int VEC, bool COMPACT, int U>
+__device__ __forceinline__ void pull_records(const unsigned char* rec_base, const GySource<T>& gs, int j, float2* t0,
+                                             float2* t1, float2* b0, float2* b1) {
+    constexpr int EPV = Elem<T>::per16;
+    const T* src[U];
+    float w[U][4];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+        if constexpr (COMPACT) {
+            const uint2 r = reinterpret_cast<const uint2*>(rec_base)[j + u];
+            // m * (hq * wq) * 2^-32 with hq, wq the 16-bit fixed-point weights
+            const float ms = from_bits(static_cast<uint16_t>(r.x >> 16), T()) * 0x1p-32f;
+            const float hq1 = static_cast<float>(r.y & 0xffff), hq0 = 65536.f - hq1;
+            const float wq1 = static_cast<float>(r.y >> 16), wq0 = 65536.f - wq1;
+            w[u][0] = ms * (hq0 * wq0);
+            w[u][1] = ms * (hq0 * wq1);
+            w[u][2] = ms * (hq1 * wq0);
+            w[u][3] = ms * (hq1 * wq1);
+            src[u] = gs.ref + static_cast<int>(r.x & 127) * gs.row + static_cast<int>((r.x >> 7) & 127) * gs.col;
+        } else {
+            const float4 r = reinterpret_cast<const float4*>(rec_base)[j + u];
+            const float lw0 = 1.f - r.w;
+            w[u][0] = r.y * lw0;
+            w[u][1] = r.y * r.w;
+            w[u][2] = r.z * lw0;
+            w[u][3] = r.z * r.w;
+            src[u] = gs.ref + __float_as_int(r.x);
+        }
+    }
+    uint4 raw[U][VEC];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+        if constexpr (VEC == 2) {
+            ld_keep32(src[u], raw[u][0], raw[u][1]);
+        } else {
+            raw[u][0] = ld_keep16(src[u]);
+        }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+        const float2 w00 = make_float2(w[u][0], w[u][0]), w01 = make_float2(w[u][1], w[u][1]);
+        const float2 w10 = make_float2(w[u][2], w[u][2]), w11 = make_float2(w[u][3], w[u][3]);
+#pragma unroll
+        for (int v = 0; v < VEC; ++v) {
+            float2 f[EPV / 2];
+            unpack(raw[u][v], f, T());
+#pragma unroll
+            for (int i = 0; i < EPV / 2; ++i) {
+                const int k = v * (EPV / 2) + i;
+                t0[k] = __ffma2_rn(w00, f[i], t0[k]);
+                t1[k] = __ffma2_rn(w01, f[i], t1[k]);
+                b0[k] = __ffma2_rn(w10, f[i], b0[k]);
+                b1[k] = __ffma2_rn(w11, f[i], b1[k]);
+            }
+        }
+    }
+}
+
+// All records [j, end) of one cell, two at a time.
 template <typename T, int VEC, bool COMPACT>
-__global__ void __launch_bounds__(512, 2) value_kernel(const Geometry g, const T* __restrict__ om,
+__device__ __forceinline__ void pull_cell(const unsigned char* rec_base, const GySource<T>& gs, int j, int end,
+                                          float2* t0, float2* t1, float2* b0, float2* b1) {
+    for (; j + 1 < end; j += 2) pull_records<T, VEC, COMPACT, 2>(rec_base, gs, j, t0, t1, b0, b1);
+    if (j < end) pull_records<T, VEC, COMPACT, 1>(rec_base, gs, j, t0, t1, b0, b1);
+}
+
+// A finished pixel row of a strip: lane cx holds the right corners (r) of
+// pixel cx and the left corners (l) of pixel cx - 1; the pixel's sum is its
+// own r plus the next lane's l.  Stores it (when `store`) and clears l, r.
+template <typename T, int VEC>
+__device__ __forceinline__ void finish_row(float2* l, float2* r, int LW, bool store, T* dst) {
+    constexpr int EPV = Elem<T>::per16;
+    constexpr int PAIRS = VEC * EPV / 2;
+    float2 out[PAIRS];
+#pragma unroll
+    for (int i = 0; i < PAIRS; ++i) {
+        out[i].x = r[i].x + __shfl_down_sync(0xffffffffu, l[i].x, 1, LW);
+        out[i].y = r[i].y + __shfl_down_sync(0xffffffffu, l[i].y, 1, LW);
+    }
+    if (store) {
+        if constexpr (VEC == 2) {
+            st_global32(dst, pack(out, T()), pack(out + EPV / 2, T()));
+        } else {
+            st_global(dst, pack(out, T()));
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < PAIRS; ++i) l[i] = r[i] = make_float2(0.f, 0.f);
+}
+
+// Exclusive scan of cnt[0, nbins) into cur, block-wide (thread-contiguous
+// chunks); every thread gets the total.  Starts and ends with a barrier.
+__device__ __forceinline__ int bins_exclusive_scan(const int* cnt, int* cur, int nbins, int* s_warp, int* s_total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+    __syncthreads();
+    const int per = (nbins + blockDim.x - 1) / blockDim.x;
+    const int b0 = threadIdx.x * per;
+    int local = 0;
+    for (int b = b0; b < min(nbins, b0 + per); ++b) local += cnt[b];
+    int incl = local;
+    for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+    }
+    if (lane == 31) s_warp[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        int v = lane < nwarps ? s_warp[lane] : 0;
+        for (int o = 1; o < 32; o <<= 1) {
+            const int u = __shfl_up_sync(0xffffffffu, v, o);
+            if (lane >= o) v += u;
+        }
+        if (lane < nwarps) s_warp[lane] = v;  // inclusive warp totals
+        if (lane == nwarps - 1) *s_total = v;
+    }
+    __syncthreads();
+    int run = incl - local + (warp > 0 ? s_warp[warp - 1] : 0);
+    for (int b = b0; b < min(nbins, b0 + per); ++b) {
+        cur[b] = run;
+        run += cnt[b];
+    }
+    __syncthreads();
+    return *s_total;
+}
+
+// Compact record of a sample of output pixel (ho, wo): false if the pixel is
+// outside the 128 x 128 window the record can name.
+__device__ __forceinline__ bool compact_source(int ho, int wo, int ho_ref, int wo_ref, uint32_t& id) {
+    const int dh = ho - ho_ref + 64, dw = wo - wo_ref + 64;
+    id = static_cast<uint32_t>(dh) | (static_cast<uint32_t>(dw) << 7);
+    return static_cast<unsigned>(dh) < 128u && static_cast<unsigned>(dw) < 128u;
+}
+
+__device__ __forceinline__ uint32_t ld_stream_u32(const void* p) {
+    unsigned r;
+    asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(r) : "l"(p));
+    return r;
+}
+
+// Records of the grad_value sort each thread keeps in flight.
+constexpr int kScanBatch = 8;
+
+template <typename T, int VEC, bool COMPACT>
+__global__ void __launch_bounds__(256, 2) value_kernel(const Geometry g, const T* __restrict__ om,
                                                        const T* __restrict__ gout, T* __restrict__ gvalue,
-                                                       const int* __restrict__ reach,
-                                                       const void* __restrict__ codes,
+                                                       const int* __restrict__ reach, const SampleArrays sa,
                                                        const uint32_t* __restrict__ boxes) {
     extern __shared__ __align__(16) unsigned char smem[];
     __shared__ int s_warp[32];
     __shared__ int s_total;
     __shared__ int s_nlist;
+    __shared__ int s_fail;
     constexpr int EPV = Elem<T>::per16;
     constexpr int PAIRS = VEC * EPV / 2;
 
@@ -359,314 +646,313 @@ __global__ void __launch_bounds__(512, 2) value_kernel(const Geometry g, const T
     const int by = tr / g.btiles_w;
     const int y0 = by * g.BH, x0 = (tr - by * g.btiles_w) * g.BW;
     const int bh = min(g.BH, g.H - y0), bw = min(g.BW, g.W - x0);
+    // Cell (bin) (cy, cx) of the tile has its top-left corner at pixel
+    // (y0 - 1 + cy, x0 - 1 + cx); cy in [0, bh], cx in [0, bw].
     const int cells_w = g.BW + 1;
     const int cells = (g.BH + 1) * cells_w;
     const int nbins = g.G * cells;
+    const int GK = g.G * g.K;
     int* cnt = reinterpret_cast<int*>(smem);
     int* cur = cnt + nbins;
     uint32_t* s_list = reinterpret_cast<uint32_t*>(cur + nbins);  // candidate pixels: (ho << 16) | wo
-    unsigned char* rec_base = smem + ((2 * nbins + kListCap) * sizeof(int) + 15) / 16 * 16;
+    int4* s_tab = reinterpret_cast<int4*>(smem + ((2 * nbins + kListCap) * sizeof(int) + 15) / 16 * 16);
+    unsigned char* rec_base = reinterpret_cast<unsigned char*>(s_tab + GK);
     float4* rec_w = reinterpret_cast<float4*>(rec_base);
     uint2* rec_c = reinterpret_cast<uint2*>(rec_base);
-
-    // Samples that can touch the tile come from output pixels whose anchor
-    // (for the sample's grid point) lies within R of the tile.
-    const int R = reach[n];
-    const int GK = g.G * g.K;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
-    const bool use_codes = R <= kCodeReach;  // else cells are re-formed from the offsets
-    const bool boxes_exact = use_codes && R + max((g.kh - 1) * g.dh, (g.kw - 1) * g.dw) <= 127;
-    int ho_lo = 0, ho_hi = -1, wo_lo = 0, wo_hi = -1;
-    if (R >= 0) {
-        ho_lo = max(0, ceil_div(y0 - R + g.ph - (g.kh - 1) * g.dh, g.sh));
-        ho_hi = min(g.Ho - 1, floor_div(y0 + bh - 1 + R + g.ph, g.sh));
-        wo_lo = max(0, ceil_div(x0 - R + g.pw - (g.kw - 1) * g.dw, g.sw));
-        wo_hi = min(g.Wo - 1, floor_div(x0 + bw - 1 + R + g.pw, g.sw));
-    }
-    const int e_w = max(0, wo_hi - wo_lo + 1);
-    const int e_cnt = e_w * max(0, ho_hi - ho_lo + 1);
+    const int nthr = blockDim.x;
     const long long pix0 = static_cast<long long>(n) * g.Ho * g.Wo;
+    // Compact records name their output pixel relative to this one (a sample
+    // of output pixel p touches the tile only if p's grid lies near it).
+    const int ho_ref = floor_div(y0 + g.ph, g.sh), wo_ref = floor_div(x0 + g.pw, g.sw);
+    // ... and the pull forms their grad_out offsets in 32 bits.
+    const bool compact_ok = !COMPACT || 128LL * (g.Wo + 1) * g.C < (1LL << 31);
 
-    if (threadIdx.x == 0) s_nlist = 0;
-    for (int i = threadIdx.x; i < nbins; i += blockDim.x) cnt[i] = 0;
-    __syncthreads();
-
-    // List the candidate pixels whose cell bounding box meets the tile's cells.
-    if (boxes_exact) {
-        for (int e0 = warp * 32; e0 < e_cnt; e0 += nwarps * 32) {
-            const int e = e0 + lane;
-            bool keep = false;
-            int ho = 0, wo = 0;
-            if (e < e_cnt) {
-                const int eh = e / e_w;
-                ho = ho_lo + eh;
-                wo = wo_lo + (e - eh * e_w);
-                const uint32_t box = boxes[pix0 + static_cast<long long>(ho) * g.Wo + wo];
-                const int bh0 = ho * g.sh - g.ph, bw0 = wo * g.sw - g.pw;
-                const int rmin = bh0 + static_cast<int8_t>(box & 0xff), rmax = bh0 + static_cast<int8_t>((box >> 8) & 0xff);
-                const int cmin = bw0 + static_cast<int8_t>((box >> 16) & 0xff), cmax = bw0 + static_cast<int8_t>(box >> 24);
-                keep = rmax >= y0 - 1 && rmin <= y0 + bh - 1 && cmax >= x0 - 1 && cmin <= x0 + bw - 1;
-            }
-            const unsigned ball = __ballot_sync(0xffffffffu, keep);
-            int base = 0;
-            if (lane == 0 && ball) base = atomicAdd(&s_nlist, __popc(ball));
-            base = __shfl_sync(0xffffffffu, base, 0);
-            const int pos = base + __popc(ball & ((1u << lane) - 1));
-            if (keep && pos < kListCap) s_list[pos] = (static_cast<uint32_t>(ho) << 16) | static_cast<uint32_t>(wo);
-        }
+    if (threadIdx.x == 0) {
+        s_nlist = 0;
+        s_fail = 0;
     }
-    __syncthreads();
-    const bool listed = boxes_exact && s_nlist <= kListCap && g.Ho <= 65535 && g.Wo <= 65535;
-    const int nlist = s_nlist;
+    for (int i = threadIdx.x; i < nbins; i += nthr) cnt[i] = 0;
 
-    // Scan mapping: each thread keeps one (group, point) and walks the listed
-    // pixels (or, without a list, every pixel whose anchor for that point is
-    // within R of the tile), a slot of pixels at a time.
-    const int spt = blockDim.x / GK;
-    const int tslot = threadIdx.x / GK;
-    const int gk = threadIdx.x - tslot * GK;
-    const bool scanner = tslot < spt;
-    const int sg = gk / g.K;
-    const int sk = gk - sg * g.K;
-    int s_ih, s_iw;
-    grid_cell_of(g, sk, s_ih, s_iw);
-    const int ah0 = s_ih * g.dh - g.ph, aw0 = s_iw * g.dw - g.pw;  // anchor = (ho*sh + ah0, wo*sw + aw0)
-    int kh_lo = 0, kh_hi = -1, kw_lo = 0, kw_hi = -1;
-    if (R >= 0) {
-        kh_lo = max(0, ceil_div(y0 - R - ah0, g.sh));
-        kh_hi = min(g.Ho - 1, floor_div(y0 + bh - 1 + R - ah0, g.sh));
-        kw_lo = max(0, ceil_div(x0 - R - aw0, g.sw));
-        kw_hi = min(g.Wo - 1, floor_div(x0 + bw - 1 + R - aw0, g.sw));
-    }
-    const int k_w = max(0, kw_hi - kw_lo + 1);
-    const int k_cnt = listed ? nlist : k_w * max(0, kh_hi - kh_lo + 1);
-    const SampleEntry<T>* code_n = static_cast<const SampleEntry<T>*>(codes) + pix0 * GK + gk;
-    const T* om_n = om + pix0 * g.P + sg * 3 * g.K;
-
-    // Pass 0 counts the samples of each (group, cell); pass 1 places their records in bin order.
-    bool sorted = true;
-    for (int pass = 0; pass < 2; ++pass) {
-        if (pass == 1) {
-            // Exclusive scan of the counts -> cursors (block-wide, thread-contiguous chunks).
-            const int per = (nbins + blockDim.x - 1) / blockDim.x;
-            const int b0 = threadIdx.x * per;
-            int local = 0;
-            for (int b = b0; b < min(nbins, b0 + per); ++b) local += cnt[b];
-            int incl = local;
-            for (int o = 1; o < 32; o <<= 1) {
-                const int v = __shfl_up_sync(0xffffffffu, incl, o);
-                if (lane >= o) incl += v;
+    bool sorted = false;
+    const int R = reach[n];
+    // The filing pass trusts the cell codes only up to kCodeReach.
+    const int nfiled = (COMPACT && g.buckets && compact_ok && R <= kCodeReach) ? sa.tile_count[blockIdx.x] : -1;
+    if (nfiled >= 0 && nfiled <= g.bcap) {
+        // The grad_offset_mask pass filed this tile's records in its bucket:
+        // count them per bin, scan, place them in bin order.
+        const uint64_t* brec = sa.bucket_rec + static_cast<long long>(blockIdx.x) * g.bcap;
+        const uint32_t* bpix = sa.bucket_pix + static_cast<long long>(blockIdx.x) * g.bcap;
+        __syncthreads();
+        for (int i0 = threadIdx.x; i0 < nfiled; i0 += kScanBatch * nthr) {
+            uint32_t bin[kScanBatch];
+#pragma unroll
+            for (int u = 0; u < kScanBatch; ++u) {
+                const int i = i0 + u * nthr;
+                bin[u] = i < nfiled ? ld_stream_u16(brec + i) : 0xffffffffu;
             }
-            if (lane == 31) s_warp[warp] = incl;
-            __syncthreads();
-            if (warp == 0) {
-                int v = lane < nwarps ? s_warp[lane] : 0;
-                for (int o = 1; o < 32; o <<= 1) {
-                    const int u = __shfl_up_sync(0xffffffffu, v, o);
-                    if (lane >= o) v += u;
-                }
-                if (lane < nwarps) s_warp[lane] = v;  // inclusive warp totals
-                if (lane == nwarps - 1) s_total = v;
-            }
-            __syncthreads();
-            int run = incl - local + (warp > 0 ? s_warp[warp - 1] : 0);
-            for (int b = b0; b < min(nbins, b0 + per); ++b) {
-                cur[b] = run;
-                run += cnt[b];
-            }
-            __syncthreads();
-            sorted = s_total <= g.bcap;
-            if (!sorted) break;
+#pragma unroll
+            for (int u = 0; u < kScanBatch; ++u)
+                if (bin[u] != 0xffffffffu) atomicAdd(&cnt[bin[u]], 1);
         }
-        if (scanner && listed) {
-            // Lean walk over the listed pixels: 32-bit math, constants hoisted.
-            const int Wo = g.Wo, sh = g.sh, sw = g.sw;
-            const int hbase = ah0 - (y0 - 1), wbase = aw0 - (x0 - 1);  // cell row/col relative to the tile's cells
-            const int binbase = sg * cells;
-            for (int e = tslot; e < nlist; e += spt) {
-                const uint32_t lv = s_list[e];
-                const int ho = static_cast<int>(lv >> 16), wo = static_cast<int>(lv & 0xffff);
-                const int pix = ho * Wo + wo;
-                SampleEntry<T> sr;
-                if constexpr (COMPACT) {
-                    sr = ld_stream_u64(code_n + static_cast<long long>(pix) * GK);
-                } else {
-                    sr = ld_stream_u16(code_n + static_cast<long long>(pix) * GK);
+        bins_exclusive_scan(cnt, cur, nbins, s_warp, &s_total);
+        for (int i0 = threadIdx.x; i0 < nfiled; i0 += kScanBatch * nthr) {
+            uint64_t r[kScanBatch];
+            uint32_t p[kScanBatch];
+#pragma unroll
+            for (int u = 0; u < kScanBatch; ++u) {
+                const int i = i0 + u * nthr;
+                r[u] = 0;
+                p[u] = 0;
+                if (i < nfiled) {
+                    r[u] = ld_stream_u64(brec + i);
+                    p[u] = ld_stream_u32(bpix + i);
                 }
-                const uint16_t cd = static_cast<uint16_t>(sr & 0xffff);
-                const int ch = ho * sh + hbase + static_cast<int8_t>(cd & 0xff);
-                const int cw = wo * sw + wbase + static_cast<int8_t>(cd >> 8);
-                if (cd == kCodeNone || static_cast<unsigned>(ch) > static_cast<unsigned>(bh) ||
-                    static_cast<unsigned>(cw) > static_cast<unsigned>(bw))
+            }
+#pragma unroll
+            for (int u = 0; u < kScanBatch; ++u) {
+                if (i0 + u * nthr >= nfiled) continue;
+                uint32_t id;
+                if (!compact_source(static_cast<int>(p[u] >> 16), static_cast<int>(p[u] & 0xffff), ho_ref, wo_ref, id)) {
+                    s_fail = 1;
                     continue;
-                const int bin = binbase + ch * cells_w + cw;
-                if (pass == 0) {
-                    atomicAdd(&cnt[bin], 1);
-                } else {
-                    const int slot = atomicAdd(&cur[bin], 1);
-                    if constexpr (COMPACT) {
-                        // the sample pass already left the mask bits and fixed-point lh, lw
-                        rec_c[slot] = make_uint2(static_cast<uint32_t>(e) | (static_cast<uint32_t>(sr) & 0xffff0000u),
-                                                 static_cast<uint32_t>(sr >> 32));
-                    } else {
-                        const T* orow = om_n + static_cast<long long>(pix) * g.P;
-                        const Candidate c = candidate(g, orow, sk, ho, wo, s_ih, s_iw);
-                        const float mf = ld_stream_elem(orow + 2 * g.K + sk);
-                        const float b = mf * c.lh;
-                        rec_w[slot] = make_float4(__int_as_float(pix), mf - b, b, c.lw);
-                    }
                 }
+                const int slot = atomicAdd(&cur[static_cast<uint32_t>(r[u]) & 0xffff], 1);
+                rec_c[slot] = make_uint2(id | (static_cast<uint32_t>(r[u]) & 0xffff0000u), static_cast<uint32_t>(r[u] >> 32));
             }
-        } else if (scanner) {
-            // Without a list: every pixel whose anchor for this point lies within R.
-            int ho = 0, wo = 0;
-            if (tslot < k_cnt) {
-                const int eh = tslot / k_w;
-                ho = kh_lo + eh;
-                wo = kw_lo + tslot - eh * k_w;
-            }
-            for (int e = tslot; e < k_cnt; e += spt) {
-                const long long pix = static_cast<long long>(ho) * g.Wo + wo;
-                int h0, w0;
-                bool any;
-                Candidate c;
-                if (use_codes) {
-                    uint16_t cd;
-                    if constexpr (COMPACT) {
-                        cd = static_cast<uint16_t>(ld_stream_u64(code_n + pix * GK) & 0xffff);
-                    } else {
-                        cd = ld_stream_u16(code_n + pix * GK);
-                    }
-                    any = cd != kCodeNone;
-                    h0 = ho * g.sh + ah0 + static_cast<int8_t>(cd & 0xff);
-                    w0 = wo * g.sw + aw0 + static_cast<int8_t>(cd >> 8);
-                } else {
-                    c = candidate(g, om_n + pix * g.P, sk, ho, wo, s_ih, s_iw);
-                    any = c.any;
-                    h0 = c.h0;
-                    w0 = c.w0;
+        }
+        __syncthreads();
+        sorted = s_fail == 0;
+    } else {
+        // Rescan: samples that can touch the tile come from output pixels
+        // whose anchor (for the sample's grid point) lies within R of the tile
+        // and whose cell box meets the tile's cells.
+        for (int gk = threadIdx.x; gk < GK; gk += nthr) {
+            // Per (group, point): bin offset of the group, and the anchor of the
+            // point relative to the tile's first cell (anchor row = ho*sh + .y,
+            // column = wo*sw + .z); .w = point | group << 16.
+            const int sg = gk / g.K, sk = gk - (gk / g.K) * g.K;
+            int ih, iw;
+            grid_cell_of(g, sk, ih, iw);
+            s_tab[gk] = make_int4(sg * cells, ih * g.dh - g.ph - (y0 - 1), iw * g.dw - g.pw - (x0 - 1), sk | (sg << 16));
+        }
+        const bool boxes_exact = R <= kCodeReach && R + max((g.kh - 1) * g.dh, (g.kw - 1) * g.dw) <= 127;
+        int ho_lo = 0, ho_hi = -1, wo_lo = 0, wo_hi = -1;
+        if (R >= 0) {
+            ho_lo = max(0, ceil_div(y0 - R + g.ph - (g.kh - 1) * g.dh, g.sh));
+            ho_hi = min(g.Ho - 1, floor_div(y0 + bh - 1 + R + g.ph, g.sh));
+            wo_lo = max(0, ceil_div(x0 - R + g.pw - (g.kw - 1) * g.dw, g.sw));
+            wo_hi = min(g.Wo - 1, floor_div(x0 + bw - 1 + R + g.pw, g.sw));
+        }
+        const int e_w = max(0, wo_hi - wo_lo + 1);
+        const int e_cnt = e_w * max(0, ho_hi - ho_lo + 1);
+        __syncthreads();
+        // List the candidate pixels; four box reads per lane in flight.
+        if (boxes_exact) {
+            for (int e0 = warp * 128; e0 < e_cnt; e0 += nwarps * 128) {
+                uint32_t box[4];
+                int hos[4], wos[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int e = e0 + u * 32 + lane;
+                    const int eh = e / e_w;
+                    hos[u] = ho_lo + eh;
+                    wos[u] = wo_lo + (e - eh * e_w);
+                    box[u] = e < e_cnt ? boxes[pix0 + static_cast<long long>(hos[u]) * g.Wo + wos[u]] : 0u;
                 }
-                const int ch = h0 - (y0 - 1), cw = w0 - (x0 - 1);
-                if (any && static_cast<unsigned>(ch) <= static_cast<unsigned>(bh) &&
-                    static_cast<unsigned>(cw) <= static_cast<unsigned>(bw)) {
-                    const int bin = sg * cells + ch * cells_w + cw;
-                    if (pass == 0) {
-                        atomicAdd(&cnt[bin], 1);
-                    } else if constexpr (!COMPACT) {  // compact records need the list (direct path instead)
-                        const T* orow = om_n + pix * g.P;
-                        if (use_codes) c = candidate(g, orow, sk, ho, wo, s_ih, s_iw);
-                        const int slot = atomicAdd(&cur[bin], 1);
-                        const float mf = ld_stream_elem(orow + 2 * g.K + sk);
-                        const float b = mf * c.lh;
-                        rec_w[slot] = make_float4(__int_as_float(static_cast<int>(pix)), mf - b, b, c.lw);
-                    }
-                }
-                wo += spt;  // next pixel of this slot
-                while (wo > kw_hi) {
-                    wo -= k_w;
-                    ++ho;
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int bh0 = hos[u] * g.sh - g.ph, bw0 = wos[u] * g.sw - g.pw;
+                    const int rmin = bh0 + static_cast<int8_t>(box[u] & 0xff);
+                    const int rmax = bh0 + static_cast<int8_t>((box[u] >> 8) & 0xff);
+                    const int cmin = bw0 + static_cast<int8_t>((box[u] >> 16) & 0xff);
+                    const int cmax = bw0 + static_cast<int8_t>(box[u] >> 24);
+                    const bool keep = e0 + u * 32 + lane < e_cnt && rmax >= y0 - 1 && rmin <= y0 + bh - 1 &&
+                                      cmax >= x0 - 1 && cmin <= x0 + bw - 1;
+                    const unsigned ball = __ballot_sync(0xffffffffu, keep);
+                    int base = 0;
+                    if (lane == 0 && ball) base = atomicAdd(&s_nlist, __popc(ball));
+                    base = __shfl_sync(0xffffffffu, base, 0);
+                    const int pos = base + __popc(ball & ((1u << lane) - 1));
+                    if (keep && pos < kListCap)
+                        s_list[pos] = (static_cast<uint32_t>(hos[u]) << 16) | static_cast<uint32_t>(wos[u]);
                 }
             }
         }
         __syncthreads();
-    }
-    // Compact records need the list; without it the tile takes the direct path.
-    if (COMPACT && !listed) sorted = false;
-
-    // Pull: thread -> (input pixel q of the tile, group, slice).
-    const int lanes_pp = g.G * g.nslice;
-    const int q = threadIdx.x / lanes_pp;
-    const int qy = q / g.BW, qx = q - (q / g.BW) * g.BW;
-    if (q >= g.BH * g.BW || qy >= bh || qx >= bw) return;
-    const int rr = threadIdx.x - q * lanes_pp;
-    const int grp = rr / g.nslice;
-    const int sl = rr - grp * g.nslice;
-    const int ch_off = grp * g.Cg + sl * (VEC * EPV);
-    const T* gy_img = gout + pix0 * g.C + ch_off;
-
-    float2 acc[PAIRS];
+        const int nlist = s_nlist;
+        sorted = boxes_exact && nlist <= kListCap && g.Ho <= 65535 && g.Wo <= 65535 && compact_ok &&
+                 static_cast<long long>(g.Ho) * g.Wo * g.C < (1LL << 31);
+        if (sorted) {
+            // Each thread keeps one (group, point) -- its bin base and anchor
+            // offset stay in registers -- and walks the listed pixels of its
+            // slot, kScanBatch code reads in flight.  Pass 0 counts the samples
+            // of each (group, cell); pass 1 places their records in bin order.
+            const int spt = GK <= nthr ? nthr / GK : 1;
+            const int tslot = GK <= nthr ? static_cast<int>(threadIdx.x) / GK : 0;
+            const int gk_first = threadIdx.x - tslot * GK;
+            const int Wo = g.Wo, sh = g.sh, sw = g.sw;
+            for (int pass = 0; pass < 2; ++pass) {
+                if (pass == 1) {
+                    sorted = bins_exclusive_scan(cnt, cur, nbins, s_warp, &s_total) <= g.bcap;
+                    if (!sorted) break;
+                }
+                for (int gk = gk_first; tslot < spt && gk < GK; gk += nthr) {
+                    const int4 tb = s_tab[gk];
+                    const long long ebase = pix0 * GK + gk;  // entry of listed pixel pix: ebase + pix * GK
+                    const int sk = tb.w & 0xffff, sg = tb.w >> 16;
+                    int ih, iw;
+                    grid_cell_of(g, sk, ih, iw);
+                    for (int e0 = tslot; e0 < nlist; e0 += kScanBatch * spt) {
+                        // Cell of each sample: fp32 from its code; 16-bit dtypes
+                        // re-form it from the offsets (the same fp32 fma).
+                        uint32_t lv[kScanBatch];
+                        int bin[kScanBatch];
+                        Candidate c[kScanBatch];
 #pragma unroll
-    for (int i = 0; i < PAIRS; ++i) acc[i] = make_float2(0.f, 0.f);
+                        for (int u = 0; u < kScanBatch; ++u) {
+                            const int e = e0 + u * spt;
+                            lv[u] = e < nlist ? s_list[e] : 0;
+                            const int ho = static_cast<int>(lv[u] >> 16), wo = static_cast<int>(lv[u] & 0xffff);
+                            const int pix = ho * Wo + wo;
+                            c[u].any = false;
+                            if (e < nlist) {
+                                if constexpr (COMPACT) {
+                                    c[u] = candidate(g, om + (pix0 + pix) * g.P + sg * 3 * g.K, sk, ho, wo, ih, iw);
+                                } else {
+                                    const uint32_t cd = ld_stream_u16(sa.code + ebase + static_cast<long long>(pix) * GK);
+                                    c[u].any = cd != kCodeNone;
+                                    c[u].h0 = ho * sh + tb.y + (y0 - 1) + static_cast<int8_t>(cd & 0xff);
+                                    c[u].w0 = wo * sw + tb.z + (x0 - 1) + static_cast<int8_t>(cd >> 8);
+                                }
+                            }
+                        }
+#pragma unroll
+                        for (int u = 0; u < kScanBatch; ++u) {
+                            const int ch = c[u].h0 - (y0 - 1), cw = c[u].w0 - (x0 - 1);
+                            const bool in = c[u].any && static_cast<unsigned>(ch) <= static_cast<unsigned>(bh) &&
+                                            static_cast<unsigned>(cw) <= static_cast<unsigned>(bw);
+                            bin[u] = in ? tb.x + ch * cells_w + cw : -1;
+                        }
+                        if (pass == 0) {
+#pragma unroll
+                            for (int u = 0; u < kScanBatch; ++u)
+                                if (bin[u] >= 0) atomicAdd(&cnt[bin[u]], 1);
+                            continue;
+                        }
+#pragma unroll
+                        for (int u = 0; u < kScanBatch; ++u) {
+                            if (bin[u] < 0) continue;
+                            const int ho = static_cast<int>(lv[u] >> 16), wo = static_cast<int>(lv[u] & 0xffff);
+                            const int pix = ho * Wo + wo;
+                            const T* orow = om + (pix0 + pix) * g.P + sg * 3 * g.K;
+                            const int slot = atomicAdd(&cur[bin[u]], 1);
+                            if constexpr (COMPACT) {
+                                uint32_t id;
+                                if (!compact_source(ho, wo, ho_ref, wo_ref, id)) s_fail = 1;
+                                const uint32_t mb = ld_stream_u16(orow + 2 * g.K + sk);
+                                rec_c[slot] = make_uint2(id | (mb << 16), fix16(c[u].lh) | (fix16(c[u].lw) << 16));
+                            } else {
+                                const Candidate cc = candidate(g, orow, sk, ho, wo, ih, iw);
+                                const float mf = ld_stream_elem(orow + 2 * g.K + sk);
+                                const float b = mf * cc.lh;
+                                rec_w[slot] = make_float4(__int_as_float(pix * g.C), mf - b, b, cc.lw);
+                            }
+                        }
+                    }
+                }
+                __syncthreads();
+            }
+            if (sorted) sorted = s_fail == 0;
+        }
+    }
 
     if (sorted) {
-        // q is corner (a, b) of the cell with top-left (qy - a, qx - b).
+        // Pull over strips.  A strip is LW lanes of a warp; lane cx owns cell
+        // column cx of one (group, channel slice) and one segment of BS pixel
+        // rows, and walks the segment's cell rows top to bottom.  Each sample
+        // of its cell is read once and added, with its four bilinear weights,
+        // to the partial sums of the cell's corners: left/right of the pixel
+        // row above the cell (top) and of the row below it (bottom).  After a
+        // cell row the pixel row above it is complete but for the left
+        // corners of the next cell column, which the next lane holds: one
+        // shuffle adds them and the lane writes its pixel.  Partial sums that
+        // fall outside the segment are dropped (the neighbouring segment
+        // forms them too).
+        const int LW = g.LW;
+        const int strips = 32 / LW;
+        const int cx = lane & (LW - 1);
+        const int gs_count = g.G * g.nslice;
+        const int items = gs_count * g.nseg;
+        for (int base = warp * strips; base < items; base += nwarps * strips) {
+            const int item = base + lane / LW;
+            const bool live = item < items;
+            const int seg = item / gs_count;
+            const int gsl = item - seg * gs_count;
+            const int grp = gsl / g.nslice, sl = gsl - (gsl / g.nslice) * g.nslice;
+            const int r0 = seg * g.BS;
+            const int r1 = min(r0 + g.BS, bh);  // pixel rows [r0, r1) of the tile
+            const int ch_off = grp * g.Cg + sl * (VEC * EPV);
+            GySource<T> gs;
+            gs.row = g.Wo * g.C;
+            gs.col = g.C;
+            gs.ref = gout + pix0 * g.C + ch_off;
+            if constexpr (COMPACT) gs.ref += (static_cast<long long>(ho_ref - 64) * g.Wo + (wo_ref - 64)) * g.C;
+            // Ping-pong partial sums: A and B alternate as the pixel row above
+            // (top) and below (bottom) the current cell row.
+            float2 a0[PAIRS], a1[PAIRS], b0[PAIRS], b1[PAIRS];
 #pragma unroll
-        for (int a = 0; a < 2; ++a) {
-#pragma unroll
-            for (int b = 0; b < 2; ++b) {
-                const int bin = grp * cells + (qy - a + 1) * cells_w + (qx - b + 1);
-                const int end = cur[bin];
-                int j = end - cnt[bin];
-                // Two records per step, so two grad_out gathers are in flight.
-                for (; j + 1 < end; j += 2) {
-                    const T* src[2];
-                    float wt[2];
-#pragma unroll
-                    for (int u = 0; u < 2; ++u) {
-                        if constexpr (COMPACT) {
-                            const uint2 r = rec_c[j + u];
-                            const uint32_t lv = s_list[r.x & 0xffff];
-                            const float m = from_bits(static_cast<uint16_t>(r.x >> 16), T());
-                            const float hq = static_cast<float>(a ? (r.y & 0xffff) : 65536u - (r.y & 0xffff));
-                            const float wq = static_cast<float>(b ? (r.y >> 16) : 65536u - (r.y >> 16));
-                            wt[u] = m * (hq * wq) * 0x1p-32f;
-                            src[u] = gy_img + ((lv >> 16) * static_cast<long long>(g.Wo) + (lv & 0xffff)) * g.C;
-                        } else {
-                            const float4 r = rec_w[j + u];
-                            wt[u] = (a ? r.z : r.y) * (b ? r.w : 1.f - r.w);
-                            src[u] = gy_img + static_cast<long long>(__float_as_int(r.x)) * g.C;
-                        }
-                    }
-                    uint4 raw[2][VEC];
-#pragma unroll
-                    for (int u = 0; u < 2; ++u) {
-                        if constexpr (VEC == 2) {
-                            ld_keep32(src[u], raw[u][0], raw[u][1]);
-                        } else {
-                            raw[u][0] = ld_keep16(src[u]);
-                        }
-                    }
-#pragma unroll
-                    for (int u = 0; u < 2; ++u) {
-                        const float2 w2 = make_float2(wt[u], wt[u]);
-#pragma unroll
-                        for (int v = 0; v < VEC; ++v) {
-                            float2 f[EPV / 2];
-                            unpack(raw[u][v], f, T());
-#pragma unroll
-                            for (int i = 0; i < EPV / 2; ++i)
-                                acc[v * (EPV / 2) + i] = __ffma2_rn(w2, f[i], acc[v * (EPV / 2) + i]);
-                        }
-                    }
+            for (int i = 0; i < PAIRS; ++i) a0[i] = a1[i] = b0[i] = b1[i] = make_float2(0.f, 0.f);
+            const bool has_col = live && cx <= bw;
+            T* dst_col = gvalue + ((static_cast<long long>(n) * g.H + y0) * g.W + x0 + cx) * g.C + ch_off;
+            const long long row_stride = static_cast<long long>(g.W) * g.C;
+            for (int t = 0; t <= g.BS; t += 2) {
+                int cy = r0 + t;
+                int end = 0, j = 0;
+                if (has_col && cy <= r1) {
+                    const int bin = grp * cells + cy * cells_w + cx;
+                    end = cur[bin];
+                    j = end - cnt[bin];
                 }
-                if (j < end) {
-                    const T* src;
-                    float wt;
-                    if constexpr (COMPACT) {
-                        const uint2 r = rec_c[j];
-                        const uint32_t lv = s_list[r.x & 0xffff];
-                        const float m = from_bits(static_cast<uint16_t>(r.x >> 16), T());
-                        const float hq = static_cast<float>(a ? (r.y & 0xffff) : 65536u - (r.y & 0xffff));
-                        const float wq = static_cast<float>(b ? (r.y >> 16) : 65536u - (r.y >> 16));
-                        wt = m * (hq * wq) * 0x1p-32f;
-                        src = gy_img + ((lv >> 16) * static_cast<long long>(g.Wo) + (lv & 0xffff)) * g.C;
-                    } else {
-                        const float4 r = rec_w[j];
-                        wt = (a ? r.z : r.y) * (b ? r.w : 1.f - r.w);
-                        src = gy_img + static_cast<long long>(__float_as_int(r.x)) * g.C;
-                    }
-                    accumulate<T, VEC>(acc, src, wt);
+                pull_cell<T, VEC, COMPACT>(rec_base, gs, j, end, a0, a1, b0, b1);
+                // pixel row cy - 1 (in A) is complete
+                finish_row<T, VEC>(a0, a1, LW, live && t > 0 && cy - 1 < r1 && cx < bw, dst_col + (cy - 1) * row_stride);
+                if (t + 1 > g.BS) break;
+                ++cy;
+                end = j = 0;
+                if (has_col && cy <= r1) {
+                    const int bin = grp * cells + cy * cells_w + cx;
+                    end = cur[bin];
+                    j = end - cnt[bin];
                 }
+                pull_cell<T, VEC, COMPACT>(rec_base, gs, j, end, b0, b1, a0, a1);
+                finish_row<T, VEC>(b0, b1, LW, live && cy - 1 < r1 && cx < bw, dst_col + (cy - 1) * row_stride);
             }
         }
-    } else {
-        // Direct path: scan every candidate sample of this group.
-        const int uh_lo = max(0, ceil_div(y0 - R + g.ph - (g.kh - 1) * g.dh, g.sh));
-        const int uh_hi = min(g.Ho - 1, floor_div(y0 + bh - 1 + R + g.ph, g.sh));
-        const int uw_lo = max(0, ceil_div(x0 - R + g.pw - (g.kw - 1) * g.dw, g.sw));
-        const int uw_hi = min(g.Wo - 1, floor_div(x0 + bw - 1 + R + g.pw, g.sw));
-        const int u_w = max(0, uw_hi - uw_lo + 1);
-        const int u_cnt = R >= 0 ? u_w * max(0, uh_hi - uh_lo + 1) : 0;
+        return;
+    }
+
+    // Direct path (records that do not fit, or a tile the sort cannot name):
+    // thread -> (input pixel, group, slice) of the tile, scanning every
+    // candidate sample of its group.
+    const int lanes_pp = g.G * g.nslice;
+    const int uh_lo = max(0, ceil_div(y0 - R + g.ph - (g.kh - 1) * g.dh, g.sh));
+    const int uh_hi = min(g.Ho - 1, floor_div(y0 + bh - 1 + R + g.ph, g.sh));
+    const int uw_lo = max(0, ceil_div(x0 - R + g.pw - (g.kw - 1) * g.dw, g.sw));
+    const int uw_hi = min(g.Wo - 1, floor_div(x0 + bw - 1 + R + g.pw, g.sw));
+    const int u_w = max(0, uw_hi - uw_lo + 1);
+    const int u_cnt = R >= 0 ? u_w * max(0, uh_hi - uh_lo + 1) : 0;
+    for (int it = threadIdx.x; it < bh * bw * lanes_pp; it += nthr) {
+        const int q = it / lanes_pp;
+        const int rr = it - q * lanes_pp;
+        const int grp = rr / g.nslice;
+        const int sl = rr - grp * g.nslice;
+        const int qy = q / bw, qx = q - (q / bw) * bw;
+        const int ch_off = grp * g.Cg + sl * (VEC * EPV);
+        const T* gy_img = gout + pix0 * g.C + ch_off;
+        float2 acc[PAIRS];
+#pragma unroll
+        for (int i = 0; i < PAIRS; ++i) acc[i] = make_float2(0.f, 0.f);
         const int gy_abs = y0 + qy, gx_abs = x0 + qx;
         const T* om_g = om + pix0 * g.P + grp * 3 * g.K;
         for (int e = 0; e < u_cnt; ++e) {
@@ -685,13 +971,12 @@ __global__ void __launch_bounds__(512, 2) value_kernel(const Geometry g, const T
                 }
             }
         }
-    }
-
-    T* dst = gvalue + ((static_cast<long long>(n) * g.H + y0 + qy) * g.W + x0 + qx) * g.C + ch_off;
-    if constexpr (VEC == 2) {
-        st_global32(dst, pack(acc, T()), pack(acc + EPV / 2, T()));
-    } else {
-        st_global(dst, pack(acc, T()));
+        T* dst = gvalue + ((static_cast<long long>(n) * g.H + gy_abs) * g.W + gx_abs) * g.C + ch_off;
+        if constexpr (VEC == 2) {
+            st_global32(dst, pack(acc, T()), pack(acc + EPV / 2, T()));
+        } else {
+            st_global(dst, pack(acc, T()));
+        }
     }
 }
 
@@ -708,85 +993,88 @@ cudaError_t allow_smem(Kern kern, size_t smem) {
 
 template <typename T, int VEC, int KH, int KW, bool RC>
 cudaError_t launch_samples_typed(const Geometry& g, const void* value, const void* om, const void* gout, void* gom,
-                                 int* reach, void* codes, uint32_t* boxes, cudaStream_t stream) {
+                                 int* reach, SampleArrays sa, uint32_t* boxes, cudaStream_t stream) {
     const size_t smem = backward_smem_bytes(g, sizeof(T));
     auto kern = samples_kernel<T, VEC, KH, KW, RC>;
     cudaError_t e = allow_smem(kern, smem);
     if (e != cudaSuccess) return e;
     const long long blocks = static_cast<long long>(g.N) * g.tiles_h * g.tiles_w;
-    const int threads = (g.pix_per_cta * g.G * g.nslice + 31) / 32 * 32;  // whole warps (shuffles)
+    const int threads = samples_threads(g);
     kern<<<static_cast<unsigned>(blocks), threads, smem, stream>>>(g, static_cast<const T*>(value),
                                                                    static_cast<const T*>(om), static_cast<const T*>(gout),
-                                                                   static_cast<T*>(gom), reach, codes, boxes);
+                                                                   static_cast<T*>(gom), reach, sa, boxes);
     return cudaGetLastError();
 }
 
 template <typename T, int VEC>
 cudaError_t launch_samples_grid(const Geometry& g, const void* value, const void* om, const void* gout, void* gom,
-                                int* reach, void* codes, uint32_t* boxes, cudaStream_t stream) {
+                                int* reach, SampleArrays sa, uint32_t* boxes, cudaStream_t stream) {
     if (g.kh == 3 && g.kw == 3) {
         return g.remove_center
-                   ? launch_samples_typed<T, VEC, 3, 3, true>(g, value, om, gout, gom, reach, codes, boxes, stream)
-                   : launch_samples_typed<T, VEC, 3, 3, false>(g, value, om, gout, gom, reach, codes, boxes, stream);
+                   ? launch_samples_typed<T, VEC, 3, 3, true>(g, value, om, gout, gom, reach, sa, boxes, stream)
+                   : launch_samples_typed<T, VEC, 3, 3, false>(g, value, om, gout, gom, reach, sa, boxes, stream);
     }
-    return launch_samples_typed<T, VEC, 0, 0, false>(g, value, om, gout, gom, reach, codes, boxes, stream);
+    return launch_samples_typed<T, VEC, 0, 0, false>(g, value, om, gout, gom, reach, sa, boxes, stream);
 }
 
 template <typename T>
 cudaError_t launch_samples_vec(const Geometry& g, const void* value, const void* om, const void* gout, void* gom,
-                               int* reach, void* codes, uint32_t* boxes, cudaStream_t stream) {
-    return g.vec == 2 ? launch_samples_grid<T, 2>(g, value, om, gout, gom, reach, codes, boxes, stream)
-                      : launch_samples_grid<T, 1>(g, value, om, gout, gom, reach, codes, boxes, stream);
+                               int* reach, SampleArrays sa, uint32_t* boxes, cudaStream_t stream) {
+    return g.vec == 2 ? launch_samples_grid<T, 2>(g, value, om, gout, gom, reach, sa, boxes, stream)
+                      : launch_samples_grid<T, 1>(g, value, om, gout, gom, reach, sa, boxes, stream);
 }
 
 template <typename T, int VEC>
 cudaError_t launch_value_typed(const Geometry& g, const void* om, const void* gout, void* gvalue, const int* reach,
-                               const void* codes, const uint32_t* boxes, cudaStream_t stream) {
+                               SampleArrays sa, const uint32_t* boxes, cudaStream_t stream) {
     const size_t smem = backward_value_smem_bytes(g);
     auto kern = value_kernel<T, VEC, sizeof(T) == 2>;
     cudaError_t e = allow_smem(kern, smem);
     if (e != cudaSuccess) return e;
     const long long blocks = static_cast<long long>(g.N) * g.btiles_h * g.btiles_w;
     kern<<<static_cast<unsigned>(blocks), g.bthreads, smem, stream>>>(
-        g, static_cast<const T*>(om), static_cast<const T*>(gout), static_cast<T*>(gvalue), reach, codes, boxes);
+        g, static_cast<const T*>(om), static_cast<const T*>(gout), static_cast<T*>(gvalue), reach, sa, boxes);
     return cudaGetLastError();
 }
 
 template <typename T>
 cudaError_t launch_value_vec(const Geometry& g, const void* om, const void* gout, void* gvalue, const int* reach,
-                             const void* codes, const uint32_t* boxes, cudaStream_t stream) {
-    return g.vec == 2 ? launch_value_typed<T, 2>(g, om, gout, gvalue, reach, codes, boxes, stream)
-                      : launch_value_typed<T, 1>(g, om, gout, gvalue, reach, codes, boxes, stream);
+                             SampleArrays sa, const uint32_t* boxes, cudaStream_t stream) {
+    return g.vec == 2 ? launch_value_typed<T, 2>(g, om, gout, gvalue, reach, sa, boxes, stream)
+                      : launch_value_typed<T, 1>(g, om, gout, gvalue, reach, sa, boxes, stream);
 }
 
 }  // namespace
 
 size_t backward_smem_bytes(const Geometry& g, int elem_bytes) {
-    return static_cast<size_t>(g.TH) * g.TW * g.P * elem_bytes * 2;
+    size_t b = static_cast<size_t>(g.TH) * g.TW * g.P * elem_bytes * 2;
+    if (elem_bytes == 2 && g.buckets) b += static_cast<size_t>(g.K) * samples_threads(g) * 16;  // filing staging
+    return b;
 }
 
 size_t backward_value_smem_bytes(const Geometry& g) {
     const size_t nbins = static_cast<size_t>(g.G) * (g.BH + 1) * (g.BW + 1);
-    return ((2 * nbins + kListCap) * sizeof(int) + 15) / 16 * 16 + static_cast<size_t>(g.bcap) * g.brec;
+    return ((2 * nbins + kListCap) * sizeof(int) + 15) / 16 * 16 + static_cast<size_t>(g.G) * g.K * sizeof(int4) +
+           static_cast<size_t>(g.bcap) * g.brec;
 }
 
 cudaError_t launch_backward_samples(const Geometry& g, int dtype, const void* value, const void* om, const void* gout,
-                                    void* gom, int* reach, void* codes, uint32_t* boxes, cudaStream_t stream) {
+                                    void* gom, int* reach, SampleArrays sa, uint32_t* boxes, cudaStream_t stream) {
     switch (dtype) {
-        case 0: return launch_samples_vec<float>(g, value, om, gout, gom, reach, codes, boxes, stream);
-        case 1: return launch_samples_vec<__half>(g, value, om, gout, gom, reach, codes, boxes, stream);
-        case 2: return launch_samples_vec<__nv_bfloat16>(g, value, om, gout, gom, reach, codes, boxes, stream);
+        case 0: return launch_samples_vec<float>(g, value, om, gout, gom, reach, sa, boxes, stream);
+        case 1: return launch_samples_vec<__half>(g, value, om, gout, gom, reach, sa, boxes, stream);
+        case 2: return launch_samples_vec<__nv_bfloat16>(g, value, om, gout, gom, reach, sa, boxes, stream);
         default: return cudaErrorInvalidValue;
     }
 }
 
 cudaError_t launch_backward_value(const Geometry& g, int dtype, const void* om, const void* gout, void* gvalue,
-                                  const int* reach, const void* codes, const uint32_t* boxes,
+                                  const int* reach, SampleArrays sa, const uint32_t* boxes,
                                   cudaStream_t stream) {
     switch (dtype) {
-        case 0: return launch_value_vec<float>(g, om, gout, gvalue, reach, codes, boxes, stream);
-        case 1: return launch_value_vec<__half>(g, om, gout, gvalue, reach, codes, boxes, stream);
-        case 2: return launch_value_vec<__nv_bfloat16>(g, om, gout, gvalue, reach, codes, boxes, stream);
+        case 0: return launch_value_vec<float>(g, om, gout, gvalue, reach, sa, boxes, stream);
+        case 1: return launch_value_vec<__half>(g, om, gout, gvalue, reach, sa, boxes, stream);
+        case 2: return launch_value_vec<__nv_bfloat16>(g, om, gout, gvalue, reach, sa, boxes, stream);
         default: return cudaErrorInvalidValue;
     }
 }

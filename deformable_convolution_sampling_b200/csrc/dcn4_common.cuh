@@ -30,7 +30,34 @@ struct Geometry {
     // room for bcap sample records in shared memory.
     int BH, BW, btiles_h, btiles_w, bthreads, bcap;
     int brec;  // bytes per sample record: 8 (16-bit dtypes) or 16 (fp32)
+    int LW;    // lanes of one strip (one lane per cell column, BW + 1 <= LW): 8, 16 or 32
+    int BS;    // pixel rows of one strip segment
+    int nseg;  // segments per tile: ceil(BH / BS)
+    // Buckets (16-bit dtypes): the grad_offset_mask pass files each sample's
+    // record under every grad_value tile whose cells hold it, up to bcap per
+    // tile.  bh_magic / bw_magic divide a pixel coordinate by BH / BW with
+    // __umulhi (exact for coordinates < 2^24).
+    int buckets;
+    uint32_t bh_magic, bw_magic;
 };
+
+// What the grad_offset_mask pass leaves for the grad_value pass.
+//   code        [N, Ho, Wo, G, K]  fp32: the cell code of every sample
+// 16-bit dtypes, when g.buckets:
+//   tile_count  [N * btiles_h * btiles_w]  records filed per grad_value tile
+//               (pre-zeroed; above bcap -- or with kBucketOverflow set -- the
+//               tile's bucket is incomplete and the tile rescans the offsets)
+//   bucket_pix  [tiles][bcap]  output pixel of the record, (ho << 16) | wo
+//   bucket_rec  [tiles][bcap]  bin (group, cell) of the record in the tile |
+//               mask bits << 16 | lh << 32 | lw << 48 (16-bit fixed point)
+// Arrays a dtype does not use are NULL.
+struct SampleArrays {
+    uint16_t* code;
+    int* tile_count;
+    uint32_t* bucket_pix;
+    uint64_t* bucket_rec;
+};
+constexpr int kBucketOverflow = 1 << 30;
 
 template <typename T>
 struct Elem;
@@ -273,16 +300,17 @@ namespace dcn4 {
 cudaError_t launch_forward(const Geometry& g, int dtype, const void* value, const void* om, void* out,
                            cudaStream_t stream);
 // grad_offset_mask and the per-image reach (int[N], pre-filled with -1).
-// Also writes one entry per sample, codes[N, Ho, Wo, G, K] (a 2-byte cell code for
-// fp32, an 8-byte record for 16-bit dtypes), and the
-// bounding box of each output pixel's cells, boxes[N, Ho, Wo].
+// Also writes the per-sample entries of `sa` and the bounding box of each
+// output pixel's cells, boxes[N, Ho, Wo].
 cudaError_t launch_backward_samples(const Geometry& g, int dtype, const void* value, const void* om,
-                                    const void* gout, void* gom, int* reach, void* codes, uint32_t* boxes,
+                                    const void* gout, void* gom, int* reach, SampleArrays sa, uint32_t* boxes,
                                     cudaStream_t stream);
-// grad_value from the reach, cell codes and boxes written by launch_backward_samples.
+// grad_value from the reach, sample entries and boxes written by launch_backward_samples.
 cudaError_t launch_backward_value(const Geometry& g, int dtype, const void* om, const void* gout, void* gvalue,
-                                  const int* reach, const void* codes, const uint32_t* boxes,
+                                  const int* reach, SampleArrays sa, const uint32_t* boxes,
                                   cudaStream_t stream);
+// Threads of one grad_offset_mask CTA: whole warps (the kernel shuffles).
+inline int samples_threads(const Geometry& g) { return (g.pix_per_cta * g.G * g.nslice + 31) / 32 * 32; }
 // Dynamic shared memory bytes of one CTA.
 size_t forward_smem_bytes(const Geometry& g, int elem_bytes);
 size_t backward_smem_bytes(const Geometry& g, int elem_bytes);

@@ -82,14 +82,21 @@ def test_output_dims_agree_with_the_oracle(dcn):
 
 
 def test_workspace_size(dcn):
-    """Per image a reach word, per output pixel a cell box (each rounded up to 256 bytes), per
-    sample a 2-byte cell code (fp32) or an 8-byte sample record (16-bit dtypes)."""
+    """Per image a reach word, per output pixel a cell box; then per sample a 2-byte cell code
+    (fp32), or (16-bit dtypes) a record counter per grad_value tile and each tile's bucket of
+    12-byte records; each array starts on a 256-byte boundary."""
     def up(x):
         return (x + 255) // 256 * 256
     p = dcn.make_params(N=64, H=56, W=56, G=4, Cg=16, dtype="f16")
-    assert dcn.dcn4_backward_workspace_size(p) == 256 + up(64 * 56 * 56 * 4) + 64 * 56 * 56 * 4 * 9 * 8
+    # grad_value tiles of 8 x 31 pixels: 7 x 2 per image; bucket room for 1.0625x the expected
+    # records (K per cell and group, (8+1) x (31+1) cells, 4 groups) + 512
+    tiles = 64 * 7 * 2
+    expect = 4 * 9 * 32 * 9
+    cap = expect + expect // 16 + 512
+    assert dcn.dcn4_backward_workspace_size(p) == (256 + up(64 * 56 * 56 * 4) + up(tiles * 4)
+                                                   + up(tiles * cap * 4) + tiles * cap * 8)
     p = dcn.make_params(N=100, H=8, W=8, G=2, Cg=8, dtype="f32", remove_center=1)
-    assert dcn.dcn4_backward_workspace_size(p) == 512 + up(100 * 64 * 4) + 100 * 64 * 2 * 8 * 2
+    assert dcn.dcn4_backward_workspace_size(p) == 512 + up(100 * 64 * 4) + up(100 * 64 * 2 * 8 * 2)
     p.Cg = 6
     assert dcn.dcn4_backward_workspace_size(p) == 0
 
