@@ -117,11 +117,16 @@ int dcn4_check_params(const dcn4_params* p);
 int dcn4_forward(const dcn4_params* p, const void* value, const void* offset_mask, void* out,
                  void* stream);
 
-/* Bytes of device workspace dcn4_backward needs: one 32-bit word per image
- * (N*4 rounded up to 256), one 32-bit cell box per output pixel (N*Ho*Wo*4
- * rounded up to 256) and one entry per sample, N*Ho*Wo*G*K of them: a 2-byte
- * cell code for fp32, an 8-byte record (cell code, mask bits, fixed-point
- * bilinear fractions) for fp16/bf16; 0 if p is invalid. */
+/* Bytes of device workspace dcn4_backward needs, each part rounded up to 256
+ * bytes: one 32-bit word per image, one 32-bit cell box per output pixel
+ * (N*Ho*Wo), then
+ *   fp32:      a 2-byte cell code per sample (N*Ho*Wo*G*K of them);
+ *   fp16/bf16: a 32-bit counter per grad_value tile and, per tile, room for
+ *              bcap 12-byte sample records (4-byte output pixel + 8 bytes of
+ *              bin, mask bits and fixed-point bilinear fractions), where the
+ *              tiles and bcap follow from the shape (about 1.06x the records
+ *              a tile expects, + 512);
+ * 0 if p is invalid. */
 size_t dcn4_backward_workspace_size(const dcn4_params* p);
 
 /* Backward of the forward for upstream gradient grad_out:
@@ -133,13 +138,15 @@ size_t dcn4_backward_workspace_size(const dcn4_params* p);
  * accumulated into); the offset_mask padding tail is written as 0.
  * `workspace` (device, 16-byte aligned, >= dcn4_backward_workspace_size bytes)
  * is scratch, clobbered by the call: it receives, per image, how far any
- * sample reaches from its grid position, and per sample the bilinear cell it
- * falls in relative to that position.
- * Launches, on `stream`: a memset of that word per image, one kernel for
- * grad_offset_mask (and the reach), and one for grad_value.  grad_value is
- * not scattered with atomics: each element is summed by one thread in fp32
- * (over the samples sorted by cell) and written once, so results are
- * deterministic up to the order in which samples of one cell are added. */
+ * sample reaches from its grid position, and per sample its bilinear cell
+ * (fp32: relative to its grid position; fp16/bf16: filed, with its weights,
+ * under every grad_value tile whose cells hold it).
+ * Launches, on `stream`: a memset of the per-image words (and, for fp16/bf16,
+ * one of the per-tile counters), one kernel for grad_offset_mask (and the
+ * workspace), and one for grad_value.  grad_value is not scattered with
+ * atomics: each element is summed by one thread in fp32 (over the samples
+ * sorted by cell) and written once, so results are deterministic up to the
+ * order in which samples of one cell are added. */
 int dcn4_backward(const dcn4_params* p, const void* value, const void* offset_mask,
                   const void* grad_out, void* grad_value, void* grad_offset_mask,
                   void* workspace, size_t workspace_bytes, void* stream);
@@ -182,8 +189,8 @@ const char* dcn4_noalloc_last_error(void);
 /* The two stages of dcn4_backward, callable on their own (same arguments,
  * layouts and errors as dcn4_backward):
  *   dcn4_backward_offset_mask writes grad_offset_mask and fills `workspace`
- *     (the per-image reach, per-pixel cell boxes and per-sample cell codes);
- *     launches a memset of one word per image and one kernel.
+ *     (the per-image reach, per-pixel cell boxes, and the per-sample cell
+ *     codes or per-tile records); launches the memsets and one kernel.
  *   dcn4_backward_value writes grad_value from offset_mask, grad_out and a
  *     workspace filled by dcn4_backward_offset_mask for the same offset_mask
  *     (and the same params), ordered before it; one kernel.
