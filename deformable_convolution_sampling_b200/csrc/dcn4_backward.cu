@@ -302,7 +302,8 @@ __global__ void __launch_bounds__(256, 3) samples_kernel(const Geometry g, const
                         const int leader = __ffs(peers) - 1;
                         int base = 0;
                         if (lane == leader) base = atomicAdd(s_fcnt + dl0, __popc(peers));
-                        base = __shfl_sync(peers, base, leader);
+                        // every lane with a record takes part (one mask for all), each reading its own leader
+                        base = __shfl_sync(okm, base, leader);
                         const int rank = base + __popc(peers & ((1u << lane) - 1));
                         meta = static_cast<uint64_t>(dl0) | (static_cast<uint64_t>(rank) << 6) | (1ull << 61);
                         // copies for the next tiles when the cell straddles a border
@@ -692,8 +693,16 @@ __global__ void __launch_bounds__(256, 2) value_kernel(const Geometry g, const T
                 bin[u] = i < nfiled ? ld_stream_u16(brec + i) : 0xffffffffu;
             }
 #pragma unroll
-            for (int u = 0; u < kScanBatch; ++u)
-                if (bin[u] != 0xffffffffu) atomicAdd(&cnt[bin[u]], 1);
+            for (int u = 0; u < kScanBatch; ++u) {
+                if (bin[u] == 0xffffffffu) continue;
+                // A bin outside the tile means a corrupt bucket: never index with it; the
+                // tile then takes the direct path.
+                if (bin[u] >= static_cast<uint32_t>(nbins)) {
+                    s_fail = 1;
+                    continue;
+                }
+                atomicAdd(&cnt[bin[u]], 1);
+            }
         }
         bins_exclusive_scan(cnt, cur, nbins, s_warp, &s_total);
         for (int i0 = threadIdx.x; i0 < nfiled; i0 += kScanBatch * nthr) {
@@ -713,11 +722,17 @@ __global__ void __launch_bounds__(256, 2) value_kernel(const Geometry g, const T
             for (int u = 0; u < kScanBatch; ++u) {
                 if (i0 + u * nthr >= nfiled) continue;
                 uint32_t id;
-                if (!compact_source(static_cast<int>(p[u] >> 16), static_cast<int>(p[u] & 0xffff), ho_ref, wo_ref, id)) {
+                const uint32_t bin = static_cast<uint32_t>(r[u]) & 0xffff;
+                if (bin >= static_cast<uint32_t>(nbins) ||
+                    !compact_source(static_cast<int>(p[u] >> 16), static_cast<int>(p[u] & 0xffff), ho_ref, wo_ref, id)) {
                     s_fail = 1;
                     continue;
                 }
-                const int slot = atomicAdd(&cur[static_cast<uint32_t>(r[u]) & 0xffff], 1);
+                const int slot = atomicAdd(&cur[bin], 1);
+                if (slot >= nfiled) {  // more records of a bin than counted: corrupt bucket
+                    s_fail = 1;
+                    continue;
+                }
                 rec_c[slot] = make_uint2(id | (static_cast<uint32_t>(r[u]) & 0xffff0000u), static_cast<uint32_t>(r[u] >> 32));
             }
         }
