@@ -299,3 +299,48 @@ def test_backward_stages_equal_backward():
     # summation noise where the sum cancels to almost nothing.
     a, b = to_f64(gv), to_f64(gv_ref)
     assert np.all(np.abs(a - b) <= 2.0 ** -7 * np.maximum(np.abs(a), np.abs(b)) + 2.0 ** -20 * np.abs(b).max())
+
+
+def test_backward_value_twice_on_one_workspace():
+    """The grad_value stage only reads the workspace: calling it twice after one
+    grad_offset_mask stage gives the same gradient (up to the summation order
+    within a cell)."""
+    import torch
+    import deformable_convolution_sampling_b200 as dcn
+    w = gen.WORKLOADS["stage1_f16"]
+    w = gen.custom(**{**w.__dict__, "N": 4, "name": "twice"})
+    inp = gen.make_inputs(w)
+    p = dcn.make_params(dtype=w.dtype, **w.geometry())
+    v, om, gy = (to_device(inp[k], w.dtype) for k in ("value", "offset_mask", "grad_out"))
+    nbytes = dcn.dcn4_backward_workspace_size(p)
+    ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    gom = torch.empty_like(om)
+    s = torch.cuda.current_stream().cuda_stream
+    dcn.check(dcn.dcn4_backward_offset_mask(p, v.data_ptr(), om.data_ptr(), gy.data_ptr(), gom.data_ptr(),
+                                            ws.data_ptr(), nbytes, s))
+    out = []
+    for _ in range(2):
+        gv = torch.full_like(v, float("nan"))
+        dcn.check(dcn.dcn4_backward_value(p, om.data_ptr(), gy.data_ptr(), gv.data_ptr(), ws.data_ptr(), nbytes, s))
+        out.append(gv)
+    torch.cuda.synchronize()
+    a, b = to_f64(out[0]), to_f64(out[1])
+    assert np.all(np.isfinite(a)) and np.all(np.isfinite(b))
+    assert np.all(np.abs(a - b) <= 2.0 ** -10 * np.maximum(np.abs(a), np.abs(b)) + 2.0 ** -20 * np.abs(b).max())
+
+
+def test_samples_beyond_the_filing_window():
+    """Third-stage-like tiles (16 groups: three rows per grad_value tile) with
+    vertical offsets of up to 20 rows: samples land outside the window of tiles
+    a grad_offset_mask CTA files into, those tiles are marked overflowed, and
+    grad_value rescans their offsets."""
+    w = gen.custom(name="window", N=2, H=48, W=14, G=16, Cg=16, Ho=48, Wo=14, K=9, P=432, dtype="bf16",
+                   offset=("normal", 0.0, 1.0))
+    inp = gen.make_inputs(w)
+    rng = np.random.default_rng(7)
+    body = inp["offset_mask"][..., : w.G * 27].reshape(w.N, w.Ho, w.Wo, w.G, 27)
+    dy = rng.uniform(-20.0, 20.0, size=body[..., 1:18:2].shape)
+    body[..., 1:18:2] = gen.to_storage(dy, w.dtype)
+    inp["offset_mask"][..., : w.G * 27] = body.reshape(w.N, w.Ho, w.Wo, w.G * 27)
+    _check_forward(w, inp)
+    _check_backward(w, inp)
