@@ -101,7 +101,9 @@ int make_geometry(const dcn4_params* p, bool backward, bool wide, dcn4::Geometry
     // Output pixels per CTA: fill kTargetThreads, then shrink until the
     // shared-memory rows fit the default 48 KB (or, for very long rows, the
     // per-CTA maximum).
-    const size_t row_bytes = static_cast<size_t>(p->P) * eb * (backward ? 2 : 1);
+    // Shared memory per output pixel: two offset_mask rows (forward: a double
+    // buffer; backward: offset_mask and grad_offset_mask rows).
+    const size_t row_bytes = static_cast<size_t>(p->P) * eb * 2;
     long long ppc = kTargetThreads / lanes_pp;
     while (ppc > 1 && ppc * row_bytes > kSmemDefault) --ppc;
     if (ppc * row_bytes > kSmemMax) return fail(DCN4_ERR_UNSUPPORTED, "P=%d rows do not fit shared memory", p->P);

@@ -18,6 +18,9 @@
 // lines) and accumulates in fp32 with packed f32x2 FMAs: the coefficient reuse
 // and vector loads of section 2.2 ("消除冗余工作量", "消除冗余内存指令").
 // Nothing is written but the output, with 256-bit stores.
+#include <algorithm>
+#include <atomic>
+
 #include "dcn4_common.cuh"
 
 namespace dcn4 {
@@ -44,76 +47,141 @@ __device__ __forceinline__ void accumulate(float2* acc, const T* src, float wt) 
     }
 }
 
+// CTAs per SM the forward kernel is compiled for (80 registers a thread).
+constexpr int kFwdCtasPerSm = 3;
+
+// SM count of the current device, queried once per device.
+cudaError_t sm_count(int* out) {
+    static std::atomic<int> cached[64];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < 64) {
+        const int c = cached[dev].load(std::memory_order_relaxed);
+        if (c > 0) {
+            *out = c;
+            return cudaSuccess;
+        }
+    }
+    int sms = 0;
+    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < 64) cached[dev].store(sms, std::memory_order_relaxed);
+    *out = sms;
+    return cudaSuccess;
+}
+
+__device__ __forceinline__ Tile tile_at(const Geometry& g, int idx) {
+    const int per_img = g.tiles_h * g.tiles_w;
+    Tile t;
+    t.n = idx / per_img;
+    const int r = idx - t.n * per_img;
+    const int ty = r / g.tiles_w;
+    const int tx = r - ty * g.tiles_w;
+    t.ho0 = ty * g.TH;
+    t.wo0 = tx * g.TW;
+    t.th = min(g.TH, g.Ho - t.ho0);
+    t.tw = min(g.TW, g.Wo - t.wo0);
+    return t;
+}
+
+// The tile's offset_mask rows into shared memory [TH][TW][P] with cp.async (16 bytes per thread per step).
+template <typename T>
+__device__ __forceinline__ void stage_tile_async(T* dst_smem, const T* src, const Geometry& g, const Tile& t) {
+    const int row_chunks = t.tw * g.P * static_cast<int>(sizeof(T)) / 16;
+    const int total = t.th * row_chunks;
+    for (int i = threadIdx.x; i < total; i += blockDim.x) {
+        const int r = i / row_chunks;
+        const int c = i - r * row_chunks;
+        const long long grow = (static_cast<long long>(t.n) * g.Ho + t.ho0 + r) * g.Wo + t.wo0;
+        const char* sp = reinterpret_cast<const char*>(src + grow * g.P) + 16ll * c;
+        char* d = reinterpret_cast<char*>(dst_smem + r * g.TW * g.P) + 16 * c;
+        const unsigned da = static_cast<unsigned>(__cvta_generic_to_shared(d));
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(da), "l"(sp));
+    }
+    asm volatile("cp.async.commit_group;");
+}
+
+// Persistent: a CTA per resident slot loops over the output tiles (tile,
+// tile + gridDim.x, ...), copying the next tile's offset_mask rows into the
+// other half of a double buffer (cp.async) while it computes the current one.
 // KH, KW > 0: compile-time grid size (fully unrolled) and RC = remove_center;
 // KH = KW = 0: sizes and remove_center from g.
 template <typename T, int VEC, int KH, int KW, bool RC>
-#ifndef DCN4_FWD_MIN_BLOCKS
-#define DCN4_FWD_MIN_BLOCKS 3
-#endif
-__global__ void __launch_bounds__(256, DCN4_FWD_MIN_BLOCKS) forward_kernel(const Geometry g, const T* __restrict__ value,
+__global__ void __launch_bounds__(256, kFwdCtasPerSm) forward_kernel(const Geometry g, const T* __restrict__ value,
                                                       const T* __restrict__ om, T* __restrict__ out) {
     extern __shared__ __align__(16) unsigned char smem[];
     constexpr int EPV = Elem<T>::per16;
     constexpr int PAIRS = VEC * EPV / 2;
-    T* om_s = reinterpret_cast<T*>(smem);
+    const int tile_elems = g.TH * g.TW * g.P;
+    T* bufs[2] = {reinterpret_cast<T*>(smem), reinterpret_cast<T*>(smem) + tile_elems};
+    const int ntiles = g.N * g.tiles_h * g.tiles_w;
+    int tile = blockIdx.x;
+    if (tile >= ntiles) return;
+    stage_tile_async(bufs[0], om, g, tile_at(g, tile));
 
-    const Tile t = tile_of_block(g);
-    stage_tile_rows(om_s, om, g, t);
-    __syncthreads();
-
-    // Thread -> (pixel of the tile, group, slice); the groups of one pixel are
-    // adjacent lanes, so their corner slices sit at distinct offsets of a line.
     const int lanes_pp = g.G * g.nslice;
     const int lp = threadIdx.x / lanes_pp;
     const int py = lp / g.TW;
     const int px = lp - py * g.TW;
-    if (py >= t.th || px >= t.tw) return;
     const int r = threadIdx.x - lp * lanes_pp;
     const int grp = r / g.nslice;
     const int sl = r - grp * g.nslice;
-    const int ho = t.ho0 + py, wo = t.wo0 + px;
-
     const int K = KH > 0 ? KH * KW - (RC ? 1 : 0) : g.K;
     const int kh = KH > 0 ? KH : g.kh;
     const int kw = KW > 0 ? KW : g.kw;
     const bool rc = KH > 0 ? RC : g.remove_center != 0;
-    const T* row = om_s + lp * g.P + grp * 3 * K;
     const int ch_off = grp * g.Cg + sl * (VEC * EPV);
-    const T* img = value + static_cast<long long>(t.n) * g.H * g.W * g.C + ch_off;
-    const int hb = ho * g.sh - g.ph, wb = wo * g.sw - g.pw;
 
-    float2 acc[PAIRS];
-#pragma unroll
-    for (int i = 0; i < PAIRS; ++i) acc[i] = make_float2(0.f, 0.f);
-
-    int k = 0;
-#pragma unroll
-    for (int iw = 0; iw < kw; ++iw) {
-        const float wbase = static_cast<float>(wb + iw * g.dw);
-#pragma unroll
-        for (int ih = 0; ih < kh; ++ih) {
-            if (rc && iw == kw / 2 && ih == kh / 2) continue;
-            const float dx = to_f32(row[2 * k]);
-            const float dy = to_f32(row[2 * k + 1]);
-            const float m = to_f32(row[2 * K + k]);
-            ++k;
-            const float h = __fmaf_rn(g.s, dy, static_cast<float>(hb + ih * g.dh));
-            const float w = __fmaf_rn(g.s, dx, wbase);
-            const Cell<T> cell = bilinear_cell(g, img, h, w);
-            const float b = m * cell.lh, a = m - b;  // m (1 - lh), m lh
-            const float wl = 1.f - cell.lw;
-            accumulate<T, VEC>(acc, cell.c[0], a * wl);
-            accumulate<T, VEC>(acc, cell.c[1], a * cell.lw);
-            accumulate<T, VEC>(acc, cell.c[2], b * wl);
-            accumulate<T, VEC>(acc, cell.c[3], b * cell.lw);
+    for (int it = 0; tile < ntiles; ++it, tile += gridDim.x) {
+        const int next = tile + gridDim.x;
+        if (next < ntiles) {
+            stage_tile_async(bufs[(it + 1) & 1], om, g, tile_at(g, next));
+            asm volatile("cp.async.wait_group 1;" ::: "memory");
+        } else {
+            asm volatile("cp.async.wait_group 0;" ::: "memory");
         }
-    }
-
-    T* dst = out + ((static_cast<long long>(t.n) * g.Ho + ho) * g.Wo + wo) * g.C + ch_off;
-    if constexpr (VEC == 2) {
-        st_global32(dst, pack(acc, T()), pack(acc + EPV / 2, T()));
-    } else {
-        st_global(dst, pack(acc, T()));
+        __syncthreads();
+        const Tile t = tile_at(g, tile);
+        const T* om_s = bufs[it & 1];
+        if (py < t.th && px < t.tw) {
+            const int ho = t.ho0 + py, wo = t.wo0 + px;
+            const T* row = om_s + lp * g.P + grp * 3 * K;
+            const T* img = value + static_cast<long long>(t.n) * g.H * g.W * g.C + ch_off;
+            const int hb = ho * g.sh - g.ph, wb = wo * g.sw - g.pw;
+            float2 acc[PAIRS];
+#pragma unroll
+            for (int i = 0; i < PAIRS; ++i) acc[i] = make_float2(0.f, 0.f);
+            int k = 0;
+#pragma unroll
+            for (int iw = 0; iw < kw; ++iw) {
+                const float wbase = static_cast<float>(wb + iw * g.dw);
+#pragma unroll
+                for (int ih = 0; ih < kh; ++ih) {
+                    if (rc && iw == kw / 2 && ih == kh / 2) continue;
+                    const float dx = to_f32(row[2 * k]);
+                    const float dy = to_f32(row[2 * k + 1]);
+                    const float m = to_f32(row[2 * K + k]);
+                    ++k;
+                    const float h = __fmaf_rn(g.s, dy, static_cast<float>(hb + ih * g.dh));
+                    const float w = __fmaf_rn(g.s, dx, wbase);
+                    const Cell<T> cell = bilinear_cell(g, img, h, w);
+                    const float b = m * cell.lh, a = m - b;
+                    const float wl = 1.f - cell.lw;
+                    accumulate<T, VEC>(acc, cell.c[0], a * wl);
+                    accumulate<T, VEC>(acc, cell.c[1], a * cell.lw);
+                    accumulate<T, VEC>(acc, cell.c[2], b * wl);
+                    accumulate<T, VEC>(acc, cell.c[3], b * cell.lw);
+                }
+            }
+            T* dst = out + ((static_cast<long long>(t.n) * g.Ho + ho) * g.Wo + wo) * g.C + ch_off;
+            if constexpr (VEC == 2) {
+                st_global32(dst, pack(acc, T()), pack(acc + EPV / 2, T()));
+            } else {
+                st_global(dst, pack(acc, T()));
+            }
+        }
+        __syncthreads();  // the buffer is refilled two tiles later
     }
 }
 
@@ -121,12 +189,18 @@ template <typename T, int VEC, int KH, int KW, bool RC>
 cudaError_t launch_typed(const Geometry& g, const void* value, const void* om, void* out, cudaStream_t stream) {
     const size_t smem = forward_smem_bytes(g, sizeof(T));
     auto kern = forward_kernel<T, VEC, KH, KW, RC>;
-    if (smem > 48 * 1024) {
-        const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-        if (e != cudaSuccess) return e;
-    }
-    const long long blocks = static_cast<long long>(g.N) * g.tiles_h * g.tiles_w;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
     const int threads = (g.pix_per_cta * g.G * g.nslice + 31) / 32 * 32;
+    int sms = 0;
+    e = sm_count(&sms);
+    if (e != cudaSuccess) return e;
+    // One CTA per resident slot (kFwdCtasPerSm by registers, fewer if the double
+    // buffer limits shared memory); each loops over tiles.
+    const long long by_smem = static_cast<long long>(227 * 1024) / static_cast<long long>(smem + 1024);
+    const long long per_sm = std::max<long long>(1, std::min<long long>(kFwdCtasPerSm, by_smem));
+    const long long ntiles = static_cast<long long>(g.N) * g.tiles_h * g.tiles_w;
+    const long long blocks = std::min<long long>(ntiles, per_sm * sms);
     kern<<<static_cast<unsigned>(blocks), threads, smem, stream>>>(g, static_cast<const T*>(value),
                                                                    static_cast<const T*>(om), static_cast<T*>(out));
     return cudaGetLastError();
@@ -149,7 +223,7 @@ cudaError_t launch_vec(const Geometry& g, int vec, const void* value, const void
 }  // namespace
 
 size_t forward_smem_bytes(const Geometry& g, int elem_bytes) {
-    return static_cast<size_t>(g.pix_per_cta) * g.P * elem_bytes;
+    return 2 * static_cast<size_t>(g.pix_per_cta) * g.P * elem_bytes;  // double buffer
 }
 
 cudaError_t launch_forward(const Geometry& g, int dtype, const void* value, const void* om, void* out,
