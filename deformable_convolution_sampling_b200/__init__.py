@@ -224,3 +224,90 @@ def backward(p: dcn4_params, value, offset_mask, grad_out, grad_value=None, grad
                         grad_value.data_ptr(), grad_offset_mask.data_ptr(), ws_ptr, ws_bytes,
                         _stream_handle(value.device)))
     return grad_value, grad_offset_mask
+
+
+# ---------------------------------------------------------------------------
+# torch.autograd wrapper (argument marshalling only: both passes run in libdcn4)
+# ---------------------------------------------------------------------------
+
+_TORCH_CODES = None
+
+
+def _dtype_code(t) -> int:
+    import torch
+    global _TORCH_CODES
+    if _TORCH_CODES is None:
+        _TORCH_CODES = {torch.float32: DCN4_F32, torch.float16: DCN4_F16, torch.bfloat16: DCN4_BF16}
+    if t.dtype not in _TORCH_CODES:
+        raise ValueError(f"dtype {t.dtype} is not float32, float16 or bfloat16")
+    return _TORCH_CODES[t.dtype]
+
+
+def _pair(v):
+    return (v, v) if isinstance(v, int) else tuple(v)
+
+
+def params_for_tensors(value, offset_mask, *, group: int, kernel=3, stride=1, pad=1, dilation=1,
+                       offset_scale: float = 1.0, remove_center: bool = False) -> dcn4_params:
+    """dcn4_params for NHWC value [N,H,W,C] and offset_mask [N,Ho,Wo,P]; checks shapes,
+    dtypes, devices and contiguity on the host (ValueError) before anything is launched."""
+    if value.dim() != 4 or offset_mask.dim() != 4:
+        raise ValueError("value must be [N,H,W,C] and offset_mask [N,Ho,Wo,P]")
+    if value.dtype != offset_mask.dtype:
+        raise ValueError("value and offset_mask must have the same dtype")
+    if not (value.is_contiguous() and offset_mask.is_contiguous()):
+        raise ValueError("value and offset_mask must be contiguous (channels last)")
+    N, H, W, C = value.shape
+    if group < 1 or C % group != 0:
+        raise ValueError(f"C={C} is not a multiple of group={group}")
+    if not (value.is_cuda and offset_mask.is_cuda):
+        raise ValueError("value and offset_mask must be CUDA tensors")
+    if value.device != offset_mask.device:
+        raise ValueError("value and offset_mask must be on the same device")
+    (kh, kw), (sh, sw), (ph, pw), (dh, dw) = _pair(kernel), _pair(stride), _pair(pad), _pair(dilation)
+    p = make_params(N=N, H=H, W=W, G=group, Cg=C // group, kh=kh, kw=kw, sh=sh, sw=sw, ph=ph, pw=pw, dh=dh,
+                    dw=dw, offset_scale=float(offset_scale), remove_center=int(bool(remove_center)),
+                    P=offset_mask.shape[-1], dtype={DCN4_F32: "f32", DCN4_F16: "f16", DCN4_BF16: "bf16"}[_dtype_code(value)])
+    st, Ho, Wo = dcn4_output_dims(p)
+    check(st)
+    if tuple(offset_mask.shape[:3]) != (N, Ho, Wo):
+        raise ValueError(f"offset_mask must be [N={N}, Ho={Ho}, Wo={Wo}, P], got {tuple(offset_mask.shape)}")
+    check(dcn4_check_params(p))
+    return p
+
+
+def _autograd_function():
+    import torch
+
+    class DCNv4Core(torch.autograd.Function):
+        """The DCNv4 core aggregation as a torch.autograd.Function: forward and backward
+        are dcn4_forward and dcn4_backward on the tensors' device and current stream."""
+
+        @staticmethod
+        def forward(ctx, value, offset_mask, p):
+            ctx.save_for_backward(value, offset_mask)
+            ctx.p = p
+            return forward(p, value, offset_mask)
+
+        @staticmethod
+        def backward(ctx, grad_out):
+            value, offset_mask = ctx.saved_tensors
+            grad_value, grad_offset_mask = backward(ctx.p, value, offset_mask, grad_out.contiguous())
+            return grad_value, grad_offset_mask, None
+
+    return DCNv4Core
+
+
+_DCNV4_CORE = None
+
+
+def dcnv4_core(value, offset_mask, *, group: int, kernel=3, stride=1, pad=1, dilation=1,
+               offset_scale: float = 1.0, remove_center: bool = False):
+    """y = DCNv4 core aggregation of value [N,H,W,C] at the offsets and masks of
+    offset_mask [N,Ho,Wo,P], differentiable in both (torch.autograd)."""
+    global _DCNV4_CORE
+    p = params_for_tensors(value, offset_mask, group=group, kernel=kernel, stride=stride, pad=pad,
+                           dilation=dilation, offset_scale=offset_scale, remove_center=remove_center)
+    if _DCNV4_CORE is None:
+        _DCNV4_CORE = _autograd_function()
+    return _DCNV4_CORE.apply(value, offset_mask, p)
