@@ -35,6 +35,7 @@ class _Problem(ctypes.Structure):
         ("P", ctypes.c_int),
         ("dtype", ctypes.c_int),
         ("location_fp32", ctypes.c_int),
+        ("softmax", ctypes.c_int),
     ]
 
 
@@ -60,6 +61,7 @@ class Problem:
     P: int | None = None          # None: the smallest multiple of 8 >= G*3K
     dtype: str = "f64"
     location_fp32: bool = False
+    softmax: bool = False         # DCNv3 variant: the masks are logits, softmax over k
 
     @property
     def K(self) -> int:
@@ -80,7 +82,7 @@ class Problem:
             self.N, self.H, self.W, self.G, self.Cg, self.kh, self.kw, self.sh, self.sw,
             self.ph, self.pw, self.dh, self.dw, float(self.offset_scale),
             1 if self.remove_center else 0, self.row, DTYPES[self.dtype],
-            1 if self.location_fp32 else 0,
+            1 if self.location_fp32 else 0, 1 if self.softmax else 0,
         )
 
 

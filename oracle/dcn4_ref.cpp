@@ -6,6 +6,7 @@
 // reordering.  Accumulation is in double.
 #include "dcn4_ref.h"
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -195,6 +196,24 @@ int ref_num_points(const ref_problem* p) {
     return p->kh * p->kw - (p->remove_center ? 1 : 0);
 }
 
+// The weights of the K points of one (pixel, group): the masks, or (softmax
+// variant) their softmax over k, exp(m_k - max) / sum_j exp(m_j - max).
+std::vector<double> point_weights(const ref_problem* p, const void* offset_mask, int64_t om, int K) {
+    std::vector<double> a(K);
+    for (int k = 0; k < K; ++k) a[k] = load(offset_mask, p->dtype, om + 2 * K + k);
+    if (p->softmax) {
+        double mx = a[0];
+        for (int k = 1; k < K; ++k) mx = std::max(mx, a[k]);
+        double sum = 0.0;
+        for (int k = 0; k < K; ++k) {
+            a[k] = std::exp(a[k] - mx);
+            sum += a[k];
+        }
+        for (int k = 0; k < K; ++k) a[k] /= sum;
+    }
+    return a;
+}
+
 void ref_decode(int dtype, const void* src, double* dst, int64_t n) {
     for (int64_t i = 0; i < n; ++i) dst[i] = load(src, dtype, i);
 }
@@ -215,12 +234,13 @@ int ref_forward(const ref_problem* p, const void* value, const void* offset_mask
             const int64_t pix = (static_cast<int64_t>(n) * Ho + ho) * Wo + wo;
             for (int g = 0; g < p->G; ++g) {
                 const int64_t om = pix * p->P + static_cast<int64_t>(g) * 3 * K;
+                const std::vector<double> a = point_weights(p, offset_mask, om, K);
                 for (int c = 0; c < p->Cg; ++c) {
                     double y = 0.0;
                     for (int k = 0; k < K; ++k) {
                         const double dx = load(offset_mask, p->dtype, om + 2 * k);
                         const double dy = load(offset_mask, p->dtype, om + 2 * k + 1);
-                        const double m = load(offset_mask, p->dtype, om + 2 * K + k);
+                        const double m = a[k];
                         double h, w;
                         sample_location(p, ho, wo, cells[k], dx, dy, &h, &w);
                         const Bilinear b = bilinear_cell(p, h, w);
@@ -259,14 +279,16 @@ int ref_backward(const ref_problem* p, const void* value, const void* offset_mas
                 for (int e = 0; e < p->P; ++e) gom[e] = 0.0;  // includes the padding tail
                 for (int g = 0; g < p->G; ++g) {
                     const int64_t om = pix * p->P + static_cast<int64_t>(g) * 3 * K;
+                    const std::vector<double> a = point_weights(p, offset_mask, om, K);
+                    std::vector<double> gw(K, 0.0);  // d loss / d (weight of point k) = <gy, S_k>
                     for (int k = 0; k < K; ++k) {
                         const double dx = load(offset_mask, p->dtype, om + 2 * k);
                         const double dy = load(offset_mask, p->dtype, om + 2 * k + 1);
-                        const double m = load(offset_mask, p->dtype, om + 2 * K + k);
+                        const double m = a[k];
                         double h, w;
                         sample_location(p, ho, wo, cells[k], dx, dy, &h, &w);
                         const Bilinear b = bilinear_cell(p, h, w);
-                        if (!b.any) continue;  // no pixel touched: all three gradients are 0
+                        if (!b.any) continue;  // no pixel touched: S_k = 0, offset gradients 0
                         // Corner values v_ab and the upstream gradient gy, per channel.
                         double gmask = 0.0, gdw = 0.0, gdh = 0.0;
                         for (int c = 0; c < p->Cg; ++c) {
@@ -299,8 +321,15 @@ int ref_backward(const ref_problem* p, const void* value, const void* offset_mas
                         // location = base + s * offset, so d/d offset = s * m * dS/d location.
                         gom[static_cast<int64_t>(g) * 3 * K + 2 * k] = s * m * gdw;
                         gom[static_cast<int64_t>(g) * 3 * K + 2 * k + 1] = s * m * gdh;
-                        gom[static_cast<int64_t>(g) * 3 * K + 2 * K + k] = gmask;
+                        gw[k] = gmask;
                     }
+                    // Mask gradient: the weight gradient itself, or through the softmax,
+                    // d/d m_j = a_j * (gw_j - sum_k a_k gw_k).
+                    double dot = 0.0;
+                    if (p->softmax)
+                        for (int k = 0; k < K; ++k) dot += a[k] * gw[k];
+                    for (int k = 0; k < K; ++k)
+                        gom[static_cast<int64_t>(g) * 3 * K + 2 * K + k] = p->softmax ? a[k] * (gw[k] - dot) : gw[k];
                 }
             }
         }

@@ -41,6 +41,14 @@
  * which bilinear cell a sample falls in — and all later arithmetic stays in
  * double.  Otherwise the location is formed in double.
  *
+ * Softmax variant (softmax != 0): the K masks of each (pixel, group) are
+ * logits, normalised over k before they weigh the samples,
+ *     m_gk -> exp(m_gk) / sum_j exp(m_gj)
+ * — the DCNv3 aggregation the CSDN summary's section 1.2 equation gives, which
+ * DCNv4 drops (section 2.1); the reference extension keeps it as a `softmax`
+ * flag (mhpn.cn page, dcnv4_cuda_forward signature).  The exponentials are
+ * taken after subtracting the largest logit (same value, no overflow).
+ *
  * Element storage: REF_F32, REF_F16 (IEEE binary16), REF_BF16 (upper half of an
  * IEEE binary32) and REF_F64 (for finite-difference tests).  Every element is
  * decoded exactly into a double by this file's own bit-level decoders.
@@ -69,6 +77,7 @@ typedef struct {
     int P;                /* row length of offset_mask, >= G*3K                */
     int dtype;            /* REF_* storage type of value/offset_mask/grad_out  */
     int location_fp32;    /* 1: form the sampling location with an fp32 fma    */
+    int softmax;          /* 1: the masks are logits, normalised over k        */
 } ref_problem;
 
 /* Output size of the grid: Ho = (H + 2ph - (dh*(kh-1)+1)) / sh + 1 (floor).

@@ -14,8 +14,8 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 SRC = os.path.join(ROOT, "oracle", "dcn4_ref.cpp")
 
 MUTATIONS = {
-    "dx_dy_swapped": ("const double dx = load(offset_mask, p->dtype, om + 2 * k);\n                        const double dy = load(offset_mask, p->dtype, om + 2 * k + 1);\n                        const double m = load(offset_mask, p->dtype, om + 2 * K + k);\n                        double h, w;\n                        sample_location(p, ho, wo, cells[k], dx, dy, &h, &w);\n                        const Bilinear b = bilinear_cell(p, h, w);\n                        y +=",
-                      "const double dy = load(offset_mask, p->dtype, om + 2 * k);\n                        const double dx = load(offset_mask, p->dtype, om + 2 * k + 1);\n                        const double m = load(offset_mask, p->dtype, om + 2 * K + k);\n                        double h, w;\n                        sample_location(p, ho, wo, cells[k], dx, dy, &h, &w);\n                        const Bilinear b = bilinear_cell(p, h, w);\n                        y +="),
+    "dx_dy_swapped": ("const double dx = load(offset_mask, p->dtype, om + 2 * k);\n                        const double dy = load(offset_mask, p->dtype, om + 2 * k + 1);\n                        const double m = a[k];\n                        double h, w;\n                        sample_location(p, ho, wo, cells[k], dx, dy, &h, &w);\n                        const Bilinear b = bilinear_cell(p, h, w);\n                        y +=",
+                      "const double dy = load(offset_mask, p->dtype, om + 2 * k);\n                        const double dx = load(offset_mask, p->dtype, om + 2 * k + 1);\n                        const double m = a[k];\n                        double h, w;\n                        sample_location(p, ho, wo, cells[k], dx, dy, &h, &w);\n                        const Bilinear b = bilinear_cell(p, h, w);\n                        y +="),
     "k_order_row_major": ("for (int iw = 0; iw < p->kw; ++iw) {\n        for (int ih = 0; ih < p->kh; ++ih) {",
                           "for (int ih = 0; ih < p->kh; ++ih) {\n        for (int iw = 0; iw < p->kw; ++iw) {"),
     "corner_dropped": ("for (int bb = 0; bb < 2; ++bb) {\n            const int y = b.h0 + a;",
@@ -30,6 +30,12 @@ MUTATIONS = {
     "stride_ignored": ("const int base_w = wo * p->sw - p->pw + c.iw * p->dw;",
                        "const int base_w = wo - p->pw + c.iw * p->dw;"),
     "bilinear_ceil_cell": ("const double fh = std::floor(h);", "const double fh = std::ceil(h) - 1.0;"),
+    # softmax variant
+    "softmax_not_normalised": ("for (int k = 0; k < K; ++k) a[k] /= sum;", ""),
+    "softmax_largest_not_subtracted": ("a[k] = std::exp(a[k] - mx);", "a[k] = std::exp(a[k]);"),
+    "softmax_jacobian_without_sum": ("p->softmax ? a[k] * (gw[k] - dot) : gw[k]", "p->softmax ? a[k] * gw[k] : gw[k]"),
+    "softmax_ignored_in_backward_offsets": ("const double m = a[k];\n                        double h, w;\n                        sample_location(p, ho, wo, cells[k], dx, dy, &h, &w);\n                        const Bilinear b = bilinear_cell(p, h, w);\n                        if (!b.any) continue;",
+                                            "const double m = load(offset_mask, p->dtype, om + 2 * K + k);\n                        double h, w;\n                        sample_location(p, ho, wo, cells[k], dx, dy, &h, &w);\n                        const Bilinear b = bilinear_cell(p, h, w);\n                        if (!b.any) continue;"),
 }
 
 

@@ -17,6 +17,8 @@ DCNv4 module signature on the mhpn.cn architecture page.
 """
 import math
 
+import dataclasses
+
 import numpy as np
 import pytest
 import torch
@@ -491,3 +493,111 @@ def test_grad_offset_zero_offsets_at_border_uses_floor_cell():
     # k = 4 is the centre (1, 1): location (0, 0): dS/dh = v[1,0]-v[0,0] = 4, dS/dw = v[0,1]-v[0,0] = 1
     assert dyg[0, 0, 0, 0, 4] == 4.0 and dxg[0, 0, 0, 0, 4] == 1.0
     assert math.isfinite(float(np.sum(gom)))
+
+
+# ---------------------------------------------------------------------------
+# Softmax variant (DCNv3 normalisation of the K masks of each (pixel, group))
+# ---------------------------------------------------------------------------
+
+def _softmax_problem(**kw):
+    return oracle.Problem(**{**dict(N=2, H=7, W=9, G=2, Cg=3, dtype="f64"), **kw})
+
+
+def _set_logits(om, prob, fn):
+    """Replace the masks of every (pixel, group) by fn(shape) (in place)."""
+    _, _, m = split_om(om, prob.G, prob.K)
+    m[...] = fn(m.shape)
+    return om
+
+
+def test_softmax_shift_invariance():
+    """Adding one constant to the K logits of a (pixel, group) changes nothing."""
+    prob = _softmax_problem(softmax=True)
+    inp, Ho, Wo = rand_problem_inputs(prob, seed=41)
+    om = inp["offset_mask"].copy()
+    y0 = oracle.forward(prob, inp["value"], om)
+    _, _, m = split_om(om, prob.G, prob.K)
+    m += np.random.default_rng(5).uniform(-30, 30, size=m.shape[:-1] + (1,))
+    y1 = oracle.forward(prob, inp["value"], om)
+    assert rel_err(y1, y0) < 1e-12
+
+
+def test_softmax_equal_logits_average_the_points():
+    """Equal logits weigh every point 1/K: the plain operator with mask 1/K."""
+    prob = _softmax_problem(softmax=True, remove_center=1)
+    inp, Ho, Wo = rand_problem_inputs(prob, seed=42)
+    om_sm = _set_logits(inp["offset_mask"].copy(), prob,
+                        lambda sh: np.repeat(np.random.default_rng(6).normal(size=sh[:-1] + (1,)), sh[-1], -1))
+    om_plain = _set_logits(inp["offset_mask"].copy(), prob, lambda sh: np.full(sh, 1.0 / prob.K))
+    y_sm = oracle.forward(prob, inp["value"], om_sm)
+    y_plain = oracle.forward(dataclasses.replace(prob, softmax=False), inp["value"], om_plain)
+    assert rel_err(y_sm, y_plain) < 1e-13
+
+
+def test_softmax_dominant_logit_selects_its_point():
+    """Logits +800 at point j and -800 elsewhere weigh point j by exactly 1 (this
+    also needs the largest logit subtracted before exp, or exp overflows)."""
+    prob = _softmax_problem(softmax=True)
+    inp, Ho, Wo = rand_problem_inputs(prob, seed=43)
+    rng = np.random.default_rng(7)
+    j = rng.integers(0, prob.K, size=(prob.N, Ho, Wo, prob.G))
+    onehot = np.eye(prob.K)[j]
+    om_sm = _set_logits(inp["offset_mask"].copy(), prob, lambda sh: 1600.0 * onehot - 800.0)
+    om_plain = _set_logits(inp["offset_mask"].copy(), prob, lambda sh: onehot)
+    y_sm = oracle.forward(prob, inp["value"], om_sm)
+    y_plain = oracle.forward(dataclasses.replace(prob, softmax=False), inp["value"], om_plain)
+    assert np.all(np.isfinite(y_sm))
+    assert rel_err(y_sm, y_plain) < 1e-15
+
+
+def test_softmax_logit_gradients_sum_to_zero():
+    """The softmax is invariant to a common shift, so the logit gradients of each
+    (pixel, group) sum to zero, while the samples' own gradients do not."""
+    prob = _softmax_problem(softmax=True)
+    inp, Ho, Wo = rand_problem_inputs(prob, seed=44)
+    _, gom = oracle.backward(prob, inp["value"], inp["offset_mask"], inp["grad_out"])
+    _, _, gm = split_om(gom, prob.G, prob.K)
+    scale = np.max(np.abs(gm))
+    assert scale > 1e-3
+    assert np.max(np.abs(gm.sum(-1))) < 1e-12 * scale * prob.K
+
+
+@pytest.mark.parametrize("remove_center", [0, 1])
+def test_softmax_backward_finite_differences(remove_center):
+    """Offsets and logits: central differences of the softmax forward."""
+    prob = oracle.Problem(N=1, H=8, W=8, G=2, Cg=4, dtype="f64", softmax=True, remove_center=remove_center,
+                          offset_scale=0.7)
+    inp, Ho, Wo = rand_problem_inputs(prob, seed=45)
+    om = inp["offset_mask"].copy()
+    om[..., prob.G * 3 * prob.K:] = 0.0
+    dx, dy, _ = split_om(om, prob.G, prob.K)
+    for d in (dx, dy):
+        frac = np.mod(prob.offset_scale * d, 1.0)
+        bad = (frac < 1e-3) | (frac > 1 - 1e-3)
+        d[bad] += 0.01
+    gy = inp["grad_out"]
+    _, gom = oracle.backward(prob, inp["value"], om, gy)
+    eps = 1e-6
+    G, K, Cg = prob.G, prob.K, prob.Cg
+    body = G * 3 * K
+    scale_ref = max(np.max(np.abs(gom[..., :body])), 1e-12)
+    for e in range(3 * K):
+        plus, minus = om.copy(), om.copy()
+        idx = np.arange(G) * 3 * K + e
+        plus[..., idx] += eps
+        minus[..., idx] -= eps
+        yp = oracle.forward(prob, inp["value"], plus).reshape(1, Ho, Wo, G, Cg)
+        ym = oracle.forward(prob, inp["value"], minus).reshape(1, Ho, Wo, G, Cg)
+        fd = np.sum(gy.reshape(1, Ho, Wo, G, Cg) * (yp - ym), axis=-1) / (2 * eps)
+        assert np.max(np.abs(gom[..., idx] - fd)) / scale_ref < 1e-6, f"entry {e}"
+
+
+def test_softmax_grad_value_is_adjoint():
+    """y is linear in value for fixed offsets and logits: <gy, y(v)> = <grad_value, v>."""
+    prob = _softmax_problem(softmax=True)
+    inp, Ho, Wo = rand_problem_inputs(prob, seed=46)
+    y = oracle.forward(prob, inp["value"], inp["offset_mask"])
+    gv, _ = oracle.backward(prob, inp["value"], inp["offset_mask"], inp["grad_out"])
+    lhs = float(np.sum(inp["grad_out"] * y))
+    rhs = float(np.sum(gv * inp["value"]))
+    assert abs(lhs - rhs) <= 1e-12 * max(abs(lhs), 1.0)
