@@ -157,6 +157,7 @@ class Workload:
     dw: int = 1
     offset_scale: float = 1.0
     remove_center: int = 0
+    softmax: int = 0          # masks are logits normalised over the K points
     seed: int = 0
     passes: str = "fwd"
     note: str = ""
@@ -169,10 +170,11 @@ class Workload:
         """Keyword arguments shared by the oracle's Problem and the library's params."""
         return dict(N=self.N, H=self.H, W=self.W, G=self.G, Cg=self.Cg, kh=self.kh, kw=self.kw,
                     sh=self.sh, sw=self.sw, ph=self.ph, pw=self.pw, dh=self.dh, dw=self.dw,
-                    offset_scale=self.offset_scale, remove_center=self.remove_center, P=self.P)
+                    offset_scale=self.offset_scale, remove_center=self.remove_center, P=self.P,
+                    softmax=self.softmax)
 
     def describe(self) -> str:
-        rc = " remove_center" if self.remove_center else ""
+        rc = (" remove_center" if self.remove_center else "") + (" softmax" if self.softmax else "")
         return (f"N{self.N} H{self.H} W{self.W} C{self.C} G{self.G} (C'={self.Cg}) "
                 f"{self.kh}x{self.kw} s{self.sh} p{self.ph} d{self.dh} K{self.K} P{self.P} "
                 f"offset_scale {self.offset_scale}{rc} {self.dtype}")

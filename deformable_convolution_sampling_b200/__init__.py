@@ -46,18 +46,20 @@ class dcn4_params(ctypes.Structure):
         ("remove_center", ctypes.c_int),
         ("P", ctypes.c_int),
         ("dtype", ctypes.c_int),
+        ("softmax", ctypes.c_int),
     ]
 
 
 def make_params(*, N, H, W, G, Cg, kh=3, kw=3, sh=1, sw=1, ph=1, pw=1, dh=1, dw=1,
-                offset_scale=1.0, remove_center=0, P=None, dtype="f32") -> dcn4_params:
-    """Build a dcn4_params; P defaults to the smallest valid padded row."""
+                offset_scale=1.0, remove_center=0, P=None, dtype="f32", softmax=0) -> dcn4_params:
+    """Build a dcn4_params; P defaults to the smallest valid padded row.  softmax=1
+    normalises the K masks of each (pixel, group) with a softmax (the DCNv3 form)."""
     if isinstance(dtype, str):
         dtype = DTYPE_NAMES[dtype]
     if P is None:
         P = dcn4_padded_offset_dim(G, kh * kw - (1 if remove_center else 0))
     return dcn4_params(N, H, W, G, Cg, kh, kw, sh, sw, ph, pw, dh, dw, float(offset_scale),
-                       1 if remove_center else 0, P, dtype)
+                       1 if remove_center else 0, P, dtype, 1 if softmax else 0)
 
 
 def _load() -> ctypes.CDLL:
@@ -248,7 +250,8 @@ def _pair(v):
 
 
 def params_for_tensors(value, offset_mask, *, group: int, kernel=3, stride=1, pad=1, dilation=1,
-                       offset_scale: float = 1.0, remove_center: bool = False) -> dcn4_params:
+                       offset_scale: float = 1.0, remove_center: bool = False,
+                       softmax: bool = False) -> dcn4_params:
     """dcn4_params for NHWC value [N,H,W,C] and offset_mask [N,Ho,Wo,P]; checks shapes,
     dtypes, devices and contiguity on the host (ValueError) before anything is launched."""
     if value.dim() != 4 or offset_mask.dim() != 4:
@@ -267,7 +270,8 @@ def params_for_tensors(value, offset_mask, *, group: int, kernel=3, stride=1, pa
     (kh, kw), (sh, sw), (ph, pw), (dh, dw) = _pair(kernel), _pair(stride), _pair(pad), _pair(dilation)
     p = make_params(N=N, H=H, W=W, G=group, Cg=C // group, kh=kh, kw=kw, sh=sh, sw=sw, ph=ph, pw=pw, dh=dh,
                     dw=dw, offset_scale=float(offset_scale), remove_center=int(bool(remove_center)),
-                    P=offset_mask.shape[-1], dtype={DCN4_F32: "f32", DCN4_F16: "f16", DCN4_BF16: "bf16"}[_dtype_code(value)])
+                    P=offset_mask.shape[-1], dtype={DCN4_F32: "f32", DCN4_F16: "f16", DCN4_BF16: "bf16"}[_dtype_code(value)],
+                    softmax=int(bool(softmax)))
     st, Ho, Wo = dcn4_output_dims(p)
     check(st)
     if tuple(offset_mask.shape[:3]) != (N, Ho, Wo):
@@ -302,12 +306,14 @@ _DCNV4_CORE = None
 
 
 def dcnv4_core(value, offset_mask, *, group: int, kernel=3, stride=1, pad=1, dilation=1,
-               offset_scale: float = 1.0, remove_center: bool = False):
+               offset_scale: float = 1.0, remove_center: bool = False, softmax: bool = False):
     """y = DCNv4 core aggregation of value [N,H,W,C] at the offsets and masks of
-    offset_mask [N,Ho,Wo,P], differentiable in both (torch.autograd)."""
+    offset_mask [N,Ho,Wo,P], differentiable in both (torch.autograd).  softmax=True
+    takes the masks as logits normalised over the K points (the DCNv3 form)."""
     global _DCNV4_CORE
     p = params_for_tensors(value, offset_mask, group=group, kernel=kernel, stride=stride, pad=pad,
-                           dilation=dilation, offset_scale=offset_scale, remove_center=remove_center)
+                           dilation=dilation, offset_scale=offset_scale, remove_center=remove_center,
+                           softmax=softmax)
     if _DCNV4_CORE is None:
         _DCNV4_CORE = _autograd_function()
     return _DCNV4_CORE.apply(value, offset_mask, p)

@@ -46,6 +46,9 @@ constexpr int kValueMaxGK = 512;   // groups x points at most
 // grad_offset_mask pass: shared memory at most for its offset_mask tiles plus
 // the staging of the records it files (beyond it the grad_value pass rescans).
 constexpr size_t kFileSmem = 96 * 1024;
+// Static shared memory of the grad_offset_mask kernel (per-pixel boxes and the
+// filing counters), an upper bound.
+constexpr size_t kSamplesStaticSmem = 8 * 1024;
 
 // Validates p and fills the kernel geometry.  Touches no GPU state.
 // wide: the gathered and stored tensors are 32-byte aligned, so a thread may
@@ -61,6 +64,7 @@ int make_geometry(const dcn4_params* p, bool backward, bool wide, dcn4::Geometry
         return fail(DCN4_ERR_BAD_SHAPE, "need kernel, stride, dilation >= 1 and padding >= 0");
     if (p->remove_center != 0 && p->remove_center != 1)
         return fail(DCN4_ERR_BAD_SHAPE, "remove_center must be 0 or 1");
+    if (p->softmax != 0 && p->softmax != 1) return fail(DCN4_ERR_BAD_SHAPE, "softmax must be 0 or 1");
     if (p->remove_center && (p->kh % 2 == 0 || p->kw % 2 == 0))
         return fail(DCN4_ERR_BAD_SHAPE, "remove_center needs odd kh and kw");
     if (!std::isfinite(p->offset_scale)) return fail(DCN4_ERR_BAD_SHAPE, "offset_scale is not finite");
@@ -102,8 +106,10 @@ int make_geometry(const dcn4_params* p, bool backward, bool wide, dcn4::Geometry
     // shared-memory rows fit the default 48 KB (or, for very long rows, the
     // per-CTA maximum).
     // Shared memory per output pixel: two offset_mask rows (forward: a double
-    // buffer; backward: offset_mask and grad_offset_mask rows).
-    const size_t row_bytes = static_cast<size_t>(p->P) * eb * 2;
+    // buffer; backward: offset_mask and grad_offset_mask rows), and with softmax
+    // (forward) its threads' fp32 exponentials.
+    const size_t row_bytes = static_cast<size_t>(p->P) * eb * 2 +
+                             (p->softmax ? static_cast<size_t>(K) * lanes_pp * sizeof(float) : 0);
     long long ppc = kTargetThreads / lanes_pp;
     while (ppc > 1 && ppc * row_bytes > kSmemDefault) --ppc;
     if (ppc * row_bytes > kSmemMax) return fail(DCN4_ERR_UNSUPPORTED, "P=%d rows do not fit shared memory", p->P);
@@ -122,6 +128,7 @@ int make_geometry(const dcn4_params* p, bool backward, bool wide, dcn4::Geometry
     g->Ho = static_cast<int>(Ho); g->Wo = static_cast<int>(Wo); g->P = p->P; g->K = K;
     g->kh = p->kh; g->kw = p->kw; g->sh = p->sh; g->sw = p->sw; g->ph = p->ph; g->pw = p->pw;
     g->dh = p->dh; g->dw = p->dw; g->s = p->offset_scale; g->remove_center = p->remove_center;
+    g->softmax = p->softmax;
     g->vec = static_cast<int>(vec);
     g->nslice = static_cast<int>(nslice);
     g->pix_per_cta = static_cast<int>(TH * TW);
@@ -187,6 +194,9 @@ int make_geometry(const dcn4_params* p, bool backward, bool wide, dcn4::Geometry
     if (g->buckets && (dcn4::backward_smem_bytes(*g, eb) > kFileSmem ||
                        static_cast<long long>(K) * dcn4::samples_threads(*g) > (1 << 13)))
         g->buckets = 0;
+    // The grad_offset_mask CTA's dynamic shared memory, next to its static arrays.
+    if (backward && dcn4::backward_smem_bytes(*g, eb) + kSamplesStaticSmem > kSmemMax)
+        return fail(DCN4_ERR_UNSUPPORTED, "the backward's rows of P=%d (K=%d) do not fit shared memory", p->P, K);
     return DCN4_OK;
 }
 

@@ -7,7 +7,11 @@
 //   d/d dx_k  = s * m_k * <gy, dS/dw>,          dS/dw = (1-lh)(v01 - v00) + lh(v11 - v10)
 //   d/d dy_k  = s * m_k * <gy, dS/dh>,          dS/dh = (1-lw)(v10 - v00) + lw(v11 - v01)
 //   grad_value[corner ab] += m_k * w_ab * gy     (every in-image corner)
-// where <.,.> sums over the group's C' channels.
+// where <.,.> sums over the group's C' channels.  With g.softmax the masks
+// are logits l_k and m_k = softmax(l)_k over the K points of the (pixel,
+// group) (the DCNv3 form); m_k then stands for that weight above, and
+//   d/d l_k   = m_k * (<gy, S_k> - sum_j m_j <gy, S_j>)
+// (the softmax Jacobian applied to the gradients of the weights).
 //
 // Two kernels, no atomics on gradient data:
 //
@@ -105,11 +109,38 @@ __device__ __forceinline__ uint16_t cell_code(bool any, int dh, int dw) {
 
 __device__ __forceinline__ uint32_t fix16(float f) { return min(65535u, static_cast<uint32_t>(f * 65536.f + 0.5f)); }
 
+// A softmax weight (in [0, 1]) in the 16 mask bits of a compact record: q / 65535
+// (absolute error below 2^-17, like the bilinear fractions).
+__device__ __forceinline__ uint32_t weight_q16(float a) { return min(65535u, static_cast<uint32_t>(a * 65535.f + 0.5f)); }
+constexpr float kWeightQ16 = 0x1p-32f / 65535.f;  // q16 weight x 2^-32 (the fractions' scale) per unit of q
+
 template <typename T>
 __device__ __forceinline__ uint16_t raw_bits(T x) {
     uint16_t b;
     memcpy(&b, &x, 2);
     return b;
+}
+
+// An fp32 value in the two elements at p (one element for fp32 storage), as
+// raw bits; get_f32 reads it back.
+__device__ __forceinline__ void put_f32(float* p, float v) { *p = v; }
+__device__ __forceinline__ float get_f32(const float* p) { return *p; }
+__device__ __forceinline__ void put_f32(__half* p, float v) {
+    const uint32_t b = __float_as_uint(v);
+    p[0] = __ushort_as_half(static_cast<unsigned short>(b & 0xffffu));
+    p[1] = __ushort_as_half(static_cast<unsigned short>(b >> 16));
+}
+__device__ __forceinline__ float get_f32(const __half* p) {
+    return __uint_as_float(static_cast<uint32_t>(__half_as_ushort(p[0])) | (static_cast<uint32_t>(__half_as_ushort(p[1])) << 16));
+}
+__device__ __forceinline__ void put_f32(__nv_bfloat16* p, float v) {
+    const uint32_t b = __float_as_uint(v);
+    p[0] = __ushort_as_bfloat16(static_cast<unsigned short>(b & 0xffffu));
+    p[1] = __ushort_as_bfloat16(static_cast<unsigned short>(b >> 16));
+}
+__device__ __forceinline__ float get_f32(const __nv_bfloat16* p) {
+    return __uint_as_float(static_cast<uint32_t>(__bfloat16_as_ushort(p[0])) |
+                           (static_cast<uint32_t>(__bfloat16_as_ushort(p[1])) << 16));
 }
 
 // Grid cell (ih, iw) of sampling point k (columns outer, rows inner, centre
@@ -168,7 +199,7 @@ __device__ __forceinline__ int tile_index(const Geometry& g, int n, int ty, int 
 // ---------------------------------------------------------------------------
 // grad_offset_mask + reach
 // ---------------------------------------------------------------------------
-template <typename T, int VEC, int KH, int KW, bool RC>
+template <typename T, int VEC, int KH, int KW, bool RC, bool SM>
 __global__ void __launch_bounds__(256, 3) samples_kernel(const Geometry g, const T* __restrict__ value,
                                                       const T* __restrict__ om, const T* __restrict__ gout,
                                                       T* __restrict__ gom, int* __restrict__ reach,
@@ -182,13 +213,13 @@ __global__ void __launch_bounds__(256, 3) samples_kernel(const Geometry g, const
     const int tile_elems = g.TH * g.TW * g.P;
     T* om_s = reinterpret_cast<T*>(smem);
     T* gom_s = reinterpret_cast<T*>(smem + tile_elems * sizeof(T));  // P % 8 == 0 keeps this 16-byte aligned
+    const bool filing = sizeof(T) == 2 && g.buckets != 0;
 
     const Tile t = tile_of_block(g);
     const int K = KH > 0 ? KH * KW - (RC ? 1 : 0) : g.K;
     const int kh = KH > 0 ? KH : g.kh;
     const int kw = KW > 0 ? KW : g.kw;
     const bool rc = KH > 0 ? RC : g.remove_center != 0;
-    const bool filing = sizeof(T) == 2 && g.buckets != 0;
     FileStage fs;
     if (filing) {
         // staging after the two offset_mask tiles
@@ -237,6 +268,10 @@ __global__ void __launch_bounds__(256, 3) samples_kernel(const Geometry g, const
     const bool writer = active && sl == 0;
     int my_reach = -1;
     int bmin_h = 127, bmax_h = -128, bmin_w = 127, bmax_w = -128;  // cells relative to (hb, wb)
+    constexpr bool smax = SM;  // masks are logits (softmax over the K points)
+    float2 stats = make_float2(0.f, 1.f);  // softmax: (l_max, 1 / sum_k exp(l_k - l_max))
+    if constexpr (SM) stats = softmax_stats(row + 2 * K, K);
+    float gdot = 0.f;  // softmax: sum_k m_k <gy, S_k>
 
     int k = 0;
 #pragma unroll
@@ -249,7 +284,8 @@ __global__ void __launch_bounds__(256, 3) samples_kernel(const Geometry g, const
             const int ah = hb + ih * g.dh;  // anchor row
             const float dx = to_f32(row[2 * kk]);
             const float dy = to_f32(row[2 * kk + 1]);
-            const float m = to_f32(row[2 * K + kk]);
+            float m = to_f32(row[2 * K + kk]);
+            if constexpr (SM) m = softmax_weight(m, stats);
             const float h = active ? __fmaf_rn(g.s, dy, static_cast<float>(ah)) : -2.f;
             const float w = __fmaf_rn(g.s, dx, static_cast<float>(aw));
             const Cell<T> cell = bilinear_cell(g, img, h, w);
@@ -263,6 +299,7 @@ __global__ void __launch_bounds__(256, 3) samples_kernel(const Geometry g, const
                 d10 += __shfl_xor_sync(0xffffffffu, d10, off);
                 d11 += __shfl_xor_sync(0xffffffffu, d11, off);
             }
+            float gw = 0.f;  // <gy, S_k>
             if (cell.any) {
                 if (sl == 0) {
                     const float hl = 1.f - cell.lh, wl = 1.f - cell.lw;
@@ -270,7 +307,8 @@ __global__ void __launch_bounds__(256, 3) samples_kernel(const Geometry g, const
                     T* gr = gom_s + lrow;  // rounded once, to the I/O dtype
                     gr[2 * kk] = from_f32<T>(sm * (hl * (d01 - d00) + cell.lh * (d11 - d10)));
                     gr[2 * kk + 1] = from_f32<T>(sm * (wl * (d10 - d00) + cell.lw * (d11 - d01)));
-                    gr[2 * K + kk] = from_f32<T>(hl * (wl * d00 + cell.lw * d01) + cell.lh * (wl * d10 + cell.lw * d11));
+                    gw = hl * (wl * d00 + cell.lw * d01) + cell.lh * (wl * d10 + cell.lw * d11);
+                    if (!smax) gr[2 * K + kk] = from_f32<T>(gw);
                 }
                 const int dh = max(abs(cell.h0 - ah), abs(cell.h0 + 1 - ah));
                 const int dw = max(abs(cell.w0 - aw), abs(cell.w0 + 1 - aw));
@@ -280,6 +318,11 @@ __global__ void __launch_bounds__(256, 3) samples_kernel(const Geometry g, const
                 bmin_w = min(bmin_w, cell.w0 - wb);
                 bmax_w = max(bmax_w, cell.w0 - wb);
             }
+            if (smax && writer) {
+                // the staged offsets of sample kk are spent: they keep <gy, S_k> (fp32 bits)
+                put_f32(om_s + lrow + 2 * kk, gw);
+                gdot = __fmaf_rn(m, gw, gdot);
+            }
             if constexpr (sizeof(T) == 2) {
                 if (filing) {
                     const bool has = writer && cell.any;
@@ -288,7 +331,8 @@ __global__ void __launch_bounds__(256, 3) samples_kernel(const Geometry g, const
                     const int ua = w0 < 0 ? 0 : g.BW == 1 ? w0 : static_cast<int>(__umulhi(static_cast<uint32_t>(w0), g.bw_magic));
                     const int cy = h0 + 1 - ta * g.BH, cx = w0 + 1 - ua * g.BW;
                     const int gbase = grp * (g.BH + 1) * (g.BW + 1);
-                    const uint64_t rec = (static_cast<uint64_t>(raw_bits(row[2 * K + kk])) << 16) |
+                    const uint64_t mbits = smax ? weight_q16(m) : raw_bits(row[2 * K + kk]);
+                    const uint64_t rec = (mbits << 16) |
                                          (static_cast<uint64_t>(fix16(cell.lh)) << 32) |
                                          (static_cast<uint64_t>(fix16(cell.lw)) << 48);
                     const int dl0 = has ? window_slot(fs, ta, ua) : -1;
@@ -332,6 +376,12 @@ __global__ void __launch_bounds__(256, 3) samples_kernel(const Geometry g, const
         }
     }
 
+    if (smax && writer) {
+        // logit gradients: the softmax Jacobian applied to the weight gradients
+        T* gr = gom_s + lrow;
+        for (int kk = 0; kk < K; ++kk)
+            gr[2 * K + kk] = from_f32<T>(softmax_weight(to_f32(row[2 * K + kk]), stats) * (get_f32(row + 2 * kk) - gdot));
+    }
     for (int off = 16; off > 0; off >>= 1) my_reach = max(my_reach, __shfl_xor_sync(0xffffffffu, my_reach, off));
     if ((threadIdx.x & 31) == 0 && my_reach >= 0) atomicMax(&s_reach, my_reach);
     if (writer && bmax_h >= bmin_h) {
@@ -486,8 +536,8 @@ struct GySource {
 // sums of its four corners: t0/t1 = top-left/top-right, b0/b1 = bottom-left/
 // bottom-right.  All U grad_out gathers are issued before any is used.
 template <typename T, int VEC, bool COMPACT, int U>
-__device__ __forceinline__ void pull_records(const unsigned char* rec_base, const GySource<T>& gs, int j, float2* t0,
-                                             float2* t1, float2* b0, float2* b1) {
+__device__ __forceinline__ void pull_records(const unsigned char* rec_base, const GySource<T>& gs, bool smax, int j,
+                                             float2* t0, float2* t1, float2* b0, float2* b1) {
     constexpr int EPV = Elem<T>::per16;
     const T* src[U];
     float w[U][4];
@@ -495,8 +545,10 @@ __device__ __forceinline__ void pull_records(const unsigned char* rec_base, cons
     for (int u = 0; u < U; ++u) {
         if constexpr (COMPACT) {
             const uint2 r = reinterpret_cast<const uint2*>(rec_base)[j + u];
-            // m * (hq * wq) * 2^-32 with hq, wq the 16-bit fixed-point weights
-            const float ms = from_bits(static_cast<uint16_t>(r.x >> 16), T()) * 0x1p-32f;
+            // m * (hq * wq) * 2^-32 with hq, wq the 16-bit fixed-point weights; m is
+            // the mask's own bits, or with softmax its weight as q / 65535
+            const uint32_t mq = r.x >> 16;
+            const float ms = smax ? static_cast<float>(mq) * kWeightQ16 : from_bits(static_cast<uint16_t>(mq), T()) * 0x1p-32f;
             const float hq1 = static_cast<float>(r.y & 0xffff), hq0 = 65536.f - hq1;
             const float wq1 = static_cast<float>(r.y >> 16), wq0 = 65536.f - wq1;
             w[u][0] = ms * (hq0 * wq0);
@@ -545,10 +597,10 @@ __device__ __forceinline__ void pull_records(const unsigned char* rec_base, cons
 
 // All records [j, end) of one cell, two at a time.
 template <typename T, int VEC, bool COMPACT>
-__device__ __forceinline__ void pull_cell(const unsigned char* rec_base, const GySource<T>& gs, int j, int end,
-                                          float2* t0, float2* t1, float2* b0, float2* b1) {
-    for (; j + 1 < end; j += 2) pull_records<T, VEC, COMPACT, 2>(rec_base, gs, j, t0, t1, b0, b1);
-    if (j < end) pull_records<T, VEC, COMPACT, 1>(rec_base, gs, j, t0, t1, b0, b1);
+__device__ __forceinline__ void pull_cell(const unsigned char* rec_base, const GySource<T>& gs, bool smax, int j,
+                                          int end, float2* t0, float2* t1, float2* b0, float2* b1) {
+    for (; j + 1 < end; j += 2) pull_records<T, VEC, COMPACT, 2>(rec_base, gs, smax, j, t0, t1, b0, b1);
+    if (j < end) pull_records<T, VEC, COMPACT, 1>(rec_base, gs, smax, j, t0, t1, b0, b1);
 }
 
 // A finished pixel row of a strip: lane cx holds the right corners (r) of
@@ -627,7 +679,7 @@ __device__ __forceinline__ uint32_t ld_stream_u32(const void* p) {
 // Records of the grad_value sort each thread keeps in flight.
 constexpr int kScanBatch = 8;
 
-template <typename T, int VEC, bool COMPACT>
+template <typename T, int VEC, bool COMPACT, bool SM>
 __global__ void __launch_bounds__(256, 2) value_kernel(const Geometry g, const T* __restrict__ om,
                                                        const T* __restrict__ gout, T* __restrict__ gvalue,
                                                        const int* __restrict__ reach, const SampleArrays sa,
@@ -663,6 +715,7 @@ __global__ void __launch_bounds__(256, 2) value_kernel(const Geometry g, const T
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
     const int nthr = blockDim.x;
     const long long pix0 = static_cast<long long>(n) * g.Ho * g.Wo;
+    constexpr bool smax = SM;  // weights are the softmax of each (pixel, group)'s logits
     // Compact records name their output pixel relative to this one (a sample
     // of output pixel p touches the tile only if p's grid lies near it).
     const int ho_ref = floor_div(y0 + g.ph, g.sh), wo_ref = floor_div(x0 + g.pw, g.sw);
@@ -865,11 +918,14 @@ __global__ void __launch_bounds__(256, 2) value_kernel(const Geometry g, const T
                             if constexpr (COMPACT) {
                                 uint32_t id;
                                 if (!compact_source(ho, wo, ho_ref, wo_ref, id)) s_fail = 1;
-                                const uint32_t mb = ld_stream_u16(orow + 2 * g.K + sk);
+                                const uint32_t mb =
+                                    smax ? weight_q16(softmax_weight(to_f32(orow[2 * g.K + sk]), softmax_stats(orow + 2 * g.K, g.K)))
+                                         : ld_stream_u16(orow + 2 * g.K + sk);
                                 rec_c[slot] = make_uint2(id | (mb << 16), fix16(c[u].lh) | (fix16(c[u].lw) << 16));
                             } else {
                                 const Candidate cc = candidate(g, orow, sk, ho, wo, ih, iw);
-                                const float mf = ld_stream_elem(orow + 2 * g.K + sk);
+                                float mf = ld_stream_elem(orow + 2 * g.K + sk);
+                                if (smax) mf = softmax_weight(mf, softmax_stats(orow + 2 * g.K, g.K));
                                 const float b = mf * cc.lh;
                                 rec_w[slot] = make_float4(__int_as_float(pix * g.C), mf - b, b, cc.lw);
                             }
@@ -929,7 +985,7 @@ __global__ void __launch_bounds__(256, 2) value_kernel(const Geometry g, const T
                     end = cur[bin];
                     j = end - cnt[bin];
                 }
-                pull_cell<T, VEC, COMPACT>(rec_base, gs, j, end, a0, a1, b0, b1);
+                pull_cell<T, VEC, COMPACT>(rec_base, gs, smax, j, end, a0, a1, b0, b1);
                 // pixel row cy - 1 (in A) is complete
                 finish_row<T, VEC>(a0, a1, LW, live && t > 0 && cy - 1 < r1 && cx < bw, dst_col + (cy - 1) * row_stride);
                 if (t + 1 > g.BS) break;
@@ -940,7 +996,7 @@ __global__ void __launch_bounds__(256, 2) value_kernel(const Geometry g, const T
                     end = cur[bin];
                     j = end - cnt[bin];
                 }
-                pull_cell<T, VEC, COMPACT>(rec_base, gs, j, end, b0, b1, a0, a1);
+                pull_cell<T, VEC, COMPACT>(rec_base, gs, smax, j, end, b0, b1, a0, a1);
                 finish_row<T, VEC>(b0, b1, LW, live && cy - 1 < r1 && cx < bw, dst_col + (cy - 1) * row_stride);
             }
         }
@@ -980,7 +1036,8 @@ __global__ void __launch_bounds__(256, 2) value_kernel(const Geometry g, const T
                 const Candidate c = candidate(g, orow, k, ho, wo, ih, iw);
                 const int a = gy_abs - c.h0, b = gx_abs - c.w0;
                 if (c.any && a >= 0 && a <= 1 && b >= 0 && b <= 1) {
-                    const float m = to_f32(orow[2 * g.K + k]);
+                    float m = to_f32(orow[2 * g.K + k]);
+                    if (smax) m = softmax_weight(m, softmax_stats(orow + 2 * g.K, g.K));
                     const float wt = m * (a ? c.lh : 1.f - c.lh) * (b ? c.lw : 1.f - c.lw);
                     accumulate<T, VEC>(acc, gy_img + static_cast<long long>(ho * g.Wo + wo) * g.C, wt);
                 }
@@ -1006,11 +1063,11 @@ cudaError_t allow_smem(Kern kern, size_t smem) {
     return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
 }
 
-template <typename T, int VEC, int KH, int KW, bool RC>
+template <typename T, int VEC, int KH, int KW, bool RC, bool SM>
 cudaError_t launch_samples_typed(const Geometry& g, const void* value, const void* om, const void* gout, void* gom,
                                  int* reach, SampleArrays sa, uint32_t* boxes, cudaStream_t stream) {
     const size_t smem = backward_smem_bytes(g, sizeof(T));
-    auto kern = samples_kernel<T, VEC, KH, KW, RC>;
+    auto kern = samples_kernel<T, VEC, KH, KW, RC, SM>;
     cudaError_t e = allow_smem(kern, smem);
     if (e != cudaSuccess) return e;
     const long long blocks = static_cast<long long>(g.N) * g.tiles_h * g.tiles_w;
@@ -1021,29 +1078,36 @@ cudaError_t launch_samples_typed(const Geometry& g, const void* value, const voi
     return cudaGetLastError();
 }
 
-template <typename T, int VEC>
+template <typename T, int VEC, bool SM>
 cudaError_t launch_samples_grid(const Geometry& g, const void* value, const void* om, const void* gout, void* gom,
                                 int* reach, SampleArrays sa, uint32_t* boxes, cudaStream_t stream) {
     if (g.kh == 3 && g.kw == 3) {
         return g.remove_center
-                   ? launch_samples_typed<T, VEC, 3, 3, true>(g, value, om, gout, gom, reach, sa, boxes, stream)
-                   : launch_samples_typed<T, VEC, 3, 3, false>(g, value, om, gout, gom, reach, sa, boxes, stream);
+                   ? launch_samples_typed<T, VEC, 3, 3, true, SM>(g, value, om, gout, gom, reach, sa, boxes, stream)
+                   : launch_samples_typed<T, VEC, 3, 3, false, SM>(g, value, om, gout, gom, reach, sa, boxes, stream);
     }
-    return launch_samples_typed<T, VEC, 0, 0, false>(g, value, om, gout, gom, reach, sa, boxes, stream);
+    return launch_samples_typed<T, VEC, 0, 0, false, SM>(g, value, om, gout, gom, reach, sa, boxes, stream);
+}
+
+template <typename T, int VEC>
+cudaError_t launch_samples_softmax(const Geometry& g, const void* value, const void* om, const void* gout, void* gom,
+                                   int* reach, SampleArrays sa, uint32_t* boxes, cudaStream_t stream) {
+    return g.softmax ? launch_samples_grid<T, VEC, true>(g, value, om, gout, gom, reach, sa, boxes, stream)
+                     : launch_samples_grid<T, VEC, false>(g, value, om, gout, gom, reach, sa, boxes, stream);
 }
 
 template <typename T>
 cudaError_t launch_samples_vec(const Geometry& g, const void* value, const void* om, const void* gout, void* gom,
                                int* reach, SampleArrays sa, uint32_t* boxes, cudaStream_t stream) {
-    return g.vec == 2 ? launch_samples_grid<T, 2>(g, value, om, gout, gom, reach, sa, boxes, stream)
-                      : launch_samples_grid<T, 1>(g, value, om, gout, gom, reach, sa, boxes, stream);
+    return g.vec == 2 ? launch_samples_softmax<T, 2>(g, value, om, gout, gom, reach, sa, boxes, stream)
+                      : launch_samples_softmax<T, 1>(g, value, om, gout, gom, reach, sa, boxes, stream);
 }
 
-template <typename T, int VEC>
+template <typename T, int VEC, bool SM>
 cudaError_t launch_value_typed(const Geometry& g, const void* om, const void* gout, void* gvalue, const int* reach,
                                SampleArrays sa, const uint32_t* boxes, cudaStream_t stream) {
     const size_t smem = backward_value_smem_bytes(g);
-    auto kern = value_kernel<T, VEC, sizeof(T) == 2>;
+    auto kern = value_kernel<T, VEC, sizeof(T) == 2, SM>;
     cudaError_t e = allow_smem(kern, smem);
     if (e != cudaSuccess) return e;
     const long long blocks = static_cast<long long>(g.N) * g.btiles_h * g.btiles_w;
@@ -1055,8 +1119,11 @@ cudaError_t launch_value_typed(const Geometry& g, const void* om, const void* go
 template <typename T>
 cudaError_t launch_value_vec(const Geometry& g, const void* om, const void* gout, void* gvalue, const int* reach,
                              SampleArrays sa, const uint32_t* boxes, cudaStream_t stream) {
-    return g.vec == 2 ? launch_value_typed<T, 2>(g, om, gout, gvalue, reach, sa, boxes, stream)
-                      : launch_value_typed<T, 1>(g, om, gout, gvalue, reach, sa, boxes, stream);
+    if (g.softmax)
+        return g.vec == 2 ? launch_value_typed<T, 2, true>(g, om, gout, gvalue, reach, sa, boxes, stream)
+                          : launch_value_typed<T, 1, true>(g, om, gout, gvalue, reach, sa, boxes, stream);
+    return g.vec == 2 ? launch_value_typed<T, 2, false>(g, om, gout, gvalue, reach, sa, boxes, stream)
+                      : launch_value_typed<T, 1, false>(g, om, gout, gvalue, reach, sa, boxes, stream);
 }
 
 }  // namespace

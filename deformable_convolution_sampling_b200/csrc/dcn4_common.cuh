@@ -20,6 +20,7 @@ struct Geometry {
     int kh, kw, sh, sw, ph, pw, dh, dw;
     float s;              // offset_scale
     int remove_center;
+    int softmax;          // masks are logits normalised by a softmax over the K points
     int vec;              // 16-byte vectors per thread slice: 2 (one 32-byte access) or 1
     int nslice;           // threads cooperating on one (pixel, group): power of two <= 32
     int pix_per_cta;      // output pixels handled by one CTA (= TH * TW)
@@ -246,6 +247,39 @@ __device__ __forceinline__ void stage_tile_rows(T* dst_smem, const T* src, const
         char* d = reinterpret_cast<char*>(dst_smem + r * g.TW * g.P) + 16 * c;
         *reinterpret_cast<uint4*>(d) = ld_stream(s);
     }
+}
+
+// ---------------------------------------------------------------------------
+// Softmax over the K mask logits of one (pixel, group) -- the DCNv3 form of the
+// modulation scalars (CSDN summary of "Efficient Deformable ConvNets", section
+// 1.2): m_k = exp(l_k - l_max) / sum_j exp(l_j - l_max), in fp32, the sum taken
+// in k order.  softmax_stats returns (l_max, 1 / sum) and softmax_weight then
+// gives m_k; softmax_exps keeps the K exponentials (e[k * stride]) and returns
+// the same (l_max, 1 / sum), m_k being e_k * (1 / sum).  All give the same fp32
+// weights.
+// ---------------------------------------------------------------------------
+template <typename T>
+__device__ __forceinline__ float2 softmax_stats(const T* logits, int K) {
+    float mx = -INFINITY;
+    for (int j = 0; j < K; ++j) mx = fmaxf(mx, to_f32(logits[j]));
+    float sum = 0.f;
+    for (int j = 0; j < K; ++j) sum += expf(to_f32(logits[j]) - mx);
+    return make_float2(mx, 1.f / sum);
+}
+__device__ __forceinline__ float softmax_weight(float logit, float2 stats) {
+    return expf(logit - stats.x) * stats.y;
+}
+template <typename T>
+__device__ __forceinline__ float2 softmax_exps(const T* logits, int K, float* e, int stride) {
+    float mx = -INFINITY;
+    for (int j = 0; j < K; ++j) mx = fmaxf(mx, to_f32(logits[j]));
+    float sum = 0.f;
+    for (int j = 0; j < K; ++j) {
+        const float x = expf(to_f32(logits[j]) - mx);
+        e[j * stride] = x;
+        sum += x;
+    }
+    return make_float2(mx, 1.f / sum);
 }
 
 // ---------------------------------------------------------------------------

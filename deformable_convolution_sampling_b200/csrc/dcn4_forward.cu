@@ -17,7 +17,10 @@
 // are adjacent lanes, so a warp's loads spread over distinct slots of the L1
 // lines) and accumulates in fp32 with packed f32x2 FMAs: the coefficient reuse
 // and vector loads of section 2.2 ("消除冗余工作量", "消除冗余内存指令").
-// Nothing is written but the output, with 256-bit stores.
+// Nothing is written but the output, with 256-bit stores.  With softmax the
+// masks are logits: before its samples each thread takes the K exponentials of
+// its (pixel, group)'s logits once, into its own slots of shared memory (no
+// barrier), and the samples read their weights from there.
 #include <algorithm>
 #include <atomic>
 
@@ -106,8 +109,8 @@ __device__ __forceinline__ void stage_tile_async(T* dst_smem, const T* src, cons
 // tile + gridDim.x, ...), copying the next tile's offset_mask rows into the
 // other half of a double buffer (cp.async) while it computes the current one.
 // KH, KW > 0: compile-time grid size (fully unrolled) and RC = remove_center;
-// KH = KW = 0: sizes and remove_center from g.
-template <typename T, int VEC, int KH, int KW, bool RC>
+// KH = KW = 0: sizes and remove_center from g.  SM: softmax over the K masks.
+template <typename T, int VEC, int KH, int KW, bool RC, bool SM>
 __global__ void __launch_bounds__(256, kFwdCtasPerSm) forward_kernel(const Geometry g, const T* __restrict__ value,
                                                       const T* __restrict__ om, T* __restrict__ out) {
     extern __shared__ __align__(16) unsigned char smem[];
@@ -115,6 +118,7 @@ __global__ void __launch_bounds__(256, kFwdCtasPerSm) forward_kernel(const Geome
     constexpr int PAIRS = VEC * EPV / 2;
     const int tile_elems = g.TH * g.TW * g.P;
     T* bufs[2] = {reinterpret_cast<T*>(smem), reinterpret_cast<T*>(smem) + tile_elems};
+    float* e_s = reinterpret_cast<float*>(bufs[1] + tile_elems);  // softmax exponentials [K][threads]
     const int ntiles = g.N * g.tiles_h * g.tiles_w;
     int tile = blockIdx.x;
     if (tile >= ntiles) return;
@@ -152,6 +156,8 @@ __global__ void __launch_bounds__(256, kFwdCtasPerSm) forward_kernel(const Geome
             float2 acc[PAIRS];
 #pragma unroll
             for (int i = 0; i < PAIRS; ++i) acc[i] = make_float2(0.f, 0.f);
+            float inv = 1.f;
+            if constexpr (SM) inv = softmax_exps(row + 2 * K, K, e_s + threadIdx.x, blockDim.x).y;
             int k = 0;
 #pragma unroll
             for (int iw = 0; iw < kw; ++iw) {
@@ -161,7 +167,8 @@ __global__ void __launch_bounds__(256, kFwdCtasPerSm) forward_kernel(const Geome
                     if (rc && iw == kw / 2 && ih == kh / 2) continue;
                     const float dx = to_f32(row[2 * k]);
                     const float dy = to_f32(row[2 * k + 1]);
-                    const float m = to_f32(row[2 * K + k]);
+                    float m = to_f32(row[2 * K + k]);
+                    if constexpr (SM) m = e_s[k * blockDim.x + threadIdx.x] * inv;
                     ++k;
                     const float h = __fmaf_rn(g.s, dy, static_cast<float>(hb + ih * g.dh));
                     const float w = __fmaf_rn(g.s, dx, wbase);
@@ -185,10 +192,10 @@ __global__ void __launch_bounds__(256, kFwdCtasPerSm) forward_kernel(const Geome
     }
 }
 
-template <typename T, int VEC, int KH, int KW, bool RC>
+template <typename T, int VEC, int KH, int KW, bool RC, bool SM>
 cudaError_t launch_typed(const Geometry& g, const void* value, const void* om, void* out, cudaStream_t stream) {
     const size_t smem = forward_smem_bytes(g, sizeof(T));
-    auto kern = forward_kernel<T, VEC, KH, KW, RC>;
+    auto kern = forward_kernel<T, VEC, KH, KW, RC, SM>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     const int threads = (g.pix_per_cta * g.G * g.nslice + 31) / 32 * 32;
@@ -206,24 +213,31 @@ cudaError_t launch_typed(const Geometry& g, const void* value, const void* om, v
     return cudaGetLastError();
 }
 
-template <typename T, int VEC>
+template <typename T, int VEC, bool SM>
 cudaError_t launch_grid(const Geometry& g, const void* value, const void* om, void* out, cudaStream_t stream) {
     if (g.kh == 3 && g.kw == 3) {
-        return g.remove_center ? launch_typed<T, VEC, 3, 3, true>(g, value, om, out, stream)
-                               : launch_typed<T, VEC, 3, 3, false>(g, value, om, out, stream);
+        return g.remove_center ? launch_typed<T, VEC, 3, 3, true, SM>(g, value, om, out, stream)
+                               : launch_typed<T, VEC, 3, 3, false, SM>(g, value, om, out, stream);
     }
-    return launch_typed<T, VEC, 0, 0, false>(g, value, om, out, stream);
+    return launch_typed<T, VEC, 0, 0, false, SM>(g, value, om, out, stream);
+}
+
+template <typename T, int VEC>
+cudaError_t launch_softmax(const Geometry& g, const void* value, const void* om, void* out, cudaStream_t stream) {
+    return g.softmax ? launch_grid<T, VEC, true>(g, value, om, out, stream)
+                     : launch_grid<T, VEC, false>(g, value, om, out, stream);
 }
 
 template <typename T>
 cudaError_t launch_vec(const Geometry& g, int vec, const void* value, const void* om, void* out, cudaStream_t stream) {
-    return vec == 2 ? launch_grid<T, 2>(g, value, om, out, stream) : launch_grid<T, 1>(g, value, om, out, stream);
+    return vec == 2 ? launch_softmax<T, 2>(g, value, om, out, stream) : launch_softmax<T, 1>(g, value, om, out, stream);
 }
 
 }  // namespace
 
 size_t forward_smem_bytes(const Geometry& g, int elem_bytes) {
-    return 2 * static_cast<size_t>(g.pix_per_cta) * g.P * elem_bytes;  // double buffer
+    return 2 * static_cast<size_t>(g.pix_per_cta) * g.P * elem_bytes +                        // double buffer
+           (g.softmax ? static_cast<size_t>(g.K) * samples_threads(g) * sizeof(float) : 0);  // exponentials
 }
 
 cudaError_t launch_forward(const Geometry& g, int dtype, const void* value, const void* om, void* out,

@@ -13,7 +13,13 @@
  * kh x kw convolution grid with stride, padding and dilation; remove_center
  * drops the centre cell so K = kh*kw - 1 (DCNv4 module / dcnv4_cuda_forward
  * signatures on the mhpn.cn architecture page).  The modulation scalars m_gk
- * are unbounded (no softmax).
+ * are unbounded (no softmax) unless `softmax` is set, which gives the DCNv3
+ * form: m_gk = exp(l_gk) / sum_j exp(l_gj) over the K mask entries l_gk of the
+ * (pixel, group) (CSDN summary, section 1.2 DCNv3 equation; the `softmax` flag
+ * of the dcnv4_cuda_forward signature on the mhpn.cn page).  The exponentials are taken
+ * after subtracting the largest l_gj, in fp32 (expf), and grad_offset_mask
+ * then holds the gradients of the logits l_gk:
+ * m_gk * (<gy, S_k> - sum_j m_gj <gy, S_j>).
  *
  * Sampling location of grid cell (ih, iw) for output pixel (ho, wo):
  *     h = ho*sh - ph + ih*dh + offset_scale*dy,   w = wo*sw - pw + iw*dw + offset_scale*dx
@@ -48,7 +54,8 @@
  *   - Cg * sizeof(dtype) a multiple of 16 bytes (fp32: Cg % 4 == 0, fp16/bf16:
  *     Cg % 8 == 0) and Cg * sizeof(dtype) / 32 (rounded up) a power of two <= 32;
  *   - H, W < 2^24 and H*W*C < 2^31 (per image), Ho >= 1, Wo >= 1;
- *   - remove_center only with odd kh and kw.
+ *   - remove_center only with odd kh and kw;
+ *   - remove_center and softmax each 0 or 1.
  * Errors are returned, never raised: no abort, no exception, no device trap.
  */
 #ifndef DCN4_H
@@ -60,7 +67,7 @@
 extern "C" {
 #endif
 
-#define DCN4_VERSION 100  /* 1.0.0 */
+#define DCN4_VERSION 110  /* 1.1.0: dcn4_params.softmax */
 
 typedef enum {
     DCN4_F32 = 0,   /* IEEE binary32            */
@@ -92,6 +99,8 @@ typedef struct {
     int remove_center;    /* 0 or 1                                             */
     int P;                /* row length of offset_mask / grad_offset_mask       */
     int dtype;            /* dcn4_dtype of every tensor argument                */
+    int softmax;          /* 0: masks used as given; 1: softmax over the K masks
+                             of each (pixel, group) (DCNv3 form)                */
 } dcn4_params;
 
 /* Library version (DCN4_VERSION of the build). */

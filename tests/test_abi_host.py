@@ -47,6 +47,22 @@ def test_every_declared_symbol_is_exported(dcn):
     assert exported == set(declared_functions()), exported ^ set(declared_functions())
 
 
+def test_params_mirror_matches_the_header(dcn):
+    """The binding's ctypes dcn4_params has the header's fields, in order, all 4 bytes."""
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    body = re.search(r"typedef struct \{(.*?)\} dcn4_params;", text, flags=re.S).group(1)
+    fields = []
+    for decl in body.split(";"):
+        decl = decl.strip()
+        if decl:
+            ctype, names = decl.split(None, 1)
+            assert ctype in ("int", "float"), decl
+            fields += [n.strip() for n in names.split(",")]
+    assert [f[0] for f in dcn.dcn4_params._fields_] == fields
+    assert ctypes.sizeof(dcn.dcn4_params) == 4 * len(fields)
+    assert dcn.dcn4_version() == 110
+
+
 def test_library_does_not_link_the_oracle(dcn):
     out = subprocess.run(["ldd", dcn.LIB_PATH], capture_output=True, text=True).stdout
     assert "oracle" not in out
@@ -103,7 +119,7 @@ def test_workspace_size(dcn):
 
 @pytest.mark.parametrize("field,value,status", [
     ("dtype", 7, -8), ("N", -1, -2), ("H", 0, -2), ("G", 0, -2), ("Cg", 0, -2), ("kh", 0, -2),
-    ("sh", 0, -2), ("ph", -1, -2), ("dh", 0, -2), ("remove_center", 2, -2), ("P", 50, -3),
+    ("sh", 0, -2), ("ph", -1, -2), ("dh", 0, -2), ("remove_center", 2, -2), ("softmax", 2, -2), ("softmax", -1, -2), ("P", 50, -3),
     ("P", 60, -3), ("Cg", 4, -5), ("Cg", 24, -5), ("Cg", 48, -5), ("H", 1 << 24, -5),
 ])
 def test_invalid_params_are_rejected_before_launch(dcn, field, value, status):
