@@ -2,7 +2,7 @@
 """Benchmark of the DCNv4 core operator on B200: one forward + backward step.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
-                    [--workload NAME] [--no-cpu-baseline] [--no-e2e]
+                    [--workload NAME] [--softmax] [--no-cpu-baseline] [--no-e2e]
 
 A step is one pass of the whole path over one batch: dcn4_forward followed by
 dcn4_backward on the first-stage backbone workload (N64 H56 W56 C64 G4, C'=16,
@@ -20,6 +20,9 @@ against the algorithmic byte model, the roofline of the dominant launch, an
 end-to-end figure through host buffers, clocks sampled during the timed loop,
 and a CPU-oracle baseline.
 
+--softmax runs the same step with the masks normalised by a softmax over the
+K points of each (pixel, group) (the DCNv3 form of the operator).
+
 --impl reference times the CPU oracle (the only other implementation of the
 operator) on the host cores, on a bounded sample of the same workload per
 step, scaled to the full batch.
@@ -27,6 +30,7 @@ step, scaled to the full batch.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import os
 import statistics
@@ -441,6 +445,8 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--workload", default="stage1_f16", choices=sorted(gen.WORKLOADS))
+    ap.add_argument("--softmax", action="store_true",
+                    help="masks are logits normalised by a softmax over the K points (DCNv3 form)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
@@ -451,6 +457,8 @@ def main(argv=None):
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     w = gen.WORKLOADS[args.workload]
+    if args.softmax:
+        w = dataclasses.replace(w, softmax=1, name=w.name + "_softmax")
     rank, world, _ = dist_env()
     if args.impl == "reference":
         res = run_reference(args, w)
