@@ -72,15 +72,25 @@ def byte_model(w: gen.Workload) -> dict:
 KERNELS = {"fwd": "forward_kernel", "bwd_offset_mask": "samples_kernel", "bwd_value": "value_kernel"}
 
 
-def kernel_sources_sha() -> str:
-    """sha256 over the CUDA sources: a DRAM-traffic capture is only reported
-    while the kernels are the ones it measured."""
-    import glob
+# Sources each kernel is built from: its own translation unit, the shared device
+# helpers, the host side that sets its launch geometry, and the ABI header.
+KERNEL_SOURCES = {
+    "forward_kernel": ["csrc/dcn4_forward.cu"],
+    "samples_kernel": ["csrc/dcn4_backward.cu"],
+    "value_kernel": ["csrc/dcn4_backward.cu"],
+}
+COMMON_SOURCES = ["csrc/dcn4_common.cuh", "csrc/dcn4_api.cu", "../include/dcn4.h"]
+
+
+def kernel_sources_sha(kernel: str) -> str:
+    """sha256 over the sources `kernel` is built from: a DRAM-traffic capture is
+    only reported while the kernel is the one it measured."""
     import hashlib
     h = hashlib.sha256()
-    for f in sorted(glob.glob(os.path.join(ROOT, "deformable_convolution_sampling_b200", "csrc", "*.cu*"))):
-        with open(f, "rb") as fh:
-            h.update(os.path.basename(f).encode())
+    pkg = os.path.join(ROOT, "deformable_convolution_sampling_b200")
+    for rel in KERNEL_SOURCES[kernel] + COMMON_SOURCES:
+        with open(os.path.normpath(os.path.join(pkg, rel)), "rb") as fh:
+            h.update(os.path.basename(rel).encode())
             h.update(fh.read())
     return h.hexdigest()
 
@@ -93,7 +103,7 @@ def recorded_traffic(kernel: str, workload: str):
         lines = open(path).read().splitlines()
     except OSError:
         return None
-    sha = kernel_sources_sha()
+    sha = kernel_sources_sha(kernel)
     for line in lines:
         parts = line.split()
         if len(parts) >= 4 and not line.startswith("#") and parts[0] == kernel and parts[1] == workload:

@@ -36,15 +36,22 @@ def test_summarize_clocks():
     assert c["samples"] == 3 and c["window"].startswith("whole run")
 
 
+def test_kernel_sources_sha_covers_the_kernels_own_sources():
+    shas = {k: bench.kernel_sources_sha(k) for k in bench.KERNELS.values()}
+    assert shas["samples_kernel"] == shas["value_kernel"]          # one translation unit
+    assert shas["forward_kernel"] != shas["value_kernel"]
+    assert all(len(v) == 64 for v in shas.values())
+
+
 def test_recorded_traffic_needs_matching_sources(tmp_path, monkeypatch):
     (tmp_path / "profiles").mkdir()
-    sha = bench.kernel_sources_sha()
+    sha = bench.kernel_sources_sha("value_kernel")
     (tmp_path / "profiles" / "dram_traffic.txt").write_text(
         "# kernel workload bytes sources_sha256\n"
         f"value_kernel stage1_f16 123456 {sha}\n"
         "forward_kernel stage1_f16 99 0000\n")
     monkeypatch.setattr(bench, "ROOT", tmp_path)
-    monkeypatch.setattr(bench, "kernel_sources_sha", lambda: sha)
+    monkeypatch.setattr(bench, "kernel_sources_sha", lambda kernel: sha)
     assert bench.recorded_traffic("value_kernel", "stage1_f16") == 123456
     assert bench.recorded_traffic("forward_kernel", "stage1_f16") is None   # other sources
     assert bench.recorded_traffic("samples_kernel", "stage1_f16") is None   # not captured
