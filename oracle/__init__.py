@@ -108,6 +108,10 @@ def lib() -> ctypes.CDLL:
         L.ref_backward.restype = ctypes.c_int
         L.ref_decode.argtypes = [ctypes.c_int, vp, dp, ctypes.c_int64]
         L.ref_decode.restype = None
+        L.ref_encode.argtypes = [ctypes.c_int, dp, vp, ctypes.c_int64]
+        L.ref_encode.restype = None
+        L.ref_linear.argtypes = [ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int, vp, vp, vp, vp]
+        L.ref_linear.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -173,6 +177,35 @@ def decode(dtype: str, arr: np.ndarray) -> np.ndarray:
         raise TypeError(f"decode {dtype}: got {arr.dtype}")
     out = np.empty(arr.shape, dtype=np.float64)
     lib().ref_decode(DTYPES[dtype], _ptr(arr), _dptr(out), arr.size)
+    return out
+
+
+def encode(dtype: str, values: np.ndarray) -> np.ndarray:
+    """values (float64) stored in `dtype`, rounded to nearest, ties to even."""
+    v = np.ascontiguousarray(values, dtype=np.float64)
+    out = np.empty(v.shape, dtype=NUMPY_STORAGE[dtype])
+    lib().ref_encode(DTYPES[dtype], _dptr(v), _ptr(out), v.size)
+    return out
+
+
+def linear(dtype: str, x: np.ndarray, weight: np.ndarray, bias: np.ndarray | None = None) -> np.ndarray:
+    """The merged offset/mask linear layer: round_dtype(x @ weight.T + bias) with x
+    [..., Cin], weight [Cout, Cin], bias [Cout] (or None), all stored in `dtype`;
+    returns [..., Cout] stored in `dtype`."""
+    want = NUMPY_STORAGE[dtype]
+    x = np.ascontiguousarray(x)
+    weight = np.ascontiguousarray(weight)
+    for name, a in (("x", x), ("weight", weight)) + ((("bias", bias),) if bias is not None else ()):
+        if a.dtype != want:
+            raise TypeError(f"{name}: storage {dtype} wants {np.dtype(want)}, got {a.dtype}")
+    Cout, Cin = weight.shape
+    if x.shape[-1] != Cin or (bias is not None and tuple(bias.shape) != (Cout,)):
+        raise ValueError("linear: shape mismatch")
+    M = int(np.prod(x.shape[:-1]))
+    out = np.empty(x.shape[:-1] + (Cout,), dtype=want)
+    b = _ptr(np.ascontiguousarray(bias)) if bias is not None else None
+    if lib().ref_linear(M, Cin, Cout, DTYPES[dtype], _ptr(x), _ptr(weight), b, _ptr(out)) != 0:
+        raise ValueError("oracle linear rejected its arguments")
     return out
 
 

@@ -44,6 +44,68 @@ double decode_bf16(uint16_t bits) {
     return static_cast<double>(f);
 }
 
+// Encoders: the nearest representable value, ties to an even last fraction bit.
+// std::nearbyint rounds to an integer in the default mode (to nearest, ties to
+// even); a / 2^k is exact, so q below is the value in units of the last place.
+
+// binary16: normal numbers 1.f x 2^E (E in [-14, 15], 10 fraction bits, unit in
+// the last place 2^(E-10)); below 2^-14 the unit is 2^-24 (subnormals).
+uint16_t encode_f16(double v) {
+    if (std::isnan(v)) return 0x7e00;
+    const uint16_t sign = std::signbit(v) ? 0x8000 : 0;
+    const double a = std::fabs(v);
+    if (a == 0.0) return sign;
+    if (std::isinf(a)) return sign | 0x7c00;
+    int e;
+    std::frexp(a, &e);  // a = m * 2^e, m in [0.5, 1): the leading bit is 2^(e-1)
+    int E = e - 1;
+    if (E < -14) {
+        const double q = std::nearbyint(std::ldexp(a, 24));  // units of 2^-24, <= 1024
+        return sign | static_cast<uint16_t>(q);              // q = 1024 is the smallest normal
+    }
+    double q = std::nearbyint(std::ldexp(a, 10 - E));        // in [1024, 2048]
+    if (q == 2048.0) {
+        q = 1024.0;
+        ++E;
+    }
+    if (E > 15) return sign | 0x7c00;
+    return sign | static_cast<uint16_t>(((E + 15) << 10) | (static_cast<int>(q) - 1024));
+}
+
+// bfloat16: binary32's exponent range (E in [-126, 127]) with 7 fraction bits;
+// below 2^-126 the unit is 2^-133.
+uint16_t encode_bf16(double v) {
+    if (std::isnan(v)) return 0x7fc0;
+    const uint16_t sign = std::signbit(v) ? 0x8000 : 0;
+    const double a = std::fabs(v);
+    if (a == 0.0) return sign;
+    if (std::isinf(a)) return sign | 0x7f80;
+    int e;
+    std::frexp(a, &e);
+    int E = e - 1;
+    if (E < -126) {
+        const double q = std::nearbyint(std::ldexp(a, 133));  // <= 128
+        return sign | static_cast<uint16_t>(q);
+    }
+    double q = std::nearbyint(std::ldexp(a, 7 - E));          // in [128, 256]
+    if (q == 256.0) {
+        q = 128.0;
+        ++E;
+    }
+    if (E > 127) return sign | 0x7f80;
+    return sign | static_cast<uint16_t>(((E + 127) << 7) | (static_cast<int>(q) - 128));
+}
+
+void store(void* buf, int dtype, int64_t i, double v) {
+    switch (dtype) {
+        case REF_F32: static_cast<float*>(buf)[i] = static_cast<float>(v); break;  // C rounds to nearest even
+        case REF_F16: static_cast<uint16_t*>(buf)[i] = encode_f16(v); break;
+        case REF_BF16: static_cast<uint16_t*>(buf)[i] = encode_bf16(v); break;
+        case REF_F64: static_cast<double*>(buf)[i] = v; break;
+        default: break;
+    }
+}
+
 double load(const void* buf, int dtype, int64_t i) {
     switch (dtype) {
         case REF_F32: return static_cast<double>(static_cast<const float*>(buf)[i]);
@@ -212,6 +274,25 @@ std::vector<double> point_weights(const ref_problem* p, const void* offset_mask,
         for (int k = 0; k < K; ++k) a[k] /= sum;
     }
     return a;
+}
+
+void ref_encode(int dtype, const double* src, void* dst, int64_t n) {
+    for (int64_t i = 0; i < n; ++i) store(dst, dtype, i, src[i]);
+}
+
+int ref_linear(int64_t M, int Cin, int Cout, int dtype, const void* x, const void* weight,
+               const void* bias, void* out) {
+    if (M < 0 || Cin < 1 || Cout < 1 || dtype < REF_F32 || dtype > REF_F64 || !x || !weight || !out) return -1;
+    for (int64_t m = 0; m < M; ++m) {
+        for (int j = 0; j < Cout; ++j) {
+            double acc = 0.0;
+            for (int c = 0; c < Cin; ++c)
+                acc += load(x, dtype, m * Cin + c) * load(weight, dtype, static_cast<int64_t>(j) * Cin + c);
+            if (bias) acc += load(bias, dtype, j);
+            store(out, dtype, m * Cout + j, acc);
+        }
+    }
+    return 0;
 }
 
 void ref_decode(int dtype, const void* src, double* dst, int64_t n) {

@@ -107,6 +107,24 @@ int ref_backward(const ref_problem* p, const void* value, const void* offset_mas
 /* Exact decode of n stored elements into doubles. */
 void ref_decode(int dtype, const void* src, double* dst, int64_t n);
 
+/* Store n doubles in `dtype`, each rounded to the nearest representable value,
+ * ties to the one with an even last fraction bit (IEEE 754 roundTiesToEven);
+ * beyond the largest finite value (by at least half a unit in its last place)
+ * the result is an infinity; NaN stays NaN.  REF_F64 copies. */
+void ref_encode(int dtype, const double* src, void* dst, int64_t n);
+
+/* The merged offset/mask linear layer of the DCNv4 module (CSDN summary,
+ * section 2.2 "DCN模块的微设计": the offsets and the dynamic weights come from a
+ * single linear layer; with latency first, the depthwise convolution before it
+ * is dropped):
+ *     out[m, j] = round_dtype( sum_c x[m, c] * weight[j, c] + bias[j] )
+ * for m < M rows (output pixels) and j < Cout (= P, the padded row length),
+ * x [M, Cin] and weight [Cout, Cin] (nn.Linear layout) stored in `dtype`, bias
+ * [Cout] in `dtype` or NULL (zero).  The sum is taken in double in c order and
+ * rounded once (ref_encode).  Returns 0, or -1 for bad sizes. */
+int ref_linear(int64_t M, int Cin, int Cout, int dtype, const void* x, const void* weight,
+               const void* bias, void* out);
+
 #ifdef __cplusplus
 }
 #endif

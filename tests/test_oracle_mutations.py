@@ -34,6 +34,13 @@ MUTATIONS = {
     "softmax_not_normalised": ("for (int k = 0; k < K; ++k) a[k] /= sum;", ""),
     "softmax_largest_not_subtracted": ("a[k] = std::exp(a[k] - mx);", "a[k] = std::exp(a[k]);"),
     "softmax_jacobian_without_sum": ("p->softmax ? a[k] * (gw[k] - dot) : gw[k]", "p->softmax ? a[k] * gw[k] : gw[k]"),
+    # storage rounding and the offset/mask linear layer
+    "encode_f16_truncates": ("double q = std::nearbyint(std::ldexp(a, 10 - E));", "double q = std::floor(std::ldexp(a, 10 - E));"),
+    "encode_bf16_ties_away": ("double q = std::nearbyint(std::ldexp(a, 7 - E));", "double q = std::round(std::ldexp(a, 7 - E));"),
+    "encode_f16_subnormal_unit": ("std::nearbyint(std::ldexp(a, 24));", "std::nearbyint(std::ldexp(a, 25));"),
+    "linear_drops_bias": ("if (bias) acc += load(bias, dtype, j);", ""),
+    "linear_weight_transposed": ("load(weight, dtype, static_cast<int64_t>(j) * Cin + c)",
+                                 "load(weight, dtype, static_cast<int64_t>(c % Cout) * Cin + (j % Cin))"),
     "softmax_ignored_in_backward_offsets": ("const double m = a[k];\n                        double h, w;\n                        sample_location(p, ho, wo, cells[k], dx, dy, &h, &w);\n                        const Bilinear b = bilinear_cell(p, h, w);\n                        if (!b.any) continue;",
                                             "const double m = load(offset_mask, p->dtype, om + 2 * K + k);\n                        double h, w;\n                        sample_location(p, ho, wo, cells[k], dx, dy, &h, &w);\n                        const Bilinear b = bilinear_cell(p, h, w);\n                        if (!b.any) continue;"),
 }

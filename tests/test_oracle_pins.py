@@ -601,3 +601,107 @@ def test_softmax_grad_value_is_adjoint():
     lhs = float(np.sum(inp["grad_out"] * y))
     rhs = float(np.sum(gv * inp["value"]))
     assert abs(lhs - rhs) <= 1e-12 * max(abs(lhs), 1.0)
+
+
+# ---------------------------------------------------------------------------
+# Rounding to storage and the merged offset/mask linear layer
+# ---------------------------------------------------------------------------
+
+def _lattice(fmt):
+    """Every finite non-negative value of the 16-bit format with its bit pattern, ascending
+    (decoded by numpy's own bit views, independent of the oracle's decoders)."""
+    bits = np.arange(0, 0x8000, dtype=np.uint16)
+    if fmt == "f16":
+        vals = bits.view(np.float16).astype(np.float64)
+    else:
+        vals = (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    keep = np.isfinite(vals)
+    return vals[keep], bits[keep]
+
+
+def _nearest_even(fmt, v):
+    """Brute force: the nearest lattice value of |v| (ties: even pattern), with v's sign;
+    beyond the largest finite value by half a unit or more: infinity."""
+    vals, bits = _lattice(fmt)
+    a = np.abs(v)
+    i = np.clip(np.searchsorted(vals, a), 1, len(vals) - 1)
+    lo, hi = vals[i - 1], vals[i]
+    pick_hi = (a - lo > hi - a) | ((a - lo == hi - a) & (bits[i] % 2 == 0))
+    out = np.where(pick_hi, bits[i], bits[i - 1]).astype(np.uint16)
+    top = vals[-1]
+    half_ulp = (vals[-1] - vals[-2]) / 2
+    inf = np.uint16(0x7c00 if fmt == "f16" else 0x7f80)
+    out = np.where(a >= top + half_ulp, inf, np.where(a > top, bits[-1], out))
+    return (out | np.where(np.signbit(v), 0x8000, 0).astype(np.uint16)).astype(np.uint16)
+
+
+@pytest.mark.parametrize("fmt", ["f16", "bf16"])
+def test_encode_round_trips_every_finite_pattern(fmt):
+    vals, bits = _lattice(fmt)
+    for sign in (0, 0x8000):
+        got = oracle.encode(fmt, vals if sign == 0 else -vals).view(np.uint16)
+        want = bits | np.uint16(sign)
+        same = got == want
+        # -0.0 encodes as 0x8000, +0.0 as 0
+        assert np.all(same), np.flatnonzero(~same)[:5]
+
+
+@pytest.mark.parametrize("fmt", ["f16", "bf16"])
+def test_encode_is_nearest_ties_to_even(fmt):
+    """Midpoints between neighbouring values (exact ties), points just either side of
+    them, random values over the whole range, subnormals and the overflow threshold."""
+    vals, _ = _lattice(fmt)
+    mids = (vals[:-1] + vals[1:]) / 2
+    rng = np.random.default_rng(3)
+    span = np.log2(vals[-1])
+    v = np.concatenate([mids, np.nextafter(mids, 0), np.nextafter(mids, np.inf),
+                        rng.uniform(-1, 1, 20000) * 2.0 ** rng.uniform(-30 if fmt == "f16" else -140, span, 20000),
+                        [vals[-1] * 1.0001, vals[-1] + (vals[-1] - vals[-2]) / 2, 1e300, -1e300]])
+    got = oracle.encode(fmt, v).view(np.uint16)
+    assert np.array_equal(got, _nearest_even(fmt, v))
+    if fmt == "f16":  # numpy's float64 -> float16 cast rounds the same way
+        with np.errstate(over="ignore"):
+            assert np.array_equal(got, v.astype(np.float16).view(np.uint16))
+
+
+def test_encode_nan_and_f32():
+    out = oracle.encode("f16", np.array([np.nan])).view(np.uint16)
+    assert (out[0] & 0x7c00) == 0x7c00 and (out[0] & 0x3ff) != 0
+    v = np.random.default_rng(4).normal(size=1000) * 1e3
+    assert np.array_equal(oracle.encode("f32", v), v.astype(np.float32))
+
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16", "f32"])
+@pytest.mark.parametrize("with_bias", [True, False])
+def test_linear_is_the_rounded_affine_map(dtype, with_bias):
+    """x @ W.T + b in float64 (numpy's matmul), rounded once to the storage format."""
+    rng = np.random.default_rng(5)
+    M, Cin, Cout = 37, 48, 40
+    x = gen.to_storage(rng.normal(size=(M, Cin)), dtype)
+    w = gen.to_storage(rng.normal(size=(Cout, Cin)) / 8, dtype)
+    b = gen.to_storage(rng.normal(size=Cout), dtype) if with_bias else None
+    got = oracle.linear(dtype, x, w, b)
+    exact = gen.storage_to_f64(x, dtype) @ gen.storage_to_f64(w, dtype).T + (gen.storage_to_f64(b, dtype) if with_bias else 0.0)
+    if dtype == "f32":
+        assert np.array_equal(got, exact.astype(np.float32))
+    else:
+        assert np.array_equal(got.view(np.uint16), _nearest_even(dtype, exact))
+    # an identity weight copies x, a zero weight gives the bias
+    eye = gen.to_storage(np.eye(Cin), dtype)
+    assert np.array_equal(gen.storage_to_f64(oracle.linear(dtype, x, eye), dtype), gen.storage_to_f64(x, dtype))
+    if with_bias:
+        zero = gen.to_storage(np.zeros((Cout, Cin)), dtype)
+        assert np.array_equal(gen.storage_to_f64(oracle.linear(dtype, x, zero, b), dtype),
+                              np.broadcast_to(gen.storage_to_f64(b, dtype), (M, Cout)))
+
+
+def test_linear_shapes_and_rows():
+    """Leading dimensions are flattened rows; row m of the output depends on row m of x only."""
+    rng = np.random.default_rng(6)
+    x = gen.to_storage(rng.normal(size=(2, 3, 5, 16)), "f16")
+    w = gen.to_storage(rng.normal(size=(24, 16)), "f16")
+    out = oracle.linear("f16", x, w)
+    assert out.shape == (2, 3, 5, 24)
+    assert np.array_equal(out[1, 2, 4], oracle.linear("f16", x[1, 2, 4][None], w)[0])
+    with pytest.raises(ValueError):
+        oracle.linear("f16", x, w[:, :8])
