@@ -2,7 +2,7 @@
 """Benchmark of the DCNv4 core operator on B200: one forward + backward step.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
-                    [--workload NAME] [--softmax] [--no-cpu-baseline] [--no-e2e]
+                    [--workload NAME] [--softmax] [--linear] [--no-cpu-baseline] [--no-e2e]
 
 A step is one pass of the whole path over one batch: dcn4_forward followed by
 dcn4_backward on the first-stage backbone workload (N64 H56 W56 C64 G4, C'=16,
@@ -22,6 +22,11 @@ and a CPU-oracle baseline.
 
 --softmax runs the same step with the masks normalised by a softmax over the
 K points of each (pixel, group) (the DCNv3 form of the operator).
+
+--linear adds a "linear" object: the forward with its producer fused in
+(dcn4_forward_linear: offset_mask = x W^T + b formed per tile on the tensor
+cores; fp16/bf16 workloads) against the same producer run as a separate
+library GEMM (torch.nn.functional.linear, cuBLAS) followed by dcn4_forward.
 
 --impl reference times the CPU oracle (the only other implementation of the
 operator) on the host cores, on a bounded sample of the same workload per
@@ -438,6 +443,8 @@ def run_native(args, w: gen.Workload) -> dict:
     }
     if e2e is not None:
         result["e2e"] = e2e
+    if args.linear:
+        result["linear"] = linear_leg(w, v, p, flush, stream, dev, world)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         n_img = oracle_sample_images(w, args.cpu_seconds)
         cb = time_oracle(w, n_img)
@@ -446,6 +453,62 @@ def run_native(args, w: gen.Workload) -> dict:
     if world > 1:
         dist.destroy_process_group()
     return result
+
+
+def linear_leg(w: gen.Workload, v, p, flush, stream, dev, world: int) -> dict:
+    """µs per call (CUDA events, L2 flushed before each, max over ranks): the fused
+    forward with and without storing its offset_mask, against cuBLAS's linear layer
+    followed by dcn4_forward, on seeded x [N,Ho,Wo,C], W [P,C], b [P]."""
+    import numpy as np
+    import torch
+    import torch.nn.functional as F
+    import deformable_convolution_sampling_b200 as dcn
+    tdt = {"f16": torch.float16, "bf16": torch.bfloat16}.get(w.dtype)
+    if tdt is None:
+        return {"unavailable": "the fused producer takes fp16 or bf16"}
+    lin = gen.make_linear_inputs(w, w.C)
+
+    def dev_t(a):
+        a = np.ascontiguousarray(a)
+        t = torch.from_numpy(a.view(np.int16)).view(tdt) if w.dtype == "bf16" else torch.from_numpy(a)
+        return t.to(dev)
+    x, wt, b = dev_t(lin["x"]), dev_t(lin["weight"]), dev_t(lin["bias"])
+    out = torch.empty((w.N, w.Ho, w.Wo, w.C), dtype=tdt, device=dev)
+    om = torch.empty((w.N, w.Ho, w.Wo, w.P), dtype=tdt, device=dev)
+    sh = stream.cuda_stream
+    ptr = dict(v=v.data_ptr(), x=x.data_ptr(), w=wt.data_ptr(), b=b.data_ptr(), out=out.data_ptr(),
+               om=om.data_ptr())
+
+    def fused():
+        dcn.check(dcn.dcn4_forward_linear(p, w.C, ptr["v"], ptr["x"], ptr["w"], ptr["b"], ptr["out"], None, sh))
+
+    def fused_om():
+        dcn.check(dcn.dcn4_forward_linear(p, w.C, ptr["v"], ptr["x"], ptr["w"], ptr["b"], ptr["out"], ptr["om"], sh))
+
+    def unfused():
+        torch.addmm(b, x.view(-1, w.C), wt.t(), out=om.view(-1, w.P))
+        dcn.check(dcn.dcn4_forward(p, ptr["v"], ptr["om"], ptr["out"], sh))
+
+    def linear_only():
+        torch.addmm(b, x.view(-1, w.C), wt.t(), out=om.view(-1, w.P))
+
+    res = {}
+    for name, fn in (("fused_us", fused), ("fused_with_offset_mask_out_us", fused_om),
+                     ("cublas_linear_then_forward_us", unfused), ("cublas_linear_us", linear_only)):
+        for _ in range(5):
+            fn()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(100)]
+        for e0, e1 in ev:
+            flush.zero_()
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+        torch.cuda.synchronize(dev)
+        res[name] = round(max_over_ranks(statistics.mean(a.elapsed_time(c) for a, c in ev) * 1e3, dev), 2)
+    res["speedup_vs_unfused"] = round(res["cublas_linear_then_forward_us"] / res["fused_us"], 3)
+    res["gemm"] = f"x [{w.N * w.Ho * w.Wo}, {w.C}] @ W^T [{w.C}, {w.P}] + b, mma.sync m16n8k16, fp32 accumulation"
+    res["launches_per_call"] = 1
+    return res
 
 
 def main(argv=None):
@@ -457,6 +520,8 @@ def main(argv=None):
     ap.add_argument("--workload", default="stage1_f16", choices=sorted(gen.WORKLOADS))
     ap.add_argument("--softmax", action="store_true",
                     help="masks are logits normalised by a softmax over the K points (DCNv3 form)")
+    ap.add_argument("--linear", action="store_true",
+                    help="also time the forward with the offset/mask linear layer fused in")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,

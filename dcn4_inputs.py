@@ -37,6 +37,7 @@ _M1 = np.uint64(0xBF58476D1CE4E5B9)
 _M2 = np.uint64(0x94D049BB133111EB)
 
 STREAM_VALUE, STREAM_OFFSET, STREAM_MASK, STREAM_GRAD = 1, 2, 3, 4
+STREAM_X, STREAM_WEIGHT, STREAM_BIAS = 5, 6, 7
 
 
 def _splitmix64(z: np.ndarray) -> np.ndarray:
@@ -247,6 +248,28 @@ def make_inputs(w: Workload, *, seed: int | None = None, tail_fill: float = math
         ng = w.N * w.Ho * w.Wo * w.C
         out["grad_out"] = to_storage(draw(w.grad_out, seed, STREAM_GRAD, ng), dtype).reshape(
             w.N, w.Ho, w.Wo, w.C)
+    return out
+
+
+def make_linear_inputs(w: Workload, Cx: int, *, seed: int | None = None, bias: bool = True,
+                       dtype: str | None = None) -> dict:
+    """Inputs of the merged offset/mask linear layer in front of the aggregation:
+    x [N,Ho,Wo,Cx] ~ N(0,1), weight [P,Cx] and bias [P] (or None), in storage form.
+    Weight rows are drawn N(0, s^2 / Cx) so that each produced entry has about the
+    spread of the workload's own offsets (offset rows) or masks (mask rows and the
+    padding rows); bias ~ N(0, 0.1^2)."""
+    seed = w.seed if seed is None else seed
+    dtype = w.dtype if dtype is None else dtype
+    x = to_storage(draw(("normal", 0.0, 1.0), seed, STREAM_X, w.N * w.Ho * w.Wo * Cx), dtype)
+    row_sd = np.full(w.P, float(w.mask[2]) if w.mask[0] == "normal" else 0.5)
+    off_sd = float(w.offset[2]) if w.offset[0] == "normal" else (w.offset[2] - w.offset[1]) / 12 ** 0.5
+    for g in range(w.G):
+        row_sd[g * 3 * w.K: g * 3 * w.K + 2 * w.K] = off_sd
+    z = draw(("normal", 0.0, 1.0), seed, STREAM_WEIGHT, w.P * Cx).reshape(w.P, Cx)
+    weight = to_storage(z * (row_sd[:, None] / np.sqrt(Cx)), dtype)
+    out = {"x": x.reshape(w.N, w.Ho, w.Wo, Cx), "weight": weight, "bias": None}
+    if bias:
+        out["bias"] = to_storage(draw(("normal", 0.0, 0.1), seed, STREAM_BIAS, w.P), dtype)
     return out
 
 

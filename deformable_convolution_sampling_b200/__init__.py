@@ -77,6 +77,7 @@ def _load() -> ctypes.CDLL:
         "dcn4_output_dims": ([P, ip, ip], ctypes.c_int),
         "dcn4_check_params": ([P], ctypes.c_int),
         "dcn4_forward": ([P, vp, vp, vp, vp], ctypes.c_int),
+        "dcn4_forward_linear": ([P, ctypes.c_int, vp, vp, vp, vp, vp, vp, vp], ctypes.c_int),
         "dcn4_backward_workspace_size": ([P], ctypes.c_size_t),
         "dcn4_backward": ([P, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp], ctypes.c_int),
         "dcn4_status_string": ([ctypes.c_int], ctypes.c_char_p),
@@ -126,6 +127,11 @@ def dcn4_check_params(p: dcn4_params) -> int:
 
 def dcn4_forward(p: dcn4_params, value, offset_mask, out, stream=None) -> int:
     return lib.dcn4_forward(ctypes.byref(p), value, offset_mask, out, stream)
+
+
+def dcn4_forward_linear(p: dcn4_params, Cx: int, value, x, weight, bias, out, offset_mask_out=None,
+                        stream=None) -> int:
+    return lib.dcn4_forward_linear(ctypes.byref(p), int(Cx), value, x, weight, bias, out, offset_mask_out, stream)
 
 
 def dcn4_backward_workspace_size(p: dcn4_params) -> int:
@@ -203,6 +209,22 @@ def forward(p: dcn4_params, value, offset_mask, out=None):
         out = torch.empty((p.N, Ho, Wo, p.G * p.Cg), dtype=_torch_dtype(p.dtype), device=value.device)
     check(dcn4_forward(p, value.data_ptr(), offset_mask.data_ptr(), out.data_ptr(),
                        _stream_handle(value.device)))
+    return out
+
+
+def forward_linear(p: dcn4_params, value, x, weight, bias=None, out=None, offset_mask_out=None):
+    """y[N,Ho,Wo,C] with the offset_mask formed in the kernel as x @ weight.T + bias
+    (x [N,Ho,Wo,Cx], weight [P,Cx], bias [P] or None); offset_mask_out, when given
+    ([N,Ho,Wo,P]), receives that offset_mask.  CUDA tensors, fp16 or bf16."""
+    import torch
+    st, Ho, Wo = dcn4_output_dims(p)
+    check(st)
+    if out is None:
+        out = torch.empty((p.N, Ho, Wo, p.G * p.Cg), dtype=_torch_dtype(p.dtype), device=value.device)
+    check(dcn4_forward_linear(p, x.shape[-1], value.data_ptr(), x.data_ptr(), weight.data_ptr(),
+                              bias.data_ptr() if bias is not None else None, out.data_ptr(),
+                              offset_mask_out.data_ptr() if offset_mask_out is not None else None,
+                              _stream_handle(value.device)))
     return out
 
 

@@ -286,6 +286,29 @@ int dcn4_forward(const dcn4_params* p, const void* value, const void* offset_mas
     return DCN4_OK;
 }
 
+int dcn4_forward_linear(const dcn4_params* p, int Cx, const void* value, const void* x, const void* weight,
+                        const void* bias, void* out, void* offset_mask_out, void* stream) {
+    dcn4::Geometry g;
+    const int st = make_geometry(p, false, aligned32(value) && aligned32(out), &g);
+    if (st != DCN4_OK) return st;
+    if (p->dtype == DCN4_F32) return fail(DCN4_ERR_UNSUPPORTED, "the fused linear producer takes fp16 or bf16");
+    if (Cx < 16 || Cx % 16 != 0 || Cx > (1 << 16))
+        return fail(DCN4_ERR_BAD_SHAPE, "Cx=%d must be a positive multiple of 16", Cx);
+    if (dcn4::forward_linear_smem_bytes(g, Cx, dcn4::forward_linear_w_smem(g, Cx)) > kSmemMax)
+        return fail(DCN4_ERR_UNSUPPORTED, "x rows of Cx=%d with P=%d do not fit shared memory", Cx, p->P);
+    if (static_cast<long long>(g.Ho) * g.Wo * Cx >= (1LL << 31) || static_cast<long long>(p->P) * Cx >= (1LL << 31))
+        return fail(DCN4_ERR_UNSUPPORTED, "x or weight too large");
+    if (g.total_pix == 0) return DCN4_OK;
+    if (!value || !x || !weight || !out) return fail(DCN4_ERR_NULL, "value, x, weight and out must be non-NULL");
+    if (!aligned16(value) || !aligned16(x) || !aligned16(weight) || !aligned16(out) || !aligned16(bias) ||
+        !aligned16(offset_mask_out))
+        return fail(DCN4_ERR_MISALIGNED, "every pointer must be 16-byte aligned");
+    const cudaError_t e = dcn4::launch_forward_linear(g, p->dtype, value, x, weight, bias, out, offset_mask_out, Cx,
+                                                      static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return fail(DCN4_ERR_LAUNCH, "forward_linear launch: %s", cudaGetErrorString(e));
+    return DCN4_OK;
+}
+
 size_t dcn4_backward_workspace_size(const dcn4_params* p) {
     dcn4::Geometry g;
     if (make_geometry(p, true, true, &g) != DCN4_OK) return 0;

@@ -347,6 +347,13 @@ cudaError_t launch_backward_value(const Geometry& g, int dtype, const void* om, 
 inline int samples_threads(const Geometry& g) { return (g.pix_per_cta * g.G * g.nslice + 31) / 32 * 32; }
 // Dynamic shared memory bytes of one CTA.
 size_t forward_smem_bytes(const Geometry& g, int elem_bytes);
+// Forward with the linear producer (16-bit dtypes): offset_mask = x W^T + b per
+// tile, x [N, Ho, Wo, Cx], w [P, Cx], b [P] or null, om_out [N, Ho, Wo, P] or null.
+cudaError_t launch_forward_linear(const Geometry& g, int dtype, const void* value, const void* x, const void* w,
+                                  const void* b, void* out, void* om_out, int Cx, cudaStream_t stream);
+size_t forward_linear_smem_bytes(const Geometry& g, int Cx, bool w_smem);
+// Whether the fused forward stages W in shared memory for this shape.
+bool forward_linear_w_smem(const Geometry& g, int Cx);
 size_t backward_smem_bytes(const Geometry& g, int elem_bytes);
 size_t backward_value_smem_bytes(const Geometry& g);
 }  // namespace dcn4

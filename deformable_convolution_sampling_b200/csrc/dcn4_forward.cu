@@ -21,8 +21,17 @@
 // masks are logits: before its samples each thread takes the K exponentials of
 // its (pixel, group)'s logits once, into its own slots of shared memory (no
 // barrier), and the samples read their weights from there.
+//
+// Fused producer (LIN).  The DCNv4 module computes the offsets and dynamic
+// weights with one merged linear layer (CSDN summary, section 2.2 "DCN模块的微设计"):
+// offset_mask = x W^T + b.  With LIN the kernel stages the tile's rows of x
+// instead (cp.async, double buffered), forms the tile's offset_mask rows on
+// the tensor cores (mma.sync m16n8k16, fp32 accumulation, bias added, rounded
+// once to the I/O dtype) into shared memory, optionally stores them, and
+// samples them as above: the offset_mask never makes a round trip through HBM.
 #include <algorithm>
 #include <atomic>
+#include <type_traits>
 
 #include "dcn4_common.cuh"
 
@@ -52,6 +61,195 @@ __device__ __forceinline__ void accumulate(float2* acc, const T* src, float wt) 
 
 // CTAs per SM the forward kernel is compiled for (80 registers a thread).
 constexpr int kFwdCtasPerSm = 3;
+
+// Arguments of the fused producer: x [N, Ho, Wo, Cx], w [P, Cx] (nn.Linear
+// layout), b [P] or null, om_out [N, Ho, Wo, P] or null.
+template <typename T>
+struct LinearArgs {
+    const T* x;
+    const T* w;
+    const T* b;
+    T* om_out;
+    int Cx;
+    int w_smem;  // 1: W is staged in shared memory once per CTA (when it fits)
+};
+
+// Rows of a staged x tile: the tile's pixels rounded up to whole 16-row MMA tiles.
+__host__ __device__ inline int linear_rows(const Geometry& g) { return (g.TH * g.TW + 15) / 16 * 16; }
+// Elements per staged x (and W) row: 8 of padding keep ldmatrix's eight row reads on distinct banks.
+__host__ __device__ inline int linear_ld(int Cx) { return Cx + 8; }
+// Column tiles (of 8 outputs) one GEMM item covers.
+constexpr int kLinNB = 4;
+// Rows of a staged W: whole items of kLinNB column tiles.
+__host__ __device__ inline int linear_w_rows(const Geometry& g) { return (g.P / 8 + kLinNB - 1) / kLinNB * kLinNB * 8; }
+
+__device__ __forceinline__ void ldmatrix_x4(uint32_t* r, unsigned addr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+
+// d += a (16x16, row-major fragment) * b (16x8, column fragment), fp32 accumulation.
+template <typename T>
+__device__ __forceinline__ void mma_16816(float* d, const uint32_t* a, const uint32_t* b) {
+    if constexpr (std::is_same<T, __half>::value) {
+        asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+                     "{%0, %1, %2, %3};"
+                     : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+                     : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+    } else {
+        asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+                     "{%0, %1, %2, %3};"
+                     : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+                     : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+    }
+}
+
+template <typename T>
+__device__ __forceinline__ uint32_t pack2(float lo, float hi) {
+    uint32_t u;
+    if constexpr (std::is_same<T, __half>::value) {
+        const __half2 h = __floats2half2_rn(lo, hi);
+        memcpy(&u, &h, 4);
+    } else {
+        const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+        memcpy(&u, &h, 4);
+    }
+    return u;
+}
+
+// The tile's rows of x into shared memory [rows][Cx + 8] with cp.async.
+template <typename T>
+__device__ __forceinline__ void stage_x_async(T* dst, const LinearArgs<T>& lin, const Geometry& g, const Tile& t) {
+    constexpr int EPV = Elem<T>::per16;
+    const int cpp = lin.Cx / EPV;  // 16-byte chunks per pixel
+    const int total = t.th * t.tw * cpp;
+    const int ld = linear_ld(lin.Cx);
+    for (int i = threadIdx.x; i < total; i += blockDim.x) {
+        const int q = i / cpp, c = i - q * cpp;
+        const int py = q / t.tw, px = q - py * t.tw;
+        const long long pix = (static_cast<long long>(t.n) * g.Ho + t.ho0 + py) * g.Wo + t.wo0 + px;
+        const T* sp = lin.x + pix * lin.Cx + c * EPV;
+        T* d = dst + (py * g.TW + px) * ld + c * EPV;
+        const unsigned da = static_cast<unsigned>(__cvta_generic_to_shared(d));
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(da), "l"(sp));
+    }
+    asm volatile("cp.async.commit_group;");
+}
+
+template <typename T>
+__device__ __forceinline__ void store_pair_rows(T* om_s, const Geometry& g, int rows, int mt, int col, const float* acc,
+                                                const float* b_s) {
+    const int lane = threadIdx.x & 31;
+    const float2 bb = *reinterpret_cast<const float2*>(b_s + col);
+    const int r0 = mt * 16 + (lane >> 2), r1 = r0 + 8;
+    if (r0 < rows) *reinterpret_cast<uint32_t*>(om_s + r0 * g.P + col) = pack2<T>(acc[0] + bb.x, acc[1] + bb.y);
+    if (r1 < rows) *reinterpret_cast<uint32_t*>(om_s + r1 * g.P + col) = pack2<T>(acc[2] + bb.x, acc[3] + bb.y);
+}
+
+// om_s = round(x_s W^T + b) with W staged and KS = Cx / 16 k-steps known at
+// compile time: a warp keeps one 16-row tile's A fragments for all k-steps in
+// registers and walks its share of the 8-column tiles, loading each tile's B
+// fragments two k-steps per ldmatrix.
+template <typename T, int KS>
+__device__ __forceinline__ void linear_tile_staged(const Geometry& g, const LinearArgs<T>& lin, const T* x_s,
+                                                   const T* w_s, T* om_s, const float* b_s) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    const int rows = g.TH * g.TW;
+    const int MT = linear_rows(g) / 16, NT = g.P / 8;
+    const int ld = linear_ld(lin.Cx);
+    const int wpm = max(1, nw / MT);  // warps per 16-row tile
+    const int sub = warp % wpm;
+    for (int mt = warp / wpm; mt < MT; mt += nw / wpm) {
+        uint32_t a[KS][4];
+        const unsigned a_addr =
+            static_cast<unsigned>(__cvta_generic_to_shared(x_s + (mt * 16 + (lane & 15)) * ld + (lane >> 4) * 8));
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) ldmatrix_x4(a[ks], a_addr + ks * 32);
+        // lane l: row l % 8 of the column tile, k offset 8 * (l / 8) within two k-steps
+        const unsigned b_base =
+            static_cast<unsigned>(__cvta_generic_to_shared(w_s + (lane & 7) * ld + (lane >> 3) * 8));
+        for (int nt = sub; nt < NT; nt += wpm) {
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+            const unsigned b_addr = b_base + nt * 8 * ld * 2;
+#pragma unroll
+            for (int ks = 0; ks < KS; ks += 2) {
+                uint32_t b[4];
+                if constexpr (KS == 1) {
+                    asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0, %1}, [%2];"
+                                 : "=r"(b[0]), "=r"(b[1])
+                                 : "r"(b_addr));
+                } else {
+                    ldmatrix_x4(b, b_addr + ks * 32);
+                }
+                mma_16816<T>(acc, a[ks], b);
+                if constexpr (KS > 1) mma_16816<T>(acc, a[ks + 1], b + 2);
+            }
+            store_pair_rows<T>(om_s, g, rows, mt, nt * 8 + (lane & 3) * 2, acc, b_s);
+        }
+    }
+}
+
+// om_s [TH*TW][P] = round(x_s W^T + b) for the tile: warps take (16-row tile,
+// 4 column tiles of 8) items; A fragments come from shared memory (ldmatrix),
+// B fragments from the staged W (ldmatrix, two column tiles per instruction)
+// or, when W does not fit shared memory, straight from global memory.
+template <typename T>
+__device__ __forceinline__ void linear_tile(const Geometry& g, const LinearArgs<T>& lin, const T* x_s, const T* w_s,
+                                            T* om_s, const float* b_s) {
+    constexpr int NB = kLinNB;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    const int rows = g.TH * g.TW;
+    const int MT = linear_rows(g) / 16, NT = g.P / 8, KS = lin.Cx / 16;
+    const int NCH = (NT + NB - 1) / NB;
+    const int ld = linear_ld(lin.Cx);
+    const int gq = lane >> 2, tq = lane & 3;
+    for (int item = warp; item < MT * NCH; item += nw) {
+        const int mt = item / NCH, nt0 = (item - mt * NCH) * NB;
+        float acc[NB][4];
+#pragma unroll
+        for (int j = 0; j < NB; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+        // lane l reads row l % 16 of the 16-row tile, column half l / 16
+        const unsigned a_addr =
+            static_cast<unsigned>(__cvta_generic_to_shared(x_s + (mt * 16 + (lane & 15)) * ld + (lane >> 4) * 8));
+        if (lin.w_smem) {
+            // lanes 0-7 / 8-15: rows of column tile nt, k halves 0 / 1; lanes 16-31: column tile nt + 1
+            const int brow = (lane & 7) + ((lane >> 4) << 3), bcol = ((lane >> 3) & 1) * 8;
+            const unsigned b_addr = static_cast<unsigned>(__cvta_generic_to_shared(w_s + (nt0 * 8 + brow) * ld + bcol));
+            for (int ks = 0; ks < KS; ++ks) {
+                uint32_t a[4], b[NB / 2][4];
+                ldmatrix_x4(a, a_addr + ks * 32);
+#pragma unroll
+                for (int jj = 0; jj < NB / 2; ++jj) ldmatrix_x4(b[jj], b_addr + (jj * 16 * ld + ks * 16) * 2);
+#pragma unroll
+                for (int j = 0; j < NB; ++j)
+                    if (nt0 + j < NT) mma_16816<T>(acc[j], a, &b[j >> 1][(j & 1) * 2]);  // uniform over the warp
+            }
+        } else {
+            for (int ks = 0; ks < KS; ++ks) {
+                uint32_t a[4];
+                ldmatrix_x4(a, a_addr + ks * 32);
+#pragma unroll
+                for (int j = 0; j < NB; ++j) {
+                    if (nt0 + j >= NT) break;  // uniform over the warp
+                    const T* wr = lin.w + static_cast<long long>((nt0 + j) * 8 + gq) * lin.Cx + ks * 16 + tq * 2;
+                    const uint32_t b[2] = {__ldg(reinterpret_cast<const unsigned*>(wr)),
+                                           __ldg(reinterpret_cast<const unsigned*>(wr + 8))};
+                    mma_16816<T>(acc[j], a, b);
+                }
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < NB; ++j) {
+            if (nt0 + j >= NT) break;
+            const int col = (nt0 + j) * 8 + tq * 2;
+            const float b0 = b_s[col], b1 = b_s[col + 1];
+            const int r0 = mt * 16 + gq, r1 = r0 + 8;
+            if (r0 < rows) *reinterpret_cast<uint32_t*>(om_s + r0 * g.P + col) = pack2<T>(acc[j][0] + b0, acc[j][1] + b1);
+            if (r1 < rows) *reinterpret_cast<uint32_t*>(om_s + r1 * g.P + col) = pack2<T>(acc[j][2] + b0, acc[j][3] + b1);
+        }
+    }
+}
 
 // SM count of the current device, queried once per device.
 cudaError_t sm_count(int* out) {
@@ -106,23 +304,56 @@ __device__ __forceinline__ void stage_tile_async(T* dst_smem, const T* src, cons
 }
 
 // Persistent: a CTA per resident slot loops over the output tiles (tile,
-// tile + gridDim.x, ...), copying the next tile's offset_mask rows into the
-// other half of a double buffer (cp.async) while it computes the current one.
-// KH, KW > 0: compile-time grid size (fully unrolled) and RC = remove_center;
-// KH = KW = 0: sizes and remove_center from g.  SM: softmax over the K masks.
-template <typename T, int VEC, int KH, int KW, bool RC, bool SM>
+// tile + gridDim.x, ...), copying the next tile's offset_mask rows (LIN: x
+// rows) into the other half of a double buffer (cp.async) while it computes
+// the current one.  KH, KW > 0: compile-time grid size (fully unrolled) and
+// RC = remove_center; KH = KW = 0: sizes and remove_center from g.  SM:
+// softmax over the K masks.  LIN: offset_mask rows from the linear producer.
+template <typename T, int VEC, int KH, int KW, bool RC, bool SM, bool LIN>
 __global__ void __launch_bounds__(256, kFwdCtasPerSm) forward_kernel(const Geometry g, const T* __restrict__ value,
-                                                      const T* __restrict__ om, T* __restrict__ out) {
+                                                      const T* __restrict__ om, T* __restrict__ out,
+                                                      const LinearArgs<T> lin) {
     extern __shared__ __align__(16) unsigned char smem[];
     constexpr int EPV = Elem<T>::per16;
     constexpr int PAIRS = VEC * EPV / 2;
     const int tile_elems = g.TH * g.TW * g.P;
-    T* bufs[2] = {reinterpret_cast<T*>(smem), reinterpret_cast<T*>(smem) + tile_elems};
-    float* e_s = reinterpret_cast<float*>(bufs[1] + tile_elems);  // softmax exponentials [K][threads]
+    // plain: two offset_mask tiles; LIN: one offset_mask tile, two x tiles, W (when
+    // staged), the bias (fp32)
+    T* bufs[2];
+    T* xbuf[2] = {nullptr, nullptr};
+    T* w_s = nullptr;
+    float* b_s = nullptr;
+    float* e_s;  // softmax exponentials [K][threads]
+    if constexpr (LIN) {
+        const int xs = linear_rows(g) * linear_ld(lin.Cx);
+        bufs[0] = bufs[1] = reinterpret_cast<T*>(smem);
+        xbuf[0] = bufs[0] + tile_elems;
+        xbuf[1] = xbuf[0] + xs;
+        w_s = xbuf[1] + xs;
+        b_s = reinterpret_cast<float*>(w_s + (lin.w_smem ? linear_w_rows(g) * linear_ld(lin.Cx) : 0));
+        e_s = b_s + g.P;
+    } else {
+        bufs[0] = reinterpret_cast<T*>(smem);
+        bufs[1] = bufs[0] + tile_elems;
+        e_s = reinterpret_cast<float*>(bufs[1] + tile_elems);
+    }
     const int ntiles = g.N * g.tiles_h * g.tiles_w;
     int tile = blockIdx.x;
     if (tile >= ntiles) return;
-    stage_tile_async(bufs[0], om, g, tile_at(g, tile));
+    if constexpr (LIN) {
+        for (int j = threadIdx.x; j < g.P; j += blockDim.x) b_s[j] = lin.b ? to_f32(lin.b[j]) : 0.f;
+        if (lin.w_smem) {  // W rows [P][Cx] -> [rows][Cx + 8]; rows past P stay unset (their columns are dropped)
+            const int cpr = lin.Cx / EPV;
+            for (int i = threadIdx.x; i < g.P * cpr; i += blockDim.x) {
+                const int r = i / cpr, c = i - r * cpr;
+                *reinterpret_cast<uint4*>(w_s + r * linear_ld(lin.Cx) + c * EPV) =
+                    ld_gather(lin.w + static_cast<long long>(r) * lin.Cx + c * EPV);
+            }
+        }
+        stage_x_async(xbuf[0], lin, g, tile_at(g, tile));
+    } else {
+        stage_tile_async(bufs[0], om, g, tile_at(g, tile));
+    }
 
     const int lanes_pp = g.G * g.nslice;
     const int lp = threadIdx.x / lanes_pp;
@@ -140,7 +371,11 @@ __global__ void __launch_bounds__(256, kFwdCtasPerSm) forward_kernel(const Geome
     for (int it = 0; tile < ntiles; ++it, tile += gridDim.x) {
         const int next = tile + gridDim.x;
         if (next < ntiles) {
-            stage_tile_async(bufs[(it + 1) & 1], om, g, tile_at(g, next));
+            if constexpr (LIN) {
+                stage_x_async(xbuf[(it + 1) & 1], lin, g, tile_at(g, next));
+            } else {
+                stage_tile_async(bufs[(it + 1) & 1], om, g, tile_at(g, next));
+            }
             asm volatile("cp.async.wait_group 1;" ::: "memory");
         } else {
             asm volatile("cp.async.wait_group 0;" ::: "memory");
@@ -148,6 +383,26 @@ __global__ void __launch_bounds__(256, kFwdCtasPerSm) forward_kernel(const Geome
         __syncthreads();
         const Tile t = tile_at(g, tile);
         const T* om_s = bufs[it & 1];
+        if constexpr (LIN) {
+            switch (lin.w_smem ? lin.Cx / 16 : 0) {
+                case 1: linear_tile_staged<T, 1>(g, lin, xbuf[it & 1], w_s, bufs[0], b_s); break;
+                case 2: linear_tile_staged<T, 2>(g, lin, xbuf[it & 1], w_s, bufs[0], b_s); break;
+                case 4: linear_tile_staged<T, 4>(g, lin, xbuf[it & 1], w_s, bufs[0], b_s); break;
+                case 8: linear_tile_staged<T, 8>(g, lin, xbuf[it & 1], w_s, bufs[0], b_s); break;
+                default: linear_tile(g, lin, xbuf[it & 1], w_s, bufs[0], b_s);
+            }
+            __syncthreads();
+            if (lin.om_out) {  // the rows the samples use, 16-byte stores
+                const int cpp = g.P / EPV;
+                for (int i = threadIdx.x; i < t.th * t.tw * cpp; i += blockDim.x) {
+                    const int q = i / cpp, c = i - q * cpp;
+                    const int qy = q / t.tw, qx = q - qy * t.tw;
+                    const long long pix = (static_cast<long long>(t.n) * g.Ho + t.ho0 + qy) * g.Wo + t.wo0 + qx;
+                    st_global(lin.om_out + pix * g.P + c * EPV,
+                              *reinterpret_cast<const uint4*>(bufs[0] + (qy * g.TW + qx) * g.P + c * EPV));
+                }
+            }
+        }
         if (py < t.th && px < t.tw) {
             const int ho = t.ho0 + py, wo = t.wo0 + px;
             const T* row = om_s + lp * g.P + grp * 3 * K;
@@ -188,14 +443,15 @@ __global__ void __launch_bounds__(256, kFwdCtasPerSm) forward_kernel(const Geome
                 st_global(dst, pack(acc, T()));
             }
         }
-        __syncthreads();  // the buffer is refilled two tiles later
+        __syncthreads();  // the buffer is refilled two tiles later (LIN: om_s at the next tile)
     }
 }
 
-template <typename T, int VEC, int KH, int KW, bool RC, bool SM>
-cudaError_t launch_typed(const Geometry& g, const void* value, const void* om, void* out, cudaStream_t stream) {
-    const size_t smem = forward_smem_bytes(g, sizeof(T));
-    auto kern = forward_kernel<T, VEC, KH, KW, RC, SM>;
+template <typename T, int VEC, int KH, int KW, bool RC, bool SM, bool LIN>
+cudaError_t launch_typed(const Geometry& g, const void* value, const void* om, void* out, const LinearArgs<T>& lin,
+                         cudaStream_t stream) {
+    const size_t smem = LIN ? forward_linear_smem_bytes(g, lin.Cx, lin.w_smem != 0) : forward_smem_bytes(g, sizeof(T));
+    auto kern = forward_kernel<T, VEC, KH, KW, RC, SM, LIN>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     const int threads = (g.pix_per_cta * g.G * g.nslice + 31) / 32 * 32;
@@ -208,32 +464,69 @@ cudaError_t launch_typed(const Geometry& g, const void* value, const void* om, v
     const long long per_sm = std::max<long long>(1, std::min<long long>(kFwdCtasPerSm, by_smem));
     const long long ntiles = static_cast<long long>(g.N) * g.tiles_h * g.tiles_w;
     const long long blocks = std::min<long long>(ntiles, per_sm * sms);
-    kern<<<static_cast<unsigned>(blocks), threads, smem, stream>>>(g, static_cast<const T*>(value),
-                                                                   static_cast<const T*>(om), static_cast<T*>(out));
+    kern<<<static_cast<unsigned>(blocks), threads, smem, stream>>>(
+        g, static_cast<const T*>(value), static_cast<const T*>(om), static_cast<T*>(out), lin);
     return cudaGetLastError();
 }
 
-template <typename T, int VEC, bool SM>
-cudaError_t launch_grid(const Geometry& g, const void* value, const void* om, void* out, cudaStream_t stream) {
+template <typename T, int VEC, bool SM, bool LIN>
+cudaError_t launch_grid(const Geometry& g, const void* value, const void* om, void* out, const LinearArgs<T>& lin,
+                        cudaStream_t stream) {
     if (g.kh == 3 && g.kw == 3) {
-        return g.remove_center ? launch_typed<T, VEC, 3, 3, true, SM>(g, value, om, out, stream)
-                               : launch_typed<T, VEC, 3, 3, false, SM>(g, value, om, out, stream);
+        return g.remove_center ? launch_typed<T, VEC, 3, 3, true, SM, LIN>(g, value, om, out, lin, stream)
+                               : launch_typed<T, VEC, 3, 3, false, SM, LIN>(g, value, om, out, lin, stream);
     }
-    return launch_typed<T, VEC, 0, 0, false, SM>(g, value, om, out, stream);
+    return launch_typed<T, VEC, 0, 0, false, SM, LIN>(g, value, om, out, lin, stream);
 }
 
-template <typename T, int VEC>
-cudaError_t launch_softmax(const Geometry& g, const void* value, const void* om, void* out, cudaStream_t stream) {
-    return g.softmax ? launch_grid<T, VEC, true>(g, value, om, out, stream)
-                     : launch_grid<T, VEC, false>(g, value, om, out, stream);
+template <typename T, int VEC, bool LIN>
+cudaError_t launch_softmax(const Geometry& g, const void* value, const void* om, void* out, const LinearArgs<T>& lin,
+                           cudaStream_t stream) {
+    return g.softmax ? launch_grid<T, VEC, true, LIN>(g, value, om, out, lin, stream)
+                     : launch_grid<T, VEC, false, LIN>(g, value, om, out, lin, stream);
 }
 
-template <typename T>
-cudaError_t launch_vec(const Geometry& g, int vec, const void* value, const void* om, void* out, cudaStream_t stream) {
-    return vec == 2 ? launch_softmax<T, 2>(g, value, om, out, stream) : launch_softmax<T, 1>(g, value, om, out, stream);
+template <typename T, bool LIN = false>
+cudaError_t launch_vec(const Geometry& g, int vec, const void* value, const void* om, void* out,
+                       const LinearArgs<T>& lin, cudaStream_t stream) {
+    return vec == 2 ? launch_softmax<T, 2, LIN>(g, value, om, out, lin, stream)
+                    : launch_softmax<T, 1, LIN>(g, value, om, out, lin, stream);
 }
 
 }  // namespace
+
+size_t forward_linear_smem_bytes(const Geometry& g, int Cx, bool w_smem) {
+    const size_t xs = static_cast<size_t>(linear_rows(g)) * linear_ld(Cx) * 2;  // 16-bit dtypes only
+    const size_t ws = w_smem ? static_cast<size_t>(linear_w_rows(g)) * linear_ld(Cx) * 2 : 0;
+    return static_cast<size_t>(g.pix_per_cta) * g.P * 2 + 2 * xs + ws + static_cast<size_t>(g.P) * sizeof(float) +
+           (g.softmax ? static_cast<size_t>(g.K) * samples_threads(g) * sizeof(float) : 0);
+}
+
+bool forward_linear_w_smem(const Geometry& g, int Cx) {
+    // W is staged when the CTA still fits three to an SM (the sampler's occupancy)
+    return forward_linear_smem_bytes(g, Cx, true) + 1024 <= 227 * 1024 / kFwdCtasPerSm;
+}
+
+cudaError_t launch_forward_linear(const Geometry& g, int dtype, const void* value, const void* x, const void* w,
+                                  const void* b, void* out, void* om_out, int Cx, cudaStream_t stream) {
+    switch (dtype) {
+        case 1: {
+            const LinearArgs<__half> lin{static_cast<const __half*>(x), static_cast<const __half*>(w),
+                                         static_cast<const __half*>(b), static_cast<__half*>(om_out), Cx,
+                                         forward_linear_w_smem(g, Cx) ? 1 : 0};
+            return launch_vec<__half, true>(g, g.vec, value, nullptr, out, lin, stream);
+        }
+        case 2: {
+            const LinearArgs<__nv_bfloat16> lin{static_cast<const __nv_bfloat16*>(x),
+                                                static_cast<const __nv_bfloat16*>(w),
+                                                static_cast<const __nv_bfloat16*>(b),
+                                                static_cast<__nv_bfloat16*>(om_out), Cx,
+                                                forward_linear_w_smem(g, Cx) ? 1 : 0};
+            return launch_vec<__nv_bfloat16, true>(g, g.vec, value, nullptr, out, lin, stream);
+        }
+        default: return cudaErrorInvalidValue;
+    }
+}
 
 size_t forward_smem_bytes(const Geometry& g, int elem_bytes) {
     return 2 * static_cast<size_t>(g.pix_per_cta) * g.P * elem_bytes +                        // double buffer
@@ -244,9 +537,9 @@ cudaError_t launch_forward(const Geometry& g, int dtype, const void* value, cons
                            cudaStream_t stream) {
     const int vec = g.vec;
     switch (dtype) {
-        case 0: return launch_vec<float>(g, vec, value, om, out, stream);
-        case 1: return launch_vec<__half>(g, vec, value, om, out, stream);
-        case 2: return launch_vec<__nv_bfloat16>(g, vec, value, om, out, stream);
+        case 0: return launch_vec<float>(g, vec, value, om, out, LinearArgs<float>{}, stream);
+        case 1: return launch_vec<__half>(g, vec, value, om, out, LinearArgs<__half>{}, stream);
+        case 2: return launch_vec<__nv_bfloat16>(g, vec, value, om, out, LinearArgs<__nv_bfloat16>{}, stream);
         default: return cudaErrorInvalidValue;
     }
 }

@@ -67,7 +67,7 @@
 extern "C" {
 #endif
 
-#define DCN4_VERSION 110  /* 1.1.0: dcn4_params.softmax */
+#define DCN4_VERSION 120  /* 1.2.0: dcn4_forward_linear */
 
 typedef enum {
     DCN4_F32 = 0,   /* IEEE binary32            */
@@ -125,6 +125,29 @@ int dcn4_check_params(const dcn4_params* p);
  * One kernel launch on `stream`. */
 int dcn4_forward(const dcn4_params* p, const void* value, const void* offset_mask, void* out,
                  void* stream);
+
+/* Forward with its producer fused in: the merged offset/mask linear layer of
+ * the DCNv4 module (CSDN summary, section 2.2 "DCN模块的微设计": one linear layer
+ * gives the offsets and the dynamic weights; with latency first the depthwise
+ * convolution before it is dropped), then the aggregation:
+ *     offset_mask[n, ho, wo, j] = round_dtype( sum_c x[n, ho, wo, c] * weight[j, c] + bias[j] )
+ *     out = dcn4_forward(value, offset_mask)
+ * formed tile by tile in the kernel (tensor cores, fp32 accumulation, the bias
+ * added in fp32, one rounding to dtype), so the offset_mask is never read from
+ * HBM.  One kernel launch on `stream`.
+ *   x                [N, Ho, Wo, Cx]  dtype: the features of each output pixel
+ *   weight           [P, Cx]          dtype (nn.Linear layout: row j gives entry j)
+ *   bias             [P]              dtype, or NULL for none
+ *   out              [N, Ho, Wo, C]   dtype
+ *   offset_mask_out  [N, Ho, Wo, P]   dtype, or NULL: receives the offset_mask the
+ *                                     samples used (for a later dcn4_backward)
+ * Rows [G*3K, P) of weight give the padding entries: computed (and stored in
+ * offset_mask_out), never sampled.  fp16 and bf16 only (DCN4_ERR_UNSUPPORTED for
+ * fp32); Cx a multiple of 16 (DCN4_ERR_BAD_SHAPE otherwise) whose staged tiles
+ * fit shared memory (DCN4_ERR_UNSUPPORTED otherwise); every non-NULL pointer
+ * 16-byte aligned.  The same checks as dcn4_forward otherwise. */
+int dcn4_forward_linear(const dcn4_params* p, int Cx, const void* value, const void* x, const void* weight,
+                        const void* bias, void* out, void* offset_mask_out, void* stream);
 
 /* Bytes of device workspace dcn4_backward needs, each part rounded up to 256
  * bytes: one 32-bit word per image, one 32-bit cell box per output pixel

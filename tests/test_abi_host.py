@@ -60,7 +60,7 @@ def test_params_mirror_matches_the_header(dcn):
             fields += [n.strip() for n in names.split(",")]
     assert [f[0] for f in dcn.dcn4_params._fields_] == fields
     assert ctypes.sizeof(dcn.dcn4_params) == 4 * len(fields)
-    assert dcn.dcn4_version() == 110
+    assert dcn.dcn4_version() == 120
 
 
 def test_library_does_not_link_the_oracle(dcn):
@@ -128,6 +128,27 @@ def test_invalid_params_are_rejected_before_launch(dcn, field, value, status):
     assert dcn.dcn4_check_params(p) == status
     # pointers that would fault if used: the call must fail before any launch
     assert dcn.dcn4_forward(p, 16, 32, 48, None) == status
+    assert dcn.dcn4_last_error() != ""
+
+
+def test_forward_linear_checks_before_launch(dcn):
+    """dcn4_forward_linear validates on the host: pointers that would fault are never used."""
+    p = dcn.make_params(N=2, H=8, W=8, G=4, Cg=16, dtype="f16")
+    ok = dict(value=16, x=32, weight=48, bias=None, out=64, om=None)
+
+    def call(params, Cx, **kw):
+        a = {**ok, **kw}
+        return dcn.dcn4_forward_linear(params, Cx, a["value"], a["x"], a["weight"], a["bias"], a["out"], a["om"],
+                                       None)
+    p32 = dcn.make_params(N=2, H=8, W=8, G=4, Cg=16, dtype="f32")
+    assert call(p32, 64) == -5                      # fp32: no fused producer
+    assert call(p, 24) == -2 and call(p, 0) == -2   # Cx not a multiple of 16
+    assert call(p, 1 << 14) == -5                   # x tiles too large for shared memory
+    assert call(p, 64, x=None) == -1
+    assert call(p, 64, bias=40) == -4 and call(p, 64, om=72) == -4 and call(p, 64, x=36) == -4
+    bad = dcn.make_params(N=2, H=8, W=8, G=4, Cg=16, dtype="f16")
+    bad.P = 100
+    assert call(bad, 64) == -3
     assert dcn.dcn4_last_error() != ""
 
 
