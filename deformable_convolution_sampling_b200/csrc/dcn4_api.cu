@@ -44,8 +44,9 @@ constexpr size_t kValueSmem = 112 * 1024;
 constexpr int kValueMaxBH = 16;    // input rows per tile at most
 constexpr int kValueMaxGK = 512;   // groups x points at most
 // grad_offset_mask pass: shared memory at most for its offset_mask tiles plus
-// the staging of the records it files (beyond it the grad_value pass rescans).
-constexpr size_t kFileSmem = 96 * 1024;
+// the staging of the records it files (beyond it the grad_value pass rescans,
+// which for large grids costs far more than the CTAs per SM the staging takes).
+constexpr size_t kFileSmem = 200 * 1024;
 // Static shared memory of the grad_offset_mask kernel (per-pixel boxes and the
 // filing counters), an upper bound.
 constexpr size_t kSamplesStaticSmem = 8 * 1024;
@@ -188,6 +189,17 @@ int make_geometry(const dcn4_params* p, bool backward, bool wide, dcn4::Geometry
     const long long nbins = static_cast<long long>(p->G) * (BH + 1) * (BW + 1);
     g->buckets = eb == 2 && Ho <= 65535 && Wo <= 65535 && nbins <= 65535;
 
+    // Filing window (64 grad_value tiles): enough tile rows for the rows a CTA's
+    // samples span -- its TH output rows, the grid, and about 8 pixels of
+    // offsets either way -- the rest of the 64 as columns.
+    {
+        const long long span = (TH - 1) * p->sh + static_cast<long long>(p->kh - 1) * p->dh + 2 * 8 + 2;
+        const long long need = (span + BH - 1) / BH + 1;
+        int wl = 3;  // 8 x 8, and always for 3 x 3 grids, whose kernels are compiled for it
+        while (wl > 0 && (64 >> wl) < need && !(p->kh == 3 && p->kw == 3)) --wl;
+        g->fwin_wl = wl;
+        g->fwin_h = 64 >> wl;
+    }
     g->bh_magic = 0xffffffffu / static_cast<uint32_t>(BH) + 1u;  // BH, BW >= 2 use __umulhi; 1 is special-cased
     g->bw_magic = 0xffffffffu / static_cast<uint32_t>(BW) + 1u;
     // ... and when the grad_offset_mask CTA can stage its records in shared memory.

@@ -164,11 +164,13 @@ __device__ __forceinline__ void grid_cell_of(const Geometry& g, int k, int& ih, 
 // the CTA's records for the same tile; after the samples the CTA takes one
 // range per tile from the tile's global counter and writes its records there
 // (records of one tile keep no particular order).  Tiles are named by their
-// place in a kFileWin x kFileWin window of tiles around the CTA's anchors; a
+// place in a window of kFileSlots tiles around the CTA's anchors (g.fwin_h
+// tile rows x 2^g.fwin_wl tile columns: square for tall tiles, tall and
+// narrow when grad_value tiles are only a row or two high); a
 // record for a tile outside the window, or beyond the staging room, marks the
 // tile kBucketOverflow instead, and that tile rescans the offsets.
 // ---------------------------------------------------------------------------
-constexpr int kFileWin = 8;
+constexpr int kFileSlots = 64;
 
 // Staging of one (sample, thread): the record for the cell's own tile (bin
 // included) and a meta word: window slot of that tile (6 bits), the record's
@@ -181,14 +183,15 @@ struct FileStage {
     uint64_t* rec;   // [K][threads]
     uint64_t* meta;  // [K][threads]
     int wy0, wx0;    // window origin (tile row, tile column)
+    int wh, wwl;     // window rows, log2 of its columns (wh << wwl == kFileSlots)
 };
 constexpr int kRankBits = 13;  // ranks < K * threads <= 2^13 (checked on the host)
 
 __device__ __forceinline__ int window_slot(const FileStage& fs, int ty, int tx) {
     const int dy = ty - fs.wy0, dx = tx - fs.wx0;
-    return (static_cast<unsigned>(dy) < static_cast<unsigned>(kFileWin) &&
-            static_cast<unsigned>(dx) < static_cast<unsigned>(kFileWin))
-               ? dy * kFileWin + dx
+    return (static_cast<unsigned>(dy) < static_cast<unsigned>(fs.wh) &&
+            static_cast<unsigned>(dx) < static_cast<unsigned>(1 << fs.wwl))
+               ? (dy << fs.wwl) + dx
                : -1;
 }
 
@@ -207,7 +210,7 @@ __global__ void __launch_bounds__(256, 3) samples_kernel(const Geometry g, const
     extern __shared__ __align__(16) unsigned char smem[];
     __shared__ int s_reach;
     __shared__ int s_box[4 * 256];  // per tile pixel: min/max cell row, min/max cell column (relative)
-    __shared__ int s_fcnt[kFileWin * kFileWin], s_fbase[kFileWin * kFileWin];
+    __shared__ int s_fcnt[kFileSlots], s_fbase[kFileSlots];
     constexpr int EPV = Elem<T>::per16;
     constexpr int PAIRS = VEC * EPV / 2;
     const int tile_elems = g.TH * g.TW * g.P;
@@ -229,9 +232,11 @@ __global__ void __launch_bounds__(256, 3) samples_kernel(const Geometry g, const
         // window of tiles centred on the anchors of this CTA's grid
         const int amid_h = t.ho0 * g.sh - g.ph + ((t.th - 1) * g.sh + (kh - 1) * g.dh) / 2;
         const int amid_w = t.wo0 * g.sw - g.pw + ((t.tw - 1) * g.sw + (kw - 1) * g.dw) / 2;
-        fs.wy0 = max(0, max(0, amid_h) / g.BH - kFileWin / 2);
-        fs.wx0 = max(0, max(0, amid_w) / g.BW - kFileWin / 2);
-        for (int i = threadIdx.x; i < kFileWin * kFileWin; i += blockDim.x) s_fcnt[i] = 0;
+        fs.wh = KH > 0 ? 8 : g.fwin_h;  // the unrolled grids are compiled for an 8 x 8 window
+        fs.wwl = KH > 0 ? 3 : g.fwin_wl;
+        fs.wy0 = max(0, max(0, amid_h) / g.BH - fs.wh / 2);
+        fs.wx0 = max(0, max(0, amid_w) / g.BW - (1 << fs.wwl) / 2);
+        for (int i = threadIdx.x; i < kFileSlots; i += blockDim.x) s_fcnt[i] = 0;
     }
     stage_tile_rows(om_s, om, g, t);
     for (int i = threadIdx.x; i < tile_elems; i += blockDim.x) gom_s[i] = static_cast<T>(0.f);
@@ -393,10 +398,11 @@ __global__ void __launch_bounds__(256, 3) samples_kernel(const Geometry g, const
     __syncthreads();
     if (filing) {
         // One range per window tile from its global counter, then the staged records.
-        for (int i = threadIdx.x; i < kFileWin * kFileWin; i += blockDim.x) {
+        const int wmask = (1 << fs.wwl) - 1;
+        for (int i = threadIdx.x; i < kFileSlots; i += blockDim.x) {
             s_fbase[i] = 0;
             if (s_fcnt[i] > 0)
-                s_fbase[i] = atomicAdd(sa.tile_count + tile_index(g, t.n, fs.wy0 + i / kFileWin, fs.wx0 + i % kFileWin),
+                s_fbase[i] = atomicAdd(sa.tile_count + tile_index(g, t.n, fs.wy0 + (i >> fs.wwl), fs.wx0 + (i & wmask)),
                                        s_fcnt[i]);
         }
         __syncthreads();
@@ -404,7 +410,7 @@ __global__ void __launch_bounds__(256, 3) samples_kernel(const Geometry g, const
         auto put = [&](int dl, int rank, uint64_t rec) {
             const int slot = s_fbase[dl] + rank;
             if (static_cast<unsigned>(slot) >= static_cast<unsigned>(g.bcap)) return;  // the tile rescans
-            const long long at = static_cast<long long>(tile_index(g, t.n, fs.wy0 + dl / kFileWin, fs.wx0 + dl % kFileWin)) *
+            const long long at = static_cast<long long>(tile_index(g, t.n, fs.wy0 + (dl >> fs.wwl), fs.wx0 + (dl & wmask))) *
                                      g.bcap + slot;
             sa.bucket_pix[at] = pixv;
             sa.bucket_rec[at] = rec;
@@ -420,12 +426,12 @@ __global__ void __launch_bounds__(256, 3) samples_kernel(const Geometry g, const
             const uint64_t body = rec & ~0xffffull;
             const int bin = static_cast<int>(rec & 0xffff);
             if ((meta >> 58) & 1)  // below: cell row 0 there
-                put(dl0 + kFileWin, static_cast<int>(meta >> (6 + kRankBits)) & rmask,
+                put(dl0 + (1 << fs.wwl), static_cast<int>(meta >> (6 + kRankBits)) & rmask,
                     body | static_cast<uint64_t>(bin - g.BH * (g.BW + 1)));
             if ((meta >> 59) & 1)  // right: cell column 0 there
                 put(dl0 + 1, static_cast<int>(meta >> (6 + 2 * kRankBits)) & rmask, body | static_cast<uint64_t>(bin - g.BW));
             if ((meta >> 60) & 1)  // below-right
-                put(dl0 + kFileWin + 1, static_cast<int>(meta >> (6 + 3 * kRankBits)) & rmask,
+                put(dl0 + (1 << fs.wwl) + 1, static_cast<int>(meta >> (6 + 3 * kRankBits)) & rmask,
                     body | static_cast<uint64_t>(bin - g.BH * (g.BW + 1) - g.BW));
         }
     }

@@ -40,6 +40,9 @@ struct Geometry {
     // __umulhi (exact for coordinates < 2^24).
     int buckets;
     uint32_t bh_magic, bw_magic;
+    // Filing window of the grad_offset_mask CTA: fwin_h tile rows x 2^fwin_wl
+    // tile columns (64 tiles).
+    int fwin_h, fwin_wl;
 };
 
 // What the grad_offset_mask pass leaves for the grad_value pass.

@@ -330,16 +330,16 @@ def test_backward_value_twice_on_one_workspace():
 
 
 def test_samples_beyond_the_filing_window():
-    """Third-stage-like tiles (16 groups: three rows per grad_value tile) with
-    vertical offsets of up to 20 rows: samples land outside the window of tiles
-    a grad_offset_mask CTA files into, those tiles are marked overflowed, and
-    grad_value rescans their offsets."""
-    w = gen.custom(name="window", N=2, H=48, W=14, G=16, Cg=16, Ho=48, Wo=14, K=9, P=432, dtype="bf16",
+    """Third-stage-like tiles (16 groups: three rows per grad_value tile, a filing
+    window of 16 x 4 tiles) with vertical offsets of up to 60 rows: samples land
+    outside the window of tiles a grad_offset_mask CTA files into, those tiles are
+    marked overflowed, and grad_value rescans their offsets."""
+    w = gen.custom(name="window", N=2, H=128, W=14, G=16, Cg=16, Ho=128, Wo=14, K=9, P=432, dtype="bf16",
                    offset=("normal", 0.0, 1.0))
     inp = gen.make_inputs(w)
     rng = np.random.default_rng(7)
     body = inp["offset_mask"][..., : w.G * 27].reshape(w.N, w.Ho, w.Wo, w.G, 27)
-    dy = rng.uniform(-20.0, 20.0, size=body[..., 1:18:2].shape)
+    dy = rng.uniform(-60.0, 60.0, size=body[..., 1:18:2].shape)
     body[..., 1:18:2] = gen.to_storage(dy, w.dtype)
     inp["offset_mask"][..., : w.G * 27] = body.reshape(w.N, w.Ho, w.Wo, w.G * 27)
     _check_forward(w, inp)

@@ -155,14 +155,14 @@ def test_clustered_samples_direct_path(dtype):
 
 
 def test_samples_beyond_the_filing_window():
-    """Vertical offsets of up to 20 rows on 16-group tiles: overflowed tiles rescan the
+    """Vertical offsets of up to 60 rows on 16-group tiles: overflowed tiles rescan the
     offsets and re-form the softmax weights from the logits."""
-    w = gen.custom(name="window", N=2, H=48, W=14, G=16, Cg=16, Ho=48, Wo=14, K=9, P=432, dtype="bf16",
+    w = gen.custom(name="window", N=2, H=128, W=14, G=16, Cg=16, Ho=128, Wo=14, K=9, P=432, dtype="bf16",
                    offset=("normal", 0.0, 1.0), softmax=1)
     inp = gen.make_inputs(w)
     rng = np.random.default_rng(7)
     body = inp["offset_mask"][..., : w.G * 27].reshape(w.N, w.Ho, w.Wo, w.G, 27)
-    body[..., 1:18:2] = gen.to_storage(rng.uniform(-20.0, 20.0, size=body[..., 1:18:2].shape), w.dtype)
+    body[..., 1:18:2] = gen.to_storage(rng.uniform(-60.0, 60.0, size=body[..., 1:18:2].shape), w.dtype)
     inp["offset_mask"][..., : w.G * 27] = body.reshape(w.N, w.Ho, w.Wo, w.G * 27)
     _check(w, inp)
 
