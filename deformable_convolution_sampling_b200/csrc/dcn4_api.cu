@@ -204,7 +204,7 @@ int make_geometry(const dcn4_params* p, bool backward, bool wide, dcn4::Geometry
     g->bw_magic = 0xffffffffu / static_cast<uint32_t>(BW) + 1u;
     // ... and when the grad_offset_mask CTA can stage its records in shared memory.
     if (g->buckets && (dcn4::backward_smem_bytes(*g, eb) > kFileSmem ||
-                       static_cast<long long>(K) * dcn4::samples_threads(*g) > (1 << 13)))
+                       static_cast<long long>(dcn4::filing_chunk(*g)) * dcn4::samples_threads(*g) > (1 << 13)))
         g->buckets = 0;
     // The grad_offset_mask CTA's dynamic shared memory, next to its static arrays.
     if (backward && dcn4::backward_smem_bytes(*g, eb) + kSamplesStaticSmem > kSmemMax)

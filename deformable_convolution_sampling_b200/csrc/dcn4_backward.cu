@@ -228,7 +228,7 @@ __global__ void __launch_bounds__(256, 3) samples_kernel(const Geometry g, const
         // staging after the two offset_mask tiles
         unsigned char* st = smem + 2 * static_cast<size_t>(tile_elems) * sizeof(T);
         fs.rec = reinterpret_cast<uint64_t*>(st);
-        fs.meta = fs.rec + K * blockDim.x;
+        fs.meta = fs.rec + (KH > 0 ? K : filing_chunk(g)) * blockDim.x;
         // window of tiles centred on the anchors of this CTA's grid
         const int amid_h = t.ho0 * g.sh - g.ph + ((t.th - 1) * g.sh + (kh - 1) * g.dh) / 2;
         const int amid_w = t.wo0 * g.sw - g.pw + ((t.tw - 1) * g.sw + (kw - 1) * g.dw) / 2;
@@ -277,6 +277,53 @@ __global__ void __launch_bounds__(256, 3) samples_kernel(const Geometry g, const
     float2 stats = make_float2(0.f, 1.f);  // softmax: (l_max, 1 / sum_k exp(l_k - l_max))
     if constexpr (SM) stats = softmax_stats(row + 2 * K, K);
     float gdot = 0.f;  // softmax: sum_k m_k <gy, S_k>
+
+    // Filing write-out: one range per window tile from its global counter, then
+    // the nk staged points of each thread.
+    auto reserve = [&]() {
+        const int wmask = (1 << fs.wwl) - 1;
+        for (int i = threadIdx.x; i < kFileSlots; i += blockDim.x) {
+            s_fbase[i] = 0;
+            if (s_fcnt[i] > 0)
+                s_fbase[i] = atomicAdd(sa.tile_count + tile_index(g, t.n, fs.wy0 + (i >> fs.wwl), fs.wx0 + (i & wmask)),
+                                       s_fcnt[i]);
+        }
+    };
+    auto write_out = [&](int nk) {
+        const int wmask = (1 << fs.wwl) - 1;
+        const uint32_t pixv = (static_cast<uint32_t>(t.ho0 + (active ? py : 0)) << 16) |
+                              static_cast<uint32_t>(t.wo0 + (active ? px : 0));
+        auto put = [&](int dl, int rank, uint64_t rec) {
+            const int slot = s_fbase[dl] + rank;
+            if (static_cast<unsigned>(slot) >= static_cast<unsigned>(g.bcap)) return;  // the tile rescans
+            const long long at = static_cast<long long>(tile_index(g, t.n, fs.wy0 + (dl >> fs.wwl), fs.wx0 + (dl & wmask))) *
+                                     g.bcap + slot;
+            sa.bucket_pix[at] = pixv;
+            sa.bucket_rec[at] = rec;
+        };
+        const int rmask = (1 << kRankBits) - 1;
+        for (int j = 0; j < nk; ++j) {
+            const int at = j * blockDim.x + threadIdx.x;
+            const uint64_t meta = fs.meta[at];
+            if (!((meta >> 61) & 1)) continue;
+            const uint64_t rec = fs.rec[at];
+            const int dl0 = static_cast<int>(meta & 63);
+            put(dl0, static_cast<int>(meta >> 6) & rmask, rec);
+            const uint64_t body = rec & ~0xffffull;
+            const int bin = static_cast<int>(rec & 0xffff);
+            if ((meta >> 58) & 1)  // below: cell row 0 there
+                put(dl0 + (1 << fs.wwl), static_cast<int>(meta >> (6 + kRankBits)) & rmask,
+                    body | static_cast<uint64_t>(bin - g.BH * (g.BW + 1)));
+            if ((meta >> 59) & 1)  // right: cell column 0 there
+                put(dl0 + 1, static_cast<int>(meta >> (6 + 2 * kRankBits)) & rmask, body | static_cast<uint64_t>(bin - g.BW));
+            if ((meta >> 60) & 1)  // below-right
+                put(dl0 + (1 << fs.wwl) + 1, static_cast<int>(meta >> (6 + 3 * kRankBits)) & rmask,
+                    body | static_cast<uint64_t>(bin - g.BH * (g.BW + 1) - g.BW));
+        }
+    };
+    // Generic grids file in chunks of filing_chunk(g) points (a bounded staging area).
+    const int fkc = KH > 0 ? K : filing_chunk(g);
+    int kc = 0;  // points staged in the current chunk
 
     int k = 0;
 #pragma unroll
@@ -371,9 +418,22 @@ __global__ void __launch_bounds__(256, 3) samples_kernel(const Geometry g, const
                             meta |= (static_cast<uint64_t>(r) << (6 + kRankBits * d)) | (1ull << (57 + d));
                         }
                     }
-                    const int at = kk * blockDim.x + threadIdx.x;
+                    const int at = (KH > 0 ? kk : kc) * blockDim.x + threadIdx.x;
                     fs.meta[at] = meta;
                     fs.rec[at] = rec | static_cast<uint64_t>(gbase + cy * (g.BW + 1) + cx);
+                    if constexpr (KH == 0) {
+                        // every thread takes the same branch: kc, kk and filing are uniform
+                        if (++kc == fkc || kk + 1 == K) {
+                            __syncthreads();
+                            reserve();
+                            __syncthreads();
+                            write_out(kc);
+                            __syncthreads();
+                            for (int i = threadIdx.x; i < kFileSlots; i += blockDim.x) s_fcnt[i] = 0;
+                            __syncthreads();
+                            kc = 0;
+                        }
+                    }
                 }
             } else {
                 if (writer) sa.code[s0 + kk] = cell_code(cell.any, cell.h0 - ah, cell.w0 - aw);
@@ -396,44 +456,10 @@ __global__ void __launch_bounds__(256, 3) samples_kernel(const Geometry g, const
         atomicMax(&s_box[4 * lp + 3], min(127, bmax_w));
     }
     __syncthreads();
-    if (filing) {
-        // One range per window tile from its global counter, then the staged records.
-        const int wmask = (1 << fs.wwl) - 1;
-        for (int i = threadIdx.x; i < kFileSlots; i += blockDim.x) {
-            s_fbase[i] = 0;
-            if (s_fcnt[i] > 0)
-                s_fbase[i] = atomicAdd(sa.tile_count + tile_index(g, t.n, fs.wy0 + (i >> fs.wwl), fs.wx0 + (i & wmask)),
-                                       s_fcnt[i]);
-        }
+    if (KH > 0 && filing) {  // the unrolled grids stage all K points and file them here
+        reserve();
         __syncthreads();
-        const uint32_t pixv = (static_cast<uint32_t>(ho) << 16) | static_cast<uint32_t>(wo);
-        auto put = [&](int dl, int rank, uint64_t rec) {
-            const int slot = s_fbase[dl] + rank;
-            if (static_cast<unsigned>(slot) >= static_cast<unsigned>(g.bcap)) return;  // the tile rescans
-            const long long at = static_cast<long long>(tile_index(g, t.n, fs.wy0 + (dl >> fs.wwl), fs.wx0 + (dl & wmask))) *
-                                     g.bcap + slot;
-            sa.bucket_pix[at] = pixv;
-            sa.bucket_rec[at] = rec;
-        };
-        const int rmask = (1 << kRankBits) - 1;
-        for (int kk = 0; kk < K; ++kk) {
-            const int at = kk * blockDim.x + threadIdx.x;
-            const uint64_t meta = fs.meta[at];
-            if (!((meta >> 61) & 1)) continue;
-            const uint64_t rec = fs.rec[at];
-            const int dl0 = static_cast<int>(meta & 63);
-            put(dl0, static_cast<int>(meta >> 6) & rmask, rec);
-            const uint64_t body = rec & ~0xffffull;
-            const int bin = static_cast<int>(rec & 0xffff);
-            if ((meta >> 58) & 1)  // below: cell row 0 there
-                put(dl0 + (1 << fs.wwl), static_cast<int>(meta >> (6 + kRankBits)) & rmask,
-                    body | static_cast<uint64_t>(bin - g.BH * (g.BW + 1)));
-            if ((meta >> 59) & 1)  // right: cell column 0 there
-                put(dl0 + 1, static_cast<int>(meta >> (6 + 2 * kRankBits)) & rmask, body | static_cast<uint64_t>(bin - g.BW));
-            if ((meta >> 60) & 1)  // below-right
-                put(dl0 + (1 << fs.wwl) + 1, static_cast<int>(meta >> (6 + 3 * kRankBits)) & rmask,
-                    body | static_cast<uint64_t>(bin - g.BH * (g.BW + 1) - g.BW));
-        }
+        write_out(K);
     }
     if (threadIdx.x == 0 && s_reach >= 0) atomicMax(reach + t.n, s_reach);
     for (int i = threadIdx.x; i < t.th * g.TW; i += blockDim.x) {
@@ -1136,7 +1162,7 @@ cudaError_t launch_value_vec(const Geometry& g, const void* om, const void* gout
 
 size_t backward_smem_bytes(const Geometry& g, int elem_bytes) {
     size_t b = static_cast<size_t>(g.TH) * g.TW * g.P * elem_bytes * 2;
-    if (elem_bytes == 2 && g.buckets) b += static_cast<size_t>(g.K) * samples_threads(g) * 16;  // filing staging
+    if (elem_bytes == 2 && g.buckets) b += static_cast<size_t>(filing_chunk(g)) * samples_threads(g) * 16;  // staging
     return b;
 }
 

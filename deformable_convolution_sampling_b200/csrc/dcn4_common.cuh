@@ -346,6 +346,9 @@ cudaError_t launch_backward_samples(const Geometry& g, int dtype, const void* va
 cudaError_t launch_backward_value(const Geometry& g, int dtype, const void* om, const void* gout, void* gvalue,
                                   const int* reach, SampleArrays sa, const uint32_t* boxes,
                                   cudaStream_t stream);
+// Points a grad_offset_mask CTA stages before filing them: all K for the 3x3
+// grids (compiled unrolled), chunks of 8 for the generic grids.
+__host__ __device__ inline int filing_chunk(const Geometry& g) { return (g.kh == 3 && g.kw == 3) ? g.K : (g.K < 8 ? g.K : 8); }
 // Threads of one grad_offset_mask CTA: whole warps (the kernel shuffles).
 inline int samples_threads(const Geometry& g) { return (g.pix_per_cta * g.G * g.nslice + 31) / 32 * 32; }
 // Dynamic shared memory bytes of one CTA.
