@@ -344,3 +344,28 @@ def test_samples_beyond_the_filing_window():
     inp["offset_mask"][..., : w.G * 27] = body.reshape(w.N, w.Ho, w.Wo, w.G * 27)
     _check_forward(w, inp)
     _check_backward(w, inp)
+
+
+# ---------------------------------------------------------------------------
+# Larger grids at a feature-map size: the generic kernels, a filing window
+# shaped by the grad_value tile height, and filing in chunks of points
+# ---------------------------------------------------------------------------
+
+LARGE_GRIDS = [
+    dict(name="k5x5_f16", k=5, dtype="f16", remove_center=0, softmax=0),
+    dict(name="k7x7_bf16_rc", k=7, dtype="bf16", remove_center=1, softmax=0),
+    dict(name="k5x5_bf16_softmax", k=5, dtype="bf16", remove_center=0, softmax=1),
+    dict(name="k5x5_f32", k=5, dtype="f32", remove_center=0, softmax=0),
+]
+
+
+@pytest.mark.parametrize("spec", LARGE_GRIDS, ids=[s["name"] for s in LARGE_GRIDS])
+def test_large_grid_forward_backward(spec):
+    k = spec["k"]
+    K = k * k - spec["remove_center"]
+    P = -(-4 * 3 * K // 8) * 8
+    w = gen.custom(name=spec["name"], N=2, H=40, W=48, G=4, Cg=16, Ho=40, Wo=48, K=K, P=P, dtype=spec["dtype"],
+                   kh=k, kw=k, ph=k // 2, pw=k // 2, remove_center=spec["remove_center"], softmax=spec["softmax"])
+    inp = gen.make_inputs(w)
+    _check_forward(w, inp)
+    _check_backward(w, inp)
