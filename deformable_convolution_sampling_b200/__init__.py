@@ -325,6 +325,42 @@ def _autograd_function():
 
 
 _DCNV4_CORE = None
+_DCNV4_CORE_LINEAR = None
+
+
+def _autograd_function_linear():
+    import torch
+
+    class DCNv4CoreLinear(torch.autograd.Function):
+        """The offset/mask linear layer fused into the aggregation as a
+        torch.autograd.Function.  Forward: dcn4_forward_linear, keeping the
+        offset_mask it formed.  Backward: dcn4_backward on that offset_mask, then the
+        linear layer's gradients (grad_x = g W, grad_W = g^T x, grad_b = sum g, with
+        g = grad_offset_mask as [M, P]) as library GEMMs."""
+
+        @staticmethod
+        def forward(ctx, value, x, weight, bias, p):
+            st, Ho, Wo = dcn4_output_dims(p)
+            check(st)
+            om = torch.empty((p.N, Ho, Wo, p.P), dtype=value.dtype, device=value.device)
+            y = forward_linear(p, value, x, weight, bias, offset_mask_out=om)
+            ctx.save_for_backward(value, x, weight, om)
+            ctx.p = p
+            ctx.has_bias = bias is not None
+            return y
+
+        @staticmethod
+        def backward(ctx, grad_out):
+            value, x, weight, om = ctx.saved_tensors
+            grad_value, gom = backward(ctx.p, value, om, grad_out.contiguous())
+            g = gom.reshape(-1, gom.shape[-1])
+            xm = x.reshape(-1, x.shape[-1])
+            grad_x = (g @ weight).reshape(x.shape)
+            grad_w = g.t() @ xm
+            grad_b = g.sum(0) if ctx.has_bias else None
+            return grad_value, grad_x, grad_w, grad_b, None
+
+    return DCNv4CoreLinear
 
 
 def dcnv4_core(value, offset_mask, *, group: int, kernel=3, stride=1, pad=1, dilation=1,
@@ -339,3 +375,44 @@ def dcnv4_core(value, offset_mask, *, group: int, kernel=3, stride=1, pad=1, dil
     if _DCNV4_CORE is None:
         _DCNV4_CORE = _autograd_function()
     return _DCNV4_CORE.apply(value, offset_mask, p)
+
+
+def dcnv4_core_linear(value, x, weight, bias=None, *, group: int, kernel=3, stride=1, pad=1, dilation=1,
+                      offset_scale: float = 1.0, remove_center: bool = False, softmax: bool = False):
+    """y = DCNv4 core aggregation of value [N,H,W,C] at offset_mask = x @ weight.T + bias,
+    formed inside the forward kernel (x [N,Ho,Wo,Cx], weight [P,Cx], bias [P] or None;
+    fp16/bf16), differentiable in value, x, weight and bias (torch.autograd)."""
+    global _DCNV4_CORE_LINEAR
+    if weight.dim() != 2 or x.dim() != 4 or x.shape[-1] != weight.shape[1]:
+        raise ValueError("x must be [N,Ho,Wo,Cx] and weight [P,Cx]")
+    if bias is not None and tuple(bias.shape) != (weight.shape[0],):
+        raise ValueError("bias must be [P]")
+    for name, t in (("x", x), ("weight", weight)) + ((("bias", bias),) if bias is not None else ()):
+        if t.dtype != value.dtype or not t.is_contiguous() or t.device != value.device:
+            raise ValueError(f"{name} must be contiguous, on value's device and of value's dtype")
+    # the shape checks of the operator itself, on an offset_mask-shaped view of the producer
+    N = value.shape[0]
+    p = params_for_tensors(value, _OffsetMaskShape(x.shape[:3], weight.shape[0], value), group=group, kernel=kernel,
+                           stride=stride, pad=pad, dilation=dilation, offset_scale=offset_scale,
+                           remove_center=remove_center, softmax=softmax)
+    if x.shape[0] != N:
+        raise ValueError("x and value must have the same batch")
+    if _DCNV4_CORE_LINEAR is None:
+        _DCNV4_CORE_LINEAR = _autograd_function_linear()
+    return _DCNV4_CORE_LINEAR.apply(value, x, weight, bias, p)
+
+
+class _OffsetMaskShape:
+    """Stands in for an offset_mask tensor [N,Ho,Wo,P] in params_for_tensors' checks."""
+
+    def __init__(self, lead, P, like):
+        self.shape = tuple(lead) + (int(P),)
+        self.dtype = like.dtype
+        self.is_cuda = like.is_cuda
+        self.device = like.device
+
+    def dim(self):
+        return 4
+
+    def is_contiguous(self):
+        return True

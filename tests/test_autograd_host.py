@@ -25,3 +25,16 @@ def test_argument_errors(value, om, kw, msg):
 def test_float64_is_refused():
     with pytest.raises(ValueError):
         dcn._dtype_code(_t(1, dtype=torch.float64))
+
+
+@pytest.mark.parametrize("x,w,b,msg", [
+    (_t(1, 8, 8, 64, dtype=torch.float16), _t(56, 64, 1, dtype=torch.float16), None, "weight"),
+    (_t(1, 8, 8, 32, dtype=torch.float16), _t(56, 64, dtype=torch.float16), None, "weight"),
+    (_t(1, 8, 8, 64, dtype=torch.float16), _t(56, 64, dtype=torch.float16), _t(55, dtype=torch.float16), "bias"),
+    (_t(1, 8, 8, 64), _t(56, 64, dtype=torch.float16), None, "dtype"),
+    (_t(1, 8, 8, 64, dtype=torch.float16), _t(56, 64, dtype=torch.float16), None, "CUDA tensors"),
+])
+def test_linear_argument_errors(x, w, b, msg):
+    value = _t(1, 8, 8, 16, dtype=torch.float16)
+    with pytest.raises(ValueError, match=msg):
+        dcn.dcnv4_core_linear(value, x, w, b, group=2)

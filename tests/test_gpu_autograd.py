@@ -30,3 +30,38 @@ def test_autograd_matches_oracle(name):
     body = w.G * 3 * w.K
     assert normwise(to_f64(om.grad)[..., :body], ref_gom[..., :body]) <= BWD_TOL[w.dtype]
     assert np.all(to_f64(om.grad)[..., body:] == 0)     # the padding tail's gradient is 0
+
+
+@pytest.mark.parametrize("dtype,bias", [("f16", True), ("bf16", False)])
+def test_autograd_linear_matches_oracle(dtype, bias):
+    """dcnv4_core_linear: y and the gradients of value, x, W and b against the oracle's
+    chain: offset_mask = linear(x, W, b), y = aggregation, then the aggregation's
+    backward and the linear layer's gradients in float64."""
+    import torch
+    import deformable_convolution_sampling_b200 as dcn
+    import oracle
+    from _parity import BWD_TOL, FWD_TOL, normwise, oracle_backward, oracle_forward, to_device, to_f64
+    w = gen.custom(name="lin_autograd", N=2, H=12, W=10, G=4, Cg=16, Ho=12, Wo=10, K=9, P=112, dtype=dtype)
+    inp = gen.make_inputs(w)
+    lin = gen.make_linear_inputs(w, w.C, bias=bias)
+    v = to_device(inp["value"], dtype).requires_grad_(True)
+    x = to_device(lin["x"], dtype).requires_grad_(True)
+    wt = to_device(lin["weight"], dtype).requires_grad_(True)
+    b = to_device(lin["bias"], dtype).requires_grad_(True) if bias else None
+    y = dcn.dcnv4_core_linear(v, x, wt, b, group=w.G)
+    y.backward(to_device(inp["grad_out"], dtype))
+    torch.cuda.synchronize()
+
+    om_ref = oracle.linear(dtype, lin["x"], lin["weight"], lin["bias"])
+    sub = {"value": inp["value"], "offset_mask": om_ref, "grad_out": inp["grad_out"]}
+    ry = oracle_forward(w, sub)
+    rgv, rgom = oracle_backward(w, sub)
+    g = rgom.reshape(-1, w.P)
+    xf = gen.storage_to_f64(lin["x"], dtype).reshape(-1, w.C)
+    wf = gen.storage_to_f64(lin["weight"], dtype)
+    assert normwise(to_f64(y), ry) <= FWD_TOL[dtype]
+    assert normwise(to_f64(v.grad), rgv) <= BWD_TOL[dtype]
+    assert normwise(to_f64(x.grad).reshape(-1, w.C), g @ wf) <= BWD_TOL[dtype]
+    assert normwise(to_f64(wt.grad), g.T @ xf) <= BWD_TOL[dtype]
+    if bias:
+        assert normwise(to_f64(b.grad), g.sum(0)) <= BWD_TOL[dtype]
