@@ -369,3 +369,21 @@ def test_large_grid_forward_backward(spec):
     inp = gen.make_inputs(w)
     _check_forward(w, inp)
     _check_backward(w, inp)
+
+
+
+def test_worked_example_2x2_exact():
+    """The hand-derived worked example (tests/golden) in fp32 through the C ABI: every
+    value is dyadic, so the kernels must reproduce it exactly."""
+    import torch
+    import _golden
+    import deformable_convolution_sampling_b200 as dcn
+    ex = _golden.load()
+    p = dcn.make_params(dtype="f32", **_golden.GEOMETRY)
+    t = {k: torch.from_numpy(ex[k].astype(np.float32)).cuda() for k in ("value", "offset_mask", "grad_out")}
+    y = dcn.forward(p, t["value"], t["offset_mask"])
+    gv, gom = dcn.backward(p, t["value"], t["offset_mask"], t["grad_out"])
+    torch.cuda.synchronize()
+    assert np.array_equal(to_f64(y), ex["y"])
+    assert np.array_equal(to_f64(gom), ex["grad_offset_mask"])
+    assert np.array_equal(to_f64(gv), ex["grad_value"])

@@ -705,3 +705,21 @@ def test_linear_shapes_and_rows():
     assert np.array_equal(out[1, 2, 4], oracle.linear("f16", x[1, 2, 4][None], w)[0])
     with pytest.raises(ValueError):
         oracle.linear("f16", x, w[:, :8])
+
+
+
+# ---------------------------------------------------------------------------
+# The hand-derived worked example (tests/golden/bilinear_2x2_worked.txt)
+# ---------------------------------------------------------------------------
+
+def test_worked_example_2x2():
+    """Fractional offsets, an out-of-image corner and a sample that touches no pixel,
+    worked out by hand from the definition: forward, grad_offset_mask and grad_value."""
+    import _golden
+    ex = _golden.load()
+    prob = oracle.Problem(dtype="f64", **_golden.GEOMETRY)
+    y = oracle.forward(prob, ex["value"], ex["offset_mask"])
+    gv, gom = oracle.backward(prob, ex["value"], ex["offset_mask"], ex["grad_out"])
+    assert np.array_equal(y, ex["y"])
+    assert np.array_equal(gom, ex["grad_offset_mask"])
+    assert np.array_equal(gv, ex["grad_value"])
