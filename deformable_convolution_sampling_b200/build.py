@@ -52,11 +52,29 @@ def build(force: bool = False, ptxas_info: bool = False) -> str:
     if not (force or ptxas_info or needs_build()):
         return LIB
     tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [nvcc(), *ARCH_FLAGS, *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC, "-shared", "-o", tmp, *sources()]
-    if ptxas_info:
-        cmd.insert(1, "-Xptxas=-v")
-    subprocess.run(cmd, check=True)
-    os.replace(tmp, LIB)
+    objdir = os.path.join(PKG, "_build")
+    os.makedirs(objdir, exist_ok=True)
+    # one nvcc per translation unit, all at once, then one link
+    procs, objs = [], []
+    for src in sources():
+        obj = os.path.join(objdir, os.path.basename(src) + f".{os.getpid()}.o")
+        cmd = [nvcc(), *ARCH_FLAGS, *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC, "-c", "-o", obj, src]
+        if ptxas_info:
+            cmd.insert(1, "-Xptxas=-v")
+        procs.append((src, subprocess.Popen(cmd)))
+        objs.append(obj)
+        if ptxas_info:  # one at a time, so the resource reports do not interleave
+            procs[-1][1].wait()
+    failed = [src for src, proc in procs if proc.wait() != 0]
+    try:
+        if failed:
+            raise subprocess.CalledProcessError(1, f"nvcc {' '.join(os.path.basename(f) for f in failed)}")
+        subprocess.run([nvcc(), *ARCH_FLAGS, "-shared", "-o", tmp, *objs], check=True)
+        os.replace(tmp, LIB)
+    finally:
+        for obj in objs:
+            if os.path.exists(obj):
+                os.remove(obj)
     return LIB
 
 
