@@ -79,3 +79,21 @@ def test_workload_table_consistent():
         assert w.P % 8 == 0 and w.P >= w.G * 3 * w.K and w.P - w.G * 3 * w.K < 8
         assert w.Ho == (w.H + 2 * w.ph - (w.dh * (w.kh - 1) + 1)) // w.sh + 1
         assert w.Wo == (w.W + 2 * w.pw - (w.dw * (w.kw - 1) + 1)) // w.sw + 1
+
+
+def test_linear_inputs_are_seeded_and_shaped():
+    """make_linear_inputs: same seed, same bits; shapes [N,Ho,Wo,Cx], [P,Cx], [P]; the
+    produced offsets and masks have about the workload's own spread."""
+    import numpy as np
+    w = gen.custom(**{**gen.WORKLOADS["stage1_f16"].__dict__, "N": 2, "name": "lin"})
+    a = gen.make_linear_inputs(w, 64)
+    b = gen.make_linear_inputs(w, 64)
+    assert all(np.array_equal(a[k], b[k]) for k in ("x", "weight", "bias"))
+    assert a["x"].shape == (2, 56, 56, 64) and a["weight"].shape == (112, 64) and a["bias"].shape == (112,)
+    assert gen.make_linear_inputs(w, 64, bias=False)["bias"] is None
+    c = gen.make_linear_inputs(w, 64, seed=1)
+    assert not np.array_equal(a["x"], c["x"])
+    om = gen.storage_to_f64(a["x"], "f16").reshape(-1, 64) @ gen.storage_to_f64(a["weight"], "f16").T
+    offs = np.concatenate([om[:, g * 27:g * 27 + 18] for g in range(4)], axis=1)
+    masks = np.concatenate([om[:, g * 27 + 18:g * 27 + 27] for g in range(4)], axis=1)
+    assert abs(offs.std() - 1.5) < 0.1 and abs(masks.std() - 0.5) < 0.05
