@@ -387,3 +387,30 @@ def test_worked_example_2x2_exact():
     assert np.array_equal(to_f64(y), ex["y"])
     assert np.array_equal(to_f64(gom), ex["grad_offset_mask"])
     assert np.array_equal(to_f64(gv), ex["grad_value"])
+
+
+def test_location_rounded_once_on_the_gpu():
+    """The kernels form s*dy + anchor with one fp32 rounding (fmaf): on the case where
+    two roundings would move the sample to the next cell row, grad_offset and
+    grad_value match the hand-derived values of the single rounding exactly
+    (1x1 grid on a 4 x 1 image; the same constants as the oracle pin)."""
+    import torch
+    import deformable_convolution_sampling_b200 as dcn
+    s, dy = 10066330 * 2.0 ** -25, -13981013 * 2.0 ** -21
+    lh = 1.0 - 2.0 ** -24
+    p = dcn.make_params(N=1, H=4, W=1, G=1, Cg=4, kh=1, kw=1, ph=0, pw=0, offset_scale=s, dtype="f32", P=8)
+    value = torch.tensor([1.0, 2.0, 10.0, 0.0], dtype=torch.float32).repeat_interleave(4).view(1, 4, 1, 4).cuda()
+    om = torch.zeros((1, 4, 1, 8), dtype=torch.float32)
+    om[..., 2] = 1.0
+    om[0, 3, 0, 1] = dy
+    om = om.cuda()
+    gy = torch.zeros((1, 4, 1, 4), dtype=torch.float32)
+    gy[0, 3, 0, 0] = 1.0                               # <gy, v> = channel 0 of v
+    gy = gy.cuda()
+    y = dcn.forward(p, value, om)
+    gv, gom = dcn.backward(p, value, om, gy)
+    torch.cuda.synchronize()
+    assert np.all(to_f64(y)[0, 3, 0] == np.float32((1.0 - lh) + lh * 2.0))
+    g = to_f64(gom)[0, 3, 0]
+    assert g[1] == np.float32(s * 1.0) and g[0] == np.float32(s * -(1.0 + lh))
+    assert np.array_equal(to_f64(gv)[0, :, 0, 0], np.float32([1.0 - lh, lh, 0.0, 0.0]).astype(np.float64))

@@ -29,6 +29,8 @@ MUTATIONS = {
     "grad_value_without_mask": ("+= m * wt * gy;", "+= wt * gy;"),
     "stride_ignored": ("const int base_w = wo * p->sw - p->pw + c.iw * p->dw;",
                        "const int base_w = wo - p->pw + c.iw * p->dw;"),
+    "location_two_roundings": ("*h = static_cast<double>(std::fmaf(s, static_cast<float>(dy), static_cast<float>(base_h)));",
+                               "*h = static_cast<double>(static_cast<float>(s * static_cast<float>(dy)) + static_cast<float>(base_h));"),
     "bilinear_ceil_cell": ("const double fh = std::floor(h);", "const double fh = std::ceil(h) - 1.0;"),
     # softmax variant
     "softmax_not_normalised": ("for (int k = 0; k < K; ++k) a[k] /= sum;", ""),

@@ -385,6 +385,53 @@ def test_location_fp32_mode():
     np.testing.assert_array_equal(oracle.forward(pa, inp["value"], om), oracle.forward(pb, inp["value"], om))
 
 
+# One location where a single rounding of s*dy + base and two roundings
+# (the product rounded to fp32 first, then the sum) pick different cells.
+# fp32 constants, checked below: s = fl(0.3) = 10066330 * 2^-25 and
+# dy = -13981013 * 2^-21 (= -6.6666665077...); their exact product is
+# -2.0000000317891... .  With base 3 the exact sum 0.99999996821... lies
+# closer to 1 - 2^-24 than to 1, so fmaf gives h = 1 - 2^-24 (cell row 0,
+# lh = 1 - 2^-24); fl(s*dy) = -2 exactly, and -2 + 3 = 1 puts h on row 1.
+FUSED_S = 10066330 * 2.0 ** -25
+FUSED_DY = -13981013 * 2.0 ** -21
+
+
+def _fused_location_case():
+    """1x1 grid on a 4 x 1 image, one group of one channel; output pixel 3 (anchor
+    row 3) samples at 3 + s*dy, every other pixel at its own anchor.  value rows
+    1, 2, 10, 0; grad_out 1 at pixel 3 only; masks 1."""
+    prob = oracle.Problem(N=1, H=4, W=1, G=1, Cg=1, kh=1, kw=1, ph=0, pw=0, offset_scale=FUSED_S,
+                          dtype="f32", P=8, location_fp32=True)
+    value = np.array([1.0, 2.0, 10.0, 0.0], dtype=np.float32).reshape(1, 4, 1, 1)
+    om = np.zeros((1, 4, 1, 8), dtype=np.float32)
+    om[..., 2] = 1.0                                   # the mask of every pixel
+    om[0, 3, 0, 1] = FUSED_DY                          # dy of pixel 3
+    gy = np.zeros((1, 4, 1, 1), dtype=np.float32)
+    gy[0, 3] = 1.0
+    return prob, value, om, gy
+
+
+def test_location_is_one_fused_rounding():
+    """The fp32 location mode rounds s*dy + base once (fmaf), as the kernels do."""
+    assert np.float32(0.3) == np.float32(FUSED_S) and float(np.float32(FUSED_S)) == FUSED_S
+    assert float(np.float32(FUSED_DY)) == FUSED_DY
+    exact = FUSED_S * FUSED_DY + 3.0                   # exact in float64 (24 x 24 bits)
+    assert 1.0 - 2.0 ** -24 < exact < 1.0 - 2.0 ** -25  # rounds down to 1 - 2^-24 in fp32
+    assert float(np.float32(FUSED_S * FUSED_DY)) == -2.0
+    prob, value, om, gy = _fused_location_case()
+    lh = 1.0 - 2.0 ** -24                              # h = 1 - 2^-24: cell rows 0 and 1
+    y = oracle.forward(prob, value, om)
+    assert y[0, 3, 0, 0] == (1.0 - lh) * 1.0 + lh * 2.0
+    assert y[0, 0, 0, 0] == 1.0 and y[0, 1, 0, 0] == 2.0 and y[0, 2, 0, 0] == 10.0
+    gv, gom = oracle.backward(prob, value, om, gy)
+    # d/d dy = s * m * <gy, dS/dh>, dS/dh = v[row 1] - v[row 0] on this cell (lw = 0)
+    assert gom[0, 3, 0, 1] == FUSED_S * (2.0 - 1.0)
+    # d/d dx: dS/dw = (1 - lh)(0 - v[row 0]) + lh (0 - v[row 1]) (the right corners are off the image)
+    assert gom[0, 3, 0, 0] == FUSED_S * -(1.0 + lh)
+    assert gom[0, 3, 0, 2] == (1.0 - lh) * 1.0 + lh * 2.0
+    np.testing.assert_array_equal(gv[0, :, 0, 0], [1.0 - lh, lh, 0.0, 0.0])
+
+
 def test_threads_do_not_change_results():
     prob = _tiny(N=3)
     inp, Ho, Wo = rand_problem_inputs(prob, seed=15)
