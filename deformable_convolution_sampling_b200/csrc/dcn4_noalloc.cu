@@ -9,7 +9,8 @@
 // every device that loads this library and keeps there until the process
 // exits.  Nothing here calls cudaMalloc, cudaFree or an allocating library
 // routine.
-#include <atomic>
+#include <cuda.h>  // CUcontext and CUresult only: the two driver calls below come from cudaGetDriverEntryPoint
+
 #include <cstdio>
 #include <mutex>
 
@@ -25,10 +26,46 @@ constexpr size_t kScratchBytes = static_cast<size_t>(DCN4_NOALLOC_SCRATCH_BYTES)
 __device__ __align__(256) unsigned char g_scratch[kScratchBytes];
 
 constexpr int kMaxDevices = 64;
-std::atomic<void*> g_scratch_ptr[kMaxDevices];
+
+// The area's address is looked up once per device and context: a device reset
+// (cudaDeviceReset, or the primary context released and made again) unloads
+// the module, so the array may come back elsewhere.  Contexts are told apart by
+// the driver's context id, which is never reused within a process.
+struct ScratchSlot {
+    unsigned long long ctx_id;  // 0: not set up
+    void* ptr;
+};
+ScratchSlot g_slot[kMaxDevices];
 std::mutex g_setup_mutex;
 
 thread_local char g_error[256] = "";
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+// Id of the calling thread's current context, or 0 when there is none yet.
+cudaError_t current_context_id(unsigned long long* id) {
+    static CtxGetCurrentFn get_current = nullptr;
+    static CtxGetIdFn get_id = nullptr;
+    static std::once_flag once;
+    static cudaError_t resolved = cudaSuccess;
+    std::call_once(once, [] {
+        void* a = nullptr;
+        void* b = nullptr;
+        cudaError_t e = cudaGetDriverEntryPoint("cuCtxGetCurrent", &a, cudaEnableDefault, nullptr);
+        if (e == cudaSuccess) e = cudaGetDriverEntryPoint("cuCtxGetId", &b, cudaEnableDefault, nullptr);
+        if (e == cudaSuccess && (a == nullptr || b == nullptr)) e = cudaErrorSymbolNotFound;
+        resolved = e;
+        get_current = reinterpret_cast<CtxGetCurrentFn>(a);
+        get_id = reinterpret_cast<CtxGetIdFn>(b);
+    });
+    if (resolved != cudaSuccess) return resolved;
+    CUcontext ctx = nullptr;
+    if (get_current(&ctx) != CUDA_SUCCESS) return cudaErrorContextIsDestroyed;
+    *id = 0;
+    if (ctx != nullptr && get_id(ctx, id) != CUDA_SUCCESS) return cudaErrorContextIsDestroyed;
+    return cudaSuccess;
+}
 
 }  // namespace
 
@@ -52,20 +89,26 @@ extern "C" int dcn4_backward_noalloc(const dcn4_params* p, const void* value, co
                  cudaGetErrorString(e));
         return DCN4_ERR_LAUNCH;
     }
-    void* scratch = g_scratch_ptr[dev].load(std::memory_order_acquire);
-    if (scratch == nullptr) {
-        // Set-up, once per device, with that device current.
+    void* scratch = nullptr;
+    {
+        // Set-up, once per device (and again after a device reset), with that
+        // device current: look the area's device address up.
         std::lock_guard<std::mutex> lock(g_setup_mutex);
-        scratch = g_scratch_ptr[dev].load(std::memory_order_acquire);
-        if (scratch == nullptr) {
-            e = cudaGetSymbolAddress(&scratch, g_scratch);
-            if (e != cudaSuccess || scratch == nullptr) {
-                snprintf(g_error, sizeof g_error, "dcn4_backward_noalloc: cudaGetSymbolAddress failed (%s)",
-                         cudaGetErrorString(e));
-                return DCN4_ERR_LAUNCH;
-            }
-            g_scratch_ptr[dev].store(scratch, std::memory_order_release);
+        unsigned long long ctx = 0;
+        e = current_context_id(&ctx);
+        if (e == cudaSuccess && (ctx == 0 || g_slot[dev].ctx_id != ctx)) {
+            e = cudaGetSymbolAddress(&scratch, g_scratch);  // makes the device's context current if none is
+            if (e == cudaSuccess) e = current_context_id(&ctx);
+            if (e == cudaSuccess && (scratch == nullptr || ctx == 0)) e = cudaErrorContextIsDestroyed;
+            if (e == cudaSuccess) g_slot[dev] = ScratchSlot{ctx, scratch};
         }
+        if (e != cudaSuccess) {
+            g_slot[dev] = ScratchSlot{0, nullptr};
+            snprintf(g_error, sizeof g_error, "dcn4_backward_noalloc: scratch look-up on device %d failed (%s)",
+                     dev, cudaGetErrorString(e));
+            return DCN4_ERR_LAUNCH;
+        }
+        scratch = g_slot[dev].ptr;
     }
     g_error[0] = '\0';
     return dcn4_backward(p, value, offset_mask, grad_out, grad_value, grad_offset_mask, scratch, kScratchBytes,

@@ -199,8 +199,8 @@ int dcn4_backward(const dcn4_params* p, const void* value, const void* offset_ma
  *     DCN4_ERR_WORKSPACE before anything is launched (detail in
  *     dcn4_noalloc_last_error()).
  *   - Set-up: the first call on a device (made with that device current) looks
- *     up the area's device address; make that first call before any stream
- *     capture begins.
+ *     up the area's device address, and so does the first call after a device
+ *     reset (a new context); make such a call before any stream capture begins.
  *   - Sharing: every call on a device uses the same area, which keeps the
  *     last call's contents (each call resets what it needs).  Calls whose
  *     executions overlap on the GPU (different streams, no ordering between

@@ -25,6 +25,16 @@ def dcn():
     return d
 
 
+def run_without_gpu(code: str):
+    """Runs `code` (with `dcn`, the binding, imported) in a child process whose
+    CUDA runtime sees no device, so that no address it passes can reach a GPU."""
+    env = dict(os.environ, CUDA_VISIBLE_DEVICES="")
+    prelude = "import sys; sys.path.insert(0, %r)\nimport deformable_convolution_sampling_b200 as dcn\n" % ROOT
+    r = subprocess.run([sys.executable, "-c", prelude + code], cwd=ROOT, env=env, capture_output=True, text=True,
+                       timeout=300)
+    assert r.returncode == 0, r.stdout[-2000:] + r.stderr[-2000:]
+
+
 def declared_functions():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
@@ -126,30 +136,36 @@ def test_invalid_params_are_rejected_before_launch(dcn, field, value, status):
     p = dcn.make_params(N=2, H=8, W=8, G=2, Cg=8, dtype="f16")
     setattr(p, field, value)
     assert dcn.dcn4_check_params(p) == status
-    # pointers that would fault if used: the call must fail before any launch
-    assert dcn.dcn4_forward(p, 16, 32, 48, None) == status
+    # NULL tensors: the parameter check must answer first (a regression would
+    # return DCN4_ERR_NULL instead, still without a launch)
+    assert dcn.dcn4_forward(p, None, None, None, None) == status
     assert dcn.dcn4_last_error() != ""
 
 
-def test_forward_linear_checks_before_launch(dcn):
-    """dcn4_forward_linear validates on the host: pointers that would fault are never used."""
-    p = dcn.make_params(N=2, H=8, W=8, G=4, Cg=16, dtype="f16")
-    ok = dict(value=16, x=32, weight=48, bias=None, out=64, om=None)
+def test_forward_linear_checks_before_launch():
+    """dcn4_forward_linear validates on the host.  The checks need non-NULL
+    (made-up, never dereferenced) addresses, so they run in a child process that
+    sees no GPU: should a check ever regress, the launch fails with "no device"
+    instead of reaching a GPU with those addresses."""
+    run_without_gpu("""
+p = dcn.make_params(N=2, H=8, W=8, G=4, Cg=16, dtype="f16")
+ok = dict(value=16, x=32, weight=48, bias=None, out=64, om=None)
 
-    def call(params, Cx, **kw):
-        a = {**ok, **kw}
-        return dcn.dcn4_forward_linear(params, Cx, a["value"], a["x"], a["weight"], a["bias"], a["out"], a["om"],
-                                       None)
-    p32 = dcn.make_params(N=2, H=8, W=8, G=4, Cg=16, dtype="f32")
-    assert call(p32, 64) == -5                      # fp32: no fused producer
-    assert call(p, 24) == -2 and call(p, 0) == -2   # Cx not a multiple of 16
-    assert call(p, 1 << 14) == -5                   # x tiles too large for shared memory
-    assert call(p, 64, x=None) == -1
-    assert call(p, 64, bias=40) == -4 and call(p, 64, om=72) == -4 and call(p, 64, x=36) == -4
-    bad = dcn.make_params(N=2, H=8, W=8, G=4, Cg=16, dtype="f16")
-    bad.P = 100
-    assert call(bad, 64) == -3
-    assert dcn.dcn4_last_error() != ""
+def call(params, Cx, **kw):
+    a = {**ok, **kw}
+    return dcn.dcn4_forward_linear(params, Cx, a["value"], a["x"], a["weight"], a["bias"], a["out"], a["om"],
+                                   None)
+p32 = dcn.make_params(N=2, H=8, W=8, G=4, Cg=16, dtype="f32")
+assert call(p32, 64) == -5                      # fp32: no fused producer
+assert call(p, 24) == -2 and call(p, 0) == -2   # Cx not a multiple of 16
+assert call(p, 1 << 14) == -5                   # x tiles too large for shared memory
+assert call(p, 64, x=None) == -1
+assert call(p, 64, bias=40) == -4 and call(p, 64, om=72) == -4 and call(p, 64, x=36) == -4
+bad = dcn.make_params(N=2, H=8, W=8, G=4, Cg=16, dtype="f16")
+bad.P = 100
+assert call(bad, 64) == -3
+assert dcn.dcn4_last_error() != ""
+""")
 
 
 def test_remove_center_needs_odd_kernel(dcn):
@@ -158,15 +174,31 @@ def test_remove_center_needs_odd_kernel(dcn):
     assert dcn.dcn4_check_params(p) == -2
 
 
-def test_null_and_misaligned_pointers(dcn):
-    p = dcn.make_params(N=1, H=8, W=8, G=2, Cg=8, dtype="f16")
-    assert dcn.dcn4_forward(p, None, 16, 32, None) == -1
-    assert dcn.dcn4_forward(p, 16, 18, 32, None) == -4
-    assert dcn.dcn4_backward(p, 16, 32, 48, 64, None, 96, 1 << 20, None) == -1
-    assert dcn.dcn4_backward(p, 16, 32, 48, 64, 80, 97, 1 << 20, None) == -4
-    assert dcn.dcn4_backward(p, 16, 32, 48, 64, 80, None, 0, None) == -6
-    assert dcn.dcn4_backward(p, 16, 32, 48, 64, 80, 96, 100, None) == -6
-    assert dcn.lib.dcn4_forward(None, None, None, None, None) == -1
+def test_null_and_misaligned_pointers():
+    """NULL, misaligned and missing-workspace arguments are refused on the host
+    (made-up addresses: checked in a child process that sees no GPU)."""
+    run_without_gpu("""
+p = dcn.make_params(N=1, H=8, W=8, G=2, Cg=8, dtype="f16")
+assert dcn.dcn4_forward(p, None, 16, 32, None) == -1
+assert dcn.dcn4_forward(p, 16, 18, 32, None) == -4
+assert dcn.dcn4_backward(p, 16, 32, 48, 64, None, 96, 1 << 20, None) == -1
+assert dcn.dcn4_backward(p, 16, 32, 48, 64, 80, 97, 1 << 20, None) == -4
+assert dcn.dcn4_backward(p, 16, 32, 48, 64, 80, None, 0, None) == -6
+assert dcn.dcn4_backward(p, 16, 32, 48, 64, 80, 96, 100, None) == -6
+assert dcn.lib.dcn4_forward(None, None, None, None, None) == -1
+""")
+
+
+def test_child_process_sees_no_gpu():
+    """The isolation the checks above rely on: with CUDA_VISIBLE_DEVICES empty the
+    library's CUDA runtime finds no device (the no-allocation entry point's device
+    look-up fails; every pointer argument is NULL)."""
+    run_without_gpu("""
+p = dcn.make_params(N=1, H=8, W=8, G=2, Cg=8, dtype="f16")
+st = dcn.dcn4_backward_noalloc(p, None, None, None, None, None, None)
+assert st == -7, st                               # DCN4_ERR_LAUNCH: no usable device
+assert "device" in dcn.dcn4_noalloc_last_error()
+""")
 
 
 def test_status_strings(dcn):
@@ -181,3 +213,21 @@ def test_missing_library_fails_loudly(tmp_path):
     r = subprocess.run([sys.executable, "-c", "import deformable_convolution_sampling_b200"], cwd=tmp_path,
                        capture_output=True, text=True)
     assert r.returncode != 0 and "ImportError" in r.stderr and "no CPU fallback" in r.stderr
+
+
+def _code_only(path: str) -> str:
+    """Source text without // and /* */ comments."""
+    text = open(path).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return re.sub(r"//[^\n]*", "", text)
+
+
+def test_backward_path_allocates_nothing():
+    """dcn4_backward_noalloc promises no device allocation: no source on the
+    backward's call path (the entry point, the C ABI, the backward kernels and
+    their shared helpers) names an allocating or freeing CUDA call."""
+    csrc = os.path.join(ROOT, "deformable_convolution_sampling_b200", "csrc")
+    pattern = re.compile(r"\b(cudaMalloc\w*|cudaFree\w*|cuMemAlloc\w*|cuMemFree\w*|cudaHostAlloc|cudaMemPool\w*)\b")
+    for name in ("dcn4_noalloc.cu", "dcn4_api.cu", "dcn4_backward.cu", "dcn4_common.cuh"):
+        found = pattern.findall(_code_only(os.path.join(csrc, name)))
+        assert not found, f"{name} calls {sorted(set(found))}"
