@@ -28,9 +28,18 @@ K points of each (pixel, group) (the DCNv3 form of the operator).
 cores; fp16/bf16 workloads) against the same producer run as a separate
 library GEMM (torch.nn.functional.linear, cuBLAS) followed by dcn4_forward.
 
+The line also carries "per_config": forward and backward µs per call,
+achieved GB/s and fractions of the measured copy bandwidth and of 8 TB/s for
+every workload of the configuration table (tiny fp32, first-stage fp16,
+third-stage bf16, high-resolution fp16, training-step bf16), each stage timed
+over --config-reps calls with the L2 flushed before every call.
+
 --impl reference times the CPU oracle (the only other implementation of the
-operator) on the host cores, on a bounded sample of the same workload per
-step, scaled to the full batch.
+operator) on the host cores: each step is one forward + backward call on the
+whole batch when the run fits about REFERENCE_BUDGET_S seconds, else on a
+sample of at least one image per host thread (value scaled to the batch;
+ms_per_step is always the measured step).  cpu_baseline in the native line
+times the same calls for about --cpu-seconds of CPU work.
 """
 from __future__ import annotations
 
@@ -52,6 +61,7 @@ import dcn4_inputs as gen  # noqa: E402
 
 METRIC = "DCNv4 core fwd/bwd µs per call and achieved HBM GB/s (% of B200 peak)"
 L2_FLUSH_BYTES = 256 << 20
+REFERENCE_BUDGET_S = 150.0
 FALLBACK_HBM_GBS = 6650.0
 ELEM_BYTES = {"f32": 4, "f16": 2, "bf16": 2}
 
@@ -225,55 +235,82 @@ def barrier(device=None):
 # CPU oracle timing (baseline / reference arm)
 # ---------------------------------------------------------------------------
 
-def time_oracle(w: gen.Workload, images: int, inp=None) -> dict:
-    """Forward + backward of the oracle on `images` images of the workload,
-    scaled to µs per full-batch call."""
+def oracle_call_seconds(w: gen.Workload, inp: dict, threads: int) -> float:
+    """Wall seconds of one oracle forward + backward on the images of `inp`."""
     import oracle
-    threads = oracle.host_threads()
-    sub = gen.custom(**{**w.__dict__, "N": images, "name": w.name + "_sample"})
-    if inp is None:
-        inp = gen.make_inputs(sub, tail_fill=0.0)
-    prob = oracle.Problem(dtype=w.dtype, location_fp32=True, **sub.geometry())
+    prob = oracle.Problem(dtype=w.dtype, location_fp32=True, **{**w.geometry(), "N": inp["value"].shape[0]})
     t0 = time.perf_counter()
     oracle.forward(prob, inp["value"], inp["offset_mask"], nthreads=threads)
     oracle.backward(prob, inp["value"], inp["offset_mask"], inp["grad_out"], nthreads=threads)
-    dt = time.perf_counter() - t0
-    us_full = dt * 1e6 * w.N / images
-    return {"value": round(us_full, 1), "unit": "us/call", "cores": threads, "kind": "oracle",
-            "sample": f"forward+backward of {images} of {w.N} images, {threads} threads, "
-                      f"{dt:.2f} s, scaled x{w.N / images:g} to the full batch",
-            "seconds": dt}
+    return time.perf_counter() - t0
 
 
-def oracle_sample_images(w: gen.Workload, target_s: float = 15.0) -> int:
-    """Images of the workload the oracle handles in about target_s seconds."""
-    probe = time_oracle(w, 1)
-    per = max(probe["seconds"], 1e-3)
-    return int(max(1, min(w.N, target_s // per)))
+def oracle_sample(w: gen.Workload, images: int) -> dict:
+    sub = gen.custom(**{**w.__dict__, "N": images, "name": w.name + "_sample"})
+    return gen.make_inputs(sub, tail_fill=0.0)
+
+
+def oracle_images(w: gen.Workload, seconds_per_call: float, threads: int) -> tuple[int, float]:
+    """Images per oracle call so that one call takes about `seconds_per_call`: the
+    whole batch when it fits, else a sample of at least `threads` images (the
+    oracle's backward runs one image per thread).  Returns (images, estimated
+    seconds of one whole-batch call)."""
+    probe_n = max(1, min(w.N, threads))
+    per_img = oracle_call_seconds(w, oracle_sample(w, probe_n), threads) / probe_n
+    full = per_img * w.N
+    if full <= seconds_per_call:
+        return w.N, full
+    n = int(seconds_per_call // max(per_img, 1e-9))
+    return max(probe_n, min(w.N, n)), full
+
+
+def time_oracle(w: gen.Workload, target_s: float) -> dict:
+    """The oracle as a baseline: forward + backward calls on the host cores for
+    about target_s seconds of CPU work, in µs per whole-batch call."""
+    import oracle
+    threads = oracle.host_threads()
+    images, _ = oracle_images(w, target_s, threads)
+    inp = oracle_sample(w, images)
+    secs = []
+    while not secs or (sum(secs) < target_s and len(secs) < 20):
+        secs.append(oracle_call_seconds(w, inp, threads))
+    per_call = statistics.mean(secs)
+    us_full = per_call * 1e6 * w.N / images
+    used = min(threads, images)
+    scaled = "" if images == w.N else f", scaled x{w.N / images:g} to the {w.N}-image batch"
+    return {"value": round(us_full, 1), "unit": "us/call", "cores": used, "kind": "oracle",
+            "sample": f"{len(secs)} calls of forward+backward on {images} of {w.N} images with {used} threads "
+                      f"(of {threads}), {sum(secs):.2f} s of CPU work{scaled}"}
 
 
 def run_reference(args, w: gen.Workload) -> dict:
+    """The oracle as the reference arm: each step is one forward + backward call on
+    the host cores, on the whole batch when the --steps/--warmup run fits about
+    REFERENCE_BUDGET_S seconds, else on a sample of images (value scaled to the
+    batch; ms_per_step is always the measured step)."""
+    import oracle
     rank, world, _ = dist_env()
     if rank != 0:
         return {}
-    imgs = max(1, min(w.N, args.reference_images))
-    sub = gen.custom(**{**w.__dict__, "N": imgs, "name": w.name + "_sample"})
-    inp = gen.make_inputs(sub, tail_fill=0.0)
+    threads = oracle.host_threads()
+    images, _ = oracle_images(w, REFERENCE_BUDGET_S / (args.steps + args.warmup), threads)
+    inp = oracle_sample(w, images)
     for _ in range(args.warmup):
-        time_oracle(w, imgs, inp)
-    times = [time_oracle(w, imgs, inp) for _ in range(args.steps)]
-    us = statistics.mean(t["value"] for t in times)
-    cb = dict(times[0])
-    cb["value"] = round(us, 1)
-    cb.pop("seconds", None)
-    cb["sample"] = f"each step: forward+backward of {imgs} of {w.N} images, scaled to the full batch"
+        oracle_call_seconds(w, inp, threads)
+    secs = [oracle_call_seconds(w, inp, threads) for _ in range(args.steps)]
+    step_s = statistics.mean(secs)
+    us = step_s * 1e6 * w.N / images
+    used = min(threads, images)
+    sample = (f"each step: forward+backward on {images} of {w.N} images with {used} threads (of {threads}), "
+              f"{step_s:.3f} s" + ("" if images == w.N else f"; value scaled x{w.N / images:g} to the batch"))
     return {
         "impl": "reference", "metric": METRIC, "value": round(us, 1), "unit": "us/call",
-        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(us / 1e3, 4),
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_s * 1e3, 3),
         "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": {"workload": f"{w.name}: {w.describe()}, forward+backward",
-                                        "parallelism": "oracle on host cores"},
-        "cpu_baseline": cb,
+                                        "parallelism": "oracle on host cores", "images_per_step": images},
+        "cpu_baseline": {"value": round(us, 1), "unit": "us/call", "cores": used, "kind": "oracle",
+                         "sample": sample},
         "e2e": {"value": round(us, 1), "unit": "us/call", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
@@ -502,14 +539,92 @@ def run_native(args, w: gen.Workload) -> dict:
         result["e2e"] = e2e
     if args.linear:
         result["linear"] = linear_leg(w, v, p, flush, stream, dev, world)
+    if not args.no_per_config:
+        sampler = ClockSampler(local if world > 1 else torch.cuda.current_device())
+        sampler.start()
+        time.sleep(0.3)
+        t2 = time.time()
+        result["per_config"] = per_config_leg(dev, world, args.config_reps, flush, stream)
+        t3 = time.time()
+        sampler.stop()
+        result["per_config_clocks"] = summarize_clocks(sampler.samples, t2, t3)
+        result["per_config_note"] = (f"{args.config_reps} calls of each stage per workload, CUDA events on the "
+                                     f"launching stream, L2 flushed before every call; fractions of the measured "
+                                     f"copy bandwidth ({measured_peaks()['hbm_gbs']} GB/s) and of 8 TB/s")
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        n_img = oracle_sample_images(w, args.cpu_seconds)
-        cb = time_oracle(w, n_img)
-        cb.pop("seconds", None)
-        result["cpu_baseline"] = cb
+        result["cpu_baseline"] = time_oracle(w, args.cpu_seconds)
     if world > 1:
         dist.destroy_process_group()
     return result
+
+
+def config_record(w: gen.Workload, stage_us: dict, peaks: dict) -> dict:
+    """µs per call and achieved HBM GB/s against the algorithmic byte model."""
+    bm = byte_model(w)
+    fwd_us = stage_us["fwd"]
+    bwd_us = stage_us["bwd_offset_mask"] + stage_us["bwd_value"]
+    rec = {"workload": f"{w.name}: {w.describe()}", "fwd_us": round(fwd_us, 2), "bwd_us": round(bwd_us, 2),
+           "kernel_us": {KERNELS[k]: round(v, 2) for k, v in stage_us.items()},
+           "fwd_bytes": bm["fwd"], "bwd_bytes": bm["bwd"]}
+    for leg, us, b in (("fwd", fwd_us, bm["fwd"]), ("bwd", bwd_us, bm["bwd"])):
+        gbs = b / (us * 1e-6) / 1e9
+        rec[f"{leg}_gbs"] = round(gbs, 1)
+        rec[f"{leg}_frac_hbm"] = round(gbs / peaks["hbm_gbs"], 4)
+        rec[f"{leg}_frac_8tbs"] = round(gbs / 8000.0, 4)
+    return rec
+
+
+def per_config_leg(dev, world: int, reps: int, flush, stream) -> dict:
+    """Every workload of the configuration table: forward, grad_offset_mask and
+    grad_value stages, each timed over `reps` calls with CUDA events on the
+    launching stream and the L2 flushed before every call (outside the events);
+    max over ranks."""
+    import numpy as np
+    import torch
+    import deformable_convolution_sampling_b200 as dcn
+    peaks = measured_peaks()
+    sh = stream.cuda_stream
+    out = {}
+    for name in gen.WORKLOAD_ORDER:
+        w = gen.WORKLOADS[name]
+        tdt = {"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16}[w.dtype]
+        inp = gen.make_inputs(w, tail_fill=0.0)
+
+        def dev_t(a):
+            a = np.ascontiguousarray(a)
+            t = torch.from_numpy(a.view(np.int16)).view(tdt) if w.dtype == "bf16" else torch.from_numpy(a)
+            return t.to(dev)
+        v, om, gy = dev_t(inp["value"]), dev_t(inp["offset_mask"]), dev_t(inp["grad_out"])
+        p = dcn.make_params(dtype=w.dtype, **w.geometry())
+        y = torch.empty((w.N, w.Ho, w.Wo, w.C), dtype=tdt, device=dev)
+        gv, gom = torch.empty_like(v), torch.empty_like(om)
+        nb = dcn.dcn4_backward_workspace_size(p)
+        ws = torch.empty(max(nb, 16), dtype=torch.uint8, device=dev)
+        calls = {
+            "fwd": lambda: dcn.check(dcn.dcn4_forward(p, v.data_ptr(), om.data_ptr(), y.data_ptr(), sh)),
+            "bwd_offset_mask": lambda: dcn.check(dcn.dcn4_backward_offset_mask(
+                p, v.data_ptr(), om.data_ptr(), gy.data_ptr(), gom.data_ptr(), ws.data_ptr(), nb, sh)),
+            "bwd_value": lambda: dcn.check(dcn.dcn4_backward_value(
+                p, om.data_ptr(), gy.data_ptr(), gv.data_ptr(), ws.data_ptr(), nb, sh)),
+        }
+        for _ in range(5):
+            for fn in calls.values():
+                fn()
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(reps)]
+        torch.cuda.synchronize(dev)
+        for e in ev:
+            flush.zero_()
+            e[0].record(stream)
+            for j, fn in enumerate(calls.values()):
+                fn()
+                e[j + 1].record(stream)
+        torch.cuda.synchronize(dev)
+        stage_us = {k: max_over_ranks(statistics.mean(e[j].elapsed_time(e[j + 1]) for e in ev) * 1e3, dev)
+                    for j, k in enumerate(calls)}
+        out[name] = config_record(w, stage_us, peaks)
+        del v, om, gy, y, gv, gom, ws
+    torch.cuda.empty_cache()
+    return out
 
 
 def linear_leg(w: gen.Workload, v, p, flush, stream, dev, world: int) -> dict:
@@ -581,10 +696,12 @@ def main(argv=None):
                     help="also time the forward with the offset/mask linear layer fused in")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="skip the per-workload forward/backward timings")
+    ap.add_argument("--config-reps", type=int, default=50,
+                    help="calls per stage and workload in the per-config timings")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="target seconds of oracle work for the cpu_baseline sample")
-    ap.add_argument("--reference-images", type=int, default=1,
-                    help="images of the batch the reference arm runs per step")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

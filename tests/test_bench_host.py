@@ -83,12 +83,30 @@ def test_max_over_ranks_two_gloo_processes():
 
 
 def test_reference_arm_tiny():
+    import time
+    t0 = time.time()
     r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload",
                         "tiny_f32", "--steps", "3", "--warmup", "3"], capture_output=True, text=True, timeout=300)
+    wall = time.time() - t0
     assert r.returncode == 0, r.stderr
     line = json.loads(r.stdout.strip().splitlines()[-1])
     assert line["impl"] == "reference" and line["unit"] == "us/call" and line["value"] > 0
     assert line["cpu_baseline"]["kind"] == "oracle" and line["e2e"]["h2d_bytes_per_step"] == 0
+    # the whole batch fits the budget: no scaling, and the measured steps fit the run
+    assert line["config"]["images_per_step"] == 1
+    assert abs(line["value"] - line["ms_per_step"] * 1e3) <= 1e-3 * line["value"] + 0.1
+    assert line["ms_per_step"] * (line["steps"] + line["warmup"]) / 1e3 <= wall
+    assert line["cpu_baseline"]["cores"] == 1          # one image: one thread does the work
+
+
+def test_config_record_fractions():
+    w = gen.WORKLOADS["stage1_f16"]
+    rec = bench.config_record(w, {"fwd": 100.0, "bwd_offset_mask": 150.0, "bwd_value": 50.0},
+                              {"hbm_gbs": 6000.0})
+    assert rec["fwd_us"] == 100.0 and rec["bwd_us"] == 200.0
+    assert rec["fwd_gbs"] == round(96_337_920 / 100e-6 / 1e9, 1)
+    assert rec["bwd_frac_hbm"] == round(166_985_728 / 200e-6 / 1e9 / 6000.0, 4)
+    assert rec["fwd_frac_8tbs"] == round(96_337_920 / 100e-6 / 1e9 / 8000.0, 4)
 
 
 def test_reference_arm_other_ranks_exit_quietly():
