@@ -87,6 +87,7 @@ def _load() -> ctypes.CDLL:
         "dcn4_backward_noalloc": ([P, vp, vp, vp, vp, vp, vp], ctypes.c_int),
         "dcn4_backward_noalloc_capacity": ([], ctypes.c_size_t),
         "dcn4_noalloc_last_error": ([], ctypes.c_char_p),
+        "dcn4_backward_diagnostics": ([P, vp, ctypes.c_size_t, ip, vp], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         fn = getattr(L, name)
@@ -154,6 +155,14 @@ def dcn4_backward_value(p: dcn4_params, offset_mask, grad_out, grad_value, works
                         stream=None) -> int:
     return lib.dcn4_backward_value(ctypes.byref(p), offset_mask, grad_out, grad_value, workspace,
                                    workspace_bytes, stream)
+
+
+def dcn4_backward_diagnostics(p: dcn4_params, workspace, workspace_bytes: int, stream=None):
+    """(status, [corrupt bucket tiles, rescanned tiles, direct-path tiles]) of the last
+    backward run on `workspace`; waits for `stream`."""
+    counts = (ctypes.c_int * 3)()
+    st = lib.dcn4_backward_diagnostics(ctypes.byref(p), workspace, workspace_bytes, counts, stream)
+    return st, list(counts)
 
 
 def dcn4_backward_noalloc(p: dcn4_params, value, offset_mask, grad_out, grad_value, grad_offset_mask,
@@ -230,7 +239,9 @@ def forward_linear(p: dcn4_params, value, x, weight, bias=None, out=None, offset
 
 def backward(p: dcn4_params, value, offset_mask, grad_out, grad_value=None, grad_offset_mask=None,
              workspace=None):
-    """(grad_value[N,H,W,C], grad_offset_mask[N,Ho,Wo,P]) for CUDA tensors."""
+    """(grad_value[N,H,W,C], grad_offset_mask[N,Ho,Wo,P]) for CUDA tensors.  `workspace`
+    (a uint8 CUDA tensor of dcn4_backward_workspace_size bytes) is allocated when not
+    given; pass one to read the call's fallback counters with backward_diagnostics."""
     import torch
     st, Ho, Wo = dcn4_output_dims(p)
     check(st)
@@ -248,6 +259,13 @@ def backward(p: dcn4_params, value, offset_mask, grad_out, grad_value=None, grad
                         grad_value.data_ptr(), grad_offset_mask.data_ptr(), ws_ptr, ws_bytes,
                         _stream_handle(value.device)))
     return grad_value, grad_offset_mask
+
+
+def backward_diagnostics(p: dcn4_params, workspace) -> dict:
+    """Fallback counters of the last backward on `workspace` (a uint8 CUDA tensor)."""
+    st, c = dcn4_backward_diagnostics(p, workspace.data_ptr(), workspace.numel(), _stream_handle(workspace.device))
+    check(st)
+    return {"corrupt_bucket_tiles": c[0], "rescanned_tiles": c[1], "direct_tiles": c[2]}
 
 
 # ---------------------------------------------------------------------------

@@ -212,34 +212,44 @@ int make_geometry(const dcn4_params* p, bool backward, bool wide, dcn4::Geometry
     return DCN4_OK;
 }
 
-// Backward workspace, each part starting on a 256-byte boundary: one reach
-// word per image, one cell bounding box (4 bytes) per output pixel; then for
-// fp32 a 2-byte cell code per sample, for 16-bit dtypes (with buckets) one
-// record counter per grad_value tile and each tile's bucket of bcap 12-byte
-// records (4-byte output pixel + 8-byte bin, mask bits and fractions).
+// Backward workspace, each part starting on a 256-byte boundary.  The header
+// (zeroed by one memset per call): kDiagWords fallback counters, one reach word
+// per image (stored as R + 1, 0: no sample touches the image), and for 16-bit
+// dtypes with buckets one record counter per grad_value tile.  Then one cell
+// box (4 bytes) per output pixel; then for fp32 a 2-byte cell code per sample,
+// for 16-bit dtypes (with buckets) each tile's bucket of bcap records: 4-byte
+// output pixels, then 8-byte bin, mask bits and fractions.
 size_t round256(size_t b) { return (b + 255) / 256 * 256; }
-size_t reach_bytes(const dcn4::Geometry& g) { return round256(static_cast<size_t>(g.N) * sizeof(int)); }
+size_t num_value_tiles(const dcn4::Geometry& g) { return static_cast<size_t>(g.N) * g.btiles_h * g.btiles_w; }
+size_t header_words(const dcn4::Geometry& g, int dtype) {
+    return dcn4::kDiagWords + static_cast<size_t>(g.N) + (dtype != DCN4_F32 && g.buckets ? num_value_tiles(g) : 0);
+}
+size_t header_bytes(const dcn4::Geometry& g, int dtype) { return round256(header_words(g, dtype) * sizeof(int)); }
 size_t box_bytes(const dcn4::Geometry& g) { return round256(static_cast<size_t>(g.total_pix) * 4); }
 size_t num_samples(const dcn4::Geometry& g) { return static_cast<size_t>(g.total_pix) * g.G * g.K; }
-size_t num_value_tiles(const dcn4::Geometry& g) { return static_cast<size_t>(g.N) * g.btiles_h * g.btiles_w; }
-size_t count_bytes(const dcn4::Geometry& g) { return round256(num_value_tiles(g) * sizeof(int)); }
 size_t workspace_bytes(const dcn4::Geometry& g, int dtype) {
-    size_t b = reach_bytes(g) + box_bytes(g);
+    size_t b = header_bytes(g, dtype) + box_bytes(g);
     if (dtype == DCN4_F32) return b + round256(num_samples(g) * 2);
     if (!g.buckets) return b;
     const size_t recs = num_value_tiles(g) * static_cast<size_t>(g.bcap);
-    return b + count_bytes(g) + round256(recs * 4) + recs * 8;
+    return b + round256(recs * 4) + recs * 8;
+}
+int* reach_words(void* workspace) { return static_cast<int*>(workspace) + dcn4::kDiagWords; }
+uint32_t* box_words(const dcn4::Geometry& g, int dtype, void* workspace) {
+    return reinterpret_cast<uint32_t*>(static_cast<char*>(workspace) + header_bytes(g, dtype));
 }
 dcn4::SampleArrays sample_arrays(const dcn4::Geometry& g, int dtype, const void* workspace) {
-    char* base = static_cast<char*>(const_cast<void*>(workspace)) + reach_bytes(g) + box_bytes(g);
+    char* ws = static_cast<char*>(const_cast<void*>(workspace));
+    char* base = ws + header_bytes(g, dtype) + box_bytes(g);
     dcn4::SampleArrays sa = {};
+    sa.diag = reinterpret_cast<int*>(ws);
     if (dtype == DCN4_F32) {
         sa.code = reinterpret_cast<uint16_t*>(base);
     } else if (g.buckets) {
         const size_t recs = num_value_tiles(g) * static_cast<size_t>(g.bcap);
-        sa.tile_count = reinterpret_cast<int*>(base);
-        sa.bucket_pix = reinterpret_cast<uint32_t*>(base + count_bytes(g));
-        sa.bucket_rec = reinterpret_cast<uint64_t*>(base + count_bytes(g) + round256(recs * 4));
+        sa.tile_count = reach_words(ws) + g.N;
+        sa.bucket_pix = reinterpret_cast<uint32_t*>(base);
+        sa.bucket_rec = reinterpret_cast<uint64_t*>(base + round256(recs * 4));
     }
     return sa;
 }
@@ -341,16 +351,13 @@ int dcn4_backward_offset_mask(const dcn4_params* p, const void* value, const voi
     if (!workspace || workspace_bytes < need)
         return fail(DCN4_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, workspace_bytes);
     if (!aligned16(workspace)) return fail(DCN4_ERR_MISALIGNED, "workspace must be 16-byte aligned");
-    int* reach = static_cast<int*>(workspace);
-    uint32_t* boxes = reinterpret_cast<uint32_t*>(static_cast<char*>(workspace) + reach_bytes(g));
+    int* reach = reach_words(workspace);
+    uint32_t* boxes = box_words(g, p->dtype, workspace);
     const dcn4::SampleArrays sa = sample_arrays(g, p->dtype, workspace);
     const cudaStream_t s = static_cast<cudaStream_t>(stream);
-    cudaError_t e = cudaMemsetAsync(reach, 0xff, static_cast<size_t>(g.N) * sizeof(int), s);  // reach = -1
-    if (e != cudaSuccess) return fail(DCN4_ERR_LAUNCH, "reach reset: %s", cudaGetErrorString(e));
-    if (g.buckets) {
-        e = cudaMemsetAsync(sa.tile_count, 0, num_value_tiles(g) * sizeof(int), s);
-        if (e != cudaSuccess) return fail(DCN4_ERR_LAUNCH, "bucket reset: %s", cudaGetErrorString(e));
-    }
+    // counters, reach words and bucket counters: one memset
+    cudaError_t e = cudaMemsetAsync(workspace, 0, header_words(g, p->dtype) * sizeof(int), s);
+    if (e != cudaSuccess) return fail(DCN4_ERR_LAUNCH, "workspace reset: %s", cudaGetErrorString(e));
     e = dcn4::launch_backward_samples(g, p->dtype, value, offset_mask, grad_out, grad_offset_mask, reach, sa, boxes, s);
     if (e != cudaSuccess) return fail(DCN4_ERR_LAUNCH, "grad_offset_mask launch: %s", cudaGetErrorString(e));
 
@@ -371,8 +378,8 @@ int dcn4_backward_value(const dcn4_params* p, const void* offset_mask, const voi
     if (!workspace || workspace_bytes < need)
         return fail(DCN4_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, workspace_bytes);
     if (!aligned16(workspace)) return fail(DCN4_ERR_MISALIGNED, "workspace must be 16-byte aligned");
-    const int* reach = static_cast<const int*>(workspace);
-    const uint32_t* boxes = reinterpret_cast<const uint32_t*>(static_cast<const char*>(workspace) + reach_bytes(g));
+    const int* reach = reach_words(const_cast<void*>(workspace));
+    const uint32_t* boxes = box_words(g, p->dtype, const_cast<void*>(workspace));
     const dcn4::SampleArrays sa = sample_arrays(g, p->dtype, workspace);
     const cudaError_t e = dcn4::launch_backward_value(g, p->dtype, offset_mask, grad_out, grad_value, reach, sa,
                                                       boxes, static_cast<cudaStream_t>(stream));
@@ -393,6 +400,29 @@ int dcn4_backward(const dcn4_params* p, const void* value, const void* offset_ma
                                             workspace_bytes, stream);
     if (a != DCN4_OK) return a;
     return dcn4_backward_value(p, offset_mask, grad_out, grad_value, workspace, workspace_bytes, stream);
+}
+
+int dcn4_backward_diagnostics(const dcn4_params* p, const void* workspace, size_t workspace_bytes, int* counts,
+                              void* stream) {
+    dcn4::Geometry g;
+    const int st = make_geometry(p, true, false, &g);
+    if (st != DCN4_OK) return st;
+    if (!counts) return fail(DCN4_ERR_NULL, "counts must be non-NULL");
+    counts[0] = counts[1] = counts[2] = 0;
+    if (g.total_pix == 0) return DCN4_OK;
+    const size_t need = dcn4_backward_workspace_size(p);
+    if (!workspace || workspace_bytes < need)
+        return fail(DCN4_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, workspace_bytes);
+    if (!aligned16(workspace)) return fail(DCN4_ERR_MISALIGNED, "workspace must be 16-byte aligned");
+    int host[dcn4::kDiagWords] = {};
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemcpyAsync(host, workspace, sizeof host, cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return fail(DCN4_ERR_LAUNCH, "diagnostics read: %s", cudaGetErrorString(e));
+    counts[0] = host[dcn4::kDiagCorruptBucket];
+    counts[1] = host[dcn4::kDiagRescan];
+    counts[2] = host[dcn4::kDiagDirect];
+    return DCN4_OK;
 }
 
 const char* dcn4_status_string(int status) {

@@ -461,7 +461,7 @@ __global__ void __launch_bounds__(256, 3) samples_kernel(const Geometry g, const
         __syncthreads();
         write_out(K);
     }
-    if (threadIdx.x == 0 && s_reach >= 0) atomicMax(reach + t.n, s_reach);
+    if (threadIdx.x == 0 && s_reach >= 0) atomicMax(reach + t.n, s_reach + 1);  // stored as R + 1; 0: no sample
     for (int i = threadIdx.x; i < t.th * g.TW; i += blockDim.x) {
         const int r2 = i / g.TW, c2 = i - r2 * g.TW;
         if (c2 >= t.tw) continue;
@@ -761,7 +761,7 @@ __global__ void __launch_bounds__(256, 2) value_kernel(const Geometry g, const T
     for (int i = threadIdx.x; i < nbins; i += nthr) cnt[i] = 0;
 
     bool sorted = false;
-    const int R = reach[n];
+    const int R = reach[n] - 1;  // -1: no sample of the image touches it
     // The filing pass trusts the cell codes only up to kCodeReach.
     const int nfiled = (COMPACT && g.buckets && compact_ok && R <= kCodeReach) ? sa.tile_count[blockIdx.x] : -1;
     if (nfiled >= 0 && nfiled <= g.bcap) {
@@ -823,7 +823,11 @@ __global__ void __launch_bounds__(256, 2) value_kernel(const Geometry g, const T
         }
         __syncthreads();
         sorted = s_fail == 0;
+        // A bucket that failed the checks: counted, so that callers and tests can
+        // tell that it happened (the tile's result is still exact).
+        if (!sorted && threadIdx.x == 0) atomicAdd(sa.diag + kDiagCorruptBucket, 1);
     } else {
+        if (COMPACT && g.buckets && threadIdx.x == 0) atomicAdd(sa.diag + kDiagRescan, 1);
         // Rescan: samples that can touch the tile come from output pixels
         // whose anchor (for the sample's grid point) lies within R of the tile
         // and whose cell box meets the tile's cells.
@@ -1038,6 +1042,7 @@ __global__ void __launch_bounds__(256, 2) value_kernel(const Geometry g, const T
     // Direct path (records that do not fit, or a tile the sort cannot name):
     // thread -> (input pixel, group, slice) of the tile, scanning every
     // candidate sample of its group.
+    if (threadIdx.x == 0) atomicAdd(sa.diag + kDiagDirect, 1);
     const int lanes_pp = g.G * g.nslice;
     const int uh_lo = max(0, ceil_div(y0 - R + g.ph - (g.kh - 1) * g.dh, g.sh));
     const int uh_hi = min(g.Ho - 1, floor_div(y0 + bh - 1 + R + g.ph, g.sh));

@@ -60,7 +60,16 @@ struct SampleArrays {
     int* tile_count;
     uint32_t* bucket_pix;
     uint64_t* bucket_rec;
+    int* diag;  // fallback counters of the grad_value pass (kDiag*)
 };
+// Counters the grad_value pass keeps per call: tiles whose bucket failed the
+// consistency checks (taken by the direct path), tiles that rescanned the
+// offsets (bucket overflow, or a sample beyond the filing window), and tiles
+// that took the direct path for any reason.
+constexpr int kDiagCorruptBucket = 0;
+constexpr int kDiagRescan = 1;
+constexpr int kDiagDirect = 2;
+constexpr int kDiagWords = 4;
 constexpr int kBucketOverflow = 1 << 30;
 
 template <typename T>

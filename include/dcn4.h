@@ -67,7 +67,7 @@
 extern "C" {
 #endif
 
-#define DCN4_VERSION 120  /* 1.2.0: dcn4_forward_linear */
+#define DCN4_VERSION 130  /* 1.3.0: dcn4_backward_diagnostics */
 
 typedef enum {
     DCN4_F32 = 0,   /* IEEE binary32            */
@@ -150,14 +150,15 @@ int dcn4_forward_linear(const dcn4_params* p, int Cx, const void* value, const v
                         const void* bias, void* out, void* offset_mask_out, void* stream);
 
 /* Bytes of device workspace dcn4_backward needs, each part rounded up to 256
- * bytes: one 32-bit word per image, one 32-bit cell box per output pixel
- * (N*Ho*Wo), then
+ * bytes: a header of 32-bit words (4 fallback counters, one word per image,
+ * and for fp16/bf16 one record counter per grad_value tile), one 32-bit cell
+ * box per output pixel (N*Ho*Wo), then
  *   fp32:      a 2-byte cell code per sample (N*Ho*Wo*G*K of them);
- *   fp16/bf16: a 32-bit counter per grad_value tile and, per tile, room for
- *              bcap 12-byte sample records (4-byte output pixel + 8 bytes of
- *              bin, mask bits and fixed-point bilinear fractions), where the
- *              tiles and bcap follow from the shape (about 1.06x the records
- *              a tile expects, + 512);
+ *   fp16/bf16: per grad_value tile, room for bcap 12-byte sample records
+ *              (4-byte output pixel + 8 bytes of bin, mask bits and
+ *              fixed-point bilinear fractions), where the tiles and bcap
+ *              follow from the shape (about 1.06x the records a tile
+ *              expects, + 512);
  * 0 if p is invalid. */
 size_t dcn4_backward_workspace_size(const dcn4_params* p);
 
@@ -233,6 +234,19 @@ int dcn4_backward_offset_mask(const dcn4_params* p, const void* value, const voi
                               size_t workspace_bytes, void* stream);
 int dcn4_backward_value(const dcn4_params* p, const void* offset_mask, const void* grad_out,
                         void* grad_value, const void* workspace, size_t workspace_bytes, void* stream);
+
+/* Fallback counters of the last dcn4_backward (or dcn4_backward_value) run on
+ * `workspace` for the same params: counts[0] = grad_value tiles whose filed
+ * sample records failed the kernel's consistency checks (each such tile is
+ * recomputed by the direct path, so the gradient stays exact; a nonzero count
+ * means a filing fault), counts[1] = tiles that rescanned the offsets instead
+ * of reading their records (bucket overflow, samples beyond the filing
+ * window, or images of very large reach), counts[2] = tiles that took the
+ * direct path for any reason.  Copies 16 bytes from the workspace to the host
+ * on `stream` and waits for it (the one synchronising call of the library).
+ * Same checks as dcn4_backward; counts must hold 3 ints. */
+int dcn4_backward_diagnostics(const dcn4_params* p, const void* workspace, size_t workspace_bytes, int* counts,
+                              void* stream);
 
 /* Name of a dcn4_status. */
 const char* dcn4_status_string(int status);

@@ -47,10 +47,18 @@ def gpu_forward(w: gen.Workload, inp: dict):
 
 
 def gpu_backward(w: gen.Workload, inp: dict):
+    """The backward through the C ABI; also checks that no grad_value tile found its
+    filed sample records inconsistent (the kernel's fallback counter stays 0)."""
+    import torch
     import deformable_convolution_sampling_b200 as dcn
     p = params_for(w)
-    return dcn.backward(p, to_device(inp["value"], w.dtype), to_device(inp["offset_mask"], w.dtype),
-                        to_device(inp["grad_out"], w.dtype))
+    ws = torch.empty(max(dcn.dcn4_backward_workspace_size(p), 16), dtype=torch.uint8, device="cuda")
+    out = dcn.backward(p, to_device(inp["value"], w.dtype), to_device(inp["offset_mask"], w.dtype),
+                       to_device(inp["grad_out"], w.dtype), workspace=ws)
+    if p.N > 0:
+        diag = dcn.backward_diagnostics(p, ws)
+        assert diag["corrupt_bucket_tiles"] == 0, diag
+    return out
 
 
 def take(inp: dict, idx) -> dict:

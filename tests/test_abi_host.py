@@ -70,7 +70,7 @@ def test_params_mirror_matches_the_header(dcn):
             fields += [n.strip() for n in names.split(",")]
     assert [f[0] for f in dcn.dcn4_params._fields_] == fields
     assert ctypes.sizeof(dcn.dcn4_params) == 4 * len(fields)
-    assert dcn.dcn4_version() == 120
+    assert dcn.dcn4_version() == 130
 
 
 def test_library_does_not_link_the_oracle(dcn):
@@ -119,10 +119,11 @@ def test_workspace_size(dcn):
     tiles = 64 * 7 * 2
     expect = 4 * 9 * 32 * 9
     cap = expect + expect // 16 + 512
-    assert dcn.dcn4_backward_workspace_size(p) == (256 + up(64 * 56 * 56 * 4) + up(tiles * 4)
+    header = up((4 + 64 + tiles) * 4)          # counters, reach words, bucket counters
+    assert dcn.dcn4_backward_workspace_size(p) == (header + up(64 * 56 * 56 * 4)
                                                    + up(tiles * cap * 4) + tiles * cap * 8)
     p = dcn.make_params(N=100, H=8, W=8, G=2, Cg=8, dtype="f32", remove_center=1)
-    assert dcn.dcn4_backward_workspace_size(p) == 512 + up(100 * 64 * 4) + up(100 * 64 * 2 * 8 * 2)
+    assert dcn.dcn4_backward_workspace_size(p) == up((4 + 100) * 4) + up(100 * 64 * 4) + up(100 * 64 * 2 * 8 * 2)
     p.Cg = 6
     assert dcn.dcn4_backward_workspace_size(p) == 0
 
@@ -186,6 +187,27 @@ assert dcn.dcn4_backward(p, 16, 32, 48, 64, 80, 97, 1 << 20, None) == -4
 assert dcn.dcn4_backward(p, 16, 32, 48, 64, 80, None, 0, None) == -6
 assert dcn.dcn4_backward(p, 16, 32, 48, 64, 80, 96, 100, None) == -6
 assert dcn.lib.dcn4_forward(None, None, None, None, None) == -1
+""")
+
+
+def test_diagnostics_checks_before_reading():
+    """dcn4_backward_diagnostics validates its arguments on the host (NULL counts,
+    missing or small workspace) before any copy; made-up addresses only in a child
+    process that sees no GPU."""
+    run_without_gpu("""
+import ctypes
+p = dcn.make_params(N=2, H=8, W=8, G=2, Cg=8, dtype="f16")
+st, c = dcn.dcn4_backward_diagnostics(p, None, 0)
+assert st == -6 and c == [0, 0, 0], (st, c)
+st, c = dcn.dcn4_backward_diagnostics(p, 256, 100)
+assert st == -6, st
+st, c = dcn.dcn4_backward_diagnostics(p, 264, 1 << 24)
+assert st == -4, st
+assert dcn.lib.dcn4_backward_diagnostics(ctypes.byref(p), None, 0, None, None) == -1
+bad = dcn.make_params(N=2, H=8, W=8, G=2, Cg=8, dtype="f16")
+bad.P = 50
+st, c = dcn.dcn4_backward_diagnostics(bad, None, 0)
+assert st == -3, st
 """)
 
 

@@ -260,6 +260,18 @@ def test_samples_clustered_on_one_cell(dtype):
     inp["offset_mask"][0, ..., : w.G * 27] = body.reshape(w.Ho, w.Wo, w.G * 27)
     _check_forward(w, inp)
     _check_backward(w, inp)
+    diag = _diagnostics(w, inp)
+    assert diag["corrupt_bucket_tiles"] == 0 and diag["direct_tiles"] > 0, diag
+
+
+def _diagnostics(w, inp):
+    """Fallback counters of one backward through the C ABI on these inputs."""
+    import torch
+    import deformable_convolution_sampling_b200 as dcn
+    p = params_for(w)
+    ws = torch.empty(dcn.dcn4_backward_workspace_size(p), dtype=torch.uint8, device="cuda")
+    dcn.backward(p, *(to_device(inp[k], w.dtype) for k in ("value", "offset_mask", "grad_out")), workspace=ws)
+    return dcn.backward_diagnostics(p, ws)
 
 
 def test_images_with_different_reach():
@@ -344,6 +356,21 @@ def test_samples_beyond_the_filing_window():
     inp["offset_mask"][..., : w.G * 27] = body.reshape(w.N, w.Ho, w.Wo, w.G * 27)
     _check_forward(w, inp)
     _check_backward(w, inp)
+    diag = _diagnostics(w, inp)
+    assert diag["corrupt_bucket_tiles"] == 0 and diag["rescanned_tiles"] > 0, diag
+
+
+@pytest.mark.parametrize("name", gen.WORKLOAD_ORDER)
+def test_no_fallback_tiles_on_the_workloads(name):
+    """On every measured workload no grad_value tile finds its filed records
+    inconsistent (the counter of tiles sent to the direct path by a failed bucket
+    check stays 0)."""
+    w = gen.WORKLOADS[name]
+    if w.N > 8:
+        w = gen.custom(**{**w.__dict__, "N": 8, "name": name + "_8"})
+    inp = gen.make_inputs(w)
+    diag = _diagnostics(w, inp)
+    assert diag["corrupt_bucket_tiles"] == 0, diag
 
 
 # ---------------------------------------------------------------------------
