@@ -382,7 +382,8 @@ __global__ void __launch_bounds__(256, kFwdCtasPerSm) forward_kernel(const Geome
         }
         __syncthreads();
         const Tile t = tile_at(g, tile);
-        const T* om_s = bufs[it & 1];
+        // the tile's rows, addressed from smem directly so the reads stay shared-space loads
+        const T* om_s = reinterpret_cast<const T*>(smem) + (LIN ? 0 : (it & 1) * tile_elems);
         if constexpr (LIN) {
             switch (lin.w_smem ? lin.Cx / 16 : 0) {
                 case 1: linear_tile_staged<T, 1>(g, lin, xbuf[it & 1], w_s, bufs[0], b_s); break;
@@ -413,27 +414,92 @@ __global__ void __launch_bounds__(256, kFwdCtasPerSm) forward_kernel(const Geome
             for (int i = 0; i < PAIRS; ++i) acc[i] = make_float2(0.f, 0.f);
             float inv = 1.f;
             if constexpr (SM) inv = softmax_exps(row + 2 * K, K, e_s + threadIdx.x, blockDim.x).y;
-            int k = 0;
-#pragma unroll
-            for (int iw = 0; iw < kw; ++iw) {
-                const float wbase = static_cast<float>(wb + iw * g.dw);
-#pragma unroll
-                for (int ih = 0; ih < kh; ++ih) {
-                    if (rc && iw == kw / 2 && ih == kh / 2) continue;
-                    const float dx = to_f32(row[2 * k]);
-                    const float dy = to_f32(row[2 * k + 1]);
-                    float m = to_f32(row[2 * K + k]);
-                    if constexpr (SM) m = e_s[k * blockDim.x + threadIdx.x] * inv;
-                    ++k;
+            if constexpr (KH > 0) {
+                // Compile-time grid: two-stage pipeline.  The four corner slices of
+                // sample k + 1 are requested before the FMAs of sample k, so each
+                // thread keeps eight 32-byte loads in flight instead of four.
+                constexpr int KK = KH * KW - (RC ? 1 : 0);
+                uint4 raw[2][4][VEC];
+                float wts[2][4];
+                auto issue = [&](int kk, int ih, int iw, uint4 (&r)[4][VEC], float (&wt)[4]) {
+                    const float dx = to_f32(row[2 * kk]);
+                    const float dy = to_f32(row[2 * kk + 1]);
+                    float m = to_f32(row[2 * K + kk]);
+                    if constexpr (SM) m = e_s[kk * blockDim.x + threadIdx.x] * inv;
                     const float h = __fmaf_rn(g.s, dy, static_cast<float>(hb + ih * g.dh));
-                    const float w = __fmaf_rn(g.s, dx, wbase);
+                    const float w = __fmaf_rn(g.s, dx, static_cast<float>(wb + iw * g.dw));
                     const Cell<T> cell = bilinear_cell(g, img, h, w);
                     const float b = m * cell.lh, a = m - b;
                     const float wl = 1.f - cell.lw;
-                    accumulate<T, VEC>(acc, cell.c[0], a * wl);
-                    accumulate<T, VEC>(acc, cell.c[1], a * cell.lw);
-                    accumulate<T, VEC>(acc, cell.c[2], b * wl);
-                    accumulate<T, VEC>(acc, cell.c[3], b * cell.lw);
+                    wt[0] = a * wl;
+                    wt[1] = a * cell.lw;
+                    wt[2] = b * wl;
+                    wt[3] = b * cell.lw;
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        if constexpr (VEC == 2) {
+                            ld_gather32(cell.c[c], r[c][0], r[c][1]);
+                        } else {
+                            r[c][0] = ld_gather(cell.c[c]);
+                        }
+                    }
+                };
+                auto consume = [&](const uint4 (&r)[4][VEC], const float (&wt)[4]) {
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        const float2 w2 = make_float2(wt[c], wt[c]);
+#pragma unroll
+                        for (int v = 0; v < VEC; ++v) {
+                            float2 f[EPV / 2];
+                            unpack(r[c][v], f, T());
+#pragma unroll
+                            for (int i = 0; i < EPV / 2; ++i)
+                                acc[v * (EPV / 2) + i] = __ffma2_rn(w2, f[i], acc[v * (EPV / 2) + i]);
+                        }
+                    }
+                };
+                // point kk -> grid cell (ih, iw): columns outer, rows inner, centre skipped
+                auto cell_of = [](int kk, int& ih, int& iw) {
+                    int idx = kk;
+                    if (RC && idx >= (KW / 2) * KH + KH / 2) ++idx;
+                    iw = idx / KH;
+                    ih = idx - iw * KH;
+                };
+                {
+                    int ih, iw;
+                    cell_of(0, ih, iw);
+                    issue(0, ih, iw, raw[0], wts[0]);
+                }
+#pragma unroll
+                for (int kk = 0; kk < KK; ++kk) {
+                    if (kk + 1 < KK) {
+                        int ih, iw;
+                        cell_of(kk + 1, ih, iw);
+                        issue(kk + 1, ih, iw, raw[(kk + 1) & 1], wts[(kk + 1) & 1]);
+                    }
+                    consume(raw[kk & 1], wts[kk & 1]);
+                }
+            } else {
+                int k = 0;
+                for (int iw = 0; iw < kw; ++iw) {
+                    const float wbase = static_cast<float>(wb + iw * g.dw);
+                    for (int ih = 0; ih < kh; ++ih) {
+                        if (rc && iw == kw / 2 && ih == kh / 2) continue;
+                        const float dx = to_f32(row[2 * k]);
+                        const float dy = to_f32(row[2 * k + 1]);
+                        float m = to_f32(row[2 * K + k]);
+                        if constexpr (SM) m = e_s[k * blockDim.x + threadIdx.x] * inv;
+                        ++k;
+                        const float h = __fmaf_rn(g.s, dy, static_cast<float>(hb + ih * g.dh));
+                        const float w = __fmaf_rn(g.s, dx, wbase);
+                        const Cell<T> cell = bilinear_cell(g, img, h, w);
+                        const float b = m * cell.lh, a = m - b;
+                        const float wl = 1.f - cell.lw;
+                        accumulate<T, VEC>(acc, cell.c[0], a * wl);
+                        accumulate<T, VEC>(acc, cell.c[1], a * cell.lw);
+                        accumulate<T, VEC>(acc, cell.c[2], b * wl);
+                        accumulate<T, VEC>(acc, cell.c[3], b * cell.lw);
+                    }
                 }
             }
             T* dst = out + ((static_cast<long long>(t.n) * g.Ho + ho) * g.Wo + wo) * g.C + ch_off;
