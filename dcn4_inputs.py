@@ -38,6 +38,7 @@ _M2 = np.uint64(0x94D049BB133111EB)
 
 STREAM_VALUE, STREAM_OFFSET, STREAM_MASK, STREAM_GRAD = 1, 2, 3, 4
 STREAM_X, STREAM_WEIGHT, STREAM_BIAS = 5, 6, 7
+STREAM_REF = 8
 
 
 def _splitmix64(z: np.ndarray) -> np.ndarray:
@@ -278,3 +279,91 @@ def custom(name: str = "custom", **kw) -> Workload:
     base = dict(value=("normal", 0.0, 1.0), offset=("normal", 0.0, 1.5), mask=("normal", 0.0, 0.5))
     base.update(kw)
     return Workload(name=name, **base)
+
+
+# ---------------------------------------------------------------------------
+# Deformable attention (single scale): value [N,H,W,G*Cg], reference points
+# ref [N,Nq,2] (fp32, (x, y) in pixel coordinates), offset_logits [N,Nq,P]
+# (per group K (dx, dy) pairs, then K logits), grad_out [N,Nq,G*Cg].
+# ---------------------------------------------------------------------------
+
+@dataclasses.dataclass(frozen=True)
+class AttnWorkload:
+    name: str
+    N: int
+    H: int
+    W: int
+    G: int
+    Cg: int
+    Nq: int
+    K: int
+    P: int
+    dtype: str
+    offset_scale: float = 1.0
+    # "pixels": one query per pixel, reference at its centre (Nq = H*W, row-major);
+    # ("uniform", margin): reference points uniform over [-margin, W-1+margin] x [-margin, H-1+margin]
+    ref: object = "pixels"
+    value: tuple = ("normal", 0.0, 1.0)
+    offset: tuple = ("normal", 0.0, 2.0)
+    logit: tuple = ("normal", 0.0, 1.0)
+    grad_out: tuple = ("normal", 0.0, 1.0)
+    seed: int = 0
+
+    @property
+    def C(self) -> int:
+        return self.G * self.Cg
+
+    def geometry(self) -> dict:
+        return dict(N=self.N, H=self.H, W=self.W, G=self.G, Cg=self.Cg, Nq=self.Nq, K=self.K, P=self.P,
+                    offset_scale=self.offset_scale)
+
+    def describe(self) -> str:
+        ref = "pixel-centre queries" if self.ref == "pixels" else f"{self.Nq} queries at random reference points"
+        return (f"N{self.N} H{self.H} W{self.W} C{self.C} G{self.G} (C'={self.Cg}) Nq{self.Nq} K{self.K} "
+                f"P{self.P} offset_scale {self.offset_scale} {self.dtype}, {ref}")
+
+
+ATTN_WORKLOADS: dict[str, AttnWorkload] = {
+    w.name: w
+    for w in [
+        AttnWorkload("attn_tiny_f32", N=1, H=8, W=8, G=2, Cg=8, Nq=32, K=4, P=24, dtype="f32",
+                     ref=("uniform", 1.0), offset=("uniform", -2.0, 2.0)),
+        # encoder-style self-attention on one 64x64 map: every pixel queries K=4 points per head
+        AttnWorkload("attn_enc_f16", N=8, H=64, W=64, G=8, Cg=32, Nq=64 * 64, K=4, P=96, dtype="f16"),
+        # decoder-style: 300 object queries per image at random reference points
+        AttnWorkload("attn_dec_bf16", N=8, H=64, W=64, G=8, Cg=32, Nq=300, K=4, P=96, dtype="bf16",
+                     ref=("uniform", 0.0), offset=("normal", 0.0, 4.0)),
+    ]
+}
+ATTN_WORKLOAD_ORDER = ["attn_tiny_f32", "attn_enc_f16", "attn_dec_bf16"]
+
+
+def attn_custom(name: str = "attn_custom", **kw) -> AttnWorkload:
+    return AttnWorkload(name=name, **kw)
+
+
+def make_attn_inputs(w: AttnWorkload, *, seed: int | None = None, tail_fill: float = math.nan,
+                     with_grad: bool = True) -> dict:
+    """value, ref_points (float32), offset_logits and (optionally) grad_out, in storage form."""
+    seed = w.seed if seed is None else seed
+    value = to_storage(draw(w.value, seed, STREAM_VALUE, w.N * w.H * w.W * w.C), w.dtype).reshape(
+        w.N, w.H, w.W, w.C)
+    if w.ref == "pixels":
+        if w.Nq != w.H * w.W:
+            raise ValueError("pixel-centre queries need Nq = H*W")
+        ys, xs = np.divmod(np.arange(w.Nq), w.W)
+        ref = np.broadcast_to(np.stack([xs, ys], axis=-1).astype(np.float32), (w.N, w.Nq, 2)).copy()
+    else:
+        kind, margin = w.ref
+        u = uniform01(seed, STREAM_REF, w.N * w.Nq * 2).reshape(w.N, w.Nq, 2)
+        span = np.array([w.W - 1 + 2 * margin, w.H - 1 + 2 * margin])
+        ref = (-margin + u * span).astype(np.float32)
+    ns = w.N * w.Nq * w.G * w.K
+    offs = to_storage(draw(w.offset, seed, STREAM_OFFSET, 2 * ns), w.dtype).reshape(w.N, w.Nq, w.G, w.K, 2)
+    logits = to_storage(draw(w.logit, seed, STREAM_MASK, ns), w.dtype).reshape(w.N, w.Nq, w.G, w.K)
+    out = {"value": value, "ref_points": ref,
+           "offset_logits": assemble_offset_mask(offs, logits, w.P, w.dtype, tail_fill)}
+    if with_grad:
+        out["grad_out"] = to_storage(draw(w.grad_out, seed, STREAM_GRAD, w.N * w.Nq * w.C), w.dtype).reshape(
+            w.N, w.Nq, w.C)
+    return out

@@ -86,6 +86,47 @@ class Problem:
         )
 
 
+class _AttnProblem(ctypes.Structure):
+    _fields_ = [
+        ("N", ctypes.c_int), ("H", ctypes.c_int), ("W", ctypes.c_int),
+        ("G", ctypes.c_int), ("Cg", ctypes.c_int),
+        ("Nq", ctypes.c_int), ("K", ctypes.c_int),
+        ("offset_scale", ctypes.c_double),
+        ("P", ctypes.c_int),
+        ("dtype", ctypes.c_int),
+        ("location_fp32", ctypes.c_int),
+    ]
+
+
+@dataclasses.dataclass
+class AttnProblem:
+    """Geometry of one single-scale deformable attention call, as the oracle sees it."""
+
+    N: int
+    H: int
+    W: int
+    G: int
+    Cg: int
+    Nq: int
+    K: int
+    offset_scale: float = 1.0
+    P: int | None = None          # None: the smallest multiple of 8 >= G*3K
+    dtype: str = "f64"
+    location_fp32: bool = False
+
+    @property
+    def C(self) -> int:
+        return self.G * self.Cg
+
+    @property
+    def row(self) -> int:
+        return self.P if self.P is not None else -(-self.G * 3 * self.K // 8) * 8
+
+    def c_struct(self) -> _AttnProblem:
+        return _AttnProblem(self.N, self.H, self.W, self.G, self.Cg, self.Nq, self.K, float(self.offset_scale),
+                            self.row, DTYPES[self.dtype], 1 if self.location_fp32 else 0)
+
+
 _lib = None
 
 
@@ -112,6 +153,11 @@ def lib() -> ctypes.CDLL:
         L.ref_encode.restype = None
         L.ref_linear.argtypes = [ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int, vp, vp, vp, vp]
         L.ref_linear.restype = ctypes.c_int
+        AP = ctypes.POINTER(_AttnProblem)
+        L.ref_attn_forward.argtypes = [AP, vp, vp, vp, dp, ctypes.c_int]
+        L.ref_attn_forward.restype = ctypes.c_int
+        L.ref_attn_backward.argtypes = [AP, vp, vp, vp, vp, dp, dp, ctypes.c_int]
+        L.ref_attn_backward.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -207,6 +253,39 @@ def linear(dtype: str, x: np.ndarray, weight: np.ndarray, bias: np.ndarray | Non
     if lib().ref_linear(M, Cin, Cout, DTYPES[dtype], _ptr(x), _ptr(weight), b, _ptr(out)) != 0:
         raise ValueError("oracle linear rejected its arguments")
     return out
+
+
+def _attn_check(prob: AttnProblem, value, ref_points, offset_logits):
+    value = _check(value, prob, (prob.N, prob.H, prob.W, prob.C), "value")
+    offset_logits = _check(offset_logits, prob, (prob.N, prob.Nq, prob.row), "offset_logits")
+    ref_points = np.ascontiguousarray(ref_points)
+    if ref_points.dtype != np.float32 or tuple(ref_points.shape) != (prob.N, prob.Nq, 2):
+        raise ValueError(f"ref_points must be float32 [{prob.N}, {prob.Nq}, 2]")
+    return value, ref_points, offset_logits
+
+
+def attn_forward(prob: AttnProblem, value, ref_points, offset_logits, nthreads: int = 1) -> np.ndarray:
+    """Single-scale deformable attention: out[N,Nq,G*Cg] in float64."""
+    value, ref_points, offset_logits = _attn_check(prob, value, ref_points, offset_logits)
+    out = np.empty((prob.N, prob.Nq, prob.C), dtype=np.float64)
+    st = prob.c_struct()
+    if lib().ref_attn_forward(ctypes.byref(st), _ptr(value), _ptr(ref_points), _ptr(offset_logits), _dptr(out),
+                              int(nthreads)) != 0:
+        raise ValueError(f"oracle attention forward rejected {prob}")
+    return out
+
+
+def attn_backward(prob: AttnProblem, value, ref_points, offset_logits, grad_out, nthreads: int = 1):
+    """(grad_value[N,H,W,C], grad_offset_logits[N,Nq,P]) in float64."""
+    value, ref_points, offset_logits = _attn_check(prob, value, ref_points, offset_logits)
+    grad_out = _check(grad_out, prob, (prob.N, prob.Nq, prob.C), "grad_out")
+    gv = np.empty((prob.N, prob.H, prob.W, prob.C), dtype=np.float64)
+    gol = np.empty((prob.N, prob.Nq, prob.row), dtype=np.float64)
+    st = prob.c_struct()
+    if lib().ref_attn_backward(ctypes.byref(st), _ptr(value), _ptr(ref_points), _ptr(offset_logits),
+                               _ptr(grad_out), _dptr(gv), _dptr(gol), int(nthreads)) != 0:
+        raise ValueError(f"oracle attention backward rejected {prob}")
+    return gv, gol
 
 
 def host_threads() -> int:

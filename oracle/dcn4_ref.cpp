@@ -418,4 +418,148 @@ int ref_backward(const ref_problem* p, const void* value, const void* offset_mas
     return 0;
 }
 
+// ---------------------------------------------------------------------------
+// Deformable attention (single scale): see dcn4_ref.h.
+// ---------------------------------------------------------------------------
+
+static bool attn_valid(const ref_attn_problem* p) {
+    if (!p) return false;
+    if (p->N < 0 || p->H <= 0 || p->W <= 0 || p->G <= 0 || p->Cg <= 0 || p->Nq < 0 || p->K <= 0) return false;
+    if (p->dtype < REF_F32 || p->dtype > REF_F64) return false;
+    return p->P >= p->G * 3 * p->K;
+}
+
+// The sampling location of one point: reference point + offset_scale * offset.
+static void attn_location(const ref_attn_problem* p, float rx, float ry, double dx, double dy, double* h,
+                          double* w) {
+    if (p->location_fp32) {
+        const float s = static_cast<float>(p->offset_scale);
+        *h = static_cast<double>(std::fmaf(s, static_cast<float>(dy), ry));
+        *w = static_cast<double>(std::fmaf(s, static_cast<float>(dx), rx));
+    } else {
+        *h = static_cast<double>(ry) + p->offset_scale * dy;
+        *w = static_cast<double>(rx) + p->offset_scale * dx;
+    }
+}
+
+// Corner (y, x) of group g, channel c of image n; 0 outside the image.
+static double attn_pixel(const ref_attn_problem* p, const void* value, int n, int y, int x, int g, int c) {
+    if (y < 0 || y >= p->H || x < 0 || x >= p->W) return 0.0;
+    const int64_t C = static_cast<int64_t>(p->G) * p->Cg;
+    return load(value, p->dtype, ((static_cast<int64_t>(n) * p->H + y) * p->W + x) * C + static_cast<int64_t>(g) * p->Cg + c);
+}
+
+// Softmax of the K logits of one (query, group), the largest subtracted first.
+static std::vector<double> attn_weights(const ref_attn_problem* p, const void* offset_logits, int64_t row) {
+    std::vector<double> a(p->K);
+    for (int k = 0; k < p->K; ++k) a[k] = load(offset_logits, p->dtype, row + 2 * p->K + k);
+    double mx = a[0];
+    for (int k = 1; k < p->K; ++k) mx = std::max(mx, a[k]);
+    double sum = 0.0;
+    for (int k = 0; k < p->K; ++k) {
+        a[k] = std::exp(a[k] - mx);
+        sum += a[k];
+    }
+    for (int k = 0; k < p->K; ++k) a[k] /= sum;
+    return a;
+}
+
+int ref_attn_forward(const ref_attn_problem* p, const void* value, const float* ref_points,
+                     const void* offset_logits, double* out, int nthreads) {
+    if (!attn_valid(p) || !value || !ref_points || !offset_logits || !out) return -1;
+    const int64_t C = static_cast<int64_t>(p->G) * p->Cg;
+    parallel_range(static_cast<int64_t>(p->N) * p->Nq, nthreads, [&](int64_t nq) {
+        const int n = static_cast<int>(nq / (p->Nq > 0 ? p->Nq : 1));
+        const float rx = ref_points[2 * nq], ry = ref_points[2 * nq + 1];
+        for (int g = 0; g < p->G; ++g) {
+            const int64_t row = nq * p->P + static_cast<int64_t>(g) * 3 * p->K;
+            const std::vector<double> a = attn_weights(p, offset_logits, row);
+            for (int c = 0; c < p->Cg; ++c) {
+                double y = 0.0;
+                for (int k = 0; k < p->K; ++k) {
+                    double h, w;
+                    attn_location(p, rx, ry, load(offset_logits, p->dtype, row + 2 * k),
+                                  load(offset_logits, p->dtype, row + 2 * k + 1), &h, &w);
+                    // bilinear sample of the zero-extended image: nothing touched beyond [-1, H) x [-1, W)
+                    if (!(h >= -1.0 && h < p->H && w >= -1.0 && w < p->W)) continue;
+                    const double fh = std::floor(h), fw = std::floor(w);
+                    const int h0 = static_cast<int>(fh), w0 = static_cast<int>(fw);
+                    const double lh = h - fh, lw = w - fw;
+                    double smp = 0.0;
+                    for (int a2 = 0; a2 < 2; ++a2)
+                        for (int b2 = 0; b2 < 2; ++b2)
+                            smp += (a2 ? lh : 1.0 - lh) * (b2 ? lw : 1.0 - lw) *
+                                   attn_pixel(p, value, n, h0 + a2, w0 + b2, g, c);
+                    y += a[k] * smp;
+                }
+                out[nq * C + static_cast<int64_t>(g) * p->Cg + c] = y;
+            }
+        }
+    });
+    return 0;
+}
+
+int ref_attn_backward(const ref_attn_problem* p, const void* value, const float* ref_points,
+                      const void* offset_logits, const void* grad_out, double* grad_value,
+                      double* grad_offset_logits, int nthreads) {
+    if (!attn_valid(p) || !value || !ref_points || !offset_logits || !grad_out || !grad_value ||
+        !grad_offset_logits)
+        return -1;
+    const int64_t C = static_cast<int64_t>(p->G) * p->Cg;
+    const int K = p->K;
+    const double s = p->location_fp32 ? static_cast<double>(static_cast<float>(p->offset_scale)) : p->offset_scale;
+    parallel_range(p->N, nthreads, [&](int64_t n64) {
+        const int n = static_cast<int>(n64);
+        const int64_t img = static_cast<int64_t>(p->H) * p->W * C;
+        for (int64_t i = 0; i < img; ++i) grad_value[n64 * img + i] = 0.0;
+        for (int q = 0; q < p->Nq; ++q) {
+            const int64_t nq = n64 * p->Nq + q;
+            const float rx = ref_points[2 * nq], ry = ref_points[2 * nq + 1];
+            double* gol = grad_offset_logits + nq * p->P;
+            for (int e = 0; e < p->P; ++e) gol[e] = 0.0;
+            for (int g = 0; g < p->G; ++g) {
+                const int64_t row = nq * p->P + static_cast<int64_t>(g) * 3 * K;
+                const std::vector<double> a = attn_weights(p, offset_logits, row);
+                std::vector<double> gw(K, 0.0);  // <gy, S_k>
+                for (int k = 0; k < K; ++k) {
+                    double h, w;
+                    attn_location(p, rx, ry, load(offset_logits, p->dtype, row + 2 * k),
+                                  load(offset_logits, p->dtype, row + 2 * k + 1), &h, &w);
+                    if (!(h >= -1.0 && h < p->H && w >= -1.0 && w < p->W)) continue;
+                    const double fh = std::floor(h), fw = std::floor(w);
+                    const int h0 = static_cast<int>(fh), w0 = static_cast<int>(fw);
+                    const double lh = h - fh, lw = w - fw;
+                    double gS = 0.0, gdw = 0.0, gdh = 0.0;
+                    for (int c = 0; c < p->Cg; ++c) {
+                        const double gy = load(grad_out, p->dtype, nq * C + static_cast<int64_t>(g) * p->Cg + c);
+                        double v[2][2];
+                        for (int a2 = 0; a2 < 2; ++a2)
+                            for (int b2 = 0; b2 < 2; ++b2) v[a2][b2] = attn_pixel(p, value, n, h0 + a2, w0 + b2, g, c);
+                        const double S = (1 - lh) * (1 - lw) * v[0][0] + (1 - lh) * lw * v[0][1] +
+                                         lh * (1 - lw) * v[1][0] + lh * lw * v[1][1];
+                        gS += gy * S;
+                        gdw += gy * ((1 - lh) * (v[0][1] - v[0][0]) + lh * (v[1][1] - v[1][0]));
+                        gdh += gy * ((1 - lw) * (v[1][0] - v[0][0]) + lw * (v[1][1] - v[0][1]));
+                        for (int a2 = 0; a2 < 2; ++a2)
+                            for (int b2 = 0; b2 < 2; ++b2) {
+                                const int y = h0 + a2, x = w0 + b2;
+                                if (y < 0 || y >= p->H || x < 0 || x >= p->W) continue;
+                                const double wt = (a2 ? lh : 1 - lh) * (b2 ? lw : 1 - lw);
+                                grad_value[((n64 * p->H + y) * p->W + x) * C + static_cast<int64_t>(g) * p->Cg + c] +=
+                                    a[k] * wt * gy;
+                            }
+                    }
+                    gol[static_cast<int64_t>(g) * 3 * K + 2 * k] = s * a[k] * gdw;
+                    gol[static_cast<int64_t>(g) * 3 * K + 2 * k + 1] = s * a[k] * gdh;
+                    gw[k] = gS;
+                }
+                double dot = 0.0;
+                for (int k = 0; k < K; ++k) dot += a[k] * gw[k];
+                for (int k = 0; k < K; ++k) gol[static_cast<int64_t>(g) * 3 * K + 2 * K + k] = a[k] * (gw[k] - dot);
+            }
+        }
+    });
+    return 0;
+}
+
 }  // extern "C"

@@ -125,6 +125,47 @@ void ref_encode(int dtype, const double* src, void* dst, int64_t n);
 int ref_linear(int64_t M, int Cin, int Cout, int dtype, const void* x, const void* weight,
                const void* bias, void* out);
 
+/* ---------------------------------------------------------------------------
+ * Deformable attention, single scale (CSDN summary of "Efficient Deformable
+ * ConvNets", section 1.1: each query attends to a selected number of key
+ * sampling points whose positions and weights are set dynamically; section 1.2:
+ * the weights are normalised with a softmax over the points, as in DCNv3).
+ * For query q of image n and group g:
+ *     y_g(q) = sum_{k<K} A_gk * x_g(r_q + offset_scale * dp_gk),
+ *     A_gk   = exp(l_gk - max_j l_gj) / sum_j exp(l_gj - max_j l_gj)
+ * with r_q the query's reference point (x, y) in pixel coordinates of value
+ * (integer coordinates are pixel centres), dp_gk = (dx, dy) its K learned
+ * offsets, l_gk its K attention logits, and x_g(.) the bilinear sample of the
+ * zero-extended image (as the aggregation above).
+ *   value          [N, H, W, G*Cg]     dtype
+ *   ref_points     [N, Nq, 2]          fp32, (x, y)
+ *   offset_logits  [N, Nq, P]          dtype: group g owns [g*3K, (g+1)*3K):
+ *                                      K (dx, dy) pairs, then K logits
+ *   out / grad_out [N, Nq, G*Cg]
+ * --------------------------------------------------------------------------- */
+typedef struct {
+    int N, H, W;          /* value batch and spatial size                      */
+    int G, Cg;            /* groups (heads) and channels per group             */
+    int Nq, K;            /* queries per image, sampling points per query      */
+    double offset_scale;  /* multiplies the learned offsets                     */
+    int P;                /* row length of offset_logits, >= G*3K              */
+    int dtype;            /* REF_* storage type of value/offset_logits/grad_out */
+    int location_fp32;    /* 1: form the location with an fp32 fma             */
+} ref_attn_problem;
+
+/* Forward: out[N,Nq,G*Cg] (double).  nthreads > 1 splits queries across
+ * std::thread workers.  Returns 0 or -1. */
+int ref_attn_forward(const ref_attn_problem* p, const void* value, const float* ref_points,
+                     const void* offset_logits, double* out, int nthreads);
+
+/* Backward for grad_out: grad_value [N,H,W,G*Cg] (adjoint in value) and
+ * grad_offset_logits [N,Nq,P]: d<grad_out, y>/d offsets and d/d logits
+ * A_k (<gy, S_k> - sum_j A_j <gy, S_j>); the padding tail is 0.  The reference
+ * points get no gradient.  nthreads > 1 splits the batch.  Returns 0 or -1. */
+int ref_attn_backward(const ref_attn_problem* p, const void* value, const float* ref_points,
+                      const void* offset_logits, const void* grad_out, double* grad_value,
+                      double* grad_offset_logits, int nthreads);
+
 #ifdef __cplusplus
 }
 #endif

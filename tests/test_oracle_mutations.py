@@ -31,6 +31,14 @@ MUTATIONS = {
                        "const int base_w = wo - p->pw + c.iw * p->dw;"),
     "location_two_roundings": ("*h = static_cast<double>(std::fmaf(s, static_cast<float>(dy), static_cast<float>(base_h)));",
                                "*h = static_cast<double>(static_cast<float>(s * static_cast<float>(dy)) + static_cast<float>(base_h));"),
+    # single-scale deformable attention
+    "attn_softmax_not_normalised": ("for (int k = 0; k < p->K; ++k) a[k] /= sum;", ""),
+    "attn_dx_dy_swapped": ("*h = static_cast<double>(ry) + p->offset_scale * dy;\n        *w = static_cast<double>(rx) + p->offset_scale * dx;",
+                           "*h = static_cast<double>(ry) + p->offset_scale * dx;\n        *w = static_cast<double>(rx) + p->offset_scale * dy;"),
+    "attn_jacobian_without_sum": ("= a[k] * (gw[k] - dot);", "= a[k] * gw[k];"),
+    "attn_offset_grad_without_weight": ("= s * a[k] * gdw;", "= s * gdw;"),
+    "attn_corner_row_swapped": ("v[a2][b2] = attn_pixel(p, value, n, h0 + a2, w0 + b2, g, c);",
+                                "v[a2][b2] = attn_pixel(p, value, n, h0 + 1 - a2, w0 + b2, g, c);"),
     "bilinear_ceil_cell": ("const double fh = std::floor(h);", "const double fh = std::ceil(h) - 1.0;"),
     # softmax variant
     "softmax_not_normalised": ("for (int k = 0; k < K; ++k) a[k] /= sum;", ""),

@@ -770,3 +770,129 @@ def test_worked_example_2x2():
     assert np.array_equal(y, ex["y"])
     assert np.array_equal(gom, ex["grad_offset_mask"])
     assert np.array_equal(gv, ex["grad_value"])
+
+
+# ---------------------------------------------------------------------------
+# Deformable attention, single scale (CSDN summary section 1.1: each query
+# attends to a selected number of sampling points whose positions and weights
+# are dynamic; the weights normalised with a softmax over the points as in the
+# section 1.2 DCNv3 equation)
+# ---------------------------------------------------------------------------
+
+def _attn_problem(w, **kw):
+    return oracle.AttnProblem(dtype=w.dtype, **{**w.geometry(), **kw})
+
+
+def _dyadic(x, bits=10):
+    return np.round(np.asarray(x) * 2.0 ** bits) / 2.0 ** bits
+
+
+def test_attn_on_the_grid_is_the_dcnv3_aggregation():
+    """Queries at the pixel centres of a 3x3, stride-1, pad-1 grid whose offsets are the
+    grid cells p_k plus DCN offsets reproduce the DCNv3 form of the aggregation (softmax
+    over the K = 9 points) bit for bit, forward and backward: the same sampling
+    locations, weights and sums.  (The DCN oracle is pinned independently above.)"""
+    N, H, W, G, Cg, K = 2, 6, 7, 2, 3, 9
+    rng = np.random.default_rng(31)
+    value = rng.standard_normal((N, H, W, G * Cg)).astype(np.float32)
+    dxy = _dyadic(rng.normal(0.0, 1.5, (N, H, W, G, K, 2))).astype(np.float32)
+    logits = _dyadic(rng.normal(0.0, 1.0, (N, H, W, G, K))).astype(np.float32)
+    gy = rng.standard_normal((N, H, W, G * Cg)).astype(np.float32)
+    P = -(-G * 3 * K // 8) * 8
+    om = gen.assemble_offset_mask(dxy, logits, P, "f32", tail_fill=0.0)
+    dcn = oracle.Problem(N=N, H=H, W=W, G=G, Cg=Cg, dtype="f32", softmax=True, P=P)
+    y_dcn = oracle.forward(dcn, value, om)
+    gv_dcn, gom_dcn = oracle.backward(dcn, value, om, gy)
+    # the same samples as queries: reference = output pixel centre (x, y), offset = p_k + dp
+    grid = np.array([(iw - 1, ih - 1) for (ih, iw) in cells(3, 3, False)], dtype=np.float32)  # (x, y) per k
+    off_attn = (dxy + grid[None, None, None, None, :, :]).astype(np.float32)
+    assert np.array_equal(off_attn.astype(np.float64), dxy.astype(np.float64) + grid)  # exact in fp32
+    ys, xs = np.divmod(np.arange(H * W), W)
+    ref = np.broadcast_to(np.stack([xs, ys], -1).astype(np.float32), (N, H * W, 2)).copy()
+    ol = gen.assemble_offset_mask(off_attn.reshape(N, H * W, G, K, 2), logits.reshape(N, H * W, G, K), P, "f32",
+                                  tail_fill=0.0)
+    attn = oracle.AttnProblem(N=N, H=H, W=W, G=G, Cg=Cg, Nq=H * W, K=K, P=P, dtype="f32")
+    y = oracle.attn_forward(attn, value, ref, ol)
+    gv, gol = oracle.attn_backward(attn, value, ref, ol, gy.reshape(N, H * W, G * Cg))
+    np.testing.assert_array_equal(y.reshape(y_dcn.shape), y_dcn)
+    np.testing.assert_array_equal(gv, gv_dcn)
+    np.testing.assert_array_equal(gol.reshape(gom_dcn.shape), gom_dcn)
+
+
+def test_attn_single_point_is_grid_sample():
+    """K = 1: the weight is 1 and the output is the bilinear sample of the zero-padded map
+    at reference + offset, which torch's grid_sample computes (align_corners=True)."""
+    w = gen.attn_custom(N=2, H=9, W=11, G=3, Cg=4, Nq=40, K=1, P=16, dtype="f64", ref=("uniform", 2.0),
+                        offset=("normal", 0.0, 3.0))
+    inp = gen.make_attn_inputs(w, tail_fill=0.0)
+    y = oracle.attn_forward(_attn_problem(w), inp["value"], inp["ref_points"], inp["offset_logits"])
+    off = inp["offset_logits"][..., :9].reshape(2, 40, 3, 3)[..., :2]            # (dx, dy) per group
+    loc = inp["ref_points"][:, :, None, :].astype(np.float64) + off               # (x, y)
+    for g in range(3):
+        img = torch.from_numpy(inp["value"][..., g * 4:(g + 1) * 4]).permute(0, 3, 1, 2)
+        gx = 2.0 * loc[..., g, 0] / (w.W - 1) - 1.0
+        gyy = 2.0 * loc[..., g, 1] / (w.H - 1) - 1.0
+        grid = torch.from_numpy(np.stack([gx, gyy], -1)[:, :, None, :])
+        ref = F.grid_sample(img, grid, mode="bilinear", padding_mode="zeros", align_corners=True)
+        np.testing.assert_allclose(y[..., g * 4:(g + 1) * 4], ref[..., 0].permute(0, 2, 1).numpy(), rtol=0,
+                                   atol=1e-12)
+
+
+def test_attn_weights_are_a_softmax():
+    """Equal logits average the K samples; one logit far above the rest selects its
+    point; adding a constant to a query's logits changes nothing."""
+    w = gen.attn_custom(N=1, H=8, W=8, G=2, Cg=3, Nq=12, K=4, P=24, dtype="f64", ref=("uniform", 1.0))
+    inp = gen.make_attn_inputs(w, tail_fill=0.0)
+    prob = _attn_problem(w)
+    ol = inp["offset_logits"].copy()
+    body = ol[..., :24].reshape(1, 12, 2, 12)
+    body[..., 8:] = 0.3
+    y_eq = oracle.attn_forward(prob, inp["value"], inp["ref_points"], ol)
+    singles = []
+    for k in range(4):
+        one = ol.copy()
+        b1 = one[..., :24].reshape(1, 12, 2, 12)
+        b1[..., 8:] = -800.0
+        b1[..., 8 + k] = 0.0
+        singles.append(oracle.attn_forward(prob, inp["value"], inp["ref_points"], one))
+    np.testing.assert_allclose(y_eq, sum(singles) / 4.0, rtol=1e-13, atol=1e-14)
+    shifted = inp["offset_logits"].copy()
+    shifted[..., :24].reshape(1, 12, 2, 12)[..., 8:] += 17.5
+    np.testing.assert_allclose(oracle.attn_forward(prob, inp["value"], inp["ref_points"], shifted),
+                               oracle.attn_forward(prob, inp["value"], inp["ref_points"], inp["offset_logits"]),
+                               rtol=1e-12, atol=1e-14)
+
+
+def test_attn_gradients():
+    """grad_value by the adjoint identity <gy, y(v)> = <grad_value, v> (y is linear in
+    value); offset and logit gradients by central differences; logit gradients of a
+    (query, group) sum to 0; the padding tail is 0."""
+    w = gen.attn_custom(N=2, H=6, W=7, G=2, Cg=3, Nq=10, K=3, P=24, dtype="f64", ref=("uniform", 0.5),
+                        offset=("uniform", -1.7, 1.7))
+    inp = gen.make_attn_inputs(w, tail_fill=0.0)
+    prob = _attn_problem(w)
+    v, ref, ol, gy = inp["value"], inp["ref_points"], inp["offset_logits"], inp["grad_out"]
+    y = oracle.attn_forward(prob, v, ref, ol)
+    gv, gol = oracle.attn_backward(prob, v, ref, ol, gy)
+    assert np.isclose(np.sum(gy * y), np.sum(gv * v), rtol=1e-12)
+    assert np.all(gol[..., 18:] == 0.0)
+    np.testing.assert_allclose(gol[..., :18].reshape(2, 10, 2, 9)[..., 6:].sum(-1), 0.0, atol=1e-12)
+    eps = 1e-6
+    rng = np.random.default_rng(5)
+    for _ in range(40):
+        n, q, e = rng.integers(2), rng.integers(10), rng.integers(18)
+        a, b = ol.copy(), ol.copy()
+        a[n, q, e] += eps
+        b[n, q, e] -= eps
+        fd = (np.sum(gy * oracle.attn_forward(prob, v, ref, a)) - np.sum(gy * oracle.attn_forward(prob, v, ref, b))) / (2 * eps)
+        assert abs(fd - gol[n, q, e]) <= 1e-6 * max(1.0, abs(fd)), (n, q, e, fd, gol[n, q, e])
+
+
+def test_attn_far_offsets_touch_nothing():
+    w = gen.attn_custom(N=1, H=5, W=6, G=2, Cg=4, Nq=8, K=3, P=24, dtype="f64", ref=("uniform", 0.0),
+                        offset=("uniform", 50.0, 60.0))
+    inp = gen.make_attn_inputs(w, tail_fill=0.0)
+    prob = _attn_problem(w)
+    assert np.all(oracle.attn_forward(prob, inp["value"], inp["ref_points"], inp["offset_logits"]) == 0.0)
+    gv, gol = oracle.attn_backward(prob, inp["value"], inp["ref_points"], inp["offset_logits"], inp["grad_out"])
+    assert np.all(gv == 0.0) and np.all(gol == 0.0)
