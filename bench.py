@@ -551,6 +551,7 @@ def run_native(args, w: gen.Workload) -> dict:
         result["per_config_note"] = (f"{args.config_reps} calls of each stage per workload, CUDA events on the "
                                      f"launching stream, L2 flushed before every call; fractions of the measured "
                                      f"copy bandwidth ({measured_peaks()['hbm_gbs']} GB/s) and of 8 TB/s")
+        result["attention"] = attention_leg(dev, world, args.config_reps, flush, stream)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = time_oracle(w, args.cpu_seconds)
     if world > 1:
@@ -625,6 +626,77 @@ def per_config_leg(dev, world: int, reps: int, flush, stream) -> dict:
         del v, om, gy, y, gv, gom, ws
     torch.cuda.empty_cache()
     return out
+
+
+def attn_byte_model(w) -> dict:
+    """Compulsory bytes of single-scale deformable attention.  forward: value,
+    reference points and offset_logits read, out written; backward: value,
+    reference points, offset_logits and grad_out read, grad_value and
+    grad_offset_logits written."""
+    b = ELEM_BYTES[w.dtype]
+    value = w.N * w.H * w.W * w.C * b
+    ref = w.N * w.Nq * 8
+    ol = w.N * w.Nq * w.P * b
+    out = w.N * w.Nq * w.C * b
+    return {"fwd": value + ref + ol + out, "bwd": value + ref + ol + out + value + ol}
+
+
+def attention_leg(dev, world: int, reps: int, flush, stream) -> dict:
+    """Single-scale deformable attention on its workloads: forward and backward
+    µs per call (CUDA events, L2 flushed before every call), achieved GB/s against
+    the byte model, fractions of the measured copy bandwidth and of 8 TB/s."""
+    import numpy as np
+    import torch
+    import deformable_convolution_sampling_b200 as dcn
+    peaks = measured_peaks()
+    sh = stream.cuda_stream
+    res = {}
+    for name in gen.ATTN_WORKLOAD_ORDER:
+        w = gen.ATTN_WORKLOADS[name]
+        tdt = {"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16}[w.dtype]
+        inp = gen.make_attn_inputs(w, tail_fill=0.0)
+
+        def dev_t(a, keep=False):
+            a = np.ascontiguousarray(a)
+            t = torch.from_numpy(a.view(np.int16)).view(tdt) if (w.dtype == "bf16" and not keep) else torch.from_numpy(a)
+            return t.to(dev)
+        v, ol, gy = dev_t(inp["value"]), dev_t(inp["offset_logits"]), dev_t(inp["grad_out"])
+        ref = dev_t(inp["ref_points"], keep=True)
+        p = dcn.make_attn_params(dtype=w.dtype, **w.geometry())
+        y = torch.empty((w.N, w.Nq, w.C), dtype=tdt, device=dev)
+        gv, gol = torch.empty_like(v), torch.empty_like(ol)
+        nb = dcn.dcn4_attn_backward_workspace_size(p)
+        ws = torch.empty(max(nb, 16), dtype=torch.uint8, device=dev)
+        calls = {
+            "fwd": lambda: dcn.check(dcn.dcn4_attn_forward(p, v.data_ptr(), ref.data_ptr(), ol.data_ptr(),
+                                                           y.data_ptr(), sh)),
+            "bwd": lambda: dcn.check(dcn.dcn4_attn_backward(p, v.data_ptr(), ref.data_ptr(), ol.data_ptr(),
+                                                            gy.data_ptr(), gv.data_ptr(), gol.data_ptr(),
+                                                            ws.data_ptr(), nb, sh)),
+        }
+        bm = attn_byte_model(w)
+        rec = {"workload": f"{w.name}: {w.describe()}"}
+        for leg, fn in calls.items():
+            for _ in range(5):
+                fn()
+            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+            for e0, e1 in ev:
+                flush.zero_()
+                e0.record(stream)
+                fn()
+                e1.record(stream)
+            torch.cuda.synchronize(dev)
+            us = max_over_ranks(statistics.mean(a.elapsed_time(c) for a, c in ev) * 1e3, dev)
+            gbs = bm[leg] / (us * 1e-6) / 1e9
+            rec[f"{leg}_us"] = round(us, 2)
+            rec[f"{leg}_bytes"] = bm[leg]
+            rec[f"{leg}_gbs"] = round(gbs, 1)
+            rec[f"{leg}_frac_hbm"] = round(gbs / peaks["hbm_gbs"], 4)
+            rec[f"{leg}_frac_8tbs"] = round(gbs / 8000.0, 4)
+        res[name] = rec
+        del v, ol, gy, ref, y, gv, gol, ws
+    torch.cuda.empty_cache()
+    return res
 
 
 def linear_leg(w: gen.Workload, v, p, flush, stream, dev, world: int) -> dict:

@@ -50,6 +50,28 @@ class dcn4_params(ctypes.Structure):
     ]
 
 
+class dcn4_attn_params(ctypes.Structure):
+    """Mirror of dcn4_attn_params in include/dcn4.h (field order matters)."""
+
+    _fields_ = [
+        ("N", ctypes.c_int), ("H", ctypes.c_int), ("W", ctypes.c_int),
+        ("G", ctypes.c_int), ("Cg", ctypes.c_int),
+        ("Nq", ctypes.c_int), ("K", ctypes.c_int),
+        ("offset_scale", ctypes.c_float),
+        ("P", ctypes.c_int),
+        ("dtype", ctypes.c_int),
+    ]
+
+
+def make_attn_params(*, N, H, W, G, Cg, Nq, K, offset_scale=1.0, P=None, dtype="f16") -> dcn4_attn_params:
+    """dcn4_attn_params for a single-scale deformable attention call; P defaults to G*3K rounded up to 8."""
+    if isinstance(dtype, str):
+        dtype = DTYPE_NAMES[dtype]
+    if P is None:
+        P = -(-G * 3 * K // 8) * 8
+    return dcn4_attn_params(N, H, W, G, Cg, Nq, K, float(offset_scale), P, dtype)
+
+
 def make_params(*, N, H, W, G, Cg, kh=3, kw=3, sh=1, sw=1, ph=1, pw=1, dh=1, dw=1,
                 offset_scale=1.0, remove_center=0, P=None, dtype="f32", softmax=0) -> dcn4_params:
     """Build a dcn4_params; P defaults to the smallest valid padded row.  softmax=1
@@ -69,6 +91,7 @@ def _load() -> ctypes.CDLL:
             "(there is no CPU fallback)")
     L = ctypes.CDLL(LIB_PATH)
     P = ctypes.POINTER(dcn4_params)
+    AP = ctypes.POINTER(dcn4_attn_params)
     vp, ip = ctypes.c_void_p, ctypes.POINTER(ctypes.c_int)
     sig = {
         "dcn4_version": ([], ctypes.c_int),
@@ -88,6 +111,10 @@ def _load() -> ctypes.CDLL:
         "dcn4_backward_noalloc_capacity": ([], ctypes.c_size_t),
         "dcn4_noalloc_last_error": ([], ctypes.c_char_p),
         "dcn4_backward_diagnostics": ([P, vp, ctypes.c_size_t, ip, vp], ctypes.c_int),
+        "dcn4_attn_check_params": ([AP], ctypes.c_int),
+        "dcn4_attn_forward": ([AP, vp, vp, vp, vp, vp], ctypes.c_int),
+        "dcn4_attn_backward_workspace_size": ([AP], ctypes.c_size_t),
+        "dcn4_attn_backward": ([AP, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         fn = getattr(L, name)
@@ -163,6 +190,24 @@ def dcn4_backward_diagnostics(p: dcn4_params, workspace, workspace_bytes: int, s
     counts = (ctypes.c_int * 3)()
     st = lib.dcn4_backward_diagnostics(ctypes.byref(p), workspace, workspace_bytes, counts, stream)
     return st, list(counts)
+
+
+def dcn4_attn_check_params(p: dcn4_attn_params) -> int:
+    return lib.dcn4_attn_check_params(ctypes.byref(p))
+
+
+def dcn4_attn_forward(p: dcn4_attn_params, value, ref_points, offset_logits, out, stream=None) -> int:
+    return lib.dcn4_attn_forward(ctypes.byref(p), value, ref_points, offset_logits, out, stream)
+
+
+def dcn4_attn_backward_workspace_size(p: dcn4_attn_params) -> int:
+    return lib.dcn4_attn_backward_workspace_size(ctypes.byref(p))
+
+
+def dcn4_attn_backward(p: dcn4_attn_params, value, ref_points, offset_logits, grad_out, grad_value,
+                       grad_offset_logits, workspace, workspace_bytes: int, stream=None) -> int:
+    return lib.dcn4_attn_backward(ctypes.byref(p), value, ref_points, offset_logits, grad_out, grad_value,
+                                  grad_offset_logits, workspace, workspace_bytes, stream)
 
 
 def dcn4_backward_noalloc(p: dcn4_params, value, offset_mask, grad_out, grad_value, grad_offset_mask,
@@ -259,6 +304,31 @@ def backward(p: dcn4_params, value, offset_mask, grad_out, grad_value=None, grad
                         grad_value.data_ptr(), grad_offset_mask.data_ptr(), ws_ptr, ws_bytes,
                         _stream_handle(value.device)))
     return grad_value, grad_offset_mask
+
+
+def attn_forward(p: dcn4_attn_params, value, ref_points, offset_logits, out=None):
+    """y[N,Nq,C] of single-scale deformable attention for CUDA tensors value [N,H,W,C],
+    ref_points [N,Nq,2] (float32) and offset_logits [N,Nq,P]."""
+    import torch
+    if out is None:
+        out = torch.empty((p.N, p.Nq, p.G * p.Cg), dtype=_torch_dtype(p.dtype), device=value.device)
+    check(dcn4_attn_forward(p, value.data_ptr(), ref_points.data_ptr(), offset_logits.data_ptr(), out.data_ptr(),
+                            _stream_handle(value.device)))
+    return out
+
+
+def attn_backward(p: dcn4_attn_params, value, ref_points, offset_logits, grad_out):
+    """(grad_value[N,H,W,C], grad_offset_logits[N,Nq,P]) for CUDA tensors."""
+    import torch
+    dt = _torch_dtype(p.dtype)
+    gv = torch.empty((p.N, p.H, p.W, p.G * p.Cg), dtype=dt, device=value.device)
+    gol = torch.empty((p.N, p.Nq, p.P), dtype=dt, device=value.device)
+    need = dcn4_attn_backward_workspace_size(p)
+    ws = torch.empty(max(need, 16), dtype=torch.uint8, device=value.device)
+    check(dcn4_attn_backward(p, value.data_ptr(), ref_points.data_ptr(), offset_logits.data_ptr(),
+                             grad_out.data_ptr(), gv.data_ptr(), gol.data_ptr(), ws.data_ptr(), need,
+                             _stream_handle(value.device)))
+    return gv, gol
 
 
 def backward_diagnostics(p: dcn4_params, workspace) -> dict:

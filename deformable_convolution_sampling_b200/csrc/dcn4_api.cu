@@ -254,6 +254,48 @@ dcn4::SampleArrays sample_arrays(const dcn4::Geometry& g, int dtype, const void*
     return sa;
 }
 
+// Validates a deformable attention call and fills the kernel geometry (value
+// map, points per query, row length, slices).  Touches no GPU state.
+int make_attn_geometry(const dcn4_attn_params* p, bool wide, dcn4::Geometry* g) {
+    if (!p) return fail(DCN4_ERR_NULL, "params is NULL");
+    if (p->dtype != DCN4_F32 && p->dtype != DCN4_F16 && p->dtype != DCN4_BF16)
+        return fail(DCN4_ERR_DTYPE, "dtype %d is not a dcn4_dtype", p->dtype);
+    if (p->N < 0 || p->H < 1 || p->W < 1 || p->G < 1 || p->Cg < 1 || p->Nq < 0 || p->K < 1)
+        return fail(DCN4_ERR_BAD_SHAPE, "need N, Nq >= 0 and H, W, G, Cg, K >= 1");
+    if (!std::isfinite(p->offset_scale)) return fail(DCN4_ERR_BAD_SHAPE, "offset_scale is not finite");
+    if (p->K > 1024) return fail(DCN4_ERR_UNSUPPORTED, "K > 1024");
+    const long long body = 3LL * p->G * p->K;
+    if (body > (1LL << 30) || p->P < body || p->P % 8 != 0)
+        return fail(DCN4_ERR_BAD_P, "P=%d must be a multiple of 8 and >= G*3K=%lld", p->P, body);
+    if (p->H >= (1 << 24) || p->W >= (1 << 24)) return fail(DCN4_ERR_UNSUPPORTED, "H, W must be < 2^24");
+    const long long C = static_cast<long long>(p->G) * p->Cg;
+    if (static_cast<long long>(p->H) * p->W * C >= (1LL << 31))
+        return fail(DCN4_ERR_UNSUPPORTED, "H*W*C must be < 2^31 per image");
+    const int eb = elem_bytes(p->dtype);
+    const long long slice_bytes = static_cast<long long>(p->Cg) * eb;
+    if (slice_bytes % 16 != 0)
+        return fail(DCN4_ERR_UNSUPPORTED, "Cg*sizeof(dtype)=%lld must be a multiple of 16 bytes", slice_bytes);
+    const long long vec = (wide && slice_bytes % 32 == 0) ? 2 : 1;
+    const long long nslice = slice_bytes / (16 * vec);
+    if (nslice > 32 || (nslice & (nslice - 1)) != 0)
+        return fail(DCN4_ERR_UNSUPPORTED, "Cg*sizeof(dtype)/32 must be a power of two <= 32 (Cg=%d)", p->Cg);
+    if (p->G * nslice > kTargetThreads)
+        return fail(DCN4_ERR_UNSUPPORTED, "G * slices per group = %lld exceeds %d threads", p->G * nslice, kTargetThreads);
+    const long long queries = static_cast<long long>(p->N) * p->Nq;
+    if (queries > (1LL << 40)) return fail(DCN4_ERR_UNSUPPORTED, "N*Nq too large");
+    *g = dcn4::Geometry{};
+    g->N = p->N; g->H = p->H; g->W = p->W; g->G = p->G; g->Cg = p->Cg; g->C = static_cast<int>(C);
+    g->K = p->K; g->P = p->P; g->s = p->offset_scale; g->softmax = 1;
+    g->vec = static_cast<int>(vec);
+    g->nslice = static_cast<int>(nslice);
+    g->Ho = 1; g->Wo = 1;
+    if (dcn4::attn_smem_bytes(*g, eb, true) > kSmemMax)
+        return fail(DCN4_ERR_UNSUPPORTED, "K=%d points and P=%d rows do not fit shared memory", p->K, p->P);
+    const long long qb = std::max(1LL, static_cast<long long>(kTargetThreads) / (p->G * nslice));
+    if ((queries + qb - 1) / qb > 0x7fffffffLL) return fail(DCN4_ERR_UNSUPPORTED, "grid too large");
+    return DCN4_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -400,6 +442,74 @@ int dcn4_backward(const dcn4_params* p, const void* value, const void* offset_ma
                                             workspace_bytes, stream);
     if (a != DCN4_OK) return a;
     return dcn4_backward_value(p, offset_mask, grad_out, grad_value, workspace, workspace_bytes, stream);
+}
+
+int dcn4_attn_check_params(const dcn4_attn_params* p) {
+    dcn4::Geometry g;
+    for (int wide = 0; wide < 2; ++wide) {
+        const int st = make_attn_geometry(p, wide, &g);
+        if (st != DCN4_OK) return st;
+    }
+    return DCN4_OK;
+}
+
+int dcn4_attn_forward(const dcn4_attn_params* p, const void* value, const float* ref_points, const void* offset_logits,
+                      void* out, void* stream) {
+    dcn4::Geometry g;
+    const int st = make_attn_geometry(p, aligned32(value) && aligned32(out), &g);
+    if (st != DCN4_OK) return st;
+    if (static_cast<long long>(p->N) * p->Nq == 0) return DCN4_OK;
+    if (!value || !ref_points || !offset_logits || !out)
+        return fail(DCN4_ERR_NULL, "value, ref_points, offset_logits and out must be non-NULL");
+    if (!aligned16(value) || !aligned16(ref_points) || !aligned16(offset_logits) || !aligned16(out))
+        return fail(DCN4_ERR_MISALIGNED, "every pointer must be 16-byte aligned");
+    const cudaError_t e = dcn4::launch_attn_forward(g, p->dtype, p->Nq, value, ref_points, offset_logits, out,
+                                                    static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return fail(DCN4_ERR_LAUNCH, "attention forward launch: %s", cudaGetErrorString(e));
+    return DCN4_OK;
+}
+
+size_t dcn4_attn_backward_workspace_size(const dcn4_attn_params* p) {
+    dcn4::Geometry g;
+    if (make_attn_geometry(p, true, &g) != DCN4_OK) return 0;
+    if (p->dtype == DCN4_F32) return 0;
+    return round256(static_cast<size_t>(p->N) * p->H * p->W * g.C * sizeof(float));
+}
+
+int dcn4_attn_backward(const dcn4_attn_params* p, const void* value, const float* ref_points, const void* offset_logits,
+                       const void* grad_out, void* grad_value, void* grad_offset_logits, void* workspace,
+                       size_t workspace_bytes, void* stream) {
+    dcn4::Geometry g;
+    const int st = make_attn_geometry(p, aligned32(value) && aligned32(grad_out), &g);
+    if (st != DCN4_OK) return st;
+    if (!grad_value && p->N > 0) return fail(DCN4_ERR_NULL, "grad_value must be non-NULL");
+    if (p->N == 0) return DCN4_OK;
+    if (!aligned16(grad_value)) return fail(DCN4_ERR_MISALIGNED, "every pointer must be 16-byte aligned");
+    const size_t need = dcn4_attn_backward_workspace_size(p);
+    if (need && (!workspace || workspace_bytes < need))
+        return fail(DCN4_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, workspace_bytes);
+    if (need && !aligned16(workspace)) return fail(DCN4_ERR_MISALIGNED, "workspace must be 16-byte aligned");
+    const bool any_query = p->Nq > 0;
+    if (any_query && (!value || !ref_points || !offset_logits || !grad_out || !grad_offset_logits))
+        return fail(DCN4_ERR_NULL, "value, ref_points, offset_logits, grad_out and grad_offset_logits must be non-NULL");
+    if (any_query && (!aligned16(value) || !aligned16(ref_points) || !aligned16(offset_logits) ||
+                      !aligned16(grad_out) || !aligned16(grad_offset_logits)))
+        return fail(DCN4_ERR_MISALIGNED, "every pointer must be 16-byte aligned");
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t elems = static_cast<size_t>(p->N) * p->H * p->W * g.C;
+    float* acc = p->dtype == DCN4_F32 ? static_cast<float*>(grad_value) : static_cast<float*>(workspace);
+    cudaError_t e = cudaMemsetAsync(acc, 0, elems * sizeof(float), s);
+    if (e != cudaSuccess) return fail(DCN4_ERR_LAUNCH, "accumulator reset: %s", cudaGetErrorString(e));
+    if (!any_query) {
+        // no query samples anything: grad_value is zero (rounded from the cleared accumulator)
+        if (p->dtype != DCN4_F32) e = cudaMemsetAsync(grad_value, 0, elems * elem_bytes(p->dtype), s);
+        if (e != cudaSuccess) return fail(DCN4_ERR_LAUNCH, "grad_value reset: %s", cudaGetErrorString(e));
+        return DCN4_OK;
+    }
+    e = dcn4::launch_attn_backward(g, p->dtype, p->Nq, value, ref_points, offset_logits, grad_out, grad_value,
+                                   grad_offset_logits, acc, s);
+    if (e != cudaSuccess) return fail(DCN4_ERR_LAUNCH, "attention backward launch: %s", cudaGetErrorString(e));
+    return DCN4_OK;
 }
 
 int dcn4_backward_diagnostics(const dcn4_params* p, const void* workspace, size_t workspace_bytes, int* counts,

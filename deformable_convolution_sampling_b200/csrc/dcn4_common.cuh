@@ -370,5 +370,16 @@ size_t forward_linear_smem_bytes(const Geometry& g, int Cx, bool w_smem);
 // Whether the fused forward stages W in shared memory for this shape.
 bool forward_linear_w_smem(const Geometry& g, int Cx);
 size_t backward_smem_bytes(const Geometry& g, int elem_bytes);
+// Single-scale deformable attention (dcn4_attn.cu): g holds the value map (N, H,
+// W, G, Cg, C), the points per query (K), the row length (P), offset_scale (s)
+// and the slice split (vec, nslice); Nq queries per image.  The backward
+// accumulates grad_value in fp32 at `acc` (grad_value itself for fp32 I/O,
+// zeroed by the caller) and rounds it into gvalue for 16-bit I/O.
+size_t attn_smem_bytes(const Geometry& g, int elem_bytes, bool backward);
+cudaError_t launch_attn_forward(const Geometry& g, int dtype, int Nq, const void* value, const float* ref,
+                                const void* ol, void* out, cudaStream_t stream);
+cudaError_t launch_attn_backward(const Geometry& g, int dtype, int Nq, const void* value, const float* ref,
+                                 const void* ol, const void* gout, void* gvalue, void* gol, float* acc,
+                                 cudaStream_t stream);
 size_t backward_value_smem_bytes(const Geometry& g);
 }  // namespace dcn4

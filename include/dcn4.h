@@ -67,7 +67,7 @@
 extern "C" {
 #endif
 
-#define DCN4_VERSION 130  /* 1.3.0: dcn4_backward_diagnostics */
+#define DCN4_VERSION 140  /* 1.4.0: deformable attention (dcn4_attn_*) */
 
 typedef enum {
     DCN4_F32 = 0,   /* IEEE binary32            */
@@ -247,6 +247,71 @@ int dcn4_backward_value(const dcn4_params* p, const void* offset_mask, const voi
  * Same checks as dcn4_backward; counts must hold 3 ints. */
 int dcn4_backward_diagnostics(const dcn4_params* p, const void* workspace, size_t workspace_bytes, int* counts,
                               void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Deformable attention, single scale.
+ *
+ * The pages describe deformable attention as letting each query attend to a
+ * selected number of key sampling points whose positions and weights are
+ * determined dynamically (CSDN summary of "Efficient Deformable ConvNets",
+ * section 1.1), and note that the aggregation's memory optimisations apply to
+ * it (section 2.2, "消除冗余内存指令").  This is that operation on one feature
+ * map, with the weights normalised by a softmax over the points as in the
+ * DCNv3 equation of section 1.2:
+ *
+ *     y_g(q) = sum_{k<K} A_gk * x_g(r_q + offset_scale * dp_gk),
+ *     A_gk   = exp(l_gk - max_j l_gj) / sum_j exp(l_gj - max_j l_gj)
+ *
+ * for every query q (reference point r_q) and group g (a head).  x_g(.) is the
+ * bilinear sample of the zero-extended map exactly as in dcn4_forward, the
+ * location formed in fp32 as fmaf(offset_scale, d, r), the exponentials in fp32
+ * (expf), sums in fp32, one rounding of each result to dtype.
+ *
+ * Layouts (dense, contiguous; C = G*Cg):
+ *   value              [N, H, W, C]    dtype
+ *   ref_points         [N, Nq, 2]      fp32 (x, y) in pixel coordinates of value;
+ *                                      integer coordinates are pixel centres
+ *   offset_logits      [N, Nq, P]      dtype.  Group g owns [g*3K, (g+1)*3K):
+ *                                      K pairs (dx, dy), then K logits l_k.
+ *                                      Entries [G*3K, P) are padding: never read.
+ *   out / grad_out     [N, Nq, C]      dtype
+ *   grad_value         [N, H, W, C]    dtype
+ *   grad_offset_logits [N, Nq, P]      dtype; the padding tail is written as 0.
+ * The reference points receive no gradient.  Preconditions as for dcn4_forward
+ * (16-byte aligned pointers, Cg*sizeof(dtype) a multiple of 16 and /32 a power
+ * of two, P >= G*3K a multiple of 8), plus K <= 1024 points whose rows fit
+ * shared memory; N*Nq == 0 is a successful no-op.
+ * ------------------------------------------------------------------------- */
+typedef struct {
+    int N, H, W;          /* value is [N, H, W, G*Cg]                          */
+    int G, Cg;            /* groups (heads), channels per group                */
+    int Nq, K;            /* queries per image, sampling points per query      */
+    float offset_scale;   /* multiplies the offsets                             */
+    int P;                /* row length of offset_logits / grad_offset_logits  */
+    int dtype;            /* dcn4_dtype of every tensor argument but ref_points */
+} dcn4_attn_params;
+
+/* Host-only validation of p; returns DCN4_OK or the status a call would return. */
+int dcn4_attn_check_params(const dcn4_attn_params* p);
+
+/* Forward: out = y.  One kernel launch on `stream`. */
+int dcn4_attn_forward(const dcn4_attn_params* p, const void* value, const float* ref_points,
+                      const void* offset_logits, void* out, void* stream);
+
+/* Bytes of workspace dcn4_attn_backward needs: 0 for fp32, else an fp32
+ * accumulator for grad_value (N*H*W*C*4, rounded up to 256); 0 if p is invalid. */
+size_t dcn4_attn_backward_workspace_size(const dcn4_attn_params* p);
+
+/* Backward for grad_out: grad_value (overwritten) and grad_offset_logits
+ * (overwritten): d/d dx_k = offset_scale * A_k * <gy, dS/dw>, likewise dy, and
+ * d/d l_k = A_k (<gy, S_k> - sum_j A_j <gy, S_j>).  grad_value is scattered
+ * with fp32 vector reductions (red.global.add.v4.f32) into the workspace (into
+ * grad_value itself for fp32), so the order of its sums, and its last bits,
+ * may differ between calls.  Launches, on `stream`: a memset of the
+ * accumulator, one kernel, and for fp16/bf16 one rounding kernel. */
+int dcn4_attn_backward(const dcn4_attn_params* p, const void* value, const float* ref_points,
+                       const void* offset_logits, const void* grad_out, void* grad_value,
+                       void* grad_offset_logits, void* workspace, size_t workspace_bytes, void* stream);
 
 /* Name of a dcn4_status. */
 const char* dcn4_status_string(int status);

@@ -70,7 +70,53 @@ def test_params_mirror_matches_the_header(dcn):
             fields += [n.strip() for n in names.split(",")]
     assert [f[0] for f in dcn.dcn4_params._fields_] == fields
     assert ctypes.sizeof(dcn.dcn4_params) == 4 * len(fields)
-    assert dcn.dcn4_version() == 130
+    assert dcn.dcn4_version() == 140
+
+
+def test_attn_params_mirror_matches_the_header(dcn):
+    """The binding's ctypes dcn4_attn_params has the header's fields, in order, all 4 bytes."""
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    body = re.search(r"typedef struct \{([^}]*)\} dcn4_attn_params;", text, flags=re.S).group(1)
+    fields = []
+    for decl in body.split(";"):
+        decl = decl.strip()
+        if decl:
+            ctype, names = decl.split(None, 1)
+            assert ctype in ("int", "float"), decl
+            fields += [n.strip() for n in names.split(",")]
+    assert [f[0] for f in dcn.dcn4_attn_params._fields_] == fields
+    assert ctypes.sizeof(dcn.dcn4_attn_params) == 4 * len(fields)
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("dtype", 5, -8), ("N", -1, -2), ("H", 0, -2), ("G", 0, -2), ("Cg", 0, -2), ("Nq", -1, -2), ("K", 0, -2),
+    ("P", 16, -3), ("P", 50, -3), ("Cg", 4, -5), ("Cg", 24, -5), ("K", 2000, -5), ("H", 1 << 24, -5),
+])
+def test_attn_invalid_params_are_rejected_before_launch(dcn, field, value, status):
+    p = dcn.make_attn_params(N=2, H=8, W=8, G=2, Cg=8, Nq=10, K=4, dtype="f16")
+    setattr(p, field, value)
+    assert dcn.dcn4_attn_check_params(p) == status
+    assert dcn.dcn4_attn_forward(p, None, None, None, None, None) == status
+    assert dcn.dcn4_attn_backward(p, None, None, None, None, None, None, None, 0, None) == status
+
+
+def test_attn_workspace_and_null_pointers():
+    """Workspace size (an fp32 grad_value accumulator for 16-bit I/O, none for fp32) and
+    the NULL / misaligned / missing-workspace refusals (made-up addresses: checked in a
+    child process that sees no GPU)."""
+    run_without_gpu("""
+p = dcn.make_attn_params(N=2, H=8, W=8, G=2, Cg=8, Nq=10, K=4, dtype="f16")
+assert dcn.dcn4_attn_check_params(p) == 0
+assert dcn.dcn4_attn_backward_workspace_size(p) == 2 * 8 * 8 * 16 * 4
+assert dcn.dcn4_attn_backward_workspace_size(dcn.make_attn_params(N=2, H=8, W=8, G=2, Cg=8, Nq=10, K=4, dtype="f32")) == 0
+assert dcn.dcn4_attn_forward(p, None, 32, 48, 64, None) == -1
+assert dcn.dcn4_attn_forward(p, 16, 36, 48, 64, None) == -4
+assert dcn.dcn4_attn_backward(p, 16, 32, 48, 64, 80, 96, None, 0, None) == -6
+assert dcn.dcn4_attn_backward(p, 16, 32, 48, 64, 80, 96, 112, 100, None) == -6
+assert dcn.dcn4_attn_backward(p, 16, 32, 48, 64, None, 96, 112, 1 << 20, None) == -1
+empty = dcn.make_attn_params(N=0, H=8, W=8, G=2, Cg=8, Nq=10, K=4, dtype="f16")
+assert dcn.dcn4_attn_forward(empty, None, None, None, None, None) == 0
+""")
 
 
 def test_library_does_not_link_the_oracle(dcn):

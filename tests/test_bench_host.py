@@ -115,3 +115,11 @@ def test_reference_arm_other_ranks_exit_quietly():
                         "tiny_f32", "--steps", "3", "--warmup", "3"], capture_output=True, text=True, timeout=300,
                        env=env)
     assert r.returncode == 0 and r.stdout.strip() == ""
+
+
+def test_attn_byte_model():
+    w = gen.ATTN_WORKLOADS["attn_enc_f16"]
+    bm = bench.attn_byte_model(w)
+    value, ref, ol, out = 8 * 64 * 64 * 256 * 2, 8 * 4096 * 8, 8 * 4096 * 96 * 2, 8 * 4096 * 256 * 2
+    assert bm["fwd"] == value + ref + ol + out
+    assert bm["bwd"] == value + ref + ol + out + value + ol
