@@ -153,6 +153,9 @@ def lib() -> ctypes.CDLL:
         L.ref_encode.restype = None
         L.ref_linear.argtypes = [ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int, vp, vp, vp, vp]
         L.ref_linear.restype = ctypes.c_int
+        L.ref_linear_backward.argtypes = [ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int, vp, vp, vp,
+                                          dp, dp, dp, ctypes.c_int]
+        L.ref_linear_backward.restype = ctypes.c_int
         AP = ctypes.POINTER(_AttnProblem)
         L.ref_attn_forward.argtypes = [AP, vp, vp, vp, dp, ctypes.c_int]
         L.ref_attn_forward.restype = ctypes.c_int
@@ -253,6 +256,32 @@ def linear(dtype: str, x: np.ndarray, weight: np.ndarray, bias: np.ndarray | Non
     if lib().ref_linear(M, Cin, Cout, DTYPES[dtype], _ptr(x), _ptr(weight), b, _ptr(out)) != 0:
         raise ValueError("oracle linear rejected its arguments")
     return out
+
+
+def linear_backward(dtype: str, x: np.ndarray, weight: np.ndarray, grad: np.ndarray, nthreads: int = 1,
+                    want_x: bool = True, want_weight: bool = True):
+    """Gradients of the merged offset/mask linear layer for the upstream gradient
+    `grad` [..., Cout] of its output (x [..., Cin], weight [Cout, Cin], all stored in
+    `dtype`): (grad_x [..., Cin], grad_weight [Cout, Cin], grad_bias [Cout]) in
+    float64, unrounded; grad_x (want_x=False) or grad_weight and grad_bias
+    (want_weight=False) come back as None when not wanted."""
+    want = NUMPY_STORAGE[dtype]
+    x, weight, grad = (np.ascontiguousarray(a) for a in (x, weight, grad))
+    for name, a in (("x", x), ("weight", weight), ("grad", grad)):
+        if a.dtype != want:
+            raise TypeError(f"{name}: storage {dtype} wants {np.dtype(want)}, got {a.dtype}")
+    Cout, Cin = weight.shape
+    if x.shape[-1] != Cin or grad.shape != x.shape[:-1] + (Cout,):
+        raise ValueError("linear_backward: shape mismatch")
+    M = int(np.prod(x.shape[:-1]))
+    gx = np.empty(x.shape, dtype=np.float64)
+    gw = np.empty((Cout, Cin), dtype=np.float64)
+    gb = np.empty((Cout,), dtype=np.float64)
+    if lib().ref_linear_backward(M, Cin, Cout, DTYPES[dtype], _ptr(x), _ptr(weight), _ptr(grad),
+                                 _dptr(gx) if want_x else None, _dptr(gw) if want_weight else None,
+                                 _dptr(gb) if want_weight else None, int(nthreads)) != 0:
+        raise ValueError("oracle linear_backward rejected its arguments")
+    return (gx if want_x else None), (gw if want_weight else None), (gb if want_weight else None)
 
 
 def _attn_check(prob: AttnProblem, value, ref_points, offset_logits):

@@ -295,6 +295,38 @@ int ref_linear(int64_t M, int Cin, int Cout, int dtype, const void* x, const voi
     return 0;
 }
 
+int ref_linear_backward(int64_t M, int Cin, int Cout, int dtype, const void* x, const void* weight, const void* g,
+                        double* grad_x, double* grad_w, double* grad_b, int nthreads) {
+    if (M < 0 || Cin < 1 || Cout < 1 || dtype < REF_F32 || dtype > REF_F64 || (M > 0 && !g)) return -1;
+    if ((grad_x && !weight) || (grad_w && !x)) return -1;
+    if (grad_x)
+        parallel_range(M, nthreads, [&](int64_t m) {
+            for (int c = 0; c < Cin; ++c) {
+                double acc = 0.0;
+                for (int j = 0; j < Cout; ++j)
+                    acc += load(g, dtype, m * Cout + j) * load(weight, dtype, static_cast<int64_t>(j) * Cin + c);
+                grad_x[m * Cin + c] = acc;
+            }
+        });
+    // For each row j of the weight, one pass over the rows m (in order) keeps the
+    // Cin sums of grad_w[j, :] and the sum of grad_b[j] side by side.
+    if (grad_w || grad_b)
+        parallel_range(Cout, nthreads, [&](int64_t j) {
+            std::vector<double> acc(Cin, 0.0);
+            double bsum = 0.0;
+            for (int64_t m = 0; m < M; ++m) {
+                const double gj = load(g, dtype, m * Cout + j);
+                bsum += gj;
+                if (grad_w)
+                    for (int c = 0; c < Cin; ++c) acc[c] += gj * load(x, dtype, m * Cin + c);
+            }
+            if (grad_w)
+                for (int c = 0; c < Cin; ++c) grad_w[j * Cin + c] = acc[c];
+            if (grad_b) grad_b[j] = bsum;
+        });
+    return 0;
+}
+
 void ref_decode(int dtype, const void* src, double* dst, int64_t n) {
     for (int64_t i = 0; i < n; ++i) dst[i] = load(src, dtype, i);
 }

@@ -125,6 +125,18 @@ void ref_encode(int dtype, const double* src, void* dst, int64_t n);
 int ref_linear(int64_t M, int Cin, int Cout, int dtype, const void* x, const void* weight,
                const void* bias, void* out);
 
+/* Gradients of ref_linear's affine map (before its rounding) for an upstream
+ * gradient g [M, Cout] stored in `dtype`:
+ *     grad_x[m, c] = sum_j g[m, j] * weight[j, c]      [M, Cin]
+ *     grad_w[j, c] = sum_m g[m, j] * x[m, c]           [Cout, Cin]
+ *     grad_b[j]    = sum_m g[m, j]                     [Cout]
+ * in double, unrounded (the derivative of a linear map is its transpose; the
+ * bias enters every row with weight 1).  Any of the three outputs may be NULL.
+ * Rows of grad_x and rows of grad_w / grad_b are spread over nthreads threads.
+ * Returns 0, or -1 for bad sizes. */
+int ref_linear_backward(int64_t M, int Cin, int Cout, int dtype, const void* x, const void* weight, const void* g,
+                        double* grad_x, double* grad_w, double* grad_b, int nthreads);
+
 /* ---------------------------------------------------------------------------
  * Deformable attention, single scale (CSDN summary of "Efficient Deformable
  * ConvNets", section 1.1: each query attends to a selected number of key

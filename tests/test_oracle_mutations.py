@@ -51,6 +51,11 @@ MUTATIONS = {
     "linear_drops_bias": ("if (bias) acc += load(bias, dtype, j);", ""),
     "linear_weight_transposed": ("load(weight, dtype, static_cast<int64_t>(j) * Cin + c)",
                                  "load(weight, dtype, static_cast<int64_t>(c % Cout) * Cin + (j % Cin))"),
+    "linear_bwd_weight_transposed": ("load(g, dtype, m * Cout + j) * load(weight, dtype, static_cast<int64_t>(j) * Cin + c)",
+                                     "load(g, dtype, m * Cout + j) * load(weight, dtype, static_cast<int64_t>(c % Cout) * Cin + (j % Cin))"),
+    "linear_bwd_x_row_shifted": ("acc[c] += gj * load(x, dtype, m * Cin + c);",
+                                 "acc[c] += gj * load(x, dtype, ((m + 1) % M) * Cin + c);"),
+    "linear_bwd_bias_skips_first_row": ("bsum += gj;", "if (m > 0) bsum += gj;"),
     "softmax_ignored_in_backward_offsets": ("const double m = a[k];\n                        double h, w;\n                        sample_location(p, ho, wo, cells[k], dx, dy, &h, &w);\n                        const Bilinear b = bilinear_cell(p, h, w);\n                        if (!b.any) continue;",
                                             "const double m = load(offset_mask, p->dtype, om + 2 * K + k);\n                        double h, w;\n                        sample_location(p, ho, wo, cells[k], dx, dy, &h, &w);\n                        const Bilinear b = bilinear_cell(p, h, w);\n                        if (!b.any) continue;"),
 }

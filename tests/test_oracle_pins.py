@@ -755,6 +755,54 @@ def test_linear_shapes_and_rows():
 
 
 
+@pytest.mark.parametrize("dtype", ["f64", "f16", "bf16"])
+def test_linear_backward_is_the_derivative_of_the_forward(dtype):
+    """Every entry of grad_x, grad_weight and grad_bias equals the central difference
+    of L = <g, linear(x, W, b)> in that coordinate, L evaluated with the forward
+    oracle.  The layer is affine, so a unit step gives the derivative exactly; with
+    small integers every forward output (and L) is exact even in 16-bit storage."""
+    rng = np.random.default_rng(11)
+    M, Cin, Cout = 5, 4, 6
+    xs = rng.integers(-2, 3, size=(M, Cin)).astype(np.float64)
+    ws = rng.integers(-2, 3, size=(Cout, Cin)).astype(np.float64)
+    bs = rng.integers(-3, 4, size=Cout).astype(np.float64)
+    gs = rng.integers(-3, 4, size=(M, Cout)).astype(np.float64)
+    st = lambda a: gen.to_storage(a, dtype) if dtype != "f64" else a.copy()
+    dec = lambda a: gen.storage_to_f64(a, dtype) if dtype != "f64" else a
+
+    def loss(x, w, b):
+        return float(np.sum(gs * dec(oracle.linear(dtype, st(x), st(w), st(b)))))
+
+    gx, gw, gb = oracle.linear_backward(dtype, st(xs), st(ws), st(gs))
+    for arr, grad, which in ((xs, gx, 0), (ws, gw, 1), (bs, gb, 2)):
+        for idx in np.ndindex(arr.shape):
+            args = [xs, ws, bs]
+            up, dn = arr.copy(), arr.copy()
+            up[idx] += 1.0
+            dn[idx] -= 1.0
+            args_up, args_dn = list(args), list(args)
+            args_up[which], args_dn[which] = up, dn
+            assert grad[idx] == (loss(*args_up) - loss(*args_dn)) / 2.0, (which, idx)
+
+
+def test_linear_backward_rows_and_shapes():
+    """Leading dimensions are rows; grad_x's row m depends on g's row m only; grad_weight
+    and grad_bias are sums of per-row contributions (so they add over a split of the rows)."""
+    rng = np.random.default_rng(12)
+    x = gen.to_storage(rng.normal(size=(2, 3, 16)), "bf16")
+    w = gen.to_storage(rng.normal(size=(8, 16)), "bf16")
+    g = gen.to_storage(rng.normal(size=(2, 3, 8)), "bf16")
+    gx, gw, gb = oracle.linear_backward("bf16", x, w, g)
+    assert gx.shape == (2, 3, 16) and gw.shape == (8, 16) and gb.shape == (8,)
+    gx1, gw1, gb1 = oracle.linear_backward("bf16", x[1, 2][None], w, g[1, 2][None])
+    assert np.array_equal(gx[1, 2], gx1[0])
+    gxa, gwa, gba = oracle.linear_backward("bf16", x[0], w, g[0])
+    gxb, gwb, gbb = oracle.linear_backward("bf16", x[1], w, g[1])
+    assert np.allclose(gw, gwa + gwb, rtol=1e-14, atol=1e-12) and np.allclose(gb, gba + gbb, rtol=1e-14, atol=1e-12)
+    with pytest.raises(ValueError):
+        oracle.linear_backward("bf16", x, w, g[..., :4])
+
+
 # ---------------------------------------------------------------------------
 # The hand-derived worked example (tests/golden/bilinear_2x2_worked.txt)
 # ---------------------------------------------------------------------------
