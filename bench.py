@@ -2,7 +2,8 @@
 """Benchmark of the DCNv4 core operator on B200: one forward + backward step.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
-                    [--workload NAME] [--softmax] [--linear] [--no-cpu-baseline] [--no-e2e]
+                    [--workload NAME] [--softmax] [--no-linear] [--no-cpu-baseline] [--no-e2e]
+    python bench.py --profile [--workload NAME] [--linear] --steps K --warmup W   (for ncu)
 
 A step is one pass of the whole path over one batch: dcn4_forward followed by
 dcn4_backward on the first-stage backbone workload (N64 H56 W56 C64 G4, C'=16,
@@ -23,10 +24,17 @@ and a CPU-oracle baseline.
 --softmax runs the same step with the masks normalised by a softmax over the
 K points of each (pixel, group) (the DCNv3 form of the operator).
 
---linear adds a "linear" object: the forward with its producer fused in
-(dcn4_forward_linear: offset_mask = x W^T + b formed per tile on the tensor
-cores; fp16/bf16 workloads) against the same producer run as a separate
-library GEMM (torch.nn.functional.linear, cuBLAS) followed by dcn4_forward.
+The "linear" object (skipped with --no-linear) times the layer with its
+producer: the forward with the producer fused in (dcn4_forward_linear:
+offset_mask = x W^T + b formed per tile on the tensor cores; fp16/bf16
+workloads) against the producer as a separate library GEMM (cuBLAS) followed
+by dcn4_forward; and the layer's backward dcn4_backward_linear (the
+aggregation's backward, then grad_x = g W, grad_W = g^T x, grad_b on the
+tensor cores in libdcn4) against dcn4_backward followed by cuBLAS products.
+
+--profile runs warm-up + steps untimed passes of the workload (forward and
+backward; with --linear also the fused forward and dcn4_backward_linear) and
+prints no JSON line: a fixed launch sequence for ncu captures.
 
 The line also carries "per_config": forward and backward µs per call,
 achieved GB/s and fractions of the measured copy bandwidth and of 8 TB/s for
@@ -537,8 +545,8 @@ def run_native(args, w: gen.Workload) -> dict:
     }
     if e2e is not None:
         result["e2e"] = e2e
-    if args.linear:
-        result["linear"] = linear_leg(w, v, p, flush, stream, dev, world)
+    if not args.no_linear:
+        result["linear"] = linear_leg(w, v, gy, p, flush, stream, dev, world)
     if not args.no_per_config:
         sampler = ClockSampler(local if world > 1 else torch.cuda.current_device())
         sampler.start()
@@ -699,10 +707,12 @@ def attention_leg(dev, world: int, reps: int, flush, stream) -> dict:
     return res
 
 
-def linear_leg(w: gen.Workload, v, p, flush, stream, dev, world: int) -> dict:
+def linear_leg(w: gen.Workload, v, gy, p, flush, stream, dev, world: int) -> dict:
     """µs per call (CUDA events, L2 flushed before each, max over ranks): the fused
     forward with and without storing its offset_mask, against cuBLAS's linear layer
-    followed by dcn4_forward, on seeded x [N,Ho,Wo,C], W [P,C], b [P]."""
+    followed by dcn4_forward, on seeded x [N,Ho,Wo,C], W [P,C], b [P]; and the
+    layer's backward (dcn4_backward_linear) against dcn4_backward followed by
+    cuBLAS products for the linear layer's gradients."""
     import numpy as np
     import torch
     import torch.nn.functional as F
@@ -752,7 +762,89 @@ def linear_leg(w: gen.Workload, v, p, flush, stream, dev, world: int) -> dict:
     res["speedup_vs_unfused"] = round(res["cublas_linear_then_forward_us"] / res["fused_us"], 3)
     res["gemm"] = f"x [{w.N * w.Ho * w.Wo}, {w.C}] @ W^T [{w.C}, {w.P}] + b, mma.sync m16n8k16, fp32 accumulation"
     res["launches_per_call"] = 1
+
+    # Backward of the layer: dcn4_backward_linear (the aggregation's backward, then the
+    # linear layer's gradients in libdcn4) against dcn4_backward followed by cuBLAS.
+    gv, gom = torch.empty_like(v), torch.empty_like(om)
+    gx, gw, gb = torch.empty_like(x), torch.empty_like(wt), torch.empty_like(b)
+    nb = dcn.dcn4_backward_workspace_size(p)
+    nbl = dcn.dcn4_backward_linear_workspace_size(p, w.C)
+    ws = torch.empty(max(nbl, 16), dtype=torch.uint8, device=dev)
+    fused_om()
+    torch.cuda.synchronize(dev)
+    g2, x2 = gom.view(-1, w.P), x.view(-1, w.C)
+
+    def bwd_chain():
+        dcn.check(dcn.dcn4_backward_linear(p, w.C, ptr["v"], ptr["om"], ptr["x"], ptr["w"], gy.data_ptr(),
+                                           gv.data_ptr(), gom.data_ptr(), gx.data_ptr(), gw.data_ptr(), gb.data_ptr(),
+                                           ws.data_ptr(), nbl, sh))
+
+    def bwd_only():
+        dcn.check(dcn.dcn4_backward(p, ptr["v"], ptr["om"], gy.data_ptr(), gv.data_ptr(), gom.data_ptr(),
+                                    ws.data_ptr(), nb, sh))
+
+    def bwd_then_cublas():
+        bwd_only()
+        torch.mm(g2, wt, out=gx.view(-1, w.C))
+        torch.mm(g2.t(), x2, out=gw)
+        torch.sum(g2, 0, out=gb)
+
+    for name, fn in (("backward_linear_us", bwd_chain), ("backward_us", bwd_only),
+                     ("backward_then_cublas_us", bwd_then_cublas)):
+        for _ in range(5):
+            fn()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(100)]
+        for e0, e1 in ev:
+            flush.zero_()
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+        torch.cuda.synchronize(dev)
+        res[name] = round(max_over_ranks(statistics.mean(a.elapsed_time(c) for a, c in ev) * 1e3, dev), 2)
+    M = w.N * w.Ho * w.Wo
+    lin_us = res["backward_linear_us"] - res["backward_us"]
+    res["linear_backward_us"] = round(lin_us, 2)
+    res["cublas_linear_backward_us"] = round(res["backward_then_cublas_us"] - res["backward_us"], 2)
+    # g, x read once and grad_x written once: the least the layer's gradients move
+    lin_bytes = M * (w.P + 2 * w.C) * 2
+    res["linear_backward_bytes"] = lin_bytes
+    if lin_us > 0:
+        res["linear_backward_gbs"] = round(lin_bytes / (lin_us * 1e-6) / 1e9, 1)
+    del gv, gom, gx, gw, gb, ws
     return res
+
+
+def run_profile(args, w: gen.Workload) -> None:
+    """--profile: warm-up + steps passes of the path (forward and backward of the
+    workload; with --linear the fused forward and dcn4_backward_linear too) with
+    no timing and no JSON line -- a short, fixed launch sequence for ncu captures."""
+    import numpy as np
+    import torch
+    import deformable_convolution_sampling_b200 as dcn
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    tdt = {"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16}[w.dtype]
+
+    def dev_t(a):
+        a = np.ascontiguousarray(a)
+        t = torch.from_numpy(a.view(np.int16)).view(tdt) if w.dtype == "bf16" else torch.from_numpy(a)
+        return t.to(dev)
+    inp = gen.make_inputs(w, tail_fill=0.0)
+    v, om, gy = dev_t(inp["value"]), dev_t(inp["offset_mask"]), dev_t(inp["grad_out"])
+    p = dcn.make_params(dtype=w.dtype, **w.geometry())
+    lin = None
+    if args.linear:
+        li = gen.make_linear_inputs(w, w.C)
+        lin = dev_t(li["x"]), dev_t(li["weight"]), dev_t(li["bias"])
+    for _ in range(args.warmup + args.steps):
+        dcn.forward(p, v, om)
+        dcn.backward(p, v, om, gy)
+        if lin is not None:
+            om_lin = torch.empty_like(om)
+            dcn.forward_linear(p, v, *lin, offset_mask_out=om_lin)
+            dcn.backward_linear(p, v, om_lin, lin[0], lin[1], gy)
+    torch.cuda.synchronize(dev)
+    print(f"profile: {w.name}: {args.warmup + args.steps} passes done", flush=True)
 
 
 def main(argv=None):
@@ -764,8 +856,11 @@ def main(argv=None):
     ap.add_argument("--workload", default="stage1_f16", choices=sorted(gen.WORKLOADS))
     ap.add_argument("--softmax", action="store_true",
                     help="masks are logits normalised by a softmax over the K points (DCNv3 form)")
+    ap.add_argument("--no-linear", action="store_true",
+                    help="skip the timings of the layer with its offset/mask linear producer (fused forward, "
+                         "dcn4_backward_linear)")
     ap.add_argument("--linear", action="store_true",
-                    help="also time the forward with the offset/mask linear layer fused in")
+                    help="with --profile: also run the fused forward and dcn4_backward_linear")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-per-config", action="store_true",
@@ -774,12 +869,17 @@ def main(argv=None):
                     help="calls per stage and workload in the per-config timings")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="target seconds of oracle work for the cpu_baseline sample")
+    ap.add_argument("--profile", action="store_true",
+                    help="run warm-up + steps untimed passes of --workload for an ncu capture; no JSON line")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     w = gen.WORKLOADS[args.workload]
     if args.softmax:
         w = dataclasses.replace(w, softmax=1, name=w.name + "_softmax")
+    if args.profile:
+        run_profile(args, w)
+        return
     rank, world, _ = dist_env()
     if args.impl == "reference":
         res = run_reference(args, w)

@@ -111,6 +111,8 @@ def _load() -> ctypes.CDLL:
         "dcn4_backward_noalloc_capacity": ([], ctypes.c_size_t),
         "dcn4_noalloc_last_error": ([], ctypes.c_char_p),
         "dcn4_backward_diagnostics": ([P, vp, ctypes.c_size_t, ip, vp], ctypes.c_int),
+        "dcn4_backward_linear_workspace_size": ([P, ctypes.c_int], ctypes.c_size_t),
+        "dcn4_backward_linear": ([P, ctypes.c_int] + [vp] * 11 + [ctypes.c_size_t, vp], ctypes.c_int),
         "dcn4_attn_check_params": ([AP], ctypes.c_int),
         "dcn4_attn_forward": ([AP, vp, vp, vp, vp, vp], ctypes.c_int),
         "dcn4_attn_backward_workspace_size": ([AP], ctypes.c_size_t),
@@ -190,6 +192,18 @@ def dcn4_backward_diagnostics(p: dcn4_params, workspace, workspace_bytes: int, s
     counts = (ctypes.c_int * 3)()
     st = lib.dcn4_backward_diagnostics(ctypes.byref(p), workspace, workspace_bytes, counts, stream)
     return st, list(counts)
+
+
+def dcn4_backward_linear_workspace_size(p: dcn4_params, Cx: int) -> int:
+    return lib.dcn4_backward_linear_workspace_size(ctypes.byref(p), int(Cx))
+
+
+def dcn4_backward_linear(p: dcn4_params, Cx: int, value, offset_mask, x, weight, grad_out, grad_value,
+                         grad_offset_mask, grad_x, grad_weight, grad_bias, workspace, workspace_bytes: int,
+                         stream=None) -> int:
+    return lib.dcn4_backward_linear(ctypes.byref(p), int(Cx), value, offset_mask, x, weight, grad_out, grad_value,
+                                    grad_offset_mask, grad_x, grad_weight, grad_bias, workspace, workspace_bytes,
+                                    stream)
 
 
 def dcn4_attn_check_params(p: dcn4_attn_params) -> int:
@@ -304,6 +318,36 @@ def backward(p: dcn4_params, value, offset_mask, grad_out, grad_value=None, grad
                         grad_value.data_ptr(), grad_offset_mask.data_ptr(), ws_ptr, ws_bytes,
                         _stream_handle(value.device)))
     return grad_value, grad_offset_mask
+
+
+def backward_linear(p: dcn4_params, value, offset_mask, x, weight, grad_out, with_bias: bool = True,
+                    want_x: bool = True, want_weight: bool = True, workspace=None):
+    """Backward of forward_linear for CUDA tensors (offset_mask: the one the forward
+    formed): (grad_value, grad_offset_mask, grad_x or None, grad_weight or None,
+    grad_bias or None), all computed in libdcn4."""
+    import torch
+    st, Ho, Wo = dcn4_output_dims(p)
+    check(st)
+    dt = _torch_dtype(p.dtype)
+    dev = value.device
+    Cx = x.shape[-1]
+    gv = torch.empty_like(value, dtype=dt)
+    gom = torch.empty((p.N, Ho, Wo, p.P), dtype=dt, device=dev)
+    gx = torch.empty_like(x) if want_x else None
+    gw = torch.empty_like(weight) if want_weight else None
+    gb = torch.empty((p.P,), dtype=dt, device=dev) if with_bias else None
+    need = dcn4_backward_linear_workspace_size(p, Cx)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+
+    def ptr(t):
+        return t.data_ptr() if t is not None else None
+
+    check(dcn4_backward_linear(p, Cx, value.data_ptr(), offset_mask.data_ptr(), x.data_ptr(), weight.data_ptr(),
+                               grad_out.data_ptr(), gv.data_ptr(), gom.data_ptr(), ptr(gx), ptr(gw), ptr(gb),
+                               workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                               _stream_handle(dev)))
+    return gv, gom, gx, gw, gb
 
 
 def attn_forward(p: dcn4_attn_params, value, ref_points, offset_logits, out=None):
@@ -422,9 +466,10 @@ def _autograd_function_linear():
     class DCNv4CoreLinear(torch.autograd.Function):
         """The offset/mask linear layer fused into the aggregation as a
         torch.autograd.Function.  Forward: dcn4_forward_linear, keeping the
-        offset_mask it formed.  Backward: dcn4_backward on that offset_mask, then the
-        linear layer's gradients (grad_x = g W, grad_W = g^T x, grad_b = sum g, with
-        g = grad_offset_mask as [M, P]) as library GEMMs."""
+        offset_mask it formed.  Backward: dcn4_backward_linear, i.e. dcn4_backward on
+        that offset_mask, then the linear layer's gradients (grad_x = g W,
+        grad_W = g^T x, grad_b = sum g, with g = grad_offset_mask as [M, P]) in
+        libdcn4's tensor-core kernels."""
 
         @staticmethod
         def forward(ctx, value, x, weight, bias, p):
@@ -440,12 +485,9 @@ def _autograd_function_linear():
         @staticmethod
         def backward(ctx, grad_out):
             value, x, weight, om = ctx.saved_tensors
-            grad_value, gom = backward(ctx.p, value, om, grad_out.contiguous())
-            g = gom.reshape(-1, gom.shape[-1])
-            xm = x.reshape(-1, x.shape[-1])
-            grad_x = (g @ weight).reshape(x.shape)
-            grad_w = g.t() @ xm
-            grad_b = g.sum(0) if ctx.has_bias else None
+            grad_value, _, grad_x, grad_w, grad_b = backward_linear(
+                ctx.p, value, om, x, weight, grad_out.contiguous(), with_bias=ctx.has_bias,
+                want_x=ctx.needs_input_grad[1], want_weight=ctx.needs_input_grad[2])
             return grad_value, grad_x, grad_w, grad_b, None
 
     return DCNv4CoreLinear

@@ -444,6 +444,53 @@ int dcn4_backward(const dcn4_params* p, const void* value, const void* offset_ma
     return dcn4_backward_value(p, offset_mask, grad_out, grad_value, workspace, workspace_bytes, stream);
 }
 
+size_t dcn4_backward_linear_workspace_size(const dcn4_params* p, int Cx) {
+    const size_t b = dcn4_backward_workspace_size(p);
+    if (b == 0 || Cx < 1 || static_cast<long long>(p->P) * Cx >= (1LL << 31)) return 0;
+    return round256(b) + round256(dcn4::linear_backward_workspace_bytes(p->P, Cx));
+}
+
+int dcn4_backward_linear(const dcn4_params* p, int Cx, const void* value, const void* offset_mask, const void* x,
+                         const void* weight, const void* grad_out, void* grad_value, void* grad_offset_mask,
+                         void* grad_x, void* grad_weight, void* grad_bias, void* workspace, size_t workspace_bytes,
+                         void* stream) {
+    dcn4::Geometry g;
+    const int st = make_geometry(p, true, false, &g);
+    if (st != DCN4_OK) return st;
+    if (p->dtype == DCN4_F32) return fail(DCN4_ERR_UNSUPPORTED, "the linear producer takes fp16 or bf16");
+    if (Cx < 16 || Cx % 16 != 0 || Cx > (1 << 16))
+        return fail(DCN4_ERR_BAD_SHAPE, "Cx=%d must be a positive multiple of 16", Cx);
+    if (static_cast<long long>(p->P) * Cx >= (1LL << 31) || (g.total_pix + 127) / 128 > 0x7fffffffLL)
+        return fail(DCN4_ERR_UNSUPPORTED, "x or weight too large");
+    if (!aligned16(x) || !aligned16(weight) || !aligned16(grad_x) || !aligned16(grad_weight) || !aligned16(grad_bias))
+        return fail(DCN4_ERR_MISALIGNED, "every pointer must be 16-byte aligned");
+    const size_t need = dcn4_backward_linear_workspace_size(p, Cx);
+    if (!workspace || workspace_bytes < need)
+        return fail(DCN4_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, workspace_bytes);
+    if (!aligned16(workspace)) return fail(DCN4_ERR_MISALIGNED, "workspace must be 16-byte aligned");
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t eb = static_cast<size_t>(elem_bytes(p->dtype));
+    if (g.total_pix == 0) {
+        // no output pixels: the weight and bias gradients are empty sums
+        cudaError_t e = cudaSuccess;
+        if (grad_weight) e = cudaMemsetAsync(grad_weight, 0, static_cast<size_t>(p->P) * Cx * eb, s);
+        if (e == cudaSuccess && grad_bias) e = cudaMemsetAsync(grad_bias, 0, static_cast<size_t>(p->P) * eb, s);
+        if (e != cudaSuccess) return fail(DCN4_ERR_LAUNCH, "zeroing grad_weight/grad_bias: %s", cudaGetErrorString(e));
+        return DCN4_OK;
+    }
+    if (!grad_offset_mask) return fail(DCN4_ERR_NULL, "grad_offset_mask must be non-NULL");
+    if ((grad_x && !weight) || (grad_weight && !x))
+        return fail(DCN4_ERR_NULL, "grad_x needs weight and grad_weight needs x");
+    const size_t lin_off = round256(dcn4_backward_workspace_size(p));
+    const int a = dcn4_backward(p, value, offset_mask, grad_out, grad_value, grad_offset_mask, workspace, lin_off, stream);
+    if (a != DCN4_OK) return a;
+    float* acc = reinterpret_cast<float*>(static_cast<char*>(workspace) + lin_off);
+    const cudaError_t e = dcn4::launch_linear_backward(p->dtype, g.total_pix, p->P, Cx, x, weight, grad_offset_mask,
+                                                       grad_x, grad_weight, grad_bias, acc, s);
+    if (e != cudaSuccess) return fail(DCN4_ERR_LAUNCH, "linear backward launch: %s", cudaGetErrorString(e));
+    return DCN4_OK;
+}
+
 int dcn4_attn_check_params(const dcn4_attn_params* p) {
     dcn4::Geometry g;
     for (int wide = 0; wide < 2; ++wide) {

@@ -369,6 +369,13 @@ cudaError_t launch_forward_linear(const Geometry& g, int dtype, const void* valu
 size_t forward_linear_smem_bytes(const Geometry& g, int Cx, bool w_smem);
 // Whether the fused forward stages W in shared memory for this shape.
 bool forward_linear_w_smem(const Geometry& g, int Cx);
+// Gradients of the linear producer from gom = grad_offset_mask as an [M, P]
+// matrix (16-bit dtypes): gx = gom W [M, Cx], gw = gom^T x [P, Cx], gb = column
+// sums of gom [P]; any of the three may be null.  ws: fp32 scratch of
+// linear_backward_workspace_bytes(P, Cx) bytes (grad_W and grad_b accumulators).
+size_t linear_backward_workspace_bytes(int P, int Cx);
+cudaError_t launch_linear_backward(int dtype, long long M, int P, int Cx, const void* x, const void* w,
+                                   const void* gom, void* gx, void* gw, void* gb, float* ws, cudaStream_t stream);
 size_t backward_smem_bytes(const Geometry& g, int elem_bytes);
 // Single-scale deformable attention (dcn4_attn.cu): g holds the value map (N, H,
 // W, G, Cg, C), the points per query (K), the row length (P), offset_scale (s)

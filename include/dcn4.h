@@ -67,7 +67,7 @@
 extern "C" {
 #endif
 
-#define DCN4_VERSION 140  /* 1.4.0: deformable attention (dcn4_attn_*) */
+#define DCN4_VERSION 150  /* 1.5.0: backward of the fused linear producer (dcn4_backward_linear) */
 
 typedef enum {
     DCN4_F32 = 0,   /* IEEE binary32            */
@@ -247,6 +247,37 @@ int dcn4_backward_value(const dcn4_params* p, const void* offset_mask, const voi
  * Same checks as dcn4_backward; counts must hold 3 ints. */
 int dcn4_backward_diagnostics(const dcn4_params* p, const void* workspace, size_t workspace_bytes, int* counts,
                               void* stream);
+
+/* Bytes of device workspace dcn4_backward_linear needs: dcn4_backward's
+ * workspace rounded up to 256 bytes, then fp32 accumulators for grad_weight
+ * (P*Cx) and grad_bias (P), rounded up to 256 bytes; 0 if p is invalid. */
+size_t dcn4_backward_linear_workspace_size(const dcn4_params* p, int Cx);
+
+/* Backward of dcn4_forward_linear, the aggregation with its offset/mask linear
+ * layer (CSDN summary, section 2.2 "DCN模块的微设计"): with
+ * offset_mask = x weight^T + bias as saved by the forward (its offset_mask_out),
+ *   grad_value, grad_offset_mask  as dcn4_backward computes them, then, with
+ *   g = grad_offset_mask as an [M = N*Ho*Wo, P] matrix (its padding columns are 0):
+ *   grad_x      [N, Ho, Wo, Cx] = g weight          (sum over j of g[m, j] * weight[j, c])
+ *   grad_weight [P, Cx]         = g^T x             (sum over m of g[m, j] * x[m, c])
+ *   grad_bias   [P]             = sum over m of g[m, j]
+ * All of dtype (fp16 or bf16; DCN4_ERR_UNSUPPORTED for fp32).  The products read
+ * g as dcn4_backward rounded it to dtype, run on the tensor cores with fp32
+ * accumulation and are rounded to dtype once; grad_weight and grad_bias sum
+ * partial products of row chunks with fp32 atomics (so their last bit may vary
+ * from call to call).  grad_x, grad_weight and grad_bias may each be NULL (not
+ * wanted); grad_value and grad_offset_mask are required.  Every pointer 16-byte
+ * aligned; Cx a positive multiple of 16 (DCN4_ERR_BAD_SHAPE); `workspace`
+ * (device, >= dcn4_backward_linear_workspace_size bytes) is clobbered, its first
+ * part exactly as by dcn4_backward (so dcn4_backward_diagnostics reads it).
+ * With N*Ho*Wo = 0 only grad_weight and grad_bias are written (zeros).
+ * Launches on `stream`: dcn4_backward's launches, then one kernel for grad_x,
+ * a memset and one kernel for the grad_weight/grad_bias accumulators, and one
+ * rounding kernel for each of grad_weight and grad_bias. */
+int dcn4_backward_linear(const dcn4_params* p, int Cx, const void* value, const void* offset_mask, const void* x,
+                         const void* weight, const void* grad_out, void* grad_value, void* grad_offset_mask,
+                         void* grad_x, void* grad_weight, void* grad_bias, void* workspace, size_t workspace_bytes,
+                         void* stream);
 
 /* ---------------------------------------------------------------------------
  * Deformable attention, single scale.

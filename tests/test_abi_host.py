@@ -70,7 +70,7 @@ def test_params_mirror_matches_the_header(dcn):
             fields += [n.strip() for n in names.split(",")]
     assert [f[0] for f in dcn.dcn4_params._fields_] == fields
     assert ctypes.sizeof(dcn.dcn4_params) == 4 * len(fields)
-    assert dcn.dcn4_version() == 140
+    assert dcn.dcn4_version() == 150
 
 
 def test_attn_params_mirror_matches_the_header(dcn):
@@ -209,6 +209,36 @@ assert call(p, 1 << 14) == -5                   # x tiles too large for shared m
 assert call(p, 64, x=None) == -1
 assert call(p, 64, bias=40) == -4 and call(p, 64, om=72) == -4 and call(p, 64, x=36) == -4
 bad = dcn.make_params(N=2, H=8, W=8, G=4, Cg=16, dtype="f16")
+bad.P = 100
+assert call(bad, 64) == -3
+assert dcn.dcn4_last_error() != ""
+""")
+
+
+def test_backward_linear_checks_before_launch():
+    """dcn4_backward_linear validates on the host before its first launch (made-up
+    addresses: checked in a child process that sees no GPU)."""
+    run_without_gpu("""
+p = dcn.make_params(N=2, H=8, W=8, G=4, Cg=16, dtype="bf16")
+need = dcn.dcn4_backward_linear_workspace_size(p, 64)
+assert need >= dcn.dcn4_backward_workspace_size(p) + 4 * (p.P * 64 + p.P)
+assert need % 256 == 0 and dcn.dcn4_backward_linear_workspace_size(p, 0) == 0
+ok = dict(value=16, om=32, x=48, w=64, gy=80, gv=96, gom=112, gx=128, gw=144, gb=160, ws=4096, nb=need)
+
+def call(params, Cx, **kw):
+    a = {**ok, **kw}
+    return dcn.dcn4_backward_linear(params, Cx, a["value"], a["om"], a["x"], a["w"], a["gy"], a["gv"], a["gom"],
+                                    a["gx"], a["gw"], a["gb"], a["ws"], a["nb"], None)
+p32 = dcn.make_params(N=2, H=8, W=8, G=4, Cg=16, dtype="f32")
+assert call(p32, 64, nb=1 << 24) == -5              # fp32: no linear producer
+assert call(p, 24) == -2 and call(p, 0) == -2       # Cx not a multiple of 16
+assert call(p, 64, nb=need - 1) == -6 and call(p, 64, ws=None) == -6
+assert call(p, 64, ws=4100) == -4                   # misaligned workspace
+assert call(p, 64, gw=148) == -4 and call(p, 64, x=52) == -4 and call(p, 64, gb=161) == -4
+assert call(p, 64, gom=None) == -1
+assert call(p, 64, w=None) == -1 and call(p, 64, x=None) == -1
+assert call(p, 64, value=None) == -1 and call(p, 64, gv=None) == -1
+bad = dcn.make_params(N=2, H=8, W=8, G=4, Cg=16, dtype="bf16")
 bad.P = 100
 assert call(bad, 64) == -3
 assert dcn.dcn4_last_error() != ""
