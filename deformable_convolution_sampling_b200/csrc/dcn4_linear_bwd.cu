@@ -172,7 +172,7 @@ __device__ __forceinline__ void red_add2(float* dst, float a, float b) {
 template <typename T>
 __global__ void __launch_bounds__(kLbThreads) linear_grad_w_kernel(const T* __restrict__ g, const T* __restrict__ x,
                                                                    float* __restrict__ wacc, float* __restrict__ bacc,
-                                                                   long long M, int P, int Cx, int mchunk) {
+                                                                   long long M, int P, int Cx, long long mchunk) {
     __shared__ __align__(16) T g_s[2][kWK][kWLd];  // [m][p]
     __shared__ __align__(16) T x_s[2][kWK][kWLd];  // [m][c]
     __shared__ float b_part[kLbThreads];
@@ -296,7 +296,7 @@ cudaError_t linear_backward_typed(long long M, int P, int Cx, const void* x, con
     const long long zc = (M + mchunk - 1) / mchunk;
     const dim3 grid(static_cast<unsigned>(pt), static_cast<unsigned>(ct), static_cast<unsigned>(std::max<long long>(1, zc)));
     linear_grad_w_kernel<T><<<grid, kLbThreads, 0, stream>>>(g, static_cast<const T*>(x), ws, gb ? ws + wsz : nullptr,
-                                                             M, P, Cx, static_cast<int>(mchunk));
+                                                             M, P, Cx, mchunk);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     if (gw) {
