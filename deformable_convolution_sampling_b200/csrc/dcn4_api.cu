@@ -114,13 +114,37 @@ int make_geometry(const dcn4_params* p, bool backward, bool wide, dcn4::Geometry
     long long ppc = kTargetThreads / lanes_pp;
     while (ppc > 1 && ppc * row_bytes > kSmemDefault) --ppc;
     if (ppc * row_bytes > kSmemMax) return fail(DCN4_ERR_UNSUPPORTED, "P=%d rows do not fit shared memory", p->P);
-    // A CTA covers a TH x TW tile of output pixels of one image: as square as
-    // the pixel budget allows (TW a power of two), clipped to the image.
-    long long TW = 1;
-    while (TW * TW < ppc && TW * 2 <= ppc) TW *= 2;
-    while (TW > 1 && TW / 2 >= Wo) TW /= 2;
-    long long TH = ppc / TW;
-    if (TH > Ho) TH = Ho;
+    // A CTA covers a TH x TW tile of output pixels of one image (TW a power of
+    // two, TH = the rest of the pixel budget, both clipped to the image): the
+    // shape that leaves the fewest threads idle on the image's ragged edges;
+    // among equals the one with more pixels, then the squarer one.  Shapes
+    // more than 4:1 are taken only when nothing squarer exists (a 14 x 1 strip
+    // fills a 14 x 14 map exactly but gathers from a wider halo per pixel).
+    long long TW = 1, TH = 1;
+    {
+        long long best_used = -1, best_slots = 1, best_px = 0, best_skew = 0;
+        for (int pass = 0; pass < 2 && best_used < 0; ++pass)
+        for (long long tw = 1; tw <= ppc; tw *= 2) {
+            if (tw > 1 && tw / 2 >= Wo) break;
+            const long long th = std::min(ppc / tw, Ho);
+            if (pass == 0 && std::max(th, tw) > 4 * std::min(th, tw)) continue;
+            const long long slots = (Ho + th - 1) / th * th * ((Wo + tw - 1) / tw * tw);
+            const long long used = Ho * Wo;
+            const long long px = th * tw, skew = std::max(th, tw) / std::min(th, tw);
+            // compare used / slots as fractions without rounding
+            const bool better = best_used < 0 || used * best_slots > best_used * slots ||
+                                (used * best_slots == best_used * slots &&
+                                 (px > best_px || (px == best_px && skew < best_skew)));
+            if (better) {
+                best_used = used;
+                best_slots = slots;
+                best_px = px;
+                best_skew = skew;
+                TW = tw;
+                TH = th;
+            }
+        }
+    }
     const long long tiles_h = (Ho + TH - 1) / TH, tiles_w = (Wo + TW - 1) / TW;
     if (static_cast<long long>(p->N) * tiles_h * tiles_w > 0x7fffffffLL)
         return fail(DCN4_ERR_UNSUPPORTED, "grid too large");

@@ -217,6 +217,11 @@ __global__ void __launch_bounds__(256, 3) samples_kernel(const Geometry g, const
     T* om_s = reinterpret_cast<T*>(smem);
     T* gom_s = reinterpret_cast<T*>(smem + tile_elems * sizeof(T));  // P % 8 == 0 keeps this 16-byte aligned
     const bool filing = sizeof(T) == 2 && g.buckets != 0;
+    // Unrolled grids without softmax stage only the meta words: the record body
+    // (bin, mask bits, fractions) is formed again at write-out from the offsets,
+    // which stay in shared memory, with the same fp32 arithmetic.  Half the
+    // staging leaves that much more of the SM's L1 to the gathers.
+    constexpr bool SLIM = KH > 0 && !SM;
 
     const Tile t = tile_of_block(g);
     const int K = KH > 0 ? KH * KW - (RC ? 1 : 0) : g.K;
@@ -228,7 +233,7 @@ __global__ void __launch_bounds__(256, 3) samples_kernel(const Geometry g, const
         // staging after the two offset_mask tiles
         unsigned char* st = smem + 2 * static_cast<size_t>(tile_elems) * sizeof(T);
         fs.rec = reinterpret_cast<uint64_t*>(st);
-        fs.meta = fs.rec + (KH > 0 ? K : filing_chunk(g)) * blockDim.x;
+        fs.meta = SLIM ? fs.rec : fs.rec + (KH > 0 ? K : filing_chunk(g)) * blockDim.x;
         // window of tiles centred on the anchors of this CTA's grid
         const int amid_h = t.ho0 * g.sh - g.ph + ((t.th - 1) * g.sh + (kh - 1) * g.dh) / 2;
         const int amid_w = t.wo0 * g.sw - g.pw + ((t.tw - 1) * g.sw + (kw - 1) * g.dw) / 2;
@@ -302,11 +307,7 @@ __global__ void __launch_bounds__(256, 3) samples_kernel(const Geometry g, const
             sa.bucket_rec[at] = rec;
         };
         const int rmask = (1 << kRankBits) - 1;
-        for (int j = 0; j < nk; ++j) {
-            const int at = j * blockDim.x + threadIdx.x;
-            const uint64_t meta = fs.meta[at];
-            if (!((meta >> 61) & 1)) continue;
-            const uint64_t rec = fs.rec[at];
+        auto emit = [&](uint64_t meta, uint64_t rec) {
             const int dl0 = static_cast<int>(meta & 63);
             put(dl0, static_cast<int>(meta >> 6) & rmask, rec);
             const uint64_t body = rec & ~0xffffull;
@@ -319,6 +320,40 @@ __global__ void __launch_bounds__(256, 3) samples_kernel(const Geometry g, const
             if ((meta >> 60) & 1)  // below-right
                 put(dl0 + (1 << fs.wwl) + 1, static_cast<int>(meta >> (6 + 3 * kRankBits)) & rmask,
                     body | static_cast<uint64_t>(bin - g.BH * (g.BW + 1) - g.BW));
+        };
+        if constexpr (SLIM) {
+            // Walk the grid as the sample loop did, so the anchors are compile-time
+            // offsets; the cell's tile comes back from the staged window slot.
+            const int gbase = grp * (g.BH + 1) * (g.BW + 1);
+            int j = 0;
+#pragma unroll
+            for (int iw = 0; iw < KW; ++iw) {
+#pragma unroll
+                for (int ih = 0; ih < KH; ++ih) {
+                    if (RC && iw == KW / 2 && ih == KH / 2) continue;
+                    const int kk = j++;
+                    const uint64_t meta = fs.meta[kk * blockDim.x + threadIdx.x];
+                    if (!((meta >> 61) & 1)) continue;
+                    const int dl0 = static_cast<int>(meta & 63);
+                    const int ta = fs.wy0 + (dl0 >> fs.wwl), ua = fs.wx0 + (dl0 & wmask);
+                    const float h = __fmaf_rn(g.s, to_f32(row[2 * kk + 1]), static_cast<float>(hb + ih * g.dh));
+                    const float w = __fmaf_rn(g.s, to_f32(row[2 * kk]), static_cast<float>(wb + iw * g.dw));
+                    const float h0f = floorf(h), w0f = floorf(w);
+                    const int cy = static_cast<int>(h0f) + 1 - ta * g.BH, cx = static_cast<int>(w0f) + 1 - ua * g.BW;
+                    const uint64_t rec = (static_cast<uint64_t>(raw_bits(row[2 * K + kk])) << 16) |
+                                         (static_cast<uint64_t>(fix16(h - h0f)) << 32) |
+                                         (static_cast<uint64_t>(fix16(w - w0f)) << 48) |
+                                         static_cast<uint64_t>(gbase + cy * (g.BW + 1) + cx);
+                    emit(meta, rec);
+                }
+            }
+        } else {
+            for (int j = 0; j < nk; ++j) {
+                const int at = j * blockDim.x + threadIdx.x;
+                const uint64_t meta = fs.meta[at];
+                if (!((meta >> 61) & 1)) continue;
+                emit(meta, fs.rec[at]);
+            }
         }
     };
     // Generic grids file in chunks of filing_chunk(g) points (a bounded staging area).
@@ -420,7 +455,7 @@ __global__ void __launch_bounds__(256, 3) samples_kernel(const Geometry g, const
                     }
                     const int at = (KH > 0 ? kk : kc) * blockDim.x + threadIdx.x;
                     fs.meta[at] = meta;
-                    fs.rec[at] = rec | static_cast<uint64_t>(gbase + cy * (g.BW + 1) + cx);
+                    if constexpr (!SLIM) fs.rec[at] = rec | static_cast<uint64_t>(gbase + cy * (g.BW + 1) + cx);
                     if constexpr (KH == 0) {
                         // every thread takes the same branch: kc, kk and filing are uniform
                         if (++kc == fkc || kk + 1 == K) {
@@ -1167,7 +1202,10 @@ cudaError_t launch_value_vec(const Geometry& g, const void* om, const void* gout
 
 size_t backward_smem_bytes(const Geometry& g, int elem_bytes) {
     size_t b = static_cast<size_t>(g.TH) * g.TW * g.P * elem_bytes * 2;
-    if (elem_bytes == 2 && g.buckets) b += static_cast<size_t>(filing_chunk(g)) * samples_threads(g) * 16;  // staging
+    if (elem_bytes == 2 && g.buckets) {  // staging: meta words only for the unrolled grids without softmax
+        const size_t per = (g.kh == 3 && g.kw == 3 && !g.softmax) ? 8 : 16;
+        b += static_cast<size_t>(filing_chunk(g)) * samples_threads(g) * per;
+    }
     return b;
 }
 
