@@ -808,6 +808,9 @@ def linear_leg(w: gen.Workload, v, gy, p, flush, stream, dev, world: int) -> dic
     # g, x read once and grad_x written once: the least the layer's gradients move
     lin_bytes = M * (w.P + 2 * w.C) * 2
     res["linear_backward_bytes"] = lin_bytes
+    res["linear_backward_gemm"] = (f"grad_x = g W ([{M}, {w.P}] x [{w.P}, {w.C}]), grad_W = g^T x, grad_b: tcgen05.mma "
+                                   f"kind::f16 from TMA-fed 128-byte-swizzled shared memory, fp32 accumulators in "
+                                   f"tensor memory, warp-specialised")
     if lin_us > 0:
         res["linear_backward_gbs"] = round(lin_bytes / (lin_us * 1e-6) / 1e9, 1)
     del gv, gom, gx, gw, gb, ws

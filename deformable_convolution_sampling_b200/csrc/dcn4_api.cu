@@ -484,8 +484,8 @@ int dcn4_backward_linear(const dcn4_params* p, int Cx, const void* value, const 
     if (p->dtype == DCN4_F32) return fail(DCN4_ERR_UNSUPPORTED, "the linear producer takes fp16 or bf16");
     if (Cx < 16 || Cx % 16 != 0 || Cx > (1 << 16))
         return fail(DCN4_ERR_BAD_SHAPE, "Cx=%d must be a positive multiple of 16", Cx);
-    if (static_cast<long long>(p->P) * Cx >= (1LL << 31) || (g.total_pix + 127) / 128 > 0x7fffffffLL)
-        return fail(DCN4_ERR_UNSUPPORTED, "x or weight too large");
+    if (static_cast<long long>(p->P) * Cx >= (1LL << 31) || g.total_pix >= (1LL << 31))
+        return fail(DCN4_ERR_UNSUPPORTED, "x or weight too large (N*Ho*Wo and P*Cx must be < 2^31)");
     if (!aligned16(x) || !aligned16(weight) || !aligned16(grad_x) || !aligned16(grad_weight) || !aligned16(grad_bias))
         return fail(DCN4_ERR_MISALIGNED, "every pointer must be 16-byte aligned");
     const size_t need = dcn4_backward_linear_workspace_size(p, Cx);

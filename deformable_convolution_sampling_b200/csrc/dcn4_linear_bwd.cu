@@ -6,17 +6,22 @@
 // Its gradients, with g = grad_offset_mask as an [M, P] matrix (M output
 // pixels; the padding columns of g are zero):
 //     grad_x [M, Cx] = g W          grad_W [P, Cx] = g^T x          grad_b [P] = sum_m g[m, :]
-// Both products run on the tensor cores (mma.sync m16n8k16, fp16/bf16 in,
-// fp32 accumulation) from tiles staged in shared memory by a cp.async ring.  They are bound by HBM (g and x read, grad_x written: 40-60
-// FLOP per byte, far below the tensor pipe's ridge), so the kernels are built
-// for streaming: long-lived CTAs whose ring runs across tile boundaries.
-//   grad_x: persistent CTAs walk (128 x 64 output tile, 32-deep chunk of P)
-//           pairs through a four-deep ring; 32 x 32 warp tiles.
-//   grad_W: a CTA per 128 x 64 output tile and range of rows (split K), 32 rows
-//           per stage, four-deep ring; 32 x 32 warp tiles.  grad_b rides on the same A
-//           fragments: one more MMA per step against a constant B whose first
-//           column is ones.  Partial tiles are added into fp32 accumulators
-//           with vector reductions; the last CTA to finish rounds them once.
+// Both products run on the fifth-generation tensor cores (tcgen05.mma,
+// fp16/bf16 operands read from shared memory by descriptor, fp32 accumulators
+// in tensor memory), fed by TMA in the 128-byte swizzled layout.  Each kernel
+// is warp-specialised: a TMA warp fills a ring of stages, an MMA warp consumes
+// them, four warps drain the accumulator.  The products are bound by HBM (g
+// and x read, grad_x written: 40-60 FLOP per byte, far below the tensor pipe's
+// ridge), so the ring is sized for bytes in flight, not for tensor throughput.
+//   grad_x: persistent CTAs walk 128 x 64 tiles of grad_x; the accumulator is
+//           double-buffered in tensor memory, so one tile's epilogue overlaps
+//           the next tile's MMAs.
+//   grad_W: a CTA per 128 x 64 tile of grad_W and range of rows (split K);
+//           grad_b rides on the same MMAs through a constant ones column of B.
+//           Partial tiles are added into fp32 accumulators with vector
+//           reductions; the last CTA of each tile rounds it once.
+#include <cuda.h>  // tensor-map types (the encoder is resolved at run time)
+
 #include <algorithm>
 #include <cstring>
 #include <type_traits>
@@ -25,43 +30,6 @@
 
 namespace dcn4 {
 namespace {
-
-constexpr int kLbThreads = 256;
-
-__device__ __forceinline__ void cp_async16(void* dst_smem, const void* src, bool valid) {
-    const unsigned da = static_cast<unsigned>(__cvta_generic_to_shared(dst_smem));
-    const int n = valid ? 16 : 0;  // 0 source bytes: the 16 bytes are zero-filled
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(da), "l"(src), "r"(n));
-}
-
-__device__ __forceinline__ void ldsm_x4(uint32_t* r, const void* p) {
-    const unsigned a = static_cast<unsigned>(__cvta_generic_to_shared(p));
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-                 : "r"(a));
-}
-__device__ __forceinline__ void ldsm_x4_t(uint32_t* r, const void* p) {
-    const unsigned a = static_cast<unsigned>(__cvta_generic_to_shared(p));
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-                 : "r"(a));
-}
-
-// d += a (16x16, row fragments) * b (16x8, column fragments), fp32 accumulation.
-template <typename T>
-__device__ __forceinline__ void mma16816(float* d, const uint32_t* a, const uint32_t* b) {
-    if constexpr (std::is_same<T, __half>::value) {
-        asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
-                     "{%0, %1, %2, %3};"
-                     : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-                     : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
-    } else {
-        asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
-                     "{%0, %1, %2, %3};"
-                     : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-                     : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
-    }
-}
 
 template <typename T>
 __device__ __forceinline__ uint32_t pack_pair(float lo, float hi) {
@@ -76,32 +44,26 @@ __device__ __forceinline__ uint32_t pack_pair(float lo, float hi) {
     return u;
 }
 
-constexpr int kPad = 8;  // padded smem rows (16 bytes): conflict-free ldmatrix
-
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
-
 // Rounds one 128 x 64 tile of the fp32 grad_W accumulator (and, for the first
 // column tile, its 128 grad_b entries) into the outputs: every load of a thread
 // is issued before the first store.
 template <typename T, int NT>
 __device__ __forceinline__ void round_tile(const float* wacc, const float* bacc, T* gw, T* gb, int P, int Cx, int p0,
                                            int c0, bool with_b) {
-    constexpr int kVec = 128 * 64 / 4 / NT;  // float4 groups per thread
+    constexpr int kGroups = 128 * 64 / 4, kVec = (kGroups + NT - 1) / NT;  // float4 groups: per tile, per thread
     if (gw) {
         float4 v[kVec];
 #pragma unroll
         for (int u = 0; u < kVec; ++u) {
             const int e = threadIdx.x + u * NT, r = e >> 4, c = (e & 15) * 4;
             v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (p0 + r < P && c0 + c < Cx)
+            if (e < kGroups && p0 + r < P && c0 + c < Cx)
                 v[u] = __ldcg(reinterpret_cast<const float4*>(wacc + static_cast<long long>(p0 + r) * Cx + c0 + c));
         }
 #pragma unroll
         for (int u = 0; u < kVec; ++u) {
             const int e = threadIdx.x + u * NT, r = e >> 4, c = (e & 15) * 4;
-            if (p0 + r < P && c0 + c < Cx)
+            if (e < kGroups && p0 + r < P && c0 + c < Cx)
                 *reinterpret_cast<uint2*>(gw + static_cast<long long>(p0 + r) * Cx + c0 + c) =
                     make_uint2(pack_pair<T>(v[u].x, v[u].y), pack_pair<T>(v[u].z, v[u].w));
         }
@@ -112,264 +74,10 @@ __device__ __forceinline__ void round_tile(const float* wacc, const float* bacc,
 }
 
 // ---------------------------------------------------------------------------
-// grad_x = g W: A = g [M, P] (row-major, k = p), B = W [P, Cx] (k-major rows).
+// tcgen05 building blocks: shared-memory matrix and instruction descriptors,
+// the MMA, its commit to an mbarrier, tensor-memory loads, bounded waits.
 // ---------------------------------------------------------------------------
-constexpr int kXM = 128, kXN = 64, kXK = 32, kXStages = 4;
-template <typename T>
-struct XStage {
-    T a[kXM][kXK + kPad];
-    T b[kXK][kXN + kPad];
-};
-
-template <typename T>
-__global__ void __launch_bounds__(kLbThreads, 3)
-    linear_grad_x_kernel(const T* __restrict__ g, const T* __restrict__ w, T* __restrict__ gx, long long M, int P,
-                         int Cx, long long ntiles, int ntiles_n, int nk) {
-    extern __shared__ __align__(16) unsigned char lin_smem[];
-    XStage<T>* st = reinterpret_cast<XStage<T>*>(lin_smem);
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int wm = warp >> 1, wn = warp & 1;  // 4 x 2 warps of 32 x 32
-    constexpr int EPV = 8;                    // 16-bit elements per 16-byte chunk
-    if (static_cast<long long>(blockIdx.x) >= ntiles) return;
-    // this thread's 16-byte chunks: A rows ar and ar + 64 at column ac; B row br at column bc
-    const int ar = threadIdx.x / (kXK / EPV), ac = (threadIdx.x % (kXK / EPV)) * EPV;
-    const int br = threadIdx.x / (kXN / EPV), bc = (threadIdx.x % (kXN / EPV)) * EPV;
-    static_assert(kXM * (kXK / EPV) == 2 * kLbThreads && kXK * (kXN / EPV) == kLbThreads, "chunk split");
-
-    // (tile, chunk) walk of the loads, kXStages - 1 ahead of the compute walk
-    long long ld_tile = blockIdx.x;
-    int ld_kc = 0;
-    auto load = [&](int slot) {
-        const long long tm = ld_tile / ntiles_n;
-        const int n0 = static_cast<int>(ld_tile - tm * ntiles_n) * kXN;
-        const long long m0 = tm * kXM;
-        const int k0 = ld_kc * kXK;
-        XStage<T>& s = st[slot];
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-            const int r = ar + (kXM / 2) * i;
-            const long long m = m0 + r;
-            const bool ok = m < M && k0 + ac < P;
-            cp_async16(&s.a[r][ac], g + (ok ? m * P + k0 + ac : 0), ok);
-        }
-        const bool okb = k0 + br < P && n0 + bc < Cx;
-        cp_async16(&s.b[br][bc], w + (okb ? static_cast<long long>(k0 + br) * Cx + n0 + bc : 0), okb);
-        if (++ld_kc == nk) {
-            ld_kc = 0;
-            ld_tile += gridDim.x;
-        }
-    };
-
-    float acc[2][4][4] = {};
-    for (int j = 0; j < kXStages - 1; ++j) {
-        if (ld_tile < ntiles) load(j);
-        cp_async_commit();
-    }
-    long long tile = blockIdx.x;
-    int kc = 0, slot = 0;
-    while (tile < ntiles) {
-        cp_async_wait<kXStages - 2>();
-        __syncthreads();  // this slot landed for every thread; the slot used last is free again
-        if (ld_tile < ntiles) load(slot == 0 ? kXStages - 1 : slot - 1);
-        cp_async_commit();
-        const XStage<T>& s = st[slot];
-#pragma unroll
-        for (int ks = 0; ks < kXK / 16; ++ks) {
-            uint32_t a[2][4], b[4][2];
-#pragma unroll
-            for (int mt = 0; mt < 2; ++mt)
-                ldsm_x4(a[mt], &s.a[wm * 32 + mt * 16 + (lane & 15)][ks * 16 + (lane >> 4) * 8]);
-#pragma unroll
-            for (int np = 0; np < 2; ++np) {
-                // two n8 tiles per x4.trans: lanes 0-15 address the k rows of tile 2np, lanes 16-31 of 2np+1
-                uint32_t r[4];
-                ldsm_x4_t(r, &s.b[ks * 16 + (lane & 15)][wn * 32 + np * 16 + (lane >> 4) * 8]);
-                b[2 * np][0] = r[0];
-                b[2 * np][1] = r[1];
-                b[2 * np + 1][0] = r[2];
-                b[2 * np + 1][1] = r[3];
-            }
-#pragma unroll
-            for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-                for (int nt = 0; nt < 4; ++nt) mma16816<T>(acc[mt][nt], a[mt], b[nt]);
-        }
-        slot = slot + 1 == kXStages ? 0 : slot + 1;
-        if (++kc == nk) {  // last chunk of this tile: round once and store
-            const long long tm = tile / ntiles_n;
-            const int n0 = static_cast<int>(tile - tm * ntiles_n) * kXN;
-            const int gq = lane >> 2, tq = lane & 3;
-#pragma unroll
-            for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-                for (int nt = 0; nt < 4; ++nt) {
-                    const int col = n0 + wn * 32 + nt * 8 + tq * 2;
-                    const long long r0 = tm * kXM + wm * 32 + mt * 16 + gq, r1 = r0 + 8;
-                    if (col < Cx) {
-                        if (r0 < M)
-                            *reinterpret_cast<uint32_t*>(gx + r0 * Cx + col) = pack_pair<T>(acc[mt][nt][0], acc[mt][nt][1]);
-                        if (r1 < M)
-                            *reinterpret_cast<uint32_t*>(gx + r1 * Cx + col) = pack_pair<T>(acc[mt][nt][2], acc[mt][nt][3]);
-                    }
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) acc[mt][nt][e] = 0.f;
-                }
-            kc = 0;
-            tile += gridDim.x;
-        }
-    }
-    cp_async_wait<0>();
-}
-
-// ---------------------------------------------------------------------------
-// grad_W += g^T x over a range of rows: A = g^T (from g [m][p] with
-// ldmatrix.trans), B = x [m][c] (k = m).  grad_b from the same A fragments.
-// ---------------------------------------------------------------------------
-constexpr int kWP = 128, kWC = 64, kWK = 32, kWStages = 4;
-template <typename T>
-struct WStage {
-    T g[kWK][kWP + kPad];  // [m][p]
-    T x[kWK][kWC + kPad];  // [m][c]
-};
-
-__device__ __forceinline__ void red_add2(float* dst, float a, float b) {
-    asm volatile("red.global.add.v2.f32 [%0], {%1, %2};" ::"l"(dst), "f"(a), "f"(b) : "memory");
-}
-
-template <typename T>
-__global__ void __launch_bounds__(kLbThreads, 3)
-    linear_grad_w_kernel(const T* __restrict__ g, const T* __restrict__ x, float* __restrict__ wacc,
-                         float* __restrict__ bacc, unsigned* __restrict__ done, T* __restrict__ gw,
-                         T* __restrict__ gb, long long M, int P, int Cx, int ntile, int ct, long long mchunk) {
-    extern __shared__ __align__(16) unsigned char lin_smem[];
-    WStage<T>* st = reinterpret_cast<WStage<T>*>(lin_smem);
-    __shared__ unsigned ticket;
-    const int tile = blockIdx.x % ntile;  // ntile = (P tiles) x (Cx tiles); blocks of one split run together
-    const long long split = blockIdx.x / ntile;
-    const int tp = tile / ct, tc = tile - tp * ct;
-    const int p0 = tp * kWP, c0 = tc * kWC;
-    const long long mb = split * mchunk;
-    const long long me = std::min<long long>(M, mb + mchunk);
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int wp = warp >> 1, wc = warp & 1;  // 4 x 2 warps of 32 (p) x 32 (c)
-    constexpr int EPV = 8;
-    const bool sum_b = bacc != nullptr && tc == 0 && wc == 0;
-    const int nk = static_cast<int>((me - mb + kWK - 1) / kWK);
-    // this thread's 16-byte chunks: g rows gr and gr + 16 at column gc; x row xr at column xc
-    const int gr = threadIdx.x / (kWP / EPV), gc = (threadIdx.x % (kWP / EPV)) * EPV;
-    const int xr = threadIdx.x / (kWC / EPV), xc = (threadIdx.x % (kWC / EPV)) * EPV;
-    static_assert(kWK * (kWP / EPV) == 2 * kLbThreads && kWK * (kWC / EPV) == kLbThreads, "chunk split");
-    const bool gcol_ok = p0 + gc < P, xcol_ok = c0 + xc < Cx;
-
-    auto load = [&](int j, int slot) {
-        const long long m = mb + static_cast<long long>(j) * kWK;
-        WStage<T>& s = st[slot];
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-            const int r = gr + (kWK / 2) * i;
-            const long long mm = m + r;
-            const bool ok = mm < me && gcol_ok;
-            cp_async16(&s.g[r][gc], g + (ok ? mm * P + p0 + gc : 0), ok);
-        }
-        const long long mm = m + xr;
-        const bool ok = mm < me && xcol_ok;
-        cp_async16(&s.x[xr][xc], x + (ok ? mm * Cx + c0 + xc : 0), ok);
-    };
-
-    // B operand whose first column is ones: A * ones_b puts the row sums of A in column 0
-    const int gq = lane >> 2, tq = lane & 3;
-    const uint32_t one2 = gq == 0 ? pack_pair<T>(1.f, 1.f) : 0u;
-    const uint32_t ones_b[2] = {one2, one2};
-
-    float acc[2][4][4] = {};
-    float accb[2][4] = {};
-    for (int j = 0; j < kWStages - 1; ++j) {
-        if (j < nk) load(j, j);
-        cp_async_commit();
-    }
-    int slot = 0;
-    for (int j = 0; j < nk; ++j) {
-        cp_async_wait<kWStages - 2>();
-        __syncthreads();
-        if (j + kWStages - 1 < nk) load(j + kWStages - 1, slot == 0 ? kWStages - 1 : slot - 1);
-        cp_async_commit();
-        const WStage<T>& s = st[slot];
-        slot = slot + 1 == kWStages ? 0 : slot + 1;
-#pragma unroll
-        for (int ks = 0; ks < kWK / 16; ++ks) {
-            uint32_t a[2][4], b[4][2];
-#pragma unroll
-            for (int mt = 0; mt < 2; ++mt) {
-                // A[p][m] = g[m][p]: submatrices (p 0-7, m 0-7), (p 8-15, m 0-7), (p 0-7, m 8-15), (p 8-15, m 8-15)
-                const int mrow = ks * 16 + (lane & 7) + ((lane >> 4) << 3);
-                const int pcol = wp * 32 + mt * 16 + (((lane >> 3) & 1) << 3);
-                ldsm_x4_t(a[mt], &s.g[mrow][pcol]);
-            }
-#pragma unroll
-            for (int np = 0; np < 2; ++np) {
-                uint32_t r[4];
-                ldsm_x4_t(r, &s.x[ks * 16 + (lane & 15)][wc * 32 + np * 16 + (lane >> 4) * 8]);
-                b[2 * np][0] = r[0];
-                b[2 * np][1] = r[1];
-                b[2 * np + 1][0] = r[2];
-                b[2 * np + 1][1] = r[3];
-            }
-#pragma unroll
-            for (int mt = 0; mt < 2; ++mt) {
-#pragma unroll
-                for (int nt = 0; nt < 4; ++nt) mma16816<T>(acc[mt][nt], a[mt], b[nt]);
-                if (sum_b) mma16816<T>(accb[mt], a[mt], ones_b);
-            }
-        }
-    }
-    cp_async_wait<0>();
-
-#pragma unroll
-    for (int mt = 0; mt < 2; ++mt) {
-        const int r0 = p0 + wp * 32 + mt * 16 + gq, r1 = r0 + 8;
-#pragma unroll
-        for (int nt = 0; nt < 4; ++nt) {
-            const int col = c0 + wc * 32 + nt * 8 + tq * 2;
-            if (col >= Cx) continue;
-            if (r0 < P) red_add2(wacc + static_cast<long long>(r0) * Cx + col, acc[mt][nt][0], acc[mt][nt][1]);
-            if (r1 < P) red_add2(wacc + static_cast<long long>(r1) * Cx + col, acc[mt][nt][2], acc[mt][nt][3]);
-        }
-        if (sum_b && tq == 0) {  // column 0 of the ones product: rows r0 and r1
-            if (r0 < P) atomicAdd(bacc + r0, accb[mt][0]);
-            if (r1 < P) atomicAdd(bacc + r1, accb[mt][2]);
-        }
-    }
-
-    // The last CTA of this output tile rounds it once (its fence orders the other
-    // CTAs' reductions, which precede their tickets, before its reads).
-    __threadfence();
-    __syncthreads();
-    if (threadIdx.x == 0) ticket = atomicAdd(done + tile, 1u);
-    __syncthreads();
-    if (ticket != gridDim.x / ntile - 1) return;
-    __threadfence();
-    round_tile<T, kLbThreads>(wacc, bacc, gw, gb, P, Cx, p0, c0, tc == 0);
-}
-
-// ---------------------------------------------------------------------------
-// grad_x = g W on the fifth-generation tensor cores (tcgen05).  One thread
-// issues the MMAs (M = 128 rows of g, N = 64 columns of grad_x, K = 16 each),
-// operands read from shared memory by descriptor, the fp32 accumulator in
-// tensor memory; the CTA's 128 threads stage the operands and read the
-// accumulator back.  Operands use the no-swizzle canonical layouts, 8 x 8
-// core matrices of 128 bytes (8 rows of 16 bytes):
-//   A = g  (K-major): element (m, k) at (m/8)*512 + (k/8)*128 + (m%8)*16 + (k%8)*2
-//   B = W  (N-major): element (k, n) at (k/8)*1024 + (n/8)*128 + (k%8)*16 + (n%8)*2
-// The ring has kTStages slots of 32 rows of K, loaded kTDepth ahead: a slot is
-// refilled two iterations after the MMAs that read it were issued, so the
-// loads never wait on the tensor cores' latency.
-// ---------------------------------------------------------------------------
-constexpr int kTM = 128, kTN = 64, kTK = 32, kTStages = 6, kTDepth = 4, kTThreads = 128;
-constexpr int kTABytes = kTM * kTK * 2;               // 8 KB
-constexpr int kTBBytes = kTK * kTN * 2;               // 4 KB
-constexpr int kTStageBytes = kTABytes + kTBBytes;     // 12 KB
-constexpr int kTSlack = 16 * 1024;                    // guard band after the ring
-constexpr int kTSmem = kTStages * kTStageBytes + kTSlack;
+constexpr int kTM = 128, kTN = 64;  // grad_x tile: 128 rows of g x 64 columns
 constexpr int kTWaitSpins = 1 << 22;                  // bound of every mbarrier wait
 constexpr unsigned kLinStatusTimeout = 1u;            // a wait gave up (status word)
 
@@ -377,12 +85,8 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
-__device__ __forceinline__ void cp_async16_s(uint32_t dst, const void* src, bool valid) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0));
-}
-
 // Shared-memory matrix descriptor: start address, leading and stride byte
-// offsets (all in 16-byte units), descriptor version 1, no swizzle.
+// offsets (all in 16-byte units), descriptor version 1; layout type in bits 61-63.
 __device__ __forceinline__ uint64_t umma_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
     return static_cast<uint64_t>((saddr >> 4) & 0x3FFFu) | (static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16) |
            (static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46);
@@ -412,21 +116,6 @@ __device__ __forceinline__ void umma_commit(uint32_t mbar) {
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
-// Waits (bounded) for the completion of the phase of parity `parity`; false if it gave up.
-__device__ __forceinline__ bool mbar_wait(uint32_t mbar, uint32_t parity) {
-    for (int i = 0; i < kTWaitSpins; ++i) {
-        uint32_t done;
-        asm volatile(
-            "{\n\t.reg .pred P1;\n\tmbarrier.try_wait.parity.shared::cta.b64 P1, [%1], %2;\n\t"
-            "selp.b32 %0, 1, 0, P1;\n\t}"
-            : "=r"(done)
-            : "r"(mbar), "r"(parity)
-            : "memory");
-        if (done) return true;
-    }
-    return false;
-}
-
 // 32 consecutive fp32 accumulator columns of this thread's TMEM lane.
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t* r) {
     asm volatile(
@@ -440,164 +129,227 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t* r) {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// ---------------------------------------------------------------------------
+// tcgen05 products fed by TMA, warp-specialised.  Warp 4 (one lane) loads the
+// stages with TMA, warp 5 (one lane) issues the MMAs, warps 0-3 read the
+// accumulator back (warp w owns TMEM lanes 32w..32w+31).  Operands use the
+// 128-byte swizzled layout: a TMA box 64 elements (128 bytes) wide with
+// SWIZZLE_128B lands rows of 128 bytes whose 16-byte chunks are permuted by the
+// row index within each 8-row, 1024-byte atom -- the permutation the
+// descriptor's SWIZZLE_128B mode undoes.  (Boxes 16 bytes wide in the
+// no-swizzle layout were tried first: every row became its own 16-byte
+// request, and grad_x took 51 us instead of 19.)
+//   K-major operand, 64-wide K slab:  row r at r*128, SBO 1024 (8 rows); the
+//       16-wide K step of an MMA moves the start address by 32 bytes.
+//   M/N-major operand, 64-wide M/N block: K row k at k*128, SBO 1024 (8 K rows),
+//       LBO = distance between 64-wide blocks; the MMA's K step moves 2048 bytes.
+// Full / empty barriers per stage, full / empty barriers per accumulator; every
+// wait is bounded and gives up at once when another role has given up.
+// ---------------------------------------------------------------------------
+constexpr int kQThreads = 192;  // 4 epilogue warps, the TMA warp, the MMA warp
+constexpr int kQProducer = 4, kQMma = 5;
+
+__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    return umma_desc(saddr, lbo, sbo) | (2ull << 61);  // layout type SWIZZLE_128B
+}
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t mbar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+            dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(mbar)
+        : "memory");
+}
+__device__ __forceinline__ void mbar_init(uint32_t mbar, int count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(mbar), "r"(count));
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t mbar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(mbar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t mbar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(mbar) : "memory");
+}
+// Bounded wait for the phase of parity `parity`; stops early once *abort is set.
+__device__ __forceinline__ bool mbar_wait_or(uint32_t mbar, uint32_t parity, volatile int* abort) {
+    for (int i = 0; i < kTWaitSpins; ++i) {
+        uint32_t done;
+        asm volatile(
+            "{\n\t.reg .pred P1;\n\tmbarrier.try_wait.parity.shared::cta.b64 P1, [%1], %2;\n\t"
+            "selp.b32 %0, 1, 0, P1;\n\t}"
+            : "=r"(done)
+            : "r"(mbar), "r"(parity)
+            : "memory");
+        if (done) return true;
+        if ((i & 63) == 63 && *abort) return false;
+    }
+    *abort = 1;
+    return false;
+}
+
+__device__ __forceinline__ void red_add4(float* dst, float a, float b, float c, float d) {
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(a), "f"(b), "f"(c), "f"(d) : "memory");
+}
+
+constexpr int kUM = 128, kUN = 64, kUTmemCols = 128;  // grad_W tile: 128 rows of W x 64 columns (80 with grad_b)
+
+// grad_x = g W: persistent CTAs walk 128 x 64 tiles of grad_x; stages of a 64
+// column slab of g (one box of 128 rows) and 64 rows of W (one box 64 wide);
+// the accumulator is double-buffered in tensor memory so the epilogue of one
+// tile overlaps the MMAs of the next.
+constexpr int kQXK = 64, kQXStages = 4;
+constexpr int kQXABytes = kTM * kQXK * 2;             // 16 KB
+constexpr int kQXBBytes = kQXK * kTN * 2;             // 8 KB
+constexpr int kQXStage = kQXABytes + kQXBBytes;
+constexpr int kQXSmem = kQXStages * kQXStage + 1024;
+
 template <typename T>
-__global__ void __launch_bounds__(kTThreads, 2)
-    linear_grad_x_tc_kernel(const T* __restrict__ g, const T* __restrict__ w, T* __restrict__ gx, long long M, int P,
-                            int Cx, long long ntiles, int ntiles_n, int nk, unsigned* __restrict__ status) {
+__global__ void __launch_bounds__(kQThreads, 2)
+    linear_grad_x_tma_kernel(const __grid_constant__ CUtensorMap map_g, const __grid_constant__ CUtensorMap map_w,
+                             T* __restrict__ gx, long long M, int Cx, long long ntiles, int ntiles_n, int nk,
+                             unsigned* __restrict__ status) {
     extern __shared__ __align__(1024) unsigned char tc_smem[];
-    __shared__ __align__(8) uint64_t mbar[kTStages];
+    __shared__ __align__(8) uint64_t full[kQXStages], empty[kQXStages], acc_full[2], acc_empty[2];
     __shared__ uint32_t taddr_s;
-    if (static_cast<long long>(blockIdx.x) >= ntiles) return;  // whole CTA, before anything is held
+    __shared__ int s_abort;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const uint32_t ring = smem_u32(tc_smem);
+    const uint32_t ring = (smem_u32(tc_smem) + 1023u) & ~1023u;
     if (tid == 0) {
-        for (int s = 0; s < kTStages; ++s) asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&mbar[s])));
+        for (int s = 0; s < kQXStages; ++s) {
+            mbar_init(smem_u32(&full[s]), 1);
+            mbar_init(smem_u32(&empty[s]), 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(smem_u32(&acc_full[a]), 1);
+            mbar_init(smem_u32(&acc_empty[a]), 4);
+        }
+        s_abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    if (warp == 0) {  // 64 fp32 columns x 128 lanes of tensor memory: the accumulator
+    if (warp == kQMma) {  // two 64-column fp32 accumulators x 128 lanes
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&taddr_s)),
-                     "r"(kTN));
+                     "r"(2 * kTN));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = taddr_s;
-    constexpr uint32_t idesc = umma_idesc<T>(kTM, kTN, 0, 1);
+    volatile int* abort = &s_abort;
+    const long long my_tiles =
+        static_cast<long long>(blockIdx.x) < ntiles ? (ntiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
 
-    // (tile, chunk) walk of the loads, kTStages - 1 ahead of the MMAs
-    long long ld_tile = blockIdx.x;
-    int ld_kc = 0;
-    auto load = [&](int slot) {
-        const long long tm = ld_tile / ntiles_n;
-        const int n0 = static_cast<int>(ld_tile - tm * ntiles_n) * kTN;
-        const long long m0 = tm * kTM;
-        const int k0 = ld_kc * kTK;
-        const uint32_t sa = ring + slot * kTStageBytes, sb = sa + kTABytes;
+    if (warp == kQProducer) {
+        if (lane == 0) {
+            long long it = 0;
+            for (long long lt = 0; lt < my_tiles && !*abort; ++lt) {
+                const long long tile = blockIdx.x + lt * gridDim.x;
+                const long long tm = tile / ntiles_n;
+                const int n0 = static_cast<int>(tile - tm * ntiles_n) * kTN;
+                const int m0 = static_cast<int>(tm * kTM);
+                for (int kc = 0; kc < nk; ++kc, ++it) {
+                    const int s = static_cast<int>(it % kQXStages);
+                    const uint32_t ph = static_cast<uint32_t>(it / kQXStages) & 1u;
+                    if (!mbar_wait_or(smem_u32(&empty[s]), ph ^ 1u, abort)) break;
+                    const uint32_t fb = smem_u32(&full[s]);
+                    mbar_expect_tx(fb, kQXStage);
+                    const uint32_t sa = ring + s * kQXStage, sb = sa + kQXABytes;
+                    const int k0 = kc * kQXK;
+                    tma_load_2d(sa, &map_g, k0, m0, fb);
+                    tma_load_2d(sb, &map_w, n0, k0, fb);
+                }
+            }
+        }
+    } else if (warp == kQMma) {
+        if (lane == 0) {
+            constexpr uint32_t idesc = umma_idesc<T>(kTM, kTN, 0, 1);
+            long long it = 0;
+            for (long long lt = 0; lt < my_tiles && !*abort; ++lt) {
+                const int a = static_cast<int>(lt & 1);
+                const uint32_t aph = static_cast<uint32_t>(lt >> 1) & 1u;
+                if (!mbar_wait_or(smem_u32(&acc_empty[a]), aph ^ 1u, abort)) break;
+                tc_fence_after();
+                const uint32_t d = tmem + a * kTN;
+                bool ok = true;
+                for (int kc = 0; kc < nk; ++kc, ++it) {
+                    const int s = static_cast<int>(it % kQXStages);
+                    const uint32_t ph = static_cast<uint32_t>(it / kQXStages) & 1u;
+                    if (!mbar_wait_or(smem_u32(&full[s]), ph, abort)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t sa = ring + s * kQXStage, sb = sa + kQXABytes;
 #pragma unroll
-        for (int u = 0; u < kTM * (kTK / 8) / kTThreads; ++u) {  // A: 128 rows x 4 chunks of 16 bytes
-            const int i = tid + u * kTThreads, m = i >> 2, kg = i & 3;
-            const bool ok = m0 + m < M && k0 + kg * 8 < P;
-            cp_async16_s(sa + (m >> 3) * 512 + kg * 128 + (m & 7) * 16, g + (ok ? (m0 + m) * P + k0 + kg * 8 : 0), ok);
+                    for (int q = 0; q < kQXK / 16; ++q)  // A: 32 bytes along its rows; B: 16 rows of 128 bytes
+                        umma_f16(d, umma_desc_sw128(sa + q * 32, 16, 1024), umma_desc_sw128(sb + q * 2048, kQXBBytes, 1024),
+                                 idesc, kc > 0 || q > 0);
+                    umma_commit(smem_u32(&empty[s]));  // the stage may be refilled once these MMAs are done
+                }
+                if (!ok) break;
+                umma_commit(smem_u32(&acc_full[a]));
+            }
         }
-#pragma unroll
-        for (int u = 0; u < kTK * (kTN / 8) / kTThreads; ++u) {  // B: 32 rows x 8 chunks
-            const int i = tid + u * kTThreads, k = i >> 3, ng = i & 7;
-            const bool ok = k0 + k < P && n0 + ng * 8 < Cx;
-            cp_async16_s(sb + (k >> 3) * 1024 + ng * 128 + (k & 7) * 16,
-                         w + (ok ? static_cast<long long>(k0 + k) * Cx + n0 + ng * 8 : 0), ok);
-        }
-        if (++ld_kc == nk) {
-            ld_kc = 0;
-            ld_tile += gridDim.x;
-        }
-    };
-
-    uint32_t phase = 0, pending = 0;  // per slot: parity of its next completion; a commit not yet waited for
-    int aborted = 0;                  // this thread gave up a wait; the CTA stops at the next barrier
-    auto wait_slot = [&](int s) {
-        if (!((pending >> s) & 1u)) return;
-        if (!mbar_wait(smem_u32(&mbar[s]), (phase >> s) & 1u)) aborted = 1;
-        phase ^= 1u << s;
-        pending &= ~(1u << s);
-    };
-
-    for (int j = 0; j < kTDepth; ++j) {
-        if (ld_tile < ntiles) load(j);
-        cp_async_commit();
-    }
-    long long tile = blockIdx.x;
-    int kc = 0, slot = 0, ld_slot = kTDepth;
-    while (tile < ntiles) {
-        wait_slot(ld_slot);  // the MMAs that last read ld_slot (two iterations ago) are done
-        if (ld_tile < ntiles) load(ld_slot);
-        cp_async_commit();
-        ld_slot = ld_slot + 1 == kTStages ? 0 : ld_slot + 1;
-        cp_async_wait<kTDepth>();                   // this thread's copies of `slot` landed
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // ... and are visible to the tensor cores
-        if (__syncthreads_or(aborted)) break;
-        if (tid == 0) {
+    } else {  // warps 0-3: read the accumulator back, round once, store
+        for (long long lt = 0; lt < my_tiles; ++lt) {
+            const int a = static_cast<int>(lt & 1);
+            const uint32_t aph = static_cast<uint32_t>(lt >> 1) & 1u;
+            if (!mbar_wait_or(smem_u32(&acc_full[a]), aph, abort)) break;
             tc_fence_after();
-            const uint32_t sa = ring + slot * kTStageBytes, sb = sa + kTABytes;
-#pragma unroll
-            for (int q = 0; q < kTK / 16; ++q)  // K = 16 per MMA: two core matrices of A, two rows of B's
-                umma_f16(tmem, umma_desc(sa + q * 256, 128, 512), umma_desc(sb + q * 2048, 1024, 128), idesc,
-                         kc > 0 || q > 0);
-            umma_commit(smem_u32(&mbar[slot]));
-        }
-        pending |= 1u << slot;
-        const int done_slot = slot;
-        slot = slot + 1 == kTStages ? 0 : slot + 1;
-        if (++kc == nk) {  // the tile's accumulator is complete: read it back, round once, store
-            wait_slot(done_slot);
-            tc_fence_after();
+            const long long tile = blockIdx.x + lt * gridDim.x;
             const long long tm = tile / ntiles_n;
             const int n0 = static_cast<int>(tile - tm * ntiles_n) * kTN;
             const long long row = tm * kTM + warp * 32 + lane;
-            const uint32_t lane_addr = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+            const uint32_t lane_addr = tmem + a * kTN + (static_cast<uint32_t>(warp * 32) << 16);
+            uint32_t r[2][32];
+            tmem_ld32(lane_addr, r[0]);
+            tmem_ld32(lane_addr + 32, r[1]);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&acc_empty[a]));  // the MMA warp may reuse this accumulator
+            if (row < M) {
 #pragma unroll
-            for (int h = 0; h < kTN / 32; ++h) {
-                uint32_t r[32];
-                tmem_ld32(lane_addr + h * 32, r);
-                if (row < M && !aborted) {
+                for (int h = 0; h < 2; ++h)
 #pragma unroll
                     for (int v = 0; v < 4; ++v) {
                         const int col = n0 + h * 32 + v * 8;
                         if (col >= Cx) continue;
                         uint4 o;
-                        o.x = pack_pair<T>(__uint_as_float(r[8 * v + 0]), __uint_as_float(r[8 * v + 1]));
-                        o.y = pack_pair<T>(__uint_as_float(r[8 * v + 2]), __uint_as_float(r[8 * v + 3]));
-                        o.z = pack_pair<T>(__uint_as_float(r[8 * v + 4]), __uint_as_float(r[8 * v + 5]));
-                        o.w = pack_pair<T>(__uint_as_float(r[8 * v + 6]), __uint_as_float(r[8 * v + 7]));
+                        o.x = pack_pair<T>(__uint_as_float(r[h][8 * v + 0]), __uint_as_float(r[h][8 * v + 1]));
+                        o.y = pack_pair<T>(__uint_as_float(r[h][8 * v + 2]), __uint_as_float(r[h][8 * v + 3]));
+                        o.z = pack_pair<T>(__uint_as_float(r[h][8 * v + 4]), __uint_as_float(r[h][8 * v + 5]));
+                        o.w = pack_pair<T>(__uint_as_float(r[h][8 * v + 6]), __uint_as_float(r[h][8 * v + 7]));
                         *reinterpret_cast<uint4*>(gx + row * Cx + col) = o;
                     }
-                }
             }
-            tc_fence_before();  // the next tile's first MMA overwrites the accumulator after the next barrier
-            kc = 0;
-            tile += gridDim.x;
         }
     }
-    cp_async_wait<0>();
-    for (int s = 0; s < kTStages; ++s) wait_slot(s);  // no MMA may still read shared or tensor memory
-    if (aborted) atomicOr(status, kLinStatusTimeout);
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTN));
+    if (tid == 0 && *abort) atomicOr(status, kLinStatusTimeout);
+    if (warp == kQMma) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(2 * kTN));
 }
 
-// ---------------------------------------------------------------------------
-// grad_W += g^T x and grad_b on tcgen05 over one range of rows (split K):
-// D [128 rows of W^T's rows p, 80 columns] in tensor memory, K = rows m of g
-// and x, 64 per stage.  A = g^T is M-major straight from g's rows (p
-// contiguous); B = x is N-major (c contiguous) with two extra column groups
-// set once: column 64 all ones, 65-79 zero, so D's column 64 sums g's columns
-// (grad_b) with the same MMAs.
-//   A: element (p, m) at (m/8)*2048 + (p/8)*128 + (m%8)*16 + (p%8)*2
-//   B: element (m, c) at (m/8)*1280 + (c/8)*128 + (m%8)*16 + (c%8)*2
-// Ring of kUStages slots of 32 rows, loaded kUDepth ahead (as for grad_x).
-// ---------------------------------------------------------------------------
-constexpr int kUM = 128, kUN = 64, kUNB = 80, kUK = 32, kUStages = 6, kUDepth = 4;
-constexpr int kUABytes = kUK * kUM * 2;               // 8 KB
-constexpr int kUBBytes = kUK * kUNB * 2;              // 5 KB
-constexpr int kUStageBytes = kUABytes + kUBBytes;     // 13 KB
-constexpr int kUSlack = 24 * 1024;
-constexpr int kUSmem = kUStages * kUStageBytes + kUSlack;
-constexpr int kUTmemCols = 128;                       // 80 used
-
-__device__ __forceinline__ void red_add4(float* dst, float a, float b, float c, float d) {
-    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(a), "f"(b), "f"(c), "f"(d) : "memory");
-}
+// grad_W += g^T x and grad_b over one range of rows (split K): a CTA per
+// 128 x 64 tile of grad_W and range; stages of 32 rows m: g^T (M-major) as two
+// 64-wide boxes, x (N-major) as one, plus a constant second block of B (its
+// first column all ones, the rest zero) so that D's column 64 sums g's columns
+// (grad_b).  One accumulator of 80 columns.
+constexpr int kQWK = 32, kQWStages = 6, kQWNB = 80;
+constexpr int kQWABytes = kQWK * kUM * 2;             // 8 KB: two 64-wide blocks of 32 rows
+constexpr int kQWBBytes = 2 * kQWK * 64 * 2;          // 8 KB: x's block and the constant block
+constexpr int kQWStage = kQWABytes + kQWBBytes;
+constexpr int kQWLoad = kQWABytes + kQWK * kUN * 2;   // bytes TMA writes per stage
+constexpr int kQWSmem = kQWStages * kQWStage + 1024;
 
 template <typename T>
-__global__ void __launch_bounds__(kTThreads, 2)
-    linear_grad_w_tc_kernel(const T* __restrict__ g, const T* __restrict__ x, float* __restrict__ wacc,
-                            float* __restrict__ bacc, unsigned* __restrict__ done, unsigned* __restrict__ status,
-                            T* __restrict__ gw, T* __restrict__ gb, long long M, int P, int Cx, int ntile, int ct,
-                            long long mchunk) {
+__global__ void __launch_bounds__(kQThreads, 2)
+    linear_grad_w_tma_kernel(const __grid_constant__ CUtensorMap map_g, const __grid_constant__ CUtensorMap map_x,
+                             float* __restrict__ wacc, float* __restrict__ bacc, unsigned* __restrict__ done,
+                             unsigned* __restrict__ status, T* __restrict__ gw, T* __restrict__ gb, long long M, int P,
+                             int Cx, int ntile, int ct, long long mchunk) {
     extern __shared__ __align__(1024) unsigned char tc_smem[];
-    __shared__ __align__(8) uint64_t mbar[kUStages];
+    __shared__ __align__(8) uint64_t full[kQWStages], empty[kQWStages], acc_full;
     __shared__ uint32_t taddr_s;
+    __shared__ int s_abort;
     __shared__ unsigned ticket;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int tile = blockIdx.x % ntile;  // blocks of one split (the same rows) run together
@@ -606,116 +358,106 @@ __global__ void __launch_bounds__(kTThreads, 2)
     const int p0 = tp * kUM, c0 = tc * kUN;
     const long long mb = split * mchunk;
     const long long me = std::min<long long>(M, mb + mchunk);
-    const int nk = static_cast<int>((me - mb + kUK - 1) / kUK);
-    const uint32_t ring = smem_u32(tc_smem);
+    const int nk = static_cast<int>((me - mb + kQWK - 1) / kQWK);
+    const uint32_t ring_off = ((smem_u32(tc_smem) + 1023u) & ~1023u) - smem_u32(tc_smem);
+    const uint32_t ring = smem_u32(tc_smem) + ring_off;
     if (tid == 0) {
-        for (int s = 0; s < kUStages; ++s) asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&mbar[s])));
+        for (int s = 0; s < kQWStages; ++s) {
+            mbar_init(smem_u32(&full[s]), 1);
+            mbar_init(smem_u32(&empty[s]), 1);
+        }
+        mbar_init(smem_u32(&acc_full), 1);
+        s_abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    if (warp == 0) {
+    if (warp == kQMma) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&taddr_s)),
                      "r"(kUTmemCols));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
     }
-    // the constant column groups of B (8: ones in column 64, 9: zeros), in every stage
-    for (int i = tid; i < kUStages * kUK * 2; i += kTThreads) {
-        const int s = i / (kUK * 2), r = i - s * (kUK * 2), m = r >> 1, grp = 8 + (r & 1);
-        unsigned char* dst = tc_smem + s * kUStageBytes + kUABytes + (m >> 3) * 1280 + grp * 128 + (m & 7) * 16;
+    // B's constant block in every stage: row m holds a one in its first column, zeros elsewhere; under
+    // the 128-byte swizzle the first 16-byte chunk of row m sits at chunk (m mod 8)
+    for (int i = tid; i < kQWStages * kQWK * 8; i += kQThreads) {
+        const int s = i / (kQWK * 8), r = i - s * (kQWK * 8), m = r >> 3, chunk = r & 7;
         uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (grp == 8) v.x = pack_pair<T>(1.f, 0.f);
-        *reinterpret_cast<uint4*>(dst) = v;
+        if (chunk == (m & 7)) v.x = pack_pair<T>(1.f, 0.f);
+        *reinterpret_cast<uint4*>(tc_smem + ring_off + s * kQWStage + kQWABytes + kQWK * 128 + m * 128 + chunk * 16) = v;
     }
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = taddr_s;
-    constexpr uint32_t idesc = umma_idesc<T>(kUM, kUNB, 1, 1);
+    volatile int* abort = &s_abort;
 
-    auto load = [&](int j, int slot) {
-        const long long m = mb + static_cast<long long>(j) * kUK;
-        const uint32_t sa = ring + slot * kUStageBytes, sb = sa + kUABytes;
-#pragma unroll
-        for (int u = 0; u < kUK * (kUM / 8) / kTThreads; ++u) {  // g rows: 32 x 16 chunks of 8 p
-            const int i = tid + u * kTThreads, r = i >> 4, pg = i & 15;
-            const bool ok = m + r < me && p0 + pg * 8 < P;
-            cp_async16_s(sa + (r >> 3) * 2048 + pg * 128 + (r & 7) * 16, g + (ok ? (m + r) * P + p0 + pg * 8 : 0), ok);
+    if (warp == kQProducer) {
+        if (lane == 0) {
+            for (int j = 0; j < nk && !*abort; ++j) {
+                const int s = j % kQWStages;
+                const uint32_t ph = static_cast<uint32_t>(j / kQWStages) & 1u;
+                if (!mbar_wait_or(smem_u32(&empty[s]), ph ^ 1u, abort)) break;
+                const uint32_t fb = smem_u32(&full[s]);
+                mbar_expect_tx(fb, kQWLoad);
+                const uint32_t sa = ring + s * kQWStage, sb = sa + kQWABytes;
+                // ranges are whole multiples of 32 rows, so a box never reaches into the next
+                // range; past the last row of the matrix TMA fills zeros
+                const int m = static_cast<int>(mb + static_cast<long long>(j) * kQWK);
+                tma_load_2d(sa, &map_g, p0, m, fb);
+                tma_load_2d(sa + kQWK * 128, &map_g, p0 + 64, m, fb);
+                tma_load_2d(sb, &map_x, c0, m, fb);
+            }
         }
+    } else if (warp == kQMma) {
+        if (lane == 0) {
+            constexpr uint32_t idesc = umma_idesc<T>(kUM, kQWNB, 1, 1);
+            bool ok = true;
+            for (int j = 0; j < nk; ++j) {
+                const int s = j % kQWStages;
+                const uint32_t ph = static_cast<uint32_t>(j / kQWStages) & 1u;
+                if (!mbar_wait_or(smem_u32(&full[s]), ph, abort)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t sa = ring + s * kQWStage, sb = sa + kQWABytes;
 #pragma unroll
-        for (int u = 0; u < kUK * (kUN / 8) / kTThreads; ++u) {  // x rows: 32 x 8 chunks of 8 c
-            const int i = tid + u * kTThreads, r = i >> 3, cg = i & 7;
-            const bool ok = m + r < me && c0 + cg * 8 < Cx;
-            cp_async16_s(sb + (r >> 3) * 1280 + cg * 128 + (r & 7) * 16, x + (ok ? (m + r) * Cx + c0 + cg * 8 : 0), ok);
+                for (int q = 0; q < kQWK / 16; ++q)  // K = 16 rows of 128 bytes; the 64-wide blocks 4 KB apart
+                    umma_f16(tmem, umma_desc_sw128(sa + q * 2048, kQWK * 128, 1024),
+                             umma_desc_sw128(sb + q * 2048, kQWK * 128, 1024), idesc, j > 0 || q > 0);
+                umma_commit(smem_u32(&empty[s]));
+            }
+            if (ok) umma_commit(smem_u32(&acc_full));
         }
-    };
-
-    uint32_t phase = 0, pending = 0;
-    int aborted = 0;
-    auto wait_slot = [&](int s) {
-        if (!((pending >> s) & 1u)) return;
-        if (!mbar_wait(smem_u32(&mbar[s]), (phase >> s) & 1u)) aborted = 1;
-        phase ^= 1u << s;
-        pending &= ~(1u << s);
-    };
-    for (int j = 0; j < kUDepth; ++j) {
-        if (j < nk) load(j, j);
-        cp_async_commit();
     }
-    int slot = 0, ld_slot = kUDepth, last_slot = -1;
-    for (int j = 0; j < nk; ++j) {
-        wait_slot(ld_slot);  // the MMAs that last read ld_slot (two iterations ago) are done
-        if (j + kUDepth < nk) load(j + kUDepth, ld_slot);
-        cp_async_commit();
-        ld_slot = ld_slot + 1 == kUStages ? 0 : ld_slot + 1;
-        cp_async_wait<kUDepth>();
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        if (__syncthreads_or(aborted)) break;
-        if (tid == 0) {
-            tc_fence_after();
-            const uint32_t sa = ring + slot * kUStageBytes, sb = sa + kUABytes;
+    // warps 0-3: the partial tile out (thread = row p), into the fp32 accumulators
+    if (warp < 4) {
+        const bool have = nk > 0 && mbar_wait_or(smem_u32(&acc_full), 0u, abort);
+        tc_fence_after();
+        const int p = p0 + warp * 32 + lane;
+        const uint32_t lane_addr = tmem + (static_cast<uint32_t>(warp * 32) << 16);
 #pragma unroll
-            for (int q = 0; q < kUK / 16; ++q)  // K = 16 rows per MMA: two row groups of A and of B
-                umma_f16(tmem, umma_desc(sa + q * 4096, 2048, 128), umma_desc(sb + q * 2560, 1280, 128), idesc,
-                         j > 0 || q > 0);
-            umma_commit(smem_u32(&mbar[slot]));
-        }
-        pending |= 1u << slot;
-        last_slot = slot;
-        slot = slot + 1 == kUStages ? 0 : slot + 1;
-    }
-    cp_async_wait<0>();
-    if (last_slot >= 0) wait_slot(last_slot);
-    for (int s = 0; s < kUStages; ++s) wait_slot(s);
-    tc_fence_after();
-
-    // Partial tile out: thread = row p of this tile (TMEM lane), 64 columns of
-    // grad_W and column 64 (grad_b), added into the fp32 accumulators.
-    const int p = p0 + warp * 32 + lane;
-    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-    const bool live = nk > 0 && !aborted;
+        for (int h = 0; h < 3; ++h) {
+            uint32_t r[32];
+            tmem_ld32(lane_addr + h * 32, r);  // columns 64-95 hold grad_b in 64
+            if (!have || p >= P) continue;
+            if (h < 2) {
 #pragma unroll
-    for (int h = 0; h < kUN / 32; ++h) {
-        uint32_t r[32];
-        tmem_ld32(lane_addr + h * 32, r);
-        if (live && p < P) {
-#pragma unroll
-            for (int v = 0; v < 8; ++v) {
-                const int col = c0 + h * 32 + v * 4;
-                if (col < Cx)
-                    red_add4(wacc + static_cast<long long>(p) * Cx + col, __uint_as_float(r[4 * v]),
-                             __uint_as_float(r[4 * v + 1]), __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
+                for (int v = 0; v < 8; ++v) {
+                    const int col = c0 + h * 32 + v * 4;
+                    if (col < Cx)
+                        red_add4(wacc + static_cast<long long>(p) * Cx + col, __uint_as_float(r[4 * v]),
+                                 __uint_as_float(r[4 * v + 1]), __uint_as_float(r[4 * v + 2]),
+                                 __uint_as_float(r[4 * v + 3]));
+                }
+            } else if (bacc != nullptr && tc == 0) {
+                atomicAdd(bacc + p, __uint_as_float(r[0]));
             }
         }
     }
-    {
-        uint32_t r[32];
-        tmem_ld32(lane_addr + kUN, r);  // columns 64-95: 64 is the ones column
-        if (live && p < P && bacc != nullptr && tc == 0) atomicAdd(bacc + p, __uint_as_float(r[0]));
-    }
-    if (aborted) atomicOr(status, kLinStatusTimeout);
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kUTmemCols));
+    if (tid == 0 && *abort) atomicOr(status, kLinStatusTimeout);
+    if (warp == kQMma) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kUTmemCols));
 
     // The last CTA of this output tile rounds it once (its fence orders the other
     // CTAs' reductions, which precede their tickets, before its reads).
@@ -725,7 +467,7 @@ __global__ void __launch_bounds__(kTThreads, 2)
     __syncthreads();
     if (ticket != gridDim.x / ntile - 1) return;
     __threadfence();
-    round_tile<T, kTThreads>(wacc, bacc, gw, gb, P, Cx, p0, c0, tc == 0);
+    round_tile<T, kQThreads>(wacc, bacc, gw, gb, P, Cx, p0, c0, tc == 0);
 }
 
 int device_sms() {
@@ -735,74 +477,84 @@ int device_sms() {
     return sms > 0 ? sms : 148;
 }
 
-constexpr bool kTcgen05 = false;  // tcgen05 products (else mma.sync)
+// cuTensorMapEncodeTiled from the driver (resolved once through the runtime).
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn encode_tiled() {
+    static EncodeTiledFn fn = [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return static_cast<EncodeTiledFn>(nullptr);
+        return reinterpret_cast<EncodeTiledFn>(p);
+    }();
+    return fn;
+}
+
+// A row-major [rows][cols] matrix of 16-bit elements as a 2-D tensor map with
+// boxes 64 elements (128 bytes) wide and box_rows high, 128-byte swizzle, zeros
+// outside the matrix.
+bool swizzled_map(CUtensorMap* map, bool half, const void* base, long long rows, int cols, int box_rows) {
+    const EncodeTiledFn fn = encode_tiled();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
+    const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(map, half ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+              const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
 
 template <typename T>
 cudaError_t linear_backward_typed(long long M, int P, int Cx, const void* x, const void* w, const void* gom,
                                   void* gx, void* gw, void* gb, float* ws, cudaStream_t stream) {
-    const T* g = static_cast<const T*>(gom);
+    constexpr bool kHalf = std::is_same<T, __half>::value;
     const int sms = device_sms();
     const long long wsz = static_cast<long long>(P) * Cx;
     float* wacc = ws;
     float* bacc = ws + wsz;
     unsigned* status = reinterpret_cast<unsigned*>(ws + wsz + P);
     unsigned* done = status + 1;  // one finishing counter per 128 x 64 tile of grad_W
-    const long long ntile = static_cast<long long>((P + 127) / 128) * ((Cx + 63) / 64);
+    const long long ntile = static_cast<long long>((P + kUM - 1) / kUM) * ((Cx + kUN - 1) / kUN);
     // accumulators, the status word and the finishing counters
     cudaError_t e = cudaMemsetAsync(ws, 0, (wsz + P + 1 + ntile) * sizeof(float), stream);
     if (e != cudaSuccess) return e;
     if (gx) {
-        if constexpr (kTcgen05) {
-            e = cudaFuncSetAttribute(linear_grad_x_tc_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, kTSmem);
-            if (e != cudaSuccess) return e;
-            const int ntiles_n = (Cx + kTN - 1) / kTN;
-            const long long ntiles = (M + kTM - 1) / kTM * ntiles_n;
-            const int nk = (P + kTK - 1) / kTK;
-            const long long grid = std::min<long long>(ntiles, 2LL * sms);
-            linear_grad_x_tc_kernel<T><<<static_cast<unsigned>(grid), kTThreads, kTSmem, stream>>>(
-                g, static_cast<const T*>(w), static_cast<T*>(gx), M, P, Cx, ntiles, ntiles_n, nk, status);
-        } else {
-            const size_t smem = kXStages * sizeof(XStage<T>);
-            e = cudaFuncSetAttribute(linear_grad_x_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     static_cast<int>(smem));
-            if (e != cudaSuccess) return e;
-            const int ntiles_n = (Cx + kXN - 1) / kXN;
-            const long long ntiles = (M + kXM - 1) / kXM * ntiles_n;
-            const int nk = (P + kXK - 1) / kXK;
-            const long long grid = std::min<long long>(ntiles, 3LL * sms);
-            linear_grad_x_kernel<T><<<static_cast<unsigned>(grid), kLbThreads, smem, stream>>>(
-                g, static_cast<const T*>(w), static_cast<T*>(gx), M, P, Cx, ntiles, ntiles_n, nk);
-        }
+        CUtensorMap map_g, map_w;
+        if (!swizzled_map(&map_g, kHalf, gom, M, P, kTM) || !swizzled_map(&map_w, kHalf, w, P, Cx, kQXK))
+            return cudaErrorInvalidValue;
+        e = cudaFuncSetAttribute(linear_grad_x_tma_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, kQXSmem);
+        if (e != cudaSuccess) return e;
+        const int ntiles_n = (Cx + kTN - 1) / kTN;
+        const long long ntiles = (M + kTM - 1) / kTM * ntiles_n;
+        const int nk = (P + kQXK - 1) / kQXK;
+        const long long grid = std::min<long long>(ntiles, 2LL * sms);
+        linear_grad_x_tma_kernel<T><<<static_cast<unsigned>(grid), kQThreads, kQXSmem, stream>>>(
+            map_g, map_w, static_cast<T*>(gx), M, Cx, ntiles, ntiles_n, nk, status);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
     if (!gw && !gb) return cudaSuccess;
-    const int pt = (P + 127) / 128, ct = (Cx + 63) / 64;
-    const int rows = kTcgen05 ? kUK : kWK;
-    const int per_sm = kTcgen05 ? 2 : 3;
-    // split the rows so that the grid holds about per_sm CTAs per SM, at least a few stages each
-    const long long want = std::max<long long>(1, (per_sm * static_cast<long long>(sms) + pt * ct - 1) / (pt * ct));
+    CUtensorMap map_g, map_x;
+    if (!swizzled_map(&map_g, kHalf, gom, M, P, kQWK) || !swizzled_map(&map_x, kHalf, x, M, Cx, kQWK))
+        return cudaErrorInvalidValue;
+    const int pt = (P + kUM - 1) / kUM, ct = (Cx + kUN - 1) / kUN;
+    // split the rows (whole multiples of 32) so that the grid holds about two CTAs per SM
+    const long long want = std::max<long long>(1, (2LL * sms + pt * ct - 1) / (pt * ct));
     long long mchunk = (M + want - 1) / want;
-    mchunk = std::max<long long>(4LL * rows, (mchunk + rows - 1) / rows * rows);
-    if (mchunk / rows >= 0x7fffffffLL) return cudaErrorInvalidValue;  // stages per CTA must fit an int
+    mchunk = std::max<long long>(4LL * kQWK, (mchunk + kQWK - 1) / kQWK * kQWK);
     const long long splits = (M + mchunk - 1) / mchunk;
     const long long grid = splits * pt * ct;
     if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-    if constexpr (kTcgen05) {
-        e = cudaFuncSetAttribute(linear_grad_w_tc_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, kUSmem);
-        if (e != cudaSuccess) return e;
-        linear_grad_w_tc_kernel<T><<<static_cast<unsigned>(grid), kTThreads, kUSmem, stream>>>(
-            g, static_cast<const T*>(x), wacc, gb ? bacc : nullptr, done, status, static_cast<T*>(gw),
-            static_cast<T*>(gb), M, P, Cx, pt * ct, ct, mchunk);
-    } else {
-        const size_t smem = kWStages * sizeof(WStage<T>);
-        e = cudaFuncSetAttribute(linear_grad_w_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(smem));
-        if (e != cudaSuccess) return e;
-        linear_grad_w_kernel<T><<<static_cast<unsigned>(grid), kLbThreads, smem, stream>>>(
-            g, static_cast<const T*>(x), wacc, gb ? bacc : nullptr, done, static_cast<T*>(gw), static_cast<T*>(gb), M,
-            P, Cx, pt * ct, ct, mchunk);
-    }
+    e = cudaFuncSetAttribute(linear_grad_w_tma_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, kQWSmem);
+    if (e != cudaSuccess) return e;
+    linear_grad_w_tma_kernel<T><<<static_cast<unsigned>(grid), kQThreads, kQWSmem, stream>>>(
+        map_g, map_x, wacc, gb ? bacc : nullptr, done, status, static_cast<T*>(gw), static_cast<T*>(gb), M, P, Cx,
+        pt * ct, ct, mchunk);
     return cudaGetLastError();
 }
 
@@ -810,7 +562,7 @@ cudaError_t linear_backward_typed(long long M, int P, int Cx, const void* x, con
 
 size_t linear_backward_workspace_bytes(int P, int Cx) {
     // grad_W and grad_b accumulators, the status word, one finishing counter per 128 x 64 tile
-    const size_t ntile = static_cast<size_t>((P + 127) / 128) * ((Cx + 63) / 64);
+    const size_t ntile = static_cast<size_t>((P + kUM - 1) / kUM) * ((Cx + kUN - 1) / kUN);
     return (static_cast<size_t>(P) * Cx + P + 1 + ntile) * sizeof(float);
 }
 

@@ -250,7 +250,10 @@ int dcn4_backward_diagnostics(const dcn4_params* p, const void* workspace, size_
 
 /* Bytes of device workspace dcn4_backward_linear needs: dcn4_backward's
  * workspace rounded up to 256 bytes, then fp32 accumulators for grad_weight
- * (P*Cx) and grad_bias (P), rounded up to 256 bytes; 0 if p is invalid. */
+ * (P*Cx) and grad_bias (P), a 32-bit status word (nonzero after the call if a
+ * bounded wait inside the linear kernels gave up; the outputs are then not
+ * valid) and one 32-bit counter per 128 x 64 tile of grad_weight, rounded up
+ * to 256 bytes; 0 if p is invalid. */
 size_t dcn4_backward_linear_workspace_size(const dcn4_params* p, int Cx);
 
 /* Backward of dcn4_forward_linear, the aggregation with its offset/mask linear
@@ -262,18 +265,19 @@ size_t dcn4_backward_linear_workspace_size(const dcn4_params* p, int Cx);
  *   grad_weight [P, Cx]         = g^T x             (sum over m of g[m, j] * x[m, c])
  *   grad_bias   [P]             = sum over m of g[m, j]
  * All of dtype (fp16 or bf16; DCN4_ERR_UNSUPPORTED for fp32).  The products read
- * g as dcn4_backward rounded it to dtype, run on the tensor cores with fp32
- * accumulation and are rounded to dtype once; grad_weight and grad_bias sum
- * partial products of row chunks with fp32 atomics (so their last bit may vary
- * from call to call).  grad_x, grad_weight and grad_bias may each be NULL (not
+ * g as dcn4_backward rounded it to dtype, run on the tensor cores (tcgen05, fed
+ * by TMA) with fp32 accumulation and are rounded to dtype once; grad_weight and
+ * grad_bias sum partial products of row chunks with fp32 atomics (so their last
+ * bit may vary from call to call).  grad_x, grad_weight and grad_bias may each be NULL (not
  * wanted); grad_value and grad_offset_mask are required.  Every pointer 16-byte
  * aligned; Cx a positive multiple of 16 (DCN4_ERR_BAD_SHAPE); `workspace`
  * (device, >= dcn4_backward_linear_workspace_size bytes) is clobbered, its first
  * part exactly as by dcn4_backward (so dcn4_backward_diagnostics reads it).
- * With N*Ho*Wo = 0 only grad_weight and grad_bias are written (zeros).
- * Launches on `stream`: dcn4_backward's launches, then one kernel for grad_x,
- * a memset and one kernel for the grad_weight/grad_bias accumulators, and one
- * rounding kernel for each of grad_weight and grad_bias. */
+ * N*Ho*Wo and P*Cx must be below 2^31 (DCN4_ERR_UNSUPPORTED).  With N*Ho*Wo = 0
+ * only grad_weight and grad_bias are written (zeros).
+ * Launches on `stream`: dcn4_backward's launches, then a memset of the linear
+ * part of the workspace, one kernel for grad_x and one for grad_weight and
+ * grad_bias (which also rounds them). */
 int dcn4_backward_linear(const dcn4_params* p, int Cx, const void* value, const void* offset_mask, const void* x,
                          const void* weight, const void* grad_out, void* grad_value, void* grad_offset_mask,
                          void* grad_x, void* grad_weight, void* grad_bias, void* workspace, size_t workspace_bytes,

@@ -241,6 +241,9 @@ assert call(p, 64, value=None) == -1 and call(p, 64, gv=None) == -1
 bad = dcn.make_params(N=2, H=8, W=8, G=4, Cg=16, dtype="bf16")
 bad.P = 100
 assert call(bad, 64) == -3
+# the tensor-map row coordinates are 32-bit: N*Ho*Wo must stay below 2^31
+big = dcn.make_params(N=2048, H=1024, W=1024, G=4, Cg=16, dtype="bf16")
+assert call(big, 64, nb=1 << 62) == -5 and "2^31" in dcn.dcn4_last_error()
 assert dcn.dcn4_last_error() != ""
 """)
 
