@@ -63,10 +63,15 @@ def _run(w, Cx, *, bias=True, sample=None, want_x=True, want_weight=True):
     b = to_device(lin["bias"], w.dtype) if bias else None
     om = torch.empty((w.N, w.Ho, w.Wo, w.P), dtype=v.dtype, device="cuda")
     dcn.forward_linear(p, v, x, wt, b, offset_mask_out=om)
+    need = dcn.dcn4_backward_linear_workspace_size(p, Cx)
+    ws = torch.empty(need, dtype=torch.uint8, device="cuda")
     gv, gom, gx, gw, gb = dcn.backward_linear(p, v, om, x, wt, gy, with_bias=bias, want_x=want_x,
-                                              want_weight=want_weight)
+                                              want_weight=want_weight, workspace=ws)
     _, gom_plain = dcn.backward(p, v, om, gy)
     torch.cuda.synchronize()
+    # the linear kernels' status word (after dcn4_backward's part and the fp32 accumulators): no wait gave up
+    off = (dcn.dcn4_backward_workspace_size(p) + 255) // 256 * 256 + 4 * (w.P * Cx + w.P)
+    assert int(ws[off:off + 4].view(torch.int32).item()) == 0, "a bounded wait in the linear kernels gave up"
     assert torch.equal(gom.view(torch.int16), gom_plain.view(torch.int16)), "grad_offset_mask differs from dcn4_backward"
     assert (gx is None) != want_x and (gw is None) != want_weight and (gb is None) != bias
 
