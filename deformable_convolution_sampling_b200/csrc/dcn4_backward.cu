@@ -217,11 +217,13 @@ __global__ void __launch_bounds__(256, 3) samples_kernel(const Geometry g, const
     T* om_s = reinterpret_cast<T*>(smem);
     T* gom_s = reinterpret_cast<T*>(smem + tile_elems * sizeof(T));  // P % 8 == 0 keeps this 16-byte aligned
     const bool filing = sizeof(T) == 2 && g.buckets != 0;
-    // Unrolled grids without softmax stage only the meta words: the record body
-    // (bin, mask bits, fractions) is formed again at write-out from the offsets,
-    // which stay in shared memory, with the same fp32 arithmetic.  Half the
-    // staging leaves that much more of the SM's L1 to the gathers.
-    constexpr bool SLIM = KH > 0 && !SM;
+    // Unrolled grids without softmax or remove_center stage only the meta words:
+    // the record body (bin, mask bits, fractions) is formed again at write-out
+    // from the offsets, which stay in shared memory, with the same fp32
+    // arithmetic.  Half the staging leaves that much more of the SM's L1 to the
+    // gathers (measured: a gain where the samples spread wide, a small loss
+    // with remove_center at every offset scale tried).
+    constexpr bool SLIM = KH > 0 && !SM && !RC;
 
     const Tile t = tile_of_block(g);
     const int K = KH > 0 ? KH * KW - (RC ? 1 : 0) : g.K;
@@ -1203,7 +1205,7 @@ cudaError_t launch_value_vec(const Geometry& g, const void* om, const void* gout
 size_t backward_smem_bytes(const Geometry& g, int elem_bytes) {
     size_t b = static_cast<size_t>(g.TH) * g.TW * g.P * elem_bytes * 2;
     if (elem_bytes == 2 && g.buckets) {  // staging: meta words only for the unrolled grids without softmax
-        const size_t per = (g.kh == 3 && g.kw == 3 && !g.softmax) ? 8 : 16;
+        const size_t per = (g.kh == 3 && g.kw == 3 && !g.softmax && !g.remove_center) ? 8 : 16;
         b += static_cast<size_t>(filing_chunk(g)) * samples_threads(g) * per;
     }
     return b;
