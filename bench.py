@@ -760,7 +760,9 @@ def linear_leg(w: gen.Workload, v, gy, p, flush, stream, dev, world: int) -> dic
         torch.cuda.synchronize(dev)
         res[name] = round(max_over_ranks(statistics.mean(a.elapsed_time(c) for a, c in ev) * 1e3, dev), 2)
     res["speedup_vs_unfused"] = round(res["cublas_linear_then_forward_us"] / res["fused_us"], 3)
-    res["gemm"] = f"x [{w.N * w.Ho * w.Wo}, {w.C}] @ W^T [{w.C}, {w.P}] + b, mma.sync m16n8k16, fp32 accumulation"
+    res["gemm"] = (f"x [{w.N * w.Ho * w.Wo}, {w.C}] @ W^T [{w.C}, {w.P}] + b per 64-pixel tile: tcgen05.mma kind::f16 "
+                   f"(M = 128 rows of W, N = 64 pixels, fp32 accumulator in tensor memory) where W fits 128 rows and "
+                   f"Cx is 64 or 128, else mma.sync m16n8k16")
     res["launches_per_call"] = 1
 
     # Backward of the layer: dcn4_backward_linear (the aggregation's backward, then the

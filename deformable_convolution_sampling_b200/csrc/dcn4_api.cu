@@ -382,7 +382,7 @@ int dcn4_forward_linear(const dcn4_params* p, int Cx, const void* value, const v
     if (p->dtype == DCN4_F32) return fail(DCN4_ERR_UNSUPPORTED, "the fused linear producer takes fp16 or bf16");
     if (Cx < 16 || Cx % 16 != 0 || Cx > (1 << 16))
         return fail(DCN4_ERR_BAD_SHAPE, "Cx=%d must be a positive multiple of 16", Cx);
-    if (dcn4::forward_linear_smem_bytes(g, Cx, dcn4::forward_linear_w_smem(g, Cx)) > kSmemMax)
+    if (dcn4::forward_linear_smem_bytes(g, Cx, dcn4::forward_linear_mode(g, Cx)) > kSmemMax)
         return fail(DCN4_ERR_UNSUPPORTED, "x rows of Cx=%d with P=%d do not fit shared memory", Cx, p->P);
     if (static_cast<long long>(g.Ho) * g.Wo * Cx >= (1LL << 31) || static_cast<long long>(p->P) * Cx >= (1LL << 31))
         return fail(DCN4_ERR_UNSUPPORTED, "x or weight too large");

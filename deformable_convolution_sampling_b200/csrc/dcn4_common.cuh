@@ -366,9 +366,11 @@ size_t forward_smem_bytes(const Geometry& g, int elem_bytes);
 // tile, x [N, Ho, Wo, Cx], w [P, Cx], b [P] or null, om_out [N, Ho, Wo, P] or null.
 cudaError_t launch_forward_linear(const Geometry& g, int dtype, const void* value, const void* x, const void* w,
                                   const void* b, void* out, void* om_out, int Cx, cudaStream_t stream);
-size_t forward_linear_smem_bytes(const Geometry& g, int Cx, bool w_smem);
-// Whether the fused forward stages W in shared memory for this shape.
-bool forward_linear_w_smem(const Geometry& g, int Cx);
+// mode 0: mma.sync, W read from global memory; 1: mma.sync, W staged in shared
+// memory; 2: tcgen05 (W and the x tiles swizzled in shared memory).
+size_t forward_linear_smem_bytes(const Geometry& g, int Cx, int mode);
+// The fused forward's producer mode for this shape.
+int forward_linear_mode(const Geometry& g, int Cx);
 // Gradients of the linear producer from gom = grad_offset_mask as an [M, P]
 // matrix (16-bit dtypes): gx = gom W [M, Cx], gw = gom^T x [P, Cx], gb = column
 // sums of gom [P]; any of the three may be null.  ws: fp32 scratch of

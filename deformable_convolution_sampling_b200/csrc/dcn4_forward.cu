@@ -34,6 +34,7 @@
 #include <type_traits>
 
 #include "dcn4_common.cuh"
+#include "dcn4_tcgen05.cuh"
 
 namespace dcn4 {
 namespace {
@@ -72,7 +73,20 @@ struct LinearArgs {
     T* om_out;
     int Cx;
     int w_smem;  // 1: W is staged in shared memory once per CTA (when it fits)
+    int tc;      // 1: the offset_mask tile is formed on tcgen05 (see stage_x_swizzled)
 };
+
+// tcgen05 form of the producer: D^T[p][pixel] = W x^T with M = 128 rows of W
+// (P <= 128, the rest zero), N = the tile's 64 pixels, K = Cx in 64-wide slabs,
+// the accumulator in tensor memory.  W and the x tiles sit in shared memory in
+// the 128-byte swizzled K-major layout: row r of a slab at r*128 bytes, its
+// 16-byte chunk c at ((c ^ (r % 8)) * 16), slabs of 64 columns one after the
+// other.  The SMs' tensor cores form the tile while the warps only stage
+// operands and read the result back into the tile's offset_mask rows.
+constexpr int kTcRows = 128, kTcPix = 64;
+__host__ __device__ inline int tc_x_bytes(int Cx) { return kTcPix * Cx * 2; }
+__host__ __device__ inline int tc_w_bytes(int Cx) { return kTcRows * Cx * 2; }
+__device__ unsigned g_fwd_linear_status;  // nonzero once a bounded wait of the tcgen05 producer gave up
 
 // Rows of a staged x tile: the tile's pixels rounded up to whole 16-row MMA tiles.
 __host__ __device__ inline int linear_rows(const Geometry& g) { return (g.TH * g.TW + 15) / 16 * 16; }
@@ -116,6 +130,24 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
         memcpy(&u, &h, 4);
     }
     return u;
+}
+
+// The tile's rows of x, swizzled for tcgen05 (see kTcRows), with cp.async.
+template <typename T>
+__device__ __forceinline__ void stage_x_swizzled(uint32_t dst, const LinearArgs<T>& lin, const Geometry& g,
+                                                 const Tile& t) {
+    const int cpp = lin.Cx / 8;  // 16-byte chunks per pixel
+    const int total = t.th * t.tw * cpp;
+    for (int i = threadIdx.x; i < total; i += blockDim.x) {
+        const int q = i / cpp, c = i - q * cpp;
+        const int py = q / t.tw, px = q - py * t.tw;
+        const int row = py * g.TW + px;
+        const long long pix = (static_cast<long long>(t.n) * g.Ho + t.ho0 + py) * g.Wo + t.wo0 + px;
+        const T* sp = lin.x + pix * lin.Cx + c * 8;
+        const uint32_t d = dst + (c >> 3) * (kTcPix * 128) + row * 128 + (((c & 7) ^ (row & 7)) << 4);
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(sp));
+    }
+    asm volatile("cp.async.commit_group;");
 }
 
 // The tile's rows of x into shared memory [rows][Cx + 8] with cp.async.
@@ -324,13 +356,26 @@ __global__ void __launch_bounds__(256, kFwdCtasPerSm) forward_kernel(const Geome
     T* w_s = nullptr;
     float* b_s = nullptr;
     float* e_s;  // softmax exponentials [K][threads]
+    // tcgen05 producer: shared addresses of the two swizzled x tiles and of W (1024-byte aligned)
+    const uint32_t sbase = tc::smem_u32(smem);
+    uint32_t tc_x[2] = {0u, 0u}, tc_w = 0u;
+    __shared__ __align__(8) uint64_t tc_mbar;
+    __shared__ uint32_t tc_taddr;
+    __shared__ int tc_abort;
     if constexpr (LIN) {
-        const int xs = linear_rows(g) * linear_ld(lin.Cx);
         bufs[0] = bufs[1] = reinterpret_cast<T*>(smem);
-        xbuf[0] = bufs[0] + tile_elems;
-        xbuf[1] = xbuf[0] + xs;
-        w_s = xbuf[1] + xs;
-        b_s = reinterpret_cast<float*>(w_s + (lin.w_smem ? linear_w_rows(g) * linear_ld(lin.Cx) : 0));
+        if (lin.tc) {
+            tc_x[0] = (sbase + static_cast<uint32_t>(tile_elems) * 2u + 1023u) & ~1023u;
+            tc_x[1] = tc_x[0] + tc_x_bytes(lin.Cx);
+            tc_w = tc_x[1] + tc_x_bytes(lin.Cx);
+            b_s = reinterpret_cast<float*>(smem + (tc_w - sbase) + tc_w_bytes(lin.Cx));
+        } else {
+            const int xs = linear_rows(g) * linear_ld(lin.Cx);
+            xbuf[0] = bufs[0] + tile_elems;
+            xbuf[1] = xbuf[0] + xs;
+            w_s = xbuf[1] + xs;
+            b_s = reinterpret_cast<float*>(w_s + (lin.w_smem ? linear_w_rows(g) * linear_ld(lin.Cx) : 0));
+        }
         e_s = b_s + g.P;
     } else {
         bufs[0] = reinterpret_cast<T*>(smem);
@@ -342,7 +387,30 @@ __global__ void __launch_bounds__(256, kFwdCtasPerSm) forward_kernel(const Geome
     if (tile >= ntiles) return;
     if constexpr (LIN) {
         for (int j = threadIdx.x; j < g.P; j += blockDim.x) b_s[j] = lin.b ? to_f32(lin.b[j]) : 0.f;
-        if (lin.w_smem) {  // W rows [P][Cx] -> [rows][Cx + 8]; rows past P stay unset (their columns are dropped)
+        if (lin.tc) {
+            // W rows [P][Cx] into 64-wide swizzled slabs; rows P..127 zero (their results are never stored)
+            const int cpr = lin.Cx / 8;
+            for (int i = threadIdx.x; i < kTcRows * cpr; i += blockDim.x) {
+                const int r = i / cpr, c = i - r * cpr;
+                uint4 v = make_uint4(0u, 0u, 0u, 0u);
+                if (r < g.P) v = ld_gather(lin.w + static_cast<long long>(r) * lin.Cx + c * 8);
+                *reinterpret_cast<uint4*>(smem + (tc_w - sbase) + (c >> 3) * (kTcRows * 128) + r * 128 +
+                                          (((c & 7) ^ (r & 7)) << 4)) = v;
+            }
+            if (threadIdx.x == 0) {
+                tc::mbar_init(tc::smem_u32(&tc_mbar), 1);
+                tc_abort = 0;
+                asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+            }
+            if (threadIdx.x < 32) {  // kTcPix fp32 columns x 128 lanes: the accumulator
+                asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                                 tc::smem_u32(&tc_taddr)),
+                             "r"(kTcPix));
+                asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+            }
+            tc::tc_fence_before();
+            stage_x_swizzled(tc_x[0], lin, g, tile_at(g, tile));
+        } else if (lin.w_smem) {  // W rows [P][Cx] -> [rows][Cx + 8]; rows past P stay unset (their columns are dropped)
             const int cpr = lin.Cx / EPV;
             for (int i = threadIdx.x; i < g.P * cpr; i += blockDim.x) {
                 const int r = i / cpr, c = i - r * cpr;
@@ -350,7 +418,7 @@ __global__ void __launch_bounds__(256, kFwdCtasPerSm) forward_kernel(const Geome
                     ld_gather(lin.w + static_cast<long long>(r) * lin.Cx + c * EPV);
             }
         }
-        stage_x_async(xbuf[0], lin, g, tile_at(g, tile));
+        if (!lin.tc) stage_x_async(xbuf[0], lin, g, tile_at(g, tile));
     } else {
         stage_tile_async(bufs[0], om, g, tile_at(g, tile));
     }
@@ -372,7 +440,11 @@ __global__ void __launch_bounds__(256, kFwdCtasPerSm) forward_kernel(const Geome
         const int next = tile + gridDim.x;
         if (next < ntiles) {
             if constexpr (LIN) {
-                stage_x_async(xbuf[(it + 1) & 1], lin, g, tile_at(g, next));
+                if (lin.tc) {
+                    stage_x_swizzled(tc_x[(it + 1) & 1], lin, g, tile_at(g, next));
+                } else {
+                    stage_x_async(xbuf[(it + 1) & 1], lin, g, tile_at(g, next));
+                }
             } else {
                 stage_tile_async(bufs[(it + 1) & 1], om, g, tile_at(g, next));
             }
@@ -380,19 +452,59 @@ __global__ void __launch_bounds__(256, kFwdCtasPerSm) forward_kernel(const Geome
         } else {
             asm volatile("cp.async.wait_group 0;" ::: "memory");
         }
+        // the tensor cores read the x tile through the async proxy
+        if constexpr (LIN) {
+            if (lin.tc) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        }
         __syncthreads();
         const Tile t = tile_at(g, tile);
         // the tile's rows, addressed from smem directly so the reads stay shared-space loads
         const T* om_s = reinterpret_cast<const T*>(smem) + (LIN ? 0 : (it & 1) * tile_elems);
         if constexpr (LIN) {
-            switch (lin.w_smem ? lin.Cx / 16 : 0) {
-                case 1: linear_tile_staged<T, 1>(g, lin, xbuf[it & 1], w_s, bufs[0], b_s); break;
-                case 2: linear_tile_staged<T, 2>(g, lin, xbuf[it & 1], w_s, bufs[0], b_s); break;
-                case 4: linear_tile_staged<T, 4>(g, lin, xbuf[it & 1], w_s, bufs[0], b_s); break;
-                case 8: linear_tile_staged<T, 8>(g, lin, xbuf[it & 1], w_s, bufs[0], b_s); break;
-                default: linear_tile(g, lin, xbuf[it & 1], w_s, bufs[0], b_s);
+            if (lin.tc) {
+                // one thread issues the tile's MMAs; all wait for them, then read the accumulator back:
+                // warp w reads TMEM lanes (rows p) 32 (w % 4) .. + 31, pixel columns 32 (w / 4) .. + 31
+                tc::tc_fence_after();
+                const uint32_t tmem = tc_taddr;
+                if (threadIdx.x == 0) {
+                    constexpr uint32_t idesc = tc::umma_idesc<T>(kTcRows, kTcPix, 0, 0);
+                    const uint32_t xb = tc_x[it & 1];
+                    for (int sb = 0; sb < lin.Cx / 64; ++sb)
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+                            tc::umma_f16(tmem, tc::umma_desc_sw128(tc_w + sb * (kTcRows * 128) + q * 32, 16, 1024),
+                                         tc::umma_desc_sw128(xb + sb * (kTcPix * 128) + q * 32, 16, 1024), idesc,
+                                         sb > 0 || q > 0);
+                    tc::umma_commit(tc::smem_u32(&tc_mbar));
+                }
+                tc::mbar_wait_or(tc::smem_u32(&tc_mbar), static_cast<uint32_t>(it) & 1u, &tc_abort);
+                tc::tc_fence_after();
+                const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+                const int sub = warp & 3, half = warp >> 2;
+                uint32_t acc32[32];
+                tc::tmem_ld32(tmem + (static_cast<uint32_t>(32 * sub) << 16) + half * 32, acc32);
+                const int pr = 32 * sub + lane;
+                if (pr < g.P && !tc_abort) {
+                    const float bp = b_s[pr];
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        bufs[0][(half * 32 + j) * g.P + pr] = from_f32<T>(__uint_as_float(acc32[j]) + bp);
+                }
+                tc::tc_fence_before();  // the next tile's MMAs overwrite the accumulator after the next barrier
+            } else {
+                switch (lin.w_smem ? lin.Cx / 16 : 0) {
+                    case 1: linear_tile_staged<T, 1>(g, lin, xbuf[it & 1], w_s, bufs[0], b_s); break;
+                    case 2: linear_tile_staged<T, 2>(g, lin, xbuf[it & 1], w_s, bufs[0], b_s); break;
+                    case 4: linear_tile_staged<T, 4>(g, lin, xbuf[it & 1], w_s, bufs[0], b_s); break;
+                    case 8: linear_tile_staged<T, 8>(g, lin, xbuf[it & 1], w_s, bufs[0], b_s); break;
+                    default: linear_tile(g, lin, xbuf[it & 1], w_s, bufs[0], b_s);
+                }
             }
             __syncthreads();
+            if (lin.tc && tc_abort) {  // a wait gave up: no further tile is formed
+                if (threadIdx.x == 0) atomicOr(&g_fwd_linear_status, 1u);
+                break;
+            }
             if (lin.om_out) {  // the rows the samples use, 16-byte stores
                 const int cpp = g.P / EPV;
                 for (int i = threadIdx.x; i < t.th * t.tw * cpp; i += blockDim.x) {
@@ -511,12 +623,22 @@ __global__ void __launch_bounds__(256, kFwdCtasPerSm) forward_kernel(const Geome
         }
         __syncthreads();  // the buffer is refilled two tiles later (LIN: om_s at the next tile)
     }
+    if constexpr (LIN) {
+        if (lin.tc) {
+            asm volatile("cp.async.wait_group 0;" ::: "memory");
+            tc::tc_fence_before();
+            __syncthreads();
+            if (threadIdx.x < 32)
+                asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tc_taddr), "r"(kTcPix));
+        }
+    }
 }
 
 template <typename T, int VEC, int KH, int KW, bool RC, bool SM, bool LIN>
 cudaError_t launch_typed(const Geometry& g, const void* value, const void* om, void* out, const LinearArgs<T>& lin,
                          cudaStream_t stream) {
-    const size_t smem = LIN ? forward_linear_smem_bytes(g, lin.Cx, lin.w_smem != 0) : forward_smem_bytes(g, sizeof(T));
+    const size_t smem = LIN ? forward_linear_smem_bytes(g, lin.Cx, lin.tc ? 2 : lin.w_smem ? 1 : 0)
+                            : forward_smem_bytes(g, sizeof(T));
     auto kern = forward_kernel<T, VEC, KH, KW, RC, SM, LIN>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
@@ -561,33 +683,44 @@ cudaError_t launch_vec(const Geometry& g, int vec, const void* value, const void
 
 }  // namespace
 
-size_t forward_linear_smem_bytes(const Geometry& g, int Cx, bool w_smem) {
-    const size_t xs = static_cast<size_t>(linear_rows(g)) * linear_ld(Cx) * 2;  // 16-bit dtypes only
-    const size_t ws = w_smem ? static_cast<size_t>(linear_w_rows(g)) * linear_ld(Cx) * 2 : 0;
-    return static_cast<size_t>(g.pix_per_cta) * g.P * 2 + 2 * xs + ws + static_cast<size_t>(g.P) * sizeof(float) +
-           (g.softmax ? static_cast<size_t>(g.K) * samples_threads(g) * sizeof(float) : 0);
+size_t forward_linear_smem_bytes(const Geometry& g, int Cx, int mode) {
+    const size_t om = static_cast<size_t>(g.pix_per_cta) * g.P * 2;  // 16-bit dtypes only
+    const size_t tail = static_cast<size_t>(g.P) * sizeof(float) +
+                        (g.softmax ? static_cast<size_t>(g.K) * samples_threads(g) * sizeof(float) : 0);
+    if (mode == 2) return om + 1024 + 2 * static_cast<size_t>(tc_x_bytes(Cx)) + tc_w_bytes(Cx) + tail;
+    const size_t xs = static_cast<size_t>(linear_rows(g)) * linear_ld(Cx) * 2;
+    const size_t ws = mode == 1 ? static_cast<size_t>(linear_w_rows(g)) * linear_ld(Cx) * 2 : 0;
+    return om + 2 * xs + ws + tail;
 }
 
-bool forward_linear_w_smem(const Geometry& g, int Cx) {
-    // W is staged when the CTA still fits three to an SM (the sampler's occupancy)
-    return forward_linear_smem_bytes(g, Cx, true) + 1024 <= 227 * 1024 / kFwdCtasPerSm;
+int forward_linear_mode(const Geometry& g, int Cx) {
+    // Both need the CTA to still fit three to an SM (the sampler's occupancy).
+    const size_t budget = 227 * 1024 / kFwdCtasPerSm;
+    // tcgen05: 64-pixel tiles of four lanes per pixel (eight warps for the read-back), W of at most 128
+    // rows and whole 64-wide slabs of at most 128 columns
+    const bool tc_shape = g.TH * g.TW == kTcPix && g.G * g.nslice == 4 && Cx % 64 == 0 && Cx <= 128 &&
+                          g.P <= kTcRows;
+    if (tc_shape && forward_linear_smem_bytes(g, Cx, 2) + 1024 <= budget) return 2;
+    return forward_linear_smem_bytes(g, Cx, 1) + 1024 <= budget ? 1 : 0;
 }
 
 cudaError_t launch_forward_linear(const Geometry& g, int dtype, const void* value, const void* x, const void* w,
                                   const void* b, void* out, void* om_out, int Cx, cudaStream_t stream) {
     switch (dtype) {
         case 1: {
+            const int mode = forward_linear_mode(g, Cx);
             const LinearArgs<__half> lin{static_cast<const __half*>(x), static_cast<const __half*>(w),
                                          static_cast<const __half*>(b), static_cast<__half*>(om_out), Cx,
-                                         forward_linear_w_smem(g, Cx) ? 1 : 0};
+                                         mode == 1 ? 1 : 0, mode == 2 ? 1 : 0};
             return launch_vec<__half, true>(g, g.vec, value, nullptr, out, lin, stream);
         }
         case 2: {
+            const int mode = forward_linear_mode(g, Cx);
             const LinearArgs<__nv_bfloat16> lin{static_cast<const __nv_bfloat16*>(x),
                                                 static_cast<const __nv_bfloat16*>(w),
                                                 static_cast<const __nv_bfloat16*>(b),
-                                                static_cast<__nv_bfloat16*>(om_out), Cx,
-                                                forward_linear_w_smem(g, Cx) ? 1 : 0};
+                                                static_cast<__nv_bfloat16*>(om_out), Cx, mode == 1 ? 1 : 0,
+                                                mode == 2 ? 1 : 0};
             return launch_vec<__nv_bfloat16, true>(g, g.vec, value, nullptr, out, lin, stream);
         }
         default: return cudaErrorInvalidValue;

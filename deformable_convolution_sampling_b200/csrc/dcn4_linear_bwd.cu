@@ -27,9 +27,12 @@
 #include <type_traits>
 
 #include "dcn4_common.cuh"
+#include "dcn4_tcgen05.cuh"
 
 namespace dcn4 {
 namespace {
+
+using namespace tc;
 
 template <typename T>
 __device__ __forceinline__ uint32_t pack_pair(float lo, float hi) {
@@ -73,62 +76,8 @@ __device__ __forceinline__ void round_tile(const float* wacc, const float* bacc,
             if (p0 + r < P) gb[p0 + r] = from_f32<T>(__ldcg(bacc + p0 + r));
 }
 
-// ---------------------------------------------------------------------------
-// tcgen05 building blocks: shared-memory matrix and instruction descriptors,
-// the MMA, its commit to an mbarrier, tensor-memory loads, bounded waits.
-// ---------------------------------------------------------------------------
 constexpr int kTM = 128, kTN = 64;  // grad_x tile: 128 rows of g x 64 columns
-constexpr int kTWaitSpins = 1 << 22;                  // bound of every mbarrier wait
-constexpr unsigned kLinStatusTimeout = 1u;            // a wait gave up (status word)
-
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-// Shared-memory matrix descriptor: start address, leading and stride byte
-// offsets (all in 16-byte units), descriptor version 1; layout type in bits 61-63.
-__device__ __forceinline__ uint64_t umma_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
-    return static_cast<uint64_t>((saddr >> 4) & 0x3FFFu) | (static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16) |
-           (static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46);
-}
-
-// Instruction descriptor of kind::f16 with fp32 accumulation: operand format
-// (0 fp16, 1 bf16) for A and B, their majorness (0 K, 1 M/N), N / 8 and M / 16.
-template <typename T>
-__host__ __device__ constexpr uint32_t umma_idesc(int M, int N, int a_mn, int b_mn) {
-    const uint32_t fmt = std::is_same<T, __half>::value ? 0u : 1u;
-    return (1u << 4) | (fmt << 7) | (fmt << 10) | (static_cast<uint32_t>(a_mn) << 15) |
-           (static_cast<uint32_t>(b_mn) << 16) | (static_cast<uint32_t>(N >> 3) << 17) |
-           (static_cast<uint32_t>(M >> 4) << 24);
-}
-
-__device__ __forceinline__ void umma_f16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc, bool accum) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
-        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accum ? 1 : 0));
-}
-
-__device__ __forceinline__ void umma_commit(uint32_t mbar) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(mbar) : "memory");
-}
-
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-
-// 32 consecutive fp32 accumulator columns of this thread's TMEM lane.
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t* r) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
-          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-        : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-}
-
+constexpr unsigned kLinStatusTimeout = 1u;  // a wait gave up (status word)
 // ---------------------------------------------------------------------------
 // tcgen05 products fed by TMA, warp-specialised.  Warp 4 (one lane) loads the
 // stages with TMA, warp 5 (one lane) issues the MMAs, warps 0-3 read the
@@ -148,42 +97,6 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t* r) {
 // ---------------------------------------------------------------------------
 constexpr int kQThreads = 192;  // 4 epilogue warps, the TMA warp, the MMA warp
 constexpr int kQProducer = 4, kQMma = 5;
-
-__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
-    return umma_desc(saddr, lbo, sbo) | (2ull << 61);  // layout type SWIZZLE_128B
-}
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t mbar) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
-            dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(mbar)
-        : "memory");
-}
-__device__ __forceinline__ void mbar_init(uint32_t mbar, int count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(mbar), "r"(count));
-}
-__device__ __forceinline__ void mbar_expect_tx(uint32_t mbar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(mbar), "r"(bytes) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint32_t mbar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(mbar) : "memory");
-}
-// Bounded wait for the phase of parity `parity`; stops early once *abort is set.
-__device__ __forceinline__ bool mbar_wait_or(uint32_t mbar, uint32_t parity, volatile int* abort) {
-    for (int i = 0; i < kTWaitSpins; ++i) {
-        uint32_t done;
-        asm volatile(
-            "{\n\t.reg .pred P1;\n\tmbarrier.try_wait.parity.shared::cta.b64 P1, [%1], %2;\n\t"
-            "selp.b32 %0, 1, 0, P1;\n\t}"
-            : "=r"(done)
-            : "r"(mbar), "r"(parity)
-            : "memory");
-        if (done) return true;
-        if ((i & 63) == 63 && *abort) return false;
-    }
-    *abort = 1;
-    return false;
-}
 
 __device__ __forceinline__ void red_add4(float* dst, float a, float b, float c, float d) {
     asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(a), "f"(b), "f"(c), "f"(d) : "memory");
