@@ -31,6 +31,11 @@ workloads) against the producer as a separate library GEMM (cuBLAS) followed
 by dcn4_forward; and the layer's backward dcn4_backward_linear (the
 aggregation's backward, then grad_x = g W, grad_W = g^T x, grad_b on the
 tensor cores in libdcn4) against dcn4_backward followed by cuBLAS products.
+The "projection" object (also skipped with --no-linear) times the output
+projection fused behind the operator (dcn4_forward_proj: y = core W^T + b per
+tile on the tensor cores, W [C, C]) against dcn4_forward followed by cuBLAS's
+linear layer, and dcn4_backward_proj against cuBLAS products followed by
+dcn4_backward.
 
 --profile runs warm-up + steps untimed passes of the workload (forward and
 backward; with --linear also the fused forward and dcn4_backward_linear) and
@@ -547,6 +552,7 @@ def run_native(args, w: gen.Workload) -> dict:
         result["e2e"] = e2e
     if not args.no_linear:
         result["linear"] = linear_leg(w, v, gy, p, flush, stream, dev, world)
+        result["projection"] = proj_leg(w, v, om, p, flush, stream, dev, world)
     if not args.no_per_config:
         sampler = ClockSampler(local if world > 1 else torch.cuda.current_device())
         sampler.start()
@@ -819,10 +825,105 @@ def linear_leg(w: gen.Workload, v, gy, p, flush, stream, dev, world: int) -> dic
     return res
 
 
+def proj_leg(w: gen.Workload, v, om, p, flush, stream, dev, world: int) -> dict:
+    """µs per call (CUDA events, L2 flushed before each, max over ranks): the forward
+    with the output projection fused behind it (dcn4_forward_proj, Cout = C), with and
+    without storing the core output, against dcn4_forward followed by cuBLAS's linear
+    layer; and dcn4_backward_proj against cuBLAS products for the projection's
+    gradients followed by dcn4_backward."""
+    import numpy as np
+    import torch
+    import deformable_convolution_sampling_b200 as dcn
+    tdt = {"f16": torch.float16, "bf16": torch.bfloat16}.get(w.dtype)
+    if tdt is None:
+        return {"unavailable": "the fused projection takes fp16 or bf16"}
+    Cout = w.C
+    if dcn.dcn4_forward_proj(p, Cout, None, None, None, None, None) == -5:
+        return {"unavailable": dcn.dcn4_last_error()}
+    pj = gen.make_proj_inputs(w, Cout)
+
+    def dev_t(a):
+        a = np.ascontiguousarray(a)
+        t = torch.from_numpy(a.view(np.int16)).view(tdt) if w.dtype == "bf16" else torch.from_numpy(a)
+        return t.to(dev)
+    wt, b, gy = dev_t(pj["weight"]), dev_t(pj["bias"]), dev_t(pj["grad_out"])
+    M = w.N * w.Ho * w.Wo
+    core = torch.empty((w.N, w.Ho, w.Wo, w.C), dtype=tdt, device=dev)
+    y = torch.empty((w.N, w.Ho, w.Wo, Cout), dtype=tdt, device=dev)
+    sh = stream.cuda_stream
+
+    def fused():
+        dcn.check(dcn.dcn4_forward_proj(p, Cout, v.data_ptr(), om.data_ptr(), wt.data_ptr(), b.data_ptr(),
+                                        y.data_ptr(), None, sh))
+
+    def fused_core():
+        dcn.check(dcn.dcn4_forward_proj(p, Cout, v.data_ptr(), om.data_ptr(), wt.data_ptr(), b.data_ptr(),
+                                        y.data_ptr(), core.data_ptr(), sh))
+
+    def unfused():
+        dcn.check(dcn.dcn4_forward(p, v.data_ptr(), om.data_ptr(), core.data_ptr(), sh))
+        torch.addmm(b, core.view(-1, w.C), wt.t(), out=y.view(-1, Cout))
+
+    def linear_only():
+        torch.addmm(b, core.view(-1, w.C), wt.t(), out=y.view(-1, Cout))
+
+    gv, gom = torch.empty_like(v), torch.empty_like(om)
+    gw, gb, gcore = torch.empty_like(wt), torch.empty_like(b), torch.empty_like(core)
+    nb = dcn.dcn4_backward_workspace_size(p)
+    nbp = dcn.dcn4_backward_proj_workspace_size(p, Cout)
+    ws = torch.empty(max(nbp, 16), dtype=torch.uint8, device=dev)
+    g2 = gy.view(-1, Cout)
+
+    def bwd_fused():
+        dcn.check(dcn.dcn4_backward_proj(p, Cout, v.data_ptr(), om.data_ptr(), core.data_ptr(), wt.data_ptr(),
+                                         gy.data_ptr(), gv.data_ptr(), gom.data_ptr(), gw.data_ptr(), gb.data_ptr(),
+                                         ws.data_ptr(), nbp, sh))
+
+    def bwd_only():
+        dcn.check(dcn.dcn4_backward(p, v.data_ptr(), om.data_ptr(), gcore.data_ptr(), gv.data_ptr(), gom.data_ptr(),
+                                    ws.data_ptr(), nb, sh))
+
+    def cublas_then_bwd():
+        torch.mm(g2, wt, out=gcore.view(-1, w.C))
+        torch.mm(g2.t(), core.view(-1, w.C), out=gw)
+        torch.sum(g2, 0, out=gb)
+        bwd_only()
+
+    res = {}
+    fused_core()
+    torch.cuda.synchronize(dev)
+    for name, fn in (("fused_us", fused), ("fused_with_core_out_us", fused_core),
+                     ("forward_then_cublas_us", unfused), ("cublas_linear_us", linear_only),
+                     ("backward_proj_us", bwd_fused), ("backward_us", bwd_only),
+                     ("cublas_then_backward_us", cublas_then_bwd)):
+        for _ in range(5):
+            fn()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(100)]
+        for e0, e1 in ev:
+            flush.zero_()
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+        torch.cuda.synchronize(dev)
+        res[name] = round(max_over_ranks(statistics.mean(a.elapsed_time(c) for a, c in ev) * 1e3, dev), 2)
+    res["speedup_vs_unfused"] = round(res["forward_then_cublas_us"] / res["fused_us"], 3)
+    res["backward_speedup_vs_unfused"] = round(res["cublas_then_backward_us"] / res["backward_proj_us"], 3)
+    res["gemm"] = (f"core [{M}, {w.C}] @ W^T [{w.C}, {Cout}] + b per tile: tcgen05.mma kind::f16 (M = 128 rows of W, "
+                   f"N = the tile's pixels, fp32 accumulator in tensor memory), core rows written to shared memory by "
+                   f"the sampling threads")
+    res["launches_per_call"] = 1
+    res["projection_backward_us"] = round(res["backward_proj_us"] - res["backward_us"], 2)
+    res["cublas_projection_backward_us"] = round(res["cublas_then_backward_us"] - res["backward_us"], 2)
+    del gv, gom, gw, gb, gcore, ws, core, y
+    return res
+
+
 def run_profile(args, w: gen.Workload) -> None:
     """--profile: warm-up + steps passes of the path (forward and backward of the
-    workload; with --linear the fused forward and dcn4_backward_linear too) with
-    no timing and no JSON line -- a short, fixed launch sequence for ncu captures."""
+    workload; with --linear the fused forward and dcn4_backward_linear too; with
+    --proj the forward with its fused output projection and dcn4_backward_proj)
+    with no timing and no JSON line -- a short, fixed launch sequence for ncu
+    captures."""
     import numpy as np
     import torch
     import deformable_convolution_sampling_b200 as dcn
@@ -841,6 +942,10 @@ def run_profile(args, w: gen.Workload) -> None:
     if args.linear:
         li = gen.make_linear_inputs(w, w.C)
         lin = dev_t(li["x"]), dev_t(li["weight"]), dev_t(li["bias"])
+    proj = None
+    if args.proj:
+        pj = gen.make_proj_inputs(w, w.C)
+        proj = dev_t(pj["weight"]), dev_t(pj["bias"]), dev_t(pj["grad_out"])
     for _ in range(args.warmup + args.steps):
         dcn.forward(p, v, om)
         dcn.backward(p, v, om, gy)
@@ -848,6 +953,10 @@ def run_profile(args, w: gen.Workload) -> None:
             om_lin = torch.empty_like(om)
             dcn.forward_linear(p, v, *lin, offset_mask_out=om_lin)
             dcn.backward_linear(p, v, om_lin, lin[0], lin[1], gy)
+        if proj is not None:
+            core = torch.empty((w.N, w.Ho, w.Wo, w.C), dtype=tdt, device=dev)
+            dcn.forward_proj(p, v, om, proj[0], proj[1], core_out=core)
+            dcn.backward_proj(p, v, om, core, proj[0], proj[2])
     torch.cuda.synchronize(dev)
     print(f"profile: {w.name}: {args.warmup + args.steps} passes done", flush=True)
 
@@ -866,6 +975,9 @@ def main(argv=None):
                          "dcn4_backward_linear)")
     ap.add_argument("--linear", action="store_true",
                     help="with --profile: also run the fused forward and dcn4_backward_linear")
+    ap.add_argument("--proj", action="store_true",
+                    help="with --profile: also run the forward with its fused output projection and "
+                         "dcn4_backward_proj")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-per-config", action="store_true",

@@ -39,6 +39,7 @@ _M2 = np.uint64(0x94D049BB133111EB)
 STREAM_VALUE, STREAM_OFFSET, STREAM_MASK, STREAM_GRAD = 1, 2, 3, 4
 STREAM_X, STREAM_WEIGHT, STREAM_BIAS = 5, 6, 7
 STREAM_REF = 8
+STREAM_PROJ_WEIGHT, STREAM_PROJ_BIAS, STREAM_PROJ_GRAD = 9, 10, 11
 
 
 def _splitmix64(z: np.ndarray) -> np.ndarray:
@@ -271,6 +272,25 @@ def make_linear_inputs(w: Workload, Cx: int, *, seed: int | None = None, bias: b
     out = {"x": x.reshape(w.N, w.Ho, w.Wo, Cx), "weight": weight, "bias": None}
     if bias:
         out["bias"] = to_storage(draw(("normal", 0.0, 0.1), seed, STREAM_BIAS, w.P), dtype)
+    return out
+
+
+def make_proj_inputs(w: Workload, Cout: int, *, seed: int | None = None, bias: bool = True,
+                     with_grad: bool = True, dtype: str | None = None) -> dict:
+    """The output projection behind the aggregation, in storage form: weight
+    [Cout, C] ~ N(0, 1 / C) (so each output has about the spread of one core
+    channel), bias [Cout] ~ N(0, 0.1^2) (or None) and, with_grad, the upstream
+    gradient of its output grad_out [N, Ho, Wo, Cout] drawn like the workload's own."""
+    seed = w.seed if seed is None else seed
+    dtype = w.dtype if dtype is None else dtype
+    z = draw(("normal", 0.0, 1.0), seed, STREAM_PROJ_WEIGHT, Cout * w.C).reshape(Cout, w.C)
+    out = {"weight": to_storage(z / np.sqrt(w.C), dtype), "bias": None}
+    if bias:
+        out["bias"] = to_storage(draw(("normal", 0.0, 0.1), seed, STREAM_PROJ_BIAS, Cout), dtype)
+    if with_grad:
+        ng = w.N * w.Ho * w.Wo * Cout
+        out["grad_out"] = to_storage(draw(w.grad_out, seed, STREAM_PROJ_GRAD, ng), dtype).reshape(
+            w.N, w.Ho, w.Wo, Cout)
     return out
 
 

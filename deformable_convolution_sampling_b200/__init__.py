@@ -113,6 +113,10 @@ def _load() -> ctypes.CDLL:
         "dcn4_backward_diagnostics": ([P, vp, ctypes.c_size_t, ip, vp], ctypes.c_int),
         "dcn4_backward_linear_workspace_size": ([P, ctypes.c_int], ctypes.c_size_t),
         "dcn4_backward_linear": ([P, ctypes.c_int] + [vp] * 11 + [ctypes.c_size_t, vp], ctypes.c_int),
+        "dcn4_forward_proj": ([P, ctypes.c_int, vp, vp, vp, vp, vp, vp, vp], ctypes.c_int),
+        "dcn4_forward_tc_status": ([ctypes.c_int], ctypes.c_int),
+        "dcn4_backward_proj_workspace_size": ([P, ctypes.c_int], ctypes.c_size_t),
+        "dcn4_backward_proj": ([P, ctypes.c_int] + [vp] * 10 + [ctypes.c_size_t, vp], ctypes.c_int),
         "dcn4_attn_check_params": ([AP], ctypes.c_int),
         "dcn4_attn_forward": ([AP, vp, vp, vp, vp, vp], ctypes.c_int),
         "dcn4_attn_backward_workspace_size": ([AP], ctypes.c_size_t),
@@ -162,6 +166,26 @@ def dcn4_forward(p: dcn4_params, value, offset_mask, out, stream=None) -> int:
 def dcn4_forward_linear(p: dcn4_params, Cx: int, value, x, weight, bias, out, offset_mask_out=None,
                         stream=None) -> int:
     return lib.dcn4_forward_linear(ctypes.byref(p), int(Cx), value, x, weight, bias, out, offset_mask_out, stream)
+
+
+def dcn4_forward_proj(p: dcn4_params, Cout: int, value, offset_mask, weight, bias, out, core_out=None,
+                      stream=None) -> int:
+    return lib.dcn4_forward_proj(ctypes.byref(p), int(Cout), value, offset_mask, weight, bias, out, core_out, stream)
+
+
+def dcn4_forward_tc_status(reset: bool = False) -> int:
+    return lib.dcn4_forward_tc_status(1 if reset else 0)
+
+
+def dcn4_backward_proj_workspace_size(p: dcn4_params, Cout: int) -> int:
+    return lib.dcn4_backward_proj_workspace_size(ctypes.byref(p), int(Cout))
+
+
+def dcn4_backward_proj(p: dcn4_params, Cout: int, value, offset_mask, core_out, weight, grad_out, grad_value,
+                       grad_offset_mask, grad_weight, grad_bias, workspace, workspace_bytes: int, stream=None) -> int:
+    return lib.dcn4_backward_proj(ctypes.byref(p), int(Cout), value, offset_mask, core_out, weight, grad_out,
+                                  grad_value, grad_offset_mask, grad_weight, grad_bias, workspace, workspace_bytes,
+                                  stream)
 
 
 def dcn4_backward_workspace_size(p: dcn4_params) -> int:
@@ -350,6 +374,52 @@ def backward_linear(p: dcn4_params, value, offset_mask, x, weight, grad_out, wit
     return gv, gom, gx, gw, gb
 
 
+def forward_proj(p: dcn4_params, value, offset_mask, weight, bias=None, out=None, core_out=None):
+    """y[N,Ho,Wo,Cout] = (aggregation of value at offset_mask) @ weight.T + bias, the
+    projection formed inside the forward kernel (weight [Cout,C], bias [Cout] or None);
+    core_out, when given ([N,Ho,Wo,C]), receives the aggregation's own output.  CUDA
+    tensors, fp16 or bf16."""
+    import torch
+    st, Ho, Wo = dcn4_output_dims(p)
+    check(st)
+    Cout = weight.shape[0]
+    if out is None:
+        out = torch.empty((p.N, Ho, Wo, Cout), dtype=_torch_dtype(p.dtype), device=value.device)
+    check(dcn4_forward_proj(p, Cout, value.data_ptr(), offset_mask.data_ptr(), weight.data_ptr(),
+                            bias.data_ptr() if bias is not None else None, out.data_ptr(),
+                            core_out.data_ptr() if core_out is not None else None, _stream_handle(value.device)))
+    return out
+
+
+def backward_proj(p: dcn4_params, value, offset_mask, core_out, weight, grad_out, with_bias: bool = True,
+                  want_weight: bool = True, workspace=None):
+    """Backward of forward_proj for CUDA tensors (core_out: the aggregation output the
+    forward saved): (grad_value, grad_offset_mask, grad_weight or None, grad_bias or
+    None), all computed in libdcn4."""
+    import torch
+    st, Ho, Wo = dcn4_output_dims(p)
+    check(st)
+    dt = _torch_dtype(p.dtype)
+    dev = value.device
+    Cout = weight.shape[0]
+    gv = torch.empty_like(value, dtype=dt)
+    gom = torch.empty((p.N, Ho, Wo, p.P), dtype=dt, device=dev)
+    gw = torch.empty_like(weight) if want_weight else None
+    gb = torch.empty((Cout,), dtype=dt, device=dev) if with_bias else None
+    need = dcn4_backward_proj_workspace_size(p, Cout)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+
+    def ptr(t):
+        return t.data_ptr() if t is not None else None
+
+    check(dcn4_backward_proj(p, Cout, value.data_ptr(), offset_mask.data_ptr(), ptr(core_out), weight.data_ptr(),
+                             grad_out.data_ptr(), gv.data_ptr(), gom.data_ptr(), ptr(gw), ptr(gb),
+                             workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                             _stream_handle(dev)))
+    return gv, gom, gw, gb
+
+
 def attn_forward(p: dcn4_attn_params, value, ref_points, offset_logits, out=None):
     """y[N,Nq,C] of single-scale deformable attention for CUDA tensors value [N,H,W,C],
     ref_points [N,Nq,2] (float32) and offset_logits [N,Nq,P]."""
@@ -458,6 +528,38 @@ def _autograd_function():
 
 _DCNV4_CORE = None
 _DCNV4_CORE_LINEAR = None
+_DCNV4_CORE_PROJ = None
+
+
+def _autograd_function_proj():
+    import torch
+
+    class DCNv4CoreProj(torch.autograd.Function):
+        """The aggregation with the output projection fused behind it as a
+        torch.autograd.Function.  Forward: dcn4_forward_proj, keeping the core output.
+        Backward: dcn4_backward_proj (the projection's gradients in libdcn4's
+        tensor-core kernels, then dcn4_backward with grad_core = grad_out W)."""
+
+        @staticmethod
+        def forward(ctx, value, offset_mask, weight, bias, p):
+            st, Ho, Wo = dcn4_output_dims(p)
+            check(st)
+            core = torch.empty((p.N, Ho, Wo, p.G * p.Cg), dtype=value.dtype, device=value.device)
+            y = forward_proj(p, value, offset_mask, weight, bias, core_out=core)
+            ctx.save_for_backward(value, offset_mask, weight, core)
+            ctx.p = p
+            ctx.has_bias = bias is not None
+            return y
+
+        @staticmethod
+        def backward(ctx, grad_out):
+            value, offset_mask, weight, core = ctx.saved_tensors
+            grad_value, grad_om, grad_w, grad_b = backward_proj(
+                ctx.p, value, offset_mask, core, weight, grad_out.contiguous(), with_bias=ctx.has_bias,
+                want_weight=ctx.needs_input_grad[2])
+            return grad_value, grad_om, grad_w, grad_b, None
+
+    return DCNv4CoreProj
 
 
 def _autograd_function_linear():
@@ -530,6 +632,28 @@ def dcnv4_core_linear(value, x, weight, bias=None, *, group: int, kernel=3, stri
     if _DCNV4_CORE_LINEAR is None:
         _DCNV4_CORE_LINEAR = _autograd_function_linear()
     return _DCNV4_CORE_LINEAR.apply(value, x, weight, bias, p)
+
+
+def dcnv4_core_proj(value, offset_mask, weight, bias=None, *, group: int, kernel=3, stride=1, pad=1, dilation=1,
+                    offset_scale: float = 1.0, remove_center: bool = False, softmax: bool = False):
+    """y = (DCNv4 core aggregation of value [N,H,W,C] at offset_mask [N,Ho,Wo,P]) @ weight.T
+    + bias, the output projection (weight [Cout,C], bias [Cout] or None; fp16/bf16)
+    formed inside the forward kernel; differentiable in value, offset_mask, weight and
+    bias (torch.autograd)."""
+    global _DCNV4_CORE_PROJ
+    p = params_for_tensors(value, offset_mask, group=group, kernel=kernel, stride=stride, pad=pad,
+                           dilation=dilation, offset_scale=offset_scale, remove_center=remove_center,
+                           softmax=softmax)
+    if weight.dim() != 2 or weight.shape[1] != value.shape[-1]:
+        raise ValueError("weight must be [Cout, C]")
+    if bias is not None and tuple(bias.shape) != (weight.shape[0],):
+        raise ValueError("bias must be [Cout]")
+    for name, t in (("weight", weight),) + ((("bias", bias),) if bias is not None else ()):
+        if t.dtype != value.dtype or not t.is_contiguous() or t.device != value.device:
+            raise ValueError(f"{name} must be contiguous, on value's device and of value's dtype")
+    if _DCNV4_CORE_PROJ is None:
+        _DCNV4_CORE_PROJ = _autograd_function_proj()
+    return _DCNV4_CORE_PROJ.apply(value, offset_mask, weight, bias, p)
 
 
 class _OffsetMaskShape:

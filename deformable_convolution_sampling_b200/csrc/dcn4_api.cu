@@ -397,6 +397,41 @@ int dcn4_forward_linear(const dcn4_params* p, int Cx, const void* value, const v
     return DCN4_OK;
 }
 
+int dcn4_forward_proj(const dcn4_params* p, int Cout, const void* value, const void* offset_mask, const void* weight,
+                      const void* bias, void* out, void* core_out, void* stream) {
+    dcn4::Geometry g;
+    const int st = make_geometry(p, false, aligned32(value), &g);
+    if (st != DCN4_OK) return st;
+    if (p->dtype == DCN4_F32) return fail(DCN4_ERR_UNSUPPORTED, "the fused output projection takes fp16 or bf16");
+    if (Cout < 16 || Cout % 16 != 0 || Cout > (1 << 16))
+        return fail(DCN4_ERR_BAD_SHAPE, "Cout=%d must be a positive multiple of 16", Cout);
+    if (Cout > 128) return fail(DCN4_ERR_UNSUPPORTED, "the fused projection forms at most 128 outputs (Cout=%d)", Cout);
+    if (!dcn4::forward_proj_shape_ok(g, Cout))
+        return fail(DCN4_ERR_UNSUPPORTED,
+                    "the fused projection needs C a multiple of 64 up to 256 and 16-, 32- or 64-pixel tiles "
+                    "(C=%d, G=%d: %d-pixel tiles)",
+                    g.C, p->G, g.pix_per_cta);
+    if (dcn4::forward_proj_smem_bytes(g, Cout) > kSmemMax)
+        return fail(DCN4_ERR_UNSUPPORTED, "P=%d rows with C=%d do not fit shared memory", p->P, g.C);
+    if (g.total_pix == 0) return DCN4_OK;
+    if (!value || !offset_mask || !weight || !out)
+        return fail(DCN4_ERR_NULL, "value, offset_mask, weight and out must be non-NULL");
+    if (!aligned16(value) || !aligned16(offset_mask) || !aligned16(weight) || !aligned16(out) || !aligned16(bias) ||
+        !aligned16(core_out))
+        return fail(DCN4_ERR_MISALIGNED, "every pointer must be 16-byte aligned");
+    const cudaError_t e = dcn4::launch_forward_proj(g, p->dtype, value, offset_mask, weight, bias, out, core_out, Cout,
+                                                    static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return fail(DCN4_ERR_LAUNCH, "forward_proj launch: %s", cudaGetErrorString(e));
+    return DCN4_OK;
+}
+
+int dcn4_forward_tc_status(int reset) {
+    unsigned v = 0u;
+    const cudaError_t e = dcn4::forward_tc_status(&v, reset != 0);
+    if (e != cudaSuccess) return fail(DCN4_ERR_LAUNCH, "reading the forward status word: %s", cudaGetErrorString(e));
+    return static_cast<int>(v & 0x7fffffffu);
+}
+
 size_t dcn4_backward_workspace_size(const dcn4_params* p) {
     dcn4::Geometry g;
     if (make_geometry(p, true, true, &g) != DCN4_OK) return 0;
@@ -513,6 +548,66 @@ int dcn4_backward_linear(const dcn4_params* p, int Cx, const void* value, const 
                                                        grad_x, grad_weight, grad_bias, acc, s);
     if (e != cudaSuccess) return fail(DCN4_ERR_LAUNCH, "linear backward launch: %s", cudaGetErrorString(e));
     return DCN4_OK;
+}
+
+size_t dcn4_backward_proj_workspace_size(const dcn4_params* p, int Cout) {
+    dcn4::Geometry g;
+    if (make_geometry(p, true, true, &g) != DCN4_OK || Cout < 1 || static_cast<long long>(Cout) * g.C >= (1LL << 31))
+        return 0;
+    const size_t b = dcn4_backward_workspace_size(p);
+    if (b == 0) return 0;
+    const size_t core = static_cast<size_t>(g.total_pix) * g.C * static_cast<size_t>(elem_bytes(p->dtype));
+    return round256(b) + round256(core) + round256(dcn4::linear_backward_workspace_bytes(Cout, g.C));
+}
+
+int dcn4_backward_proj(const dcn4_params* p, int Cout, const void* value, const void* offset_mask,
+                       const void* core_out, const void* weight, const void* grad_out, void* grad_value,
+                       void* grad_offset_mask, void* grad_weight, void* grad_bias, void* workspace,
+                       size_t workspace_bytes, void* stream) {
+    dcn4::Geometry g;
+    const int st = make_geometry(p, true, false, &g);
+    if (st != DCN4_OK) return st;
+    if (p->dtype == DCN4_F32) return fail(DCN4_ERR_UNSUPPORTED, "the output projection takes fp16 or bf16");
+    if (Cout < 16 || Cout % 16 != 0 || Cout > (1 << 16))
+        return fail(DCN4_ERR_BAD_SHAPE, "Cout=%d must be a positive multiple of 16", Cout);
+    if (g.C % 16 != 0) return fail(DCN4_ERR_BAD_SHAPE, "C=%d must be a multiple of 16", g.C);
+    if (static_cast<long long>(Cout) * g.C >= (1LL << 31) || g.total_pix >= (1LL << 31))
+        return fail(DCN4_ERR_UNSUPPORTED, "too large (N*Ho*Wo and Cout*C must be < 2^31)");
+    if (!aligned16(core_out) || !aligned16(weight) || !aligned16(grad_out) || !aligned16(grad_weight) ||
+        !aligned16(grad_bias))
+        return fail(DCN4_ERR_MISALIGNED, "every pointer must be 16-byte aligned");
+    const size_t need = dcn4_backward_proj_workspace_size(p, Cout);
+    if (!workspace || workspace_bytes < need)
+        return fail(DCN4_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, workspace_bytes);
+    if (!aligned16(workspace)) return fail(DCN4_ERR_MISALIGNED, "workspace must be 16-byte aligned");
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t eb = static_cast<size_t>(elem_bytes(p->dtype));
+    if (g.total_pix == 0) {
+        // no output pixels: the weight and bias gradients are empty sums
+        cudaError_t e = cudaSuccess;
+        if (grad_weight) e = cudaMemsetAsync(grad_weight, 0, static_cast<size_t>(Cout) * g.C * eb, s);
+        if (e == cudaSuccess && grad_bias) e = cudaMemsetAsync(grad_bias, 0, static_cast<size_t>(Cout) * eb, s);
+        if (e != cudaSuccess) return fail(DCN4_ERR_LAUNCH, "zeroing grad_weight/grad_bias: %s", cudaGetErrorString(e));
+        return DCN4_OK;
+    }
+    // everything the aggregation's backward checks, before the first launch
+    if (!value || !offset_mask || !weight || !grad_out || !grad_value || !grad_offset_mask)
+        return fail(DCN4_ERR_NULL,
+                    "value, offset_mask, weight, grad_out, grad_value and grad_offset_mask must be non-NULL");
+    if (!aligned16(value) || !aligned16(offset_mask) || !aligned16(grad_value) || !aligned16(grad_offset_mask))
+        return fail(DCN4_ERR_MISALIGNED, "every pointer must be 16-byte aligned");
+    if (grad_weight && !core_out) return fail(DCN4_ERR_NULL, "grad_weight needs core_out");
+    // [core backward workspace][grad of the core output, N*Ho*Wo*C][grad_W / grad_b accumulators]
+    const size_t core_ws = round256(dcn4_backward_workspace_size(p));
+    const size_t gcore_bytes = round256(static_cast<size_t>(g.total_pix) * g.C * eb);
+    void* gcore = static_cast<char*>(workspace) + core_ws;
+    float* acc = reinterpret_cast<float*>(static_cast<char*>(workspace) + core_ws + gcore_bytes);
+    // the projection's gradients first: grad_core = grad_out W (rounded to the dtype, as the
+    // unfused pair would store it), grad_W = grad_out^T core_out, grad_b = column sums of grad_out
+    const cudaError_t e = dcn4::launch_linear_backward(p->dtype, g.total_pix, Cout, g.C, core_out, weight, grad_out,
+                                                       gcore, grad_weight, grad_bias, acc, s);
+    if (e != cudaSuccess) return fail(DCN4_ERR_LAUNCH, "projection backward launch: %s", cudaGetErrorString(e));
+    return dcn4_backward(p, value, offset_mask, gcore, grad_value, grad_offset_mask, workspace, core_ws, stream);
 }
 
 int dcn4_attn_check_params(const dcn4_attn_params* p) {

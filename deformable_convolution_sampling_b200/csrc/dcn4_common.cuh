@@ -371,6 +371,17 @@ cudaError_t launch_forward_linear(const Geometry& g, int dtype, const void* valu
 size_t forward_linear_smem_bytes(const Geometry& g, int Cx, int mode);
 // The fused forward's producer mode for this shape.
 int forward_linear_mode(const Geometry& g, int Cx);
+// Forward with the output projection behind the sampler (16-bit dtypes): out =
+// core W^T + b per tile, w [Cout, C], b [Cout] or null, core_out [N, Ho, Wo, C]
+// or null.  Shapes: 16-, 32- or 64-pixel tiles, C a multiple of 64 up to 256,
+// Cout a multiple of 16 up to 128 (forward_proj_shape_ok).
+bool forward_proj_shape_ok(const Geometry& g, int Cout);
+size_t forward_proj_smem_bytes(const Geometry& g, int Cout);
+cudaError_t launch_forward_proj(const Geometry& g, int dtype, const void* value, const void* om, const void* w,
+                                const void* b, void* out, void* core_out, int Cout, cudaStream_t stream);
+// The status word of the forward's tcgen05 paths (producer and projection):
+// nonzero once a bounded wait gave up.  Synchronous; reset clears it.
+cudaError_t forward_tc_status(unsigned* status, bool reset);
 // Gradients of the linear producer from gom = grad_offset_mask as an [M, P]
 // matrix (16-bit dtypes): gx = gom W [M, Cx], gw = gom^T x [P, Cx], gb = column
 // sums of gom [P]; any of the three may be null.  ws: fp32 scratch of

@@ -64,7 +64,9 @@ __device__ __forceinline__ void accumulate(float2* acc, const T* src, float wt) 
 constexpr int kFwdCtasPerSm = 3;
 
 // Arguments of the fused producer: x [N, Ho, Wo, Cx], w [P, Cx] (nn.Linear
-// layout), b [P] or null, om_out [N, Ho, Wo, P] or null.
+// layout), b [P] or null, om_out [N, Ho, Wo, P] or null; and of the fused
+// output projection: pw [Cout, C], pb [Cout] or null, core_out [N, Ho, Wo, C]
+// (the aggregation's own output) or null.
 template <typename T>
 struct LinearArgs {
     const T* x;
@@ -74,6 +76,10 @@ struct LinearArgs {
     int Cx;
     int w_smem;  // 1: W is staged in shared memory once per CTA (when it fits)
     int tc;      // 1: the offset_mask tile is formed on tcgen05 (see stage_x_swizzled)
+    const T* pw;
+    const T* pb;
+    T* core_out;
+    int Cout;
 };
 
 // tcgen05 form of the producer: D^T[p][pixel] = W x^T with M = 128 rows of W
@@ -87,6 +93,17 @@ constexpr int kTcRows = 128, kTcPix = 64;
 __host__ __device__ inline int tc_x_bytes(int Cx) { return kTcPix * Cx * 2; }
 __host__ __device__ inline int tc_w_bytes(int Cx) { return kTcRows * Cx * 2; }
 __device__ unsigned g_fwd_linear_status;  // nonzero once a bounded wait of the tcgen05 producer gave up
+
+// Output projection y = core W_out^T + b_out fused behind the sampler (PROJ): per
+// tile D^T[o][pixel] = W_out core^T with M = 128 rows of W_out (Cout <= 128, the
+// rest zero), N = the tile's pixels (16, 32 or 64), K = C in 64-wide slabs; the
+// same swizzled K-major operand layout as the producer.  The core tile is written
+// by the sampling threads themselves (their fp32 sums rounded to the I/O dtype,
+// as the unfused pair stores them), the result read back into a [pixels][Cout]
+// staging tile and stored with 16-byte writes.
+__host__ __device__ inline int proj_core_bytes(const Geometry& g) { return g.pix_per_cta * g.C * 2; }
+__host__ __device__ inline int proj_w_bytes(const Geometry& g) { return kTcRows * g.C * 2; }
+__host__ __device__ inline int proj_tmem_cols(const Geometry& g) { return g.pix_per_cta < 32 ? 32 : g.pix_per_cta; }
 
 // Rows of a staged x tile: the tile's pixels rounded up to whole 16-row MMA tiles.
 __host__ __device__ inline int linear_rows(const Geometry& g) { return (g.TH * g.TW + 15) / 16 * 16; }
@@ -341,10 +358,12 @@ __device__ __forceinline__ void stage_tile_async(T* dst_smem, const T* src, cons
 // the current one.  KH, KW > 0: compile-time grid size (fully unrolled) and
 // RC = remove_center; KH = KW = 0: sizes and remove_center from g.  SM:
 // softmax over the K masks.  LIN: offset_mask rows from the linear producer.
-template <typename T, int VEC, int KH, int KW, bool RC, bool SM, bool LIN>
+// PROJ: the output projection behind the sampler (see proj_core_bytes).
+template <typename T, int VEC, int KH, int KW, bool RC, bool SM, bool LIN, bool PROJ>
 __global__ void __launch_bounds__(256, kFwdCtasPerSm) forward_kernel(const Geometry g, const T* __restrict__ value,
                                                       const T* __restrict__ om, T* __restrict__ out,
                                                       const LinearArgs<T> lin) {
+    static_assert(!(LIN && PROJ), "the producer and the projection are separate instantiations");
     extern __shared__ __align__(16) unsigned char smem[];
     constexpr int EPV = Elem<T>::per16;
     constexpr int PAIRS = VEC * EPV / 2;
@@ -382,9 +401,46 @@ __global__ void __launch_bounds__(256, kFwdCtasPerSm) forward_kernel(const Geome
         bufs[1] = bufs[0] + tile_elems;
         e_s = reinterpret_cast<float*>(bufs[1] + tile_elems);
     }
+    // PROJ: the swizzled core tile and W_out (1024-byte aligned), the [pixels][Cout]
+    // result tile and the bias (fp32), after the exponentials
+    uint32_t pj_a = 0u, pj_w = 0u;
+    T* pj_o = nullptr;
+    float* pj_b = nullptr;
+    if constexpr (PROJ) {
+        const uint32_t end = sbase + static_cast<uint32_t>(2 * tile_elems * sizeof(T)) +
+                             (SM ? static_cast<uint32_t>(g.K * blockDim.x * sizeof(float)) : 0u);
+        pj_a = (end + 1023u) & ~1023u;
+        pj_w = pj_a + proj_core_bytes(g);
+        pj_o = reinterpret_cast<T*>(smem + (pj_w - sbase) + proj_w_bytes(g));
+        pj_b = reinterpret_cast<float*>(pj_o + g.pix_per_cta * lin.Cout);
+    }
     const int ntiles = g.N * g.tiles_h * g.tiles_w;
     int tile = blockIdx.x;
     if (tile >= ntiles) return;
+    if constexpr (PROJ) {
+        for (int j = threadIdx.x; j < lin.Cout; j += blockDim.x) pj_b[j] = lin.pb ? to_f32(lin.pb[j]) : 0.f;
+        // W_out rows [Cout][C] into 64-wide swizzled slabs; rows Cout..127 zero (their results are never read)
+        const int cpr = g.C / 8;
+        for (int i = threadIdx.x; i < kTcRows * cpr; i += blockDim.x) {
+            const int r = i / cpr, c = i - r * cpr;
+            uint4 v = make_uint4(0u, 0u, 0u, 0u);
+            if (r < lin.Cout) v = ld_gather(lin.pw + static_cast<long long>(r) * g.C + c * 8);
+            *reinterpret_cast<uint4*>(smem + (pj_w - sbase) + (c >> 3) * (kTcRows * 128) + r * 128 +
+                                      (((c & 7) ^ (r & 7)) << 4)) = v;
+        }
+        if (threadIdx.x == 0) {
+            tc::mbar_init(tc::smem_u32(&tc_mbar), 1);
+            tc_abort = 0;
+            asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        }
+        if (threadIdx.x < 32) {  // proj_tmem_cols fp32 columns x 128 lanes: the accumulator
+            asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                             tc::smem_u32(&tc_taddr)),
+                         "r"(proj_tmem_cols(g)));
+            asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+        }
+        tc::tc_fence_before();
+    }
     if constexpr (LIN) {
         for (int j = threadIdx.x; j < g.P; j += blockDim.x) b_s[j] = lin.b ? to_f32(lin.b[j]) : 0.f;
         if (lin.tc) {
@@ -614,14 +670,92 @@ __global__ void __launch_bounds__(256, kFwdCtasPerSm) forward_kernel(const Geome
                     }
                 }
             }
-            T* dst = out + ((static_cast<long long>(t.n) * g.Ho + ho) * g.Wo + wo) * g.C + ch_off;
-            if constexpr (VEC == 2) {
-                st_global32(dst, pack(acc, T()), pack(acc + EPV / 2, T()));
+            const long long o_off = ((static_cast<long long>(t.n) * g.Ho + ho) * g.Wo + wo) * g.C + ch_off;
+            if constexpr (PROJ) {
+                // the rounded sums into row lp of the swizzled core tile, 8 channels a chunk
+#pragma unroll
+                for (int v = 0; v < VEC; ++v) {
+                    const uint4 q = pack(acc + v * (EPV / 2), T());
+                    const int c = ch_off / 8 + v;
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(
+                                     pj_a + (c >> 3) * (g.pix_per_cta * 128) + lp * 128 + (((c & 7) ^ (lp & 7)) << 4)),
+                                 "r"(q.x), "r"(q.y), "r"(q.z), "r"(q.w)
+                                 : "memory");
+                    if (lin.core_out) st_global(lin.core_out + o_off + v * EPV, q);
+                }
+            } else if constexpr (VEC == 2) {
+                st_global32(out + o_off, pack(acc, T()), pack(acc + EPV / 2, T()));
             } else {
-                st_global(dst, pack(acc, T()));
+                st_global(out + o_off, pack(acc, T()));
+            }
+        } else if (PROJ && lp < g.pix_per_cta) {
+            // a pixel past the image edge: its row is zero (its column of the result is not stored)
+#pragma unroll
+            for (int v = 0; v < VEC; ++v) {
+                const int c = ch_off / 8 + v;
+                asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(
+                                 pj_a + (c >> 3) * (g.pix_per_cta * 128) + lp * 128 + (((c & 7) ^ (lp & 7)) << 4)),
+                             "r"(0u)
+                             : "memory");
+            }
+        }
+        if constexpr (PROJ) {
+            // the core tile is complete: one thread issues the MMAs, all wait, then the warps read the
+            // accumulator back (warp w: TMEM lanes = rows o 32 (w % 4) .. + 31, pixel columns 32 (w / 4) ..)
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            __syncthreads();
+            const uint32_t tmem = tc_taddr;
+            const int npix = g.pix_per_cta;
+            if (threadIdx.x == 0) {
+                tc::tc_fence_after();
+                const uint32_t idesc = tc::umma_idesc<T>(kTcRows, npix, 0, 0);
+                for (int sb = 0; sb < g.C / 64; ++sb)
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        tc::umma_f16(tmem, tc::umma_desc_sw128(pj_w + sb * (kTcRows * 128) + q * 32, 16, 1024),
+                                     tc::umma_desc_sw128(pj_a + sb * (npix * 128) + q * 32, 16, 1024), idesc,
+                                     sb > 0 || q > 0);
+                tc::umma_commit(tc::smem_u32(&tc_mbar));
+            }
+            tc::mbar_wait_or(tc::smem_u32(&tc_mbar), static_cast<uint32_t>(it) & 1u, &tc_abort);
+            tc::tc_fence_after();
+            const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+            const int sub = warp & 3, half = warp >> 2;
+            const int o = 32 * sub + lane;
+            for (int j0 = half * 32; j0 < half * 32 + 32 && j0 < npix; j0 += 16) {  // whole warps
+                uint32_t acc16[16];
+                tc::tmem_ld16(tmem + (static_cast<uint32_t>(32 * sub) << 16) + j0, acc16);
+                if (o < lin.Cout && !tc_abort) {
+                    const float bo = pj_b[o];
+#pragma unroll
+                    for (int j = 0; j < 16; ++j)
+                        pj_o[(j0 + j) * lin.Cout + o] = from_f32<T>(__uint_as_float(acc16[j]) + bo);
+                }
+            }
+            tc::tc_fence_before();  // the next tile's MMAs overwrite the accumulator after the next barrier
+            __syncthreads();
+            if (tc_abort) {  // a wait gave up: no further tile is formed
+                if (threadIdx.x == 0) atomicOr(&g_fwd_linear_status, 1u);
+                break;
+            }
+            const int cpp = lin.Cout / EPV;  // the tile's y rows, 16-byte stores
+            for (int i = threadIdx.x; i < t.th * t.tw * cpp; i += blockDim.x) {
+                const int q = i / cpp, c = i - q * cpp;
+                const int qy = q / t.tw, qx = q - qy * t.tw;
+                const long long pix = (static_cast<long long>(t.n) * g.Ho + t.ho0 + qy) * g.Wo + t.wo0 + qx;
+                st_global(out + pix * lin.Cout + c * EPV,
+                          *reinterpret_cast<const uint4*>(pj_o + (qy * g.TW + qx) * lin.Cout + c * EPV));
             }
         }
         __syncthreads();  // the buffer is refilled two tiles later (LIN: om_s at the next tile)
+    }
+    if constexpr (PROJ) {
+        asm volatile("cp.async.wait_group 0;" ::: "memory");
+        tc::tc_fence_before();
+        __syncthreads();
+        if (threadIdx.x < 32)
+            asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tc_taddr),
+                         "r"(proj_tmem_cols(g)));
     }
     if constexpr (LIN) {
         if (lin.tc) {
@@ -634,12 +768,13 @@ __global__ void __launch_bounds__(256, kFwdCtasPerSm) forward_kernel(const Geome
     }
 }
 
-template <typename T, int VEC, int KH, int KW, bool RC, bool SM, bool LIN>
+template <typename T, int VEC, int KH, int KW, bool RC, bool SM, bool LIN, bool PROJ>
 cudaError_t launch_typed(const Geometry& g, const void* value, const void* om, void* out, const LinearArgs<T>& lin,
                          cudaStream_t stream) {
-    const size_t smem = LIN ? forward_linear_smem_bytes(g, lin.Cx, lin.tc ? 2 : lin.w_smem ? 1 : 0)
-                            : forward_smem_bytes(g, sizeof(T));
-    auto kern = forward_kernel<T, VEC, KH, KW, RC, SM, LIN>;
+    const size_t smem = LIN    ? forward_linear_smem_bytes(g, lin.Cx, lin.tc ? 2 : lin.w_smem ? 1 : 0)
+                        : PROJ ? forward_proj_smem_bytes(g, lin.Cout)
+                               : forward_smem_bytes(g, sizeof(T));
+    auto kern = forward_kernel<T, VEC, KH, KW, RC, SM, LIN, PROJ>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     const int threads = (g.pix_per_cta * g.G * g.nslice + 31) / 32 * 32;
@@ -657,28 +792,28 @@ cudaError_t launch_typed(const Geometry& g, const void* value, const void* om, v
     return cudaGetLastError();
 }
 
-template <typename T, int VEC, bool SM, bool LIN>
+template <typename T, int VEC, bool SM, bool LIN, bool PROJ>
 cudaError_t launch_grid(const Geometry& g, const void* value, const void* om, void* out, const LinearArgs<T>& lin,
                         cudaStream_t stream) {
     if (g.kh == 3 && g.kw == 3) {
-        return g.remove_center ? launch_typed<T, VEC, 3, 3, true, SM, LIN>(g, value, om, out, lin, stream)
-                               : launch_typed<T, VEC, 3, 3, false, SM, LIN>(g, value, om, out, lin, stream);
+        return g.remove_center ? launch_typed<T, VEC, 3, 3, true, SM, LIN, PROJ>(g, value, om, out, lin, stream)
+                               : launch_typed<T, VEC, 3, 3, false, SM, LIN, PROJ>(g, value, om, out, lin, stream);
     }
-    return launch_typed<T, VEC, 0, 0, false, SM, LIN>(g, value, om, out, lin, stream);
+    return launch_typed<T, VEC, 0, 0, false, SM, LIN, PROJ>(g, value, om, out, lin, stream);
 }
 
-template <typename T, int VEC, bool LIN>
+template <typename T, int VEC, bool LIN, bool PROJ>
 cudaError_t launch_softmax(const Geometry& g, const void* value, const void* om, void* out, const LinearArgs<T>& lin,
                            cudaStream_t stream) {
-    return g.softmax ? launch_grid<T, VEC, true, LIN>(g, value, om, out, lin, stream)
-                     : launch_grid<T, VEC, false, LIN>(g, value, om, out, lin, stream);
+    return g.softmax ? launch_grid<T, VEC, true, LIN, PROJ>(g, value, om, out, lin, stream)
+                     : launch_grid<T, VEC, false, LIN, PROJ>(g, value, om, out, lin, stream);
 }
 
-template <typename T, bool LIN = false>
+template <typename T, bool LIN = false, bool PROJ = false>
 cudaError_t launch_vec(const Geometry& g, int vec, const void* value, const void* om, void* out,
                        const LinearArgs<T>& lin, cudaStream_t stream) {
-    return vec == 2 ? launch_softmax<T, 2, LIN>(g, value, om, out, lin, stream)
-                    : launch_softmax<T, 1, LIN>(g, value, om, out, lin, stream);
+    return vec == 2 ? launch_softmax<T, 2, LIN, PROJ>(g, value, om, out, lin, stream)
+                    : launch_softmax<T, 1, LIN, PROJ>(g, value, om, out, lin, stream);
 }
 
 }  // namespace
@@ -725,6 +860,49 @@ cudaError_t launch_forward_linear(const Geometry& g, int dtype, const void* valu
         }
         default: return cudaErrorInvalidValue;
     }
+}
+
+bool forward_proj_shape_ok(const Geometry& g, int Cout) {
+    const int npix = g.pix_per_cta;
+    return (npix == 16 || npix == 32 || npix == 64) && g.TH * g.TW == npix && g.C % 64 == 0 && g.C <= 256 &&
+           Cout >= 16 && Cout % 16 == 0 && Cout <= kTcRows && samples_threads(g) == npix * g.G * g.nslice;
+}
+
+size_t forward_proj_smem_bytes(const Geometry& g, int Cout) {
+    return forward_smem_bytes(g, 2) + 1024 + proj_core_bytes(g) + proj_w_bytes(g) +
+           static_cast<size_t>(g.pix_per_cta) * Cout * 2 + static_cast<size_t>(Cout) * sizeof(float);
+}
+
+cudaError_t launch_forward_proj(const Geometry& g, int dtype, const void* value, const void* om, const void* w,
+                                const void* b, void* out, void* core_out, int Cout, cudaStream_t stream) {
+    switch (dtype) {
+        case 1: {
+            LinearArgs<__half> a{};
+            a.pw = static_cast<const __half*>(w);
+            a.pb = static_cast<const __half*>(b);
+            a.core_out = static_cast<__half*>(core_out);
+            a.Cout = Cout;
+            return launch_vec<__half, false, true>(g, g.vec, value, om, out, a, stream);
+        }
+        case 2: {
+            LinearArgs<__nv_bfloat16> a{};
+            a.pw = static_cast<const __nv_bfloat16*>(w);
+            a.pb = static_cast<const __nv_bfloat16*>(b);
+            a.core_out = static_cast<__nv_bfloat16*>(core_out);
+            a.Cout = Cout;
+            return launch_vec<__nv_bfloat16, false, true>(g, g.vec, value, om, out, a, stream);
+        }
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t forward_tc_status(unsigned* status, bool reset) {
+    cudaError_t e = cudaMemcpyFromSymbol(status, g_fwd_linear_status, sizeof(unsigned));
+    if (e == cudaSuccess && reset) {
+        const unsigned zero = 0u;
+        e = cudaMemcpyToSymbol(g_fwd_linear_status, &zero, sizeof(unsigned));
+    }
+    return e;
 }
 
 size_t forward_smem_bytes(const Geometry& g, int elem_bytes) {

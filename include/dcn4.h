@@ -67,7 +67,7 @@
 extern "C" {
 #endif
 
-#define DCN4_VERSION 150  /* 1.5.0: backward of the fused linear producer (dcn4_backward_linear) */
+#define DCN4_VERSION 160  /* 1.6.0: the output projection fused behind the sampler (dcn4_forward_proj) */
 
 typedef enum {
     DCN4_F32 = 0,   /* IEEE binary32            */
@@ -282,6 +282,71 @@ int dcn4_backward_linear(const dcn4_params* p, int Cx, const void* value, const 
                          const void* weight, const void* grad_out, void* grad_value, void* grad_offset_mask,
                          void* grad_x, void* grad_weight, void* grad_bias, void* workspace, size_t workspace_bytes,
                          void* stream);
+
+/* Forward with the output projection fused behind it: the DCNv4 module puts a
+ * linear layer on each side of the core operator (CSDN summary, section 2.2
+ * "DCN模块的微设计", which merges the layers around the core); this is the
+ * aggregation followed by the one after it:
+ *     core = dcn4_forward(value, offset_mask)          (rounded to dtype)
+ *     out[n, ho, wo, o] = round_dtype( sum_c core[n, ho, wo, c] * weight[o, c] + bias[o] )
+ * formed tile by tile in the kernel: the sampling threads leave the tile's core
+ * rows in shared memory, the tensor cores (tcgen05, fp32 accumulation in tensor
+ * memory) multiply them by weight, the bias is added in fp32 and the result
+ * rounded once, so the core output need not go through HBM.  One kernel launch
+ * on `stream`.
+ *   offset_mask [N, Ho, Wo, P]     dtype, as for dcn4_forward
+ *   weight      [Cout, C]          dtype (nn.Linear layout: row o gives output o)
+ *   bias        [Cout]             dtype, or NULL for none
+ *   out         [N, Ho, Wo, Cout]  dtype
+ *   core_out    [N, Ho, Wo, C]     dtype, or NULL: receives the core output (for
+ *                                  a later dcn4_backward_proj)
+ * fp16 and bf16 only (DCN4_ERR_UNSUPPORTED for fp32).  Cout a positive multiple
+ * of 16 (DCN4_ERR_BAD_SHAPE), at most 128 (DCN4_ERR_UNSUPPORTED: the kernel
+ * forms M = 128 rows of weight per tile against the tile's pixels).  It needs
+ * C a multiple of 64 up to 256 and
+ * 16-, 32- or 64-pixel tiles, as C = 64 with G = 4, C = 128 with G = 4 or 8 and
+ * C = 256 with G = 16 give (DCN4_ERR_UNSUPPORTED otherwise, or when the tiles
+ * do not fit shared memory).  Every non-NULL pointer 16-byte aligned.  The
+ * same checks as dcn4_forward otherwise.  A bounded wait of the tensor-core
+ * step that gives up sets the status word dcn4_forward_tc_status reads. */
+int dcn4_forward_proj(const dcn4_params* p, int Cout, const void* value, const void* offset_mask, const void* weight,
+                      const void* bias, void* out, void* core_out, void* stream);
+
+/* The status word of the forward's tensor-core steps (dcn4_forward_linear's
+ * tcgen05 producer and dcn4_forward_proj): 0 while every wait on the tensor
+ * cores has completed, nonzero once one gave up (its tile's results are then
+ * not written).  Synchronous (waits for the device); reset != 0 clears it.
+ * Returns the word, or a negative DCN4_ERR_* status if it cannot be read. */
+int dcn4_forward_tc_status(int reset);
+
+/* Bytes of device workspace dcn4_backward_proj needs: dcn4_backward's, then
+ * room for the gradient of the core output (N*Ho*Wo*C elements of dtype), then
+ * the projection's fp32 accumulators and counters, each rounded up to 256
+ * bytes; 0 if p is invalid. */
+size_t dcn4_backward_proj_workspace_size(const dcn4_params* p, int Cout);
+
+/* Backward of dcn4_forward_proj.  With core = the core output the forward saved
+ * (its core_out) and g = grad_out [M = N*Ho*Wo, Cout]:
+ *   grad_core   [N, Ho, Wo, C]  = g weight      (in the workspace, rounded to dtype)
+ *   grad_weight [Cout, C]       = g^T core
+ *   grad_bias   [Cout]          = sum over m of g[m, o]
+ *   grad_value, grad_offset_mask = dcn4_backward(value, offset_mask, grad_core)
+ * All of dtype (fp16 or bf16; DCN4_ERR_UNSUPPORTED for fp32).  The products run
+ * on the tensor cores (tcgen05, fed by TMA) with fp32 accumulation, rounded to
+ * dtype once; grad_weight and grad_bias sum row chunks with fp32 atomics (their
+ * last bit may vary from call to call).  grad_weight and grad_bias may be NULL
+ * (not wanted; core_out is needed only for grad_weight); grad_value and
+ * grad_offset_mask are required.  Every pointer 16-byte aligned; Cout and C
+ * multiples of 16 (DCN4_ERR_BAD_SHAPE); N*Ho*Wo and Cout*C below 2^31
+ * (DCN4_ERR_UNSUPPORTED); `workspace` (device, >= dcn4_backward_proj_workspace_size
+ * bytes) is clobbered, its first part exactly as by dcn4_backward (so
+ * dcn4_backward_diagnostics reads it).  With N*Ho*Wo = 0 only grad_weight and
+ * grad_bias are written (zeros).  Launches on `stream`: a memset and one or two
+ * kernels for the projection's gradients, then dcn4_backward's launches. */
+int dcn4_backward_proj(const dcn4_params* p, int Cout, const void* value, const void* offset_mask,
+                       const void* core_out, const void* weight, const void* grad_out, void* grad_value,
+                       void* grad_offset_mask, void* grad_weight, void* grad_bias, void* workspace,
+                       size_t workspace_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
  * Deformable attention, single scale.

@@ -70,7 +70,7 @@ def test_params_mirror_matches_the_header(dcn):
             fields += [n.strip() for n in names.split(",")]
     assert [f[0] for f in dcn.dcn4_params._fields_] == fields
     assert ctypes.sizeof(dcn.dcn4_params) == 4 * len(fields)
-    assert dcn.dcn4_version() == 150
+    assert dcn.dcn4_version() == 160
 
 
 def test_attn_params_mirror_matches_the_header(dcn):
@@ -245,6 +245,68 @@ assert call(bad, 64) == -3
 big = dcn.make_params(N=2048, H=1024, W=1024, G=4, Cg=16, dtype="bf16")
 assert call(big, 64, nb=1 << 62) == -5 and "2^31" in dcn.dcn4_last_error()
 assert dcn.dcn4_last_error() != ""
+""")
+
+
+def test_forward_proj_checks_before_launch():
+    """dcn4_forward_proj validates on the host (made-up addresses: checked in a child
+    process that sees no GPU)."""
+    run_without_gpu("""
+p = dcn.make_params(N=2, H=8, W=8, G=4, Cg=16, dtype="f16")
+ok = dict(value=16, om=32, w=48, b=None, out=64, core=None)
+
+def call(params, Cout, **kw):
+    a = {**ok, **kw}
+    return dcn.dcn4_forward_proj(params, Cout, a["value"], a["om"], a["w"], a["b"], a["out"], a["core"], None)
+p32 = dcn.make_params(N=2, H=8, W=8, G=4, Cg=16, dtype="f32")
+assert call(p32, 64) == -5                                           # fp32: no fused projection
+assert call(p, 24) == -2 and call(p, 0) == -2 and call(p, 8) == -2   # Cout not a multiple of 16
+assert call(p, 144) == -5 and "128" in dcn.dcn4_last_error()         # more outputs than one tile forms
+c32 = dcn.make_params(N=2, H=8, W=8, G=2, Cg=16, dtype="f16")
+assert call(c32, 64) == -5 and "multiple of 64" in dcn.dcn4_last_error()
+c512 = dcn.make_params(N=2, H=8, W=8, G=32, Cg=16, dtype="f16")
+assert call(c512, 64) == -5
+assert call(p, 64, w=None) == -1 and call(p, 64, om=None) == -1 and call(p, 64, out=None) == -1
+assert call(p, 64, b=40) == -4 and call(p, 64, core=72) == -4 and call(p, 64, w=52) == -4
+bad = dcn.make_params(N=2, H=8, W=8, G=4, Cg=16, dtype="f16")
+bad.P = 100
+assert call(bad, 64) == -3
+assert dcn.dcn4_last_error() != ""
+""")
+
+
+def test_backward_proj_checks_before_launch():
+    """dcn4_backward_proj validates on the host before its first launch (made-up
+    addresses: checked in a child process that sees no GPU)."""
+    run_without_gpu("""
+p = dcn.make_params(N=2, H=8, W=8, G=4, Cg=16, dtype="bf16")
+need = dcn.dcn4_backward_proj_workspace_size(p, 64)
+assert need >= dcn.dcn4_backward_workspace_size(p) + 2 * 8 * 8 * 64 * 2 + 4 * (64 * 64 + 64)
+assert need % 256 == 0 and dcn.dcn4_backward_proj_workspace_size(p, 0) == 0
+ok = dict(value=16, om=32, core=48, w=64, gy=80, gv=96, gom=112, gw=144, gb=160, ws=4096, nb=need)
+
+def call(params, Cout, **kw):
+    a = {**ok, **kw}
+    return dcn.dcn4_backward_proj(params, Cout, a["value"], a["om"], a["core"], a["w"], a["gy"], a["gv"], a["gom"],
+                                  a["gw"], a["gb"], a["ws"], a["nb"], None)
+p32 = dcn.make_params(N=2, H=8, W=8, G=4, Cg=16, dtype="f32")
+assert call(p32, 64, nb=1 << 24) == -5              # fp32: no projection
+assert call(p, 24) == -2 and call(p, 0) == -2       # Cout not a multiple of 16
+c8 = dcn.make_params(N=2, H=8, W=8, G=1, Cg=8, dtype="bf16", P=32)
+assert call(c8, 64, nb=1 << 24) == -2               # C not a multiple of 16
+assert call(p, 64, nb=need - 1) == -6 and call(p, 64, ws=None) == -6
+assert call(p, 64, ws=4100) == -4                   # misaligned workspace
+assert call(p, 64, gw=148) == -4 and call(p, 64, core=52) == -4 and call(p, 64, gb=161) == -4
+assert call(p, 64, gom=None) == -1 and call(p, 64, gv=None) == -1
+assert call(p, 64, w=None) == -1 and call(p, 64, gy=None) == -1
+assert call(p, 64, value=None) == -1 and call(p, 64, om=None) == -1
+assert call(p, 64, value=20) == -4 and call(p, 64, gv=100) == -4
+assert call(p, 64, core=None) == -1 and "core_out" in dcn.dcn4_last_error()
+bad = dcn.make_params(N=2, H=8, W=8, G=4, Cg=16, dtype="bf16")
+bad.P = 100
+assert call(bad, 64) == -3
+big = dcn.make_params(N=2048, H=1024, W=1024, G=4, Cg=16, dtype="bf16")
+assert call(big, 64, nb=1 << 62) == -5 and "2^31" in dcn.dcn4_last_error()
 """)
 
 
