@@ -641,9 +641,6 @@ def dcnv4_core_proj(value, offset_mask, weight, bias=None, *, group: int, kernel
     formed inside the forward kernel; differentiable in value, offset_mask, weight and
     bias (torch.autograd)."""
     global _DCNV4_CORE_PROJ
-    p = params_for_tensors(value, offset_mask, group=group, kernel=kernel, stride=stride, pad=pad,
-                           dilation=dilation, offset_scale=offset_scale, remove_center=remove_center,
-                           softmax=softmax)
     if weight.dim() != 2 or weight.shape[1] != value.shape[-1]:
         raise ValueError("weight must be [Cout, C]")
     if bias is not None and tuple(bias.shape) != (weight.shape[0],):
@@ -651,6 +648,9 @@ def dcnv4_core_proj(value, offset_mask, weight, bias=None, *, group: int, kernel
     for name, t in (("weight", weight),) + ((("bias", bias),) if bias is not None else ()):
         if t.dtype != value.dtype or not t.is_contiguous() or t.device != value.device:
             raise ValueError(f"{name} must be contiguous, on value's device and of value's dtype")
+    p = params_for_tensors(value, offset_mask, group=group, kernel=kernel, stride=stride, pad=pad,
+                           dilation=dilation, offset_scale=offset_scale, remove_center=remove_center,
+                           softmax=softmax)
     if _DCNV4_CORE_PROJ is None:
         _DCNV4_CORE_PROJ = _autograd_function_proj()
     return _DCNV4_CORE_PROJ.apply(value, offset_mask, weight, bias, p)

@@ -54,7 +54,7 @@ constexpr size_t kSamplesStaticSmem = 8 * 1024;
 // Validates p and fills the kernel geometry.  Touches no GPU state.
 // wide: the gathered and stored tensors are 32-byte aligned, so a thread may
 // move a 32-byte channel slice with one 256-bit access.
-int make_geometry(const dcn4_params* p, bool backward, bool wide, dcn4::Geometry* g) {
+int make_geometry(const dcn4_params* p, bool backward, bool wide, dcn4::Geometry* g, bool full_tiles = false) {
     if (!p) return fail(DCN4_ERR_NULL, "params is NULL");
     if (p->dtype != DCN4_F32 && p->dtype != DCN4_F16 && p->dtype != DCN4_BF16)
         return fail(DCN4_ERR_DTYPE, "dtype %d is not a dcn4_dtype", p->dtype);
@@ -106,27 +106,35 @@ int make_geometry(const dcn4_params* p, bool backward, bool wide, dcn4::Geometry
     // Output pixels per CTA: fill kTargetThreads, then shrink until the
     // shared-memory rows fit the default 48 KB (or, for very long rows, the
     // per-CTA maximum).
-    // Shared memory per output pixel: two offset_mask rows (forward: a double
-    // buffer; backward: offset_mask and grad_offset_mask rows), and with softmax
-    // (forward) its threads' fp32 exponentials.
+    // Shared memory per output pixel: two offset_mask rows (forward: the tiles in
+    // flight, a third one only where it still fits three CTAs to an SM; backward:
+    // offset_mask and grad_offset_mask rows), and with softmax (forward) its
+    // threads' fp32 exponentials.
     const size_t row_bytes = static_cast<size_t>(p->P) * eb * 2 +
                              (p->softmax ? static_cast<size_t>(K) * lanes_pp * sizeof(float) : 0);
     long long ppc = kTargetThreads / lanes_pp;
     while (ppc > 1 && ppc * row_bytes > kSmemDefault) --ppc;
     if (ppc * row_bytes > kSmemMax) return fail(DCN4_ERR_UNSUPPORTED, "P=%d rows do not fit shared memory", p->P);
+    if (full_tiles) {  // a power of two of pixels (see below)
+        long long q = 1;
+        while (q * 2 <= ppc) q *= 2;
+        ppc = q;
+    }
     // A CTA covers a TH x TW tile of output pixels of one image (TW a power of
     // two, TH = the rest of the pixel budget, both clipped to the image): the
     // shape that leaves the fewest threads idle on the image's ragged edges;
     // among equals the one with more pixels, then the squarer one.  Shapes
     // more than 4:1 are taken only when nothing squarer exists (a 14 x 1 strip
     // fills a 14 x 14 map exactly but gathers from a wider halo per pixel).
+    // full_tiles: TH is not clipped to the image, so every tile holds the whole
+    // pixel budget (the fused projection's MMA takes N = the tile's pixels).
     long long TW = 1, TH = 1;
     {
         long long best_used = -1, best_slots = 1, best_px = 0, best_skew = 0;
         for (int pass = 0; pass < 2 && best_used < 0; ++pass)
         for (long long tw = 1; tw <= ppc; tw *= 2) {
             if (tw > 1 && tw / 2 >= Wo) break;
-            const long long th = std::min(ppc / tw, Ho);
+            const long long th = full_tiles ? ppc / tw : std::min(ppc / tw, Ho);
             if (pass == 0 && std::max(th, tw) > 4 * std::min(th, tw)) continue;
             const long long slots = (Ho + th - 1) / th * th * ((Wo + tw - 1) / tw * tw);
             const long long used = Ho * Wo;
@@ -400,7 +408,7 @@ int dcn4_forward_linear(const dcn4_params* p, int Cx, const void* value, const v
 int dcn4_forward_proj(const dcn4_params* p, int Cout, const void* value, const void* offset_mask, const void* weight,
                       const void* bias, void* out, void* core_out, void* stream) {
     dcn4::Geometry g;
-    const int st = make_geometry(p, false, aligned32(value), &g);
+    const int st = make_geometry(p, false, aligned32(value), &g, true);
     if (st != DCN4_OK) return st;
     if (p->dtype == DCN4_F32) return fail(DCN4_ERR_UNSUPPORTED, "the fused output projection takes fp16 or bf16");
     if (Cout < 16 || Cout % 16 != 0 || Cout > (1 << 16))

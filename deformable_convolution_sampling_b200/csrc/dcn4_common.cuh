@@ -43,6 +43,8 @@ struct Geometry {
     // Filing window of the grad_offset_mask CTA: fwin_h tile rows x 2^fwin_wl
     // tile columns (64 tiles).
     int fwin_h, fwin_wl;
+    // Forward: offset_mask tiles in flight per CTA (set by the forward's launcher).
+    int fbufs;
 };
 
 // What the grad_offset_mask pass leaves for the grad_value pass.

@@ -62,6 +62,11 @@ __device__ __forceinline__ void accumulate(float2* acc, const T* src, float wt) 
 
 // CTAs per SM the forward kernel is compiled for (80 registers a thread).
 constexpr int kFwdCtasPerSm = 3;
+// offset_mask tiles in flight per CTA (plain and PROJ, g.fbufs): three when they still
+// leave room for kFwdCtasPerSm CTAs an SM, else two.  With three, the buffer a tile is
+// copied into was last read two tiles earlier, before a barrier every thread has since
+// passed, so a tile needs one barrier, not two.
+constexpr int kFwdMaxBufs = 3;
 
 // Arguments of the fused producer: x [N, Ho, Wo, Cx], w [P, Cx] (nn.Linear
 // layout), b [P] or null, om_out [N, Ho, Wo, P] or null; and of the fused
@@ -104,6 +109,21 @@ __device__ unsigned g_fwd_linear_status;  // nonzero once a bounded wait of the 
 __host__ __device__ inline int proj_core_bytes(const Geometry& g) { return g.pix_per_cta * g.C * 2; }
 __host__ __device__ inline int proj_w_bytes(const Geometry& g) { return kTcRows * g.C * 2; }
 __host__ __device__ inline int proj_tmem_cols(const Geometry& g) { return g.pix_per_cta < 32 ? 32 : g.pix_per_cta; }
+// Shared memory of the projection beyond the offset_mask tiles and exponentials: the
+// 1024-byte alignment slack, the core tile, W_out, the result tile and the bias.
+inline size_t proj_extra_bytes(const Geometry& g, int Cout) {
+    return 1024 + static_cast<size_t>(proj_core_bytes(g)) + proj_w_bytes(g) +
+           static_cast<size_t>(g.pix_per_cta) * Cout * 2 + static_cast<size_t>(Cout) * sizeof(float);
+}
+// The softmax exponentials [K][threads] (fp32), when the masks are logits.
+inline size_t forward_exps_bytes(const Geometry& g) {
+    return g.softmax ? static_cast<size_t>(g.K) * samples_threads(g) * sizeof(float) : 0;
+}
+// offset_mask tiles per CTA for a CTA that also holds `extra` bytes (see kFwdMaxBufs).
+inline int forward_bufs(const Geometry& g, int elem_bytes, size_t extra) {
+    const size_t tile = static_cast<size_t>(g.pix_per_cta) * g.P * elem_bytes;
+    return kFwdMaxBufs * tile + forward_exps_bytes(g) + extra + 1024 <= 227 * 1024 / kFwdCtasPerSm ? kFwdMaxBufs : 2;
+}
 
 // Rows of a staged x tile: the tile's pixels rounded up to whole 16-row MMA tiles.
 __host__ __device__ inline int linear_rows(const Geometry& g) { return (g.TH * g.TW + 15) / 16 * 16; }
@@ -368,9 +388,9 @@ __global__ void __launch_bounds__(256, kFwdCtasPerSm) forward_kernel(const Geome
     constexpr int EPV = Elem<T>::per16;
     constexpr int PAIRS = VEC * EPV / 2;
     const int tile_elems = g.TH * g.TW * g.P;
-    // plain: two offset_mask tiles; LIN: one offset_mask tile, two x tiles, W (when
-    // staged), the bias (fp32)
-    T* bufs[2];
+    // plain: g.fbufs offset_mask tiles, the exponentials; LIN: one offset_mask tile, two x
+    // tiles, W (when staged), the bias (fp32); PROJ: as plain, then the projection's tiles
+    T* om_buf;  // the first offset_mask tile (plain and PROJ: g.fbufs of them follow one another)
     T* xbuf[2] = {nullptr, nullptr};
     T* w_s = nullptr;
     float* b_s = nullptr;
@@ -382,7 +402,7 @@ __global__ void __launch_bounds__(256, kFwdCtasPerSm) forward_kernel(const Geome
     __shared__ uint32_t tc_taddr;
     __shared__ int tc_abort;
     if constexpr (LIN) {
-        bufs[0] = bufs[1] = reinterpret_cast<T*>(smem);
+        om_buf = reinterpret_cast<T*>(smem);
         if (lin.tc) {
             tc_x[0] = (sbase + static_cast<uint32_t>(tile_elems) * 2u + 1023u) & ~1023u;
             tc_x[1] = tc_x[0] + tc_x_bytes(lin.Cx);
@@ -390,16 +410,15 @@ __global__ void __launch_bounds__(256, kFwdCtasPerSm) forward_kernel(const Geome
             b_s = reinterpret_cast<float*>(smem + (tc_w - sbase) + tc_w_bytes(lin.Cx));
         } else {
             const int xs = linear_rows(g) * linear_ld(lin.Cx);
-            xbuf[0] = bufs[0] + tile_elems;
+            xbuf[0] = om_buf + tile_elems;
             xbuf[1] = xbuf[0] + xs;
             w_s = xbuf[1] + xs;
             b_s = reinterpret_cast<float*>(w_s + (lin.w_smem ? linear_w_rows(g) * linear_ld(lin.Cx) : 0));
         }
         e_s = b_s + g.P;
     } else {
-        bufs[0] = reinterpret_cast<T*>(smem);
-        bufs[1] = bufs[0] + tile_elems;
-        e_s = reinterpret_cast<float*>(bufs[1] + tile_elems);
+        om_buf = reinterpret_cast<T*>(smem);
+        e_s = reinterpret_cast<float*>(om_buf + g.fbufs * tile_elems);
     }
     // PROJ: the swizzled core tile and W_out (1024-byte aligned), the [pixels][Cout]
     // result tile and the bias (fp32), after the exponentials
@@ -407,7 +426,7 @@ __global__ void __launch_bounds__(256, kFwdCtasPerSm) forward_kernel(const Geome
     T* pj_o = nullptr;
     float* pj_b = nullptr;
     if constexpr (PROJ) {
-        const uint32_t end = sbase + static_cast<uint32_t>(2 * tile_elems * sizeof(T)) +
+        const uint32_t end = sbase + static_cast<uint32_t>(g.fbufs * tile_elems * sizeof(T)) +
                              (SM ? static_cast<uint32_t>(g.K * blockDim.x * sizeof(float)) : 0u);
         pj_a = (end + 1023u) & ~1023u;
         pj_w = pj_a + proj_core_bytes(g);
@@ -476,7 +495,7 @@ __global__ void __launch_bounds__(256, kFwdCtasPerSm) forward_kernel(const Geome
         }
         if (!lin.tc) stage_x_async(xbuf[0], lin, g, tile_at(g, tile));
     } else {
-        stage_tile_async(bufs[0], om, g, tile_at(g, tile));
+        stage_tile_async(om_buf, om, g, tile_at(g, tile));
     }
 
     const int lanes_pp = g.G * g.nslice;
@@ -492,8 +511,10 @@ __global__ void __launch_bounds__(256, kFwdCtasPerSm) forward_kernel(const Geome
     const bool rc = KH > 0 ? RC : g.remove_center != 0;
     const int ch_off = grp * g.Cg + sl * (VEC * EPV);
 
+    int cur = 0;  // the buffer of this tile's offset_mask rows (plain and PROJ)
     for (int it = 0; tile < ntiles; ++it, tile += gridDim.x) {
         const int next = tile + gridDim.x;
+        const int nxt = cur + 1 == g.fbufs ? 0 : cur + 1;
         if (next < ntiles) {
             if constexpr (LIN) {
                 if (lin.tc) {
@@ -502,7 +523,7 @@ __global__ void __launch_bounds__(256, kFwdCtasPerSm) forward_kernel(const Geome
                     stage_x_async(xbuf[(it + 1) & 1], lin, g, tile_at(g, next));
                 }
             } else {
-                stage_tile_async(bufs[(it + 1) & 1], om, g, tile_at(g, next));
+                stage_tile_async(reinterpret_cast<T*>(smem) + nxt * tile_elems, om, g, tile_at(g, next));
             }
             asm volatile("cp.async.wait_group 1;" ::: "memory");
         } else {
@@ -515,7 +536,7 @@ __global__ void __launch_bounds__(256, kFwdCtasPerSm) forward_kernel(const Geome
         __syncthreads();
         const Tile t = tile_at(g, tile);
         // the tile's rows, addressed from smem directly so the reads stay shared-space loads
-        const T* om_s = reinterpret_cast<const T*>(smem) + (LIN ? 0 : (it & 1) * tile_elems);
+        const T* om_s = reinterpret_cast<const T*>(smem) + (LIN ? 0 : cur * tile_elems);
         if constexpr (LIN) {
             if (lin.tc) {
                 // one thread issues the tile's MMAs; all wait for them, then read the accumulator back:
@@ -544,16 +565,16 @@ __global__ void __launch_bounds__(256, kFwdCtasPerSm) forward_kernel(const Geome
                     const float bp = b_s[pr];
 #pragma unroll
                     for (int j = 0; j < 32; ++j)
-                        bufs[0][(half * 32 + j) * g.P + pr] = from_f32<T>(__uint_as_float(acc32[j]) + bp);
+                        om_buf[(half * 32 + j) * g.P + pr] = from_f32<T>(__uint_as_float(acc32[j]) + bp);
                 }
                 tc::tc_fence_before();  // the next tile's MMAs overwrite the accumulator after the next barrier
             } else {
                 switch (lin.w_smem ? lin.Cx / 16 : 0) {
-                    case 1: linear_tile_staged<T, 1>(g, lin, xbuf[it & 1], w_s, bufs[0], b_s); break;
-                    case 2: linear_tile_staged<T, 2>(g, lin, xbuf[it & 1], w_s, bufs[0], b_s); break;
-                    case 4: linear_tile_staged<T, 4>(g, lin, xbuf[it & 1], w_s, bufs[0], b_s); break;
-                    case 8: linear_tile_staged<T, 8>(g, lin, xbuf[it & 1], w_s, bufs[0], b_s); break;
-                    default: linear_tile(g, lin, xbuf[it & 1], w_s, bufs[0], b_s);
+                    case 1: linear_tile_staged<T, 1>(g, lin, xbuf[it & 1], w_s, om_buf, b_s); break;
+                    case 2: linear_tile_staged<T, 2>(g, lin, xbuf[it & 1], w_s, om_buf, b_s); break;
+                    case 4: linear_tile_staged<T, 4>(g, lin, xbuf[it & 1], w_s, om_buf, b_s); break;
+                    case 8: linear_tile_staged<T, 8>(g, lin, xbuf[it & 1], w_s, om_buf, b_s); break;
+                    default: linear_tile(g, lin, xbuf[it & 1], w_s, om_buf, b_s);
                 }
             }
             __syncthreads();
@@ -568,7 +589,7 @@ __global__ void __launch_bounds__(256, kFwdCtasPerSm) forward_kernel(const Geome
                     const int qy = q / t.tw, qx = q - qy * t.tw;
                     const long long pix = (static_cast<long long>(t.n) * g.Ho + t.ho0 + qy) * g.Wo + t.wo0 + qx;
                     st_global(lin.om_out + pix * g.P + c * EPV,
-                              *reinterpret_cast<const uint4*>(bufs[0] + (qy * g.TW + qx) * g.P + c * EPV));
+                              *reinterpret_cast<const uint4*>(om_buf + (qy * g.TW + qx) * g.P + c * EPV));
                 }
             }
         }
@@ -747,7 +768,10 @@ __global__ void __launch_bounds__(256, kFwdCtasPerSm) forward_kernel(const Geome
                           *reinterpret_cast<const uint4*>(pj_o + (qy * g.TW + qx) * lin.Cout + c * EPV));
             }
         }
-        __syncthreads();  // the buffer is refilled two tiles later (LIN: om_s at the next tile)
+        // LIN: the producer rewrites om_s at the next tile; plain and PROJ with two buffers: the
+        // next copy goes to this tile's buffer (with three, to the one read two tiles ago)
+        if (LIN || g.fbufs < 3) __syncthreads();
+        cur = nxt;
     }
     if constexpr (PROJ) {
         asm volatile("cp.async.wait_group 0;" ::: "memory");
@@ -774,6 +798,8 @@ cudaError_t launch_typed(const Geometry& g, const void* value, const void* om, v
     const size_t smem = LIN    ? forward_linear_smem_bytes(g, lin.Cx, lin.tc ? 2 : lin.w_smem ? 1 : 0)
                         : PROJ ? forward_proj_smem_bytes(g, lin.Cout)
                                : forward_smem_bytes(g, sizeof(T));
+    Geometry gk = g;
+    gk.fbufs = LIN ? 1 : forward_bufs(g, sizeof(T), PROJ ? proj_extra_bytes(g, lin.Cout) : 0);
     auto kern = forward_kernel<T, VEC, KH, KW, RC, SM, LIN, PROJ>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
@@ -788,7 +814,7 @@ cudaError_t launch_typed(const Geometry& g, const void* value, const void* om, v
     const long long ntiles = static_cast<long long>(g.N) * g.tiles_h * g.tiles_w;
     const long long blocks = std::min<long long>(ntiles, per_sm * sms);
     kern<<<static_cast<unsigned>(blocks), threads, smem, stream>>>(
-        g, static_cast<const T*>(value), static_cast<const T*>(om), static_cast<T*>(out), lin);
+        gk, static_cast<const T*>(value), static_cast<const T*>(om), static_cast<T*>(out), lin);
     return cudaGetLastError();
 }
 
@@ -869,8 +895,8 @@ bool forward_proj_shape_ok(const Geometry& g, int Cout) {
 }
 
 size_t forward_proj_smem_bytes(const Geometry& g, int Cout) {
-    return forward_smem_bytes(g, 2) + 1024 + proj_core_bytes(g) + proj_w_bytes(g) +
-           static_cast<size_t>(g.pix_per_cta) * Cout * 2 + static_cast<size_t>(Cout) * sizeof(float);
+    const size_t extra = proj_extra_bytes(g, Cout);
+    return forward_bufs(g, 2, extra) * static_cast<size_t>(g.pix_per_cta) * g.P * 2 + forward_exps_bytes(g) + extra;
 }
 
 cudaError_t launch_forward_proj(const Geometry& g, int dtype, const void* value, const void* om, const void* w,
@@ -906,8 +932,8 @@ cudaError_t forward_tc_status(unsigned* status, bool reset) {
 }
 
 size_t forward_smem_bytes(const Geometry& g, int elem_bytes) {
-    return 2 * static_cast<size_t>(g.pix_per_cta) * g.P * elem_bytes +                        // double buffer
-           (g.softmax ? static_cast<size_t>(g.K) * samples_threads(g) * sizeof(float) : 0);  // exponentials
+    return forward_bufs(g, elem_bytes, 0) * static_cast<size_t>(g.pix_per_cta) * g.P * elem_bytes +
+           forward_exps_bytes(g);
 }
 
 cudaError_t launch_forward(const Geometry& g, int dtype, const void* value, const void* om, void* out,

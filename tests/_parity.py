@@ -29,8 +29,13 @@ def to_f64(t) -> np.ndarray:
 
 
 def params_for(w: gen.Workload, dtype: str | None = None):
+    """The workload's dcn4_params, after checking that the library's output grid is the
+    one the workload's tensors are sized for."""
     import deformable_convolution_sampling_b200 as dcn
-    return dcn.make_params(dtype=dtype or w.dtype, **w.geometry())
+    p = dcn.make_params(dtype=dtype or w.dtype, **w.geometry())
+    st, Ho, Wo = dcn.dcn4_output_dims(p)
+    assert st == 0 and (Ho, Wo) == (w.Ho, w.Wo), f"{w.name}: the library's output is {Ho}x{Wo}, not {w.Ho}x{w.Wo}"
+    return p
 
 
 def problem_for(w: gen.Workload, n: int | None = None, dtype: str | None = None) -> oracle.Problem:

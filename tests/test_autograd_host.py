@@ -38,3 +38,18 @@ def test_linear_argument_errors(x, w, b, msg):
     value = _t(1, 8, 8, 16, dtype=torch.float16)
     with pytest.raises(ValueError, match=msg):
         dcn.dcnv4_core_linear(value, x, w, b, group=2)
+
+
+@pytest.mark.parametrize("w,b,msg", [
+    (_t(64, 16, 1, dtype=torch.float16), None, "weight"),
+    (_t(64, 32, dtype=torch.float16), None, "weight"),
+    (_t(64, 16, dtype=torch.float16), _t(63, dtype=torch.float16), "bias"),
+    (_t(64, 16), None, "dtype"),
+    (_t(64, 16, dtype=torch.float16).t().contiguous().t(), None, "contiguous"),
+    (_t(64, 16, dtype=torch.float16), None, "CUDA tensors"),
+])
+def test_proj_argument_errors(w, b, msg):
+    value = _t(1, 8, 8, 16, dtype=torch.float16)
+    om = _t(1, 8, 8, 56, dtype=torch.float16)
+    with pytest.raises(ValueError, match=msg):
+        dcn.dcnv4_core_proj(value, om, w, b, group=2)

@@ -21,7 +21,7 @@ import pytest
 
 import dcn4_inputs as gen
 import oracle
-from _parity import FWD_TOL, gpu_forward, normwise, oracle_forward, take, to_device, to_f64
+from _parity import FWD_TOL, gpu_forward, normwise, oracle_forward, params_for, take, to_device, to_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -45,7 +45,7 @@ def _run(w, Cx, *, bias=True, sample=None, seed=None):
     import deformable_convolution_sampling_b200 as dcn
     inp = gen.make_inputs(w, with_grad=False, seed=seed)
     lin = gen.make_linear_inputs(w, Cx, bias=bias, seed=seed)
-    p = dcn.make_params(dtype=w.dtype, **w.geometry())
+    p = params_for(w)
     v = to_device(inp["value"], w.dtype)
     x = to_device(lin["x"], w.dtype)
     wt = to_device(lin["weight"], w.dtype)
@@ -119,7 +119,7 @@ def test_identity_weight_reproduces_offset_mask():
     import deformable_convolution_sampling_b200 as dcn
     w = gen.custom(name="ident", N=2, H=9, W=10, G=4, Cg=16, Ho=9, Wo=10, K=9, P=112, dtype="f16")
     inp = gen.make_inputs(w, with_grad=False, tail_fill=0.0)
-    p = dcn.make_params(dtype=w.dtype, **w.geometry())
+    p = params_for(w)
     v = to_device(inp["value"], w.dtype)
     om = to_device(inp["offset_mask"], w.dtype)
     eye = torch.eye(w.P, dtype=v.dtype, device="cuda")

@@ -22,7 +22,7 @@ import pytest
 
 import dcn4_inputs as gen
 import oracle
-from _parity import BWD_TOL, normwise, to_device, to_f64
+from _parity import BWD_TOL, normwise, params_for, to_device, to_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -57,7 +57,7 @@ def _run(w, Cx, *, bias=True, sample=None, want_x=True, want_weight=True):
     import deformable_convolution_sampling_b200 as dcn
     inp = gen.make_inputs(w, tail_fill=0.0)
     lin = gen.make_linear_inputs(w, Cx, bias=bias)
-    p = dcn.make_params(dtype=w.dtype, **w.geometry())
+    p = params_for(w)
     v, gy = to_device(inp["value"], w.dtype), to_device(inp["grad_out"], w.dtype)
     x, wt = to_device(lin["x"], w.dtype), to_device(lin["weight"], w.dtype)
     b = to_device(lin["bias"], w.dtype) if bias else None
@@ -184,7 +184,7 @@ def test_autograd_linear_uses_the_library_backward():
     gy = to_device(inp["grad_out"], w.dtype)
     y = dcn.dcnv4_core_linear(v, x, wt, b, group=w.G)
     y.backward(gy)
-    p = dcn.make_params(dtype=w.dtype, **w.geometry())
+    p = params_for(w)
     om = torch.empty((w.N, w.Ho, w.Wo, w.P), dtype=v.dtype, device="cuda")
     dcn.forward_linear(p, v.detach(), x.detach(), wt.detach(), b.detach(), offset_mask_out=om)
     _, _, gx, gw, gb = dcn.backward_linear(p, v.detach(), om, x.detach(), wt.detach(), gy)

@@ -27,7 +27,7 @@ import pytest
 
 import dcn4_inputs as gen
 import oracle
-from _parity import BWD_TOL, FWD_TOL, normwise, oracle_forward, to_device, to_f64
+from _parity import BWD_TOL, FWD_TOL, normwise, oracle_forward, params_for, to_device, to_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -67,7 +67,7 @@ def _run(w, Cout, *, bias=True, sample=None, want_weight=True):
     import deformable_convolution_sampling_b200 as dcn
     inp = gen.make_inputs(w, with_grad=False, tail_fill=0.0)
     pj = gen.make_proj_inputs(w, Cout, bias=bias)
-    p = dcn.make_params(dtype=w.dtype, **w.geometry())
+    p = params_for(w)  # also checks the output grid the tensors are sized for
     v, om = to_device(inp["value"], w.dtype), to_device(inp["offset_mask"], w.dtype)
     wt = to_device(pj["weight"], w.dtype)
     b = to_device(pj["bias"], w.dtype) if bias else None
@@ -168,7 +168,7 @@ VARIANTS = [
     dict(name="c128_g4_32px_f16", Cout=64, N=2, H=9, W=10, G=4, Cg=32, Ho=9, Wo=10, K=9, P=112, dtype="f16"),
     dict(name="c128_g8_32px_bf16", Cout=96, N=2, H=9, W=10, G=8, Cg=16, Ho=9, Wo=10, K=9, P=216, dtype="bf16"),
     dict(name="c256_g16_16px_bf16", Cout=128, N=2, H=9, W=9, G=16, Cg=16, Ho=9, Wo=9, K=9, P=432, dtype="bf16"),
-    dict(name="ragged_s2_d2_rc_f16", Cout=64, N=3, H=11, W=9, G=4, Cg=16, Ho=5, Wo=4, K=8, P=96, dtype="f16",
+    dict(name="ragged_s2_d2_rc_f16", Cout=64, N=3, H=11, W=9, G=4, Cg=16, Ho=5, Wo=5, K=8, P=96, dtype="f16",
          sh=2, sw=2, ph=1, pw=2, dh=2, dw=2, remove_center=1, offset_scale=0.7),
     dict(name="softmax_f16", Cout=64, N=2, H=10, W=12, G=4, Cg=16, Ho=10, Wo=12, K=9, P=112, dtype="f16", softmax=1),
     dict(name="k5x5_bf16", Cout=64, N=2, H=9, W=11, G=4, Cg=16, Ho=9, Wo=11, K=25, P=304, dtype="bf16", kh=5, kw=5,
@@ -196,7 +196,7 @@ def test_identity_weight_reproduces_the_core():
     import deformable_convolution_sampling_b200 as dcn
     w = gen.custom(name="ident", N=2, H=9, W=10, G=4, Cg=16, Ho=9, Wo=10, K=9, P=112, dtype="f16")
     inp = gen.make_inputs(w, with_grad=False, tail_fill=0.0)
-    p = dcn.make_params(dtype=w.dtype, **w.geometry())
+    p = params_for(w)
     v, om = to_device(inp["value"], w.dtype), to_device(inp["offset_mask"], w.dtype)
     eye = torch.eye(w.C, dtype=v.dtype, device="cuda")
     y = dcn.forward_proj(p, v, om, eye)
@@ -211,7 +211,7 @@ def test_unsupported_shapes_are_refused():
     import deformable_convolution_sampling_b200 as dcn
     w = gen.custom(name="c32", N=1, H=8, W=8, G=2, Cg=16, Ho=8, Wo=8, K=9, P=56, dtype="f16")  # C = 32
     inp = gen.make_inputs(w, with_grad=False, tail_fill=0.0)
-    p = dcn.make_params(dtype=w.dtype, **w.geometry())
+    p = params_for(w)
     v, om = to_device(inp["value"], w.dtype), to_device(inp["offset_mask"], w.dtype)
     wt = torch.zeros((64, 32), dtype=v.dtype, device="cuda")
     out = torch.empty((1, 8, 8, 64), dtype=v.dtype, device="cuda")
@@ -251,7 +251,7 @@ def test_autograd():
     gy = to_device(pj["grad_out"], w.dtype)
     y = dcn.dcnv4_core_proj(v, om, wt, b, group=w.G)
     y.backward(gy)
-    p = dcn.make_params(dtype=w.dtype, **w.geometry())
+    p = params_for(w)
     core = dcn.forward(p, v.detach(), om.detach())
     gv, gom, gw, gb = dcn.backward_proj(p, v.detach(), om.detach(), core, wt.detach(), gy)
     torch.cuda.synchronize()
