@@ -303,10 +303,11 @@ int dcn4_backward_linear(const dcn4_params* p, int Cx, const void* value, const 
  * fp16 and bf16 only (DCN4_ERR_UNSUPPORTED for fp32).  Cout a positive multiple
  * of 16 (DCN4_ERR_BAD_SHAPE), at most 128 (DCN4_ERR_UNSUPPORTED: the kernel
  * forms M = 128 rows of weight per tile against the tile's pixels).  It needs
- * C a multiple of 64 up to 256 and
- * 16-, 32- or 64-pixel tiles, as C = 64 with G = 4, C = 128 with G = 4 or 8 and
- * C = 256 with G = 16 give (DCN4_ERR_UNSUPPORTED otherwise, or when the tiles
- * do not fit shared memory).  Every non-NULL pointer 16-byte aligned.  The
+ * C a multiple of 64 up to 256 and tiles of 16, 32 or 64 pixels (the power of
+ * two of pixels that 256 threads over the groups' channel slices give, fewer
+ * for long offset_mask rows: C = 64 with G = 4, C = 128 with G = 4 or 8 and
+ * C = 256 with G = 16 give 64, 32 and 16); DCN4_ERR_UNSUPPORTED otherwise, or
+ * when the tiles do not fit shared memory.  Every non-NULL pointer 16-byte aligned.  The
  * same checks as dcn4_forward otherwise.  A bounded wait of the tensor-core
  * step that gives up sets the status word dcn4_forward_tc_status reads. */
 int dcn4_forward_proj(const dcn4_params* p, int Cout, const void* value, const void* offset_mask, const void* weight,
