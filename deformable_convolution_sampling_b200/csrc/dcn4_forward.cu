@@ -100,21 +100,31 @@ __host__ __device__ inline int tc_w_bytes(int Cx) { return kTcRows * Cx * 2; }
 __device__ unsigned g_fwd_linear_status;  // nonzero once a bounded wait of the tcgen05 producer gave up
 
 // Output projection y = core W_out^T + b_out fused behind the sampler (PROJ): per
-// tile D^T[o][pixel] = W_out core^T with M = 128 rows of W_out (Cout <= 128, the
-// rest zero), N = the tile's pixels (16, 32 or 64), K = C in 64-wide slabs; the
-// same swizzled K-major operand layout as the producer.  The core tile is written
-// by the sampling threads themselves (their fp32 sums rounded to the I/O dtype,
-// as the unfused pair stores them), the result read back into a [pixels][Cout]
-// staging tile and stored with 16-byte writes.
-__host__ __device__ inline int proj_core_bytes(const Geometry& g) { return g.pix_per_cta * g.C * 2; }
-__host__ __device__ inline int proj_w_bytes(const Geometry& g) { return kTcRows * g.C * 2; }
-__host__ __device__ inline int proj_tmem_cols(const Geometry& g) { return g.pix_per_cta < 32 ? 32 : g.pix_per_cta; }
-// Shared memory of the projection beyond the offset_mask tiles and exponentials: the
-// 1024-byte alignment slack, the core tile, W_out, the result tile and the bias.
-inline size_t proj_extra_bytes(const Geometry& g, int Cout) {
-    return 1024 + static_cast<size_t>(proj_core_bytes(g)) + proj_w_bytes(g) +
-           static_cast<size_t>(g.pix_per_cta) * Cout * 2 + static_cast<size_t>(Cout) * sizeof(float);
+// tile D^T[o][pixel] = W_out core^T with M = 128 rows (Cout <= 128), N = the tile's
+// pixels (16, 32 or 64), K = C in 64-wide slabs; the same swizzled K-major operand
+// layout as the producer.  W_out keeps only its Cout rows per slab (slab stride
+// Cout * 128 bytes): the MMA's rows past Cout read whatever follows (the next slab,
+// the core tile), and those result rows are never read.  The core tile is written by
+// the sampling threads themselves (their fp32 sums rounded to the I/O dtype, as the
+// unfused pair stores them); once the MMAs have completed, the same memory takes
+// the [pixels][Cout] result, which 16-byte writes store.  Every byte of shared
+// memory kept small here is L1 left to the sampler's gathers.
+__host__ __device__ inline int proj_slab_bytes(int Cout) { return Cout * 128; }
+__host__ __device__ inline int proj_tile_bytes(const Geometry& g, int Cout) {
+    return g.pix_per_cta * (g.C > Cout ? g.C : Cout) * 2;  // the core tile, then the result tile
 }
+__host__ __device__ inline int proj_tmem_cols(const Geometry& g) { return g.pix_per_cta < 32 ? 32 : g.pix_per_cta; }
+// W_out's slabs, the shared tile and the bias, and at least as far as the last slab's
+// 128-row operand reads.
+__host__ __device__ inline int proj_area_bytes(const Geometry& g, int Cout) {
+    const int nslab = g.C / 64, slab = proj_slab_bytes(Cout);
+    const int body = nslab * slab + proj_tile_bytes(g, Cout) + Cout * static_cast<int>(sizeof(float));
+    const int reach = (nslab - 1) * slab + kTcRows * 128;
+    return body > reach ? body : reach;
+}
+// Shared memory of the projection beyond the offset_mask tiles and exponentials
+// (with the 1024-byte alignment slack of the swizzled operands).
+inline size_t proj_extra_bytes(const Geometry& g, int Cout) { return 1024 + static_cast<size_t>(proj_area_bytes(g, Cout)); }
 // The softmax exponentials [K][threads] (fp32), when the masks are logits.
 inline size_t forward_exps_bytes(const Geometry& g) {
     return g.softmax ? static_cast<size_t>(g.K) * samples_threads(g) * sizeof(float) : 0;
@@ -378,7 +388,7 @@ __device__ __forceinline__ void stage_tile_async(T* dst_smem, const T* src, cons
 // the current one.  KH, KW > 0: compile-time grid size (fully unrolled) and
 // RC = remove_center; KH = KW = 0: sizes and remove_center from g.  SM:
 // softmax over the K masks.  LIN: offset_mask rows from the linear producer.
-// PROJ: the output projection behind the sampler (see proj_core_bytes).
+// PROJ: the output projection behind the sampler (see proj_slab_bytes).
 template <typename T, int VEC, int KH, int KW, bool RC, bool SM, bool LIN, bool PROJ>
 __global__ void __launch_bounds__(256, kFwdCtasPerSm) forward_kernel(const Geometry g, const T* __restrict__ value,
                                                       const T* __restrict__ om, T* __restrict__ out,
@@ -420,32 +430,31 @@ __global__ void __launch_bounds__(256, kFwdCtasPerSm) forward_kernel(const Geome
         om_buf = reinterpret_cast<T*>(smem);
         e_s = reinterpret_cast<float*>(om_buf + g.fbufs * tile_elems);
     }
-    // PROJ: the swizzled core tile and W_out (1024-byte aligned), the [pixels][Cout]
-    // result tile and the bias (fp32), after the exponentials
+    // PROJ: W_out's swizzled slabs (1024-byte aligned), the swizzled core tile (later the
+    // [pixels][Cout] result tile) and the bias (fp32), after the exponentials
     uint32_t pj_a = 0u, pj_w = 0u;
     T* pj_o = nullptr;
     float* pj_b = nullptr;
     if constexpr (PROJ) {
         const uint32_t end = sbase + static_cast<uint32_t>(g.fbufs * tile_elems * sizeof(T)) +
                              (SM ? static_cast<uint32_t>(g.K * blockDim.x * sizeof(float)) : 0u);
-        pj_a = (end + 1023u) & ~1023u;
-        pj_w = pj_a + proj_core_bytes(g);
-        pj_o = reinterpret_cast<T*>(smem + (pj_w - sbase) + proj_w_bytes(g));
-        pj_b = reinterpret_cast<float*>(pj_o + g.pix_per_cta * lin.Cout);
+        pj_w = (end + 1023u) & ~1023u;
+        pj_a = pj_w + (g.C / 64) * proj_slab_bytes(lin.Cout);  // Cout * 128 is a multiple of 2048
+        pj_o = reinterpret_cast<T*>(smem + (pj_a - sbase));
+        pj_b = reinterpret_cast<float*>(smem + (pj_a - sbase) + proj_tile_bytes(g, lin.Cout));
     }
     const int ntiles = g.N * g.tiles_h * g.tiles_w;
     int tile = blockIdx.x;
     if (tile >= ntiles) return;
     if constexpr (PROJ) {
         for (int j = threadIdx.x; j < lin.Cout; j += blockDim.x) pj_b[j] = lin.pb ? to_f32(lin.pb[j]) : 0.f;
-        // W_out rows [Cout][C] into 64-wide swizzled slabs; rows Cout..127 zero (their results are never read)
+        // W_out rows [Cout][C] into 64-wide swizzled slabs of Cout rows
         const int cpr = g.C / 8;
-        for (int i = threadIdx.x; i < kTcRows * cpr; i += blockDim.x) {
+        for (int i = threadIdx.x; i < lin.Cout * cpr; i += blockDim.x) {
             const int r = i / cpr, c = i - r * cpr;
-            uint4 v = make_uint4(0u, 0u, 0u, 0u);
-            if (r < lin.Cout) v = ld_gather(lin.pw + static_cast<long long>(r) * g.C + c * 8);
-            *reinterpret_cast<uint4*>(smem + (pj_w - sbase) + (c >> 3) * (kTcRows * 128) + r * 128 +
-                                      (((c & 7) ^ (r & 7)) << 4)) = v;
+            *reinterpret_cast<uint4*>(smem + (pj_w - sbase) + (c >> 3) * proj_slab_bytes(lin.Cout) + r * 128 +
+                                      (((c & 7) ^ (r & 7)) << 4)) =
+                ld_gather(lin.pw + static_cast<long long>(r) * g.C + c * 8);
         }
         if (threadIdx.x == 0) {
             tc::mbar_init(tc::smem_u32(&tc_mbar), 1);
@@ -733,7 +742,7 @@ __global__ void __launch_bounds__(256, kFwdCtasPerSm) forward_kernel(const Geome
                 for (int sb = 0; sb < g.C / 64; ++sb)
 #pragma unroll
                     for (int q = 0; q < 4; ++q)
-                        tc::umma_f16(tmem, tc::umma_desc_sw128(pj_w + sb * (kTcRows * 128) + q * 32, 16, 1024),
+                        tc::umma_f16(tmem, tc::umma_desc_sw128(pj_w + sb * proj_slab_bytes(lin.Cout) + q * 32, 16, 1024),
                                      tc::umma_desc_sw128(pj_a + sb * (npix * 128) + q * 32, 16, 1024), idesc,
                                      sb > 0 || q > 0);
                 tc::umma_commit(tc::smem_u32(&tc_mbar));
@@ -799,7 +808,9 @@ cudaError_t launch_typed(const Geometry& g, const void* value, const void* om, v
                         : PROJ ? forward_proj_smem_bytes(g, lin.Cout)
                                : forward_smem_bytes(g, sizeof(T));
     Geometry gk = g;
-    gk.fbufs = LIN ? 1 : forward_bufs(g, sizeof(T), PROJ ? proj_extra_bytes(g, lin.Cout) : 0);
+    // PROJ keeps two offset_mask tiles: its own tiles already take shared memory, and what is
+    // left is L1 for the gathers (a third tile was measured slower on every workload)
+    gk.fbufs = LIN ? 1 : PROJ ? 2 : forward_bufs(g, sizeof(T), 0);
     auto kern = forward_kernel<T, VEC, KH, KW, RC, SM, LIN, PROJ>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
@@ -895,8 +906,7 @@ bool forward_proj_shape_ok(const Geometry& g, int Cout) {
 }
 
 size_t forward_proj_smem_bytes(const Geometry& g, int Cout) {
-    const size_t extra = proj_extra_bytes(g, Cout);
-    return forward_bufs(g, 2, extra) * static_cast<size_t>(g.pix_per_cta) * g.P * 2 + forward_exps_bytes(g) + extra;
+    return 2 * static_cast<size_t>(g.pix_per_cta) * g.P * 2 + forward_exps_bytes(g) + proj_extra_bytes(g, Cout);
 }
 
 cudaError_t launch_forward_proj(const Geometry& g, int dtype, const void* value, const void* om, const void* w,
