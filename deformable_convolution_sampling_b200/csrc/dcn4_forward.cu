@@ -777,9 +777,12 @@ __global__ void __launch_bounds__(256, kFwdCtasPerSm) forward_kernel(const Geome
                           *reinterpret_cast<const uint4*>(pj_o + (qy * g.TW + qx) * lin.Cout + c * EPV));
             }
         }
-        // LIN: the producer rewrites om_s at the next tile; plain and PROJ with two buffers: the
-        // next copy goes to this tile's buffer (with three, to the one read two tiles ago)
-        if (LIN || g.fbufs < 3) __syncthreads();
+        // Plain with two buffers: the next tile's copy (issued before the next top barrier) goes
+        // to the buffer read two tiles ago only with three, so with two a barrier must come first.
+        // LIN and PROJ need none here: LIN's next copies go to x buffers whose last reads precede
+        // the post-GEMM barrier, and its om_s is rewritten only after the next top barrier; PROJ
+        // reads om_s only before its first barrier, which precedes its second.
+        if (!LIN && !PROJ && g.fbufs < 3) __syncthreads();
         cur = nxt;
     }
     if constexpr (PROJ) {
