@@ -425,7 +425,16 @@ __global__ void __launch_bounds__(256, 3) samples_kernel(const Geometry g, const
                                          (static_cast<uint64_t>(fix16(cell.lh)) << 32) |
                                          (static_cast<uint64_t>(fix16(cell.lw)) << 48);
                     const int dl0 = has ? window_slot(fs, ta, ua) : -1;
-                    if (has && dl0 < 0) atomicOr(sa.tile_count + tile_index(g, t.n, ta, ua), kBucketOverflow);
+                    if (has && dl0 < 0) {
+                        // The own tile is outside the window: it rescans, and so do the tiles this
+                        // sample's copies would have gone to, since none of them gets its record.
+                        atomicOr(sa.tile_count + tile_index(g, t.n, ta, ua), kBucketOverflow);
+                        const bool sr = h0 >= 0 && h0 + 1 < g.H && h0 + 1 == (ta + 1) * g.BH;
+                        const bool sc = w0 >= 0 && w0 + 1 < g.W && w0 + 1 == (ua + 1) * g.BW;
+                        if (sr) atomicOr(sa.tile_count + tile_index(g, t.n, ta + 1, ua), kBucketOverflow);
+                        if (sc) atomicOr(sa.tile_count + tile_index(g, t.n, ta, ua + 1), kBucketOverflow);
+                        if (sr && sc) atomicOr(sa.tile_count + tile_index(g, t.n, ta + 1, ua + 1), kBucketOverflow);
+                    }
                     // rank among the CTA's records for the tile: one shared atomic per distinct tile in the warp
                     const unsigned okm = __ballot_sync(0xffffffffu, dl0 >= 0);
                     uint64_t meta = 0;
