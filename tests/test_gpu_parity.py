@@ -360,6 +360,20 @@ def test_samples_beyond_the_filing_window():
     assert diag["corrupt_bucket_tiles"] == 0 and diag["rescanned_tiles"] > 0, diag
 
 
+def test_copies_of_samples_filed_outside_the_window():
+    """32 groups of 8 channels on a 14 x 14 map: grad_value tiles of two rows, so the filing
+    window of the bottom grad_offset_mask CTAs leaves out the top tile rows.  With offsets
+    N(0, 4^2) some of their samples land in a cell on the border of an excluded tile and the
+    next one down: the excluded tile rescans, and the tile below (inside every CTA's window)
+    must rescan too, since it does not get the sample's copy.  Both against the oracle."""
+    w = gen.custom(name="window_copies", N=4, H=14, W=14, G=32, Cg=8, Ho=14, Wo=14, K=9, P=864, dtype="bf16",
+                   offset=("normal", 0.0, 4.0))
+    inp = gen.make_inputs(w)
+    _check_backward(w, inp)
+    diag = _diagnostics(w, inp)
+    assert diag["corrupt_bucket_tiles"] == 0 and diag["rescanned_tiles"] > 0, diag
+
+
 @pytest.mark.parametrize("name", gen.WORKLOAD_ORDER)
 def test_no_fallback_tiles_on_the_workloads(name):
     """On every measured workload no grad_value tile finds its filed records
